@@ -1,0 +1,113 @@
+/*
+ * rq_oracle.h -- CPU oracle for the ResidualQuant hot path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file and rq_oracle.c are the slow, plain,
+ * obviously-correct restatement of the method that the CUDA library is
+ * checked against.  Only the test-suite, the smoke check and the CPU-baseline
+ * leg of the benchmark may load it.  It shares no code, header, table or
+ * constant with the CUDA library under kv_cache_residual_rq_b200/csrc, and
+ * the library never loads it.
+ *
+ * Method source: "ResidualQuant: KV Cache Quantization for Looped
+ * Transformers with 2-Bit Residuals" (newx.sg page, Abstract and AI Summary):
+ * the final loop's K/V is kept as a reference, every other loop is stored as
+ * a low-bit residual against it, the residual is rotated, quantised per group
+ * down to INT2 with a least-squares scale, and the bit width may differ per
+ * loop.  Everything finer than that (the Walsh-Hadamard rotation, the code
+ * grid, the rounding rule, the group size, the packing) is a reading of the
+ * pages that is written down in DESIGN.md, section "Readings".
+ *
+ * Two levels:
+ *   - the fp32 exact-spec path (orq_*_f32): the encoder step by step, in
+ *     the fp32 operation order the spec fixes.  Codes from this path are the
+ *     bit-exact target for the GPU encoder.
+ *   - the fp64 definitional path (orq_*_f64): the rotation as an explicit
+ *     d x d matrix, reconstruction and softmax attention in double.  This is
+ *     the reference for decode-attention outputs.
+ *
+ * Data formats (all little-endian, all arrays row-major):
+ *   bf16  : uint16_t, the top half of an IEEE binary32
+ *   fp16  : uint16_t, IEEE binary16
+ *   codes : per row of d elements, ceil(d*bits/32) uint32 words; element j lives
+ *           in word j / (32/bits) at bit offset bits * (j % (32/bits))
+ *   scales: per row, d/g fp16 values, one per contiguous group of g rotated
+ *           coordinates
+ */
+#ifndef RQ_ORACLE_H
+#define RQ_ORACLE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ORQ_MAX_D 4096
+
+/* ---- scalar formats ---------------------------------------------------- */
+float    orq_bf16_to_f32(uint16_t h);
+double   orq_f16_to_f64(uint16_t h);
+uint16_t orq_f64_to_f16(double x);          /* IEEE round-to-nearest-even */
+
+/* ---- seeded sign vector (counter-based splitmix64) --------------------- */
+uint64_t orq_splitmix64(uint64_t seed, uint64_t i);
+void     orq_signs(uint64_t seed, int d, int8_t *D);
+
+/* ---- rotation ----------------------------------------------------------- */
+float orq_cd_f32(int d);                                 /* RN_f32(1/sqrt(d)) */
+int   orq_hadamard_entry(int i, int j);                  /* Sylvester, +-1 */
+void  orq_rotation_matrix_f64(int d, const int8_t *D, double *R);
+void  orq_rotate_f32(int d, const int8_t *D, const float *r, float *y);
+void  orq_fwht_f64(int d, double *v);                    /* in place, unnormalised */
+
+/* ---- quantiser (fp32 exact-spec) ---------------------------------------- */
+void orq_quantize_group_f32(int g, int bits, const float *y, uint8_t *codes,
+                            double *s_exact, uint16_t *s_f16, int *ties);
+void orq_pack_codes(int d, int bits, const uint8_t *codes, uint32_t *words);
+void orq_unpack_codes(int d, int bits, const uint32_t *words, uint8_t *codes);
+
+/* ---- encoder ------------------------------------------------------------ */
+/* One row: r = x - ref, y = Rot r, per-group codes and scale. */
+void orq_encode_row_f32(int d, int g, int bits, const int8_t *D,
+                        const uint16_t *x, const uint16_t *ref,
+                        uint32_t *words, uint16_t *scales, int *ties);
+
+/* n_rows contiguous rows of d elements. Returns the total tie count. */
+long orq_encode_rows_f32(long n_rows, int d, int g, int bits, uint64_t seed,
+                         const uint16_t *x, const uint16_t *ref,
+                         uint32_t *words, uint16_t *scales);
+
+/* fp64 definitional encoder for one row.  Also returns, per element, the
+ * distance of u from the nearest decision boundary (an integer) so that
+ * disagreement with the fp32 path can be attributed to boundary proximity. */
+void orq_encode_row_f64(int d, int g, int bits, const int8_t *D,
+                        const uint16_t *x, const uint16_t *ref,
+                        uint8_t *codes, double *scales, double *bdist);
+
+/* ---- reconstruction and attention (fp64 definitional) ------------------- */
+/* out[d] = f64(ref) + Rot^T (s16 * level), for one row. bits==16 => ref. */
+void orq_reconstruct_row_f64(int d, int g, int bits, const int8_t *D,
+                             const uint16_t *ref, const uint32_t *words,
+                             const uint16_t *scales, double *out);
+
+/* Softmax attention of G query rows over T keys/values, all in double:
+ * out[r] = sum_t softmax_t(scale * <q_r, K_t>) V_t. */
+void orq_attention_f64(int T, int d, int G, const double *q, const double *K,
+                       const double *V, double scale, double *out);
+
+/* Decode attention at one loop for one (batch, kv-head): reconstruct every
+ * cached K/V row of that loop, then exact attention.  q is bf16 [G][d];
+ * ref_k/ref_v bf16 [T][d]; codes [T][d*bits/32]; scales fp16 [T][d/g].
+ * bits == 16 means the loop is the reference (codes/scales unused).
+ * scale <= 0 selects 1/sqrt(d).  out is [G][d] double.  Returns 0 on success. */
+int orq_decode_attention_f64(int T, int d, int g, int G, int bits, uint64_t seed,
+                             double scale, const uint16_t *q,
+                             const uint16_t *ref_k, const uint16_t *ref_v,
+                             const uint32_t *codes_k, const uint32_t *codes_v,
+                             const uint16_t *scales_k, const uint16_t *scales_v,
+                             double *out);
+
+#ifdef __cplusplus
+}
+#endif
+#endif
