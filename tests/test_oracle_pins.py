@@ -326,6 +326,10 @@ def test_attention_matches_sdpa(T, G, d):
     V = rng.standard_normal((T, d))
     out = oracle.attention_f64(q, K, V, 1 / math.sqrt(d))
     assert np.abs(out - _sdpa64(q, K, V, 1 / math.sqrt(d))).max() < 1e-12
+    # scores far beyond exp's range: only a max-subtracted softmax survives
+    out = oracle.attention_f64(q, K * 400, V, 1 / math.sqrt(d))
+    assert np.isfinite(out).all()
+    assert np.abs(out - _sdpa64(q, K * 400, V, 1 / math.sqrt(d))).max() < 1e-9
 
 
 @pytest.mark.parametrize("T,G,d,g", [(1, 4, 64, 32), (100, 1, 128, 32), (77, 4, 128, 64)])
