@@ -1,0 +1,189 @@
+/*
+ * rq.h -- C ABI of librq.so, the B200 (sm_100a) hot path of ResidualQuant.
+ *
+ * Method: "ResidualQuant: KV Cache Quantization for Looped Transformers with
+ * 2-Bit Residuals" (newx.sg page, Abstract).  A looped Transformer writes one
+ * K/V per loop.  The final loop's K/V is kept in BF16 as the reference; every
+ * other loop is stored as its residual against the reference, rotated,
+ * quantised per group to INT2 (or INT4 for loops given more bits) with a
+ * least-squares fp16 scale.  Decode attention reads the reference plus the
+ * codes and rebuilds the loop's K/V on the fly.
+ *
+ * Conventions for every entry point:
+ *   - Data pointers are DEVICE pointers unless a parameter says "host".
+ *     The caller allocates and owns every buffer, including the workspace;
+ *     the library allocates nothing and never synchronises the stream.
+ *   - `stream` is a cudaStream_t passed as void*; NULL means the legacy
+ *     default stream.  Work is enqueued in order on that stream and the call
+ *     returns before it runs.
+ *   - Arguments are validated before anything is enqueued.  A call that
+ *     returns an error has enqueued nothing and written nothing.
+ *   - Device pointers must be 16-byte aligned (RQ_ERR_ALIGNMENT otherwise).
+ *   - Buffers must be at least the size the matching rq_*_bytes() query
+ *     returns; those sizes are rounded up to 16 bytes and the kernels may
+ *     read (never write) the padding.
+ *   - No C++ exception, abort or CUDA error escapes: launch failures come
+ *     back as RQ_ERR_CUDA.
+ *   - bf16 / fp16 values are passed as uint16_t bit patterns.
+ *
+ * Layouts (row-major, T = ctx, d = head_dim, g = group, b = bits):
+ *   K/V of one loop, reference : bf16 [rows][kv_heads][T][d]
+ *   query                      : bf16 [batch][q_heads][d]
+ *   codes of one loop          : uint32 [rows][kv_heads][T][d*b/32];
+ *                                element j of a row is in word j/(32/b) at
+ *                                bit offset b*(j mod 32/b), LSB first;
+ *                                code c stands for level 2c - (2^b - 1)
+ *   scales of one loop         : fp16 [rows][kv_heads][T][d/g], one per
+ *                                contiguous group of g rotated coordinates
+ *   output                     : fp32 [batch][q_heads][d]
+ * Query head j attends with kv head j / (q_heads / kv_heads).
+ *
+ * Rotation: Rot = (1/sqrt(d)) * H_d * D, H_d the Sylvester Hadamard matrix,
+ * D = diag(+-1) with D_i = -1 iff bit 63 of splitmix64 output i of `seed`
+ * is set (output i = mix(seed + (i+1) * 0x9E3779B97F4A7C15)).  The same seed
+ * must be given to rq_encode and rq_decode_attention.
+ */
+#ifndef RQ_H
+#define RQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    RQ_OK = 0,
+    RQ_ERR_INVALID_ARG = 1,   /* null pointer, non-positive size, bad shape */
+    RQ_ERR_UNSUPPORTED = 2,   /* head_dim, group, bits or GQA ratio not built */
+    RQ_ERR_ALIGNMENT = 3,     /* a device pointer is not 16-byte aligned */
+    RQ_ERR_WORKSPACE = 4,     /* workspace missing or smaller than required */
+    RQ_ERR_CUDA = 5           /* a CUDA launch or query failed */
+} rq_status;
+
+#define RQ_MAX_LOOPS 16       /* non-final loops one rq_encode call takes */
+
+typedef struct {
+    int32_t batch;      /* leading rows: B for decode; any flattened count
+                           (e.g. layers * B) for encode */
+    int32_t kv_heads;   /* Hkv >= 1 */
+    int32_t q_heads;    /* Hq, a multiple of Hkv (decode only; encode ignores) */
+    int32_t ctx;        /* T: cached tokens per (row, kv head) */
+    int32_t head_dim;   /* d: 64 or 128 */
+    int32_t group;      /* g: 32 or 64, divides d */
+} rq_shape;
+
+/* Library version as major*10000 + minor*100 + patch. */
+int rq_version(void);
+
+/* Static text for a status code; never NULL. */
+const char *rq_status_string(rq_status s);
+
+/* Bytes of the codes of ONE loop at `bits` (2 or 4) for `shape`:
+ * batch*kv_heads*ctx*head_dim*bits/8 rounded up to 16.  0 for bits == 16 or
+ * an invalid shape.  Host-only arithmetic. */
+size_t rq_codes_bytes(const rq_shape *shape, int bits);
+
+/* Bytes of the fp16 scales of ONE loop: batch*kv_heads*ctx*(head_dim/group)*2
+ * rounded up to 16.  0 for bits == 16 or an invalid shape. */
+size_t rq_scales_bytes(const rq_shape *shape, int bits);
+
+/* Workspace bytes rq_decode_attention needs for `shape` (partial softmax
+ * states of the context splits, one arrival counter per (batch, kv head) and
+ * a status word).  0 for an invalid shape.  Host-only arithmetic. */
+size_t rq_decode_workspace_bytes(const rq_shape *shape);
+
+/*
+ * rq_encode -- ResidualQuant encoder (Abstract: the non-final loops are
+ * stored as residuals against the final-loop reference, rotated, and
+ * quantised per group with a least-squares scale; the bit width is chosen
+ * per loop).
+ *
+ * For every row (r, h, t) and every loop l < n_loops with bits[l] != 16:
+ *   e   = f32(kv_loops[l][r,h,t,:]) - f32(ref[r,h,t,:])       (binary32, RN)
+ *   y   = RN(c_d * FWHT(D e)), butterfly stages h = 1, 2, ..., d/2, each
+ *         (a, b) -> (a + b, a - b) in binary32 RN, c_d = RN(1/sqrt(d))
+ *   per group of g coordinates: amax = max |y_i|;
+ *         inv = (2^(b-1) - 1/2) / amax (binary32 RN), or 0 if amax < 2^-126;
+ *         c_i = clamp(floor(RN(y_i * inv)) + 2^(b-1), 0, 2^b - 1);
+ *         l_i = 2 c_i - (2^b - 1);
+ *         s = <y, l> / <l, l>, clamped to +-65504, stored as fp16 RN.
+ * Codes are bit-identical to that sequence; the scale's dot product is
+ * summed in an unspecified order (at most one fp16 ulp from the exact value).
+ *
+ *   shape          : batch = number of leading rows, kv_heads, ctx, head_dim,
+ *                    group used; q_heads ignored.  ctx == 0 is a no-op.
+ *   kv_loops       : HOST array of n_loops device pointers, bf16 K (or V) of
+ *                    each non-final loop, layout [rows][Hkv][T][d].
+ *   n_loops        : 1 .. RQ_MAX_LOOPS.
+ *   ref            : device bf16, the final loop, same layout.  Read only.
+ *   bits_per_loop  : HOST array of n_loops values, each 2, 4 or 16.
+ *                    16 marks a loop kept in BF16 by the caller: nothing is
+ *                    written for it and its pointers may be NULL.
+ *   seed           : rotation seed.
+ *   codes_out      : HOST array of n_loops device pointers, each
+ *                    rq_codes_bytes(shape, bits_per_loop[l]) bytes.
+ *   scales_out     : HOST array of n_loops device pointers (fp16 bits), each
+ *                    rq_scales_bytes(shape, bits_per_loop[l]) bytes.
+ * The host arrays are read before the call returns.  Outputs must not
+ * overlap inputs.
+ */
+rq_status rq_encode(const rq_shape *shape, const uint16_t *const *kv_loops, int n_loops,
+                    const uint16_t *ref, const uint8_t *bits_per_loop, uint64_t seed,
+                    uint32_t *const *codes_out, uint16_t *const *scales_out, void *stream);
+
+/*
+ * rq_decode_attention -- fused ResidualQuant decode attention for one loop
+ * (Abstract: the reconstruction stays efficient; the reduced KV traffic is
+ * what speeds decode up).
+ *
+ * For each batch b and query head j (kv head h = j / G, G = Hq / Hkv), with
+ * K_hat_t = ref_k[b,h,t] + Rot^T (s^K_t * l^K_t) and likewise V_hat:
+ *   out[b,j,:] = sum_t softmax_t(sigma * <q[b,j], K_hat_t>) V_hat_t
+ * computed without materialising K_hat or V_hat: the query is rotated once
+ * (q~ = Rot q), scores are <q, ref_k_t> + sum_groups s_t,g <q~_g, l_t,g>, the
+ * V residual is accumulated in the rotated domain and rotated back once per
+ * output row.  The context is split across CTAs (split-K) and the partial
+ * softmax states are merged in the same launch.
+ *
+ *   shape          : batch, kv_heads, q_heads (multiple of kv_heads, ratio
+ *                    1..8), ctx >= 1, head_dim 64|128, group 32|64.
+ *   q              : device bf16 [batch][q_heads][d].
+ *   ref_k, ref_v   : device bf16 [batch][Hkv][T][d], the final loop.
+ *   codes_k/v      : device, this loop's codes (rq_codes_bytes); ignored and
+ *                    may be NULL when bits == 16.
+ *   scales_k/v     : device fp16 bits, this loop's scales (rq_scales_bytes);
+ *                    ignored and may be NULL when bits == 16.
+ *   bits           : 2 or 4 for a residual loop; 16 for the reference loop
+ *                    itself (plain attention over ref_k/ref_v).
+ *   seed           : the seed the codes were encoded with.
+ *   softmax_scale  : sigma; <= 0 selects 1/sqrt(head_dim).
+ *   out            : device fp32 [batch][q_heads][d].
+ *   workspace      : device, >= rq_decode_workspace_bytes(shape) bytes,
+ *                    ZERO-FILLED before its first use.  Every successful call
+ *                    leaves it ready for the next; calls sharing a workspace
+ *                    must be ordered on one stream.
+ * The split of the context depends only on (batch, kv_heads, ctx), never on
+ * bits, so a residual loop whose scales are all zero gives bit-for-bit the
+ * output of the reference loop.
+ */
+rq_status rq_decode_attention(const rq_shape *shape, const uint16_t *q,
+                              const uint16_t *ref_k, const uint16_t *ref_v,
+                              const uint32_t *codes_k, const uint32_t *codes_v,
+                              const uint16_t *scales_k, const uint16_t *scales_v,
+                              int bits, uint64_t seed, float softmax_scale, float *out,
+                              void *workspace, size_t workspace_bytes, void *stream);
+
+/* Copies the workspace's device status word to *host_status (blocking read
+ * on `stream`).  0 means every decode call since the workspace was zeroed
+ * ran clean; non-zero means a bounded wait inside a kernel ran out, its
+ * output is invalid, and the workspace must be zeroed again.  This is the
+ * only entry point that synchronises. */
+rq_status rq_workspace_status(const void *workspace, size_t workspace_bytes,
+                              uint32_t *host_status, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* RQ_H */

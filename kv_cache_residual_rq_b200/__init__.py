@@ -1,0 +1,75 @@
+"""ResidualQuant KV cache for looped Transformers on B200 (sm_100a).
+
+The compute path is librq.so (hand-written CUDA, C ABI in include/rq.h);
+this package is its Python binding.  torch is used for device memory and
+streams only: the helpers below allocate buffers with the sizes the library
+reports and pass pointers through.
+
+    from kv_cache_residual_rq_b200 import make_shape, encode, decode_attention
+"""
+from ._abi import (RQ_ERR_ALIGNMENT, RQ_ERR_CUDA, RQ_ERR_INVALID_ARG, RQ_ERR_UNSUPPORTED,
+                   RQ_ERR_WORKSPACE, RQ_MAX_LOOPS, RQ_OK, RqError, lib, make_shape,
+                   rq_codes_bytes, rq_decode_attention, rq_decode_workspace_bytes, rq_encode,
+                   rq_scales_bytes, rq_shape, rq_status_string, rq_version,
+                   rq_workspace_status)
+
+__all__ = [
+    "RQ_OK", "RQ_ERR_INVALID_ARG", "RQ_ERR_UNSUPPORTED", "RQ_ERR_ALIGNMENT", "RQ_ERR_WORKSPACE",
+    "RQ_ERR_CUDA", "RQ_MAX_LOOPS", "RqError", "lib", "rq_shape", "make_shape", "rq_version",
+    "rq_status_string", "rq_codes_bytes", "rq_scales_bytes", "rq_decode_workspace_bytes",
+    "rq_encode", "rq_decode_attention", "rq_workspace_status",
+    "alloc_codes", "alloc_scales", "alloc_workspace", "encode", "decode_attention",
+]
+
+
+def alloc_codes(shape, bits, device="cuda"):
+    """uint8 device buffer of rq_codes_bytes(shape, bits) bytes (None for bits 16)."""
+    import torch
+    n = rq_codes_bytes(shape, bits)
+    return torch.empty(n, dtype=torch.uint8, device=device) if n else None
+
+
+def alloc_scales(shape, bits, device="cuda"):
+    import torch
+    n = rq_scales_bytes(shape, bits)
+    return torch.empty(n, dtype=torch.uint8, device=device) if n else None
+
+
+def alloc_workspace(shape, device="cuda"):
+    """Zero-filled decode workspace, as rq_decode_attention requires."""
+    import torch
+    n = rq_decode_workspace_bytes(shape)
+    if n == 0:
+        raise RqError(RQ_ERR_INVALID_ARG, "rq_decode_workspace_bytes")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def encode(kv_loops, ref, bits_per_loop, group, seed, stream=None):
+    """Encode non-final loops (bf16 tensors [rows, Hkv, T, d]) against `ref`.
+
+    Returns (codes, scales): per loop a uint8 device buffer, or None for a
+    loop kept in BF16 (bits 16)."""
+    rows, hkv, t, d = ref.shape
+    shape = make_shape(rows, hkv, t, d, group)
+    codes = [alloc_codes(shape, b, ref.device) for b in bits_per_loop]
+    scales = [alloc_scales(shape, b, ref.device) for b in bits_per_loop]
+    rq_encode(shape, kv_loops, ref, bits_per_loop, seed, codes, scales, stream)
+    return codes, scales
+
+
+def decode_attention(q, ref_k, ref_v, codes_k, codes_v, scales_k, scales_v, bits, group, seed,
+                     softmax_scale=0.0, out=None, workspace=None, stream=None):
+    """Decode attention of one loop.  q [B, Hq, d] bf16; ref_k/ref_v
+    [B, Hkv, T, d] bf16; codes/scales as returned by encode (None for bits 16).
+    Returns out [B, Hq, d] fp32."""
+    import torch
+    b, hq, d = q.shape
+    _, hkv, t, _ = ref_k.shape
+    shape = make_shape(b, hkv, t, d, group, q_heads=hq)
+    if out is None:
+        out = torch.empty((b, hq, d), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(shape, q.device)
+    rq_decode_attention(shape, q, ref_k, ref_v, codes_k, codes_v, scales_k, scales_v, bits, seed,
+                        softmax_scale, out, workspace, stream=stream)
+    return out

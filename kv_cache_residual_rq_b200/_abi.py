@@ -1,0 +1,165 @@
+"""ctypes binding of librq.so: the C ABI of include/rq.h, names unchanged.
+
+Argument marshalling only.  Each function takes what the C function takes;
+a torch tensor may stand in for a device pointer (its data_ptr() is passed)
+and `stream=None` means torch's current CUDA stream.  A non-zero rq_status
+raises RqError.  There is no fallback: if librq.so is missing or fails to
+load, every call raises.
+"""
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "librq.so")
+
+RQ_OK = 0
+RQ_ERR_INVALID_ARG = 1
+RQ_ERR_UNSUPPORTED = 2
+RQ_ERR_ALIGNMENT = 3
+RQ_ERR_WORKSPACE = 4
+RQ_ERR_CUDA = 5
+RQ_MAX_LOOPS = 16
+
+
+class RqError(RuntimeError):
+    def __init__(self, status, what):
+        self.status = status
+        super().__init__(f"{what}: rq_status {status} ({rq_status_string(status)})")
+
+
+class rq_shape(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("kv_heads", ctypes.c_int32),
+                ("q_heads", ctypes.c_int32), ("ctx", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("group", ctypes.c_int32)]
+
+    def __repr__(self):
+        return ("rq_shape(batch=%d, kv_heads=%d, q_heads=%d, ctx=%d, head_dim=%d, group=%d)"
+                % (self.batch, self.kv_heads, self.q_heads, self.ctx, self.head_dim, self.group))
+
+
+def make_shape(batch, kv_heads, ctx, head_dim, group, q_heads=None):
+    return rq_shape(batch, kv_heads, kv_heads if q_heads is None else q_heads, ctx, head_dim, group)
+
+
+_lib = None
+
+
+def lib():
+    """Load librq.so once; raise if it is absent (no CPU fallback exists)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is not built; run `python -m kv_cache_residual_rq_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        c = ctypes
+        sp = c.POINTER(rq_shape)
+        L.rq_version.argtypes = []
+        L.rq_version.restype = c.c_int
+        L.rq_status_string.argtypes = [c.c_int]
+        L.rq_status_string.restype = c.c_char_p
+        L.rq_codes_bytes.argtypes = [sp, c.c_int]
+        L.rq_codes_bytes.restype = c.c_size_t
+        L.rq_scales_bytes.argtypes = [sp, c.c_int]
+        L.rq_scales_bytes.restype = c.c_size_t
+        L.rq_decode_workspace_bytes.argtypes = [sp]
+        L.rq_decode_workspace_bytes.restype = c.c_size_t
+        L.rq_encode.argtypes = [sp, c.POINTER(c.c_void_p), c.c_int, c.c_void_p,
+                                c.POINTER(c.c_uint8), c.c_uint64, c.POINTER(c.c_void_p),
+                                c.POINTER(c.c_void_p), c.c_void_p]
+        L.rq_encode.restype = c.c_int
+        L.rq_decode_attention.argtypes = [sp, c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p,
+                                          c.c_void_p, c.c_void_p, c.c_void_p, c.c_int, c.c_uint64,
+                                          c.c_float, c.c_void_p, c.c_void_p, c.c_size_t, c.c_void_p]
+        L.rq_decode_attention.restype = c.c_int
+        L.rq_workspace_status.argtypes = [c.c_void_p, c.c_size_t, c.POINTER(c.c_uint32), c.c_void_p]
+        L.rq_workspace_status.restype = c.c_int
+        _lib = L
+    return _lib
+
+
+def _ptr(x):
+    """Device pointer of a tensor, an int, or None (NULL)."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _shp(shape):
+    return None if shape is None else ctypes.byref(shape)
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(status, what):
+    if status != RQ_OK:
+        raise RqError(status, what)
+
+
+# ---- the C ABI, one function per entry point ---------------------------------
+
+def rq_version():
+    return lib().rq_version()
+
+
+def rq_status_string(status):
+    return lib().rq_status_string(int(status)).decode()
+
+
+def rq_codes_bytes(shape, bits):
+    return lib().rq_codes_bytes(_shp(shape), int(bits))
+
+
+def rq_scales_bytes(shape, bits):
+    return lib().rq_scales_bytes(_shp(shape), int(bits))
+
+
+def rq_decode_workspace_bytes(shape):
+    return lib().rq_decode_workspace_bytes(_shp(shape))
+
+
+def rq_encode(shape, kv_loops, ref, bits_per_loop, seed, codes_out, scales_out, stream=None,
+              check=True):
+    """kv_loops / codes_out / scales_out: sequences (one entry per non-final
+    loop) of tensors, ints or None.  Returns the rq_status."""
+    n = len(bits_per_loop)
+    ptrs = lambda seq: (ctypes.c_void_p * max(n, 1))(*[_ptr(v) for v in seq])
+    bits = (ctypes.c_uint8 * max(n, 1))(*[int(b) for b in bits_per_loop])
+    st = lib().rq_encode(_shp(shape), ptrs(kv_loops), n, _ptr(ref), bits,
+                         ctypes.c_uint64(seed), ptrs(codes_out), ptrs(scales_out),
+                         _stream(stream))
+    if check:
+        _check(st, "rq_encode")
+    return st
+
+
+def rq_decode_attention(shape, q, ref_k, ref_v, codes_k, codes_v, scales_k, scales_v, bits,
+                        seed, softmax_scale, out, workspace, workspace_bytes=None, stream=None,
+                        check=True):
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    st = lib().rq_decode_attention(_shp(shape), _ptr(q), _ptr(ref_k), _ptr(ref_v),
+                                   _ptr(codes_k), _ptr(codes_v), _ptr(scales_k), _ptr(scales_v),
+                                   int(bits), ctypes.c_uint64(seed), float(softmax_scale),
+                                   _ptr(out), _ptr(workspace), int(workspace_bytes),
+                                   _stream(stream))
+    if check:
+        _check(st, "rq_decode_attention")
+    return st
+
+
+def rq_workspace_status(workspace, workspace_bytes=None, stream=None):
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    v = ctypes.c_uint32(0)
+    _check(lib().rq_workspace_status(_ptr(workspace), int(workspace_bytes), ctypes.byref(v),
+                                     _stream(stream)), "rq_workspace_status")
+    return v.value

@@ -1,0 +1,224 @@
+// rq_api.cu -- the C ABI of librq.so (declared in include/rq.h).
+//
+// Host side only: argument validation (before anything is enqueued), the
+// size queries, the work plan of a decode call, and dispatch to the kernels.
+// Nothing here allocates device memory or synchronises, except
+// rq_workspace_status, whose job is to read a status word back.
+#include <climits>
+#include <cmath>
+#include <cstring>
+
+#include "rq_internal.h"
+
+namespace rq {
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t round16(size_t n) { return (n + 15) / 16 * 16; }
+
+bool supported_dims(int head_dim, int group) {
+  return (head_dim == 64 || head_dim == 128) && (group == 32 || group == 64) &&
+         head_dim % group == 0;
+}
+
+// basic shape check shared by the size queries; false for anything invalid
+bool shape_ok(const rq_shape* s, bool need_ctx) {
+  if (!s) return false;
+  if (s->batch < 1 || s->kv_heads < 1 || s->ctx < 0) return false;
+  if (need_ctx && s->ctx < 1) return false;
+  return supported_dims(s->head_dim, s->group);
+}
+
+bool decode_shape_ok(const rq_shape* s) {
+  if (!shape_ok(s, true)) return false;
+  if (s->q_heads < s->kv_heads || s->q_heads % s->kv_heads) return false;
+  const int G = s->q_heads / s->kv_heads;
+  return G == 1 || G == 2 || G == 4 || G == 8;
+}
+
+}  // namespace
+
+int device_sm_count() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 0;
+  if (dev < 64 && cache[dev] > 0) return cache[dev];
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (dev < 64) cache[dev] = sms;
+  return sms;
+}
+
+DecodePlan plan_decode(const rq_shape& s, int num_sms) {
+  DecodePlan pl;
+  pl.heads = (long long)s.batch * s.kv_heads;
+  pl.nt = (s.ctx + kDecodeTile - 1) / kDecodeTile;
+  pl.n_tiles = pl.heads * pl.nt;
+  long long P = (long long)num_sms * kDecodeCtasPerSm;
+  if (P > kDecodeMaxCtas) P = kDecodeMaxCtas;
+  if (P > pl.n_tiles) P = pl.n_tiles;
+  if (P < 1) P = 1;
+  pl.ctas = (int)P;
+  // a head spans at most floor(P / heads) + 2 CTA runs; bound with the
+  // largest P any device can get so the workspace size is device independent
+  long long mc = kDecodeMaxCtas / pl.heads + 2;
+  if (mc > pl.nt) mc = pl.nt;
+  pl.max_contrib = (int)mc;
+  return pl;
+}
+
+size_t decode_workspace_bytes(const rq_shape& s) {
+  const DecodePlan pl = plan_decode(s, 1);
+  const int G = s.q_heads / s.kv_heads;
+  return kWsHeaderBytes + ws_counters_bytes(pl.heads) +
+         (size_t)pl.heads * pl.max_contrib * G * ws_record_floats(s.head_dim) * sizeof(float);
+}
+
+}  // namespace rq
+
+using namespace rq;
+
+extern "C" {
+
+int rq_version(void) { return 100; }   // 0.1.0
+
+const char* rq_status_string(rq_status s) {
+  switch (s) {
+    case RQ_OK: return "ok";
+    case RQ_ERR_INVALID_ARG: return "invalid argument";
+    case RQ_ERR_UNSUPPORTED: return "unsupported head_dim, group, bits or GQA ratio";
+    case RQ_ERR_ALIGNMENT: return "device pointer not 16-byte aligned";
+    case RQ_ERR_WORKSPACE: return "workspace missing or too small";
+    case RQ_ERR_CUDA: return "CUDA launch or query failed";
+  }
+  return "unknown status";
+}
+
+size_t rq_codes_bytes(const rq_shape* shape, int bits) {
+  if (!shape_ok(shape, false) || (bits != 2 && bits != 4)) return 0;
+  const size_t elems =
+      (size_t)shape->batch * shape->kv_heads * shape->ctx * (size_t)shape->head_dim;
+  return round16(elems * bits / 8);
+}
+
+size_t rq_scales_bytes(const rq_shape* shape, int bits) {
+  if (!shape_ok(shape, false) || (bits != 2 && bits != 4)) return 0;
+  const size_t groups = (size_t)shape->batch * shape->kv_heads * shape->ctx *
+                        (size_t)(shape->head_dim / shape->group);
+  return round16(groups * 2);
+}
+
+size_t rq_decode_workspace_bytes(const rq_shape* shape) {
+  if (!decode_shape_ok(shape)) return 0;
+  return decode_workspace_bytes(*shape);
+}
+
+rq_status rq_encode(const rq_shape* shape, const uint16_t* const* kv_loops, int n_loops,
+                    const uint16_t* ref, const uint8_t* bits_per_loop, uint64_t seed,
+                    uint32_t* const* codes_out, uint16_t* const* scales_out, void* stream) {
+  if (!shape || !kv_loops || !bits_per_loop || !codes_out || !scales_out)
+    return RQ_ERR_INVALID_ARG;
+  if (shape->batch < 1 || shape->kv_heads < 1 || shape->ctx < 0) return RQ_ERR_INVALID_ARG;
+  if (n_loops < 1 || n_loops > RQ_MAX_LOOPS) return RQ_ERR_INVALID_ARG;
+  if (!supported_dims(shape->head_dim, shape->group)) return RQ_ERR_UNSUPPORTED;
+  if (!ref) return RQ_ERR_INVALID_ARG;
+  if (!aligned16(ref)) return RQ_ERR_ALIGNMENT;
+  EncodeParams p;
+  std::memset(&p, 0, sizeof p);
+  int active = 0;
+  for (int l = 0; l < n_loops; ++l) {
+    const int b = bits_per_loop[l];
+    if (b != 2 && b != 4 && b != 16) return RQ_ERR_UNSUPPORTED;
+    p.bits[l] = b;
+    if (b == 16) continue;
+    if (!kv_loops[l] || !codes_out[l] || !scales_out[l]) return RQ_ERR_INVALID_ARG;
+    if (!aligned16(kv_loops[l]) || !aligned16(codes_out[l]) || !aligned16(scales_out[l]))
+      return RQ_ERR_ALIGNMENT;
+    p.x[l] = kv_loops[l];
+    p.codes[l] = codes_out[l];
+    p.scales[l] = scales_out[l];
+    ++active;
+  }
+  p.ref = ref;
+  p.n_loops = n_loops;
+  p.seed = seed;
+  p.n_rows = (long long)shape->batch * shape->kv_heads * shape->ctx;
+  if (p.n_rows == 0 || active == 0) return RQ_OK;
+  const int sms = device_sm_count();
+  if (sms <= 0) return RQ_ERR_CUDA;
+  cudaError_t e = launch_encode(shape->head_dim, shape->group, p, sms,
+                                static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? RQ_OK : RQ_ERR_CUDA;
+}
+
+rq_status rq_decode_attention(const rq_shape* shape, const uint16_t* q, const uint16_t* ref_k,
+                              const uint16_t* ref_v, const uint32_t* codes_k,
+                              const uint32_t* codes_v, const uint16_t* scales_k,
+                              const uint16_t* scales_v, int bits, uint64_t seed,
+                              float softmax_scale, float* out, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  if (!shape) return RQ_ERR_INVALID_ARG;
+  if (shape->batch < 1 || shape->kv_heads < 1 || shape->ctx < 1 ||
+      shape->q_heads < shape->kv_heads)
+    return RQ_ERR_INVALID_ARG;
+  if (shape->q_heads % shape->kv_heads) return RQ_ERR_INVALID_ARG;
+  if (!decode_shape_ok(shape)) return RQ_ERR_UNSUPPORTED;
+  if (bits != 2 && bits != 4 && bits != 16) return RQ_ERR_UNSUPPORTED;
+  if (!q || !ref_k || !ref_v || !out) return RQ_ERR_INVALID_ARG;
+  if (bits != 16 && (!codes_k || !codes_v || !scales_k || !scales_v)) return RQ_ERR_INVALID_ARG;
+  if (!(softmax_scale <= 0.0f || std::isfinite(softmax_scale))) return RQ_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(ref_k) || !aligned16(ref_v) || !aligned16(out))
+    return RQ_ERR_ALIGNMENT;
+  if (bits != 16 && (!aligned16(codes_k) || !aligned16(codes_v) || !aligned16(scales_k) ||
+                     !aligned16(scales_v)))
+    return RQ_ERR_ALIGNMENT;
+  if (!workspace || workspace_bytes < decode_workspace_bytes(*shape)) return RQ_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return RQ_ERR_ALIGNMENT;
+
+  const int sms = device_sm_count();
+  if (sms <= 0) return RQ_ERR_CUDA;
+  const DecodePlan pl = plan_decode(*shape, sms);
+  const int G = shape->q_heads / shape->kv_heads;
+  DecodeParams p;
+  p.q = q;
+  p.ref_k = ref_k;
+  p.ref_v = ref_v;
+  p.codes_k = bits == 16 ? nullptr : codes_k;
+  p.codes_v = bits == 16 ? nullptr : codes_v;
+  p.scales_k = bits == 16 ? nullptr : scales_k;
+  p.scales_v = bits == 16 ? nullptr : scales_v;
+  p.out = out;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  p.status = reinterpret_cast<uint32_t*>(ws);
+  p.counters = reinterpret_cast<uint32_t*>(ws + kWsHeaderBytes);
+  p.records = reinterpret_cast<float*>(ws + kWsHeaderBytes + ws_counters_bytes(pl.heads));
+  p.batch = shape->batch;
+  p.kv_heads = shape->kv_heads;
+  p.q_heads = shape->q_heads;
+  p.ctx = shape->ctx;
+  p.group = shape->group;
+  p.nt = pl.nt;
+  p.n_tiles = pl.n_tiles;
+  p.ctas = pl.ctas;
+  p.max_contrib = pl.max_contrib;
+  p.seed = seed;
+  const float sigma =
+      softmax_scale > 0.0f ? softmax_scale : 1.0f / std::sqrt((float)shape->head_dim);
+  p.score_scale = sigma * 1.4426950408889634f;   // log2(e)
+  cudaError_t e = launch_decode(shape->head_dim, G, bits, p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? RQ_OK : RQ_ERR_CUDA;
+}
+
+rq_status rq_workspace_status(const void* workspace, size_t workspace_bytes,
+                              uint32_t* host_status, void* stream) {
+  if (!workspace || !host_status || workspace_bytes < kWsHeaderBytes) return RQ_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(host_status, workspace, sizeof(uint32_t), cudaMemcpyDeviceToHost, st) !=
+      cudaSuccess)
+    return RQ_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return RQ_ERR_CUDA;
+  return RQ_OK;
+}
+
+}  // extern "C"

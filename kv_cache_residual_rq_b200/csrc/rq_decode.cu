@@ -1,0 +1,577 @@
+// rq_decode.cu -- fused ResidualQuant decode attention for sm_100a.
+//
+// Method: "ResidualQuant: KV Cache Quantization for Looped Transformers with
+// 2-Bit Residuals", Abstract -- decode reads the BF16 final-loop reference
+// plus each other loop's low-bit rotated residual and rebuilds that loop's
+// K/V efficiently; the saving is KV memory traffic.
+//
+// For one loop the kernel computes, per (batch b, query head j, kv head h):
+//   score_t = sigma * ( <q, refK_t> + sum_g s^K_t,g <q~_g, l^K_t,g> ),  q~ = Rot q
+//   out     = ( sum_t p_t refV_t + Rot^T sum_t p_t s^V_t l^V_t ) / sum_t p_t
+// so K_hat and V_hat are never built: the query is rotated once per head
+// and the V residual is accumulated in the rotated domain and rotated back
+// once per output row.  The level l = 2c - (2^b - 1) is split as
+// 2c - (2^b - 1): the code c enters the inner products and the constant is
+// folded into one per-lane offset (scores) or one per-lane weight sum (V).
+//
+// Structure (one launch per call):
+//   - P = 2 x SMs persistent CTAs.  The (head, tile) space -- heads are
+//     (b, h) pairs, tiles are 64-token runs of the context -- is numbered
+//     head-major and cut into P equal runs, one per CTA, so each CTA streams
+//     the same number of tiles.
+//   - Warp 4 is the producer: one lane issues cp.async.bulk copies of a
+//     tile's reference K/V rows, codes and scales (all contiguous runs in
+//     HBM) into a ring of shared-memory stages, completion tracked by
+//     mbarrier transaction counts.
+//   - Warps 0-3 consume: lanes split head_dim, so one 16- or 8-byte shared
+//     load per lane reads a token row; partial dot products are reduced with
+//     shfl.xor; online softmax in base 2 per warp.
+//   - At the end of a head's run the consumer warps merge their states and
+//     write one partial record; the last CTA to arrive for that head (an
+//     atomic ticket, no waiting) merges all records, applies the inverse
+//     rotation once and writes the output.
+// Every mbarrier wait is bounded; a wait that runs out raises the workspace
+// status word, and the kernel still finishes (its output is then invalid).
+#include <cmath>
+
+#include "rq_device.cuh"
+#include "rq_internal.h"
+
+namespace rq {
+namespace {
+
+constexpr int kConsumerWarps = 4;
+constexpr int kConsumerThreads = kConsumerWarps * 32;
+constexpr int kThreads = kConsumerThreads + 32;
+constexpr float kNegInf = -INFINITY;
+
+template <int D, int G, int BITS>
+struct Cfg {
+  static constexpr int DPL = (G >= 4) ? 4 : 8;              // dims per lane
+  static constexpr int LPT = D / DPL;                       // lanes per token
+  static constexpr int TPS = 32 / LPT;                      // tokens per warp step
+  static constexpr int TILE = kDecodeTile;
+  static constexpr int TPW = TILE / kConsumerWarps;         // tokens per warp per tile
+  static constexpr int STEPS = TPW / TPS;                   // warp steps per tile
+  static constexpr int CH = (G == 1) ? (STEPS < 8 ? STEPS : 8) : (STEPS < 4 ? STEPS : 4);
+  static constexpr bool RES = (BITS != 16);
+  static constexpr int KROW = D * 2;                        // bytes of a bf16 row
+  static constexpr int CROW = RES ? D * BITS / 8 : 0;       // code bytes per token
+  static constexpr int CWORDS = CROW / 4;
+  static constexpr int SC_BYTES = RES ? TILE * (2 * D / 32) + 32 : 0;
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + TILE * KROW;
+  static constexpr int OFF_CK = OFF_V + TILE * KROW;
+  static constexpr int OFF_CV = OFF_CK + TILE * CROW;
+  static constexpr int OFF_SK = OFF_CV + TILE * CROW;
+  static constexpr int OFF_SV = OFF_SK + SC_BYTES;
+  static constexpr int STAGE_BYTES = OFF_SV + SC_BYTES;
+  static constexpr int STAGES = RES ? 2 : 3;
+  static constexpr int RING_BYTES = STAGES * STAGE_BYTES;
+  // merge area: per warp and query row {m, l} + accRef[D] + accRes[D]
+  static constexpr int MERGE_FLOATS = kConsumerWarps * G * (2 + 2 * D);
+  static constexpr int QBUF_FLOATS = 2 * G * D;             // q and q~
+  static constexpr int SMEM_BYTES =
+      RING_BYTES + 4 * (MERGE_FLOATS + QBUF_FLOATS) + 2 * STAGES * 8 + 16;
+  static_assert(TPW % TPS == 0 && STEPS % CH == 0, "tile split");
+  static_assert(STAGE_BYTES % 16 == 0, "stage alignment");
+};
+
+__device__ __forceinline__ float code_as_float(uint32_t c) {
+  // c < 2^23: exact via the 2^23 exponent trick
+  return __uint_as_float(0x4B000000u | c) - 8388608.0f;
+}
+
+__device__ __forceinline__ void flag_error(uint32_t* status, uint32_t bit) {
+  atomicOr(status, bit);
+}
+
+template <int D, int G, int BITS>
+__global__ void __launch_bounds__(kThreads, 2)
+decode_kernel(const DecodeParams p) {
+  using C = Cfg<D, G, BITS>;
+  constexpr int DPL = C::DPL, LPT = C::LPT, TPS = C::TPS, TILE = C::TILE;
+  constexpr int STAGES = C::STAGES, CH = C::CH;
+  constexpr unsigned FULL = 0xffffffffu;
+  constexpr int TOPLVL = C::RES ? (1 << BITS) - 1 : 0;
+
+  extern __shared__ __align__(128) unsigned char smem[];
+  unsigned char* ring = smem;
+  float* merge = reinterpret_cast<float*>(smem + C::RING_BYTES);
+  float* qbuf = merge + C::MERGE_FLOATS;
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(qbuf + C::QBUF_FLOATS);
+  uint64_t* empty_bar = full_bar + STAGES;
+  volatile int* flags = reinterpret_cast<volatile int*>(empty_bar + STAGES);  // [0] abort, [1] last
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int cta = blockIdx.x;
+  if (cta >= p.ctas) return;
+
+  const long long tile_begin = (long long)cta * p.n_tiles / p.ctas;
+  const long long tile_end = (long long)(cta + 1) * p.n_tiles / p.ctas;
+  const int n_my = (int)(tile_end - tile_begin);
+
+  if (tid == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], kConsumerWarps);
+    }
+    flags[0] = 0;
+    flags[1] = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  const int T = p.ctx;
+  const int SB = (D / p.group) * 2;     // scale bytes per token
+
+  // ========================= producer warp ================================
+  if (warp == kConsumerWarps) {
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < n_my; ++i) {
+        const int s = i % STAGES;
+        if (i >= STAGES) {
+          if (!mbar_wait_bounded(&empty_bar[s], ((i / STAGES) - 1) & 1)) {
+            flag_error(p.status, 1u);
+            flags[0] = 1;
+            break;
+          }
+        }
+        if (flags[0]) break;
+        const long long tile = tile_begin + i;
+        const long long hd = tile / p.nt;
+        const int t0 = (int)(tile % p.nt) * TILE;
+        const int n = min(TILE, T - t0);
+        const size_t row = (size_t)hd * T + t0;       // first token row of the tile
+        unsigned char* st = ring + s * C::STAGE_BYTES;
+        uint32_t bytes = 2u * n * C::KROW;
+        size_t sc_lo = 0;
+        uint32_t sc_bytes = 0;
+        if constexpr (C::RES) {
+          const size_t start = row * SB;
+          sc_lo = start & ~(size_t)15;
+          sc_bytes = (uint32_t)(((start + (size_t)n * SB + 15) & ~(size_t)15) - sc_lo);
+          bytes += 2u * n * C::CROW + 2u * sc_bytes;
+        }
+        mbar_arrive_expect_tx(&full_bar[s], bytes);
+        bulk_g2s(st + C::OFF_K, p.ref_k + row * D, n * C::KROW, &full_bar[s]);
+        bulk_g2s(st + C::OFF_V, p.ref_v + row * D, n * C::KROW, &full_bar[s]);
+        if constexpr (C::RES) {
+          bulk_g2s(st + C::OFF_CK, p.codes_k + row * C::CWORDS, n * C::CROW, &full_bar[s]);
+          bulk_g2s(st + C::OFF_CV, p.codes_v + row * C::CWORDS, n * C::CROW, &full_bar[s]);
+          bulk_g2s(st + C::OFF_SK, reinterpret_cast<const unsigned char*>(p.scales_k) + sc_lo,
+                   sc_bytes, &full_bar[s]);
+          bulk_g2s(st + C::OFF_SV, reinterpret_cast<const unsigned char*>(p.scales_v) + sc_lo,
+                   sc_bytes, &full_bar[s]);
+        }
+        ++issued;
+      }
+      // never leave with copies in flight into this CTA's shared memory
+      for (int j = (issued > STAGES ? issued - STAGES : 0); j < issued; ++j)
+        if (!mbar_wait_bounded(&full_bar[j % STAGES], (j / STAGES) & 1)) flag_error(p.status, 2u);
+    }
+    return;
+  }
+
+  // ========================= consumer warps ===============================
+  const int li = lane % LPT;          // lane within its token
+  const int slot = lane / LPT;        // token slot within a warp step
+  const int dim0 = li * DPL;          // first dim this lane owns
+  const float score_scale = p.score_scale;
+
+  // per-lane constants of the current head
+  float qa[G][DPL];                   // score_scale * q
+  float qc[G][DPL];                   // 2 * score_scale * q~
+  float qoff[G];                      // (2^b - 1) * score_scale * sum q~ (lane's dims)
+  // running state
+  float m_run[G], l_run[G], accV[G][DPL], accC[G][DPL], wsum[G];
+
+  auto reset_state = [&]() {
+#pragma unroll
+    for (int r = 0; r < G; ++r) {
+      m_run[r] = kNegInf;
+      l_run[r] = 0.0f;
+      wsum[r] = 0.0f;
+#pragma unroll
+      for (int k = 0; k < DPL; ++k) {
+        accV[r][k] = 0.0f;
+        accC[r][k] = 0.0f;
+      }
+    }
+  };
+
+  // load and rotate the G query rows of head hd; all consumer threads
+  auto setup_head = [&](long long hd) {
+    const int b = (int)(hd / p.kv_heads);
+    const int h = (int)(hd % p.kv_heads);
+    float* qs = qbuf;              // [G][D] raw q
+    float* qt = qbuf + G * D;      // [G][D] rotated
+    named_bar_sync(1, kConsumerThreads);          // previous users of qbuf done
+    for (int e = tid; e < G * D; e += kConsumerThreads) {
+      const int r = e / D, i = e % D;
+      const uint16_t raw = p.q[((size_t)b * p.q_heads + (size_t)h * G + r) * D + i];
+      const float v = __uint_as_float((uint32_t)raw << 16);
+      qs[e] = v;
+      qt[e] = flip_sign(v, sign_bit(p.seed, i));
+    }
+    for (int hs = 1; hs < D; hs <<= 1) {
+      named_bar_sync(1, kConsumerThreads);
+      for (int e = tid; e < G * D / 2; e += kConsumerThreads) {
+        const int r = e / (D / 2), pr = e % (D / 2);
+        const int i = (pr / hs) * 2 * hs + (pr % hs);
+        float* row = qt + r * D;
+        const float a = row[i], c = row[i + hs];
+        row[i] = a + c;
+        row[i + hs] = a - c;
+      }
+    }
+    named_bar_sync(1, kConsumerThreads);
+    const float cd = rot_scale<D>();
+#pragma unroll
+    for (int r = 0; r < G; ++r) {
+      float sum = 0.0f;
+#pragma unroll
+      for (int k = 0; k < DPL; ++k) {
+        qa[r][k] = score_scale * qs[r * D + dim0 + k];
+        const float t = cd * qt[r * D + dim0 + k];
+        qc[r][k] = 2.0f * score_scale * t;
+        sum += t;
+      }
+      qoff[r] = (float)TOPLVL * score_scale * sum;
+    }
+  };
+
+  // merge the 4 warps' states, write the head's partial record, and if this
+  // CTA is the last contributor, finish the head
+  auto flush_head = [&](long long hd) {
+    const int b = (int)(hd / p.kv_heads);
+    const int h = (int)(hd % p.kv_heads);
+    // fold the token slots of the warp together
+#pragma unroll
+    for (int r = 0; r < G; ++r) {
+#pragma unroll
+      for (int m = LPT; m < 32; m <<= 1) {
+        l_run[r] += __shfl_xor_sync(FULL, l_run[r], m);
+        if constexpr (C::RES) wsum[r] += __shfl_xor_sync(FULL, wsum[r], m);
+#pragma unroll
+        for (int k = 0; k < DPL; ++k) {
+          accV[r][k] += __shfl_xor_sync(FULL, accV[r][k], m);
+          if constexpr (C::RES) accC[r][k] += __shfl_xor_sync(FULL, accC[r][k], m);
+        }
+      }
+    }
+    named_bar_sync(1, kConsumerThreads);          // merge area free
+    float* mw = merge + warp * G * (2 + 2 * D);
+    if (slot == 0) {
+#pragma unroll
+      for (int r = 0; r < G; ++r) {
+        float* rec = mw + r * (2 + 2 * D);
+        if (li == 0) {
+          rec[0] = m_run[r];
+          rec[1] = l_run[r];
+        }
+#pragma unroll
+        for (int k = 0; k < DPL; ++k) {
+          rec[2 + dim0 + k] = accV[r][k];
+          rec[2 + D + dim0 + k] =
+              C::RES ? (2.0f * accC[r][k] - (float)TOPLVL * wsum[r]) : 0.0f;
+        }
+      }
+    }
+    named_bar_sync(1, kConsumerThreads);
+
+    // which records belong to this head, and which one is ours
+    const long long f = hd * p.nt, e = f + p.nt - 1;
+    const int c_first = (int)(((f + 1) * p.ctas - 1) / p.n_tiles);
+    const int c_last = (int)(((e + 1) * p.ctas - 1) / p.n_tiles);
+    const int ncontrib = c_last - c_first + 1;
+    const int j = cta - c_first;
+    if (j < 0 || j >= p.max_contrib || ncontrib > p.max_contrib) {
+      if (tid == 0) flag_error(p.status, 4u);
+      return;
+    }
+    float* recs = p.records + (size_t)hd * p.max_contrib * G * (4 + 2 * D);
+    for (int eidx = tid; eidx < G * (2 * D + 2); eidx += kConsumerThreads) {
+      const int r = eidx / (2 * D + 2), q = eidx % (2 * D + 2);
+      float M = kNegInf;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w)
+        M = fmaxf(M, merge[(w * G + r) * (2 + 2 * D)]);
+      float* out_rec = recs + ((size_t)j * G + r) * (4 + 2 * D);
+      if (q == 0) {
+        out_rec[0] = M;
+      } else {
+        float acc = 0.0f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) {
+          const float* mr = merge + (w * G + r) * (2 + 2 * D);
+          const float wt = (mr[0] == kNegInf) ? 0.0f : exp2f(mr[0] - M);
+          acc += wt * mr[q];
+        }
+        out_rec[q == 1 ? 1 : q + 2] = acc;   // l at 1; accRef/accRes from 4
+      }
+    }
+    __threadfence();
+    named_bar_sync(1, kConsumerThreads);
+    if (tid == 0) {
+      const uint32_t old = atomicAdd(&p.counters[hd], 1u);
+      const int last = (old == (uint32_t)(ncontrib - 1));
+      if (last) {
+        p.counters[hd] = 0u;      // ready for the next call
+        __threadfence();
+      }
+      flags[1] = last;
+    }
+    named_bar_sync(1, kConsumerThreads);
+    if (!flags[1]) return;
+
+    // ---- last contributor: merge all records of the head, finish ----
+    float* zres = merge;          // [G][D] rotated-domain residual sums
+    float* zref = merge + G * D;  // [G][D]
+    float* lsum = merge + 2 * G * D;   // [G]
+    for (int eidx = tid; eidx < G * D; eidx += kConsumerThreads) {
+      const int r = eidx / D, i = eidx % D;
+      float M = kNegInf;
+      for (int c = 0; c < ncontrib; ++c)
+        M = fmaxf(M, __ldcg(recs + ((size_t)c * G + r) * (4 + 2 * D)));
+      float aref = 0.0f, ares = 0.0f, l = 0.0f;
+      for (int c = 0; c < ncontrib; ++c) {
+        const float* rc = recs + ((size_t)c * G + r) * (4 + 2 * D);
+        const float mc = __ldcg(rc);
+        const float wt = (mc == kNegInf) ? 0.0f : exp2f(mc - M);
+        l += wt * __ldcg(rc + 1);
+        aref += wt * __ldcg(rc + 4 + i);
+        if constexpr (C::RES) ares += wt * __ldcg(rc + 4 + D + i);
+      }
+      zref[eidx] = aref;
+      zres[eidx] = ares;
+      if (i == 0) lsum[r] = l;
+    }
+    if constexpr (C::RES) {
+      // Rot^T z = D (c_d H z): butterflies, then scale and signs
+      for (int hs = 1; hs < D; hs <<= 1) {
+        named_bar_sync(1, kConsumerThreads);
+        for (int eidx = tid; eidx < G * D / 2; eidx += kConsumerThreads) {
+          const int r = eidx / (D / 2), pr = eidx % (D / 2);
+          const int i = (pr / hs) * 2 * hs + (pr % hs);
+          float* row = zres + r * D;
+          const float a = row[i], c = row[i + hs];
+          row[i] = a + c;
+          row[i + hs] = a - c;
+        }
+      }
+    }
+    named_bar_sync(1, kConsumerThreads);
+    const float cd = rot_scale<D>();
+    for (int eidx = tid; eidx < G * D; eidx += kConsumerThreads) {
+      const int r = eidx / D, i = eidx % D;
+      float num = zref[eidx];
+      if constexpr (C::RES) num += flip_sign(cd * zres[eidx], sign_bit(p.seed, i));
+      p.out[((size_t)b * p.q_heads + (size_t)h * G + r) * D + i] = num / lsum[r];
+    }
+  };
+
+  // ---- main loop over this CTA's tiles ----
+  long long cur_head = -1;
+  bool aborted = false;
+  reset_state();
+  for (int i = 0; i < n_my; ++i) {
+    const long long tile = tile_begin + i;
+    const long long hd = tile / p.nt;
+    if (hd != cur_head) {
+      if (cur_head >= 0) {
+        flush_head(cur_head);
+        reset_state();
+      }
+      cur_head = hd;
+      setup_head(hd);
+    }
+    const int s = i % STAGES;
+    bool ok = !aborted && !flags[0];
+    if (ok) ok = mbar_wait_bounded(&full_bar[s], (i / STAGES) & 1);
+    ok = __all_sync(FULL, ok);            // one decision per warp
+    if (!ok) {
+      if (!aborted && lane == 0) flag_error(p.status, 8u);
+      aborted = true;
+      flags[0] = 1;
+    }
+    if (!aborted) {
+      const int t0 = (int)(tile % p.nt) * TILE;
+      const int n = min(TILE, T - t0);
+      const unsigned char* st = ring + s * C::STAGE_BYTES;
+      const size_t row = (size_t)hd * T + t0;
+      const int sc_off = (int)((row * SB) & 15);
+      const int grp = dim0 / p.group;
+      const int cw = (dim0 * BITS) / 32;                   // code word of this lane
+      const int csh = (dim0 * BITS) % 32;                  // bit offset in it
+
+#pragma unroll 1
+      for (int c0 = 0; c0 < C::STEPS; c0 += CH) {
+        float sc[G][CH];
+        // ---- scores ----
+#pragma unroll
+        for (int u = 0; u < CH; ++u) {
+          const int tok = warp * C::TPW + (c0 + u) * TPS + slot;
+          float kf[DPL];
+          const unsigned char* kp = st + C::OFF_K + tok * C::KROW + dim0 * 2;
+          if constexpr (DPL == 8) {
+            const uint4 w = *reinterpret_cast<const uint4*>(kp);
+            kf[0] = bf16lo(w.x); kf[1] = bf16hi(w.x); kf[2] = bf16lo(w.y); kf[3] = bf16hi(w.y);
+            kf[4] = bf16lo(w.z); kf[5] = bf16hi(w.z); kf[6] = bf16lo(w.w); kf[7] = bf16hi(w.w);
+          } else {
+            const uint2 w = *reinterpret_cast<const uint2*>(kp);
+            kf[0] = bf16lo(w.x); kf[1] = bf16hi(w.x); kf[2] = bf16lo(w.y); kf[3] = bf16hi(w.y);
+          }
+          float dot[G];
+#pragma unroll
+          for (int r = 0; r < G; ++r) {
+            dot[r] = 0.0f;
+#pragma unroll
+            for (int k = 0; k < DPL; ++k) dot[r] = fmaf(qa[r][k], kf[k], dot[r]);
+          }
+          if constexpr (C::RES) {
+            const uint32_t word =
+                reinterpret_cast<const uint32_t*>(st + C::OFF_CK)[tok * C::CWORDS + cw] >> csh;
+            const float s_k = __half2float(__ushort_as_half(
+                *reinterpret_cast<const uint16_t*>(st + C::OFF_SK + sc_off + tok * SB + grp * 2)));
+            float cf[DPL];
+#pragma unroll
+            for (int k = 0; k < DPL; ++k) cf[k] = code_as_float((word >> (BITS * k)) & ((1u << BITS) - 1));
+#pragma unroll
+            for (int r = 0; r < G; ++r) {
+              float res = -qoff[r];
+#pragma unroll
+              for (int k = 0; k < DPL; ++k) res = fmaf(qc[r][k], cf[k], res);
+              dot[r] = fmaf(s_k, res, dot[r]);
+            }
+          }
+#pragma unroll
+          for (int r = 0; r < G; ++r) {
+#pragma unroll
+            for (int m = 1; m < LPT; m <<= 1) dot[r] += __shfl_xor_sync(FULL, dot[r], m);
+            sc[r][u] = (tok < n) ? dot[r] : kNegInf;
+          }
+        }
+        // ---- online softmax (base 2) ----
+        float pw[G][CH];
+#pragma unroll
+        for (int r = 0; r < G; ++r) {
+          float mc = sc[r][0];
+#pragma unroll
+          for (int u = 1; u < CH; ++u) mc = fmaxf(mc, sc[r][u]);
+#pragma unroll
+          for (int m = LPT; m < 32; m <<= 1) mc = fmaxf(mc, __shfl_xor_sync(FULL, mc, m));
+          const float m_new = fmaxf(m_run[r], mc);
+          if (m_new != m_run[r]) {
+            const float alpha = (m_run[r] == kNegInf) ? 0.0f : exp2f(m_run[r] - m_new);
+            l_run[r] *= alpha;
+            if constexpr (C::RES) wsum[r] *= alpha;
+#pragma unroll
+            for (int k = 0; k < DPL; ++k) {
+              accV[r][k] *= alpha;
+              if constexpr (C::RES) accC[r][k] *= alpha;
+            }
+            m_run[r] = m_new;
+          }
+#pragma unroll
+          for (int u = 0; u < CH; ++u) {
+            pw[r][u] = (sc[r][u] == kNegInf) ? 0.0f : exp2f(sc[r][u] - m_new);
+            l_run[r] += pw[r][u];
+          }
+        }
+        // ---- values ----
+#pragma unroll
+        for (int u = 0; u < CH; ++u) {
+          const int tok = warp * C::TPW + (c0 + u) * TPS + slot;
+          if (tok < n) {
+            float vf[DPL];
+            const unsigned char* vp = st + C::OFF_V + tok * C::KROW + dim0 * 2;
+            if constexpr (DPL == 8) {
+              const uint4 w = *reinterpret_cast<const uint4*>(vp);
+              vf[0] = bf16lo(w.x); vf[1] = bf16hi(w.x); vf[2] = bf16lo(w.y); vf[3] = bf16hi(w.y);
+              vf[4] = bf16lo(w.z); vf[5] = bf16hi(w.z); vf[6] = bf16lo(w.w); vf[7] = bf16hi(w.w);
+            } else {
+              const uint2 w = *reinterpret_cast<const uint2*>(vp);
+              vf[0] = bf16lo(w.x); vf[1] = bf16hi(w.x); vf[2] = bf16lo(w.y); vf[3] = bf16hi(w.y);
+            }
+#pragma unroll
+            for (int r = 0; r < G; ++r) {
+#pragma unroll
+              for (int k = 0; k < DPL; ++k) accV[r][k] = fmaf(pw[r][u], vf[k], accV[r][k]);
+            }
+            if constexpr (C::RES) {
+              const uint32_t word =
+                  reinterpret_cast<const uint32_t*>(st + C::OFF_CV)[tok * C::CWORDS + cw] >> csh;
+              const float s_v = __half2float(__ushort_as_half(
+                  *reinterpret_cast<const uint16_t*>(st + C::OFF_SV + sc_off + tok * SB + grp * 2)));
+              float cf[DPL];
+#pragma unroll
+              for (int k = 0; k < DPL; ++k) cf[k] = code_as_float((word >> (BITS * k)) & ((1u << BITS) - 1));
+#pragma unroll
+              for (int r = 0; r < G; ++r) {
+                const float wv = pw[r][u] * s_v;
+                wsum[r] += wv;
+#pragma unroll
+                for (int k = 0; k < DPL; ++k) accC[r][k] = fmaf(wv, cf[k], accC[r][k]);
+              }
+            }
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty_bar[s]);
+  }
+  // After an abort the flush still runs (on whatever the state holds) so that
+  // every consumer thread takes the same barrier sequence; the status word
+  // marks the output invalid.
+  if (cur_head >= 0) flush_head(cur_head);
+}
+
+template <int D, int G, int BITS>
+cudaError_t launch_decode_t(const DecodeParams& p, cudaStream_t stream) {
+  using C = Cfg<D, G, BITS>;
+  static bool attr_set = false;   // per process; harmless to repeat
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, G, BITS>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  decode_kernel<D, G, BITS><<<p.ctas, kThreads, C::SMEM_BYTES, stream>>>(p);
+  return cudaGetLastError();
+}
+
+template <int D, int G>
+cudaError_t launch_decode_g(int bits, const DecodeParams& p, cudaStream_t stream) {
+  if (bits == 2) return launch_decode_t<D, G, 2>(p, stream);
+  if (bits == 4) return launch_decode_t<D, G, 4>(p, stream);
+  if (bits == 16) return launch_decode_t<D, G, 16>(p, stream);
+  return cudaErrorInvalidValue;
+}
+
+template <int D>
+cudaError_t launch_decode_d(int G, int bits, const DecodeParams& p, cudaStream_t stream) {
+  switch (G) {
+    case 1: return launch_decode_g<D, 1>(bits, p, stream);
+    case 2: return launch_decode_g<D, 2>(bits, p, stream);
+    case 4: return launch_decode_g<D, 4>(bits, p, stream);
+    case 8: return launch_decode_g<D, 8>(bits, p, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_decode(int head_dim, int G, int bits, const DecodeParams& p,
+                          cudaStream_t stream) {
+  if (head_dim == 128) return launch_decode_d<128>(G, bits, p, stream);
+  if (head_dim == 64) return launch_decode_d<64>(G, bits, p, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace rq

@@ -1,0 +1,89 @@
+// rq_internal.h -- launch parameters shared by the C ABI layer and the kernels.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "rq.h"
+
+namespace rq {
+
+// ---------------------------------------------------------------------------
+// encoder
+// ---------------------------------------------------------------------------
+struct EncodeParams {
+  const uint16_t* x[RQ_MAX_LOOPS];   // bf16 rows of each non-final loop
+  uint32_t* codes[RQ_MAX_LOOPS];
+  uint16_t* scales[RQ_MAX_LOOPS];
+  int bits[RQ_MAX_LOOPS];
+  const uint16_t* ref;               // bf16 rows of the final loop
+  long long n_rows;                  // rows of head_dim elements
+  int n_loops;
+  uint64_t seed;
+};
+
+cudaError_t launch_encode(int head_dim, int group, const EncodeParams& p, int num_sms,
+                          cudaStream_t stream);
+
+// ---------------------------------------------------------------------------
+// decode attention
+// ---------------------------------------------------------------------------
+
+// Work split of one decode call.  The context of each (batch, kv head) --
+// a "head" -- is cut into tiles of kDecodeTile tokens; the heads' tiles are
+// numbered head-major and the P CTAs take equal contiguous runs of that
+// numbering, so every CTA streams the same number of tiles whatever the
+// shape.  A head touched by several CTAs is merged by the last to finish.
+constexpr int kDecodeTile = 64;
+constexpr int kDecodeCtasPerSm = 2;
+constexpr int kDecodeMaxCtas = 1024;     // bound used to size the workspace
+
+struct DecodePlan {
+  long long heads;      // batch * kv_heads
+  int nt;               // tiles per head
+  long long n_tiles;    // heads * nt
+  int ctas;             // P
+  int max_contrib;      // partial records reserved per head
+};
+
+// Host arithmetic shared by the size query and the launch.
+DecodePlan plan_decode(const rq_shape& s, int num_sms);
+size_t decode_workspace_bytes(const rq_shape& s);
+
+// Workspace layout: [status u32, pad to 16][counters u32 per head, pad to 16]
+//                   [partial records: heads * max_contrib * G records]
+// A record is {m, l, pad, pad, accRef[d], accRes[d]} as fp32.
+constexpr size_t kWsHeaderBytes = 16;
+inline size_t ws_counters_bytes(long long heads) {
+  return ((size_t)heads * 4 + 15) / 16 * 16;
+}
+inline size_t ws_record_floats(int head_dim) { return 4 + 2 * (size_t)head_dim; }
+
+struct DecodeParams {
+  const uint16_t* q;
+  const uint16_t* ref_k;
+  const uint16_t* ref_v;
+  const uint32_t* codes_k;
+  const uint32_t* codes_v;
+  const uint16_t* scales_k;
+  const uint16_t* scales_v;
+  float* out;
+  uint32_t* status;
+  uint32_t* counters;
+  float* records;
+  int batch, kv_heads, q_heads, ctx, group;
+  int nt;
+  long long n_tiles;
+  int ctas;
+  int max_contrib;
+  uint64_t seed;
+  float score_scale;     // softmax scale * log2(e)
+};
+
+cudaError_t launch_decode(int head_dim, int G, int bits, const DecodeParams& p,
+                          cudaStream_t stream);
+
+int device_sm_count();   // SMs of the current device, cached per device
+
+}  // namespace rq

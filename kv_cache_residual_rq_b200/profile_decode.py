@@ -1,0 +1,67 @@
+"""Small, self-contained decode case for profiler captures.
+
+    python -m kv_cache_residual_rq_b200.profile_decode [--workload NAME] [--calls N] [--bits B]
+
+Builds ONE layer of a workload on cuda:0 (for the Ouro-shaped decode: 537 MB
+of reference K/V plus 84 MB of codes and scales, above the 126 MB L2),
+encodes it, and runs the decode kernel `--calls` times on the same inputs,
+so a profiler can capture a handful of launches of exactly the kernel the
+benchmark times without holding the whole 24-layer cache on the device.
+"""
+import argparse
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def main(argv=None):
+    import torch
+    import kv_cache_residual_rq_b200 as rq
+    from kv_cache_residual_rq_b200 import synth
+
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--workload", default="ouro1.4b_decode")
+    ap.add_argument("--calls", type=int, default=4)
+    ap.add_argument("--bits", type=int, default=0, help="0: the workload's first loop")
+    ap.add_argument("--encode", action="store_true", help="also time rq_encode of the layer")
+    args = ap.parse_args(argv)
+    w = synth.BY_NAME[args.workload]
+    bits = args.bits or w.bits[0]
+    dev = torch.device("cuda:0")
+    refk = synth.reference(w, 0, 0, dev)
+    refv = synth.reference(w, 0, 1, dev)
+    q = synth.query(w, 0, 1, dev)
+    ck = cv = sk = sv = None
+    if bits != 16:
+        xk = [synth.loop_kv(w, 0, 0, l, refk) for l in range(1, w.loops)]
+        xv = [synth.loop_kv(w, 0, 1, l, refv) for l in range(1, w.loops)]
+        bl = [bits] * (w.loops - 1)
+        cks, sks = rq.encode(xk, refk, bl, w.group, w.seed)
+        cvs, svs = rq.encode(xv, refv, bl, w.group, w.seed)
+        if args.encode:
+            for _ in range(args.calls):
+                rq.encode(xk, refk, bl, w.group, w.seed)
+        ck, cv, sk, sv = cks[0], cvs[0], sks[0], svs[0]
+        del xk, xv
+    shape = rq.make_shape(w.batch, w.kv_heads, w.ctx, w.head_dim, w.group, w.q_heads)
+    ws = rq.alloc_workspace(shape, dev)
+    out = torch.empty((w.batch, w.q_heads, w.head_dim), dtype=torch.float32, device=dev)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    times = []
+    for _ in range(args.calls):
+        start.record()
+        rq.decode_attention(q, refk, refv, ck, cv, sk, sv, bits, w.group, w.seed, out=out,
+                            workspace=ws)
+        end.record()
+        torch.cuda.synchronize()
+        times.append(start.elapsed_time(end))
+    print(f"{w.name} bits={bits}: decode call ms {['%.3f' % t for t in times]}, "
+          f"status {rq.rq_workspace_status(ws)}")
+
+
+if __name__ == "__main__":
+    main()

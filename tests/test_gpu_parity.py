@@ -1,0 +1,272 @@
+"""Parity of the CUDA path (librq.so, through its C ABI) with the CPU oracle.
+
+Inputs are the seeded synthetic workloads; both sides get exactly the same
+bf16 tensors (the oracle a host copy).  The oracle never sees a value the
+GPU produced: for decode checks it encodes the sampled heads itself.
+
+Bars (from the method's specification of this build):
+  codes   bit-identical
+  scales  within 1e-3 relative (one fp16 step; one subnormal step near 0)
+  outputs within 1e-2 max-abs of the fp64 oracle (fp32 accumulation)
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import kv_cache_residual_rq_b200 as rq
+from kv_cache_residual_rq_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+OUT_TOL = 1e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def cuda_ready():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from kv_cache_residual_rq_b200 import build
+    build.build()
+    rq.lib()
+    torch.cuda.init()
+
+
+def u16(t):
+    return t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def codes_view(buf, shape_prefix, d, bits):
+    wpr = d * bits // 32
+    n = int(np.prod(shape_prefix)) * wpr
+    return buf[: n * 4].view(torch.int32).view(*shape_prefix, wpr)
+
+
+def scales_view(buf, shape_prefix, d, group):
+    n = int(np.prod(shape_prefix)) * (d // group)
+    return buf[: n * 2].view(torch.int16).view(*shape_prefix, d // group)
+
+
+def check_scales(got_u16, want_u16):
+    g = np.array([oracle.f16_to_f64(int(h)) for h in got_u16.ravel()])
+    w = np.array([oracle.f16_to_f64(int(h)) for h in want_u16.ravel()])
+    bad = np.abs(g - w) > np.maximum(1e-3 * np.abs(w), 2.0 ** -24)
+    assert not bad.any(), f"{bad.sum()} scales off, e.g. {g[bad][:4]} vs {w[bad][:4]}"
+
+
+# ---------------------------------------------------------------------------
+# encoder
+# ---------------------------------------------------------------------------
+
+def encode_layer(w, layer, kind, device="cuda", batch=None, ctx=None):
+    ref = synth.reference(w, layer, kind, device, batch=batch, ctx=ctx)
+    loops = [synth.loop_kv(w, layer, kind, l, ref) for l in range(1, w.loops)]
+    codes, scales = rq.encode(loops, ref, list(w.bits), w.group, seed=w.seed)
+    return ref, loops, codes, scales
+
+
+def compare_encode_rows(w, ref, loops, codes, scales, rows):
+    """rows: flat row indices into [B*Hkv*T]."""
+    d = w.head_dim
+    rows_t = torch.as_tensor(rows, device=ref.device)
+    r_flat = ref.reshape(-1, d)
+    ties = 0
+    for l, bits in enumerate(w.bits):
+        if bits == 16:
+            assert codes[l] is None and scales[l] is None
+            continue
+        x_flat = loops[l].reshape(-1, d)
+        gw = codes_view(codes[l], (r_flat.shape[0],), d, bits)[rows_t]
+        gs = scales_view(scales[l], (r_flat.shape[0],), d, w.group)[rows_t]
+        want_w, want_s, t = oracle.encode_rows_f32(u16(x_flat[rows_t]), u16(r_flat[rows_t]), bits,
+                                                   w.group, w.seed)
+        ties += t
+        got_w = gw.cpu().numpy().view(np.uint32)
+        mism = (got_w != want_w)
+        assert not mism.any(), f"loop {l + 1}: {mism.sum()} code words differ"
+        check_scales(gs.cpu().numpy().view(np.uint16), want_s)
+    return ties
+
+
+def test_encode_tiny_full():
+    w = synth.TINY
+    for kind in (0, 1):
+        ref, loops, codes, scales = encode_layer(w, 0, kind)
+        n = ref.numel() // w.head_dim
+        ties = compare_encode_rows(w, ref, loops, codes, scales, np.arange(n))
+        print(f"tiny kind={kind}: {n} rows x {w.loops - 1} loops bit-exact, ties={ties}")
+
+
+@pytest.mark.parametrize("name", ["ouro1.4b_decode", "mixed_precision_32k", "deep_loop_gqa",
+                                  "encode_prefill_32k"])
+def test_encode_full_size_sampled(name):
+    w = synth.BY_NAME[name]
+    layer = w.layers - 1
+    ref, loops, codes, scales = encode_layer(w, layer, 1)
+    n = ref.numel() // w.head_dim
+    rng = np.random.default_rng(7)
+    rows = np.unique(np.concatenate([rng.integers(0, n, 3000), [0, 1, n - 1]]))
+    ties = compare_encode_rows(w, ref, loops, codes, scales, rows)
+    print(f"{name}: {rows.size} sampled rows bit-exact, ties={ties}")
+
+
+@pytest.mark.parametrize("d,group,bits", [(64, 64, 2), (128, 64, 4), (64, 32, 4)])
+@pytest.mark.parametrize("ctx", [1, 3, 65])
+def test_encode_edge_shapes(d, group, bits, ctx):
+    w = synth.Workload("edge", 3, 1, 2, ctx, 4, 4, d, group, (bits, 16), (0.2, 0.1), 11)
+    ref, loops, codes, scales = encode_layer(w, 0, 0)
+    n = ref.numel() // d
+    compare_encode_rows(w, ref, loops, codes, scales, np.arange(n))
+
+
+def test_encode_zero_residual_and_bf16_loop_untouched():
+    w = synth.Workload("zero", 3, 1, 1, 100, 2, 2, 128, 32, (2, 16), (0.0, 0.0), 5)
+    ref = synth.reference(w, 0, 0)
+    shape = rq.make_shape(1, 2, 100, 128, 32)
+    codes = rq.alloc_codes(shape, 2)
+    scales = rq.alloc_scales(shape, 2)
+    codes.fill_(0xAB)
+    scales.fill_(0xCD)
+    rq.rq_encode(shape, [ref, None], ref, [2, 16], 5, [codes, None], [scales, None])
+    torch.cuda.synchronize()
+    cw = codes_view(codes, (200,), 128, 2).cpu().numpy().view(np.uint32)
+    assert (cw == 0xAAAAAAAA).all()            # every code 2 = level +1
+    assert (scales_view(scales, (200,), 128, 32) == 0).all()
+    # ctx = 0 is a no-op that writes nothing
+    empty = rq.make_shape(1, 2, 0, 128, 32)
+    rq.rq_encode(empty, [ref], ref, [2], 5, [codes], [scales])
+    torch.cuda.synchronize()
+
+
+# ---------------------------------------------------------------------------
+# decode attention
+# ---------------------------------------------------------------------------
+
+def oracle_head(w, q, refk, refv, xk, xv, bits, b, h):
+    """Oracle decode of one (b, kv head): encodes that head itself."""
+    G, d = w.G, w.head_dim
+    qh = u16(q[b, h * G:(h + 1) * G])
+    rk = u16(refk[b, h])
+    rv = u16(refv[b, h])
+    if bits == 16:
+        return oracle.decode_attention_f64(qh, rk, rv, None, None, None, None, 16, w.group, w.seed)
+    ck, sk, _ = oracle.encode_rows_f32(u16(xk[b, h]), rk, bits, w.group, w.seed)
+    cv, sv, _ = oracle.encode_rows_f32(u16(xv[b, h]), rv, bits, w.group, w.seed)
+    return oracle.decode_attention_f64(qh, rk, rv, ck, cv, sk, sv, bits, w.group, w.seed)
+
+
+def run_decode_loop(w, layer, loop, batch=None, ctx=None):
+    """GPU decode for 1-based `loop` (loop == w.loops is the reference)."""
+    refk = synth.reference(w, layer, 0, batch=batch, ctx=ctx)
+    refv = synth.reference(w, layer, 1, batch=batch, ctx=ctx)
+    q = synth.query(w, layer, loop, batch=batch)
+    if loop == w.loops:
+        out = rq.decode_attention(q, refk, refv, None, None, None, None, 16, w.group, w.seed)
+        return q, refk, refv, None, None, 16, out
+    bits = w.bits[loop - 1]
+    xk = synth.loop_kv(w, layer, 0, loop, refk)
+    xv = synth.loop_kv(w, layer, 1, loop, refv)
+    (ck,), (sk,) = rq.encode([xk], refk, [bits], w.group, w.seed)
+    (cv,), (sv,) = rq.encode([xv], refv, [bits], w.group, w.seed)
+    out = rq.decode_attention(q, refk, refv, ck, cv, sk, sv, bits, w.group, w.seed)
+    return q, refk, refv, xk, xv, bits, out
+
+
+def assert_heads_match(w, res, heads):
+    q, refk, refv, xk, xv, bits, out = res
+    torch.cuda.synchronize()
+    worst = 0.0
+    for b, h in heads:
+        want = oracle_head(w, q, refk, refv, xk, xv, bits, b, h)
+        got = out[b, h * w.G:(h + 1) * w.G].double().cpu().numpy()
+        err = np.abs(got - want).max()
+        worst = max(worst, err)
+        assert err <= OUT_TOL, f"head ({b},{h}) max-abs {err}"
+    return worst
+
+
+@pytest.mark.parametrize("loop", [1, 2, 3, 4])
+def test_decode_tiny_full(loop):
+    w = synth.TINY
+    res = run_decode_loop(w, 0, loop)
+    worst = assert_heads_match(w, res, [(0, h) for h in range(w.kv_heads)])
+    print(f"tiny loop {loop}: max-abs {worst:.2e}")
+
+
+@pytest.mark.parametrize("name,loops", [("ouro1.4b_decode", (1, 3, 4)),
+                                        ("mixed_precision_32k", (1, 2, 4)),
+                                        ("deep_loop_gqa", (1, 7, 8))])
+def test_decode_full_size_sampled(name, loops):
+    w = synth.BY_NAME[name]
+    rng = np.random.default_rng(3)
+    for loop in loops:
+        res = run_decode_loop(w, 0, loop)
+        heads = {(0, 0), (w.batch - 1, w.kv_heads - 1)}
+        heads |= {(int(rng.integers(w.batch)), int(rng.integers(w.kv_heads))) for _ in range(2)}
+        worst = assert_heads_match(w, res, sorted(heads))
+        print(f"{name} loop {loop}: {len(heads)} heads, max-abs {worst:.2e}")
+        del res
+        torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("d,group,G,bits,ctx,batch,hkv", [
+    (128, 32, 1, 2, 1, 1, 1),          # single token
+    (128, 32, 1, 2, 65, 3, 2),         # one full tile + 1
+    (128, 64, 2, 4, 1000, 2, 3),       # ragged, odd head count
+    (64, 32, 8, 2, 130, 1, 2),         # G = 8
+    (64, 64, 4, 4, 257, 2, 1),
+    (128, 32, 1, 16, 333, 2, 2),       # reference loop, ragged
+    (128, 32, 4, 2, 20000, 1, 1),      # one head spread over many CTAs
+])
+def test_decode_edge_shapes(d, group, G, bits, ctx, batch, hkv):
+    bl = (bits, 16) if bits != 16 else (2, 16)
+    w = synth.Workload("edge", 3, 1, batch, ctx, hkv * G, hkv, d, group, bl, (0.25, 0.1), 21)
+    loop = 1 if bits != 16 else 3
+    res = run_decode_loop(w, 0, loop)
+    heads = [(b, h) for b in range(batch) for h in range(hkv)]
+    worst = assert_heads_match(w, res, heads)
+    print(f"edge {d}/{group}/G{G}/b{bits}/T{ctx}: max-abs {worst:.2e}")
+
+
+def test_zero_scales_reproduce_reference_loop_bit_for_bit():
+    # a residual loop equal to the reference encodes to all-zero scales; its
+    # decode must then be bit-identical to decoding the reference loop
+    w = synth.OURO
+    refk = synth.reference(w, 2, 0, batch=4, ctx=1500)
+    refv = synth.reference(w, 2, 1, batch=4, ctx=1500)
+    q = synth.query(w, 2, 1, batch=4)
+    (ck,), (sk,) = rq.encode([refk], refk, [2], w.group, w.seed)
+    (cv,), (sv,) = rq.encode([refv], refv, [2], w.group, w.seed)
+    out_res = rq.decode_attention(q, refk, refv, ck, cv, sk, sv, 2, w.group, w.seed)
+    out_ref = rq.decode_attention(q, refk, refv, None, None, None, None, 16, w.group, w.seed)
+    torch.cuda.synchronize()
+    assert torch.equal(out_res, out_ref)
+    # and the reference loop matches plain attention (torch SDPA, fp64 on CPU)
+    want = torch.nn.functional.scaled_dot_product_attention(
+        q.double().cpu().unsqueeze(2), refk.double().cpu(), refv.double().cpu(),
+        scale=1 / math.sqrt(w.head_dim)).squeeze(2)
+    assert (out_ref.double().cpu() - want).abs().max().item() < 1e-4
+
+
+def test_repeated_calls_are_deterministic_and_status_clean():
+    w = synth.OURO
+    refk = synth.reference(w, 1, 0, batch=2, ctx=3000)
+    refv = synth.reference(w, 1, 1, batch=2, ctx=3000)
+    xk = synth.loop_kv(w, 1, 0, 1, refk)
+    xv = synth.loop_kv(w, 1, 1, 1, refv)
+    q = synth.query(w, 1, 1, batch=2)
+    (ck,), (sk,) = rq.encode([xk], refk, [2], w.group, w.seed)
+    (cv,), (sv,) = rq.encode([xv], refv, [2], w.group, w.seed)
+    shape = rq.make_shape(2, 16, 3000, 128, 32, q_heads=16)
+    ws = rq.alloc_workspace(shape)
+    outs = [rq.decode_attention(q, refk, refv, ck, cv, sk, sv, 2, w.group, w.seed, workspace=ws)
+            for _ in range(3)]
+    torch.cuda.synchronize()
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[1], outs[2])
+    assert rq.rq_workspace_status(ws) == 0
+    # the arrival counters are back at zero after every call
+    heads = 2 * 16
+    counters = ws[16:16 + 4 * heads].view(torch.int32)
+    assert (counters == 0).all()
