@@ -10,9 +10,7 @@
 //   out     = ( sum_t p_t refV_t + Rot^T sum_t p_t s^V_t l^V_t ) / sum_t p_t
 // so K_hat and V_hat are never built: the query is rotated once per head
 // and the V residual is accumulated in the rotated domain and rotated back
-// once per output row.  The level l = 2c - (2^b - 1) is split as
-// 2c - (2^b - 1): the code c enters the inner products and the constant is
-// folded into one per-lane offset (scores) or one per-lane weight sum (V).
+// once per output row.
 //
 // Structure (one launch per call):
 //   - P = 2 x SMs persistent CTAs.  The (head, tile) space -- heads are
@@ -24,12 +22,23 @@
 //     HBM) into a ring of shared-memory stages, completion tracked by
 //     mbarrier transaction counts.
 //   - Warps 0-3 consume: lanes split head_dim, so one 16- or 8-byte shared
-//     load per lane reads a token row; partial dot products are reduced with
-//     shfl.xor; online softmax in base 2 per warp.
+//     load per lane reads a token row.  Base-2 online softmax per warp.
 //   - At the end of a head's run the consumer warps merge their states and
 //     write one partial record; the last CTA to arrive for that head (an
 //     atomic ticket, no waiting) merges all records, applies the inverse
 //     rotation once and writes the output.
+//
+// Arithmetic per token is what limits this kernel once the copies stream, so
+// the single-query (G = 1) path is shaped to issue few instructions:
+//   - INT2 K residual: per head, a shared-memory table holds, for every
+//     4-dim slice of q~ and every byte of 4 codes, the partial product
+//     sum_k q~_k l(c_k); a lane's 8 dims cost two table reads.
+//   - Codes become floats with one AND/OR and one subtract (the 2^23
+//     exponent trick, the code left at its bit position); the position's
+//     power of two is folded into the query constants or applied once when
+//     the V accumulator is flushed.
+//   - Scores are reduce-scattered across the lanes of a token (one shuffle
+//     per value instead of four), so each lane evaluates one exp per chunk.
 // Every mbarrier wait is bounded; a wait that runs out raises the workspace
 // status word, and the kernel still finishes (its output is then invalid).
 #include <cmath>
@@ -53,8 +62,10 @@ struct Cfg {
   static constexpr int TILE = kDecodeTile;
   static constexpr int TPW = TILE / kConsumerWarps;         // tokens per warp per tile
   static constexpr int STEPS = TPW / TPS;                   // warp steps per tile
-  static constexpr int CH = (G == 1) ? (STEPS < 8 ? STEPS : 8) : (STEPS < 4 ? STEPS : 4);
+  // G == 1 reduce-scatters LPT/2 partial scores per chunk
+  static constexpr int CH = (G == 1) ? LPT / 2 : (STEPS < 4 ? STEPS : 4);
   static constexpr bool RES = (BITS != 16);
+  static constexpr bool LUT = (G == 1 && BITS == 2);
   static constexpr int KROW = D * 2;                        // bytes of a bf16 row
   static constexpr int CROW = RES ? D * BITS / 8 : 0;       // code bytes per token
   static constexpr int CWORDS = CROW / 4;
@@ -68,22 +79,69 @@ struct Cfg {
   static constexpr int STAGE_BYTES = OFF_SV + SC_BYTES;
   static constexpr int STAGES = RES ? 2 : 3;
   static constexpr int RING_BYTES = STAGES * STAGE_BYTES;
-  // merge area: per warp and query row {m, l} + accRef[D] + accRes[D]
+  // K-residual table: [256 byte values][32 slices] floats
+  static constexpr int LUT_FLOATS = LUT ? 256 * 32 : 0;
+  // merge area: per warp and query row {m, l} + accRef[D] + accRes[D]; it
+  // shares the table's space when there is one (never live at once)
   static constexpr int MERGE_FLOATS = kConsumerWarps * G * (2 + 2 * D);
+  static constexpr int AREA_FLOATS = LUT_FLOATS > MERGE_FLOATS ? LUT_FLOATS : MERGE_FLOATS;
   static constexpr int QBUF_FLOATS = 2 * G * D;             // q and q~
   static constexpr int SMEM_BYTES =
-      RING_BYTES + 4 * (MERGE_FLOATS + QBUF_FLOATS) + 2 * STAGES * 8 + 16;
+      RING_BYTES + 4 * (AREA_FLOATS + QBUF_FLOATS) + 2 * STAGES * 8 + 16;
   static_assert(TPW % TPS == 0 && STEPS % CH == 0, "tile split");
+  static_assert(G != 1 || CH == STEPS, "G == 1 processes a whole tile per chunk");
   static_assert(STAGE_BYTES % 16 == 0, "stage alignment");
 };
 
-__device__ __forceinline__ float code_as_float(uint32_t c) {
-  // c < 2^23: exact via the 2^23 exponent trick
-  return __uint_as_float(0x4B000000u | c) - 8388608.0f;
+// code c (already masked, left at its bit position) -> exact float
+__device__ __forceinline__ float code_at(uint32_t masked) {
+  return __uint_as_float(0x4B000000u | masked) - 8388608.0f;
+}
+
+// The lane's DPL codes as floats c_k * 2^pos_k (pos_k = the bit position the
+// code sits at inside `x`, the lane's bits already shifted down to bit 0).
+template <int BITS, int DPL>
+__device__ __forceinline__ void codes_positional(uint32_t x, float (&f)[DPL]) {
+  constexpr uint32_t M = (1u << BITS) - 1u;
+  if constexpr (BITS * DPL > 16) {
+    // 8 INT4 codes: split so no code sits above bit 16 (exactness needs < 2^23)
+    const uint32_t lo = x & 0xFFFFu, hi = x >> 16;
+#pragma unroll
+    for (int k = 0; k < DPL / 2; ++k) {
+      f[k] = code_at(lo & (M << (BITS * k)));
+      f[k + DPL / 2] = code_at(hi & (M << (BITS * k)));
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < DPL; ++k) f[k] = code_at(x & (M << (BITS * k)));
+  }
+}
+
+// 2^-pos of code k in codes_positional
+template <int BITS, int DPL>
+__host__ __device__ constexpr float pos_factor(int k) {
+  return (BITS * DPL > 16) ? 1.0f / (float)(1u << (BITS * (k % (DPL / 2))))
+                           : 1.0f / (float)(1u << (BITS * k));
 }
 
 __device__ __forceinline__ void flag_error(uint32_t* status, uint32_t bit) {
   atomicOr(status, bit);
+}
+
+template <int DPL>
+__device__ __forceinline__ void load_row(const unsigned char* p, float (&f)[DPL]) {
+  if constexpr (DPL == 8) {
+    const uint4 w = *reinterpret_cast<const uint4*>(p);
+    f[0] = bf16lo(w.x); f[1] = bf16hi(w.x); f[2] = bf16lo(w.y); f[3] = bf16hi(w.y);
+    f[4] = bf16lo(w.z); f[5] = bf16hi(w.z); f[6] = bf16lo(w.w); f[7] = bf16hi(w.w);
+  } else {
+    const uint2 w = *reinterpret_cast<const uint2*>(p);
+    f[0] = bf16lo(w.x); f[1] = bf16hi(w.x); f[2] = bf16lo(w.y); f[3] = bf16hi(w.y);
+  }
+}
+
+__device__ __forceinline__ float half_at(const unsigned char* p) {
+  return __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t*>(p)));
 }
 
 template <int D, int G, int BITS>
@@ -94,11 +152,14 @@ decode_kernel(const DecodeParams p) {
   constexpr int STAGES = C::STAGES, CH = C::CH;
   constexpr unsigned FULL = 0xffffffffu;
   constexpr int TOPLVL = C::RES ? (1 << BITS) - 1 : 0;
+  constexpr int PB = C::RES ? BITS : 2;     // bit width used for position factors
 
   extern __shared__ __align__(128) unsigned char smem[];
   unsigned char* ring = smem;
-  float* merge = reinterpret_cast<float*>(smem + C::RING_BYTES);
-  float* qbuf = merge + C::MERGE_FLOATS;
+  float* area = reinterpret_cast<float*>(smem + C::RING_BYTES);  // table / merge
+  float* merge = area;
+  float* lut = area;
+  float* qbuf = area + C::AREA_FLOATS;
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(qbuf + C::QBUF_FLOATS);
   uint64_t* empty_bar = full_bar + STAGES;
   volatile int* flags = reinterpret_cast<volatile int*>(empty_bar + STAGES);  // [0] abort, [1] last
@@ -181,10 +242,23 @@ decode_kernel(const DecodeParams p) {
   const int slot = lane / LPT;        // token slot within a warp step
   const int dim0 = li * DPL;          // first dim this lane owns
   const float score_scale = p.score_scale;
+  const int cw = (dim0 * PB) / 32;    // code word of this lane
+  const int csh = (dim0 * PB) % 32;   // bit offset of the lane's codes in it
+
+  // table slices and byte selectors of this lane (G == 1, INT2): the lane's
+  // 16 code bits are bytes 2*(li&1) and 2*(li&1)+1 of word cw, for slices
+  // 2li and 2li+1.  The two token slots of a warp step read the slices in
+  // opposite order so the 32 lanes hit 32 different banks.
+  const int slice_a = 2 * li + (slot & 1);
+  const int slice_b = 2 * li + 1 - (slot & 1);
+  const uint32_t sel_a = 0x4440u | (uint32_t)(2 * (li & 1) + (slot & 1));
+  const uint32_t sel_b = 0x4440u | (uint32_t)(2 * (li & 1) + 1 - (slot & 1));
+  // with head_dim 64 there are 16 slices; slots 2 and 3 read a second copy
+  const int lut_copy = (D == 64) ? 16 * ((slot >> 1) & 1) : 0;
 
   // per-lane constants of the current head
   float qa[G][DPL];                   // score_scale * q
-  float qc[G][DPL];                   // 2 * score_scale * q~
+  float qc[G][DPL];                   // 2 * score_scale * q~ * 2^-pos
   float qoff[G];                      // (2^b - 1) * score_scale * sum q~ (lane's dims)
   // running state
   float m_run[G], l_run[G], accV[G][DPL], accC[G][DPL], wsum[G];
@@ -203,13 +277,14 @@ decode_kernel(const DecodeParams p) {
     }
   };
 
-  // load and rotate the G query rows of head hd; all consumer threads
+  // load and rotate the G query rows of head hd (and fill the K table);
+  // all consumer threads
   auto setup_head = [&](long long hd) {
     const int b = (int)(hd / p.kv_heads);
     const int h = (int)(hd % p.kv_heads);
     float* qs = qbuf;              // [G][D] raw q
     float* qt = qbuf + G * D;      // [G][D] rotated
-    named_bar_sync(1, kConsumerThreads);          // previous users of qbuf done
+    named_bar_sync(1, kConsumerThreads);          // previous users of qbuf / area done
     for (int e = tid; e < G * D; e += kConsumerThreads) {
       const int r = e / D, i = e % D;
       const uint16_t raw = p.q[((size_t)b * p.q_heads + (size_t)h * G + r) * D + i];
@@ -230,6 +305,30 @@ decode_kernel(const DecodeParams p) {
     }
     named_bar_sync(1, kConsumerThreads);
     const float cd = rot_scale<D>();
+    if constexpr (C::LUT) {
+      // lut[byte][slice] = score_scale * sum_k q~[4 slice + k] * l(c_k(byte)),
+      // l(c) = 2c - 3, c_k = bits 2k..2k+1 of the byte.  Thread: slice =
+      // tid % S and c0 = (tid / S) % 4 fixed; it writes the 64 bytes with
+      // that c0 (and, for head_dim 64, a second copy at slice + 16).
+      constexpr int S = D / 4;
+      const int slice = tid % S;
+      const int c0 = (tid / S) & 3;
+      const int copy = (D == 64) ? 16 * ((tid / (4 * S)) & 1) : 0;
+      float lv[4][4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float qk = score_scale * cd * qt[4 * slice + k];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) lv[k][c] = qk * (float)(2 * c - 3);
+      }
+      const float base = (c0 == 0) ? lv[0][0] : (c0 == 1) ? lv[0][1] : (c0 == 2) ? lv[0][2] : lv[0][3];
+#pragma unroll
+      for (int n = 0; n < 64; ++n) {
+        const float e = base + lv[1][n & 3] + lv[2][(n >> 2) & 3] + lv[3][n >> 4];
+        lut[(c0 + 4 * n) * 32 + copy + slice] = e;
+      }
+      named_bar_sync(1, kConsumerThreads);
+    }
 #pragma unroll
     for (int r = 0; r < G; ++r) {
       float sum = 0.0f;
@@ -237,7 +336,7 @@ decode_kernel(const DecodeParams p) {
       for (int k = 0; k < DPL; ++k) {
         qa[r][k] = score_scale * qs[r * D + dim0 + k];
         const float t = cd * qt[r * D + dim0 + k];
-        qc[r][k] = 2.0f * score_scale * t;
+        qc[r][k] = 2.0f * score_scale * t * pos_factor<PB, DPL>(k);
         sum += t;
       }
       qoff[r] = (float)TOPLVL * score_scale * sum;
@@ -252,9 +351,17 @@ decode_kernel(const DecodeParams p) {
     // fold the token slots of the warp together
 #pragma unroll
     for (int r = 0; r < G; ++r) {
+      if constexpr (G == 1) {
+        // every token's weight sits in two lanes (li, li ^ 1)
+#pragma unroll
+        for (int m = 1; m < 32; m <<= 1) l_run[r] += __shfl_xor_sync(FULL, l_run[r], m);
+        l_run[r] *= 0.5f;
+      } else {
+#pragma unroll
+        for (int m = LPT; m < 32; m <<= 1) l_run[r] += __shfl_xor_sync(FULL, l_run[r], m);
+      }
 #pragma unroll
       for (int m = LPT; m < 32; m <<= 1) {
-        l_run[r] += __shfl_xor_sync(FULL, l_run[r], m);
         if constexpr (C::RES) wsum[r] += __shfl_xor_sync(FULL, wsum[r], m);
 #pragma unroll
         for (int k = 0; k < DPL; ++k) {
@@ -263,7 +370,7 @@ decode_kernel(const DecodeParams p) {
         }
       }
     }
-    named_bar_sync(1, kConsumerThreads);          // merge area free
+    named_bar_sync(1, kConsumerThreads);          // merge area (and table) free
     float* mw = merge + warp * G * (2 + 2 * D);
     if (slot == 0) {
 #pragma unroll
@@ -277,7 +384,8 @@ decode_kernel(const DecodeParams p) {
         for (int k = 0; k < DPL; ++k) {
           rec[2 + dim0 + k] = accV[r][k];
           rec[2 + D + dim0 + k] =
-              C::RES ? (2.0f * accC[r][k] - (float)TOPLVL * wsum[r]) : 0.0f;
+              C::RES ? (2.0f * pos_factor<PB, DPL>(k) * accC[r][k] - (float)TOPLVL * wsum[r])
+                     : 0.0f;
         }
       }
     }
@@ -374,6 +482,187 @@ decode_kernel(const DecodeParams p) {
     }
   };
 
+  // ---- one tile, single query row per kv head ----
+  auto tile_g1 = [&](const unsigned char* st, int n, int sc_off, int grp) {
+    float part[CH];
+#pragma unroll
+    for (int u = 0; u < CH; ++u) {
+      const int tok = warp * C::TPW + u * TPS + slot;
+      float kf[DPL];
+      load_row<DPL>(st + C::OFF_K + tok * C::KROW + dim0 * 2, kf);
+      float dot = 0.0f;
+#pragma unroll
+      for (int k = 0; k < DPL; ++k) dot = fmaf(qa[0][k], kf[k], dot);
+      if constexpr (C::RES) {
+        const uint32_t word = reinterpret_cast<const uint32_t*>(st + C::OFF_CK)[tok * C::CWORDS + cw];
+        const float s_k = half_at(st + C::OFF_SK + sc_off + tok * SB + grp * 2);
+        float res;
+        if constexpr (C::LUT) {
+          const uint32_t ba = __byte_perm(word, 0u, sel_a);
+          const uint32_t bb = __byte_perm(word, 0u, sel_b);
+          res = lut[ba * 32 + lut_copy + slice_a] + lut[bb * 32 + lut_copy + slice_b];
+        } else {
+          float cf[DPL];
+          codes_positional<PB, DPL>(word >> csh, cf);
+          res = -qoff[0];
+#pragma unroll
+          for (int k = 0; k < DPL; ++k) res = fmaf(qc[0][k], cf[k], res);
+        }
+        dot = fmaf(s_k, res, dot);
+      }
+      part[u] = dot;
+    }
+    // reduce-scatter over the LPT lanes of a token: afterwards lane li holds
+    // the full score of step li >> 1 (lanes li and li ^ 1 agree)
+#pragma unroll
+    for (int half = CH / 2, m = LPT / 2; half >= 1; half >>= 1, m >>= 1) {
+      const bool upper = (li & m) != 0;
+#pragma unroll
+      for (int i = 0; i < half; ++i) {
+        const float send = upper ? part[i] : part[i + half];
+        const float keep = upper ? part[i + half] : part[i];
+        part[i] = keep + __shfl_xor_sync(FULL, send, m);
+      }
+    }
+    float sc = part[0] + __shfl_xor_sync(FULL, part[0], 1);
+    const int own_tok = warp * C::TPW + (li >> 1) * TPS + slot;
+    if (own_tok >= n) sc = kNegInf;
+    // online softmax, base 2
+    float mc = sc;
+#pragma unroll
+    for (int m = 2; m < 32; m <<= 1) mc = fmaxf(mc, __shfl_xor_sync(FULL, mc, m));
+    const float m_new = fmaxf(m_run[0], mc);
+    if (m_new != m_run[0]) {
+      const float alpha = (m_run[0] == kNegInf) ? 0.0f : exp2f(m_run[0] - m_new);
+      l_run[0] *= alpha;
+      if constexpr (C::RES) wsum[0] *= alpha;
+#pragma unroll
+      for (int k = 0; k < DPL; ++k) {
+        accV[0][k] *= alpha;
+        if constexpr (C::RES) accC[0][k] *= alpha;
+      }
+      m_run[0] = m_new;
+    }
+    const float pme = (sc == kNegInf) ? 0.0f : exp2f(sc - m_new);
+    l_run[0] += pme;
+    // values
+#pragma unroll
+    for (int u = 0; u < CH; ++u) {
+      const float pu = __shfl_sync(FULL, pme, slot * LPT + 2 * u);
+      const int tok = warp * C::TPW + u * TPS + slot;
+      if (tok < n) {
+        float vf[DPL];
+        load_row<DPL>(st + C::OFF_V + tok * C::KROW + dim0 * 2, vf);
+#pragma unroll
+        for (int k = 0; k < DPL; ++k) accV[0][k] = fmaf(pu, vf[k], accV[0][k]);
+        if constexpr (C::RES) {
+          const uint32_t word =
+              reinterpret_cast<const uint32_t*>(st + C::OFF_CV)[tok * C::CWORDS + cw];
+          const float wv = pu * half_at(st + C::OFF_SV + sc_off + tok * SB + grp * 2);
+          float cf[DPL];
+          codes_positional<PB, DPL>(word >> csh, cf);
+          wsum[0] += wv;
+#pragma unroll
+          for (int k = 0; k < DPL; ++k) accC[0][k] = fmaf(wv, cf[k], accC[0][k]);
+        }
+      }
+    }
+  };
+
+  // ---- one tile, G query rows per kv head ----
+  auto tile_gn = [&](const unsigned char* st, int n, int sc_off, int grp) {
+#pragma unroll 1
+    for (int c0 = 0; c0 < C::STEPS; c0 += CH) {
+      float sc[G][CH];
+#pragma unroll
+      for (int u = 0; u < CH; ++u) {
+        const int tok = warp * C::TPW + (c0 + u) * TPS + slot;
+        float kf[DPL];
+        load_row<DPL>(st + C::OFF_K + tok * C::KROW + dim0 * 2, kf);
+        float dot[G];
+#pragma unroll
+        for (int r = 0; r < G; ++r) {
+          dot[r] = 0.0f;
+#pragma unroll
+          for (int k = 0; k < DPL; ++k) dot[r] = fmaf(qa[r][k], kf[k], dot[r]);
+        }
+        if constexpr (C::RES) {
+          const uint32_t word =
+              reinterpret_cast<const uint32_t*>(st + C::OFF_CK)[tok * C::CWORDS + cw];
+          const float s_k = half_at(st + C::OFF_SK + sc_off + tok * SB + grp * 2);
+          float cf[DPL];
+          codes_positional<PB, DPL>(word >> csh, cf);
+#pragma unroll
+          for (int r = 0; r < G; ++r) {
+            float res = -qoff[r];
+#pragma unroll
+            for (int k = 0; k < DPL; ++k) res = fmaf(qc[r][k], cf[k], res);
+            dot[r] = fmaf(s_k, res, dot[r]);
+          }
+        }
+#pragma unroll
+        for (int r = 0; r < G; ++r) {
+#pragma unroll
+          for (int m = 1; m < LPT; m <<= 1) dot[r] += __shfl_xor_sync(FULL, dot[r], m);
+          sc[r][u] = (tok < n) ? dot[r] : kNegInf;
+        }
+      }
+      float pw[G][CH];
+#pragma unroll
+      for (int r = 0; r < G; ++r) {
+        float mc = sc[r][0];
+#pragma unroll
+        for (int u = 1; u < CH; ++u) mc = fmaxf(mc, sc[r][u]);
+#pragma unroll
+        for (int m = LPT; m < 32; m <<= 1) mc = fmaxf(mc, __shfl_xor_sync(FULL, mc, m));
+        const float m_new = fmaxf(m_run[r], mc);
+        if (m_new != m_run[r]) {
+          const float alpha = (m_run[r] == kNegInf) ? 0.0f : exp2f(m_run[r] - m_new);
+          l_run[r] *= alpha;
+          if constexpr (C::RES) wsum[r] *= alpha;
+#pragma unroll
+          for (int k = 0; k < DPL; ++k) {
+            accV[r][k] *= alpha;
+            if constexpr (C::RES) accC[r][k] *= alpha;
+          }
+          m_run[r] = m_new;
+        }
+#pragma unroll
+        for (int u = 0; u < CH; ++u) {
+          pw[r][u] = (sc[r][u] == kNegInf) ? 0.0f : exp2f(sc[r][u] - m_new);
+          l_run[r] += pw[r][u];
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < CH; ++u) {
+        const int tok = warp * C::TPW + (c0 + u) * TPS + slot;
+        if (tok < n) {
+          float vf[DPL];
+          load_row<DPL>(st + C::OFF_V + tok * C::KROW + dim0 * 2, vf);
+#pragma unroll
+          for (int r = 0; r < G; ++r) {
+#pragma unroll
+            for (int k = 0; k < DPL; ++k) accV[r][k] = fmaf(pw[r][u], vf[k], accV[r][k]);
+          }
+          if constexpr (C::RES) {
+            const uint32_t word =
+                reinterpret_cast<const uint32_t*>(st + C::OFF_CV)[tok * C::CWORDS + cw];
+            const float s_v = half_at(st + C::OFF_SV + sc_off + tok * SB + grp * 2);
+            float cf[DPL];
+            codes_positional<PB, DPL>(word >> csh, cf);
+#pragma unroll
+            for (int r = 0; r < G; ++r) {
+              const float wv = pw[r][u] * s_v;
+              wsum[r] += wv;
+#pragma unroll
+              for (int k = 0; k < DPL; ++k) accC[r][k] = fmaf(wv, cf[k], accC[r][k]);
+            }
+          }
+        }
+      }
+    }
+  };
+
   // ---- main loop over this CTA's tiles ----
   long long cur_head = -1;
   bool aborted = false;
@@ -405,122 +694,8 @@ decode_kernel(const DecodeParams p) {
       const size_t row = (size_t)hd * T + t0;
       const int sc_off = (int)((row * SB) & 15);
       const int grp = dim0 / p.group;
-      const int cw = (dim0 * BITS) / 32;                   // code word of this lane
-      const int csh = (dim0 * BITS) % 32;                  // bit offset in it
-
-#pragma unroll 1
-      for (int c0 = 0; c0 < C::STEPS; c0 += CH) {
-        float sc[G][CH];
-        // ---- scores ----
-#pragma unroll
-        for (int u = 0; u < CH; ++u) {
-          const int tok = warp * C::TPW + (c0 + u) * TPS + slot;
-          float kf[DPL];
-          const unsigned char* kp = st + C::OFF_K + tok * C::KROW + dim0 * 2;
-          if constexpr (DPL == 8) {
-            const uint4 w = *reinterpret_cast<const uint4*>(kp);
-            kf[0] = bf16lo(w.x); kf[1] = bf16hi(w.x); kf[2] = bf16lo(w.y); kf[3] = bf16hi(w.y);
-            kf[4] = bf16lo(w.z); kf[5] = bf16hi(w.z); kf[6] = bf16lo(w.w); kf[7] = bf16hi(w.w);
-          } else {
-            const uint2 w = *reinterpret_cast<const uint2*>(kp);
-            kf[0] = bf16lo(w.x); kf[1] = bf16hi(w.x); kf[2] = bf16lo(w.y); kf[3] = bf16hi(w.y);
-          }
-          float dot[G];
-#pragma unroll
-          for (int r = 0; r < G; ++r) {
-            dot[r] = 0.0f;
-#pragma unroll
-            for (int k = 0; k < DPL; ++k) dot[r] = fmaf(qa[r][k], kf[k], dot[r]);
-          }
-          if constexpr (C::RES) {
-            const uint32_t word =
-                reinterpret_cast<const uint32_t*>(st + C::OFF_CK)[tok * C::CWORDS + cw] >> csh;
-            const float s_k = __half2float(__ushort_as_half(
-                *reinterpret_cast<const uint16_t*>(st + C::OFF_SK + sc_off + tok * SB + grp * 2)));
-            float cf[DPL];
-#pragma unroll
-            for (int k = 0; k < DPL; ++k) cf[k] = code_as_float((word >> (BITS * k)) & ((1u << BITS) - 1));
-#pragma unroll
-            for (int r = 0; r < G; ++r) {
-              float res = -qoff[r];
-#pragma unroll
-              for (int k = 0; k < DPL; ++k) res = fmaf(qc[r][k], cf[k], res);
-              dot[r] = fmaf(s_k, res, dot[r]);
-            }
-          }
-#pragma unroll
-          for (int r = 0; r < G; ++r) {
-#pragma unroll
-            for (int m = 1; m < LPT; m <<= 1) dot[r] += __shfl_xor_sync(FULL, dot[r], m);
-            sc[r][u] = (tok < n) ? dot[r] : kNegInf;
-          }
-        }
-        // ---- online softmax (base 2) ----
-        float pw[G][CH];
-#pragma unroll
-        for (int r = 0; r < G; ++r) {
-          float mc = sc[r][0];
-#pragma unroll
-          for (int u = 1; u < CH; ++u) mc = fmaxf(mc, sc[r][u]);
-#pragma unroll
-          for (int m = LPT; m < 32; m <<= 1) mc = fmaxf(mc, __shfl_xor_sync(FULL, mc, m));
-          const float m_new = fmaxf(m_run[r], mc);
-          if (m_new != m_run[r]) {
-            const float alpha = (m_run[r] == kNegInf) ? 0.0f : exp2f(m_run[r] - m_new);
-            l_run[r] *= alpha;
-            if constexpr (C::RES) wsum[r] *= alpha;
-#pragma unroll
-            for (int k = 0; k < DPL; ++k) {
-              accV[r][k] *= alpha;
-              if constexpr (C::RES) accC[r][k] *= alpha;
-            }
-            m_run[r] = m_new;
-          }
-#pragma unroll
-          for (int u = 0; u < CH; ++u) {
-            pw[r][u] = (sc[r][u] == kNegInf) ? 0.0f : exp2f(sc[r][u] - m_new);
-            l_run[r] += pw[r][u];
-          }
-        }
-        // ---- values ----
-#pragma unroll
-        for (int u = 0; u < CH; ++u) {
-          const int tok = warp * C::TPW + (c0 + u) * TPS + slot;
-          if (tok < n) {
-            float vf[DPL];
-            const unsigned char* vp = st + C::OFF_V + tok * C::KROW + dim0 * 2;
-            if constexpr (DPL == 8) {
-              const uint4 w = *reinterpret_cast<const uint4*>(vp);
-              vf[0] = bf16lo(w.x); vf[1] = bf16hi(w.x); vf[2] = bf16lo(w.y); vf[3] = bf16hi(w.y);
-              vf[4] = bf16lo(w.z); vf[5] = bf16hi(w.z); vf[6] = bf16lo(w.w); vf[7] = bf16hi(w.w);
-            } else {
-              const uint2 w = *reinterpret_cast<const uint2*>(vp);
-              vf[0] = bf16lo(w.x); vf[1] = bf16hi(w.x); vf[2] = bf16lo(w.y); vf[3] = bf16hi(w.y);
-            }
-#pragma unroll
-            for (int r = 0; r < G; ++r) {
-#pragma unroll
-              for (int k = 0; k < DPL; ++k) accV[r][k] = fmaf(pw[r][u], vf[k], accV[r][k]);
-            }
-            if constexpr (C::RES) {
-              const uint32_t word =
-                  reinterpret_cast<const uint32_t*>(st + C::OFF_CV)[tok * C::CWORDS + cw] >> csh;
-              const float s_v = __half2float(__ushort_as_half(
-                  *reinterpret_cast<const uint16_t*>(st + C::OFF_SV + sc_off + tok * SB + grp * 2)));
-              float cf[DPL];
-#pragma unroll
-              for (int k = 0; k < DPL; ++k) cf[k] = code_as_float((word >> (BITS * k)) & ((1u << BITS) - 1));
-#pragma unroll
-              for (int r = 0; r < G; ++r) {
-                const float wv = pw[r][u] * s_v;
-                wsum[r] += wv;
-#pragma unroll
-                for (int k = 0; k < DPL; ++k) accC[r][k] = fmaf(wv, cf[k], accC[r][k]);
-              }
-            }
-          }
-        }
-      }
+      if constexpr (G == 1) tile_g1(st, n, sc_off, grp);
+      else tile_gn(st, n, sc_off, grp);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty_bar[s]);
