@@ -175,6 +175,41 @@ rq_status rq_decode_attention(const rq_shape *shape, const uint16_t *q,
                               int bits, uint64_t seed, float softmax_scale, float *out,
                               void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * rq_decode_attention_noalloc -- rq_decode_attention without a workspace
+ * argument, for callers that cannot allocate device memory (for example code
+ * hosted by an application that owns every allocation, or a path that must
+ * not call cudaMalloc because it may synchronise the device).  The paper has
+ * no counterpart: this is a property of the library, not of the method.
+ *
+ * Same arguments, layouts, results and validation as rq_decode_attention,
+ * minus `workspace` and `workspace_bytes`.  The scratch is a fixed array of
+ * RQ_NOALLOC_SCRATCH_BYTES in the library's own device memory; every GPU on
+ * which this entry point is used keeps that much until the process exits.
+ *   - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library
+ *     routine.  It clears the scratch's status word and arrival counters
+ *     (cudaMemsetAsync on `stream`) before each launch.
+ *   - A shape needing more than RQ_NOALLOC_SCRATCH_BYTES
+ *     (rq_decode_workspace_bytes(shape) > RQ_NOALLOC_SCRATCH_BYTES) is
+ *     rejected with RQ_ERR_WORKSPACE before anything is enqueued.
+ *   - The first call on a device looks up the array's device address (once
+ *     per device, with that device current); make that first call before any
+ *     stream capture.
+ *   - Every call shares the one array per device and it keeps the last
+ *     call's contents: calls whose executions overlap on the GPU (other
+ *     streams, other host threads on the same device) race and give wrong
+ *     results; order them on one stream.
+ *   - There is no status readback for this scratch.
+ */
+#define RQ_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+rq_status rq_decode_attention_noalloc(const rq_shape *shape, const uint16_t *q,
+                                      const uint16_t *ref_k, const uint16_t *ref_v,
+                                      const uint32_t *codes_k, const uint32_t *codes_v,
+                                      const uint16_t *scales_k, const uint16_t *scales_v,
+                                      int bits, uint64_t seed, float softmax_scale, float *out,
+                                      void *stream);
+
 /* Copies the workspace's device status word to *host_status (blocking read
  * on `stream`).  0 means every decode call since the workspace was zeroed
  * ran clean; non-zero means a bounded wait inside a kernel ran out, its

@@ -9,7 +9,8 @@ reports and pass pointers through.
 """
 from ._abi import (RQ_ERR_ALIGNMENT, RQ_ERR_CUDA, RQ_ERR_INVALID_ARG, RQ_ERR_UNSUPPORTED,
                    RQ_ERR_WORKSPACE, RQ_MAX_LOOPS, RQ_OK, RqError, lib, make_shape,
-                   rq_codes_bytes, rq_decode_attention, rq_decode_workspace_bytes, rq_encode,
+                   rq_codes_bytes, rq_decode_attention, rq_decode_attention_noalloc,
+                   rq_decode_workspace_bytes, rq_encode,
                    rq_scales_bytes, rq_shape, rq_status_string, rq_version,
                    rq_workspace_status)
 
@@ -17,7 +18,7 @@ __all__ = [
     "RQ_OK", "RQ_ERR_INVALID_ARG", "RQ_ERR_UNSUPPORTED", "RQ_ERR_ALIGNMENT", "RQ_ERR_WORKSPACE",
     "RQ_ERR_CUDA", "RQ_MAX_LOOPS", "RqError", "lib", "rq_shape", "make_shape", "rq_version",
     "rq_status_string", "rq_codes_bytes", "rq_scales_bytes", "rq_decode_workspace_bytes",
-    "rq_encode", "rq_decode_attention", "rq_workspace_status",
+    "rq_encode", "rq_decode_attention", "rq_decode_attention_noalloc", "rq_workspace_status",
     "alloc_codes", "alloc_scales", "alloc_workspace", "encode", "decode_attention",
 ]
 

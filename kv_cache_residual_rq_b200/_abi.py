@@ -71,6 +71,11 @@ def lib():
                                           c.c_void_p, c.c_void_p, c.c_void_p, c.c_int, c.c_uint64,
                                           c.c_float, c.c_void_p, c.c_void_p, c.c_size_t, c.c_void_p]
         L.rq_decode_attention.restype = c.c_int
+        L.rq_decode_attention_noalloc.argtypes = [sp, c.c_void_p, c.c_void_p, c.c_void_p,
+                                                  c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p,
+                                                  c.c_int, c.c_uint64, c.c_float, c.c_void_p,
+                                                  c.c_void_p]
+        L.rq_decode_attention_noalloc.restype = c.c_int
         L.rq_workspace_status.argtypes = [c.c_void_p, c.c_size_t, c.POINTER(c.c_uint32), c.c_void_p]
         L.rq_workspace_status.restype = c.c_int
         _lib = L
@@ -153,6 +158,19 @@ def rq_decode_attention(shape, q, ref_k, ref_v, codes_k, codes_v, scales_k, scal
                                    _stream(stream))
     if check:
         _check(st, "rq_decode_attention")
+    return st
+
+
+def rq_decode_attention_noalloc(shape, q, ref_k, ref_v, codes_k, codes_v, scales_k, scales_v,
+                                bits, seed, softmax_scale, out, stream=None, check=True):
+    """rq_decode_attention with the library's fixed scratch instead of a
+    caller workspace (for callers that cannot allocate)."""
+    st = lib().rq_decode_attention_noalloc(_shp(shape), _ptr(q), _ptr(ref_k), _ptr(ref_v),
+                                           _ptr(codes_k), _ptr(codes_v), _ptr(scales_k),
+                                           _ptr(scales_v), int(bits), ctypes.c_uint64(seed),
+                                           float(softmax_scale), _ptr(out), _stream(stream))
+    if check:
+        _check(st, "rq_decode_attention_noalloc")
     return st
 
 
