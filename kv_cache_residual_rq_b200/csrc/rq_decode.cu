@@ -39,6 +39,9 @@
 //     the V accumulator is flushed.
 //   - Scores are reduce-scattered across the lanes of a token (one shuffle
 //     per value instead of four), so each lane evaluates one exp per chunk.
+//   - <q, refK> uses the sm_100 fp32 += bf16 x bf16 fused multiply-add on
+//     the packed rows (no unpacking; the products are exact), and the V
+//     accumulators are packed fp32 pairs updated with the paired FMA.
 // Every mbarrier wait is bounded; a wait that runs out raises the workspace
 // status word, and the kernel still finishes (its output is then invalid).
 #include <cmath>
@@ -126,18 +129,6 @@ __host__ __device__ constexpr float pos_factor(int k) {
 
 __device__ __forceinline__ void flag_error(uint32_t* status, uint32_t bit) {
   atomicOr(status, bit);
-}
-
-template <int DPL>
-__device__ __forceinline__ void load_row(const unsigned char* p, float (&f)[DPL]) {
-  if constexpr (DPL == 8) {
-    const uint4 w = *reinterpret_cast<const uint4*>(p);
-    f[0] = bf16lo(w.x); f[1] = bf16hi(w.x); f[2] = bf16lo(w.y); f[3] = bf16hi(w.y);
-    f[4] = bf16lo(w.z); f[5] = bf16hi(w.z); f[6] = bf16lo(w.w); f[7] = bf16hi(w.w);
-  } else {
-    const uint2 w = *reinterpret_cast<const uint2*>(p);
-    f[0] = bf16lo(w.x); f[1] = bf16hi(w.x); f[2] = bf16lo(w.y); f[3] = bf16hi(w.y);
-  }
 }
 
 __device__ __forceinline__ float half_at(const unsigned char* p) {
@@ -244,6 +235,7 @@ decode_kernel(const DecodeParams p) {
   const float score_scale = p.score_scale;
   const int cw = (dim0 * PB) / 32;    // code word of this lane
   const int csh = (dim0 * PB) % 32;   // bit offset of the lane's codes in it
+  constexpr int NP = DPL / 2;         // packed pairs per lane
 
   // table slices and byte selectors of this lane (G == 1, INT2): the lane's
   // 16 code bits are bytes 2*(li&1) and 2*(li&1)+1 of word cw, for slices
@@ -256,12 +248,14 @@ decode_kernel(const DecodeParams p) {
   // with head_dim 64 there are 16 slices; slots 2 and 3 read a second copy
   const int lut_copy = (D == 64) ? 16 * ((slot >> 1) & 1) : 0;
 
-  // per-lane constants of the current head
-  float qa[G][DPL];                   // score_scale * q
-  float qc[G][DPL];                   // 2 * score_scale * q~ * 2^-pos
-  float qoff[G];                      // (2^b - 1) * score_scale * sum q~ (lane's dims)
+  // per-lane constants of the current head (scores are accumulated without
+  // the softmax scale, which multiplies each reduced score once)
+  uint32_t qbf[G][NP];                // q as packed bf16 pairs
+  float2 qc[G][NP];                   // 2 q~ 2^-pos (codes at their bit position)
+  float qoff[G];                      // (2^b - 1) * sum q~ over the lane's dims
   // running state
-  float m_run[G], l_run[G], accV[G][DPL], accC[G][DPL], wsum[G];
+  float m_run[G], l_run[G], wsum[G];
+  float2 accV[G][NP], accC[G][NP];
 
   auto reset_state = [&]() {
 #pragma unroll
@@ -270,9 +264,9 @@ decode_kernel(const DecodeParams p) {
       l_run[r] = 0.0f;
       wsum[r] = 0.0f;
 #pragma unroll
-      for (int k = 0; k < DPL; ++k) {
-        accV[r][k] = 0.0f;
-        accC[r][k] = 0.0f;
+      for (int j = 0; j < NP; ++j) {
+        accV[r][j] = make_float2(0.0f, 0.0f);
+        accC[r][j] = make_float2(0.0f, 0.0f);
       }
     }
   };
@@ -306,10 +300,10 @@ decode_kernel(const DecodeParams p) {
     named_bar_sync(1, kConsumerThreads);
     const float cd = rot_scale<D>();
     if constexpr (C::LUT) {
-      // lut[byte][slice] = score_scale * sum_k q~[4 slice + k] * l(c_k(byte)),
-      // l(c) = 2c - 3, c_k = bits 2k..2k+1 of the byte.  Thread: slice =
-      // tid % S and c0 = (tid / S) % 4 fixed; it writes the 64 bytes with
-      // that c0 (and, for head_dim 64, a second copy at slice + 16).
+      // lut[byte][slice] = sum_k q~[4 slice + k] * l(c_k(byte)), l(c) = 2c - 3,
+      // c_k = bits 2k..2k+1 of the byte.  Thread: slice = tid % S and
+      // c0 = (tid / S) % 4 fixed; it writes the 64 bytes with that c0 (and,
+      // for head_dim 64, a second copy at slice + 16).
       constexpr int S = D / 4;
       const int slice = tid % S;
       const int c0 = (tid / S) & 3;
@@ -317,7 +311,7 @@ decode_kernel(const DecodeParams p) {
       float lv[4][4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const float qk = score_scale * cd * qt[4 * slice + k];
+        const float qk = cd * qt[4 * slice + k];
 #pragma unroll
         for (int c = 0; c < 4; ++c) lv[k][c] = qk * (float)(2 * c - 3);
       }
@@ -333,13 +327,16 @@ decode_kernel(const DecodeParams p) {
     for (int r = 0; r < G; ++r) {
       float sum = 0.0f;
 #pragma unroll
-      for (int k = 0; k < DPL; ++k) {
-        qa[r][k] = score_scale * qs[r * D + dim0 + k];
-        const float t = cd * qt[r * D + dim0 + k];
-        qc[r][k] = 2.0f * score_scale * t * pos_factor<PB, DPL>(k);
-        sum += t;
+      for (int j = 0; j < NP; ++j) {
+        const float q0 = qs[r * D + dim0 + 2 * j], q1 = qs[r * D + dim0 + 2 * j + 1];
+        qbf[r][j] = (__float_as_uint(q0) >> 16) | (__float_as_uint(q1) & 0xFFFF0000u);
+        const float t0 = cd * qt[r * D + dim0 + 2 * j];
+        const float t1 = cd * qt[r * D + dim0 + 2 * j + 1];
+        qc[r][j] = make_float2(2.0f * t0 * pos_factor<PB, DPL>(2 * j),
+                               2.0f * t1 * pos_factor<PB, DPL>(2 * j + 1));
+        sum += t0 + t1;
       }
-      qoff[r] = (float)TOPLVL * score_scale * sum;
+      qoff[r] = (float)TOPLVL * sum;
     }
   };
 
@@ -364,9 +361,13 @@ decode_kernel(const DecodeParams p) {
       for (int m = LPT; m < 32; m <<= 1) {
         if constexpr (C::RES) wsum[r] += __shfl_xor_sync(FULL, wsum[r], m);
 #pragma unroll
-        for (int k = 0; k < DPL; ++k) {
-          accV[r][k] += __shfl_xor_sync(FULL, accV[r][k], m);
-          if constexpr (C::RES) accC[r][k] += __shfl_xor_sync(FULL, accC[r][k], m);
+        for (int j = 0; j < NP; ++j) {
+          accV[r][j].x += __shfl_xor_sync(FULL, accV[r][j].x, m);
+          accV[r][j].y += __shfl_xor_sync(FULL, accV[r][j].y, m);
+          if constexpr (C::RES) {
+            accC[r][j].x += __shfl_xor_sync(FULL, accC[r][j].x, m);
+            accC[r][j].y += __shfl_xor_sync(FULL, accC[r][j].y, m);
+          }
         }
       }
     }
@@ -381,11 +382,18 @@ decode_kernel(const DecodeParams p) {
           rec[1] = l_run[r];
         }
 #pragma unroll
-        for (int k = 0; k < DPL; ++k) {
-          rec[2 + dim0 + k] = accV[r][k];
-          rec[2 + D + dim0 + k] =
-              C::RES ? (2.0f * pos_factor<PB, DPL>(k) * accC[r][k] - (float)TOPLVL * wsum[r])
-                     : 0.0f;
+        for (int j = 0; j < NP; ++j) {
+          rec[2 + dim0 + 2 * j] = accV[r][j].x;
+          rec[2 + dim0 + 2 * j + 1] = accV[r][j].y;
+          if constexpr (C::RES) {
+            rec[2 + D + dim0 + 2 * j] =
+                2.0f * pos_factor<PB, DPL>(2 * j) * accC[r][j].x - (float)TOPLVL * wsum[r];
+            rec[2 + D + dim0 + 2 * j + 1] =
+                2.0f * pos_factor<PB, DPL>(2 * j + 1) * accC[r][j].y - (float)TOPLVL * wsum[r];
+          } else {
+            rec[2 + D + dim0 + 2 * j] = 0.0f;
+            rec[2 + D + dim0 + 2 * j + 1] = 0.0f;
+          }
         }
       }
     }
@@ -482,17 +490,79 @@ decode_kernel(const DecodeParams p) {
     }
   };
 
+  // <q, K row> of the lane's dims, straight from the packed bf16 row
+  auto ref_dot = [&](const unsigned char* kp, int r) {
+    float dot = 0.0f;
+    if constexpr (DPL == 8) {
+      const uint4 w = *reinterpret_cast<const uint4*>(kp);
+      dot = fma_bf16x2(qbf[r][0], w.x, dot);
+      dot = fma_bf16x2(qbf[r][1], w.y, dot);
+      dot = fma_bf16x2(qbf[r][2], w.z, dot);
+      dot = fma_bf16x2(qbf[r][3], w.w, dot);
+    } else {
+      const uint2 w = *reinterpret_cast<const uint2*>(kp);
+      dot = fma_bf16x2(qbf[r][0], w.x, dot);
+      dot = fma_bf16x2(qbf[r][1], w.y, dot);
+    }
+    return dot;
+  };
+
+  // the V row of the lane's dims as NP float pairs
+  auto v_pairs = [&](const unsigned char* vp, float2 (&vf)[NP]) {
+    if constexpr (DPL == 8) {
+      const uint4 w = *reinterpret_cast<const uint4*>(vp);
+      vf[0] = make_float2(bf16lo(w.x), bf16hi(w.x));
+      vf[1] = make_float2(bf16lo(w.y), bf16hi(w.y));
+      vf[2] = make_float2(bf16lo(w.z), bf16hi(w.z));
+      vf[3] = make_float2(bf16lo(w.w), bf16hi(w.w));
+    } else {
+      const uint2 w = *reinterpret_cast<const uint2*>(vp);
+      vf[0] = make_float2(bf16lo(w.x), bf16hi(w.x));
+      vf[1] = make_float2(bf16lo(w.y), bf16hi(w.y));
+    }
+  };
+
+  // the lane's codes as float pairs c * 2^pos
+  auto code_pairs = [&](uint32_t word, float2 (&cf)[NP]) {
+    float f[DPL];
+    codes_positional<PB, DPL>(word >> csh, f);
+#pragma unroll
+    for (int j = 0; j < NP; ++j) cf[j] = make_float2(f[2 * j], f[2 * j + 1]);
+  };
+
+  auto rescale = [&](int r, float alpha) {
+    const float2 a2 = make_float2(alpha, alpha);
+    l_run[r] *= alpha;
+    if constexpr (C::RES) wsum[r] *= alpha;
+#pragma unroll
+    for (int j = 0; j < NP; ++j) {
+      accV[r][j] = __fmul2_rn(accV[r][j], a2);
+      if constexpr (C::RES) accC[r][j] = __fmul2_rn(accC[r][j], a2);
+    }
+  };
+
+  // adds weight pw of one token (lane's V row vf, codes word, scale s_v)
+  auto accumulate_v = [&](int r, float pw, const float2 (&vf)[NP], const float2 (&cf)[NP],
+                          float s_v) {
+    const float2 p2 = make_float2(pw, pw);
+#pragma unroll
+    for (int j = 0; j < NP; ++j) accV[r][j] = __ffma2_rn(p2, vf[j], accV[r][j]);
+    if constexpr (C::RES) {
+      const float wv = pw * s_v;
+      const float2 w2 = make_float2(wv, wv);
+      wsum[r] += wv;
+#pragma unroll
+      for (int j = 0; j < NP; ++j) accC[r][j] = __ffma2_rn(w2, cf[j], accC[r][j]);
+    }
+  };
+
   // ---- one tile, single query row per kv head ----
   auto tile_g1 = [&](const unsigned char* st, int n, int sc_off, int grp) {
     float part[CH];
 #pragma unroll
     for (int u = 0; u < CH; ++u) {
       const int tok = warp * C::TPW + u * TPS + slot;
-      float kf[DPL];
-      load_row<DPL>(st + C::OFF_K + tok * C::KROW + dim0 * 2, kf);
-      float dot = 0.0f;
-#pragma unroll
-      for (int k = 0; k < DPL; ++k) dot = fmaf(qa[0][k], kf[k], dot);
+      float dot = ref_dot(st + C::OFF_K + tok * C::KROW + dim0 * 2, 0);
       if constexpr (C::RES) {
         const uint32_t word = reinterpret_cast<const uint32_t*>(st + C::OFF_CK)[tok * C::CWORDS + cw];
         const float s_k = half_at(st + C::OFF_SK + sc_off + tok * SB + grp * 2);
@@ -502,11 +572,12 @@ decode_kernel(const DecodeParams p) {
           const uint32_t bb = __byte_perm(word, 0u, sel_b);
           res = lut[ba * 32 + lut_copy + slice_a] + lut[bb * 32 + lut_copy + slice_b];
         } else {
-          float cf[DPL];
-          codes_positional<PB, DPL>(word >> csh, cf);
-          res = -qoff[0];
+          float2 cf[NP];
+          code_pairs(word, cf);
+          float2 acc = make_float2(-qoff[0], 0.0f);
 #pragma unroll
-          for (int k = 0; k < DPL; ++k) res = fmaf(qc[0][k], cf[k], res);
+          for (int j = 0; j < NP; ++j) acc = __ffma2_rn(qc[0][j], cf[j], acc);
+          res = acc.x + acc.y;
         }
         dot = fmaf(s_k, res, dot);
       }
@@ -524,7 +595,7 @@ decode_kernel(const DecodeParams p) {
         part[i] = keep + __shfl_xor_sync(FULL, send, m);
       }
     }
-    float sc = part[0] + __shfl_xor_sync(FULL, part[0], 1);
+    float sc = score_scale * (part[0] + __shfl_xor_sync(FULL, part[0], 1));
     const int own_tok = warp * C::TPW + (li >> 1) * TPS + slot;
     if (own_tok >= n) sc = kNegInf;
     // online softmax, base 2
@@ -533,14 +604,7 @@ decode_kernel(const DecodeParams p) {
     for (int m = 2; m < 32; m <<= 1) mc = fmaxf(mc, __shfl_xor_sync(FULL, mc, m));
     const float m_new = fmaxf(m_run[0], mc);
     if (m_new != m_run[0]) {
-      const float alpha = (m_run[0] == kNegInf) ? 0.0f : exp2f(m_run[0] - m_new);
-      l_run[0] *= alpha;
-      if constexpr (C::RES) wsum[0] *= alpha;
-#pragma unroll
-      for (int k = 0; k < DPL; ++k) {
-        accV[0][k] *= alpha;
-        if constexpr (C::RES) accC[0][k] *= alpha;
-      }
+      rescale(0, (m_run[0] == kNegInf) ? 0.0f : exp2f(m_run[0] - m_new));
       m_run[0] = m_new;
     }
     const float pme = (sc == kNegInf) ? 0.0f : exp2f(sc - m_new);
@@ -551,20 +615,14 @@ decode_kernel(const DecodeParams p) {
       const float pu = __shfl_sync(FULL, pme, slot * LPT + 2 * u);
       const int tok = warp * C::TPW + u * TPS + slot;
       if (tok < n) {
-        float vf[DPL];
-        load_row<DPL>(st + C::OFF_V + tok * C::KROW + dim0 * 2, vf);
-#pragma unroll
-        for (int k = 0; k < DPL; ++k) accV[0][k] = fmaf(pu, vf[k], accV[0][k]);
+        float2 vf[NP], cf[NP];
+        v_pairs(st + C::OFF_V + tok * C::KROW + dim0 * 2, vf);
+        float s_v = 0.0f;
         if constexpr (C::RES) {
-          const uint32_t word =
-              reinterpret_cast<const uint32_t*>(st + C::OFF_CV)[tok * C::CWORDS + cw];
-          const float wv = pu * half_at(st + C::OFF_SV + sc_off + tok * SB + grp * 2);
-          float cf[DPL];
-          codes_positional<PB, DPL>(word >> csh, cf);
-          wsum[0] += wv;
-#pragma unroll
-          for (int k = 0; k < DPL; ++k) accC[0][k] = fmaf(wv, cf[k], accC[0][k]);
+          code_pairs(reinterpret_cast<const uint32_t*>(st + C::OFF_CV)[tok * C::CWORDS + cw], cf);
+          s_v = half_at(st + C::OFF_SV + sc_off + tok * SB + grp * 2);
         }
+        accumulate_v(0, pu, vf, cf, s_v);
       }
     }
   };
@@ -577,34 +635,29 @@ decode_kernel(const DecodeParams p) {
 #pragma unroll
       for (int u = 0; u < CH; ++u) {
         const int tok = warp * C::TPW + (c0 + u) * TPS + slot;
-        float kf[DPL];
-        load_row<DPL>(st + C::OFF_K + tok * C::KROW + dim0 * 2, kf);
+        const unsigned char* kp = st + C::OFF_K + tok * C::KROW + dim0 * 2;
         float dot[G];
 #pragma unroll
-        for (int r = 0; r < G; ++r) {
-          dot[r] = 0.0f;
-#pragma unroll
-          for (int k = 0; k < DPL; ++k) dot[r] = fmaf(qa[r][k], kf[k], dot[r]);
-        }
+        for (int r = 0; r < G; ++r) dot[r] = ref_dot(kp, r);
         if constexpr (C::RES) {
           const uint32_t word =
               reinterpret_cast<const uint32_t*>(st + C::OFF_CK)[tok * C::CWORDS + cw];
           const float s_k = half_at(st + C::OFF_SK + sc_off + tok * SB + grp * 2);
-          float cf[DPL];
-          codes_positional<PB, DPL>(word >> csh, cf);
+          float2 cf[NP];
+          code_pairs(word, cf);
 #pragma unroll
           for (int r = 0; r < G; ++r) {
-            float res = -qoff[r];
+            float2 acc = make_float2(-qoff[r], 0.0f);
 #pragma unroll
-            for (int k = 0; k < DPL; ++k) res = fmaf(qc[r][k], cf[k], res);
-            dot[r] = fmaf(s_k, res, dot[r]);
+            for (int j = 0; j < NP; ++j) acc = __ffma2_rn(qc[r][j], cf[j], acc);
+            dot[r] = fmaf(s_k, acc.x + acc.y, dot[r]);
           }
         }
 #pragma unroll
         for (int r = 0; r < G; ++r) {
 #pragma unroll
           for (int m = 1; m < LPT; m <<= 1) dot[r] += __shfl_xor_sync(FULL, dot[r], m);
-          sc[r][u] = (tok < n) ? dot[r] : kNegInf;
+          sc[r][u] = (tok < n) ? score_scale * dot[r] : kNegInf;
         }
       }
       float pw[G][CH];
@@ -617,14 +670,7 @@ decode_kernel(const DecodeParams p) {
         for (int m = LPT; m < 32; m <<= 1) mc = fmaxf(mc, __shfl_xor_sync(FULL, mc, m));
         const float m_new = fmaxf(m_run[r], mc);
         if (m_new != m_run[r]) {
-          const float alpha = (m_run[r] == kNegInf) ? 0.0f : exp2f(m_run[r] - m_new);
-          l_run[r] *= alpha;
-          if constexpr (C::RES) wsum[r] *= alpha;
-#pragma unroll
-          for (int k = 0; k < DPL; ++k) {
-            accV[r][k] *= alpha;
-            if constexpr (C::RES) accC[r][k] *= alpha;
-          }
+          rescale(r, (m_run[r] == kNegInf) ? 0.0f : exp2f(m_run[r] - m_new));
           m_run[r] = m_new;
         }
 #pragma unroll
@@ -637,27 +683,16 @@ decode_kernel(const DecodeParams p) {
       for (int u = 0; u < CH; ++u) {
         const int tok = warp * C::TPW + (c0 + u) * TPS + slot;
         if (tok < n) {
-          float vf[DPL];
-          load_row<DPL>(st + C::OFF_V + tok * C::KROW + dim0 * 2, vf);
-#pragma unroll
-          for (int r = 0; r < G; ++r) {
-#pragma unroll
-            for (int k = 0; k < DPL; ++k) accV[r][k] = fmaf(pw[r][u], vf[k], accV[r][k]);
-          }
+          float2 vf[NP], cf[NP];
+          v_pairs(st + C::OFF_V + tok * C::KROW + dim0 * 2, vf);
+          float s_v = 0.0f;
           if constexpr (C::RES) {
-            const uint32_t word =
-                reinterpret_cast<const uint32_t*>(st + C::OFF_CV)[tok * C::CWORDS + cw];
-            const float s_v = half_at(st + C::OFF_SV + sc_off + tok * SB + grp * 2);
-            float cf[DPL];
-            codes_positional<PB, DPL>(word >> csh, cf);
-#pragma unroll
-            for (int r = 0; r < G; ++r) {
-              const float wv = pw[r][u] * s_v;
-              wsum[r] += wv;
-#pragma unroll
-              for (int k = 0; k < DPL; ++k) accC[r][k] = fmaf(wv, cf[k], accC[r][k]);
-            }
+            code_pairs(reinterpret_cast<const uint32_t*>(st + C::OFF_CV)[tok * C::CWORDS + cw],
+                       cf);
+            s_v = half_at(st + C::OFF_SV + sc_off + tok * SB + grp * 2);
           }
+#pragma unroll
+          for (int r = 0; r < G; ++r) accumulate_v(r, pw[r][u], vf, cf, s_v);
         }
       }
     }

@@ -39,6 +39,20 @@ __device__ __forceinline__ float rot_scale() {
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
+// acc + a.lo * b.lo + a.hi * b.hi for two packed bf16 pairs, each step one
+// fused multiply-add with an fp32 accumulator (bf16 x bf16 products are exact
+// in fp32, so this equals widening both operands and using fmaf).
+__device__ __forceinline__ float fma_bf16x2(uint32_t a2, uint32_t b2, float acc) {
+  asm("{\n\t.reg .b16 al, ah, bl, bh;\n\t"
+      "mov.b32 {al, ah}, %1;\n\t"
+      "mov.b32 {bl, bh}, %2;\n\t"
+      "fma.rn.f32.bf16 %0, al, bl, %0;\n\t"
+      "fma.rn.f32.bf16 %0, ah, bh, %0;\n\t}"
+      : "+f"(acc)
+      : "r"(a2), "r"(b2));
+  return acc;
+}
+
 __device__ __forceinline__ float flip_sign(float x, uint32_t neg) {
   return __uint_as_float(__float_as_uint(x) ^ (neg << 31));
 }

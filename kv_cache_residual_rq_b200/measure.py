@@ -1,0 +1,114 @@
+"""Per-workload kernel timings (one layer each), for the measured tables.
+
+    python -m kv_cache_residual_rq_b200.measure [--workloads a,b] [--reps N]
+
+For every workload: the decode call of each distinct loop kind (residual INT2,
+INT4, BF16 reference) over one full layer, and rq_encode of one layer's K
+(all non-final loops), timed with CUDA events on the launching stream after
+warm-up, inputs larger than L2 or the L2 flushed between repetitions.
+Prints one JSON line per measurement with algorithmic bytes, GB/s and the
+fraction of the measured HBM copy bandwidth.
+"""
+import argparse
+import json
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def _peak():
+    try:
+        return float(json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["hbm_gbs"])
+    except (OSError, ValueError, KeyError):
+        return 6650.0
+
+
+def decode_bytes(w, bits, batch=None):
+    b = w.batch if batch is None else batch
+    heads_t = b * w.kv_heads * w.ctx
+    n = 2 * heads_t * w.head_dim * 2
+    if bits != 16:
+        n += 2 * heads_t * w.head_dim * bits // 8 + 2 * heads_t * (w.head_dim // w.group) * 2
+    return n + b * w.q_heads * w.head_dim * 6
+
+
+def encode_bytes(w, rows):
+    active = [b for b in w.bits if b != 16]
+    read = rows * w.head_dim * 2 * (1 + len(active))
+    written = sum(rows * (w.head_dim * b // 8 + 2 * w.head_dim // w.group) for b in active)
+    return read + written
+
+
+def _time(fn, reps, flush):
+    import torch
+    for _ in range(3):
+        fn()
+    times = []
+    for _ in range(reps):
+        if flush is not None:
+            flush.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b) / 1e3)
+    times.sort()
+    return times[len(times) // 2]
+
+
+def measure(w, reps, peak, emit):
+    import torch
+    import kv_cache_residual_rq_b200 as rq
+    from kv_cache_residual_rq_b200 import synth
+    dev = torch.device("cuda:0")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > L2
+    refk = synth.reference(w, 0, 0, dev)
+    refv = synth.reference(w, 0, 1, dev)
+    q = synth.query(w, 0, 1, dev)
+    xk = [synth.loop_kv(w, 0, 0, l, refk) for l in range(1, w.loops)]
+    rows = refk.numel() // w.head_dim
+    t = _time(lambda: rq.encode(xk, refk, list(w.bits), w.group, w.seed), reps, flush)
+    nb = encode_bytes(w, rows)
+    emit({"workload": w.name, "kernel": "encode", "rows": rows, "loops": len(w.bits),
+          "us": t * 1e6, "bytes": nb, "gbs": nb / t / 1e9, "frac": nb / t / 1e9 / peak})
+    ck, sk = rq.encode(xk, refk, list(w.bits), w.group, w.seed)
+    xv = [synth.loop_kv(w, 0, 1, l, refv) for l in range(1, w.loops)]
+    cv, sv = rq.encode(xv, refv, list(w.bits), w.group, w.seed)
+    del xk, xv
+    torch.cuda.empty_cache()
+    shape = rq.make_shape(w.batch, w.kv_heads, w.ctx, w.head_dim, w.group, w.q_heads)
+    ws = rq.alloc_workspace(shape, dev)
+    out = torch.empty((w.batch, w.q_heads, w.head_dim), dtype=torch.float32, device=dev)
+    kinds = {}
+    for l, b in enumerate(w.bits):
+        kinds.setdefault(b, l)
+    kinds.setdefault(16, None)
+    for b, l in sorted(kinds.items()):
+        args = (None,) * 4 if b == 16 else (ck[l], cv[l], sk[l], sv[l])
+        fn = lambda: rq.rq_decode_attention(shape, q, refk, refv, *args, b, w.seed, 0.0, out, ws)
+        t = _time(fn, reps, None)
+        nb = decode_bytes(w, b)
+        emit({"workload": w.name, "kernel": f"decode bits={b}", "G": w.G, "us": t * 1e6,
+              "bytes": nb, "gbs": nb / t / 1e9, "frac": nb / t / 1e9 / peak,
+              "tokens_per_s_per_head_call": w.batch / t})
+    assert rq.rq_workspace_status(ws) == 0
+
+
+def main(argv=None):
+    from kv_cache_residual_rq_b200 import synth
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--workloads", default=",".join(w.name for w in synth.WORKLOADS))
+    ap.add_argument("--reps", type=int, default=20)
+    args = ap.parse_args(argv)
+    peak = _peak()
+    for name in args.workloads.split(","):
+        measure(synth.BY_NAME[name], args.reps, peak, lambda d: print(json.dumps(d), flush=True))
+
+
+if __name__ == "__main__":
+    main()
