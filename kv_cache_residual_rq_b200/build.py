@@ -22,6 +22,7 @@ NVCC_FLAGS = [
     "-Xcompiler", "-fPIC,-O2,-Wall",
     "-Xptxas", "-v",
     "--expt-relaxed-constexpr",
+    "-diag-suppress=177",
     "-cudart", "static",
 ]
 

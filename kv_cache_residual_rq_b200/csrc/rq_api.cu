@@ -206,7 +206,10 @@ rq_status rq_decode_attention(const rq_shape* shape, const uint16_t* q, const ui
   const float sigma =
       softmax_scale > 0.0f ? softmax_scale : 1.0f / std::sqrt((float)shape->head_dim);
   p.score_scale = sigma * 1.4426950408889634f;   // log2(e)
-  cudaError_t e = launch_decode(shape->head_dim, G, bits, p, static_cast<cudaStream_t>(stream));
+  cudaError_t e = (G == 1)
+                      ? launch_decode(shape->head_dim, G, bits, p, static_cast<cudaStream_t>(stream))
+                      : launch_decode_gqa(shape->head_dim, G, bits, p,
+                                          static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? RQ_OK : RQ_ERR_CUDA;
 }
 

@@ -44,18 +44,12 @@
 //     accumulators are packed fp32 pairs updated with the paired FMA.
 // Every mbarrier wait is bounded; a wait that runs out raises the workspace
 // status word, and the kernel still finishes (its output is then invalid).
-#include <cmath>
-
-#include "rq_device.cuh"
-#include "rq_internal.h"
+#include "rq_decode_common.cuh"
 
 namespace rq {
 namespace {
 
-constexpr int kConsumerWarps = 4;
-constexpr int kConsumerThreads = kConsumerWarps * 32;
-constexpr int kThreads = kConsumerThreads + 32;
-constexpr float kNegInf = -INFINITY;
+constexpr int kThreads = kDecodeThreads;
 
 template <int D, int G, int BITS>
 struct Cfg {
@@ -125,14 +119,6 @@ template <int BITS, int DPL>
 __host__ __device__ constexpr float pos_factor(int k) {
   return (BITS * DPL > 16) ? 1.0f / (float)(1u << (BITS * (k % (DPL / 2))))
                            : 1.0f / (float)(1u << (BITS * k));
-}
-
-__device__ __forceinline__ void flag_error(uint32_t* status, uint32_t bit) {
-  atomicOr(status, bit);
-}
-
-__device__ __forceinline__ float half_at(const unsigned char* p) {
-  return __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t*>(p)));
 }
 
 template <int D, int G, int BITS>
@@ -274,30 +260,9 @@ decode_kernel(const DecodeParams p) {
   // load and rotate the G query rows of head hd (and fill the K table);
   // all consumer threads
   auto setup_head = [&](long long hd) {
-    const int b = (int)(hd / p.kv_heads);
-    const int h = (int)(hd % p.kv_heads);
     float* qs = qbuf;              // [G][D] raw q
-    float* qt = qbuf + G * D;      // [G][D] rotated
-    named_bar_sync(1, kConsumerThreads);          // previous users of qbuf / area done
-    for (int e = tid; e < G * D; e += kConsumerThreads) {
-      const int r = e / D, i = e % D;
-      const uint16_t raw = p.q[((size_t)b * p.q_heads + (size_t)h * G + r) * D + i];
-      const float v = __uint_as_float((uint32_t)raw << 16);
-      qs[e] = v;
-      qt[e] = flip_sign(v, sign_bit(p.seed, i));
-    }
-    for (int hs = 1; hs < D; hs <<= 1) {
-      named_bar_sync(1, kConsumerThreads);
-      for (int e = tid; e < G * D / 2; e += kConsumerThreads) {
-        const int r = e / (D / 2), pr = e % (D / 2);
-        const int i = (pr / hs) * 2 * hs + (pr % hs);
-        float* row = qt + r * D;
-        const float a = row[i], c = row[i + hs];
-        row[i] = a + c;
-        row[i + hs] = a - c;
-      }
-    }
-    named_bar_sync(1, kConsumerThreads);
+    float* qt = qbuf + G * D;      // [G][D] FWHT(D q)
+    load_rotate_queries<D, G>(p, hd, qs, qt, tid);
     const float cd = rot_scale<D>();
     if constexpr (C::LUT) {
       // lut[byte][slice] = sum_k q~[4 slice + k] * l(c_k(byte)), l(c) = 2c - 3,
@@ -343,8 +308,6 @@ decode_kernel(const DecodeParams p) {
   // merge the 4 warps' states, write the head's partial record, and if this
   // CTA is the last contributor, finish the head
   auto flush_head = [&](long long hd) {
-    const int b = (int)(hd / p.kv_heads);
-    const int h = (int)(hd % p.kv_heads);
     // fold the token slots of the warp together
 #pragma unroll
     for (int r = 0; r < G; ++r) {
@@ -399,95 +362,7 @@ decode_kernel(const DecodeParams p) {
     }
     named_bar_sync(1, kConsumerThreads);
 
-    // which records belong to this head, and which one is ours
-    const long long f = hd * p.nt, e = f + p.nt - 1;
-    const int c_first = (int)(((f + 1) * p.ctas - 1) / p.n_tiles);
-    const int c_last = (int)(((e + 1) * p.ctas - 1) / p.n_tiles);
-    const int ncontrib = c_last - c_first + 1;
-    const int j = cta - c_first;
-    if (j < 0 || j >= p.max_contrib || ncontrib > p.max_contrib) {
-      if (tid == 0) flag_error(p.status, 4u);
-      return;
-    }
-    float* recs = p.records + (size_t)hd * p.max_contrib * G * (4 + 2 * D);
-    for (int eidx = tid; eidx < G * (2 * D + 2); eidx += kConsumerThreads) {
-      const int r = eidx / (2 * D + 2), q = eidx % (2 * D + 2);
-      float M = kNegInf;
-#pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w)
-        M = fmaxf(M, merge[(w * G + r) * (2 + 2 * D)]);
-      float* out_rec = recs + ((size_t)j * G + r) * (4 + 2 * D);
-      if (q == 0) {
-        out_rec[0] = M;
-      } else {
-        float acc = 0.0f;
-#pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) {
-          const float* mr = merge + (w * G + r) * (2 + 2 * D);
-          const float wt = (mr[0] == kNegInf) ? 0.0f : exp2f(mr[0] - M);
-          acc += wt * mr[q];
-        }
-        out_rec[q == 1 ? 1 : q + 2] = acc;   // l at 1; accRef/accRes from 4
-      }
-    }
-    __threadfence();
-    named_bar_sync(1, kConsumerThreads);
-    if (tid == 0) {
-      const uint32_t old = atomicAdd(&p.counters[hd], 1u);
-      const int last = (old == (uint32_t)(ncontrib - 1));
-      if (last) {
-        p.counters[hd] = 0u;      // ready for the next call
-        __threadfence();
-      }
-      flags[1] = last;
-    }
-    named_bar_sync(1, kConsumerThreads);
-    if (!flags[1]) return;
-
-    // ---- last contributor: merge all records of the head, finish ----
-    float* zres = merge;          // [G][D] rotated-domain residual sums
-    float* zref = merge + G * D;  // [G][D]
-    float* lsum = merge + 2 * G * D;   // [G]
-    for (int eidx = tid; eidx < G * D; eidx += kConsumerThreads) {
-      const int r = eidx / D, i = eidx % D;
-      float M = kNegInf;
-      for (int c = 0; c < ncontrib; ++c)
-        M = fmaxf(M, __ldcg(recs + ((size_t)c * G + r) * (4 + 2 * D)));
-      float aref = 0.0f, ares = 0.0f, l = 0.0f;
-      for (int c = 0; c < ncontrib; ++c) {
-        const float* rc = recs + ((size_t)c * G + r) * (4 + 2 * D);
-        const float mc = __ldcg(rc);
-        const float wt = (mc == kNegInf) ? 0.0f : exp2f(mc - M);
-        l += wt * __ldcg(rc + 1);
-        aref += wt * __ldcg(rc + 4 + i);
-        if constexpr (C::RES) ares += wt * __ldcg(rc + 4 + D + i);
-      }
-      zref[eidx] = aref;
-      zres[eidx] = ares;
-      if (i == 0) lsum[r] = l;
-    }
-    if constexpr (C::RES) {
-      // Rot^T z = D (c_d H z): butterflies, then scale and signs
-      for (int hs = 1; hs < D; hs <<= 1) {
-        named_bar_sync(1, kConsumerThreads);
-        for (int eidx = tid; eidx < G * D / 2; eidx += kConsumerThreads) {
-          const int r = eidx / (D / 2), pr = eidx % (D / 2);
-          const int i = (pr / hs) * 2 * hs + (pr % hs);
-          float* row = zres + r * D;
-          const float a = row[i], c = row[i + hs];
-          row[i] = a + c;
-          row[i + hs] = a - c;
-        }
-      }
-    }
-    named_bar_sync(1, kConsumerThreads);
-    const float cd = rot_scale<D>();
-    for (int eidx = tid; eidx < G * D; eidx += kConsumerThreads) {
-      const int r = eidx / D, i = eidx % D;
-      float num = zref[eidx];
-      if constexpr (C::RES) num += flip_sign(cd * zres[eidx], sign_bit(p.seed, i));
-      p.out[((size_t)b * p.q_heads + (size_t)h * G + r) * D + i] = num / lsum[r];
-    }
+    finish_head<D, G, C::RES>(p, hd, cta, merge, flags, tid);
   };
 
   // <q, K row> of the lane's dims, straight from the packed bf16 row
@@ -766,13 +641,8 @@ cudaError_t launch_decode_g(int bits, const DecodeParams& p, cudaStream_t stream
 
 template <int D>
 cudaError_t launch_decode_d(int G, int bits, const DecodeParams& p, cudaStream_t stream) {
-  switch (G) {
-    case 1: return launch_decode_g<D, 1>(bits, p, stream);
-    case 2: return launch_decode_g<D, 2>(bits, p, stream);
-    case 4: return launch_decode_g<D, 4>(bits, p, stream);
-    case 8: return launch_decode_g<D, 8>(bits, p, stream);
-    default: return cudaErrorInvalidValue;
-  }
+  if (G == 1) return launch_decode_g<D, 1>(bits, p, stream);
+  return cudaErrorInvalidValue;     // grouped queries: rq_decode_gqa.cu
 }
 
 }  // namespace

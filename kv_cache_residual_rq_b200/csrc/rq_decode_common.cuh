@@ -1,0 +1,163 @@
+// rq_decode_common.cuh -- pieces shared by the decode-attention kernels.
+//
+// Both decode kernels (the CUDA-core kernel for one query row per kv head and
+// the tensor-core kernel for grouped queries) split a call the same way: the
+// (head, tile) space is cut into equal runs, one per persistent CTA; at the
+// end of a head's run the CTA's consumer warps leave their softmax states in
+// shared memory and call finish_head, which writes the CTA's partial record
+// and, in the last CTA to arrive for the head, merges all records and applies
+// the inverse rotation once per output row.
+#pragma once
+
+#include <cmath>
+
+#include "rq_device.cuh"
+#include "rq_internal.h"
+
+namespace rq {
+
+constexpr int kConsumerWarps = 4;
+constexpr int kConsumerThreads = kConsumerWarps * 32;
+constexpr int kDecodeThreads = kConsumerThreads + 32;   // + one producer warp
+constexpr float kNegInf = -INFINITY;
+
+__device__ __forceinline__ void flag_error(uint32_t* status, uint32_t bit) {
+  atomicOr(status, bit);
+}
+
+// fp16 value (bits in shared memory) as float
+__device__ __forceinline__ float half_at(const unsigned char* p) {
+  return __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t*>(p)));
+}
+
+// Loads the G query rows of head hd into qs[G][D] (fp32) and FWHT(D q) into
+// qt[G][D]: the rotation q~ = Rot q without its 1/sqrt(d) factor, which the
+// caller applies.  All consumer threads; ends with a consumer barrier.
+template <int D, int G>
+__device__ __forceinline__ void load_rotate_queries(const DecodeParams& p, long long hd,
+                                                    float* qs, float* qt, int tid) {
+  const int b = (int)(hd / p.kv_heads);
+  const int h = (int)(hd % p.kv_heads);
+  named_bar_sync(1, kConsumerThreads);          // previous users of the buffers done
+  for (int e = tid; e < G * D; e += kConsumerThreads) {
+    const int r = e / D, i = e % D;
+    const uint16_t raw = p.q[((size_t)b * p.q_heads + (size_t)h * G + r) * D + i];
+    const float v = __uint_as_float((uint32_t)raw << 16);
+    qs[e] = v;
+    qt[e] = flip_sign(v, sign_bit(p.seed, i));
+  }
+  for (int hs = 1; hs < D; hs <<= 1) {
+    named_bar_sync(1, kConsumerThreads);
+    for (int e = tid; e < G * D / 2; e += kConsumerThreads) {
+      const int r = e / (D / 2), pr = e % (D / 2);
+      const int i = (pr / hs) * 2 * hs + (pr % hs);
+      float* row = qt + r * D;
+      const float a = row[i], c = row[i + hs];
+      row[i] = a + c;
+      row[i + hs] = a - c;
+    }
+  }
+  named_bar_sync(1, kConsumerThreads);
+}
+
+// merge[w][r] = {m, l, accRef[D], accRes[D]} of consumer warp w and query row
+// r (m in base-2 units, accRes in the rotated domain) must be complete and
+// visible to all consumer threads.  Writes this CTA's record of head hd and,
+// if it is the last CTA of the head to arrive, the head's output.  All
+// consumer threads call it; `merge` is reused as scratch.
+template <int D, int G, bool RES>
+__device__ __forceinline__ void finish_head(const DecodeParams& p, long long hd, int cta,
+                                            float* merge, volatile int* flags, int tid) {
+  const int b = (int)(hd / p.kv_heads);
+  const int h = (int)(hd % p.kv_heads);
+  // which records belong to this head, and which one is ours
+  const long long f = hd * p.nt, e = f + p.nt - 1;
+  const int c_first = (int)(((f + 1) * p.ctas - 1) / p.n_tiles);
+  const int c_last = (int)(((e + 1) * p.ctas - 1) / p.n_tiles);
+  const int ncontrib = c_last - c_first + 1;
+  const int j = cta - c_first;
+  if (j < 0 || j >= p.max_contrib || ncontrib > p.max_contrib) {
+    if (tid == 0) flag_error(p.status, 4u);
+    return;
+  }
+  float* recs = p.records + (size_t)hd * p.max_contrib * G * (4 + 2 * D);
+  for (int eidx = tid; eidx < G * (2 * D + 2); eidx += kConsumerThreads) {
+    const int r = eidx / (2 * D + 2), q = eidx % (2 * D + 2);
+    float M = kNegInf;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, merge[(w * G + r) * (2 + 2 * D)]);
+    float* out_rec = recs + ((size_t)j * G + r) * (4 + 2 * D);
+    if (q == 0) {
+      out_rec[0] = M;
+    } else {
+      float acc = 0.0f;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) {
+        const float* mr = merge + (w * G + r) * (2 + 2 * D);
+        const float wt = (mr[0] == kNegInf) ? 0.0f : exp2f(mr[0] - M);
+        acc += wt * mr[q];
+      }
+      out_rec[q == 1 ? 1 : q + 2] = acc;   // l at 1; accRef/accRes from 4
+    }
+  }
+  __threadfence();
+  named_bar_sync(1, kConsumerThreads);
+  if (tid == 0) {
+    const uint32_t old = atomicAdd(&p.counters[hd], 1u);
+    const int last = (old == (uint32_t)(ncontrib - 1));
+    if (last) {
+      p.counters[hd] = 0u;      // ready for the next call
+      __threadfence();
+    }
+    flags[1] = last;
+  }
+  named_bar_sync(1, kConsumerThreads);
+  if (!flags[1]) return;
+
+  // ---- last contributor: merge all records of the head, finish ----
+  float* zres = merge;               // [G][D] rotated-domain residual sums
+  float* zref = merge + G * D;       // [G][D]
+  float* lsum = merge + 2 * G * D;   // [G]
+  for (int eidx = tid; eidx < G * D; eidx += kConsumerThreads) {
+    const int r = eidx / D, i = eidx % D;
+    float M = kNegInf;
+    for (int c = 0; c < ncontrib; ++c)
+      M = fmaxf(M, __ldcg(recs + ((size_t)c * G + r) * (4 + 2 * D)));
+    float aref = 0.0f, ares = 0.0f, l = 0.0f;
+    for (int c = 0; c < ncontrib; ++c) {
+      const float* rc = recs + ((size_t)c * G + r) * (4 + 2 * D);
+      const float mc = __ldcg(rc);
+      const float wt = (mc == kNegInf) ? 0.0f : exp2f(mc - M);
+      l += wt * __ldcg(rc + 1);
+      aref += wt * __ldcg(rc + 4 + i);
+      if constexpr (RES) ares += wt * __ldcg(rc + 4 + D + i);
+    }
+    zref[eidx] = aref;
+    zres[eidx] = ares;
+    if (i == 0) lsum[r] = l;
+  }
+  if constexpr (RES) {
+    // Rot^T z = D (c_d H z): butterflies, then scale and signs
+    for (int hs = 1; hs < D; hs <<= 1) {
+      named_bar_sync(1, kConsumerThreads);
+      for (int eidx = tid; eidx < G * D / 2; eidx += kConsumerThreads) {
+        const int r = eidx / (D / 2), pr = eidx % (D / 2);
+        const int i = (pr / hs) * 2 * hs + (pr % hs);
+        float* row = zres + r * D;
+        const float a = row[i], c = row[i + hs];
+        row[i] = a + c;
+        row[i + hs] = a - c;
+      }
+    }
+  }
+  named_bar_sync(1, kConsumerThreads);
+  const float cd = rot_scale<D>();
+  for (int eidx = tid; eidx < G * D; eidx += kConsumerThreads) {
+    const int r = eidx / D, i = eidx % D;
+    float num = zref[eidx];
+    if constexpr (RES) num += flip_sign(cd * zres[eidx], sign_bit(p.seed, i));
+    p.out[((size_t)b * p.q_heads + (size_t)h * G + r) * D + i] = num / lsum[r];
+  }
+}
+
+}  // namespace rq

@@ -1,0 +1,652 @@
+// rq_decode_gqa.cu -- ResidualQuant decode attention for grouped queries
+// (G = q_heads / kv_heads in {2, 4, 8}) on the sm_100a tensor cores.
+//
+// Method: "ResidualQuant: KV Cache Quantization for Looped Transformers with
+// 2-Bit Residuals", Abstract -- decode rebuilds each non-final loop's K/V
+// from the BF16 final-loop reference plus the loop's rotated low-bit residual.
+//
+// With G query rows per kv head every K/V tile is shared by G rows, so the
+// four products of the fused attention are small dense contractions and go to
+// the tensor cores (mma.sync m16n8k16, fp32 accumulation), per warp and per
+// 16 tokens of a 64-token tile:
+//   S_ref = Q  K^T          bf16 x bf16      (K from shared memory, ldmatrix)
+//   S_res = Q~ L_K^T        fp16 x fp16      per scale group, then x s^K
+//   O_ref^T += V^T P^T      bf16 x bf16      (V via ldmatrix.trans; P split
+//                                             into bf16 hi + lo, so the
+//                                             weights keep ~16 bits)
+//   O_res^T += C_V^T (P s^V)^T  fp16 x fp16  (C_V = codes, exact in fp16)
+// L_K are the levels 2c - (2^b - 1) and C_V the codes c, both built from the
+// packed words in registers; sum_t p s (2c - (2^b-1)) = 2 (C_V^T (P s)^T) -
+// (2^b - 1) sum_t p s is completed when the warp flushes.  Rows beyond G are
+// zero and their weights are forced to zero.
+//
+// The reference K/V tiles arrive by TMA tensor copies with the 128-byte
+// swizzle (conflict-free ldmatrix); codes and scales by plain bulk copies, as
+// in the single-query kernel.  The work split, the partial records and the
+// last-arriving-CTA merge with the single inverse rotation are shared with it
+// (rq_decode_common.cuh).  Every mbarrier wait is bounded.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+
+#include "rq_decode_common.cuh"
+
+namespace rq {
+namespace {
+
+struct alignas(64) GqaParams {
+  CUtensorMap tmap_k;        // reference K viewed as [rows][d] bf16, box 64 x 64, swizzle 128B
+  CUtensorMap tmap_v;
+  DecodeParams p;
+};
+
+template <int D, int G, int BITS, int GROUP>
+struct GCfg {
+  static constexpr int TILE = kDecodeTile;                 // 64 tokens
+  static constexpr int WTOK = TILE / kConsumerWarps;       // 16 tokens per warp
+  static constexpr bool RES = (BITS != 16);
+  static constexpr int NBOX = D / 64;                      // 64-column boxes per row
+  static constexpr int BOX_BYTES = 64 * 128;               // 64 rows x 128 B
+  static constexpr int KT = D / 16;                        // k-steps of 16 dims
+  static constexpr int CROW = RES ? D * BITS / 8 : 0;      // code bytes per token
+  static constexpr int CWORDS = CROW / 4;
+  static constexpr int SC_BYTES = RES ? TILE * (2 * D / 32) + 32 : 0;
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + NBOX * BOX_BYTES;
+  static constexpr int OFF_CK = OFF_V + NBOX * BOX_BYTES;
+  static constexpr int OFF_CV = OFF_CK + TILE * CROW;
+  static constexpr int OFF_SK = OFF_CV + TILE * CROW;
+  static constexpr int OFF_SV = OFF_SK + SC_BYTES;
+  static constexpr int STAGE_BYTES = (OFF_SV + SC_BYTES + 1023) / 1024 * 1024;
+  static constexpr int STAGES = 2;
+  static constexpr int RING_BYTES = STAGES * STAGE_BYTES;
+  static constexpr int MERGE_FLOATS = kConsumerWarps * G * (2 + 2 * D);
+  static constexpr int QBUF_FLOATS = 2 * G * D;
+  static constexpr int NG = D / GROUP;                      // scale groups per token
+  static constexpr int KSG = GROUP / 16;                   // k-steps per scale group
+  static constexpr int SB = 2 * NG;                        // scale bytes per token
+  static constexpr int WSUM_FLOATS = kConsumerWarps * G * NG;
+  static constexpr int QFRAG_WORDS = 2 * KT * 32 * 2;       // bf16 q and fp16 q~ A fragments
+  static constexpr int SMEM_BYTES = 1024 /* base alignment slack */ + RING_BYTES +
+                                    4 * (MERGE_FLOATS + QBUF_FLOATS + WSUM_FLOATS +
+                                         QFRAG_WORDS) +
+                                    2 * STAGES * 8 + 16;
+  static_assert(G == 2 || G == 4 || G == 8, "grouped queries");
+  static_assert(GROUP == 32 || GROUP == 64, "scale group");
+  static_assert(D == 64 || D == 128, "head_dim");
+};
+
+// ---- PTX wrappers -----------------------------------------------------------
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+// D(16x8, f32) += A(16x16) B(16x8); A row-major, B column-major fragments.
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                        uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// {lo, hi} -> packed bf16x2 / f16x2 (round to nearest)
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ uint32_t hfma2_u(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t r;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+  return r;
+}
+__device__ __forceinline__ uint32_t hadd2_u(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ float bf16_lo_f(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi_f(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+constexpr uint32_t kMagic = 0x64006400u;   // fp16 1024 in both halves
+
+// Levels of the K codes for the B fragment of one k-step (16 dims) of one
+// token: b0 = {l(2q), l(2q+1)}, b1 = {l(2q+8), l(2q+9)}, fp16, exact.  INT2:
+// w0 is the k-step's word (code j at bits 2j); INT4: w0, w1 are its two words
+// (code j at bits 4j of word j / 8).
+template <int BITS>
+__device__ __forceinline__ void k_levels(uint32_t w0, uint32_t w1, int q, uint32_t& b0,
+                                         uint32_t& b1) {
+  if constexpr (BITS == 2) {
+    // lo halves take the code at bit 1 (value 1024 + 2c, level = v - 1027),
+    // hi halves at bit 18 (value 1024 + 4c, level = v/2 - 515)
+    const uint32_t x = w0 >> (4 * q);
+    const uint32_t v0 = ((x << 1) & 0x6u) | ((x << 16) & 0xC0000u) | kMagic;
+    const uint32_t v1 = ((x >> 15) & 0x6u) | (x & 0xC0000u) | kMagic;
+    const uint32_t mul = 0x38003C00u;   // {1.0, 0.5}
+    const uint32_t add = 0xE006E403u;   // {-1027, -515}
+    b0 = hfma2_u(v0, mul, add);
+    b1 = hfma2_u(v1, mul, add);
+  } else {
+    // both halves take the code at bit 1 (value 1024 + 2c, level 2c - 15 = v - 1039)
+    const uint32_t x0 = w0 >> (8 * q);
+    const uint32_t x1 = w1 >> (8 * q);
+    const uint32_t v0 = ((x0 << 1) & 0x1Eu) | ((x0 << 13) & 0x1E0000u) | kMagic;
+    const uint32_t v1 = ((x1 << 1) & 0x1Eu) | ((x1 << 13) & 0x1E0000u) | kMagic;
+    const uint32_t add = 0xE40FE40Fu;   // {-1039, -1039}
+    b0 = hadd2_u(v0, add);
+    b1 = hadd2_u(v1, add);
+  }
+}
+
+template <int D, int G, int BITS, int GROUP>
+__global__ void __launch_bounds__(kDecodeThreads, 2)
+decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
+  using C = GCfg<D, G, BITS, GROUP>;
+  const DecodeParams& p = gp.p;
+  constexpr int STAGES = C::STAGES, TILE = C::TILE, KT = C::KT;
+  constexpr unsigned FULL = 0xffffffffu;
+  constexpr int TOPLVL = C::RES ? (1 << BITS) - 1 : 0;
+  constexpr int NG = C::NG, KSG = C::KSG, SB = C::SB;
+
+  extern __shared__ unsigned char smem_raw[];
+  // the swizzled boxes need 1024-byte alignment
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  unsigned char* ring = smem;
+  float* merge = reinterpret_cast<float*>(smem + C::RING_BYTES);
+  float* qbuf = merge + C::MERGE_FLOATS;
+  float* wsum_s = qbuf + C::QBUF_FLOATS;
+  uint32_t* qfrag = reinterpret_cast<uint32_t*>(wsum_s + C::WSUM_FLOATS);  // [2][KT][32][2]
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(qfrag + C::QFRAG_WORDS);
+  uint64_t* empty_bar = full_bar + STAGES;
+  volatile int* flags = reinterpret_cast<volatile int*>(empty_bar + STAGES);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int cta = blockIdx.x;
+  if (cta >= p.ctas) return;
+
+  const long long tile_begin = (long long)cta * p.n_tiles / p.ctas;
+  const long long tile_end = (long long)(cta + 1) * p.n_tiles / p.ctas;
+  const int n_my = (int)(tile_end - tile_begin);
+
+  if (tid == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], kConsumerWarps);
+    }
+    flags[0] = 0;
+    flags[1] = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  const int T = p.ctx;
+
+  // ========================= producer warp ================================
+  if (warp == kConsumerWarps) {
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < n_my; ++i) {
+        const int s = i % STAGES;
+        if (i >= STAGES) {
+          if (!mbar_wait_bounded(&empty_bar[s], ((i / STAGES) - 1) & 1)) {
+            flag_error(p.status, 1u);
+            flags[0] = 1;
+            break;
+          }
+        }
+        if (flags[0]) break;
+        const long long tile = tile_begin + i;
+        const long long hd = tile / p.nt;
+        const int t0 = (int)(tile % p.nt) * TILE;
+        const int n = min(TILE, T - t0);
+        const size_t row = (size_t)hd * T + t0;
+        unsigned char* st = ring + s * C::STAGE_BYTES;
+        uint32_t bytes = 2u * C::NBOX * C::BOX_BYTES;     // full boxes, OOB rows zero-filled
+        size_t sc_lo = 0;
+        uint32_t sc_bytes = 0;
+        if constexpr (C::RES) {
+          const size_t start = row * SB;
+          sc_lo = start & ~(size_t)15;
+          sc_bytes = (uint32_t)(((start + (size_t)n * SB + 15) & ~(size_t)15) - sc_lo);
+          bytes += 2u * n * C::CROW + 2u * sc_bytes;
+        }
+        mbar_arrive_expect_tx(&full_bar[s], bytes);
+#pragma unroll
+        for (int bx = 0; bx < C::NBOX; ++bx) {
+          tma_load_2d(st + C::OFF_K + bx * C::BOX_BYTES, &gp.tmap_k, 64 * bx, (int)row, &full_bar[s]);
+          tma_load_2d(st + C::OFF_V + bx * C::BOX_BYTES, &gp.tmap_v, 64 * bx, (int)row, &full_bar[s]);
+        }
+        if constexpr (C::RES) {
+          bulk_g2s(st + C::OFF_CK, p.codes_k + row * C::CWORDS, n * C::CROW, &full_bar[s]);
+          bulk_g2s(st + C::OFF_CV, p.codes_v + row * C::CWORDS, n * C::CROW, &full_bar[s]);
+          bulk_g2s(st + C::OFF_SK, reinterpret_cast<const unsigned char*>(p.scales_k) + sc_lo,
+                   sc_bytes, &full_bar[s]);
+          bulk_g2s(st + C::OFF_SV, reinterpret_cast<const unsigned char*>(p.scales_v) + sc_lo,
+                   sc_bytes, &full_bar[s]);
+        }
+        ++issued;
+      }
+      for (int j = (issued > STAGES ? issued - STAGES : 0); j < issued; ++j)
+        if (!mbar_wait_bounded(&full_bar[j % STAGES], (j / STAGES) & 1)) flag_error(p.status, 2u);
+    }
+    return;
+  }
+
+  // ========================= consumer warps ===============================
+  const int g = lane >> 2;            // fragment row group
+  const int q = lane & 3;             // fragment column pair
+  const int wtok = warp * C::WTOK;    // this warp's first token in a tile
+  const bool row_ok = g < G;          // lanes whose S/P row is a real query row
+  const float score_scale = p.score_scale;
+
+  // The per-head Q A-fragments live in shared memory (qfrag): for k-step kk
+  // and lane, {a0, a2} of the bf16 query (kind 0) and of the fp16 rotated
+  // query q~ (kind 1): rows g, dims 16kk + 2q.. and 16kk + 2q + 8..; rows
+  // g >= G are zero, and a1 = a3 = 0 (rows g + 8).
+  auto qfrag_addr = [&](int kind, int kk) {
+    return smem_u32(qfrag + ((kind * KT + kk) * 32 + lane) * 2);
+  };
+  // softmax state of row g (lanes with row_ok), and the output accumulators
+  // (O^T fragments: dims 16mt + g (+8), rows 2q, 2q + 1)
+  float m_run = kNegInf, l_run = 0.0f;
+  float wsum[NG];
+  float oref[KT][4], ores[KT][4];
+
+  auto reset_state = [&]() {
+    m_run = kNegInf;
+    l_run = 0.0f;
+#pragma unroll
+    for (int j = 0; j < NG; ++j) wsum[j] = 0.0f;
+#pragma unroll
+    for (int mt = 0; mt < KT; ++mt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        oref[mt][e] = 0.0f;
+        ores[mt][e] = 0.0f;
+      }
+  };
+
+  auto setup_head = [&](long long hd) {
+    float* qs = qbuf;
+    float* qt = qbuf + G * D;
+    load_rotate_queries<D, G>(p, hd, qs, qt, tid);
+    const float cd = rot_scale<D>();
+    if (warp == 0) {
+#pragma unroll
+      for (int kk = 0; kk < KT; ++kk) {
+        uint32_t* fa = qfrag + ((0 * KT + kk) * 32 + lane) * 2;
+        uint32_t* fr = qfrag + ((1 * KT + kk) * 32 + lane) * 2;
+        if (row_ok) {
+          const float* qrow = qs + g * D + 16 * kk + 2 * q;
+          const float* trow = qt + g * D + 16 * kk + 2 * q;
+          fa[0] = pack_bf16(qrow[0], qrow[1]);       // exact: q is bf16
+          fa[1] = pack_bf16(qrow[8], qrow[9]);
+          fr[0] = pack_f16(cd * trow[0], cd * trow[1]);
+          fr[1] = pack_f16(cd * trow[8], cd * trow[9]);
+        } else {
+          fa[0] = fa[1] = fr[0] = fr[1] = 0u;
+        }
+      }
+    }
+    named_bar_sync(1, kConsumerThreads);
+  };
+
+  auto flush_head = [&](long long hd) {
+    // l and the V weight sums of row g over the four lanes of its row group
+    l_run += __shfl_xor_sync(FULL, l_run, 1);
+    l_run += __shfl_xor_sync(FULL, l_run, 2);
+#pragma unroll
+    for (int j = 0; j < NG; ++j) {
+      wsum[j] += __shfl_xor_sync(FULL, wsum[j], 1);
+      wsum[j] += __shfl_xor_sync(FULL, wsum[j], 2);
+    }
+    named_bar_sync(1, kConsumerThreads);          // merge area free
+    float* mw = merge + warp * G * (2 + 2 * D);
+    if (row_ok && q == 0) {
+      mw[g * (2 + 2 * D)] = m_run;
+      mw[g * (2 + 2 * D) + 1] = l_run;
+      if constexpr (C::RES) {
+#pragma unroll
+        for (int j = 0; j < NG; ++j) wsum_s[(warp * G + g) * NG + j] = wsum[j];
+      }
+    }
+    // O^T fragments: c0 (dim 16mt+g, row 2q), c1 (.., row 2q+1), c2/c3 dim +8
+#pragma unroll
+    for (int mt = 0; mt < KT; ++mt) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int r = 2 * q + (e & 1);
+        const int dim = 16 * mt + g + 8 * (e >> 1);
+        if (r < G) {
+          mw[r * (2 + 2 * D) + 2 + dim] = oref[mt][e];
+          if constexpr (C::RES) mw[r * (2 + 2 * D) + 2 + D + dim] = 2.0f * ores[mt][e] * (1.0f / 4096.0f);
+          else mw[r * (2 + 2 * D) + 2 + D + dim] = 0.0f;
+        }
+      }
+    }
+    named_bar_sync(1, kConsumerThreads);
+    if constexpr (C::RES) {
+      // complete sum_t p s (2c - top) = 2 sum p s c - top sum p s
+      for (int e = tid; e < kConsumerWarps * G * D; e += kConsumerThreads) {
+        const int w = e / (G * D), r = (e / D) % G, dim = e % D;
+        merge[(w * G + r) * (2 + 2 * D) + 2 + D + dim] -=
+            (float)TOPLVL * wsum_s[(w * G + r) * NG + dim / GROUP];
+      }
+      named_bar_sync(1, kConsumerThreads);
+    }
+    finish_head<D, G, C::RES>(p, hd, cta, merge, flags, tid);
+  };
+
+  // ---- one tile ----
+  auto tile_mma = [&](const unsigned char* st, int n, int sc_off) {
+    const uint32_t sK = smem_u32(st + C::OFF_K);
+    const uint32_t sV = smem_u32(st + C::OFF_V);
+    const int r7 = lane & 7;
+    // ---- scores for the warp's two 8-token tiles, k-steps outermost ----
+    // c[nt]: S_ref (then + s x S_res) fragments, row g, tokens 2q, 2q+1 of nt
+    float cref[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
+    float ct[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
+    const int tok0[2] = {wtok + 2 * q, wtok + 8 + 2 * q};     // tokens of c0 per tile
+    const int tb[2] = {wtok + g, wtok + 8 + g};               // B-fragment token per tile
+    // ldmatrix: matrices (tile 0, dims +0..7), (tile 0, +8..15), (tile 1, ..), (tile 1, ..)
+    const int ktr = wtok + ((lane >> 4) & 1) * 8 + r7;
+    const int kch = (lane >> 3) & 1;
+#pragma unroll
+    for (int kk = 0; kk < KT; ++kk) {
+      const int chunk = 2 * kk + kch;
+      uint32_t b[4];
+      ldsm_x4(sK + (chunk >> 3) * C::BOX_BYTES + ktr * 128 + (((chunk & 7) ^ r7) << 4), b);
+      uint32_t a[4] = {0u, 0u, 0u, 0u};
+      {
+        const uint2 f = *reinterpret_cast<const uint2*>(qfrag + ((0 * KT + kk) * 32 + lane) * 2);
+        a[0] = f.x;
+        a[2] = f.y;
+      }
+      mma_bf16(cref[0], a, b[0], b[1]);
+      mma_bf16(cref[1], a, b[2], b[3]);
+      if constexpr (C::RES) {
+        const uint2 f = *reinterpret_cast<const uint2*>(qfrag + ((1 * KT + kk) * 32 + lane) * 2);
+        a[0] = f.x;
+        a[2] = f.y;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          const uint32_t* cw = reinterpret_cast<const uint32_t*>(st + C::OFF_CK + tb[nt] * C::CROW);
+          uint32_t b0, b1;
+          if constexpr (BITS == 2) {
+            k_levels<2>(cw[kk], 0u, q, b0, b1);
+          } else {
+            const uint2 w2 = *reinterpret_cast<const uint2*>(cw + 2 * kk);
+            k_levels<4>(w2.x, w2.y, q, b0, b1);
+          }
+          mma_f16(ct[nt], a, b0, b1);
+        }
+        if ((kk + 1) % KSG == 0) {
+          // end of scale group j: S += s^K_{t, j} x (q~_j . l_j) for c0, c1
+          const int j = kk / KSG;
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) {
+            const float sk0 = half_at(st + C::OFF_SK + sc_off + tok0[nt] * SB + 2 * j);
+            const float sk1 = half_at(st + C::OFF_SK + sc_off + (tok0[nt] + 1) * SB + 2 * j);
+            cref[nt][0] = fmaf(sk0, ct[nt][0], cref[nt][0]);
+            cref[nt][1] = fmaf(sk1, ct[nt][1], cref[nt][1]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) ct[nt][e] = 0.0f;
+          }
+        }
+      }
+    }
+    float sc[2][2];          // row g, tokens 2q, 2q+1 of tile nt
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      sc[nt][0] = (row_ok && tok0[nt] < n) ? score_scale * cref[nt][0] : kNegInf;
+      sc[nt][1] = (row_ok && tok0[nt] + 1 < n) ? score_scale * cref[nt][1] : kNegInf;
+    }
+    // ---- online softmax of row g (four lanes per row) ----
+    float mc = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
+    mc = fmaxf(mc, __shfl_xor_sync(FULL, mc, 1));
+    mc = fmaxf(mc, __shfl_xor_sync(FULL, mc, 2));
+    const float m_new = fmaxf(m_run, mc);
+    const float alpha = (m_new == m_run) ? 1.0f : (m_run == kNegInf ? 0.0f : exp2f(m_run - m_new));
+    m_run = m_new;
+    float pr[2][2];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) pr[nt][e] = (sc[nt][e] == kNegInf) ? 0.0f : exp2f(sc[nt][e] - m_new);
+    l_run = l_run * alpha + (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
+    if (!__all_sync(FULL, alpha == 1.0f)) {
+      // rows 2q and 2q+1 of the O^T fragments: their alphas live in lanes 8q, 8q+4
+      const float a0 = __shfl_sync(FULL, alpha, 8 * q);
+      const float a1 = __shfl_sync(FULL, alpha, 8 * q + 4);
+      const float2 a01 = make_float2(a0, a1);
+#pragma unroll
+      for (int mt = 0; mt < KT; ++mt) {
+        float2 x = __fmul2_rn(make_float2(oref[mt][0], oref[mt][1]), a01);
+        float2 y = __fmul2_rn(make_float2(oref[mt][2], oref[mt][3]), a01);
+        oref[mt][0] = x.x; oref[mt][1] = x.y; oref[mt][2] = y.x; oref[mt][3] = y.y;
+        if constexpr (C::RES) {
+          x = __fmul2_rn(make_float2(ores[mt][0], ores[mt][1]), a01);
+          y = __fmul2_rn(make_float2(ores[mt][2], ores[mt][3]), a01);
+          ores[mt][0] = x.x; ores[mt][1] = x.y; ores[mt][2] = y.x; ores[mt][3] = y.y;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < NG; ++j) wsum[j] *= alpha;
+    }
+    // P^T fragments (k = tokens 2q, 2q+1 / +8, n = row g): bf16 hi + lo
+    const uint32_t ph0 = pack_bf16(pr[0][0], pr[0][1]);
+    const uint32_t ph1 = pack_bf16(pr[1][0], pr[1][1]);
+    const uint32_t pl0 = pack_bf16(pr[0][0] - bf16_lo_f(ph0), pr[0][1] - bf16_hi_f(ph0));
+    const uint32_t pl1 = pack_bf16(pr[1][0] - bf16_lo_f(ph1), pr[1][1] - bf16_hi_f(ph1));
+    // ---- O_ref^T += V^T P^T ----
+#pragma unroll
+    for (int mt = 0; mt < KT; ++mt) {
+      const int m = lane >> 3;                         // matrix this lane addresses
+      const int tr = wtok + (m >> 1) * 8 + r7;
+      const int chunk = 2 * mt + (m & 1);
+      const uint32_t addr = sV + (chunk >> 3) * C::BOX_BYTES + tr * 128 +
+                            ((((chunk & 7) ^ r7)) << 4);
+      uint32_t a[4];
+      ldsm_x4_trans(addr, a);
+      mma_bf16(oref[mt], a, ph0, ph1);
+      mma_bf16(oref[mt], a, pl0, pl1);
+    }
+    // ---- O_res^T += C_V^T (P s^V)^T ----
+    if constexpr (C::RES) {
+      const int tk[4] = {wtok + 2 * q, wtok + 2 * q + 1, wtok + 2 * q + 8, wtok + 2 * q + 9};
+      const float pk[4] = {pr[0][0], pr[0][1], pr[1][0], pr[1][1]};
+#pragma unroll
+      for (int j = 0; j < NG; ++j) {
+        float wv[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float sv = half_at(st + C::OFF_SV + sc_off + tk[k] * SB + 2 * j);
+          wv[k] = (tk[k] < n) ? pk[k] * sv : 0.0f;       // weight 0 beyond the tile
+        }
+        wsum[j] += (wv[0] + wv[1]) + (wv[2] + wv[3]);
+        const uint32_t bw0 = pack_f16(wv[0] * 4096.0f, wv[1] * 4096.0f);
+        const uint32_t bw1 = pack_f16(wv[2] * 4096.0f, wv[3] * 4096.0f);
+#pragma unroll
+        for (int mt = j * KSG; mt < (j + 1) * KSG; ++mt) {
+          // codes of dims 16mt + g (lo halves) and 16mt + g + 8 (hi halves)
+          uint32_t x[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t* cw = reinterpret_cast<const uint32_t*>(st + C::OFF_CV + tk[k] * C::CROW);
+            if constexpr (BITS == 2) {
+              x[k] = ((cw[mt] >> (2 * g)) & 0x00030003u) | kMagic;
+            } else {
+              const uint32_t lo = (cw[2 * mt] >> (4 * g)) & 0xFu;
+              const uint32_t hi = (cw[2 * mt + 1] >> (4 * g)) & 0xFu;
+              x[k] = lo | (hi << 16) | kMagic;
+            }
+          }
+          const uint32_t m1024 = 0xE400E400u;   // {-1024, -1024}
+          uint32_t a[4];
+          a[0] = hadd2_u(__byte_perm(x[0], x[1], 0x5410), m1024);   // dim g,   tokens 2q, 2q+1
+          a[1] = hadd2_u(__byte_perm(x[0], x[1], 0x7632), m1024);   // dim g+8
+          a[2] = hadd2_u(__byte_perm(x[2], x[3], 0x5410), m1024);   // dim g,   tokens 2q+8, 2q+9
+          a[3] = hadd2_u(__byte_perm(x[2], x[3], 0x7632), m1024);   // dim g+8
+          mma_f16(ores[mt], a, bw0, bw1);
+        }
+      }
+    }
+  };
+
+  // ---- main loop over this CTA's tiles ----
+  long long cur_head = -1;
+  bool aborted = false;
+  reset_state();
+  for (int i = 0; i < n_my; ++i) {
+    const long long tile = tile_begin + i;
+    const long long hd = tile / p.nt;
+    if (hd != cur_head) {
+      if (cur_head >= 0) {
+        flush_head(cur_head);
+        reset_state();
+      }
+      cur_head = hd;
+      setup_head(hd);
+    }
+    const int s = i % STAGES;
+    bool ok = !aborted && !flags[0];
+    if (ok) ok = mbar_wait_bounded(&full_bar[s], (i / STAGES) & 1);
+    ok = __all_sync(FULL, ok);
+    if (!ok) {
+      if (!aborted && lane == 0) flag_error(p.status, 8u);
+      aborted = true;
+      flags[0] = 1;
+    }
+    if (!aborted) {
+      const int t0 = (int)(tile % p.nt) * TILE;
+      const int n = min(TILE, T - t0);
+      const size_t row = (size_t)hd * T + t0;
+      tile_mma(ring + s * C::STAGE_BYTES, n, (int)((row * SB) & 15));
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty_bar[s]);
+  }
+  if (cur_head >= 0) flush_head(cur_head);
+}
+
+// ---- host side ---------------------------------------------------------------
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult qres;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &qres) ==
+            cudaSuccess &&
+        qres == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }
+  return fn;
+}
+
+// [rows][d] bf16 viewed 2-D, box = 64 columns x 64 rows, 128-byte swizzle.
+bool encode_kv_map(CUtensorMap* map, const void* base, unsigned long long rows, int d) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)kDecodeTile};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D, int G, int BITS, int GROUP>
+cudaError_t launch_gqa_t(const GqaParams& gp, cudaStream_t stream) {
+  using C = GCfg<D, G, BITS, GROUP>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(decode_gqa_kernel<D, G, BITS, GROUP>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  decode_gqa_kernel<D, G, BITS, GROUP><<<gp.p.ctas, kDecodeThreads, C::SMEM_BYTES, stream>>>(gp);
+  return cudaGetLastError();
+}
+
+template <int D, int G>
+cudaError_t launch_gqa_g(int bits, const GqaParams& gp, cudaStream_t stream) {
+  const int group = gp.p.group;
+  if (bits == 16) return launch_gqa_t<D, G, 16, 32>(gp, stream);   // no scales are read
+  if (bits == 2)
+    return group == 32 ? launch_gqa_t<D, G, 2, 32>(gp, stream) : launch_gqa_t<D, G, 2, 64>(gp, stream);
+  if (bits == 4)
+    return group == 32 ? launch_gqa_t<D, G, 4, 32>(gp, stream) : launch_gqa_t<D, G, 4, 64>(gp, stream);
+  return cudaErrorInvalidValue;
+}
+
+template <int D>
+cudaError_t launch_gqa_d(int G, int bits, const GqaParams& gp, cudaStream_t stream) {
+  switch (G) {
+    case 2: return launch_gqa_g<D, 2>(bits, gp, stream);
+    case 4: return launch_gqa_g<D, 4>(bits, gp, stream);
+    case 8: return launch_gqa_g<D, 8>(bits, gp, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_decode_gqa(int head_dim, int G, int bits, const DecodeParams& p,
+                              cudaStream_t stream) {
+  GqaParams gp;
+  gp.p = p;
+  const unsigned long long rows = (unsigned long long)p.batch * p.kv_heads * p.ctx;
+  if (!encode_kv_map(&gp.tmap_k, p.ref_k, rows, head_dim) ||
+      !encode_kv_map(&gp.tmap_v, p.ref_v, rows, head_dim))
+    return cudaErrorInvalidValue;
+  if (head_dim == 128) return launch_gqa_d<128>(G, bits, gp, stream);
+  if (head_dim == 64) return launch_gqa_d<64>(G, bits, gp, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace rq

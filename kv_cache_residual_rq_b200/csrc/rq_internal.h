@@ -81,8 +81,12 @@ struct DecodeParams {
   float score_scale;     // softmax scale * log2(e)
 };
 
+// one query row per kv head (CUDA cores)
 cudaError_t launch_decode(int head_dim, int G, int bits, const DecodeParams& p,
                           cudaStream_t stream);
+// grouped queries, G in {2, 4, 8} (tensor cores, TMA tensor copies)
+cudaError_t launch_decode_gqa(int head_dim, int G, int bits, const DecodeParams& p,
+                              cudaStream_t stream);
 
 int device_sm_count();   // SMs of the current device, cached per device
 
