@@ -473,16 +473,18 @@ decode_kernel(const DecodeParams p) {
     float sc = score_scale * (part[0] + __shfl_xor_sync(FULL, part[0], 1));
     const int own_tok = warp * C::TPW + (li >> 1) * TPS + slot;
     if (own_tok >= n) sc = kNegInf;
-    // online softmax, base 2
-    float mc = sc;
+    // online softmax, base 2, rescaled lazily: the running max moves only when
+    // a score exceeds it by more than kLazyMax, so weights stay <= 2^kLazyMax
+    // and most tiles need one vote instead of a shuffle-max chain
+    if (__any_sync(FULL, sc > m_run[0] + kLazyMax)) {
+      float mc = sc;
 #pragma unroll
-    for (int m = 2; m < 32; m <<= 1) mc = fmaxf(mc, __shfl_xor_sync(FULL, mc, m));
-    const float m_new = fmaxf(m_run[0], mc);
-    if (m_new != m_run[0]) {
+      for (int m = 2; m < 32; m <<= 1) mc = fmaxf(mc, __shfl_xor_sync(FULL, mc, m));
+      const float m_new = fmaxf(m_run[0], mc);
       rescale(0, (m_run[0] == kNegInf) ? 0.0f : exp2f(m_run[0] - m_new));
       m_run[0] = m_new;
     }
-    const float pme = (sc == kNegInf) ? 0.0f : exp2f(sc - m_new);
+    const float pme = (sc == kNegInf) ? 0.0f : exp2f(sc - m_run[0]);
     l_run[0] += pme;
     // values
 #pragma unroll

@@ -20,6 +20,8 @@ constexpr int kConsumerWarps = 4;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kDecodeThreads = kConsumerThreads + 32;   // + one producer warp
 constexpr float kNegInf = -INFINITY;
+// lazy rescaling threshold of the online softmax (base-2 units)
+constexpr float kLazyMax = 8.0f;
 
 __device__ __forceinline__ void flag_error(uint32_t* status, uint32_t bit) {
   atomicOr(status, bit);

@@ -439,18 +439,21 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
       sc[nt][0] = (row_ok && tok0[nt] < n) ? score_scale * cref[nt][0] : kNegInf;
       sc[nt][1] = (row_ok && tok0[nt] + 1 < n) ? score_scale * cref[nt][1] : kNegInf;
     }
-    // ---- online softmax of row g (four lanes per row) ----
+    // ---- online softmax of row g (four lanes per row), rescaled lazily ----
     float mc = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
-    mc = fmaxf(mc, __shfl_xor_sync(FULL, mc, 1));
-    mc = fmaxf(mc, __shfl_xor_sync(FULL, mc, 2));
-    const float m_new = fmaxf(m_run, mc);
-    const float alpha = (m_new == m_run) ? 1.0f : (m_run == kNegInf ? 0.0f : exp2f(m_run - m_new));
-    m_run = m_new;
+    float alpha = 1.0f;
+    if (__any_sync(FULL, mc > m_run + kLazyMax)) {
+      mc = fmaxf(mc, __shfl_xor_sync(FULL, mc, 1));
+      mc = fmaxf(mc, __shfl_xor_sync(FULL, mc, 2));
+      const float m_new = fmaxf(m_run, mc);
+      alpha = (m_new == m_run) ? 1.0f : (m_run == kNegInf ? 0.0f : exp2f(m_run - m_new));
+      m_run = m_new;
+    }
     float pr[2][2];
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-      for (int e = 0; e < 2; ++e) pr[nt][e] = (sc[nt][e] == kNegInf) ? 0.0f : exp2f(sc[nt][e] - m_new);
+      for (int e = 0; e < 2; ++e) pr[nt][e] = (sc[nt][e] == kNegInf) ? 0.0f : exp2f(sc[nt][e] - m_run);
     l_run = l_run * alpha + (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
     if (!__all_sync(FULL, alpha == 1.0f)) {
       // rows 2q and 2q+1 of the O^T fragments: their alphas live in lanes 8q, 8q+4
