@@ -26,7 +26,8 @@
  *     back as RQ_ERR_CUDA.
  *   - bf16 / fp16 values are passed as uint16_t bit patterns.
  *
- * Layouts (row-major, T = ctx, d = head_dim, g = group, b = bits):
+ * Layouts (row-major, T = ctx_cap (ctx when 0), d = head_dim, g = group,
+ * b = bits):
  *   K/V of one loop, reference : bf16 [rows][kv_heads][T][d]
  *   query                      : bf16 [batch][q_heads][d]
  *   codes of one loop          : uint32 [rows][kv_heads][T][d*b/32];
@@ -69,9 +70,13 @@ typedef struct {
                            (e.g. layers * B) for encode */
     int32_t kv_heads;   /* Hkv >= 1 */
     int32_t q_heads;    /* Hq, a multiple of Hkv (decode only; encode ignores) */
-    int32_t ctx;        /* T: cached tokens per (row, kv head) */
+    int32_t ctx;        /* T: tokens per (row, kv head) the call covers */
     int32_t head_dim;   /* d: 64 or 128 */
     int32_t group;      /* g: 32 or 64, divides d */
+    int32_t ctx_cap;    /* token capacity (pitch) of the K/V, codes and scales
+                           arrays per (row, kv head); 0 means ctx.  A cache
+                           allocated for ctx_cap tokens holds its first ctx
+                           tokens valid, so it can grow in place. */
 } rq_shape;
 
 /* Library version as major*10000 + minor*100 + patch. */
@@ -81,12 +86,13 @@ int rq_version(void);
 const char *rq_status_string(rq_status s);
 
 /* Bytes of the codes of ONE loop at `bits` (2 or 4) for `shape`:
- * batch*kv_heads*ctx*head_dim*bits/8 rounded up to 16.  0 for bits == 16 or
- * an invalid shape.  Host-only arithmetic. */
+ * batch*kv_heads*T*head_dim*bits/8 rounded up to 16, T = ctx_cap (ctx when
+ * 0).  0 for bits == 16 or an invalid shape.  Host-only arithmetic. */
 size_t rq_codes_bytes(const rq_shape *shape, int bits);
 
-/* Bytes of the fp16 scales of ONE loop: batch*kv_heads*ctx*(head_dim/group)*2
- * rounded up to 16.  0 for bits == 16 or an invalid shape. */
+/* Bytes of the fp16 scales of ONE loop: batch*kv_heads*T*(head_dim/group)*2
+ * rounded up to 16, T = ctx_cap (ctx when 0).  0 for bits == 16 or an
+ * invalid shape. */
 size_t rq_scales_bytes(const rq_shape *shape, int bits);
 
 /* Workspace bytes rq_decode_attention needs for `shape` (partial softmax
@@ -134,6 +140,33 @@ rq_status rq_encode(const rq_shape *shape, const uint16_t *const *kv_loops, int 
                     uint32_t *const *codes_out, uint16_t *const *scales_out, void *stream);
 
 /*
+ * rq_encode_at -- rq_encode from a token window into a cache position (the
+ * encode-on-arrival step of a decode loop: a token's non-final loops can be
+ * encoded only once its final loop exists; until then they stay in BF16 in a
+ * window, the same constraint the LoopVQ page describes for its serving
+ * integration).
+ *
+ * Same arithmetic as rq_encode.  For every (row r, kv head h) and token
+ * t < shape->ctx it reads source token src_offset + t of arrays whose token
+ * pitch is src_pitch, and writes destination token dst_offset + t of arrays
+ * whose token pitch is dst_pitch:
+ *   kv_loops[l], ref   : bf16 [rows][Hkv][src_pitch][d]
+ *   codes_out[l]       : [rows][Hkv][dst_pitch][d*b/32]
+ *   scales_out[l]      : [rows][Hkv][dst_pitch][d/g]
+ *   ref_out (optional) : bf16 [rows][Hkv][dst_pitch][d]; when not NULL the
+ *                        final-loop rows are copied there too, so a window
+ *                        slot can be retired into the cache in one call.
+ * shape->ctx_cap is ignored.  Requires src_offset + ctx <= src_pitch and
+ * dst_offset + ctx <= dst_pitch.  Destination tokens outside the written
+ * range are not touched.
+ */
+rq_status rq_encode_at(const rq_shape *shape, int src_pitch, int src_offset, int dst_pitch,
+                       int dst_offset, const uint16_t *const *kv_loops, int n_loops,
+                       const uint16_t *ref, const uint8_t *bits_per_loop, uint64_t seed,
+                       uint32_t *const *codes_out, uint16_t *const *scales_out,
+                       uint16_t *ref_out, void *stream);
+
+/*
  * rq_decode_attention -- fused ResidualQuant decode attention for one loop
  * (Abstract: the reconstruction stays efficient; the reduced KV traffic is
  * what speeds decode up).
@@ -174,6 +207,29 @@ rq_status rq_decode_attention(const rq_shape *shape, const uint16_t *q,
                               const uint16_t *scales_k, const uint16_t *scales_v,
                               int bits, uint64_t seed, float softmax_scale, float *out,
                               void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * rq_decode_attention_tail -- rq_decode_attention over the shape->ctx cached
+ * tokens plus n_tail BF16 tokens of the same loop that are not encoded yet
+ * (the current token and any others still in the window):
+ *   out[b,j,:] = softmax over { K_hat_t, t < ctx } U { tail_k[b,h,i], i < n_tail }
+ * applied to the matching V rows.  The tail is folded into the merge that
+ * finishes each head, in the same launch.
+ *   tail_k, tail_v : device bf16 [batch][Hkv][tail_pitch][d], tokens
+ *                    0..n_tail-1 used; may be NULL when n_tail == 0.
+ *   n_tail         : 0 .. 256 (RQ_MAX_TAIL); tail_pitch >= n_tail.
+ * Everything else as rq_decode_attention (which is this call with n_tail 0).
+ */
+#define RQ_MAX_TAIL 256
+
+rq_status rq_decode_attention_tail(const rq_shape *shape, const uint16_t *q,
+                                   const uint16_t *ref_k, const uint16_t *ref_v,
+                                   const uint32_t *codes_k, const uint32_t *codes_v,
+                                   const uint16_t *scales_k, const uint16_t *scales_v,
+                                   int bits, uint64_t seed, float softmax_scale,
+                                   const uint16_t *tail_k, const uint16_t *tail_v, int n_tail,
+                                   int tail_pitch, float *out, void *workspace,
+                                   size_t workspace_bytes, void *stream);
 
 /*
  * rq_decode_attention_noalloc -- rq_decode_attention without a workspace

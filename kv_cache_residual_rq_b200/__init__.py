@@ -10,7 +10,7 @@ reports and pass pointers through.
 from ._abi import (RQ_ERR_ALIGNMENT, RQ_ERR_CUDA, RQ_ERR_INVALID_ARG, RQ_ERR_UNSUPPORTED,
                    RQ_ERR_WORKSPACE, RQ_MAX_LOOPS, RQ_OK, RqError, lib, make_shape,
                    rq_codes_bytes, rq_decode_attention, rq_decode_attention_noalloc,
-                   rq_decode_workspace_bytes, rq_encode,
+                   rq_decode_attention_tail, rq_decode_workspace_bytes, rq_encode, rq_encode_at,
                    rq_scales_bytes, rq_shape, rq_status_string, rq_version,
                    rq_workspace_status)
 
@@ -18,7 +18,8 @@ __all__ = [
     "RQ_OK", "RQ_ERR_INVALID_ARG", "RQ_ERR_UNSUPPORTED", "RQ_ERR_ALIGNMENT", "RQ_ERR_WORKSPACE",
     "RQ_ERR_CUDA", "RQ_MAX_LOOPS", "RqError", "lib", "rq_shape", "make_shape", "rq_version",
     "rq_status_string", "rq_codes_bytes", "rq_scales_bytes", "rq_decode_workspace_bytes",
-    "rq_encode", "rq_decode_attention", "rq_decode_attention_noalloc", "rq_workspace_status",
+    "rq_encode", "rq_encode_at", "rq_decode_attention", "rq_decode_attention_tail",
+    "rq_decode_attention_noalloc", "rq_workspace_status",
     "alloc_codes", "alloc_scales", "alloc_workspace", "encode", "decode_attention",
 ]
 
@@ -59,18 +60,27 @@ def encode(kv_loops, ref, bits_per_loop, group, seed, stream=None):
 
 
 def decode_attention(q, ref_k, ref_v, codes_k, codes_v, scales_k, scales_v, bits, group, seed,
-                     softmax_scale=0.0, out=None, workspace=None, stream=None):
+                     softmax_scale=0.0, out=None, workspace=None, stream=None, ctx=None,
+                     tail_k=None, tail_v=None, n_tail=0):
     """Decode attention of one loop.  q [B, Hq, d] bf16; ref_k/ref_v
-    [B, Hkv, T, d] bf16; codes/scales as returned by encode (None for bits 16).
-    Returns out [B, Hq, d] fp32."""
+    [B, Hkv, T_cap, d] bf16 of which the first `ctx` tokens (default T_cap) are
+    attended; codes/scales as returned by encode (None for bits 16); optional
+    BF16 tail tokens tail_k/tail_v [B, Hkv, W, d], the first n_tail attended
+    too.  Returns out [B, Hq, d] fp32."""
     import torch
     b, hq, d = q.shape
-    _, hkv, t, _ = ref_k.shape
-    shape = make_shape(b, hkv, t, d, group, q_heads=hq)
+    _, hkv, t_cap, _ = ref_k.shape
+    t = t_cap if ctx is None else ctx
+    shape = make_shape(b, hkv, t, d, group, q_heads=hq, ctx_cap=t_cap)
     if out is None:
         out = torch.empty((b, hq, d), dtype=torch.float32, device=q.device)
     if workspace is None:
         workspace = alloc_workspace(shape, q.device)
-    rq_decode_attention(shape, q, ref_k, ref_v, codes_k, codes_v, scales_k, scales_v, bits, seed,
-                        softmax_scale, out, workspace, stream=stream)
+    if n_tail:
+        rq_decode_attention_tail(shape, q, ref_k, ref_v, codes_k, codes_v, scales_k, scales_v,
+                                 bits, seed, softmax_scale, tail_k, tail_v, n_tail,
+                                 tail_k.shape[2], out, workspace, stream=stream)
+    else:
+        rq_decode_attention(shape, q, ref_k, ref_v, codes_k, codes_v, scales_k, scales_v, bits,
+                            seed, softmax_scale, out, workspace, stream=stream)
     return out

@@ -30,15 +30,18 @@ class RqError(RuntimeError):
 class rq_shape(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("kv_heads", ctypes.c_int32),
                 ("q_heads", ctypes.c_int32), ("ctx", ctypes.c_int32),
-                ("head_dim", ctypes.c_int32), ("group", ctypes.c_int32)]
+                ("head_dim", ctypes.c_int32), ("group", ctypes.c_int32),
+                ("ctx_cap", ctypes.c_int32)]
 
     def __repr__(self):
-        return ("rq_shape(batch=%d, kv_heads=%d, q_heads=%d, ctx=%d, head_dim=%d, group=%d)"
-                % (self.batch, self.kv_heads, self.q_heads, self.ctx, self.head_dim, self.group))
+        return ("rq_shape(batch=%d, kv_heads=%d, q_heads=%d, ctx=%d, head_dim=%d, group=%d, "
+                "ctx_cap=%d)" % (self.batch, self.kv_heads, self.q_heads, self.ctx, self.head_dim,
+                                 self.group, self.ctx_cap))
 
 
-def make_shape(batch, kv_heads, ctx, head_dim, group, q_heads=None):
-    return rq_shape(batch, kv_heads, kv_heads if q_heads is None else q_heads, ctx, head_dim, group)
+def make_shape(batch, kv_heads, ctx, head_dim, group, q_heads=None, ctx_cap=0):
+    return rq_shape(batch, kv_heads, kv_heads if q_heads is None else q_heads, ctx, head_dim,
+                    group, ctx_cap)
 
 
 _lib = None
@@ -71,6 +74,17 @@ def lib():
                                           c.c_void_p, c.c_void_p, c.c_void_p, c.c_int, c.c_uint64,
                                           c.c_float, c.c_void_p, c.c_void_p, c.c_size_t, c.c_void_p]
         L.rq_decode_attention.restype = c.c_int
+        L.rq_encode_at.argtypes = [sp, c.c_int, c.c_int, c.c_int, c.c_int,
+                                   c.POINTER(c.c_void_p), c.c_int, c.c_void_p,
+                                   c.POINTER(c.c_uint8), c.c_uint64, c.POINTER(c.c_void_p),
+                                   c.POINTER(c.c_void_p), c.c_void_p, c.c_void_p]
+        L.rq_encode_at.restype = c.c_int
+        L.rq_decode_attention_tail.argtypes = [sp, c.c_void_p, c.c_void_p, c.c_void_p,
+                                               c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p,
+                                               c.c_int, c.c_uint64, c.c_float, c.c_void_p,
+                                               c.c_void_p, c.c_int, c.c_int, c.c_void_p,
+                                               c.c_void_p, c.c_size_t, c.c_void_p]
+        L.rq_decode_attention_tail.restype = c.c_int
         L.rq_decode_attention_noalloc.argtypes = [sp, c.c_void_p, c.c_void_p, c.c_void_p,
                                                   c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p,
                                                   c.c_int, c.c_uint64, c.c_float, c.c_void_p,
@@ -143,6 +157,36 @@ def rq_encode(shape, kv_loops, ref, bits_per_loop, seed, codes_out, scales_out, 
                          _stream(stream))
     if check:
         _check(st, "rq_encode")
+    return st
+
+
+def rq_encode_at(shape, src_pitch, src_offset, dst_pitch, dst_offset, kv_loops, ref,
+                 bits_per_loop, seed, codes_out, scales_out, ref_out=None, stream=None,
+                 check=True):
+    n = len(bits_per_loop)
+    ptrs = lambda seq: (ctypes.c_void_p * max(n, 1))(*[_ptr(v) for v in seq])
+    bits = (ctypes.c_uint8 * max(n, 1))(*[int(b) for b in bits_per_loop])
+    st = lib().rq_encode_at(_shp(shape), int(src_pitch), int(src_offset), int(dst_pitch),
+                            int(dst_offset), ptrs(kv_loops), n, _ptr(ref), bits,
+                            ctypes.c_uint64(seed), ptrs(codes_out), ptrs(scales_out),
+                            _ptr(ref_out), _stream(stream))
+    if check:
+        _check(st, "rq_encode_at")
+    return st
+
+
+def rq_decode_attention_tail(shape, q, ref_k, ref_v, codes_k, codes_v, scales_k, scales_v,
+                             bits, seed, softmax_scale, tail_k, tail_v, n_tail, tail_pitch, out,
+                             workspace, workspace_bytes=None, stream=None, check=True):
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    st = lib().rq_decode_attention_tail(
+        _shp(shape), _ptr(q), _ptr(ref_k), _ptr(ref_v), _ptr(codes_k), _ptr(codes_v),
+        _ptr(scales_k), _ptr(scales_v), int(bits), ctypes.c_uint64(seed), float(softmax_scale),
+        _ptr(tail_k), _ptr(tail_v), int(n_tail), int(tail_pitch), _ptr(out), _ptr(workspace),
+        int(workspace_bytes), _stream(stream))
+    if check:
+        _check(st, "rq_decode_attention_tail")
     return st
 
 

@@ -22,10 +22,14 @@ bool supported_dims(int head_dim, int group) {
          head_dim % group == 0;
 }
 
+// token pitch of the arrays a shape describes
+int pitch_of(const rq_shape* s) { return s->ctx_cap ? s->ctx_cap : s->ctx; }
+
 // basic shape check shared by the size queries; false for anything invalid
 bool shape_ok(const rq_shape* s, bool need_ctx) {
   if (!s) return false;
   if (s->batch < 1 || s->kv_heads < 1 || s->ctx < 0) return false;
+  if (s->ctx_cap != 0 && s->ctx_cap < s->ctx) return false;
   if (need_ctx && s->ctx < 1) return false;
   return supported_dims(s->head_dim, s->group);
 }
@@ -98,13 +102,13 @@ const char* rq_status_string(rq_status s) {
 size_t rq_codes_bytes(const rq_shape* shape, int bits) {
   if (!shape_ok(shape, false) || (bits != 2 && bits != 4)) return 0;
   const size_t elems =
-      (size_t)shape->batch * shape->kv_heads * shape->ctx * (size_t)shape->head_dim;
+      (size_t)shape->batch * shape->kv_heads * pitch_of(shape) * (size_t)shape->head_dim;
   return round16(elems * bits / 8);
 }
 
 size_t rq_scales_bytes(const rq_shape* shape, int bits) {
   if (!shape_ok(shape, false) || (bits != 2 && bits != 4)) return 0;
-  const size_t groups = (size_t)shape->batch * shape->kv_heads * shape->ctx *
+  const size_t groups = (size_t)shape->batch * shape->kv_heads * pitch_of(shape) *
                         (size_t)(shape->head_dim / shape->group);
   return round16(groups * 2);
 }
@@ -114,16 +118,22 @@ size_t rq_decode_workspace_bytes(const rq_shape* shape) {
   return decode_workspace_bytes(*shape);
 }
 
-rq_status rq_encode(const rq_shape* shape, const uint16_t* const* kv_loops, int n_loops,
-                    const uint16_t* ref, const uint8_t* bits_per_loop, uint64_t seed,
-                    uint32_t* const* codes_out, uint16_t* const* scales_out, void* stream) {
+rq_status rq_encode_at(const rq_shape* shape, int src_pitch, int src_offset, int dst_pitch,
+                       int dst_offset, const uint16_t* const* kv_loops, int n_loops,
+                       const uint16_t* ref, const uint8_t* bits_per_loop, uint64_t seed,
+                       uint32_t* const* codes_out, uint16_t* const* scales_out,
+                       uint16_t* ref_out, void* stream) {
   if (!shape || !kv_loops || !bits_per_loop || !codes_out || !scales_out)
     return RQ_ERR_INVALID_ARG;
   if (shape->batch < 1 || shape->kv_heads < 1 || shape->ctx < 0) return RQ_ERR_INVALID_ARG;
+  if (src_offset < 0 || dst_offset < 0 || src_pitch < 1 || dst_pitch < 1 ||
+      (long long)src_offset + shape->ctx > src_pitch ||
+      (long long)dst_offset + shape->ctx > dst_pitch)
+    return RQ_ERR_INVALID_ARG;
   if (n_loops < 1 || n_loops > RQ_MAX_LOOPS) return RQ_ERR_INVALID_ARG;
   if (!supported_dims(shape->head_dim, shape->group)) return RQ_ERR_UNSUPPORTED;
   if (!ref) return RQ_ERR_INVALID_ARG;
-  if (!aligned16(ref)) return RQ_ERR_ALIGNMENT;
+  if (!aligned16(ref) || (ref_out && !aligned16(ref_out))) return RQ_ERR_ALIGNMENT;
   EncodeParams p;
   std::memset(&p, 0, sizeof p);
   int active = 0;
@@ -141,10 +151,16 @@ rq_status rq_encode(const rq_shape* shape, const uint16_t* const* kv_loops, int 
     ++active;
   }
   p.ref = ref;
+  p.ref_out = ref_out;
   p.n_loops = n_loops;
   p.seed = seed;
+  p.ctx = shape->ctx;
+  p.src_pitch = src_pitch;
+  p.src_offset = src_offset;
+  p.dst_pitch = dst_pitch;
+  p.dst_offset = dst_offset;
   p.n_rows = (long long)shape->batch * shape->kv_heads * shape->ctx;
-  if (p.n_rows == 0 || active == 0) return RQ_OK;
+  if (p.n_rows == 0 || (active == 0 && !ref_out)) return RQ_OK;
   const int sms = device_sm_count();
   if (sms <= 0) return RQ_ERR_CUDA;
   cudaError_t e = launch_encode(shape->head_dim, shape->group, p, sms,
@@ -152,16 +168,32 @@ rq_status rq_encode(const rq_shape* shape, const uint16_t* const* kv_loops, int 
   return e == cudaSuccess ? RQ_OK : RQ_ERR_CUDA;
 }
 
-rq_status rq_decode_attention(const rq_shape* shape, const uint16_t* q, const uint16_t* ref_k,
-                              const uint16_t* ref_v, const uint32_t* codes_k,
-                              const uint32_t* codes_v, const uint16_t* scales_k,
-                              const uint16_t* scales_v, int bits, uint64_t seed,
-                              float softmax_scale, float* out, void* workspace,
-                              size_t workspace_bytes, void* stream) {
+rq_status rq_encode(const rq_shape* shape, const uint16_t* const* kv_loops, int n_loops,
+                    const uint16_t* ref, const uint8_t* bits_per_loop, uint64_t seed,
+                    uint32_t* const* codes_out, uint16_t* const* scales_out, void* stream) {
+  if (!shape) return RQ_ERR_INVALID_ARG;
+  if (shape->ctx_cap != 0 && shape->ctx_cap < shape->ctx) return RQ_ERR_INVALID_ARG;
+  const int pitch = pitch_of(shape) > 0 ? pitch_of(shape) : 1;
+  return rq_encode_at(shape, pitch, 0, pitch, 0, kv_loops, n_loops, ref, bits_per_loop, seed,
+                      codes_out, scales_out, nullptr, stream);
+}
+
+rq_status rq_decode_attention_tail(const rq_shape* shape, const uint16_t* q,
+                                   const uint16_t* ref_k, const uint16_t* ref_v,
+                                   const uint32_t* codes_k, const uint32_t* codes_v,
+                                   const uint16_t* scales_k, const uint16_t* scales_v, int bits,
+                                   uint64_t seed, float softmax_scale, const uint16_t* tail_k,
+                                   const uint16_t* tail_v, int n_tail, int tail_pitch,
+                                   float* out, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
   if (!shape) return RQ_ERR_INVALID_ARG;
   if (shape->batch < 1 || shape->kv_heads < 1 || shape->ctx < 1 ||
       shape->q_heads < shape->kv_heads)
     return RQ_ERR_INVALID_ARG;
+  if (shape->ctx_cap != 0 && shape->ctx_cap < shape->ctx) return RQ_ERR_INVALID_ARG;
+  if (n_tail < 0 || n_tail > RQ_MAX_TAIL) return RQ_ERR_INVALID_ARG;
+  if (n_tail > 0 && (!tail_k || !tail_v || tail_pitch < n_tail)) return RQ_ERR_INVALID_ARG;
+  if (n_tail > 0 && (!aligned16(tail_k) || !aligned16(tail_v))) return RQ_ERR_ALIGNMENT;
   if (shape->q_heads % shape->kv_heads) return RQ_ERR_INVALID_ARG;
   if (!decode_shape_ok(shape)) return RQ_ERR_UNSUPPORTED;
   if (bits != 2 && bits != 4 && bits != 16) return RQ_ERR_UNSUPPORTED;
@@ -198,6 +230,11 @@ rq_status rq_decode_attention(const rq_shape* shape, const uint16_t* q, const ui
   p.q_heads = shape->q_heads;
   p.ctx = shape->ctx;
   p.group = shape->group;
+  p.ctx_pitch = pitch_of(shape);
+  p.tail_k = n_tail > 0 ? tail_k : nullptr;
+  p.tail_v = n_tail > 0 ? tail_v : nullptr;
+  p.n_tail = n_tail;
+  p.tail_pitch = n_tail > 0 ? tail_pitch : 0;
   p.nt = pl.nt;
   p.n_tiles = pl.n_tiles;
   p.ctas = pl.ctas;
@@ -211,6 +248,17 @@ rq_status rq_decode_attention(const rq_shape* shape, const uint16_t* q, const ui
                       : launch_decode_gqa(shape->head_dim, G, bits, p,
                                           static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? RQ_OK : RQ_ERR_CUDA;
+}
+
+rq_status rq_decode_attention(const rq_shape* shape, const uint16_t* q, const uint16_t* ref_k,
+                              const uint16_t* ref_v, const uint32_t* codes_k,
+                              const uint32_t* codes_v, const uint16_t* scales_k,
+                              const uint16_t* scales_v, int bits, uint64_t seed,
+                              float softmax_scale, float* out, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  return rq_decode_attention_tail(shape, q, ref_k, ref_v, codes_k, codes_v, scales_k, scales_v,
+                                  bits, seed, softmax_scale, nullptr, nullptr, 0, 0, out,
+                                  workspace, workspace_bytes, stream);
 }
 
 rq_status rq_workspace_status(const void* workspace, size_t workspace_bytes,

@@ -183,7 +183,7 @@ decode_kernel(const DecodeParams p) {
         const long long hd = tile / p.nt;
         const int t0 = (int)(tile % p.nt) * TILE;
         const int n = min(TILE, T - t0);
-        const size_t row = (size_t)hd * T + t0;       // first token row of the tile
+        const size_t row = (size_t)hd * p.ctx_pitch + t0;       // first token row of the tile
         unsigned char* st = ring + s * C::STAGE_BYTES;
         uint32_t bytes = 2u * n * C::KROW;
         size_t sc_lo = 0;
@@ -362,7 +362,7 @@ decode_kernel(const DecodeParams p) {
     }
     named_bar_sync(1, kConsumerThreads);
 
-    finish_head<D, G, C::RES>(p, hd, cta, merge, flags, tid);
+    finish_head<D, G, C::RES>(p, hd, cta, merge, qbuf, flags, tid);
   };
 
   // <q, K row> of the lane's dims, straight from the packed bf16 row
@@ -603,7 +603,7 @@ decode_kernel(const DecodeParams p) {
       const int t0 = (int)(tile % p.nt) * TILE;
       const int n = min(TILE, T - t0);
       const unsigned char* st = ring + s * C::STAGE_BYTES;
-      const size_t row = (size_t)hd * T + t0;
+      const size_t row = (size_t)hd * p.ctx_pitch + t0;
       const int sc_off = (int)((row * SB) & 15);
       const int grp = dim0 / p.group;
       if constexpr (G == 1) tile_g1(st, n, sc_off, grp);

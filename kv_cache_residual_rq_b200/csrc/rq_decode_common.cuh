@@ -65,11 +65,16 @@ __device__ __forceinline__ void load_rotate_queries(const DecodeParams& p, long 
 // merge[w][r] = {m, l, accRef[D], accRes[D]} of consumer warp w and query row
 // r (m in base-2 units, accRes in the rotated domain) must be complete and
 // visible to all consumer threads.  Writes this CTA's record of head hd and,
-// if it is the last CTA of the head to arrive, the head's output.  All
-// consumer threads call it; `merge` is reused as scratch.
+// if it is the last CTA of the head to arrive, the head's output, after
+// folding in the head's BF16 tail tokens (if any).  qs holds the head's raw
+// query rows [G][D] as floats.  All consumer threads call it; `merge` is
+// reused as scratch (it holds at least 4 G (2 + 2 D) floats).
 template <int D, int G, bool RES>
 __device__ __forceinline__ void finish_head(const DecodeParams& p, long long hd, int cta,
-                                            float* merge, volatile int* flags, int tid) {
+                                            float* merge, const float* qs,
+                                            volatile int* flags, int tid) {
+  static_assert(2 * G * D + 3 * G + G * RQ_MAX_TAIL <= 4 * G * (2 + 2 * D),
+                "merge area too small for the tail scratch");
   const int b = (int)(hd / p.kv_heads);
   const int h = (int)(hd % p.kv_heads);
   // which records belong to this head, and which one is ours
@@ -120,6 +125,9 @@ __device__ __forceinline__ void finish_head(const DecodeParams& p, long long hd,
   float* zres = merge;               // [G][D] rotated-domain residual sums
   float* zref = merge + G * D;       // [G][D]
   float* lsum = merge + 2 * G * D;   // [G]
+  float* mrow = lsum + G;            // [G] running max (base 2)
+  float* arow = mrow + G;            // [G] rescale of the cached part
+  float* tsc = arow + G;             // [G][n_tail] tail scores, then weights
   for (int eidx = tid; eidx < G * D; eidx += kConsumerThreads) {
     const int r = eidx / D, i = eidx % D;
     float M = kNegInf;
@@ -136,7 +144,54 @@ __device__ __forceinline__ void finish_head(const DecodeParams& p, long long hd,
     }
     zref[eidx] = aref;
     zres[eidx] = ares;
-    if (i == 0) lsum[r] = l;
+    if (i == 0) {
+      lsum[r] = l;
+      mrow[r] = M;
+    }
+  }
+  const int nt = p.n_tail;
+  if (nt > 0) {
+    // BF16 tail tokens of this head (not encoded yet): same base-2 scores,
+    // merged into the running state before the normalisation
+    const size_t tail0 = (size_t)hd * p.tail_pitch;
+    named_bar_sync(1, kConsumerThreads);
+    for (int e = tid; e < G * nt; e += kConsumerThreads) {
+      const int r = e / nt, jt = e % nt;
+      const uint16_t* kr = p.tail_k + (tail0 + jt) * D;
+      float acc = 0.0f;
+      for (int i = 0; i < D; i += 2) {
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(kr + i);
+        acc = fmaf(qs[r * D + i], __uint_as_float(w << 16), acc);
+        acc = fmaf(qs[r * D + i + 1], __uint_as_float(w & 0xFFFF0000u), acc);
+      }
+      tsc[e] = p.score_scale * acc;
+    }
+    named_bar_sync(1, kConsumerThreads);
+    if (tid < G) {
+      const int r = tid;
+      float mt = mrow[r];
+      for (int jt = 0; jt < nt; ++jt) mt = fmaxf(mt, tsc[r * nt + jt]);
+      const float alpha = (mrow[r] == kNegInf) ? 0.0f : exp2f(mrow[r] - mt);
+      float l = lsum[r] * alpha;
+      for (int jt = 0; jt < nt; ++jt) {
+        const float w = exp2f(tsc[r * nt + jt] - mt);
+        tsc[r * nt + jt] = w;
+        l += w;
+      }
+      lsum[r] = l;
+      mrow[r] = mt;
+      arow[r] = alpha;
+    }
+    named_bar_sync(1, kConsumerThreads);
+    for (int eidx = tid; eidx < G * D; eidx += kConsumerThreads) {
+      const int r = eidx / D, i = eidx % D;
+      float aref = zref[eidx] * arow[r];
+      for (int jt = 0; jt < nt; ++jt)
+        aref = fmaf(tsc[r * nt + jt], __uint_as_float((uint32_t)p.tail_v[(tail0 + jt) * D + i] << 16),
+                    aref);
+      zref[eidx] = aref;
+      if constexpr (RES) zres[eidx] *= arow[r];
+    }
   }
   if constexpr (RES) {
     // Rot^T z = D (c_d H z): butterflies, then scale and signs

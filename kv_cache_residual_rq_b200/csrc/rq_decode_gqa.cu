@@ -9,16 +9,18 @@
 // four products of the fused attention are small dense contractions and go to
 // the tensor cores (mma.sync m16n8k16, fp32 accumulation), per warp and per
 // 16 tokens of a 64-token tile:
-//   S_ref = Q  K^T          bf16 x bf16      (K from shared memory, ldmatrix)
-//   S_res = Q~ L_K^T        fp16 x fp16      per scale group, then x s^K
-//   O_ref^T += V^T P^T      bf16 x bf16      (V via ldmatrix.trans; P split
-//                                             into bf16 hi + lo, so the
-//                                             weights keep ~16 bits)
-//   O_res^T += C_V^T (P s^V)^T  fp16 x fp16  (C_V = codes, exact in fp16)
-// L_K are the levels 2c - (2^b - 1) and C_V the codes c, both built from the
-// packed words in registers; sum_t p s (2c - (2^b-1)) = 2 (C_V^T (P s)^T) -
-// (2^b - 1) sum_t p s is completed when the warp flushes.  Rows beyond G are
-// zero and their weights are forced to zero.
+//   S_ref = Q  K^T              (K from shared memory, ldmatrix)
+//   S_res = Q~ L_K^T            per scale group, then x s^K
+//   O_ref^T += V^T P^T          (V via ldmatrix.trans)
+//   O_res^T += C_V^T (P s^V)^T
+// all in bf16 x bf16 with fp32 accumulation.  L_K are the levels
+// 2c - (2^b - 1) and C_V the codes c, small integers that bf16 holds exactly,
+// built from the packed words in registers; q~, P and P s^V, which are not
+// bf16 values, are split into a bf16 high part and a bf16 remainder and
+// multiplied twice, so they keep ~16 significant bits and bf16's range.
+// sum_t p s (2c - (2^b-1)) = 2 (C_V^T (P s)^T) - (2^b - 1) sum_t p s is
+// completed when the warp flushes.  Rows beyond G are zero and their weights
+// are forced to zero.
 //
 // The reference K/V tiles arrive by TMA tensor copies with the 128-byte
 // swizzle (conflict-free ldmatrix); codes and scales by plain bulk copies, as
@@ -66,7 +68,7 @@ struct GCfg {
   static constexpr int KSG = GROUP / 16;                   // k-steps per scale group
   static constexpr int SB = 2 * NG;                        // scale bytes per token
   static constexpr int WSUM_FLOATS = kConsumerWarps * G * NG;
-  static constexpr int QFRAG_WORDS = 2 * KT * 32 * 2;       // bf16 q and fp16 q~ A fragments
+  static constexpr int QFRAG_WORDS = 3 * KT * 32 * 2;       // q, q~ high, q~ remainder (bf16)
   static constexpr int SMEM_BYTES = 1024 /* base alignment slack */ + RING_BYTES +
                                     4 * (MERGE_FLOATS + QBUF_FLOATS + WSUM_FLOATS +
                                          QFRAG_WORDS) +
@@ -109,14 +111,6 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
-                                        uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, "
-      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
 
 // {lo, hi} -> packed bf16x2 / f16x2 (round to nearest)
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -124,52 +118,55 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
-__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+__device__ __forceinline__ uint32_t bfma2_u(uint32_t a, uint32_t b, uint32_t c) {
   uint32_t r;
-  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
   return r;
 }
-__device__ __forceinline__ uint32_t hfma2_u(uint32_t a, uint32_t b, uint32_t c) {
+__device__ __forceinline__ uint32_t badd2_u(uint32_t a, uint32_t b) {
   uint32_t r;
-  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
-  return r;
-}
-__device__ __forceinline__ uint32_t hadd2_u(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
   return r;
 }
 __device__ __forceinline__ float bf16_lo_f(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi_f(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-constexpr uint32_t kMagic = 0x64006400u;   // fp16 1024 in both halves
+// {lo, hi} as a bf16 pair h plus a bf16 pair of remainders r, lo ~ h.lo + r.lo
+__device__ __forceinline__ void split_bf16(float lo, float hi, uint32_t& h, uint32_t& r) {
+  h = pack_bf16(lo, hi);
+  r = pack_bf16(lo - bf16_lo_f(h), hi - bf16_hi_f(h));
+}
+
+constexpr uint32_t kMagic = 0x43004300u;   // bf16 128.0 in both halves (mantissa unit 1)
 
 // Levels of the K codes for the B fragment of one k-step (16 dims) of one
-// token: b0 = {l(2q), l(2q+1)}, b1 = {l(2q+8), l(2q+9)}, fp16, exact.  INT2:
+// token: b0 = {l(2q), l(2q+1)}, b1 = {l(2q+8), l(2q+9)}, bf16, exact.  INT2:
 // w0 is the k-step's word (code j at bits 2j); INT4: w0, w1 are its two words
 // (code j at bits 4j of word j / 8).
 template <int BITS>
 __device__ __forceinline__ void k_levels(uint32_t w0, uint32_t w1, int q, uint32_t& b0,
                                          uint32_t& b1) {
   if constexpr (BITS == 2) {
-    // lo halves take the code at bit 1 (value 1024 + 2c, level = v - 1027),
-    // hi halves at bit 18 (value 1024 + 4c, level = v/2 - 515)
+    // lo halves take the code at mantissa bit 1 (value 128 + 2c, level =
+    // v - 131), hi halves at bit 18 = mantissa bit 2 (value 128 + 4c,
+    // level = v/2 - 67); every step is exact in bf16
     const uint32_t x = w0 >> (4 * q);
     const uint32_t v0 = ((x << 1) & 0x6u) | ((x << 16) & 0xC0000u) | kMagic;
     const uint32_t v1 = ((x >> 15) & 0x6u) | (x & 0xC0000u) | kMagic;
-    const uint32_t mul = 0x38003C00u;   // {1.0, 0.5}
-    const uint32_t add = 0xE006E403u;   // {-1027, -515}
-    b0 = hfma2_u(v0, mul, add);
-    b1 = hfma2_u(v1, mul, add);
+    const uint32_t mul = 0x3F003F80u;   // {1.0, 0.5}
+    const uint32_t add = 0xC286C303u;   // {-131, -67}
+    b0 = bfma2_u(v0, mul, add);
+    b1 = bfma2_u(v1, mul, add);
   } else {
-    // both halves take the code at bit 1 (value 1024 + 2c, level 2c - 15 = v - 1039)
+    // both halves take the code at mantissa bit 1 (value 128 + 2c, level
+    // 2c - 15 = v - 143)
     const uint32_t x0 = w0 >> (8 * q);
     const uint32_t x1 = w1 >> (8 * q);
     const uint32_t v0 = ((x0 << 1) & 0x1Eu) | ((x0 << 13) & 0x1E0000u) | kMagic;
     const uint32_t v1 = ((x1 << 1) & 0x1Eu) | ((x1 << 13) & 0x1E0000u) | kMagic;
-    const uint32_t add = 0xE40FE40Fu;   // {-1039, -1039}
-    b0 = hadd2_u(v0, add);
-    b1 = hadd2_u(v1, add);
+    const uint32_t add = 0xC30FC30Fu;   // {-143, -143}
+    b0 = badd2_u(v0, add);
+    b1 = badd2_u(v1, add);
   }
 }
 
@@ -191,7 +188,7 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
   float* merge = reinterpret_cast<float*>(smem + C::RING_BYTES);
   float* qbuf = merge + C::MERGE_FLOATS;
   float* wsum_s = qbuf + C::QBUF_FLOATS;
-  uint32_t* qfrag = reinterpret_cast<uint32_t*>(wsum_s + C::WSUM_FLOATS);  // [2][KT][32][2]
+  uint32_t* qfrag = reinterpret_cast<uint32_t*>(wsum_s + C::WSUM_FLOATS);  // [3][KT][32][2]
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(qfrag + C::QFRAG_WORDS);
   uint64_t* empty_bar = full_bar + STAGES;
   volatile int* flags = reinterpret_cast<volatile int*>(empty_bar + STAGES);
@@ -237,7 +234,7 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
         const long long hd = tile / p.nt;
         const int t0 = (int)(tile % p.nt) * TILE;
         const int n = min(TILE, T - t0);
-        const size_t row = (size_t)hd * T + t0;
+        const size_t row = (size_t)hd * p.ctx_pitch + t0;
         unsigned char* st = ring + s * C::STAGE_BYTES;
         uint32_t bytes = 2u * C::NBOX * C::BOX_BYTES;     // full boxes, OOB rows zero-filled
         size_t sc_lo = 0;
@@ -278,9 +275,10 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
   const float score_scale = p.score_scale;
 
   // The per-head Q A-fragments live in shared memory (qfrag): for k-step kk
-  // and lane, {a0, a2} of the bf16 query (kind 0) and of the fp16 rotated
-  // query q~ (kind 1): rows g, dims 16kk + 2q.. and 16kk + 2q + 8..; rows
-  // g >= G are zero, and a1 = a3 = 0 (rows g + 8).
+  // and lane, {a0, a2} of the bf16 query (kind 0) and of the rotated query
+  // q~ as bf16 high part (kind 1) and bf16 remainder (kind 2): rows g, dims
+  // 16kk + 2q.. and 16kk + 2q + 8..; rows g >= G are zero, and a1 = a3 = 0
+  // (rows g + 8).
   auto qfrag_addr = [&](int kind, int kk) {
     return smem_u32(qfrag + ((kind * KT + kk) * 32 + lane) * 2);
   };
@@ -313,16 +311,17 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
 #pragma unroll
       for (int kk = 0; kk < KT; ++kk) {
         uint32_t* fa = qfrag + ((0 * KT + kk) * 32 + lane) * 2;
-        uint32_t* fr = qfrag + ((1 * KT + kk) * 32 + lane) * 2;
+        uint32_t* fh = qfrag + ((1 * KT + kk) * 32 + lane) * 2;
+        uint32_t* fl = qfrag + ((2 * KT + kk) * 32 + lane) * 2;
         if (row_ok) {
           const float* qrow = qs + g * D + 16 * kk + 2 * q;
           const float* trow = qt + g * D + 16 * kk + 2 * q;
           fa[0] = pack_bf16(qrow[0], qrow[1]);       // exact: q is bf16
           fa[1] = pack_bf16(qrow[8], qrow[9]);
-          fr[0] = pack_f16(cd * trow[0], cd * trow[1]);
-          fr[1] = pack_f16(cd * trow[8], cd * trow[9]);
+          split_bf16(cd * trow[0], cd * trow[1], fh[0], fl[0]);
+          split_bf16(cd * trow[8], cd * trow[9], fh[1], fl[1]);
         } else {
-          fa[0] = fa[1] = fr[0] = fr[1] = 0u;
+          fa[0] = fa[1] = fh[0] = fh[1] = fl[0] = fl[1] = 0u;
         }
       }
     }
@@ -357,7 +356,7 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
         const int dim = 16 * mt + g + 8 * (e >> 1);
         if (r < G) {
           mw[r * (2 + 2 * D) + 2 + dim] = oref[mt][e];
-          if constexpr (C::RES) mw[r * (2 + 2 * D) + 2 + D + dim] = 2.0f * ores[mt][e] * (1.0f / 4096.0f);
+          if constexpr (C::RES) mw[r * (2 + 2 * D) + 2 + D + dim] = 2.0f * ores[mt][e];
           else mw[r * (2 + 2 * D) + 2 + D + dim] = 0.0f;
         }
       }
@@ -372,7 +371,7 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
       }
       named_bar_sync(1, kConsumerThreads);
     }
-    finish_head<D, G, C::RES>(p, hd, cta, merge, flags, tid);
+    finish_head<D, G, C::RES>(p, hd, cta, merge, qbuf, flags, tid);
   };
 
   // ---- one tile ----
@@ -403,9 +402,10 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
       mma_bf16(cref[0], a, b[0], b[1]);
       mma_bf16(cref[1], a, b[2], b[3]);
       if constexpr (C::RES) {
-        const uint2 f = *reinterpret_cast<const uint2*>(qfrag + ((1 * KT + kk) * 32 + lane) * 2);
-        a[0] = f.x;
-        a[2] = f.y;
+        const uint2 fh = *reinterpret_cast<const uint2*>(qfrag + ((1 * KT + kk) * 32 + lane) * 2);
+        const uint2 fl = *reinterpret_cast<const uint2*>(qfrag + ((2 * KT + kk) * 32 + lane) * 2);
+        const uint32_t ah[4] = {fh.x, 0u, fh.y, 0u};
+        const uint32_t al[4] = {fl.x, 0u, fl.y, 0u};
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
           const uint32_t* cw = reinterpret_cast<const uint32_t*>(st + C::OFF_CK + tb[nt] * C::CROW);
@@ -416,7 +416,8 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
             const uint2 w2 = *reinterpret_cast<const uint2*>(cw + 2 * kk);
             k_levels<4>(w2.x, w2.y, q, b0, b1);
           }
-          mma_f16(ct[nt], a, b0, b1);
+          mma_bf16(ct[nt], ah, b0, b1);
+          mma_bf16(ct[nt], al, b0, b1);
         }
         if ((kk + 1) % KSG == 0) {
           // end of scale group j: S += s^K_{t, j} x (q~_j . l_j) for c0, c1
@@ -505,8 +506,9 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
           wv[k] = (tk[k] < n) ? pk[k] * sv : 0.0f;       // weight 0 beyond the tile
         }
         wsum[j] += (wv[0] + wv[1]) + (wv[2] + wv[3]);
-        const uint32_t bw0 = pack_f16(wv[0] * 4096.0f, wv[1] * 4096.0f);
-        const uint32_t bw1 = pack_f16(wv[2] * 4096.0f, wv[3] * 4096.0f);
+        uint32_t bh0, bl0, bh1, bl1;
+        split_bf16(wv[0], wv[1], bh0, bl0);
+        split_bf16(wv[2], wv[3], bh1, bl1);
 #pragma unroll
         for (int mt = j * KSG; mt < (j + 1) * KSG; ++mt) {
           // codes of dims 16mt + g (lo halves) and 16mt + g + 8 (hi halves)
@@ -522,13 +524,14 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
               x[k] = lo | (hi << 16) | kMagic;
             }
           }
-          const uint32_t m1024 = 0xE400E400u;   // {-1024, -1024}
+          const uint32_t m128 = 0xC300C300u;   // {-128, -128}
           uint32_t a[4];
-          a[0] = hadd2_u(__byte_perm(x[0], x[1], 0x5410), m1024);   // dim g,   tokens 2q, 2q+1
-          a[1] = hadd2_u(__byte_perm(x[0], x[1], 0x7632), m1024);   // dim g+8
-          a[2] = hadd2_u(__byte_perm(x[2], x[3], 0x5410), m1024);   // dim g,   tokens 2q+8, 2q+9
-          a[3] = hadd2_u(__byte_perm(x[2], x[3], 0x7632), m1024);   // dim g+8
-          mma_f16(ores[mt], a, bw0, bw1);
+          a[0] = badd2_u(__byte_perm(x[0], x[1], 0x5410), m128);   // dim g,   tokens 2q, 2q+1
+          a[1] = badd2_u(__byte_perm(x[0], x[1], 0x7632), m128);   // dim g+8
+          a[2] = badd2_u(__byte_perm(x[2], x[3], 0x5410), m128);   // dim g,   tokens 2q+8, 2q+9
+          a[3] = badd2_u(__byte_perm(x[2], x[3], 0x7632), m128);   // dim g+8
+          mma_bf16(ores[mt], a, bh0, bh1);
+          mma_bf16(ores[mt], a, bl0, bl1);
         }
       }
     }
@@ -561,7 +564,7 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
     if (!aborted) {
       const int t0 = (int)(tile % p.nt) * TILE;
       const int n = min(TILE, T - t0);
-      const size_t row = (size_t)hd * T + t0;
+      const size_t row = (size_t)hd * p.ctx_pitch + t0;
       tile_mma(ring + s * C::STAGE_BYTES, n, (int)((row * SB) & 15));
     }
     __syncwarp();
@@ -643,7 +646,7 @@ cudaError_t launch_decode_gqa(int head_dim, int G, int bits, const DecodeParams&
                               cudaStream_t stream) {
   GqaParams gp;
   gp.p = p;
-  const unsigned long long rows = (unsigned long long)p.batch * p.kv_heads * p.ctx;
+  const unsigned long long rows = (unsigned long long)p.batch * p.kv_heads * p.ctx_pitch;
   if (!encode_kv_map(&gp.tmap_k, p.ref_k, rows, head_dim) ||
       !encode_kv_map(&gp.tmap_v, p.ref_v, rows, head_dim))
     return cudaErrorInvalidValue;

@@ -5,7 +5,9 @@
 // against the final-loop reference, rotated, and quantised per group to INT2
 // (INT4 where the loop is given more bits) with a least-squares scale.
 //
-// Mapping: a row is one (row, kv head, token) vector of head_dim elements.
+// Mapping: a row is one (row, kv head, token) vector of head_dim elements;
+// source and destination rows may sit in arrays of different token pitch
+// (encoding a window slot into a cache position).
 // 16 lanes (head_dim 128) or 8 lanes (64) own a row, 8 consecutive elements
 // per lane, so each lane moves its slice of every loop with one 16-byte
 // load.  The reference slice is loaded once and reused for every loop.  The
@@ -48,10 +50,15 @@ encode_kernel(const EncodeParams p) {
   const float cd = rot_scale<D>();
 
   for (long long row0 = warp * RPW; row0 < p.n_rows; row0 += nwarps * RPW) {
-    const long long row = row0 + slot;
-    const bool valid = row < p.n_rows;
-    const size_t eoff = (size_t)row * D + li * DPL;
+    const long long idx = row0 + slot;             // (head, token) index of this call
+    const bool valid = idx < p.n_rows;
+    const long long hd = idx / p.ctx, t = idx % p.ctx;
+    const long long src_row = hd * p.src_pitch + p.src_offset + t;
+    const long long row = hd * p.dst_pitch + p.dst_offset + t;    // destination row
+    const size_t eoff = (size_t)src_row * D + li * DPL;
     const uint4 rw = valid ? ld_stream(p.ref + eoff) : make_uint4(0, 0, 0, 0);
+    if (valid && p.ref_out)
+      *reinterpret_cast<uint4*>(p.ref_out + (size_t)row * D + li * DPL) = rw;
 
     for (int lb = 0; lb < p.n_loops; lb += kLoopBatch) {
       uint4 xw[kLoopBatch];

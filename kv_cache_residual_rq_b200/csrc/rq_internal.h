@@ -18,7 +18,11 @@ struct EncodeParams {
   uint16_t* scales[RQ_MAX_LOOPS];
   int bits[RQ_MAX_LOOPS];
   const uint16_t* ref;               // bf16 rows of the final loop
-  long long n_rows;                  // rows of head_dim elements
+  uint16_t* ref_out;                 // optional copy of the reference rows
+  long long n_rows;                  // (head, token) rows to encode = heads * ctx
+  int ctx;                           // tokens per head in this call
+  int src_pitch, src_offset;         // token pitch / first token of the inputs
+  int dst_pitch, dst_offset;         // token pitch / first token of the outputs
   int n_loops;
   uint64_t seed;
 };
@@ -73,6 +77,10 @@ struct DecodeParams {
   uint32_t* counters;
   float* records;
   int batch, kv_heads, q_heads, ctx, group;
+  int ctx_pitch;         // token pitch of ref/codes/scales per head (>= ctx)
+  const uint16_t* tail_k;   // optional BF16 tail tokens [heads][tail_pitch][d]
+  const uint16_t* tail_v;
+  int n_tail, tail_pitch;
   int nt;
   long long n_tiles;
   int ctas;

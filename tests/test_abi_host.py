@@ -161,3 +161,34 @@ def test_decode_split_covers_each_head_within_its_record_budget(batch, kv_heads,
         assert start[c_first] <= f < start[c_first + 1]
         assert start[c_last] <= e < start[c_last + 1]
         assert c_last - c_first + 1 <= max_contrib
+
+
+def test_capacity_and_window_arguments_are_checked():
+    E = rq
+    # ctx_cap below ctx is rejected; size queries follow the capacity
+    bad = rq.make_shape(2, 2, 100, 128, 32, q_heads=2, ctx_cap=50)
+    assert rq.rq_codes_bytes(bad, 2) == 0
+    assert _decode(bad) == E.RQ_ERR_INVALID_ARG
+    grown = rq.make_shape(2, 2, 100, 128, 32, ctx_cap=300)
+    assert rq.rq_codes_bytes(grown, 2) == 2 * 2 * 300 * 128 * 2 // 8
+    assert rq.rq_scales_bytes(grown, 2) == 2 * 2 * 300 * 4 * 2
+    # encode_at: ranges must fit their pitches
+    s = rq.make_shape(2, 2, 5, 128, 32)
+    enc = lambda sp, so, dp, do, ref_out=None: rq.rq_encode_at(
+        s, sp, so, dp, do, [FAKE], FAKE, [2], 0, [FAKE], [FAKE], ref_out, stream=0, check=False)
+    assert enc(4, 0, 10, 0) == E.RQ_ERR_INVALID_ARG
+    assert enc(10, 6, 10, 0) == E.RQ_ERR_INVALID_ARG
+    assert enc(10, 0, 10, 6) == E.RQ_ERR_INVALID_ARG
+    assert enc(10, -1, 10, 0) == E.RQ_ERR_INVALID_ARG
+    assert enc(10, 0, 10, 0, ref_out=MISALIGNED) == E.RQ_ERR_ALIGNMENT
+    # decode with a tail: count, pointers, pitch, alignment
+    good = rq.make_shape(2, 2, 100, 128, 32, q_heads=8)
+    ws = rq.rq_decode_workspace_bytes(good)
+    tail = lambda tk, tv, n, pitch: rq.rq_decode_attention_tail(
+        good, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, 1, 0.0, tk, tv, n, pitch, FAKE, FAKE,
+        ws, stream=0, check=False)
+    assert tail(FAKE, FAKE, 257, 300) == E.RQ_ERR_INVALID_ARG
+    assert tail(FAKE, FAKE, -1, 300) == E.RQ_ERR_INVALID_ARG
+    assert tail(None, FAKE, 3, 4) == E.RQ_ERR_INVALID_ARG
+    assert tail(FAKE, FAKE, 3, 2) == E.RQ_ERR_INVALID_ARG
+    assert tail(FAKE, MISALIGNED, 3, 4) == E.RQ_ERR_ALIGNMENT
