@@ -2,9 +2,10 @@
 """Benchmark of the ResidualQuant decode step on B200.
 
 One step = one decode step of the looped model over every layer and loop
-(loop 1 .. L-1 read residual codes, loop L the BF16 reference), followed by
-the append-encode of the step's new token (its L-1 non-final loops against
-its final loop, all layers in one call).  Workload: the Ouro-1.4B-shaped
+(loop 1 .. L-1 read residual codes, loop L the BF16 reference); each call
+attends over the cached tokens plus the new token's own BF16 K/V of that loop,
+and the step ends with the append-encode of the new token into the cache (its
+L-1 non-final loops against its final loop, all layers in one call).  Workload: the Ouro-1.4B-shaped
 decode (24 layers x 4 loops, batch 16, ctx 4096, 16 heads MHA, head_dim 128,
 INT2 residuals with group 32), synthetic seeded data.
 
@@ -139,73 +140,91 @@ def algorithmic_bytes(w, bits):
 
 
 class DecodeStep:
-    """Device-resident cache of every layer plus the per-step inputs."""
+    """Device-resident cache of every layer plus the per-step inputs.
+
+    Cache arrays are contiguous across layers, [layers][K, V][B][Hkv][T][...],
+    so the step's append-encode covers every layer in one call."""
 
     def __init__(self, w, device):
         import torch
         import kv_cache_residual_rq_b200 as rq
         from kv_cache_residual_rq_b200 import synth
         self.w, self.rq, self.torch = w, rq, torch
-        L, N = w.loops, w.layers
-        self.shape = rq.make_shape(w.batch, w.kv_heads, w.ctx, w.head_dim, w.group, w.q_heads)
-        self.refk, self.refv, self.codes, self.scales = [], [], [], []
+        L, N, B, H, T, d = w.loops, w.layers, w.batch, w.kv_heads, w.ctx, w.head_dim
+        self.shape = rq.make_shape(B, H, T, d, w.group, w.q_heads)
+        cache_shape = rq.make_shape(N * 2 * B, H, T, d, w.group)
+        self.ref = torch.empty((N, 2, B, H, T, d), dtype=torch.bfloat16, device=device)
+        self.codes = [rq.alloc_codes(cache_shape, b, device) for b in w.bits]
+        self.scales = [rq.alloc_scales(cache_shape, b, device) for b in w.bits]
+        # exact bytes of one (layer, K or V) part: parts are packed back to back
+        self.code_bytes = [B * H * T * d * b // 8 for b in w.bits]
+        self.scale_bytes = [B * H * T * (d // w.group) * 2 for b in w.bits]
+        assert all(n % 16 == 0 for n in self.code_bytes + self.scale_bytes)
+        layer_shape = rq.make_shape(B, H, T, d, w.group)
         for layer in range(N):
-            rk = synth.reference(w, layer, 0, device)
-            rv = synth.reference(w, layer, 1, device)
-            ck, sk = rq.encode([synth.loop_kv(w, layer, 0, l, rk) for l in range(1, L)], rk,
-                               list(w.bits), w.group, w.seed)
-            cv, sv = rq.encode([synth.loop_kv(w, layer, 1, l, rv) for l in range(1, L)], rv,
-                               list(w.bits), w.group, w.seed)
-            self.refk.append(rk)
-            self.refv.append(rv)
-            self.codes.append((ck, cv))
-            self.scales.append((sk, sv))
+            for kind in (0, 1):
+                r = synth.reference(w, layer, kind, device)
+                self.ref[layer, kind].copy_(r)
+                loops = [synth.loop_kv(w, layer, kind, l, r) for l in range(1, L)]
+                part = layer * 2 + kind
+                rq.rq_encode(layer_shape, loops, self.ref[layer, kind], list(w.bits), w.seed,
+                             [self._slice(self.codes[l], self.code_bytes[l], part)
+                              for l in range(L - 1)],
+                             [self._slice(self.scales[l], self.scale_bytes[l], part)
+                              for l in range(L - 1)])
+                del loops, r
             torch.cuda.empty_cache()
-        # per-step inputs: one query per (loop, layer); the new token's K/V of
-        # every loop, layer-major with K and V stacked as leading rows
+        # per-step inputs: one query per (loop, layer), and the new token's K/V
+        # of every loop and layer ([loop][layer][K, V][B][Hkv][1][d])
         self.q = torch.stack([torch.stack([synth.query(w, layer, loop, device)
                                            for layer in range(N)]) for loop in range(1, L + 1)])
         g = torch.Generator(device=device)
         g.manual_seed(w.seed * 31 + 7)
-        newref = torch.randn((N * 2 * w.batch, w.kv_heads, 1, w.head_dim), generator=g,
-                             device=device)
-        self.new_ref = newref.to(torch.bfloat16)
-        self.new_loops = torch.stack([
-            (newref + w.sigma[l] * torch.randn(newref.shape, generator=g, device=device))
-            .to(torch.bfloat16) for l in range(L - 1)])
-        self.enc_shape = rq.make_shape(N * 2 * w.batch, w.kv_heads, 1, w.head_dim, w.group)
-        self.new_codes = [rq.alloc_codes(self.enc_shape, b, device) for b in w.bits]
-        self.new_scales = [rq.alloc_scales(self.enc_shape, b, device) for b in w.bits]
-        self.out = torch.empty((L, N, w.batch, w.q_heads, w.head_dim), dtype=torch.float32,
-                               device=device)
+        newref = torch.randn((N, 2, B, H, 1, d), generator=g, device=device)
+        self.new_kv = torch.stack(
+            [(newref + w.sigma[l] * torch.randn(newref.shape, generator=g, device=device))
+             .to(torch.bfloat16) for l in range(L - 1)] + [newref.to(torch.bfloat16)])
+        self.append_shape = rq.make_shape(N * 2 * B, H, 1, d, w.group)
+        self.out = torch.empty((L, N, B, w.q_heads, d), dtype=torch.float32, device=device)
         self.ws = rq.alloc_workspace(self.shape, device)
         self.ws_bytes = self.ws.numel()
         self.launches_per_step = L * N + 1
 
+    @staticmethod
+    def _slice(buf, nbytes, part):
+        return buf[part * nbytes:(part + 1) * nbytes]
+
     def run(self, stream, timers=None):
-        """One step.  timers: list to append (start, end, bits) event pairs."""
+        """One decode step: every (loop, layer) attends over the cache plus the
+        new token's BF16 K/V of that loop; then the new token is encoded into
+        the cache (the last slot is reused every step, so T stays fixed).
+        timers: list to append (start, end, bits) event pairs."""
         rq, w, torch = self.rq, self.w, self.torch
         st = stream.cuda_stream
+        T = w.ctx
         for li in range(w.loops):
             bits = w.bits[li] if li < w.loops - 1 else 16
             for layer in range(w.layers):
-                if bits == 16:
-                    ck = cv = sk = sv = None
-                else:
-                    ck, cv = self.codes[layer][0][li], self.codes[layer][1][li]
-                    sk, sv = self.scales[layer][0][li], self.scales[layer][1][li]
+                ck = cv = sk = sv = None
+                if bits != 16:
+                    ck = self._slice(self.codes[li], self.code_bytes[li], 2 * layer)
+                    cv = self._slice(self.codes[li], self.code_bytes[li], 2 * layer + 1)
+                    sk = self._slice(self.scales[li], self.scale_bytes[li], 2 * layer)
+                    sv = self._slice(self.scales[li], self.scale_bytes[li], 2 * layer + 1)
                 ev = None
                 if timers is not None:
                     ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                     ev[0].record(stream)
-                rq.rq_decode_attention(self.shape, self.q[li, layer], self.refk[layer],
-                                       self.refv[layer], ck, cv, sk, sv, bits, w.seed, 0.0,
-                                       self.out[li, layer], self.ws, self.ws_bytes, st)
+                rq.rq_decode_attention_tail(
+                    self.shape, self.q[li, layer], self.ref[layer, 0], self.ref[layer, 1],
+                    ck, cv, sk, sv, bits, w.seed, 0.0, self.new_kv[li, layer, 0],
+                    self.new_kv[li, layer, 1], 1, 1, self.out[li, layer], self.ws, self.ws_bytes, st)
                 if ev is not None:
                     ev[1].record(stream)
                     timers.append((ev[0], ev[1], bits))
-        rq.rq_encode(self.enc_shape, list(self.new_loops), self.new_ref, list(w.bits), w.seed,
-                     self.new_codes, self.new_scales, st)
+        rq.rq_encode_at(self.append_shape, 1, 0, T, T - 1, list(self.new_kv[:w.loops - 1]),
+                        self.new_kv[w.loops - 1], list(w.bits), w.seed, self.codes, self.scales,
+                        self.ref, st)
 
     def step_bytes(self):
         w = self.w
@@ -412,16 +431,14 @@ def run_ours(args, w):
 
     # ---- end-to-end through the public API with host buffers ----
     q_host = state.q.cpu().pin_memory()
-    new_loops_host = state.new_loops.cpu().pin_memory()
-    new_ref_host = state.new_ref.cpu().pin_memory()
+    new_kv_host = state.new_kv.cpu().pin_memory()
     out_host = torch.empty(state.out.shape, dtype=state.out.dtype).pin_memory()
-    h2d = q_host.numel() * 2 + new_loops_host.numel() * 2 + new_ref_host.numel() * 2
+    h2d = q_host.numel() * 2 + new_kv_host.numel() * 2
     d2h = out_host.numel() * 4
 
     def e2e_step():
         state.q.copy_(q_host, non_blocking=True)
-        state.new_loops.copy_(new_loops_host, non_blocking=True)
-        state.new_ref.copy_(new_ref_host, non_blocking=True)
+        state.new_kv.copy_(new_kv_host, non_blocking=True)
         state.run(stream)
         out_host.copy_(state.out, non_blocking=True)
 
