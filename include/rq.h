@@ -266,6 +266,25 @@ rq_status rq_decode_attention_noalloc(const rq_shape *shape, const uint16_t *q,
                                       int bits, uint64_t seed, float softmax_scale, float *out,
                                       void *stream);
 
+/*
+ * rq_reconstruct -- the format's decoder: rebuilds one loop's K (or V) rows
+ * (Abstract: a non-final loop is the final-loop reference plus its rotated,
+ * least-squares-scaled low-bit residual) for consumers that want the loop's
+ * values themselves rather than the fused attention:
+ *   out[r,h,t,:] = f32(ref[r,h,t,:]) + Rot^T (s_g * l)      (bits 2 or 4)
+ *   out[r,h,t,:] = f32(ref[r,h,t,:])                        (bits 16)
+ * computed in fp32 (the inverse rotation summed in butterfly order), written
+ * as fp32, or as bf16 rounded to nearest when out_bf16 != 0.
+ *   shape  : batch, kv_heads, ctx (tokens rebuilt per row and head), head_dim,
+ *            group, ctx_cap (token pitch of ref, codes, scales and out).
+ *   out    : device [rows][Hkv][T][d], T = ctx_cap (ctx when 0); tokens
+ *            beyond ctx are not written.
+ * ref and codes must come from the same rq_encode seed.
+ */
+rq_status rq_reconstruct(const rq_shape *shape, const uint16_t *ref, const uint32_t *codes,
+                         const uint16_t *scales, int bits, uint64_t seed, void *out,
+                         int out_bf16, void *stream);
+
 /* Copies the workspace's device status word to *host_status (blocking read
  * on `stream`).  0 means every decode call since the workspace was zeroed
  * ran clean; non-zero means a bounded wait inside a kernel ran out, its

@@ -11,6 +11,7 @@ from ._abi import (RQ_ERR_ALIGNMENT, RQ_ERR_CUDA, RQ_ERR_INVALID_ARG, RQ_ERR_UNS
                    RQ_ERR_WORKSPACE, RQ_MAX_LOOPS, RQ_OK, RqError, lib, make_shape,
                    rq_codes_bytes, rq_decode_attention, rq_decode_attention_noalloc,
                    rq_decode_attention_tail, rq_decode_workspace_bytes, rq_encode, rq_encode_at,
+                   rq_reconstruct,
                    rq_scales_bytes, rq_shape, rq_status_string, rq_version,
                    rq_workspace_status)
 
@@ -19,8 +20,8 @@ __all__ = [
     "RQ_ERR_CUDA", "RQ_MAX_LOOPS", "RqError", "lib", "rq_shape", "make_shape", "rq_version",
     "rq_status_string", "rq_codes_bytes", "rq_scales_bytes", "rq_decode_workspace_bytes",
     "rq_encode", "rq_encode_at", "rq_decode_attention", "rq_decode_attention_tail",
-    "rq_decode_attention_noalloc", "rq_workspace_status",
-    "alloc_codes", "alloc_scales", "alloc_workspace", "encode", "decode_attention",
+    "rq_decode_attention_noalloc", "rq_reconstruct", "rq_workspace_status",
+    "alloc_codes", "alloc_scales", "alloc_workspace", "encode", "decode_attention", "reconstruct",
 ]
 
 
@@ -57,6 +58,18 @@ def encode(kv_loops, ref, bits_per_loop, group, seed, stream=None):
     scales = [alloc_scales(shape, b, ref.device) for b in bits_per_loop]
     rq_encode(shape, kv_loops, ref, bits_per_loop, seed, codes, scales, stream)
     return codes, scales
+
+
+def reconstruct(ref, codes, scales, bits, group, seed, out_bf16=False, stream=None):
+    """Rebuild a loop's rows [rows, Hkv, T, d] from ref (bf16) and its codes/scales
+    (as returned by encode; None for bits 16).  Returns fp32 (or bf16) rows."""
+    import torch
+    rows, hkv, t, d = ref.shape
+    shape = make_shape(rows, hkv, t, d, group)
+    out = torch.empty(ref.shape, dtype=torch.bfloat16 if out_bf16 else torch.float32,
+                      device=ref.device)
+    rq_reconstruct(shape, ref, codes, scales, bits, seed, out, out_bf16, stream)
+    return out
 
 
 def decode_attention(q, ref_k, ref_v, codes_k, codes_v, scales_k, scales_v, bits, group, seed,

@@ -90,6 +90,9 @@ def lib():
                                                   c.c_int, c.c_uint64, c.c_float, c.c_void_p,
                                                   c.c_void_p]
         L.rq_decode_attention_noalloc.restype = c.c_int
+        L.rq_reconstruct.argtypes = [sp, c.c_void_p, c.c_void_p, c.c_void_p, c.c_int,
+                                     c.c_uint64, c.c_void_p, c.c_int, c.c_void_p]
+        L.rq_reconstruct.restype = c.c_int
         L.rq_workspace_status.argtypes = [c.c_void_p, c.c_size_t, c.POINTER(c.c_uint32), c.c_void_p]
         L.rq_workspace_status.restype = c.c_int
         _lib = L
@@ -215,6 +218,16 @@ def rq_decode_attention_noalloc(shape, q, ref_k, ref_v, codes_k, codes_v, scales
                                            float(softmax_scale), _ptr(out), _stream(stream))
     if check:
         _check(st, "rq_decode_attention_noalloc")
+    return st
+
+
+def rq_reconstruct(shape, ref, codes, scales, bits, seed, out, out_bf16=False, stream=None,
+                   check=True):
+    st = lib().rq_reconstruct(_shp(shape), _ptr(ref), _ptr(codes), _ptr(scales), int(bits),
+                              ctypes.c_uint64(seed), _ptr(out), 1 if out_bf16 else 0,
+                              _stream(stream))
+    if check:
+        _check(st, "rq_reconstruct")
     return st
 
 

@@ -261,6 +261,36 @@ rq_status rq_decode_attention(const rq_shape* shape, const uint16_t* q, const ui
                                   workspace, workspace_bytes, stream);
 }
 
+rq_status rq_reconstruct(const rq_shape* shape, const uint16_t* ref, const uint32_t* codes,
+                         const uint16_t* scales, int bits, uint64_t seed, void* out, int out_bf16,
+                         void* stream) {
+  if (!shape || !ref || !out) return RQ_ERR_INVALID_ARG;
+  if (shape->batch < 1 || shape->kv_heads < 1 || shape->ctx < 0) return RQ_ERR_INVALID_ARG;
+  if (shape->ctx_cap != 0 && shape->ctx_cap < shape->ctx) return RQ_ERR_INVALID_ARG;
+  if (!supported_dims(shape->head_dim, shape->group)) return RQ_ERR_UNSUPPORTED;
+  if (bits != 2 && bits != 4 && bits != 16) return RQ_ERR_UNSUPPORTED;
+  if (bits != 16 && (!codes || !scales)) return RQ_ERR_INVALID_ARG;
+  if (!aligned16(ref) || !aligned16(out) ||
+      (bits != 16 && (!aligned16(codes) || !aligned16(scales))))
+    return RQ_ERR_ALIGNMENT;
+  ReconstructParams p;
+  p.ref = ref;
+  p.codes = bits == 16 ? nullptr : codes;
+  p.scales = bits == 16 ? nullptr : scales;
+  p.out = out;
+  p.ctx = shape->ctx;
+  p.pitch = pitch_of(shape);
+  p.n_rows = (long long)shape->batch * shape->kv_heads * shape->ctx;
+  p.out_bf16 = out_bf16 ? 1 : 0;
+  p.seed = seed;
+  if (p.n_rows == 0) return RQ_OK;
+  const int sms = device_sm_count();
+  if (sms <= 0) return RQ_ERR_CUDA;
+  cudaError_t e = launch_reconstruct(shape->head_dim, shape->group, bits, p, sms,
+                                     static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? RQ_OK : RQ_ERR_CUDA;
+}
+
 rq_status rq_workspace_status(const void* workspace, size_t workspace_bytes,
                               uint32_t* host_status, void* stream) {
   if (!workspace || !host_status || workspace_bytes < kWsHeaderBytes) return RQ_ERR_INVALID_ARG;

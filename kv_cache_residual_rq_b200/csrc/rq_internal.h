@@ -31,6 +31,23 @@ cudaError_t launch_encode(int head_dim, int group, const EncodeParams& p, int nu
                           cudaStream_t stream);
 
 // ---------------------------------------------------------------------------
+// reconstruction (the format's decoder)
+// ---------------------------------------------------------------------------
+struct ReconstructParams {
+  const uint16_t* ref;
+  const uint32_t* codes;      // unused for bits 16
+  const uint16_t* scales;
+  void* out;                  // fp32 or bf16 rows
+  long long n_rows;           // heads * ctx
+  int ctx, pitch;
+  int out_bf16;
+  uint64_t seed;
+};
+
+cudaError_t launch_reconstruct(int head_dim, int group, int bits, const ReconstructParams& p,
+                               int num_sms, cudaStream_t stream);
+
+// ---------------------------------------------------------------------------
 // decode attention
 // ---------------------------------------------------------------------------
 

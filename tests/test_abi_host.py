@@ -192,3 +192,18 @@ def test_capacity_and_window_arguments_are_checked():
     assert tail(None, FAKE, 3, 4) == E.RQ_ERR_INVALID_ARG
     assert tail(FAKE, FAKE, 3, 2) == E.RQ_ERR_INVALID_ARG
     assert tail(FAKE, MISALIGNED, 3, 4) == E.RQ_ERR_ALIGNMENT
+
+
+def test_reconstruct_rejects_bad_arguments_before_launch():
+    E = rq
+    s = rq.make_shape(2, 2, 10, 128, 32)
+    rec = lambda shape=s, bits=2, ref=FAKE, codes=FAKE, scales=FAKE, out=FAKE: rq.rq_reconstruct(
+        shape, ref, codes, scales, bits, 0, out, stream=0, check=False)
+    assert rec(ref=None) == E.RQ_ERR_INVALID_ARG
+    assert rec(out=None) == E.RQ_ERR_INVALID_ARG
+    assert rec(codes=None) == E.RQ_ERR_INVALID_ARG
+    assert rec(bits=3) == E.RQ_ERR_UNSUPPORTED
+    assert rec(shape=rq.make_shape(2, 2, 10, 96, 32)) == E.RQ_ERR_UNSUPPORTED
+    assert rec(shape=rq.make_shape(2, 2, 10, 128, 32, ctx_cap=5)) == E.RQ_ERR_INVALID_ARG
+    assert rec(scales=MISALIGNED) == E.RQ_ERR_ALIGNMENT
+    assert rec(shape=rq.make_shape(2, 2, 0, 128, 32)) == E.RQ_OK      # nothing to rebuild
