@@ -235,20 +235,61 @@ class DecodeStep:
         return total
 
 
+# the sources that make up the single-query decode kernel the roofline names
+DECODE_SOURCES = ("rq_decode.cu", "rq_decode_common.cuh", "rq_device.cuh", "rq_internal.h")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_ouro1.4b_traffic.json")
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "kv_cache_residual_rq_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
-        if fn.endswith((".cu", ".cuh", ".h")):
-            h.update(open(os.path.join(csrc, fn), "rb").read())
+    for fn in DECODE_SOURCES:
+        h.update(open(os.path.join(csrc, fn), "rb").read())
     return h.hexdigest()[:16]
+
+
+def record_traffic(csv_path):
+    """Write the traffic file from an ncu CSV (`--csv --log-file`) of the
+    decode kernel with dram__bytes_read.sum and dram__bytes_write.sum, taken
+    on `python -m kv_cache_residual_rq_b200.profile_decode --tail 1` (one
+    layer of the bench's workload, the bench's launch shape)."""
+    import csv
+    rows = [r for r in csv.reader(l for l in open(csv_path) if not l.startswith("=="))]
+    head = rows[0]
+    ki, mi, vi = head.index("Kernel Name"), head.index("Metric Name"), head.index("Metric Value")
+    ui, idi = head.index("Metric Unit"), head.index("ID")
+    scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9,
+             "B": 1, "KB": 1e3, "MB": 1e6, "GB": 1e9}
+    per = {}
+    for r in rows[1:]:
+        if len(r) <= vi or "decode_kernel<" not in r[ki]:
+            continue
+        if r[mi] in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
+            val = float(r[vi].replace(",", "")) * scale[r[ui]]
+            per.setdefault(r[idi], {})[r[mi]] = val
+    launches = [v for v in per.values() if len(v) == 2]
+    if not launches:
+        raise SystemExit(f"no decode_kernel launches with both DRAM metrics in {csv_path}")
+    rd = sum(v["dram__bytes_read.sum"] for v in launches) / len(launches)
+    wr = sum(v["dram__bytes_write.sum"] for v in launches) / len(launches)
+    rec = {"kernel": "decode_kernel<128, 1, 2> (residual INT2, G = 1)",
+           "workload": "ouro1.4b_decode, one call: B 16, Hkv 16, T 4096 + 1 BF16 tail token",
+           "command": ("ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,"
+                       "gpu__time_duration.sum --clock-control none -k regex:decode_kernel "
+                       "-s 1 -c 2 --csv --log-file <csv> python -m "
+                       "kv_cache_residual_rq_b200.profile_decode --tail 1 --calls 3"),
+           "launches": len(launches), "dram_bytes_read": rd, "dram_bytes_write": wr,
+           "dram_bytes_per_launch": rd + wr, "kernel_source_hash": kernel_source_hash()}
+    with open(TRAFFIC_FILE, "w") as f:
+        json.dump(rec, f, indent=1)
+        f.write("\n")
+    print(json.dumps(rec))
 
 
 def measured_traffic(kernel_hash):
     """ncu DRAM bytes per launch of the decode kernel, if taken on this source."""
-    path = os.path.join(ROOT, "profiles", "decode_ouro1.4b_traffic.json")
     try:
-        rec = json.load(open(path))
+        rec = json.load(open(TRAFFIC_FILE))
     except (OSError, ValueError):
         return None
     if rec.get("kernel_source_hash") != kernel_hash:
@@ -497,7 +538,12 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--record-traffic", metavar="NCU_CSV",
+                    help="write the decode kernel's ncu DRAM bytes into profiles/ and exit")
     args = ap.parse_args(argv)
+    if args.record_traffic:
+        record_traffic(args.record_traffic)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     from kv_cache_residual_rq_b200 import synth

@@ -27,6 +27,8 @@ def main(argv=None):
     ap.add_argument("--calls", type=int, default=4)
     ap.add_argument("--bits", type=int, default=0, help="0: the workload's first loop")
     ap.add_argument("--encode", action="store_true", help="also time rq_encode of the layer")
+    ap.add_argument("--tail", type=int, default=0,
+                    help="BF16 tail tokens per call (1 = the benchmark's launch: cache + new token)")
     args = ap.parse_args(argv)
     w = synth.BY_NAME[args.workload]
     bits = args.bits or w.bits[0]
@@ -52,10 +54,17 @@ def main(argv=None):
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     times = []
+    tail_k = tail_v = None
+    if args.tail:
+        g = torch.Generator(device=dev)
+        g.manual_seed(w.seed * 31 + 7)
+        tail_k = torch.randn((w.batch, w.kv_heads, args.tail, w.head_dim), generator=g,
+                             device=dev).to(torch.bfloat16)
+        tail_v = torch.randn(tail_k.shape, generator=g, device=dev).to(torch.bfloat16)
     for _ in range(args.calls):
         start.record()
         rq.decode_attention(q, refk, refv, ck, cv, sk, sv, bits, w.group, w.seed, out=out,
-                            workspace=ws)
+                            workspace=ws, tail_k=tail_k, tail_v=tail_v, n_tail=args.tail)
         end.record()
         torch.cuda.synchronize()
         times.append(start.elapsed_time(end))

@@ -1,0 +1,31 @@
+"""Host arithmetic of the measurement scripts (no GPU): byte counts and the
+budgeted batch plan, against figures computed by hand from the workload
+shapes (24 layers, 4 loops, 16 KV heads, head_dim 128, ctx 32768, group 32)."""
+from kv_cache_residual_rq_b200 import capacity, synth
+
+W = synth.ENCODE
+CTX = 32768
+
+
+def test_kv_bytes_per_sequence_by_hand():
+    elems = 2 * 24 * 16 * CTX * 128              # K and V elements per loop
+    assert synth.kv_bytes_per_sequence(W, CTX, False) == elems * 2 * 4     # 25.77 GB
+    # reference bf16 + three INT2 loops (2 bits + one fp16 scale per 32)
+    assert synth.kv_bytes_per_sequence(W, CTX, True) == elems * 2 + 3 * elems * (2 + 0.5) // 8
+
+
+def test_budget_plan_max_batches():
+    rows, maxb = capacity.plan(W, CTX, synth.SWEEP_BATCHES, 120e9)
+    assert maxb == {"bf16": 4, "rq": 12}
+    fits = {(s, b) for s, b, _, ok in rows if ok}
+    assert fits == {("bf16", 1), ("bf16", 2), ("bf16", 4),
+                    ("rq", 1), ("rq", 2), ("rq", 4), ("rq", 8), ("rq", 12)}
+
+
+def test_step_bytes_reread_reference_each_loop():
+    # one sequence: BF16 reads 4 loops of K/V; ResidualQuant reads the BF16
+    # reference in each of its 4 calls plus codes and scales of 3 loops
+    elems = 2 * 24 * 16 * CTX * 128
+    qo = 4 * 24 * 16 * 128 * 6
+    assert capacity.step_bytes(W, CTX, 1, "bf16") == elems * 2 * 4 + qo
+    assert capacity.step_bytes(W, CTX, 1, "rq") == elems * 2 * 4 + 3 * elems * 5 // 16 + qo
