@@ -285,6 +285,14 @@ rq_status rq_reconstruct(const rq_shape *shape, const uint16_t *ref, const uint3
                          const uint16_t *scales, int bits, uint64_t seed, void *out,
                          int out_bf16, void *stream);
 
+/* Reads and clears the encoders' sticky status word of the current device
+ * (blocking; waits for all work on the device).  0 means every rq_encode /
+ * rq_encode_at since the last read ran clean; non-zero means a bounded wait
+ * inside the encoder ran out (bit 0: the copy engine's slot was never
+ * released, bit 1: a copy never completed, bit 2: a consumer's tile never
+ * arrived) and the codes written since then are invalid. */
+rq_status rq_encode_take_status(uint32_t *host_status);
+
 /* Copies the workspace's device status word to *host_status (blocking read
  * on `stream`).  0 means every decode call since the workspace was zeroed
  * ran clean; non-zero means a bounded wait inside a kernel ran out, its

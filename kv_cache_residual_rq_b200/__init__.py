@@ -11,7 +11,7 @@ from ._abi import (RQ_ERR_ALIGNMENT, RQ_ERR_CUDA, RQ_ERR_INVALID_ARG, RQ_ERR_UNS
                    RQ_ERR_WORKSPACE, RQ_MAX_LOOPS, RQ_OK, RqError, lib, make_shape,
                    rq_codes_bytes, rq_decode_attention, rq_decode_attention_noalloc,
                    rq_decode_attention_tail, rq_decode_workspace_bytes, rq_encode, rq_encode_at,
-                   rq_reconstruct,
+                   rq_encode_take_status, rq_reconstruct,
                    rq_scales_bytes, rq_shape, rq_status_string, rq_version,
                    rq_workspace_status)
 
@@ -20,7 +20,7 @@ __all__ = [
     "RQ_ERR_CUDA", "RQ_MAX_LOOPS", "RqError", "lib", "rq_shape", "make_shape", "rq_version",
     "rq_status_string", "rq_codes_bytes", "rq_scales_bytes", "rq_decode_workspace_bytes",
     "rq_encode", "rq_encode_at", "rq_decode_attention", "rq_decode_attention_tail",
-    "rq_decode_attention_noalloc", "rq_reconstruct", "rq_workspace_status",
+    "rq_decode_attention_noalloc", "rq_reconstruct", "rq_workspace_status", "rq_encode_take_status",
     "alloc_codes", "alloc_scales", "alloc_workspace", "encode", "decode_attention", "reconstruct",
 ]
 

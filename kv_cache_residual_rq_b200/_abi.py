@@ -95,6 +95,8 @@ def lib():
         L.rq_reconstruct.restype = c.c_int
         L.rq_workspace_status.argtypes = [c.c_void_p, c.c_size_t, c.POINTER(c.c_uint32), c.c_void_p]
         L.rq_workspace_status.restype = c.c_int
+        L.rq_encode_take_status.argtypes = [c.POINTER(c.c_uint32)]
+        L.rq_encode_take_status.restype = c.c_int
         _lib = L
     return _lib
 
@@ -237,4 +239,11 @@ def rq_workspace_status(workspace, workspace_bytes=None, stream=None):
     v = ctypes.c_uint32(0)
     _check(lib().rq_workspace_status(_ptr(workspace), int(workspace_bytes), ctypes.byref(v),
                                      _stream(stream)), "rq_workspace_status")
+    return v.value
+
+
+def rq_encode_take_status():
+    """Read and clear the encoders' sticky status word of the current device."""
+    v = ctypes.c_uint32(0)
+    _check(lib().rq_encode_take_status(ctypes.byref(v)), "rq_encode_take_status")
     return v.value

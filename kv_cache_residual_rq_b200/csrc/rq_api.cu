@@ -3,7 +3,8 @@
 // Host side only: argument validation (before anything is enqueued), the
 // size queries, the work plan of a decode call, and dispatch to the kernels.
 // Nothing here allocates device memory or synchronises, except
-// rq_workspace_status, whose job is to read a status word back.
+// rq_workspace_status and rq_encode_take_status, whose job is to read a
+// status word back.
 #include <climits>
 #include <cmath>
 #include <cstring>
@@ -163,8 +164,12 @@ rq_status rq_encode_at(const rq_shape* shape, int src_pitch, int src_offset, int
   if (p.n_rows == 0 || (active == 0 && !ref_out)) return RQ_OK;
   const int sms = device_sm_count();
   if (sms <= 0) return RQ_ERR_CUDA;
-  cudaError_t e = launch_encode(shape->head_dim, shape->group, p, sms,
-                                static_cast<cudaStream_t>(stream));
+  const bool contiguous = src_pitch == shape->ctx && src_offset == 0 &&
+                          p.n_rows <= kEncodeTmaMaxRows;
+  cudaError_t e = contiguous ? launch_encode_tma(shape->head_dim, shape->group, p, sms,
+                                                 static_cast<cudaStream_t>(stream))
+                             : launch_encode(shape->head_dim, shape->group, p, sms,
+                                             static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? RQ_OK : RQ_ERR_CUDA;
 }
 
@@ -289,6 +294,12 @@ rq_status rq_reconstruct(const rq_shape* shape, const uint16_t* ref, const uint3
   cudaError_t e = launch_reconstruct(shape->head_dim, shape->group, bits, p, sms,
                                      static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? RQ_OK : RQ_ERR_CUDA;
+}
+
+rq_status rq_encode_take_status(uint32_t* host_status) {
+  if (!host_status) return RQ_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return RQ_ERR_CUDA;
+  return encode_take_status(host_status) == cudaSuccess ? RQ_OK : RQ_ERR_CUDA;
 }
 
 rq_status rq_workspace_status(const void* workspace, size_t workspace_bytes,

@@ -575,35 +575,6 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
 
 // ---- host side ---------------------------------------------------------------
 
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult qres;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &qres) ==
-            cudaSuccess &&
-        qres == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-  }
-  return fn;
-}
-
-// [rows][d] bf16 viewed 2-D, box = 64 columns x 64 rows, 128-byte swizzle.
-bool encode_kv_map(CUtensorMap* map, const void* base, unsigned long long rows, int d) {
-  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
-  if (!enc) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)d * 2};
-  cuuint32_t box[2] = {64, (cuuint32_t)kDecodeTile};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
-                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 template <int D, int G, int BITS, int GROUP>
 cudaError_t launch_gqa_t(const GqaParams& gp, cudaStream_t stream) {
   using C = GCfg<D, G, BITS, GROUP>;
@@ -647,8 +618,8 @@ cudaError_t launch_decode_gqa(int head_dim, int G, int bits, const DecodeParams&
   GqaParams gp;
   gp.p = p;
   const unsigned long long rows = (unsigned long long)p.batch * p.kv_heads * p.ctx_pitch;
-  if (!encode_kv_map(&gp.tmap_k, p.ref_k, rows, head_dim) ||
-      !encode_kv_map(&gp.tmap_v, p.ref_v, rows, head_dim))
+  if (!encode_rows_map(&gp.tmap_k, p.ref_k, rows, head_dim, kDecodeTile) ||
+      !encode_rows_map(&gp.tmap_v, p.ref_v, rows, head_dim, kDecodeTile))
     return cudaErrorInvalidValue;
   if (head_dim == 128) return launch_gqa_d<128>(G, bits, gp, stream);
   if (head_dim == 64) return launch_gqa_d<64>(G, bits, gp, stream);

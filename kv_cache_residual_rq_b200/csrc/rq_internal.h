@@ -3,6 +3,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "rq.h"
@@ -27,8 +28,17 @@ struct EncodeParams {
   uint64_t seed;
 };
 
+// streaming encoder: any token pitch and offset (rq_encode.cu)
 cudaError_t launch_encode(int head_dim, int group, const EncodeParams& p, int num_sms,
                           cudaStream_t stream);
+// encoder fed by tensor copies: every source a contiguous [n_rows][head_dim]
+// block (src_pitch == ctx, src_offset == 0), n_rows <= kEncodeTmaMaxRows
+// (rq_encode_tma.cu)
+constexpr long long kEncodeTmaMaxRows = (1ll << 31) - 512;
+cudaError_t launch_encode_tma(int head_dim, int group, const EncodeParams& p, int num_sms,
+                              cudaStream_t stream);
+// read and clear the sticky error bits of the encoders on the current device
+cudaError_t encode_take_status(uint32_t* bits);
 
 // ---------------------------------------------------------------------------
 // reconstruction (the format's decoder)
@@ -114,5 +124,10 @@ cudaError_t launch_decode_gqa(int head_dim, int G, int bits, const DecodeParams&
                               cudaStream_t stream);
 
 int device_sm_count();   // SMs of the current device, cached per device
+
+// TMA map of a row-major [rows][d] bf16 array: box 64 columns x box_rows
+// rows, 128-byte swizzle, rows past the end read as zeros (rq_tma.cu).
+bool encode_rows_map(CUtensorMap* map, const void* base, unsigned long long rows, int d,
+                     int box_rows);
 
 }  // namespace rq
