@@ -194,16 +194,26 @@ class DecodeStep:
     def _slice(buf, nbytes, part):
         return buf[part * nbytes:(part + 1) * nbytes]
 
-    def run(self, stream, timers=None):
+    def run(self, stream, timers=None, bufs=None):
         """One decode step: every (loop, layer) attends over the cache plus the
         new token's BF16 K/V of that loop; then the new token is encoded into
         the cache (the last slot is reused every step, so T stays fixed).
-        timers: list to append (start, end, bits) event pairs."""
+        timers: list to append (start, end, bits, calls) per loop segment --
+        events only at loop boundaries, so consecutive calls of a loop stay
+        back to back and each launch overlaps its predecessor's tail
+        (programmatic dependent launch); an event between two launches would
+        serialise them.  bufs: (q, new_kv, out) tensors to use instead of the
+        step's own (double-buffered end-to-end loop)."""
         rq, w, torch = self.rq, self.w, self.torch
         st = stream.cuda_stream
+        q_all, kv_all, out_all = bufs if bufs is not None else (self.q, self.new_kv, self.out)
         T = w.ctx
         for li in range(w.loops):
             bits = w.bits[li] if li < w.loops - 1 else 16
+            ev = None
+            if timers is not None:
+                ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                ev[0].record(stream)
             for layer in range(w.layers):
                 ck = cv = sk = sv = None
                 if bits != 16:
@@ -211,19 +221,15 @@ class DecodeStep:
                     cv = self._slice(self.codes[li], self.code_bytes[li], 2 * layer + 1)
                     sk = self._slice(self.scales[li], self.scale_bytes[li], 2 * layer)
                     sv = self._slice(self.scales[li], self.scale_bytes[li], 2 * layer + 1)
-                ev = None
-                if timers is not None:
-                    ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                    ev[0].record(stream)
                 rq.rq_decode_attention_tail(
-                    self.shape, self.q[li, layer], self.ref[layer, 0], self.ref[layer, 1],
-                    ck, cv, sk, sv, bits, w.seed, 0.0, self.new_kv[li, layer, 0],
-                    self.new_kv[li, layer, 1], 1, 1, self.out[li, layer], self.ws, self.ws_bytes, st)
-                if ev is not None:
-                    ev[1].record(stream)
-                    timers.append((ev[0], ev[1], bits))
-        rq.rq_encode_at(self.append_shape, 1, 0, T, T - 1, list(self.new_kv[:w.loops - 1]),
-                        self.new_kv[w.loops - 1], list(w.bits), w.seed, self.codes, self.scales,
+                    self.shape, q_all[li, layer], self.ref[layer, 0], self.ref[layer, 1],
+                    ck, cv, sk, sv, bits, w.seed, 0.0, kv_all[li, layer, 0],
+                    kv_all[li, layer, 1], 1, 1, out_all[li, layer], self.ws, self.ws_bytes, st)
+            if ev is not None:
+                ev[1].record(stream)
+                timers.append((ev[0], ev[1], bits, w.layers))
+        rq.rq_encode_at(self.append_shape, 1, 0, T, T - 1, list(kv_all[:w.loops - 1]),
+                        kv_all[w.loops - 1], list(w.bits), w.seed, self.codes, self.scales,
                         self.ref, st)
 
     def step_bytes(self):
@@ -461,8 +467,9 @@ def run_ours(args, w):
     max_elapsed, tokens = aggregate(elapsed, w.batch * args.steps)
     value = tokens / max_elapsed
 
-    res_ms = [a.elapsed_time(b) for a, b, bits in timers if bits != 16]
-    ref_ms = [a.elapsed_time(b) for a, b, bits in timers if bits == 16]
+    # average launch duration = loop segment time / calls in the segment
+    res_ms = [a.elapsed_time(b) / n for a, b, bits, n in timers if bits != 16]
+    ref_ms = [a.elapsed_time(b) / n for a, b, bits, n in timers if bits == 16]
     avg_res_s = statistics.mean(res_ms) / 1e3
     bytes_res = algorithmic_bytes(w, w.bits[0])
     peak, peak_kind = hbm_peak()
@@ -471,28 +478,56 @@ def run_ours(args, w):
     traffic = measured_traffic(khash)
 
     # ---- end-to-end through the public API with host buffers ----
+    # Like a serving loop, inputs and outputs are double-buffered: step k+1's
+    # queries and new-token K/V go up on a copy stream while step k computes,
+    # and step k's outputs come back while step k+1 computes.  Every step
+    # still moves its own inputs and outputs between pinned host memory and
+    # the device inside the timed region.
     q_host = state.q.cpu().pin_memory()
     new_kv_host = state.new_kv.cpu().pin_memory()
-    out_host = torch.empty(state.out.shape, dtype=state.out.dtype).pin_memory()
+    out_host = [torch.empty(state.out.shape, dtype=state.out.dtype).pin_memory()
+                for _ in range(2)]
+    bufs = [(state.q, state.new_kv, state.out),
+            (torch.empty_like(state.q), torch.empty_like(state.new_kv),
+             torch.empty_like(state.out))]
     h2d = q_host.numel() * 2 + new_kv_host.numel() * 2
-    d2h = out_host.numel() * 4
+    d2h = out_host[0].numel() * 4
+    copy = torch.cuda.Stream(device)
 
-    def e2e_step():
-        state.q.copy_(q_host, non_blocking=True)
-        state.new_kv.copy_(new_kv_host, non_blocking=True)
-        state.run(stream)
-        out_host.copy_(state.out, non_blocking=True)
+    def e2e_loop(n, e_start=None, e_end=None):
+        up = [None] * n
 
-    for _ in range(args.warmup):
-        e2e_step()
+        def upload(k):
+            qd, kvd, _ = bufs[k % 2]
+            with torch.cuda.stream(copy):
+                qd.copy_(q_host, non_blocking=True)
+                kvd.copy_(new_kv_host, non_blocking=True)
+            up[k] = torch.cuda.Event()
+            up[k].record(copy)
+
+        if e_start is not None:
+            e_start.record(copy)
+        for k in range(min(2, n)):
+            upload(k)
+        for k in range(n):
+            stream.wait_event(up[k])
+            state.run(stream, bufs=bufs[k % 2])
+            done = torch.cuda.Event()
+            done.record(stream)
+            copy.wait_event(done)
+            with torch.cuda.stream(copy):
+                out_host[k % 2].copy_(bufs[k % 2][2], non_blocking=True)
+            if k + 2 < n:
+                upload(k + 2)      # after step k's download: its buffers are free
+        if e_end is not None:
+            e_end.record(copy)
+
+    e2e_loop(args.warmup)
     barrier()
     torch.cuda.synchronize(device)
     e_start = torch.cuda.Event(enable_timing=True)
     e_end = torch.cuda.Event(enable_timing=True)
-    e_start.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e_end.record(stream)
+    e2e_loop(args.steps, e_start, e_end)
     torch.cuda.synchronize(device)
     barrier()
     e_elapsed, e_tokens = aggregate(e_start.elapsed_time(e_end) / 1e3, w.batch * args.steps)
@@ -518,7 +553,9 @@ def run_ours(args, w):
                          "kernel": f"decode_kernel<128,1,{w.bits[0]}> (residual loop)",
                          "algorithmic_bytes_per_launch": bytes_res,
                          "avg_launch_us": avg_res_s * 1e6, "peak_source": peak_kind + " hbm_gbs",
-                         "launches_timed": len(res_ms)},
+                         "launches_timed": len(res_ms) * w.layers,
+                         "timing": ("CUDA events at the loop boundaries of every timed step: "
+                                    "segment time / 24 back-to-back launches")},
             "step_hbm_gbs_per_gpu": step_bytes / (max_elapsed / args.steps) / 1e9,
             "ref_loop_avg_launch_us": statistics.mean(ref_ms) * 1e3 if ref_ms else None,
             "workspace_status": status,

@@ -145,6 +145,7 @@ decode_kernel(const DecodeParams p) {
   const int warp = tid >> 5;
   const int lane = tid & 31;
   const int cta = blockIdx.x;
+  pdl_allow_next();
   if (cta >= p.ctas) return;
 
   const long long tile_begin = (long long)cta * p.n_tiles / p.ctas;
@@ -161,6 +162,7 @@ decode_kernel(const DecodeParams p) {
     fence_mbar_init();
   }
   __syncthreads();
+  pdl_wait_prev();     // inputs and workspace may come from the previous kernel
 
   const int T = p.ctx;
   const int SB = (D / p.group) * 2;     // scale bytes per token
@@ -629,8 +631,7 @@ cudaError_t launch_decode_t(const DecodeParams& p, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  decode_kernel<D, G, BITS><<<p.ctas, kThreads, C::SMEM_BYTES, stream>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(decode_kernel<D, G, BITS>, p.ctas, kThreads, C::SMEM_BYTES, stream, p);
 }
 
 template <int D, int G>

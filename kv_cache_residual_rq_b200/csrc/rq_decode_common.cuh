@@ -32,32 +32,55 @@ __device__ __forceinline__ float half_at(const unsigned char* p) {
   return __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t*>(p)));
 }
 
+// Walsh-Hadamard transform (no scaling) of a D-vector spread over a warp:
+// lane owns coordinates lane*E .. lane*E+E-1, E = D/32.  Strides below E in
+// registers, the rest by shfl.xor; ascending strides, butterfly (a+b, a-b).
+template <int D>
+__device__ __forceinline__ void warp_fwht(float (&v)[D / 32], int lane) {
+  constexpr int E = D / 32;
+#pragma unroll
+  for (int h = 1; h < E; h <<= 1) {
+#pragma unroll
+    for (int k = 0; k < E; ++k) {
+      if (!(k & h)) {
+        const float a = v[k], c = v[k + h];
+        v[k] = a + c;
+        v[k + h] = a - c;
+      }
+    }
+  }
+#pragma unroll
+  for (int m = 1; m < 32; m <<= 1) {
+    const float sg = (lane & m) ? -1.0f : 1.0f;
+#pragma unroll
+    for (int k = 0; k < E; ++k) v[k] = fmaf(sg, v[k], __shfl_xor_sync(0xffffffffu, v[k], m));
+  }
+}
+
 // Loads the G query rows of head hd into qs[G][D] (fp32) and FWHT(D q) into
 // qt[G][D]: the rotation q~ = Rot q without its 1/sqrt(d) factor, which the
-// caller applies.  All consumer threads; ends with a consumer barrier.
+// caller applies.  One warp per row; all consumer threads call it, and it
+// ends with a consumer barrier.
 template <int D, int G>
 __device__ __forceinline__ void load_rotate_queries(const DecodeParams& p, long long hd,
                                                     float* qs, float* qt, int tid) {
+  constexpr int E = D / 32;
   const int b = (int)(hd / p.kv_heads);
   const int h = (int)(hd % p.kv_heads);
+  const int warp = tid >> 5, lane = tid & 31;
   named_bar_sync(1, kConsumerThreads);          // previous users of the buffers done
-  for (int e = tid; e < G * D; e += kConsumerThreads) {
-    const int r = e / D, i = e % D;
-    const uint16_t raw = p.q[((size_t)b * p.q_heads + (size_t)h * G + r) * D + i];
-    const float v = __uint_as_float((uint32_t)raw << 16);
-    qs[e] = v;
-    qt[e] = flip_sign(v, sign_bit(p.seed, i));
-  }
-  for (int hs = 1; hs < D; hs <<= 1) {
-    named_bar_sync(1, kConsumerThreads);
-    for (int e = tid; e < G * D / 2; e += kConsumerThreads) {
-      const int r = e / (D / 2), pr = e % (D / 2);
-      const int i = (pr / hs) * 2 * hs + (pr % hs);
-      float* row = qt + r * D;
-      const float a = row[i], c = row[i + hs];
-      row[i] = a + c;
-      row[i + hs] = a - c;
+  for (int r = warp; r < G; r += kConsumerWarps) {
+    const uint16_t* qr = p.q + ((size_t)b * p.q_heads + (size_t)h * G + r) * D + lane * E;
+    float v[E];
+#pragma unroll
+    for (int k = 0; k < E; ++k) {
+      const float x = __uint_as_float((uint32_t)qr[k] << 16);
+      qs[r * D + lane * E + k] = x;
+      v[k] = flip_sign(x, sign_bit(p.seed, lane * E + k));
     }
+    warp_fwht<D>(v, lane);
+#pragma unroll
+    for (int k = 0; k < E; ++k) qt[r * D + lane * E + k] = v[k];
   }
   named_bar_sync(1, kConsumerThreads);
 }
@@ -88,22 +111,31 @@ __device__ __forceinline__ void finish_head(const DecodeParams& p, long long hd,
     return;
   }
   float* recs = p.records + (size_t)hd * p.max_contrib * G * (4 + 2 * D);
-  for (int eidx = tid; eidx < G * (2 * D + 2); eidx += kConsumerThreads) {
-    const int r = eidx / (2 * D + 2), q = eidx % (2 * D + 2);
+  // per query row: the warps' common max and each warp's weight, once
+  float* wts = const_cast<float*>(qs) + G * D;    // [G][1 + warps], the rotated-query buffer
+  if (tid < G) {
+    const int r = tid;
     float M = kNegInf;
 #pragma unroll
     for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, merge[(w * G + r) * (2 + 2 * D)]);
+    wts[r * (1 + kConsumerWarps)] = M;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) {
+      const float mw = merge[(w * G + r) * (2 + 2 * D)];
+      wts[r * (1 + kConsumerWarps) + 1 + w] = (mw == kNegInf) ? 0.0f : exp2f(mw - M);
+    }
+  }
+  named_bar_sync(1, kConsumerThreads);
+  for (int eidx = tid; eidx < G * (2 * D + 2); eidx += kConsumerThreads) {
+    const int r = eidx / (2 * D + 2), q = eidx % (2 * D + 2);
+    const float* wr = wts + r * (1 + kConsumerWarps);
     float* out_rec = recs + ((size_t)j * G + r) * (4 + 2 * D);
     if (q == 0) {
-      out_rec[0] = M;
+      out_rec[0] = wr[0];
     } else {
       float acc = 0.0f;
 #pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) {
-        const float* mr = merge + (w * G + r) * (2 + 2 * D);
-        const float wt = (mr[0] == kNegInf) ? 0.0f : exp2f(mr[0] - M);
-        acc += wt * mr[q];
-      }
+      for (int w = 0; w < kConsumerWarps; ++w) acc += wr[1 + w] * merge[(w * G + r) * (2 + 2 * D) + q];
       out_rec[q == 1 ? 1 : q + 2] = acc;   // l at 1; accRef/accRes from 4
     }
   }
@@ -155,16 +187,21 @@ __device__ __forceinline__ void finish_head(const DecodeParams& p, long long hd,
     // merged into the running state before the normalisation
     const size_t tail0 = (size_t)hd * p.tail_pitch;
     named_bar_sync(1, kConsumerThreads);
-    for (int e = tid; e < G * nt; e += kConsumerThreads) {
-      const int r = e / nt, jt = e % nt;
-      const uint16_t* kr = p.tail_k + (tail0 + jt) * D;
-      float acc = 0.0f;
-      for (int i = 0; i < D; i += 2) {
-        const uint32_t w = *reinterpret_cast<const uint32_t*>(kr + i);
-        acc = fmaf(qs[r * D + i], __uint_as_float(w << 16), acc);
-        acc = fmaf(qs[r * D + i + 1], __uint_as_float(w & 0xFFFF0000u), acc);
+    {
+      // one warp per (query row, tail token): lane-parallel dot product
+      constexpr int E = D / 32;
+      const int warp = tid >> 5, lane = tid & 31;
+      for (int e = warp; e < G * nt; e += kConsumerWarps) {
+        const int r = e / nt, jt = e % nt;
+        const uint16_t* kr = p.tail_k + (tail0 + jt) * D + lane * E;
+        float acc = 0.0f;
+#pragma unroll
+        for (int k = 0; k < E; ++k)
+          acc = fmaf(qs[r * D + lane * E + k], __uint_as_float((uint32_t)kr[k] << 16), acc);
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+        if (lane == 0) tsc[e] = p.score_scale * acc;
       }
-      tsc[e] = p.score_scale * acc;
     }
     named_bar_sync(1, kConsumerThreads);
     if (tid < G) {
@@ -193,27 +230,31 @@ __device__ __forceinline__ void finish_head(const DecodeParams& p, long long hd,
       if constexpr (RES) zres[eidx] *= arow[r];
     }
   }
-  if constexpr (RES) {
-    // Rot^T z = D (c_d H z): butterflies, then scale and signs
-    for (int hs = 1; hs < D; hs <<= 1) {
-      named_bar_sync(1, kConsumerThreads);
-      for (int eidx = tid; eidx < G * D / 2; eidx += kConsumerThreads) {
-        const int r = eidx / (D / 2), pr = eidx % (D / 2);
-        const int i = (pr / hs) * 2 * hs + (pr % hs);
-        float* row = zres + r * D;
-        const float a = row[i], c = row[i + hs];
-        row[i] = a + c;
-        row[i + hs] = a - c;
-      }
-    }
-  }
+  // out = (zref + Rot^T zres) / l, Rot^T z = D (c_d H z): one warp per row
   named_bar_sync(1, kConsumerThreads);
-  const float cd = rot_scale<D>();
-  for (int eidx = tid; eidx < G * D; eidx += kConsumerThreads) {
-    const int r = eidx / D, i = eidx % D;
-    float num = zref[eidx];
-    if constexpr (RES) num += flip_sign(cd * zres[eidx], sign_bit(p.seed, i));
-    p.out[((size_t)b * p.q_heads + (size_t)h * G + r) * D + i] = num / lsum[r];
+  {
+    constexpr int E = D / 32;
+    const int warp = tid >> 5, lane = tid & 31;
+    const float cd = rot_scale<D>();
+    for (int r = warp; r < G; r += kConsumerWarps) {
+      float z[E];
+#pragma unroll
+      for (int k = 0; k < E; ++k) z[k] = RES ? zres[r * D + lane * E + k] : 0.0f;
+      if constexpr (RES) warp_fwht<D>(z, lane);
+      const float inv_l = 1.0f / lsum[r];
+      float o[E];
+#pragma unroll
+      for (int k = 0; k < E; ++k) {
+        float num = zref[r * D + lane * E + k];
+        if constexpr (RES) num += flip_sign(cd * z[k], sign_bit(p.seed, lane * E + k));
+        o[k] = num * inv_l;
+      }
+      float* dst = p.out + ((size_t)b * p.q_heads + (size_t)h * G + r) * D + lane * E;
+      if constexpr (E == 4)
+        *reinterpret_cast<float4*>(dst) = make_float4(o[0], o[1], o[2], o[3]);
+      else
+        *reinterpret_cast<float2*>(dst) = make_float2(o[0], o[1]);
+    }
   }
 }
 

@@ -197,6 +197,7 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
   const int warp = tid >> 5;
   const int lane = tid & 31;
   const int cta = blockIdx.x;
+  pdl_allow_next();
   if (cta >= p.ctas) return;
 
   const long long tile_begin = (long long)cta * p.n_tiles / p.ctas;
@@ -213,6 +214,7 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
     fence_mbar_init();
   }
   __syncthreads();
+  pdl_wait_prev();     // inputs and workspace may come from the previous kernel
 
   const int T = p.ctx;
 
@@ -586,8 +588,8 @@ cudaError_t launch_gqa_t(const GqaParams& gp, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  decode_gqa_kernel<D, G, BITS, GROUP><<<gp.p.ctas, kDecodeThreads, C::SMEM_BYTES, stream>>>(gp);
-  return cudaGetLastError();
+  return launch_pdl(decode_gqa_kernel<D, G, BITS, GROUP>, gp.p.ctas, kDecodeThreads,
+                    C::SMEM_BYTES, stream, gp);
 }
 
 template <int D, int G>

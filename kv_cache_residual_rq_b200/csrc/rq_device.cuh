@@ -124,6 +124,17 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
+// Programmatic dependent launch (sm_90 and later).  pdl_allow_next lets the
+// next kernel of the stream be scheduled once every CTA of this grid has
+// started; pdl_wait_prev blocks until the grids before this one have
+// completed and their writes are visible.  A kernel launched with the
+// programmatic-serialization attribute must call pdl_wait_prev before its
+// first global memory access.
+__device__ __forceinline__ void pdl_allow_next() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait_prev() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // named barrier over `nthreads` threads (a multiple of 32)
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");

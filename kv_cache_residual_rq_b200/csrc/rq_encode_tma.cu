@@ -88,6 +88,13 @@ __device__ __forceinline__ float fma_bf16(uint32_t a2, uint32_t b2, float c) {
   return d;
 }
 
+// max(m, |a|, |b|) for m >= 0
+__device__ __forceinline__ float fmax3_abs(float m, float a, float b) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(m), "f"(fabsf(a)), "f"(fabsf(b)));
+  return r;
+}
+
 __device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
   float2 r;
   asm("{\n\t.reg .b64 ra, rb, rr;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
@@ -120,7 +127,7 @@ __device__ __forceinline__ void quantize_store(const float2 (&P)[16], uint32_t* 
                                                uint16_t* scales_row, int q, bool valid) {
   float amax = 0.0f;
 #pragma unroll
-  for (int m = 0; m < 16; ++m) amax = fmaxf(amax, fmaxf(fabsf(P[m].x), fabsf(P[m].y)));
+  for (int m = 0; m < 16; ++m) amax = fmax3_abs(amax, P[m].x, P[m].y);
   if (GROUP == 64) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, RPW));
   constexpr float outer = (float)(1 << (BITS - 1)) - 0.5f;
   const float inv = (amax < 1.17549435e-38f) ? 0.0f : __fdiv_rn(outer, amax);
@@ -146,14 +153,23 @@ __device__ __forceinline__ void quantize_store(const float2 (&P)[16], uint32_t* 
     const float2 fl = fsub2(t, mg);                 // floor(u)
     const float2 lv = __ffma2_rn(fl, two, one);     // level 2 floor(u) + 1 = 2c - (2^b - 1)
     dot = __ffma2_rn(P[m], lv, dot);
-    nrm = __ffma2_rn(lv, lv, nrm);
+    if constexpr (BITS == 4) nrm = __ffma2_rn(lv, lv, nrm);
   }
   // every field received (0x4B400000 + floor(u)); code c = floor(u) + 2^(b-1)
   constexpr uint32_t kOff = kFloorMagicBits - (1u << (BITS - 1));
   constexpr uint32_t kSpread = BITS == 2 ? 0x55555555u : 0x11111111u;
 #pragma unroll
   for (int k = 0; k < NW; ++k) w[k] -= kOff * kSpread;
-  float d = dot.x + dot.y, n = nrm.x + nrm.y;
+  float d = dot.x + dot.y, n;
+  if constexpr (BITS == 2) {
+    // <l, l> = 32 + 8 * (number of outer levels +-3, i.e. codes 0 and 3,
+    // whose two bits are equal): an exact integer either way
+    const uint32_t e = __popc(~(w[0] ^ (w[0] >> 1)) & 0x55555555u) +
+                       __popc(~(w[1] ^ (w[1] >> 1)) & 0x55555555u);
+    n = (float)(32u + 8u * e);
+  } else {
+    n = nrm.x + nrm.y;
+  }
   if (GROUP == 64) {
     d += __shfl_xor_sync(kFull, d, RPW);
     n += __shfl_xor_sync(kFull, n, RPW);
@@ -184,6 +200,7 @@ encode_tma_kernel(const __grid_constant__ EncodeTmaParams tp) {
   uint64_t* empty = full + kSlots;
   const EncodeParams& p = tp.p;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_allow_next();
 
   for (int i = threadIdx.x; i < D / 2; i += blockDim.x) {
     const uint32_t lo = sign_bit(p.seed, 2 * i) ? 0xBF80u : 0x3F80u;
@@ -199,6 +216,7 @@ encode_tma_kernel(const __grid_constant__ EncodeTmaParams tp) {
     fence_mbar_init();
   }
   __syncthreads();
+  pdl_wait_prev();     // the sources may come from the previous kernel
 
   const int per_tile = 1 + tp.n_active;
   if (warp == CW) {
@@ -356,8 +374,8 @@ cudaError_t launch_t(const EncodeTmaParams& tp, int num_sms, cudaStream_t stream
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   const int grid = tp.n_tiles < num_sms ? tp.n_tiles : num_sms;
-  encode_tma_kernel<D, GROUP, kConsumerWarps><<<grid, C::THREADS, C::SMEM, stream>>>(tp);
-  return cudaGetLastError();
+  return launch_pdl(encode_tma_kernel<D, GROUP, kConsumerWarps>, (unsigned)grid, C::THREADS,
+                    C::SMEM, stream, tp);
 }
 
 }  // namespace

@@ -3,12 +3,41 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <utility>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "rq.h"
 
 namespace rq {
+
+// Launch with programmatic stream serialization: the kernel may be scheduled
+// while the previous kernel of the stream is finishing, and waits for it
+// (pdl_wait_prev) before touching global memory.  Only for kernels that call
+// pdl_wait_prev first.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+  if (e == cudaErrorNotSupported || e == cudaErrorInvalidValue) {
+    // a stream that cannot take the attribute: plain stream order (the
+    // kernel's wait then returns at once)
+    (void)cudaGetLastError();
+    cfg.numAttrs = 0;
+    e = cudaLaunchKernelEx(&cfg, kernel, args...);
+  }
+  return e;
+}
 
 // ---------------------------------------------------------------------------
 // encoder
