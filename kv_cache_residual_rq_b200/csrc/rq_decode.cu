@@ -83,8 +83,11 @@ struct Cfg {
   static constexpr int MERGE_FLOATS = kConsumerWarps * G * (2 + 2 * D);
   static constexpr int AREA_FLOATS = LUT_FLOATS > MERGE_FLOATS ? LUT_FLOATS : MERGE_FLOATS;
   static constexpr int QBUF_FLOATS = 2 * G * D;             // q and q~
+  // bf16 query rows of the first heads of a CTA's run, fetched at the start
+  static constexpr int QPRE_HEADS = 4;
+  static constexpr int QPRE_BYTES = QPRE_HEADS * G * D * 2;
   static constexpr int SMEM_BYTES =
-      RING_BYTES + 4 * (AREA_FLOATS + QBUF_FLOATS) + 2 * STAGES * 8 + 16;
+      RING_BYTES + 4 * (AREA_FLOATS + QBUF_FLOATS) + 2 * STAGES * 8 + 16 + QPRE_BYTES;
   static_assert(TPW % TPS == 0 && STEPS % CH == 0, "tile split");
   static_assert(G != 1 || CH == STEPS, "G == 1 processes a whole tile per chunk");
   static_assert(STAGE_BYTES % 16 == 0, "stage alignment");
@@ -140,6 +143,8 @@ decode_kernel(const DecodeParams p) {
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(qbuf + C::QBUF_FLOATS);
   uint64_t* empty_bar = full_bar + STAGES;
   volatile int* flags = reinterpret_cast<volatile int*>(empty_bar + STAGES);  // [0] abort, [1] last
+  uint16_t* qpre = reinterpret_cast<uint16_t*>(
+      reinterpret_cast<unsigned char*>(empty_bar + STAGES) + 16);      // [QPRE_HEADS][G][D]
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -217,6 +222,19 @@ decode_kernel(const DecodeParams p) {
   }
 
   // ========================= consumer warps ===============================
+  // the query rows of the first heads of the run, while the first tiles are
+  // in flight (made visible by the barrier that starts load_rotate_queries)
+  const long long h_first = tile_begin / p.nt;
+  const int n_pre =
+      n_my > 0 ? (int)min((long long)C::QPRE_HEADS, (tile_end - 1) / p.nt - h_first + 1) : 0;
+  for (int e = tid; e < n_pre * G * D / 8; e += kConsumerThreads) {
+    const int hh = e / (G * D / 8), rem = e % (G * D / 8);
+    const long long hd = h_first + hh;
+    const int b = (int)(hd / p.kv_heads), h = (int)(hd % p.kv_heads);
+    reinterpret_cast<uint4*>(qpre)[e] =
+        reinterpret_cast<const uint4*>(p.q + ((size_t)b * p.q_heads + (size_t)h * G) * D)[rem];
+  }
+
   const int li = lane % LPT;          // lane within its token
   const int slot = lane / LPT;        // token slot within a warp step
   const int dim0 = li * DPL;          // first dim this lane owns
@@ -264,7 +282,8 @@ decode_kernel(const DecodeParams p) {
   auto setup_head = [&](long long hd) {
     float* qs = qbuf;              // [G][D] raw q
     float* qt = qbuf + G * D;      // [G][D] FWHT(D q)
-    load_rotate_queries<D, G>(p, hd, qs, qt, tid);
+    load_rotate_queries<D, G>(p, hd, qs, qt, tid,
+                              hd - h_first < n_pre ? qpre + (hd - h_first) * G * D : nullptr);
     const float cd = rot_scale<D>();
     if constexpr (C::LUT) {
       // lut[byte][slice] = sum_k q~[4 slice + k] * l(c_k(byte)), l(c) = 2c - 3,

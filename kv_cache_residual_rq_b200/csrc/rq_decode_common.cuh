@@ -59,18 +59,21 @@ __device__ __forceinline__ void warp_fwht(float (&v)[D / 32], int lane) {
 
 // Loads the G query rows of head hd into qs[G][D] (fp32) and FWHT(D q) into
 // qt[G][D]: the rotation q~ = Rot q without its 1/sqrt(d) factor, which the
-// caller applies.  One warp per row; all consumer threads call it, and it
-// ends with a consumer barrier.
+// caller applies.  qrows: the head's G bf16 rows if already in shared memory,
+// else null (read from p.q).  One warp per row; all consumer threads call
+// it, and it ends with a consumer barrier.
 template <int D, int G>
 __device__ __forceinline__ void load_rotate_queries(const DecodeParams& p, long long hd,
-                                                    float* qs, float* qt, int tid) {
+                                                    float* qs, float* qt, int tid,
+                                                    const uint16_t* qrows = nullptr) {
   constexpr int E = D / 32;
   const int b = (int)(hd / p.kv_heads);
   const int h = (int)(hd % p.kv_heads);
   const int warp = tid >> 5, lane = tid & 31;
   named_bar_sync(1, kConsumerThreads);          // previous users of the buffers done
+  const uint16_t* qbase = qrows ? qrows : p.q + ((size_t)b * p.q_heads + (size_t)h * G) * D;
   for (int r = warp; r < G; r += kConsumerWarps) {
-    const uint16_t* qr = p.q + ((size_t)b * p.q_heads + (size_t)h * G + r) * D + lane * E;
+    const uint16_t* qr = qbase + (size_t)r * D + lane * E;
     float v[E];
 #pragma unroll
     for (int k = 0; k < E; ++k) {
@@ -139,9 +142,11 @@ __device__ __forceinline__ void finish_head(const DecodeParams& p, long long hd,
       out_rec[q == 1 ? 1 : q + 2] = acc;   // l at 1; accRef/accRes from 4
     }
   }
-  __threadfence();
-  named_bar_sync(1, kConsumerThreads);
+  named_bar_sync(1, kConsumerThreads);      // every record store of the CTA issued
   if (tid == 0) {
+    // the barrier orders the other threads' record stores before this fence,
+    // which makes them visible at GPU scope before the ticket (cumulativity)
+    __threadfence();
     const uint32_t old = atomicAdd(&p.counters[hd], 1u);
     const int last = (old == (uint32_t)(ncontrib - 1));
     if (last) {
@@ -162,17 +167,28 @@ __device__ __forceinline__ void finish_head(const DecodeParams& p, long long hd,
   float* tsc = arow + G;             // [G][n_tail] tail scores, then weights
   for (int eidx = tid; eidx < G * D; eidx += kConsumerThreads) {
     const int r = eidx / D, i = eidx % D;
-    float M = kNegInf;
-    for (int c = 0; c < ncontrib; ++c)
-      M = fmaxf(M, __ldcg(recs + ((size_t)c * G + r) * (4 + 2 * D)));
-    float aref = 0.0f, ares = 0.0f, l = 0.0f;
+    // one pass with a running max: the loads of every record are independent
+    // of the combining, so they are all in flight together
+    float M = kNegInf, aref = 0.0f, ares = 0.0f, l = 0.0f;
+#pragma unroll 4
     for (int c = 0; c < ncontrib; ++c) {
       const float* rc = recs + ((size_t)c * G + r) * (4 + 2 * D);
       const float mc = __ldcg(rc);
-      const float wt = (mc == kNegInf) ? 0.0f : exp2f(mc - M);
-      l += wt * __ldcg(rc + 1);
-      aref += wt * __ldcg(rc + 4 + i);
-      if constexpr (RES) ares += wt * __ldcg(rc + 4 + D + i);
+      const float lc = __ldcg(rc + 1);
+      const float ac = __ldcg(rc + 4 + i);
+      const float rcv = RES ? __ldcg(rc + 4 + D + i) : 0.0f;
+      if (mc == kNegInf) continue;
+      if (mc > M) {
+        const float sc = (M == kNegInf) ? 0.0f : exp2f(M - mc);
+        l *= sc;
+        aref *= sc;
+        ares *= sc;
+        M = mc;
+      }
+      const float wt = exp2f(mc - M);
+      l = fmaf(wt, lc, l);
+      aref = fmaf(wt, ac, aref);
+      if constexpr (RES) ares = fmaf(wt, rcv, ares);
     }
     zref[eidx] = aref;
     zres[eidx] = ares;
