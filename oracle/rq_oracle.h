@@ -15,7 +15,8 @@
  * down to INT2 with a least-squares scale, and the bit width may differ per
  * loop.  Everything finer than that (the Walsh-Hadamard rotation, the code
  * grid, the rounding rule, the group size, the packing) is a reading of the
- * pages that is written down in DESIGN.md, section "Readings".
+ * pages; each is stated below where the function that implements it is
+ * declared.
  *
  * Two levels:
  *   - the fp32 exact-spec path (orq_*_f32): the encoder step by step, in
