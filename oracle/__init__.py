@@ -73,6 +73,19 @@ def lib():
                                                c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p,
                                                f64p]
         L.orq_decode_attention_f64.restype = c.c_int
+        i32p = np.ctypeslib.ndpointer(np.int32, flags="C_CONTIGUOUS")
+        L.orq_ls_dot_f32.argtypes = [c.c_int, f32p, i32p]
+        L.orq_ls_dot_f32.restype = c.c_float
+        L.orq_quantize_group_refined_f32.argtypes = [c.c_int, c.c_int, f32p, c.c_int, u8p,
+                                                     c.POINTER(c.c_float),
+                                                     c.POINTER(c.c_uint16)]
+        L.orq_quantize_group_refined_f32.restype = None
+        L.orq_encode_rows_refined_f32.argtypes = [c.c_long, c.c_int, c.c_int, c.c_int,
+                                                  c.c_uint64, c.c_int, u16p, u16p, u32p, u16p]
+        L.orq_encode_rows_refined_f32.restype = None
+        L.orq_quantize_group_refined_f64.argtypes = [c.c_int, c.c_int, f64p, c.c_int, u8p,
+                                                     c.POINTER(c.c_double), f64p]
+        L.orq_quantize_group_refined_f64.restype = c.c_int
         _lib = L
     return _lib
 
@@ -190,6 +203,49 @@ def encode_rows_f32(x, ref, bits, group, seed):
     scales = np.empty(x.shape[:-1] + (d // group,), dtype=np.uint16)
     ties = lib().orq_encode_rows_f32(n, d, group, bits, seed, x, ref, words, scales)
     return words, scales, int(ties)
+
+
+def ls_dot_f32(y, lvl):
+    """<y, l> in the refinement's fixed binary32 order."""
+    y = np.ascontiguousarray(y, dtype=np.float32)
+    lvl = np.ascontiguousarray(lvl, dtype=np.int32)
+    return float(lib().orq_ls_dot_f32(y.size, y, lvl))
+
+
+def quantize_group_refined_f32(y, bits, iters):
+    """Alternating refits of one group (fp32 spec).  Returns (codes, s_f32, s_f16)."""
+    y = np.ascontiguousarray(y, dtype=np.float32)
+    codes = np.empty(y.size, dtype=np.uint8)
+    sv = ctypes.c_float(0.0)
+    h = ctypes.c_uint16(0)
+    lib().orq_quantize_group_refined_f32(y.size, bits, y, iters, codes, ctypes.byref(sv),
+                                         ctypes.byref(h))
+    return codes, sv.value, h.value
+
+
+def quantize_group_refined_f64(y, bits, iters):
+    """The refits in double.  Returns (codes, s, err[0..done], done)."""
+    y = np.ascontiguousarray(y, dtype=np.float64)
+    codes = np.empty(y.size, dtype=np.uint8)
+    sv = ctypes.c_double(0.0)
+    err = np.zeros(iters + 1, dtype=np.float64)
+    done = lib().orq_quantize_group_refined_f64(y.size, bits, y, iters, codes,
+                                                ctypes.byref(sv), err)
+    return codes, sv.value, err[:done + 1], done
+
+
+def encode_rows_refined_f32(x, ref, bits, group, seed, iters):
+    """fp32 spec encode with `iters` least-squares refits per group.
+    Returns (words, scales)."""
+    x = _u16(x)
+    ref = _u16(ref)
+    assert x.shape == ref.shape
+    d = x.shape[-1]
+    n = int(np.prod(x.shape[:-1])) if x.ndim > 1 else 1
+    words = np.empty(x.shape[:-1] + ((d * bits + 31) // 32,), dtype=np.uint32)
+    scales = np.empty(x.shape[:-1] + (d // group,), dtype=np.uint16)
+    lib().orq_encode_rows_refined_f32(n, d, group, bits, seed, iters, x, ref, words, scales)
+    return words, scales
 
 
 def encode_row_f64(x, ref, bits, group, seed):

@@ -258,6 +258,164 @@ long orq_encode_rows_f32(long n_rows, int d, int g, int bits, uint64_t seed,
     return ties;
 }
 
+/* ------------------------------------------------------------------------ */
+/* least-squares refinement                                                  */
+/* ------------------------------------------------------------------------ */
+
+float orq_ls_dot_f32(int g, const float *y, const int *lvl)
+{
+    if (g < 32) {                       /* a single chain */
+        float acc = 0.0f;
+        for (int i = 0; i < g; ++i)
+            acc = fmaf(y[i], (float)lvl[i], acc);
+        return acc;
+    }
+    float total = 0.0f;
+    for (int b = 0; b < g / 32; ++b) {
+        float run[2];
+        for (int h = 0; h < 2; ++h) {
+            float acc = 0.0f;
+            for (int i = 0; i < 16; ++i) {
+                const int j = 32 * b + 16 * h + i;
+                acc = fmaf(y[j], (float)lvl[j], acc);
+            }
+            run[h] = acc;
+        }
+        const float blk = run[0] + run[1];
+        total = (b == 0) ? blk : total + blk;
+    }
+    return total;
+}
+
+/* codes of one group for the step 1 / (2 inv): nearest odd level, ties up */
+static void quantize_with_inv_f32(int g, int bits, const float *y, float inv,
+                                  uint8_t *codes, int *lvl)
+{
+    const int nlev = 1 << bits;
+    const int half = 1 << (bits - 1);
+    for (int i = 0; i < g; ++i) {
+        float fl = floorf(y[i] * inv);
+        if (fl < (float)-half)
+            fl = (float)-half;
+        if (fl > (float)(half - 1))
+            fl = (float)(half - 1);
+        const int c = (int)fl + half;
+        codes[i] = (uint8_t)c;
+        lvl[i] = 2 * c - (nlev - 1);
+    }
+}
+
+static float ls_scale_f32(int g, const float *y, const int *lvl)
+{
+    int nrm = 0;
+    for (int i = 0; i < g; ++i)
+        nrm += lvl[i] * lvl[i];
+    return orq_ls_dot_f32(g, y, lvl) / (float)nrm;
+}
+
+void orq_quantize_group_refined_f32(int g, int bits, const float *y, int iters,
+                                    uint8_t *codes, float *s_out, uint16_t *s_f16)
+{
+    const int half = 1 << (bits - 1);
+    int lvl[ORQ_MAX_D];
+    float amax = 0.0f;
+    for (int i = 0; i < g; ++i) {
+        const float a = fabsf(y[i]);
+        if (a > amax)
+            amax = a;
+    }
+    const float outer = (float)half - 0.5f;
+    const float inv0 = (amax < FLT_MIN) ? 0.0f : outer / amax;
+    quantize_with_inv_f32(g, bits, y, inv0, codes, lvl);
+    float s = ls_scale_f32(g, y, lvl);
+    for (int k = 0; k < iters; ++k) {
+        if (!(s >= FLT_MIN))
+            break;
+        quantize_with_inv_f32(g, bits, y, 0.5f / s, codes, lvl);
+        s = ls_scale_f32(g, y, lvl);
+    }
+    if (s > 65504.0f)
+        s = 65504.0f;
+    if (s < -65504.0f)
+        s = -65504.0f;
+    if (s_out)
+        *s_out = s;
+    *s_f16 = orq_f64_to_f16((double)s);
+}
+
+void orq_encode_row_refined_f32(int d, int g, int bits, const int8_t *D, int iters,
+                                const uint16_t *x, const uint16_t *ref,
+                                uint32_t *words, uint16_t *scales)
+{
+    float r[ORQ_MAX_D], y[ORQ_MAX_D];
+    uint8_t c[ORQ_MAX_D];
+    for (int i = 0; i < d; ++i)
+        r[i] = orq_bf16_to_f32(x[i]) - orq_bf16_to_f32(ref[i]);
+    orq_rotate_f32(d, D, r, y);
+    for (int k = 0; k < d / g; ++k)
+        orq_quantize_group_refined_f32(g, bits, y + k * g, iters, c + k * g, NULL, scales + k);
+    orq_pack_codes(d, bits, c, words);
+}
+
+void orq_encode_rows_refined_f32(long n_rows, int d, int g, int bits, uint64_t seed,
+                                 int iters, const uint16_t *x, const uint16_t *ref,
+                                 uint32_t *words, uint16_t *scales)
+{
+    int8_t D[ORQ_MAX_D];
+    orq_signs(seed, d, D);
+    const int wpr = (d * bits + 31) / 32;
+    for (long row = 0; row < n_rows; ++row)
+        orq_encode_row_refined_f32(d, g, bits, D, iters, x + row * d, ref + row * d,
+                                   words + row * wpr, scales + row * (d / g));
+}
+
+int orq_quantize_group_refined_f64(int g, int bits, const double *y, int iters,
+                                   uint8_t *codes, double *s_out, double *err)
+{
+    const int nlev = 1 << bits;
+    const int half = 1 << (bits - 1);
+    double amax = 0.0;
+    for (int i = 0; i < g; ++i)
+        if (fabs(y[i]) > amax)
+            amax = fabs(y[i]);
+    double inv = (amax < (double)FLT_MIN) ? 0.0 : ((double)half - 0.5) / amax;
+    double s = 0.0;
+    int done = 0;
+    for (int k = 0; k <= iters; ++k) {
+        if (k > 0) {
+            if (!(s >= (double)FLT_MIN))
+                break;
+            inv = 0.5 / s;
+            ++done;
+        }
+        double num = 0.0, den = 0.0;
+        for (int i = 0; i < g; ++i) {
+            double fl = floor(y[i] * inv);
+            if (fl < -half)
+                fl = -half;
+            if (fl > half - 1)
+                fl = half - 1;
+            const int c = (int)fl + half;
+            codes[i] = (uint8_t)c;
+            const int l = 2 * c - (nlev - 1);
+            num += y[i] * l;
+            den += (double)(l * l);
+        }
+        s = num / den;
+        if (err) {
+            double e = 0.0;
+            for (int i = 0; i < g; ++i) {
+                const double dv = y[i] - s * (2 * codes[i] - (nlev - 1));
+                e += dv * dv;
+            }
+            err[k] = e;
+        }
+    }
+    if (s_out)
+        *s_out = s;
+    return done;
+}
+
 /* fp64 definitional encoder: y = R r with the explicit matrix, the same code
  * rule evaluated in double, and the least-squares scale in double. */
 void orq_encode_row_f64(int d, int g, int bits, const int8_t *D,

@@ -85,6 +85,34 @@ void orq_encode_row_f64(int d, int g, int bits, const int8_t *D,
                         const uint16_t *x, const uint16_t *ref,
                         uint8_t *codes, double *scales, double *bdist);
 
+/* ---- least-squares refinement (alternating code / scale refits) --------- */
+/* Reading of the pages' "least-squares scaling" taken one step further, as
+ * alternating refits: from the absmax codes and their least-squares scale
+ * s_0, each refit k = 1..iters re-quantises every coordinate to the nearest
+ * level of the current scale (inv = RN(0.5 / s), c = clamp(floor(RN(y inv))
+ * + 2^(b-1), 0, 2^b - 1), ties to the upper level) and refits
+ * s = <y,l>/<l,l>.  Refits stop early if s falls below FLT_MIN.  Because each
+ * scale decides the next codes, the binary32 order of <y,l> is fixed: fused
+ * multiply-add chains over runs of 16 consecutive coordinates (first to last,
+ * from 0), the two runs of each 32-coordinate block added, then the blocks
+ * added in order (a group shorter than 32 is a single chain).  Scales stay in
+ * binary32 between refits; the stored scale is the last one, clamped to
+ * +-65504 and rounded to fp16. */
+float orq_ls_dot_f32(int g, const float *y, const int *lvl);
+void orq_quantize_group_refined_f32(int g, int bits, const float *y, int iters,
+                                    uint8_t *codes, float *s_out, uint16_t *s_f16);
+void orq_encode_row_refined_f32(int d, int g, int bits, const int8_t *D, int iters,
+                                const uint16_t *x, const uint16_t *ref,
+                                uint32_t *words, uint16_t *scales);
+void orq_encode_rows_refined_f32(long n_rows, int d, int g, int bits, uint64_t seed,
+                                 int iters, const uint16_t *x, const uint16_t *ref,
+                                 uint32_t *words, uint16_t *scales);
+/* The same refits in double on given rotated coordinates y; err[k] receives
+ * ||y - s_k l_k||^2 after refit k (err[0]: the absmax codes with s_0), so
+ * err has iters + 1 entries.  Returns the number of refits done. */
+int orq_quantize_group_refined_f64(int g, int bits, const double *y, int iters,
+                                   uint8_t *codes, double *s_out, double *err);
+
 /* ---- reconstruction and attention (fp64 definitional) ------------------- */
 /* out[d] = f64(ref) + Rot^T (s16 * level), for one row. bits==16 => ref. */
 void orq_reconstruct_row_f64(int d, int g, int bits, const int8_t *D,

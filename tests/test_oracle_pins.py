@@ -377,3 +377,101 @@ def test_residual_loop_decode_is_attention_over_reconstruction(bits):
                     oracle.bf16_to_f32(xv).astype(np.float64), 1 / math.sqrt(d))
     err = np.abs(out - exact).max()
     assert 0 < err < 0.5
+
+
+# ---------------------------------------------------------------------------
+# least-squares refinement (alternating code / scale refits)
+# ---------------------------------------------------------------------------
+
+def _levels(codes, bits):
+    return 2 * codes.astype(np.int64) - ((1 << bits) - 1)
+
+
+def test_refinement_worked_example(golden):
+    # hand-derived in tests/golden/ls_refinement_g8.txt
+    g = golden("ls_refinement_g8.txt")
+    y = np.array([float(v) for v in g["y"].split()], dtype=np.float32)
+    for it, ck, sk in ((0, "codes0", "s0"), (1, "codes1", "s1"), (2, "codes2", "s2")):
+        codes, s32, _ = oracle.quantize_group_refined_f32(y, 2, it)
+        assert codes.tolist() == [int(v) for v in g[ck].split()]
+        assert abs(s32 - float(g[sk])) <= 1e-6
+        c64, s64, err, done = oracle.quantize_group_refined_f64(y.astype(np.float64), 2, it)
+        assert c64.tolist() == codes.tolist()
+    _, _, err, _ = oracle.quantize_group_refined_f64(y.astype(np.float64), 2, 1)
+    assert abs(err[0] - float(g["err0"])) < 1e-3 and abs(err[1] - float(g["err1"])) < 1e-3
+
+
+@pytest.mark.parametrize("bits,group", [(2, 32), (2, 64), (4, 32), (4, 64)])
+def test_refinement_error_never_increases(bits, group):
+    # nearest-level codes minimise the error for a fixed scale, and the
+    # least-squares scale minimises it for fixed codes: the error of the
+    # alternation can only go down
+    rng = np.random.default_rng(100 + bits + group)
+    for trial in range(300):
+        kind = trial % 3
+        if kind == 0:
+            y = rng.standard_normal(group)
+        elif kind == 1:
+            y = rng.laplace(size=group)
+        else:
+            y = rng.standard_normal(group) * 0.1
+            y[rng.integers(group)] = 5.0          # one outlier sets the absmax
+        _, _, err, done = oracle.quantize_group_refined_f64(y, bits, 8)
+        assert np.all(np.diff(err) <= 1e-12 * err[0]), (trial, err)
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_refit_codes_are_the_nearest_levels(bits):
+    # brute force over every level, independent of the floor rule
+    rng = np.random.default_rng(7 + bits)
+    top = (1 << bits) - 1
+    all_levels = np.arange(-top, top + 1, 2)
+    for _ in range(200):
+        y = rng.standard_normal(32)
+        _, s0, _, _ = oracle.quantize_group_refined_f64(y, bits, 0)
+        c1, _, _, _ = oracle.quantize_group_refined_f64(y, bits, 1)
+        best = all_levels[np.argmin(np.abs(y[:, None] - s0 * all_levels[None, :]), axis=1)]
+        assert np.array_equal(_levels(c1, bits), best)
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_refinement_fixed_point_on_an_exact_grid(bits):
+    # y = s l with s a power of two and levels that include the outermost:
+    # every quantity is exact, the first step already lands on the grid and
+    # no refit moves it
+    rng = np.random.default_rng(3)
+    top = (1 << bits) - 1
+    lv = rng.choice(np.arange(-top, top + 1, 2), size=32)
+    lv[5] = top
+    y = (0.25 * lv).astype(np.float32)
+    for it in (0, 1, 4):
+        codes, s32, h = oracle.quantize_group_refined_f32(y, bits, it)
+        assert np.array_equal(_levels(codes, bits), lv)
+        assert s32 == 0.25 and oracle.f16_to_f64(h) == 0.25
+
+
+@pytest.mark.parametrize("bits,group", [(2, 32), (4, 64)])
+def test_zero_refits_keep_the_unrefined_codes(bits, group):
+    rng = np.random.default_rng(11)
+    for _ in range(100):
+        y = rng.standard_normal(group).astype(np.float32)
+        c_ref, _, s_ref, _ = oracle.quantize_group_f32(y, bits)
+        codes, _, h = oracle.quantize_group_refined_f32(y, bits, 0)
+        assert np.array_equal(codes, c_ref)
+        a, b = oracle.f16_to_f64(h), oracle.f16_to_f64(s_ref)
+        assert abs(a - b) <= 1e-3 * abs(b) + 2.0 ** -24
+
+
+def test_fixed_order_dot_within_its_rounding_bound():
+    rng = np.random.default_rng(5)
+    for g in (8, 32, 64):
+        for _ in range(100):
+            y = rng.standard_normal(g).astype(np.float32)
+            lv = rng.choice([-3, -1, 1, 3], size=g)
+            exact = float(np.sum(y.astype(np.float64) * lv))
+            got = oracle.ls_dot_f32(y, lv)
+            bound = g * 2.0 ** -23 * float(np.sum(np.abs(y.astype(np.float64) * lv)))
+            assert abs(got - exact) <= bound
+        yi = rng.integers(-50, 50, size=g).astype(np.float32)     # all sums exact
+        lv = rng.choice([-3, -1, 1, 3], size=g)
+        assert oracle.ls_dot_f32(yi, lv) == float(np.sum(yi.astype(np.int64) * lv))
