@@ -166,6 +166,33 @@ rq_status rq_encode_at(const rq_shape *shape, int src_pitch, int src_offset, int
                        uint32_t *const *codes_out, uint16_t *const *scales_out,
                        uint16_t *ref_out, void *stream);
 
+/* Most least-squares refits rq_encode_at_ex accepts. */
+#define RQ_MAX_REFINE 8
+
+/*
+ * rq_encode_at_ex -- rq_encode_at with least-squares refinement (the pages'
+ * least-squares scaling, iterated: ResidualQuant page, Abstract).
+ *
+ * refine_iters (0 .. RQ_MAX_REFINE): after the absmax codes and their
+ * least-squares scale s, each refit re-quantises every coordinate of the
+ * group to the nearest level of the current scale (step 2s: inv = RN(0.5/s),
+ * c = clamp(floor(RN(y inv)) + 2^(b-1), 0, 2^b - 1), ties to the upper
+ * level) and refits s = <y,l>/<l,l>; a group whose scale is below FLT_MIN
+ * keeps its codes.  <y,l> is summed in a fixed binary32 order (fma chains
+ * over runs of 16 coordinates, the runs of each 32-block added, then the
+ * blocks), so codes and scales are reproducible bit for bit.  The error
+ * ||y - s l|| never increases from one refit to the next.  The stored
+ * format is unchanged: every decoder reads the refined codes as any others.
+ * refine_iters = 0 is rq_encode_at.  Other arguments and errors as
+ * rq_encode_at; a refine_iters outside 0 .. RQ_MAX_REFINE is
+ * RQ_ERR_INVALID_ARG.
+ */
+rq_status rq_encode_at_ex(const rq_shape *shape, int src_pitch, int src_offset,
+                          int dst_pitch, int dst_offset, const uint16_t *const *kv_loops,
+                          int n_loops, const uint16_t *ref, const uint8_t *bits_per_loop,
+                          uint64_t seed, int refine_iters, uint32_t *const *codes_out,
+                          uint16_t *const *scales_out, uint16_t *ref_out, void *stream);
+
 /*
  * rq_decode_attention -- fused ResidualQuant decode attention for one loop
  * (Abstract: the reconstruction stays efficient; the reduced KV traffic is

@@ -11,7 +11,7 @@ from ._abi import (RQ_ERR_ALIGNMENT, RQ_ERR_CUDA, RQ_ERR_INVALID_ARG, RQ_ERR_UNS
                    RQ_ERR_WORKSPACE, RQ_MAX_LOOPS, RQ_OK, RqError, lib, make_shape,
                    rq_codes_bytes, rq_decode_attention, rq_decode_attention_noalloc,
                    rq_decode_attention_tail, rq_decode_workspace_bytes, rq_encode, rq_encode_at,
-                   rq_encode_take_status, rq_reconstruct,
+                   rq_encode_at_ex, rq_encode_take_status, rq_reconstruct, RQ_MAX_REFINE,
                    rq_scales_bytes, rq_shape, rq_status_string, rq_version,
                    rq_workspace_status)
 
@@ -19,7 +19,7 @@ __all__ = [
     "RQ_OK", "RQ_ERR_INVALID_ARG", "RQ_ERR_UNSUPPORTED", "RQ_ERR_ALIGNMENT", "RQ_ERR_WORKSPACE",
     "RQ_ERR_CUDA", "RQ_MAX_LOOPS", "RqError", "lib", "rq_shape", "make_shape", "rq_version",
     "rq_status_string", "rq_codes_bytes", "rq_scales_bytes", "rq_decode_workspace_bytes",
-    "rq_encode", "rq_encode_at", "rq_decode_attention", "rq_decode_attention_tail",
+    "rq_encode", "rq_encode_at", "rq_encode_at_ex", "RQ_MAX_REFINE", "rq_decode_attention", "rq_decode_attention_tail",
     "rq_decode_attention_noalloc", "rq_reconstruct", "rq_workspace_status", "rq_encode_take_status",
     "alloc_codes", "alloc_scales", "alloc_workspace", "encode", "decode_attention", "reconstruct",
 ]
@@ -47,8 +47,9 @@ def alloc_workspace(shape, device="cuda"):
     return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
-def encode(kv_loops, ref, bits_per_loop, group, seed, stream=None):
-    """Encode non-final loops (bf16 tensors [rows, Hkv, T, d]) against `ref`.
+def encode(kv_loops, ref, bits_per_loop, group, seed, stream=None, refine_iters=0):
+    """Encode non-final loops (bf16 tensors [rows, Hkv, T, d]) against `ref`,
+    with `refine_iters` least-squares refits per group.
 
     Returns (codes, scales): per loop a uint8 device buffer, or None for a
     loop kept in BF16 (bits 16)."""
@@ -56,7 +57,11 @@ def encode(kv_loops, ref, bits_per_loop, group, seed, stream=None):
     shape = make_shape(rows, hkv, t, d, group)
     codes = [alloc_codes(shape, b, ref.device) for b in bits_per_loop]
     scales = [alloc_scales(shape, b, ref.device) for b in bits_per_loop]
-    rq_encode(shape, kv_loops, ref, bits_per_loop, seed, codes, scales, stream)
+    if refine_iters:
+        rq_encode_at_ex(shape, t, 0, t, 0, kv_loops, ref, bits_per_loop, seed, refine_iters,
+                        codes, scales, stream=stream)
+    else:
+        rq_encode(shape, kv_loops, ref, bits_per_loop, seed, codes, scales, stream)
     return codes, scales
 
 

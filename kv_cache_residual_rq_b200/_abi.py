@@ -19,6 +19,7 @@ RQ_ERR_ALIGNMENT = 3
 RQ_ERR_WORKSPACE = 4
 RQ_ERR_CUDA = 5
 RQ_MAX_LOOPS = 16
+RQ_MAX_REFINE = 8
 
 
 class RqError(RuntimeError):
@@ -79,6 +80,12 @@ def lib():
                                    c.POINTER(c.c_uint8), c.c_uint64, c.POINTER(c.c_void_p),
                                    c.POINTER(c.c_void_p), c.c_void_p, c.c_void_p]
         L.rq_encode_at.restype = c.c_int
+        L.rq_encode_at_ex.argtypes = [sp, c.c_int, c.c_int, c.c_int, c.c_int,
+                                      c.POINTER(c.c_void_p), c.c_int, c.c_void_p,
+                                      c.POINTER(c.c_uint8), c.c_uint64, c.c_int,
+                                      c.POINTER(c.c_void_p), c.POINTER(c.c_void_p), c.c_void_p,
+                                      c.c_void_p]
+        L.rq_encode_at_ex.restype = c.c_int
         L.rq_decode_attention_tail.argtypes = [sp, c.c_void_p, c.c_void_p, c.c_void_p,
                                                c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p,
                                                c.c_int, c.c_uint64, c.c_float, c.c_void_p,
@@ -177,6 +184,21 @@ def rq_encode_at(shape, src_pitch, src_offset, dst_pitch, dst_offset, kv_loops, 
                             _ptr(ref_out), _stream(stream))
     if check:
         _check(st, "rq_encode_at")
+    return st
+
+
+def rq_encode_at_ex(shape, src_pitch, src_offset, dst_pitch, dst_offset, kv_loops, ref,
+                    bits_per_loop, seed, refine_iters, codes_out, scales_out, ref_out=None,
+                    stream=None, check=True):
+    n = len(bits_per_loop)
+    ptrs = lambda seq: (ctypes.c_void_p * max(n, 1))(*[_ptr(v) for v in seq])
+    bits = (ctypes.c_uint8 * max(n, 1))(*[int(b) for b in bits_per_loop])
+    st = lib().rq_encode_at_ex(_shp(shape), int(src_pitch), int(src_offset), int(dst_pitch),
+                               int(dst_offset), ptrs(kv_loops), n, _ptr(ref), bits,
+                               ctypes.c_uint64(seed), int(refine_iters), ptrs(codes_out),
+                               ptrs(scales_out), _ptr(ref_out), _stream(stream))
+    if check:
+        _check(st, "rq_encode_at_ex")
     return st
 
 

@@ -119,13 +119,14 @@ size_t rq_decode_workspace_bytes(const rq_shape* shape) {
   return decode_workspace_bytes(*shape);
 }
 
-rq_status rq_encode_at(const rq_shape* shape, int src_pitch, int src_offset, int dst_pitch,
-                       int dst_offset, const uint16_t* const* kv_loops, int n_loops,
-                       const uint16_t* ref, const uint8_t* bits_per_loop, uint64_t seed,
-                       uint32_t* const* codes_out, uint16_t* const* scales_out,
-                       uint16_t* ref_out, void* stream) {
+rq_status rq_encode_at_ex(const rq_shape* shape, int src_pitch, int src_offset,
+                          int dst_pitch, int dst_offset, const uint16_t* const* kv_loops,
+                          int n_loops, const uint16_t* ref, const uint8_t* bits_per_loop,
+                          uint64_t seed, int refine_iters, uint32_t* const* codes_out,
+                          uint16_t* const* scales_out, uint16_t* ref_out, void* stream) {
   if (!shape || !kv_loops || !bits_per_loop || !codes_out || !scales_out)
     return RQ_ERR_INVALID_ARG;
+  if (refine_iters < 0 || refine_iters > RQ_MAX_REFINE) return RQ_ERR_INVALID_ARG;
   if (shape->batch < 1 || shape->kv_heads < 1 || shape->ctx < 0) return RQ_ERR_INVALID_ARG;
   if (src_offset < 0 || dst_offset < 0 || src_pitch < 1 || dst_pitch < 1 ||
       (long long)src_offset + shape->ctx > src_pitch ||
@@ -154,6 +155,7 @@ rq_status rq_encode_at(const rq_shape* shape, int src_pitch, int src_offset, int
   p.ref = ref;
   p.ref_out = ref_out;
   p.n_loops = n_loops;
+  p.refine_iters = refine_iters;
   p.seed = seed;
   p.ctx = shape->ctx;
   p.src_pitch = src_pitch;
@@ -171,6 +173,15 @@ rq_status rq_encode_at(const rq_shape* shape, int src_pitch, int src_offset, int
                              : launch_encode(shape->head_dim, shape->group, p, sms,
                                              static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? RQ_OK : RQ_ERR_CUDA;
+}
+
+rq_status rq_encode_at(const rq_shape* shape, int src_pitch, int src_offset, int dst_pitch,
+                       int dst_offset, const uint16_t* const* kv_loops, int n_loops,
+                       const uint16_t* ref, const uint8_t* bits_per_loop, uint64_t seed,
+                       uint32_t* const* codes_out, uint16_t* const* scales_out,
+                       uint16_t* ref_out, void* stream) {
+  return rq_encode_at_ex(shape, src_pitch, src_offset, dst_pitch, dst_offset, kv_loops, n_loops,
+                         ref, bits_per_loop, seed, 0, codes_out, scales_out, ref_out, stream);
 }
 
 rq_status rq_encode(const rq_shape* shape, const uint16_t* const* kv_loops, int n_loops,

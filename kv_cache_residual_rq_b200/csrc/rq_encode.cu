@@ -125,25 +125,75 @@ encode_kernel(const EncodeParams p) {
         const float outer = (float)half - 0.5f;
         const float inv = (amax < 1.17549435e-38f) ? 0.0f : __fdiv_rn(outer, amax);
 
-        uint32_t packed = 0;
-        float dot = 0.0f;
-        int nrm = 0;
+        // one quantisation pass with step 1/(2 iv): codes (clamped), the
+        // lane's levels, and <l,l> of the group
+        float lvl[DPL];
+        auto pass = [&](float iv, uint32_t& packed, int& nrm) {
+          packed = 0;
+          nrm = 0;
 #pragma unroll
-        for (int k = 0; k < DPL; ++k) {
-          const float u = __fmul_rn(v[k], inv);
-          int c = __float2int_rd(u) + half;       // floor(u) + 2^(b-1)
-          c = min(max(c, 0), top);
-          const int lvl = 2 * c - top;
-          dot = fmaf(v[k], (float)lvl, dot);
-          nrm += lvl * lvl;
-          packed |= (uint32_t)c << (bits * k);
-        }
+          for (int k = 0; k < DPL; ++k) {
+            const float u = __fmul_rn(v[k], iv);
+            int c = __float2int_rd(u) + half;     // floor(u) + 2^(b-1)
+            c = min(max(c, 0), top);
+            const int l2 = 2 * c - top;
+            lvl[k] = (float)l2;
+            nrm += l2 * l2;
+            packed |= (uint32_t)c << (bits * k);
+          }
 #pragma unroll
-        for (int m = 1; m < LPG; m <<= 1) {
-          dot += __shfl_xor_sync(FULL, dot, m);
-          nrm += __shfl_xor_sync(FULL, nrm, m);
+          for (int m = 1; m < LPG; m <<= 1) nrm += __shfl_xor_sync(FULL, nrm, m);
+        };
+        // <y,l> of the group in the order that refits depend on: fma chains
+        // over runs of 16 coordinates (lanes 2j, 2j+1: the odd lane continues
+        // its even neighbour's chain), the two runs of each 32-block added,
+        // then the blocks of a 64-group added; the total is broadcast from
+        // the group's last lane
+        auto fixed_dot = [&]() {
+          float a = 0.0f;
+#pragma unroll
+          for (int k = 0; k < DPL; ++k) a = fmaf(v[k], lvl[k], a);
+          const float prev = __shfl_up_sync(FULL, a, 1);
+          if (li & 1) {
+            a = prev;
+#pragma unroll
+            for (int k = 0; k < DPL; ++k) a = fmaf(v[k], lvl[k], a);
+          }
+          const float run0 = __shfl_up_sync(FULL, a, 2);
+          float tot = ((li & 3) == 3) ? run0 + a : a;
+          if (GROUP == 64) {
+            const float blk0 = __shfl_up_sync(FULL, tot, 4);
+            if ((li & 7) == 7) tot = blk0 + tot;
+          }
+          return __shfl_sync(FULL, tot, lane | (LPG - 1));
+        };
+
+        uint32_t packed;
+        int nrm;
+        pass(inv, packed, nrm);
+        float dot;
+        if (p.refine_iters == 0) {
+          dot = 0.0f;
+#pragma unroll
+          for (int k = 0; k < DPL; ++k) dot = fmaf(v[k], lvl[k], dot);
+#pragma unroll
+          for (int m = 1; m < LPG; m <<= 1) dot += __shfl_xor_sync(FULL, dot, m);
+        } else {
+          dot = fixed_dot();
         }
         float s = dot / (float)nrm;               // least-squares scale
+        for (int it = 0; it < p.refine_iters; ++it) {
+          // refit: nearest level of the current scale, then the scale
+          const bool live = s >= 1.17549435e-38f;   // the same in every lane of the group
+          uint32_t packed2;
+          int nrm2;
+          pass(live ? __fdiv_rn(0.5f, s) : 0.0f, packed2, nrm2);
+          const float dot2 = fixed_dot();
+          if (live) {
+            packed = packed2;
+            s = dot2 / (float)nrm2;
+          }
+        }
         s = fminf(fmaxf(s, -65504.0f), 65504.0f);
 
         if (bits == 2) {

@@ -121,28 +121,29 @@ __device__ __forceinline__ void load_row(const uint8_t* slot, int r, int q, uint
   }
 }
 
-// codes and scale of one lane's 32 rotated coordinates P[m] = {y_m, y_{m+16}}
-template <int BITS, int GROUP, int RPW>
-__device__ __forceinline__ void quantize_store(const float2 (&P)[16], uint32_t* codes_row,
-                                               uint16_t* scales_row, int q, bool valid) {
-  float amax = 0.0f;
-#pragma unroll
-  for (int m = 0; m < 16; ++m) amax = fmax3_abs(amax, P[m].x, P[m].y);
-  if (GROUP == 64) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, RPW));
-  constexpr float outer = (float)(1 << (BITS - 1)) - 0.5f;
-  const float inv = (amax < 1.17549435e-38f) ? 0.0f : __fdiv_rn(outer, amax);
+// One quantisation pass of a lane's 32 rotated coordinates P[m] = {y_m,
+// y_{m+16}} with step 1/(2 inv): packed code words, <y,l> in the fixed order
+// (fma chains over coordinates 0..15 and 16..31, the two runs added; the
+// partner lane's block added for groups of 64) and <l,l> (exact).
+template <int BITS, int GROUP, int RPW, bool CLAMP>
+__device__ __forceinline__ void quant_pass(const float2 (&P)[16], float inv, uint32_t (&w)[BITS],
+                                           float& dot_out, float& nrm_out) {
   const float2 inv2 = make_float2(inv, inv);
   const float2 mg = make_float2(kFloorMagic, kFloorMagic);
   const float2 two = make_float2(2.0f, 2.0f), one = make_float2(1.0f, 1.0f);
+  constexpr float lo = kFloorMagic - (float)(1 << (BITS - 1));
+  constexpr float hi = kFloorMagic + (float)((1 << (BITS - 1)) - 1);
   float2 dot = make_float2(0.0f, 0.0f), nrm = make_float2(0.0f, 0.0f);
-  constexpr int NW = BITS;                          // words per lane (32 codes)
-  uint32_t w[NW];
 #pragma unroll
-  for (int k = 0; k < NW; ++k) w[k] = 0;
+  for (int k = 0; k < BITS; ++k) w[k] = 0;
 #pragma unroll
   for (int m = 0; m < 16; ++m) {
     const float2 u = __fmul2_rn(P[m], inv2);
-    const float2 t = __fadd2_rd(u, mg);             // 1.5*2^23 + floor(u), exact
+    float2 t = __fadd2_rd(u, mg);                   // 1.5*2^23 + floor(u), exact
+    if constexpr (CLAMP) {
+      t.x = fminf(fmaxf(t.x, lo), hi);
+      t.y = fminf(fmaxf(t.y, lo), hi);
+    }
     if constexpr (BITS == 2) {
       w[0] += __float_as_uint(t.x) << (2 * m);
       w[1] += __float_as_uint(t.y) << (2 * m);
@@ -159,7 +160,7 @@ __device__ __forceinline__ void quantize_store(const float2 (&P)[16], uint32_t* 
   constexpr uint32_t kOff = kFloorMagicBits - (1u << (BITS - 1));
   constexpr uint32_t kSpread = BITS == 2 ? 0x55555555u : 0x11111111u;
 #pragma unroll
-  for (int k = 0; k < NW; ++k) w[k] -= kOff * kSpread;
+  for (int k = 0; k < BITS; ++k) w[k] -= kOff * kSpread;
   float d = dot.x + dot.y, n;
   if constexpr (BITS == 2) {
     // <l, l> = 32 + 8 * (number of outer levels +-3, i.e. codes 0 and 3,
@@ -174,7 +175,39 @@ __device__ __forceinline__ void quantize_store(const float2 (&P)[16], uint32_t* 
     d += __shfl_xor_sync(kFull, d, RPW);
     n += __shfl_xor_sync(kFull, n, RPW);
   }
+  dot_out = d;
+  nrm_out = n;
+}
+
+// codes and scale of one lane's 32 rotated coordinates: the absmax step,
+// then `iters` least-squares refits (nearest level of the current scale,
+// then the scale refitted); a group whose scale is below FLT_MIN keeps its
+// codes.  The loop runs the same number of times in every lane.
+template <int BITS, int GROUP, int RPW>
+__device__ __forceinline__ void quantize_store(const float2 (&P)[16], uint32_t* codes_row,
+                                               uint16_t* scales_row, int q, bool valid,
+                                               int iters) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int m = 0; m < 16; ++m) amax = fmax3_abs(amax, P[m].x, P[m].y);
+  if (GROUP == 64) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, RPW));
+  constexpr float outer = (float)(1 << (BITS - 1)) - 0.5f;
+  const float inv = (amax < 1.17549435e-38f) ? 0.0f : __fdiv_rn(outer, amax);
+  uint32_t w[BITS];
+  float d, n;
+  quant_pass<BITS, GROUP, RPW, false>(P, inv, w, d, n);
   float s = d / n;                                  // least-squares scale
+  for (int k = 0; k < iters; ++k) {
+    const bool live = s >= 1.17549435e-38f;
+    uint32_t w2[BITS];
+    float d2, n2;
+    quant_pass<BITS, GROUP, RPW, true>(P, live ? __fdiv_rn(0.5f, s) : 0.0f, w2, d2, n2);
+    if (live) {
+#pragma unroll
+      for (int j = 0; j < BITS; ++j) w[j] = w2[j];
+      s = d2 / n2;
+    }
+  }
   s = fminf(fmaxf(s, -65504.0f), 65504.0f);
   if (!valid) return;
   if constexpr (BITS == 2)
@@ -357,10 +390,12 @@ encode_tma_kernel(const __grid_constant__ EncodeTmaParams tp) {
       const int l = tp.active[j];
       if (p.bits[l] == 2)
         quantize_store<2, GROUP, C::RPW>(P, p.codes[l] + (size_t)row * (D / 16),
-                                         p.scales[l] + (size_t)row * (D / GROUP), q, valid);
+                                         p.scales[l] + (size_t)row * (D / GROUP), q, valid,
+                                         p.refine_iters);
       else
         quantize_store<4, GROUP, C::RPW>(P, p.codes[l] + (size_t)row * (D / 8),
-                                         p.scales[l] + (size_t)row * (D / GROUP), q, valid);
+                                         p.scales[l] + (size_t)row * (D / GROUP), q, valid,
+                                         p.refine_iters);
     }
   }
 }

@@ -54,6 +54,7 @@ struct EncodeParams {
   int src_pitch, src_offset;         // token pitch / first token of the inputs
   int dst_pitch, dst_offset;         // token pitch / first token of the outputs
   int n_loops;
+  int refine_iters;                  // least-squares refits after the absmax codes
   uint64_t seed;
 };
 

@@ -76,6 +76,12 @@ def measure(w, reps, peak, emit):
     nb = encode_bytes(w, rows)
     emit({"workload": w.name, "kernel": "encode", "rows": rows, "loops": len(w.bits),
           "us": t * 1e6, "bytes": nb, "gbs": nb / t / 1e9, "frac": nb / t / 1e9 / peak})
+    for it in (1, 4):
+        t = _time(lambda: rq.encode(xk, refk, list(w.bits), w.group, w.seed, refine_iters=it),
+                  reps, flush)
+        emit({"workload": w.name, "kernel": f"encode refits={it}", "rows": rows,
+              "loops": len(w.bits), "us": t * 1e6, "bytes": nb, "gbs": nb / t / 1e9,
+              "frac": nb / t / 1e9 / peak})
     ck, sk = rq.encode(xk, refk, list(w.bits), w.group, w.seed)
     xv = [synth.loop_kv(w, 0, 1, l, refv) for l in range(1, w.loops)]
     cv, sv = rq.encode(xv, refv, list(w.bits), w.group, w.seed)

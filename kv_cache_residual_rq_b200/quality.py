@@ -9,6 +9,7 @@ compares the two encodings directly on the synthetic looped-KV data:
 
   ResidualQuant : the final loop kept in BF16, every other loop as its
                   rotated residual against it (rq_encode with the reference)
+  ResidualQuant with 4 least-squares refits (rq_encode_at_ex)
   rotation-only : every loop quantised on its own with the same rotation,
                   grid and least-squares scale (rq_encode with a zero
                   reference), at INT2 and INT4
@@ -49,18 +50,20 @@ def study(w, emit):
         for l in range(1, w.loops):
             x = synth.loop_kv(w, 0, kind, l, ref)
             xf = x.float()
-            schemes = [("residualquant", w.bits[l - 1], ref)]
-            schemes += [(f"rotation_only_int{b}", b, zero) for b in (2, 4)]
-            for scheme, bits, base in schemes:
+            schemes = [("residualquant", w.bits[l - 1], ref, 0),
+                       ("residualquant_ls4", w.bits[l - 1], ref, 4)]
+            schemes += [(f"rotation_only_int{b}", b, zero, 0) for b in (2, 4)]
+            for scheme, bits, base, it in schemes:
                 if bits == 16:
                     continue
-                (c,), (s,) = rq.encode([x], base, [bits], w.group, w.seed)
+                (c,), (s,) = rq.encode([x], base, [bits], w.group, w.seed, refine_iters=it)
                 xh = rq.reconstruct(base, c, s, bits, w.group, w.seed)
                 rel = (torch.linalg.vector_norm(xh - xf) / torch.linalg.vector_norm(xf)).item()
                 emit({"workload": w.name, "tensor": name, "loop": l, "scheme": scheme,
                       "bits": bits, "rel_recon_err": rel,
                       "bits_per_position_all_loops": bits_per_position(
-                          w, "residualquant" if scheme == "residualquant" else "rot", bits)})
+                          w, "residualquant" if scheme.startswith("residualquant") else "rot",
+                          bits)})
                 del c, s, xh
             del x, xf
             torch.cuda.empty_cache()
@@ -73,13 +76,14 @@ def study(w, emit):
     exact = F.scaled_dot_product_attention(
         q.float().unsqueeze(2), xk.float().repeat_interleave(G, dim=1),
         xv.float().repeat_interleave(G, dim=1)).squeeze(2)
-    for scheme, bits, use_ref in (("residualquant", w.bits[0], True),
-                                  ("rotation_only_int2", 2, False),
-                                  ("rotation_only_int4", 4, False)):
+    for scheme, bits, use_ref, it in (("residualquant", w.bits[0], True, 0),
+                                      ("residualquant_ls4", w.bits[0], True, 4),
+                                      ("rotation_only_int2", 2, False, 0),
+                                      ("rotation_only_int4", 4, False, 0)):
         bk = refk if use_ref else torch.zeros_like(refk)
         bv = refv if use_ref else torch.zeros_like(refv)
-        (ck,), (sk,) = rq.encode([xk], bk, [bits], w.group, w.seed)
-        (cv,), (sv,) = rq.encode([xv], bv, [bits], w.group, w.seed)
+        (ck,), (sk,) = rq.encode([xk], bk, [bits], w.group, w.seed, refine_iters=it)
+        (cv,), (sv,) = rq.encode([xv], bv, [bits], w.group, w.seed, refine_iters=it)
         out = rq.decode_attention(q, bk, bv, ck, cv, sk, sv, bits, w.group, w.seed)
         err = (torch.linalg.vector_norm(out - exact) / torch.linalg.vector_norm(exact)).item()
         emit({"workload": w.name, "tensor": "attention(loop 1)", "scheme": scheme, "bits": bits,

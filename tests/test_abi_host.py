@@ -207,3 +207,15 @@ def test_reconstruct_rejects_bad_arguments_before_launch():
     assert rec(shape=rq.make_shape(2, 2, 10, 128, 32, ctx_cap=5)) == E.RQ_ERR_INVALID_ARG
     assert rec(scales=MISALIGNED) == E.RQ_ERR_ALIGNMENT
     assert rec(shape=rq.make_shape(2, 2, 0, 128, 32)) == E.RQ_OK      # nothing to rebuild
+
+
+def test_encode_at_ex_rejects_refits_out_of_range():
+    s = rq.make_shape(1, 2, 10, 128, 32)
+    call = lambda it: rq.rq_encode_at_ex(s, 10, 0, 10, 0, [FAKE], FAKE, [2], 0, it, [FAKE],
+                                         [FAKE], stream=0, check=False)
+    assert call(-1) == rq.RQ_ERR_INVALID_ARG
+    assert call(rq.RQ_MAX_REFINE + 1) == rq.RQ_ERR_INVALID_ARG
+    # in range but nothing to do (ctx 0) is fine without a device
+    z = rq.make_shape(1, 2, 0, 128, 32)
+    assert rq.rq_encode_at_ex(z, 1, 0, 1, 0, [FAKE], FAKE, [2], 0, rq.RQ_MAX_REFINE, [FAKE],
+                              [FAKE], stream=0, check=False) == rq.RQ_OK
