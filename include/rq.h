@@ -258,6 +258,44 @@ rq_status rq_decode_attention_tail(const rq_shape *shape, const uint16_t *q,
                                    int tail_pitch, float *out, void *workspace,
                                    size_t workspace_bytes, void *stream);
 
+/* Most sequences of one variable-length call. */
+#define RQ_MAX_VARLEN_BATCH 1024
+
+/*
+ * rq_decode_attention_varlen -- rq_decode_attention_tail for a batch whose
+ * sequences hold different numbers of cached tokens (continuous batching;
+ * the lengths live on the device, so one captured graph serves every step).
+ *
+ *   ctx_lens : DEVICE int32 [shape->batch], 4-byte aligned; sequence b
+ *              attends over its first ctx_lens[b] cached tokens (plus the
+ *              n_tail tail tokens).  Read by the kernel, so it may be written
+ *              by the preceding kernel of the stream.  A length outside
+ *              0 .. capacity is clamped and sets status bit 16; a sequence
+ *              with 0 cached tokens attends over its tail only (with no tail
+ *              its output is 0/0, NaN).
+ *   shape    : capacity per head = shape->ctx_cap (or shape->ctx when
+ *              ctx_cap is 0): the token pitch of ref_k/ref_v/codes/scales.
+ *              batch <= RQ_MAX_VARLEN_BATCH.
+ *   workspace: rq_decode_workspace_bytes_varlen(shape) bytes, zeroed once.
+ * The work is split evenly over the tokens actually present (computed on the
+ * device), not over the capacity.  Other arguments as rq_decode_attention_tail.
+ * Errors: RQ_ERR_INVALID_ARG for a null ctx_lens or batch above the limit,
+ * RQ_ERR_ALIGNMENT for a misaligned ctx_lens, else as the tail variant.
+ */
+rq_status rq_decode_attention_varlen(const rq_shape *shape, const int32_t *ctx_lens,
+                                     const uint16_t *q, const uint16_t *ref_k,
+                                     const uint16_t *ref_v, const uint32_t *codes_k,
+                                     const uint32_t *codes_v, const uint16_t *scales_k,
+                                     const uint16_t *scales_v, int bits, uint64_t seed,
+                                     float softmax_scale, const uint16_t *tail_k,
+                                     const uint16_t *tail_v, int n_tail, int tail_pitch,
+                                     float *out, void *workspace, size_t workspace_bytes,
+                                     void *stream);
+
+/* Workspace bytes for rq_decode_attention_varlen with this shape (any
+ * lengths up to the capacity); 0 if the shape is unsupported. */
+size_t rq_decode_workspace_bytes_varlen(const rq_shape *shape);
+
 /*
  * rq_decode_attention_noalloc -- rq_decode_attention without a workspace
  * argument, for callers that cannot allocate device memory (for example code

@@ -12,6 +12,8 @@ from ._abi import (RQ_ERR_ALIGNMENT, RQ_ERR_CUDA, RQ_ERR_INVALID_ARG, RQ_ERR_UNS
                    rq_codes_bytes, rq_decode_attention, rq_decode_attention_noalloc,
                    rq_decode_attention_tail, rq_decode_workspace_bytes, rq_encode, rq_encode_at,
                    rq_encode_at_ex, rq_encode_take_status, rq_reconstruct, RQ_MAX_REFINE,
+                   RQ_MAX_VARLEN_BATCH, rq_decode_attention_varlen,
+                   rq_decode_workspace_bytes_varlen,
                    rq_scales_bytes, rq_shape, rq_status_string, rq_version,
                    rq_workspace_status)
 
@@ -20,7 +22,8 @@ __all__ = [
     "RQ_ERR_CUDA", "RQ_MAX_LOOPS", "RqError", "lib", "rq_shape", "make_shape", "rq_version",
     "rq_status_string", "rq_codes_bytes", "rq_scales_bytes", "rq_decode_workspace_bytes",
     "rq_encode", "rq_encode_at", "rq_encode_at_ex", "RQ_MAX_REFINE", "rq_decode_attention", "rq_decode_attention_tail",
-    "rq_decode_attention_noalloc", "rq_reconstruct", "rq_workspace_status", "rq_encode_take_status",
+    "rq_decode_attention_noalloc", "rq_decode_attention_varlen", "rq_decode_workspace_bytes_varlen",
+    "RQ_MAX_VARLEN_BATCH", "rq_reconstruct", "rq_workspace_status", "rq_encode_take_status",
     "alloc_codes", "alloc_scales", "alloc_workspace", "encode", "decode_attention", "reconstruct",
 ]
 
@@ -38,10 +41,11 @@ def alloc_scales(shape, bits, device="cuda"):
     return torch.empty(n, dtype=torch.uint8, device=device) if n else None
 
 
-def alloc_workspace(shape, device="cuda"):
-    """Zero-filled decode workspace, as rq_decode_attention requires."""
+def alloc_workspace(shape, device="cuda", varlen=False):
+    """Zero-filled decode workspace, as rq_decode_attention (or, with
+    varlen, rq_decode_attention_varlen) requires."""
     import torch
-    n = rq_decode_workspace_bytes(shape)
+    n = rq_decode_workspace_bytes_varlen(shape) if varlen else rq_decode_workspace_bytes(shape)
     if n == 0:
         raise RqError(RQ_ERR_INVALID_ARG, "rq_decode_workspace_bytes")
     return torch.zeros(n, dtype=torch.uint8, device=device)

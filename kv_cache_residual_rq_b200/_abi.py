@@ -20,6 +20,7 @@ RQ_ERR_WORKSPACE = 4
 RQ_ERR_CUDA = 5
 RQ_MAX_LOOPS = 16
 RQ_MAX_REFINE = 8
+RQ_MAX_VARLEN_BATCH = 1024
 
 
 class RqError(RuntimeError):
@@ -86,6 +87,15 @@ def lib():
                                       c.POINTER(c.c_void_p), c.POINTER(c.c_void_p), c.c_void_p,
                                       c.c_void_p]
         L.rq_encode_at_ex.restype = c.c_int
+        L.rq_decode_attention_varlen.argtypes = [sp, c.c_void_p, c.c_void_p, c.c_void_p,
+                                                 c.c_void_p, c.c_void_p, c.c_void_p,
+                                                 c.c_void_p, c.c_void_p, c.c_int, c.c_uint64,
+                                                 c.c_float, c.c_void_p, c.c_void_p, c.c_int,
+                                                 c.c_int, c.c_void_p, c.c_void_p, c.c_size_t,
+                                                 c.c_void_p]
+        L.rq_decode_attention_varlen.restype = c.c_int
+        L.rq_decode_workspace_bytes_varlen.argtypes = [sp]
+        L.rq_decode_workspace_bytes_varlen.restype = c.c_size_t
         L.rq_decode_attention_tail.argtypes = [sp, c.c_void_p, c.c_void_p, c.c_void_p,
                                                c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p,
                                                c.c_int, c.c_uint64, c.c_float, c.c_void_p,
@@ -199,6 +209,26 @@ def rq_encode_at_ex(shape, src_pitch, src_offset, dst_pitch, dst_offset, kv_loop
                                ptrs(scales_out), _ptr(ref_out), _stream(stream))
     if check:
         _check(st, "rq_encode_at_ex")
+    return st
+
+
+def rq_decode_workspace_bytes_varlen(shape):
+    return lib().rq_decode_workspace_bytes_varlen(_shp(shape))
+
+
+def rq_decode_attention_varlen(shape, ctx_lens, q, ref_k, ref_v, codes_k, codes_v, scales_k,
+                               scales_v, bits, seed, softmax_scale, tail_k, tail_v, n_tail,
+                               tail_pitch, out, workspace, workspace_bytes=None, stream=None,
+                               check=True):
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    st = lib().rq_decode_attention_varlen(
+        _shp(shape), _ptr(ctx_lens), _ptr(q), _ptr(ref_k), _ptr(ref_v), _ptr(codes_k),
+        _ptr(codes_v), _ptr(scales_k), _ptr(scales_v), int(bits), ctypes.c_uint64(seed),
+        float(softmax_scale), _ptr(tail_k), _ptr(tail_v), int(n_tail), int(tail_pitch), _ptr(out),
+        _ptr(workspace), int(workspace_bytes), _stream(stream))
+    if check:
+        _check(st, "rq_decode_attention_varlen")
     return st
 
 

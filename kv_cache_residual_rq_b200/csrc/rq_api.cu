@@ -55,9 +55,22 @@ int device_sm_count() {
   return sms;
 }
 
-DecodePlan plan_decode(const rq_shape& s, int num_sms) {
+DecodePlan plan_decode(const rq_shape& s, int num_sms, bool varlen) {
   DecodePlan pl;
   pl.heads = (long long)s.batch * s.kv_heads;
+  if (varlen) {
+    // tiles are counted on the device; a head of a sequence at full
+    // capacity has nt tiles and can meet at most one CTA run per tile
+    const int cap = s.ctx_cap ? s.ctx_cap : s.ctx;
+    pl.nt = cap > 0 ? (cap + kDecodeTile - 1) / kDecodeTile : 1;
+    pl.n_tiles = 0;
+    long long P = (long long)num_sms * kDecodeCtasPerSm;
+    if (P > kDecodeMaxCtas) P = kDecodeMaxCtas;
+    if (P < 1) P = 1;
+    pl.ctas = (int)P;
+    pl.max_contrib = pl.nt < kDecodeMaxCtas ? pl.nt : kDecodeMaxCtas;
+    return pl;
+  }
   pl.nt = (s.ctx + kDecodeTile - 1) / kDecodeTile;
   pl.n_tiles = pl.heads * pl.nt;
   long long P = (long long)num_sms * kDecodeCtasPerSm;
@@ -73,8 +86,8 @@ DecodePlan plan_decode(const rq_shape& s, int num_sms) {
   return pl;
 }
 
-size_t decode_workspace_bytes(const rq_shape& s) {
-  const DecodePlan pl = plan_decode(s, 1);
+size_t decode_workspace_bytes(const rq_shape& s, bool varlen) {
+  const DecodePlan pl = plan_decode(s, 1, varlen);
   const int G = s.q_heads / s.kv_heads;
   return kWsHeaderBytes + ws_counters_bytes(pl.heads) +
          (size_t)pl.heads * pl.max_contrib * G * ws_record_floats(s.head_dim) * sizeof(float);
@@ -194,18 +207,26 @@ rq_status rq_encode(const rq_shape* shape, const uint16_t* const* kv_loops, int 
                       codes_out, scales_out, nullptr, stream);
 }
 
-rq_status rq_decode_attention_tail(const rq_shape* shape, const uint16_t* q,
-                                   const uint16_t* ref_k, const uint16_t* ref_v,
-                                   const uint32_t* codes_k, const uint32_t* codes_v,
-                                   const uint16_t* scales_k, const uint16_t* scales_v, int bits,
-                                   uint64_t seed, float softmax_scale, const uint16_t* tail_k,
-                                   const uint16_t* tail_v, int n_tail, int tail_pitch,
-                                   float* out, void* workspace, size_t workspace_bytes,
-                                   void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Shared body of the decode entry points; ctx_lens null: every sequence has
+// shape->ctx cached tokens.
+rq_status decode_impl(const rq_shape* shape, const int32_t* ctx_lens, const uint16_t* q,
+                      const uint16_t* ref_k, const uint16_t* ref_v, const uint32_t* codes_k,
+                      const uint32_t* codes_v, const uint16_t* scales_k,
+                      const uint16_t* scales_v, int bits, uint64_t seed, float softmax_scale,
+                      const uint16_t* tail_k, const uint16_t* tail_v, int n_tail,
+                      int tail_pitch, float* out, void* workspace, size_t workspace_bytes,
+                      void* stream) {
+  const bool varlen = ctx_lens != nullptr;
   if (!shape) return RQ_ERR_INVALID_ARG;
   if (shape->batch < 1 || shape->kv_heads < 1 || shape->ctx < 1 ||
       shape->q_heads < shape->kv_heads)
     return RQ_ERR_INVALID_ARG;
+  if (varlen && shape->batch > RQ_MAX_VARLEN_BATCH) return RQ_ERR_INVALID_ARG;
+  if (varlen && (reinterpret_cast<uintptr_t>(ctx_lens) & 3u)) return RQ_ERR_ALIGNMENT;
   if (shape->ctx_cap != 0 && shape->ctx_cap < shape->ctx) return RQ_ERR_INVALID_ARG;
   if (n_tail < 0 || n_tail > RQ_MAX_TAIL) return RQ_ERR_INVALID_ARG;
   if (n_tail > 0 && (!tail_k || !tail_v || tail_pitch < n_tail)) return RQ_ERR_INVALID_ARG;
@@ -221,12 +242,13 @@ rq_status rq_decode_attention_tail(const rq_shape* shape, const uint16_t* q,
   if (bits != 16 && (!aligned16(codes_k) || !aligned16(codes_v) || !aligned16(scales_k) ||
                      !aligned16(scales_v)))
     return RQ_ERR_ALIGNMENT;
-  if (!workspace || workspace_bytes < decode_workspace_bytes(*shape)) return RQ_ERR_WORKSPACE;
+  if (!workspace || workspace_bytes < decode_workspace_bytes(*shape, varlen))
+    return RQ_ERR_WORKSPACE;
   if (!aligned16(workspace)) return RQ_ERR_ALIGNMENT;
 
   const int sms = device_sm_count();
   if (sms <= 0) return RQ_ERR_CUDA;
-  const DecodePlan pl = plan_decode(*shape, sms);
+  const DecodePlan pl = plan_decode(*shape, sms, varlen);
   const int G = shape->q_heads / shape->kv_heads;
   DecodeParams p;
   p.q = q;
@@ -251,6 +273,8 @@ rq_status rq_decode_attention_tail(const rq_shape* shape, const uint16_t* q,
   p.tail_v = n_tail > 0 ? tail_v : nullptr;
   p.n_tail = n_tail;
   p.tail_pitch = n_tail > 0 ? tail_pitch : 0;
+  p.ctx_lens = ctx_lens;
+  if (varlen) p.ctx = pitch_of(shape);
   p.nt = pl.nt;
   p.n_tiles = pl.n_tiles;
   p.ctas = pl.ctas;
@@ -264,6 +288,43 @@ rq_status rq_decode_attention_tail(const rq_shape* shape, const uint16_t* q,
                       : launch_decode_gqa(shape->head_dim, G, bits, p,
                                           static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? RQ_OK : RQ_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+rq_status rq_decode_attention_tail(const rq_shape* shape, const uint16_t* q,
+                                   const uint16_t* ref_k, const uint16_t* ref_v,
+                                   const uint32_t* codes_k, const uint32_t* codes_v,
+                                   const uint16_t* scales_k, const uint16_t* scales_v, int bits,
+                                   uint64_t seed, float softmax_scale, const uint16_t* tail_k,
+                                   const uint16_t* tail_v, int n_tail, int tail_pitch,
+                                   float* out, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
+  return decode_impl(shape, nullptr, q, ref_k, ref_v, codes_k, codes_v, scales_k, scales_v, bits,
+                     seed, softmax_scale, tail_k, tail_v, n_tail, tail_pitch, out, workspace,
+                     workspace_bytes, stream);
+}
+
+rq_status rq_decode_attention_varlen(const rq_shape* shape, const int32_t* ctx_lens,
+                                     const uint16_t* q, const uint16_t* ref_k,
+                                     const uint16_t* ref_v, const uint32_t* codes_k,
+                                     const uint32_t* codes_v, const uint16_t* scales_k,
+                                     const uint16_t* scales_v, int bits, uint64_t seed,
+                                     float softmax_scale, const uint16_t* tail_k,
+                                     const uint16_t* tail_v, int n_tail, int tail_pitch,
+                                     float* out, void* workspace, size_t workspace_bytes,
+                                     void* stream) {
+  if (!ctx_lens) return RQ_ERR_INVALID_ARG;
+  return decode_impl(shape, ctx_lens, q, ref_k, ref_v, codes_k, codes_v, scales_k, scales_v,
+                     bits, seed, softmax_scale, tail_k, tail_v, n_tail, tail_pitch, out,
+                     workspace, workspace_bytes, stream);
+}
+
+size_t rq_decode_workspace_bytes_varlen(const rq_shape* shape) {
+  if (!decode_shape_ok(shape) || shape->batch > RQ_MAX_VARLEN_BATCH) return 0;
+  return decode_workspace_bytes(*shape, true);
 }
 
 rq_status rq_decode_attention(const rq_shape* shape, const uint16_t* q, const uint16_t* ref_k,

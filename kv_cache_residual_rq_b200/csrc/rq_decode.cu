@@ -81,7 +81,10 @@ struct Cfg {
   // merge area: per warp and query row {m, l} + accRef[D] + accRes[D]; it
   // shares the table's space when there is one (never live at once)
   static constexpr int MERGE_FLOATS = kConsumerWarps * G * (2 + 2 * D);
-  static constexpr int AREA_FLOATS = LUT_FLOATS > MERGE_FLOATS ? LUT_FLOATS : MERGE_FLOATS;
+  // ... and serves as scratch for the sequence-length scan of a
+  // variable-length call before the first head
+  static constexpr int AREA_0 = LUT_FLOATS > MERGE_FLOATS ? LUT_FLOATS : MERGE_FLOATS;
+  static constexpr int AREA_FLOATS = AREA_0 > kVarlenMaxBatch + 4 ? AREA_0 : kVarlenMaxBatch + 4;
   static constexpr int QBUF_FLOATS = 2 * G * D;             // q and q~
   // bf16 query rows of the first heads of a CTA's run, fetched at the start
   static constexpr int QPRE_HEADS = 4;
@@ -153,10 +156,6 @@ decode_kernel(const DecodeParams p) {
   pdl_allow_next();
   if (cta >= p.ctas) return;
 
-  const long long tile_begin = (long long)cta * p.n_tiles / p.ctas;
-  const long long tile_end = (long long)(cta + 1) * p.n_tiles / p.ctas;
-  const int n_my = (int)(tile_end - tile_begin);
-
   if (tid == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full_bar[s], 1);
@@ -169,13 +168,20 @@ decode_kernel(const DecodeParams p) {
   __syncthreads();
   pdl_wait_prev();     // inputs and workspace may come from the previous kernel
 
-  const int T = p.ctx;
+  // this CTA's run of tiles (the merge area is free scratch until the first head)
+  CallSplit split;
+  long long tile_begin, tile_end;
+  TileCursor first_cur;
+  if (!plan_cta(p, cta, reinterpret_cast<int*>(area), split, tile_begin, tile_end, first_cur))
+    return;
+  const int n_my = (int)(tile_end - tile_begin);
   const int SB = (D / p.group) * 2;     // scale bytes per token
 
   // ========================= producer warp ================================
   if (warp == kConsumerWarps) {
     if (lane == 0) {
       int issued = 0;
+      TileCursor cur = first_cur;
       for (int i = 0; i < n_my; ++i) {
         const int s = i % STAGES;
         if (i >= STAGES) {
@@ -186,12 +192,17 @@ decode_kernel(const DecodeParams p) {
           }
         }
         if (flags[0]) break;
-        const long long tile = tile_begin + i;
-        const long long hd = tile / p.nt;
-        const int t0 = (int)(tile % p.nt) * TILE;
-        const int n = min(TILE, T - t0);
+        const long long hd = cur.hd;
+        const int t0 = cur.t0();
+        const int n = cur.n();
+        cur.next(p);
         const size_t row = (size_t)hd * p.ctx_pitch + t0;       // first token row of the tile
         unsigned char* st = ring + s * C::STAGE_BYTES;
+        if (n <= 0) {                   // the empty tile of an empty sequence
+          mbar_arrive(&full_bar[s]);
+          ++issued;
+          continue;
+        }
         uint32_t bytes = 2u * n * C::KROW;
         size_t sc_lo = 0;
         uint32_t sc_bytes = 0;
@@ -224,9 +235,9 @@ decode_kernel(const DecodeParams p) {
   // ========================= consumer warps ===============================
   // the query rows of the first heads of the run, while the first tiles are
   // in flight (made visible by the barrier that starts load_rotate_queries)
-  const long long h_first = tile_begin / p.nt;
+  const long long h_first = first_cur.hd;
   const int n_pre =
-      n_my > 0 ? (int)min((long long)C::QPRE_HEADS, (tile_end - 1) / p.nt - h_first + 1) : 0;
+      (int)min((long long)C::QPRE_HEADS, (long long)p.batch * p.kv_heads - h_first);
   for (int e = tid; e < n_pre * G * D / 8; e += kConsumerThreads) {
     const int hh = e / (G * D / 8), rem = e % (G * D / 8);
     const long long hd = h_first + hh;
@@ -328,7 +339,7 @@ decode_kernel(const DecodeParams p) {
 
   // merge the 4 warps' states, write the head's partial record, and if this
   // CTA is the last contributor, finish the head
-  auto flush_head = [&](long long hd) {
+  auto flush_head = [&](long long hd, long long first_tile, int nt_h) {
     // fold the token slots of the warp together
 #pragma unroll
     for (int r = 0; r < G; ++r) {
@@ -383,7 +394,7 @@ decode_kernel(const DecodeParams p) {
     }
     named_bar_sync(1, kConsumerThreads);
 
-    finish_head<D, G, C::RES>(p, hd, cta, merge, qbuf, flags, tid);
+    finish_head<D, G, C::RES>(p, hd, first_tile, nt_h, split, cta, merge, qbuf, flags, tid);
   };
 
   // <q, K row> of the lane's dims, straight from the packed bf16 row
@@ -597,20 +608,26 @@ decode_kernel(const DecodeParams p) {
   };
 
   // ---- main loop over this CTA's tiles ----
-  long long cur_head = -1;
+  long long cur_head = -1, cur_first = 0;
+  int cur_nt = 0;
   bool aborted = false;
   reset_state();
+  TileCursor cur = first_cur;
   for (int i = 0; i < n_my; ++i) {
-    const long long tile = tile_begin + i;
-    const long long hd = tile / p.nt;
+    const long long hd = cur.hd;
+    const int t0 = cur.t0();
+    const int n = cur.n();
     if (hd != cur_head) {
       if (cur_head >= 0) {
-        flush_head(cur_head);
+        flush_head(cur_head, cur_first, cur_nt);
         reset_state();
       }
       cur_head = hd;
+      cur_first = cur.head_first();
+      cur_nt = cur.nt;
       setup_head(hd);
     }
+    cur.next(p);
     const int s = i % STAGES;
     bool ok = !aborted && !flags[0];
     if (ok) ok = mbar_wait_bounded(&full_bar[s], (i / STAGES) & 1);
@@ -620,9 +637,7 @@ decode_kernel(const DecodeParams p) {
       aborted = true;
       flags[0] = 1;
     }
-    if (!aborted) {
-      const int t0 = (int)(tile % p.nt) * TILE;
-      const int n = min(TILE, T - t0);
+    if (!aborted && n > 0) {
       const unsigned char* st = ring + s * C::STAGE_BYTES;
       const size_t row = (size_t)hd * p.ctx_pitch + t0;
       const int sc_off = (int)((row * SB) & 15);
@@ -636,7 +651,7 @@ decode_kernel(const DecodeParams p) {
   // After an abort the flush still runs (on whatever the state holds) so that
   // every consumer thread takes the same barrier sequence; the status word
   // marks the output invalid.
-  if (cur_head >= 0) flush_head(cur_head);
+  if (cur_head >= 0) flush_head(cur_head, cur_first, cur_nt);
 }
 
 template <int D, int G, int BITS>

@@ -32,6 +32,128 @@ __device__ __forceinline__ float half_at(const unsigned char* p) {
   return __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t*>(p)));
 }
 
+// ---------------------------------------------------------------------------
+// Tile numbering of a call: heads hd = b * kv_heads + h in order, each head's
+// tiles in token order.  A head of sequence b has nt_b tiles: p.nt for every
+// sequence of a uniform call; max(1, ceil(len_b / 64)) with len_b =
+// p.ctx_lens[b] clamped to [0, ctx_pitch] in a variable-length call (an empty
+// sequence keeps one empty tile, so its heads are still finished from the
+// tail).  A CTA walks its run of tiles with a cursor.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int seq_len(const DecodeParams& p, int b) {
+  if (!p.ctx_lens) return p.ctx;
+  return min(max(p.ctx_lens[b], 0), p.ctx_pitch);
+}
+
+__device__ __forceinline__ int seq_tiles(const DecodeParams& p, int len) {
+  return p.ctx_lens ? max(1, (len + kDecodeTile - 1) / kDecodeTile) : p.nt;
+}
+
+struct TileCursor {
+  long long seq_first;   // number of the first tile of sequence b
+  long long hd;          // head: b * kv_heads + h
+  int b, h, j;           // sequence, kv head, tile within the head
+  int nt, len;           // tiles per head and cached tokens of sequence b
+
+  __device__ int t0() const { return j * kDecodeTile; }
+  // tokens of the tile (0 for the empty tile of an empty sequence)
+  __device__ int n() const { return min(kDecodeTile, len - j * kDecodeTile); }
+  __device__ long long head_first() const { return seq_first + (long long)h * nt; }
+  __device__ void next(const DecodeParams& p) {
+    if (++j < nt) return;
+    j = 0;
+    ++hd;
+    if (++h < p.kv_heads) return;
+    h = 0;
+    seq_first += (long long)p.kv_heads * nt;
+    if (++b < p.batch) {
+      len = seq_len(p, b);
+      nt = seq_tiles(p, len);
+    }
+  }
+};
+
+// The split of a call over its CTAs: n_tiles tiles in `ctas` equal runs.
+struct CallSplit {
+  long long n_tiles;
+  int ctas;
+};
+
+// Work split and start cursor of this CTA.  Uniform calls: from the host's
+// plan.  Variable-length calls: every CTA scans the sequence lengths (one
+// warp, into `scratch`, which must hold batch + 1 ints and is free until the
+// caller's next barrier-protected use), uses min(p.ctas, n_tiles) CTAs and
+// finds the sequence of its first tile by binary search.  All threads of the
+// CTA call it (it contains __syncthreads); returns false for a CTA without
+// work.  Lengths outside [0, ctx_pitch] are clamped and raise status bit 16.
+__device__ __forceinline__ bool plan_cta(const DecodeParams& p, int cta, int* scratch,
+                                         CallSplit& split, long long& tile_begin,
+                                         long long& tile_end, TileCursor& cur) {
+  if (!p.ctx_lens) {
+    split.n_tiles = p.n_tiles;
+    split.ctas = p.ctas;
+  } else {
+    const int tid = threadIdx.x;
+    if (tid < 32) {
+      // exclusive prefix of per-head tile counts over the sequences
+      const int per = (p.batch + 31) / 32;
+      const int b0 = tid * per, b1 = min(p.batch, b0 + per);
+      int sum = 0;
+      bool bad = false;
+      for (int b = b0; b < b1; ++b) {
+        const int raw = p.ctx_lens[b];
+        bad |= raw < 0 || raw > p.ctx_pitch;
+        sum += seq_tiles(p, seq_len(p, b));
+      }
+      int incl = sum;
+#pragma unroll
+      for (int m = 1; m < 32; m <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, m);
+        if (tid >= m) incl += o;
+      }
+      int run = incl - sum;
+      for (int b = b0; b < b1; ++b) {
+        scratch[b] = run;
+        run += seq_tiles(p, seq_len(p, b));
+      }
+      if (tid == 31) scratch[p.batch] = incl;
+      if (__any_sync(0xffffffffu, bad) && tid == 0 && cta == 0) flag_error(p.status, 16u);
+    }
+    __syncthreads();
+    split.n_tiles = (long long)p.kv_heads * scratch[p.batch];
+    split.ctas = (int)min((long long)p.ctas, split.n_tiles);
+  }
+  if (cta >= split.ctas) return false;
+  tile_begin = (long long)cta * split.n_tiles / split.ctas;
+  tile_end = (long long)(cta + 1) * split.n_tiles / split.ctas;
+  int b;
+  long long seq_first;
+  if (!p.ctx_lens) {
+    const long long per_seq = (long long)p.kv_heads * p.nt;
+    b = (int)(tile_begin / per_seq);
+    seq_first = (long long)b * per_seq;
+  } else {
+    // last sequence whose first tile is <= tile_begin (prefixes strictly increase)
+    int lo = 0, hi = p.batch - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if ((long long)p.kv_heads * scratch[mid] <= tile_begin) lo = mid; else hi = mid - 1;
+    }
+    b = lo;
+    seq_first = (long long)p.kv_heads * scratch[b];
+  }
+  cur.b = b;
+  cur.seq_first = seq_first;
+  cur.len = seq_len(p, b);
+  cur.nt = seq_tiles(p, cur.len);
+  const long long rel = tile_begin - seq_first;
+  cur.h = (int)(rel / cur.nt);
+  cur.j = (int)(rel % cur.nt);
+  cur.hd = (long long)b * p.kv_heads + cur.h;
+  if (p.ctx_lens) __syncthreads();   // scratch free again
+  return true;
+}
+
 // Walsh-Hadamard transform (no scaling) of a D-vector spread over a warp:
 // lane owns coordinates lane*E .. lane*E+E-1, E = D/32.  Strides below E in
 // registers, the rest by shfl.xor; ascending strides, butterfly (a+b, a-b).
@@ -96,17 +218,18 @@ __device__ __forceinline__ void load_rotate_queries(const DecodeParams& p, long 
 // query rows [G][D] as floats.  All consumer threads call it; `merge` is
 // reused as scratch (it holds at least 4 G (2 + 2 D) floats).
 template <int D, int G, bool RES>
-__device__ __forceinline__ void finish_head(const DecodeParams& p, long long hd, int cta,
-                                            float* merge, const float* qs,
-                                            volatile int* flags, int tid) {
+__device__ __forceinline__ void finish_head(const DecodeParams& p, long long hd,
+                                            long long first_tile, int nt_h,
+                                            const CallSplit& split, int cta, float* merge,
+                                            const float* qs, volatile int* flags, int tid) {
   static_assert(2 * G * D + 3 * G + G * RQ_MAX_TAIL <= 4 * G * (2 + 2 * D),
                 "merge area too small for the tail scratch");
   const int b = (int)(hd / p.kv_heads);
   const int h = (int)(hd % p.kv_heads);
   // which records belong to this head, and which one is ours
-  const long long f = hd * p.nt, e = f + p.nt - 1;
-  const int c_first = (int)(((f + 1) * p.ctas - 1) / p.n_tiles);
-  const int c_last = (int)(((e + 1) * p.ctas - 1) / p.n_tiles);
+  const long long f = first_tile, e = f + nt_h - 1;
+  const int c_first = (int)(((f + 1) * split.ctas - 1) / split.n_tiles);
+  const int c_last = (int)(((e + 1) * split.ctas - 1) / split.n_tiles);
   const int ncontrib = c_last - c_first + 1;
   const int j = cta - c_first;
   if (j < 0 || j >= p.max_contrib || ncontrib > p.max_contrib) {

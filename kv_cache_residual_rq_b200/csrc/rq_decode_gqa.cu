@@ -74,6 +74,7 @@ struct GCfg {
                                          QFRAG_WORDS) +
                                     2 * STAGES * 8 + 16;
   static_assert(G == 2 || G == 4 || G == 8, "grouped queries");
+  static_assert(MERGE_FLOATS >= kVarlenMaxBatch + 1, "merge area holds the length scan");
   static_assert(GROUP == 32 || GROUP == 64, "scale group");
   static_assert(D == 64 || D == 128, "head_dim");
 };
@@ -200,10 +201,6 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
   pdl_allow_next();
   if (cta >= p.ctas) return;
 
-  const long long tile_begin = (long long)cta * p.n_tiles / p.ctas;
-  const long long tile_end = (long long)(cta + 1) * p.n_tiles / p.ctas;
-  const int n_my = (int)(tile_end - tile_begin);
-
   if (tid == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full_bar[s], 1);
@@ -216,12 +213,19 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
   __syncthreads();
   pdl_wait_prev();     // inputs and workspace may come from the previous kernel
 
-  const int T = p.ctx;
+  // this CTA's run of tiles (the merge area is free scratch until the first head)
+  CallSplit split;
+  long long tile_begin, tile_end;
+  TileCursor first_cur;
+  if (!plan_cta(p, cta, reinterpret_cast<int*>(merge), split, tile_begin, tile_end, first_cur))
+    return;
+  const int n_my = (int)(tile_end - tile_begin);
 
   // ========================= producer warp ================================
   if (warp == kConsumerWarps) {
     if (lane == 0) {
       int issued = 0;
+      TileCursor cur = first_cur;
       for (int i = 0; i < n_my; ++i) {
         const int s = i % STAGES;
         if (i >= STAGES) {
@@ -232,12 +236,17 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
           }
         }
         if (flags[0]) break;
-        const long long tile = tile_begin + i;
-        const long long hd = tile / p.nt;
-        const int t0 = (int)(tile % p.nt) * TILE;
-        const int n = min(TILE, T - t0);
+        const long long hd = cur.hd;
+        const int t0 = cur.t0();
+        const int n = cur.n();
+        cur.next(p);
         const size_t row = (size_t)hd * p.ctx_pitch + t0;
         unsigned char* st = ring + s * C::STAGE_BYTES;
+        if (n <= 0) {                   // the empty tile of an empty sequence
+          mbar_arrive(&full_bar[s]);
+          ++issued;
+          continue;
+        }
         uint32_t bytes = 2u * C::NBOX * C::BOX_BYTES;     // full boxes, OOB rows zero-filled
         size_t sc_lo = 0;
         uint32_t sc_bytes = 0;
@@ -330,7 +339,7 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
     named_bar_sync(1, kConsumerThreads);
   };
 
-  auto flush_head = [&](long long hd) {
+  auto flush_head = [&](long long hd, long long first_tile, int nt_h) {
     // l and the V weight sums of row g over the four lanes of its row group
     l_run += __shfl_xor_sync(FULL, l_run, 1);
     l_run += __shfl_xor_sync(FULL, l_run, 2);
@@ -373,11 +382,25 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
       }
       named_bar_sync(1, kConsumerThreads);
     }
-    finish_head<D, G, C::RES>(p, hd, cta, merge, qbuf, flags, tid);
+    finish_head<D, G, C::RES>(p, hd, first_tile, nt_h, split, cta, merge, qbuf, flags, tid);
   };
 
   // ---- one tile ----
   auto tile_mma = [&](const unsigned char* st, int n, int sc_off) {
+    if (n < TILE) {
+      // rows past the head's last token (spare capacity, the next head, or
+      // nothing ever written) are not part of the context: their weights are
+      // 0, and zeroing this warp's such V rows keeps a non-finite value there
+      // out of the products
+      unsigned char* vrows = const_cast<unsigned char*>(st) + C::OFF_V;
+      for (int e = lane; e < C::WTOK * C::NBOX * 8; e += 32) {
+        const int tok = wtok + e / (C::NBOX * 8), c = e % (C::NBOX * 8);
+        if (tok >= n)
+          *reinterpret_cast<uint4*>(vrows + (c >> 3) * C::BOX_BYTES + tok * 128 + (c & 7) * 16) =
+              make_uint4(0u, 0u, 0u, 0u);
+      }
+      __syncwarp();
+    }
     const uint32_t sK = smem_u32(st + C::OFF_K);
     const uint32_t sV = smem_u32(st + C::OFF_V);
     const int r7 = lane & 7;
@@ -540,20 +563,26 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
   };
 
   // ---- main loop over this CTA's tiles ----
-  long long cur_head = -1;
+  long long cur_head = -1, cur_first = 0;
+  int cur_nt = 0;
   bool aborted = false;
   reset_state();
+  TileCursor cur = first_cur;
   for (int i = 0; i < n_my; ++i) {
-    const long long tile = tile_begin + i;
-    const long long hd = tile / p.nt;
+    const long long hd = cur.hd;
+    const int t0 = cur.t0();
+    const int n = cur.n();
     if (hd != cur_head) {
       if (cur_head >= 0) {
-        flush_head(cur_head);
+        flush_head(cur_head, cur_first, cur_nt);
         reset_state();
       }
       cur_head = hd;
+      cur_first = cur.head_first();
+      cur_nt = cur.nt;
       setup_head(hd);
     }
+    cur.next(p);
     const int s = i % STAGES;
     bool ok = !aborted && !flags[0];
     if (ok) ok = mbar_wait_bounded(&full_bar[s], (i / STAGES) & 1);
@@ -563,16 +592,14 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
       aborted = true;
       flags[0] = 1;
     }
-    if (!aborted) {
-      const int t0 = (int)(tile % p.nt) * TILE;
-      const int n = min(TILE, T - t0);
+    if (!aborted && n > 0) {
       const size_t row = (size_t)hd * p.ctx_pitch + t0;
       tile_mma(ring + s * C::STAGE_BYTES, n, (int)((row * SB) & 15));
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty_bar[s]);
   }
-  if (cur_head >= 0) flush_head(cur_head);
+  if (cur_head >= 0) flush_head(cur_head, cur_first, cur_nt);
 }
 
 // ---- host side ---------------------------------------------------------------

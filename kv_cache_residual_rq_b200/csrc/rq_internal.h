@@ -99,6 +99,8 @@ cudaError_t launch_reconstruct(int head_dim, int group, int bits, const Reconstr
 constexpr int kDecodeTile = 64;
 constexpr int kDecodeCtasPerSm = 2;
 constexpr int kDecodeMaxCtas = 1024;     // bound used to size the workspace
+constexpr int kVarlenMaxBatch = 1024;    // sequences of a variable-length call
+static_assert(kVarlenMaxBatch == RQ_MAX_VARLEN_BATCH, "one limit");
 
 struct DecodePlan {
   long long heads;      // batch * kv_heads
@@ -109,8 +111,10 @@ struct DecodePlan {
 };
 
 // Host arithmetic shared by the size query and the launch.
-DecodePlan plan_decode(const rq_shape& s, int num_sms);
-size_t decode_workspace_bytes(const rq_shape& s);
+// varlen: the tile count is known only on the device; the plan then holds
+// the CTA count and a record bound that holds for any lengths <= capacity.
+DecodePlan plan_decode(const rq_shape& s, int num_sms, bool varlen = false);
+size_t decode_workspace_bytes(const rq_shape& s, bool varlen = false);
 
 // Workspace layout: [status u32, pad to 16][counters u32 per head, pad to 16]
 //                   [partial records: heads * max_contrib * G records]
@@ -138,6 +142,8 @@ struct DecodeParams {
   const uint16_t* tail_k;   // optional BF16 tail tokens [heads][tail_pitch][d]
   const uint16_t* tail_v;
   int n_tail, tail_pitch;
+  const int* ctx_lens;   // variable-length call: cached tokens per sequence
+                         // [batch] (device int32), else null (ctx for all)
   int nt;
   long long n_tiles;
   int ctas;

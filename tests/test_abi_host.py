@@ -219,3 +219,23 @@ def test_encode_at_ex_rejects_refits_out_of_range():
     z = rq.make_shape(1, 2, 0, 128, 32)
     assert rq.rq_encode_at_ex(z, 1, 0, 1, 0, [FAKE], FAKE, [2], 0, rq.RQ_MAX_REFINE, [FAKE],
                               [FAKE], stream=0, check=False) == rq.RQ_OK
+
+
+def test_varlen_decode_rejects_bad_arguments_before_launch():
+    s = rq.make_shape(4, 2, 100, 128, 32, q_heads=8)
+    call = lambda shape=s, lens=FAKE: rq.rq_decode_attention_varlen(
+        shape, lens, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, 0, 0.0, None, None, 0, 0, FAKE,
+        FAKE, 1 << 30, stream=0, check=False)
+    assert call(lens=None) == rq.RQ_ERR_INVALID_ARG
+    assert call(lens=FAKE + 2) == rq.RQ_ERR_ALIGNMENT
+    big = rq.make_shape(rq.RQ_MAX_VARLEN_BATCH + 1, 2, 100, 128, 32, q_heads=8)
+    assert call(shape=big) == rq.RQ_ERR_INVALID_ARG
+    assert rq.rq_decode_workspace_bytes_varlen(big) == 0
+    # the workspace bound covers any lengths up to the capacity
+    cap = rq.make_shape(4, 2, 64, 128, 32, q_heads=8, ctx_cap=640)
+    assert rq.rq_decode_workspace_bytes_varlen(cap) >= rq.rq_decode_workspace_bytes(
+        rq.make_shape(4, 2, 640, 128, 32, q_heads=8))
+    small_ws = rq.rq_decode_attention_varlen(
+        cap, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, 0, 0.0, None, None, 0, 0, FAKE,
+        FAKE, 64, stream=0, check=False)
+    assert small_ws == rq.RQ_ERR_WORKSPACE
