@@ -103,6 +103,24 @@ def measure(w, reps, peak, emit):
               "bytes": nb, "gbs": nb / t / 1e9, "frac": nb / t / 1e9 / peak,
               "tokens_per_s_per_head_call": w.batch / t})
     assert rq.rq_workspace_status(ws) == 0
+    if w.G == 1 and w.name == "ouro1.4b_decode":
+        # variable-length batch: seeded lengths in [ctx/8, ctx], the cache at
+        # full capacity; bytes are those of the tokens actually present
+        g = torch.Generator().manual_seed(w.seed * 977 + 5)
+        lens = torch.randint(w.ctx // 8, w.ctx + 1, (w.batch,), generator=g, dtype=torch.int32)
+        lens_d = lens.to(dev)
+        wsv = rq.alloc_workspace(shape, dev, varlen=True)
+        b = w.bits[0]
+        fn = lambda: rq.rq_decode_attention_varlen(shape, lens_d, q, refk, refv, ck[0], cv[0],
+                                                   sk[0], sv[0], b, w.seed, 0.0, None, None, 0,
+                                                   0, out, wsv)
+        t = _time(fn, reps, None)
+        per_tok = 4 * w.head_dim + 2 * w.head_dim * b // 8 + 4 * (w.head_dim // w.group)
+        nb = int(lens.sum()) * w.kv_heads * per_tok + w.batch * w.q_heads * w.head_dim * 6
+        emit({"workload": w.name, "kernel": f"decode varlen bits={b}", "G": w.G,
+              "lens": lens.tolist(), "us": t * 1e6, "bytes": nb, "gbs": nb / t / 1e9,
+              "frac": nb / t / 1e9 / peak})
+        assert rq.rq_workspace_status(wsv) == 0
 
 
 def main(argv=None):
