@@ -86,6 +86,13 @@ def lib():
         L.orq_quantize_group_refined_f64.argtypes = [c.c_int, c.c_int, f64p, c.c_int, u8p,
                                                      c.POINTER(c.c_double), f64p]
         L.orq_quantize_group_refined_f64.restype = c.c_int
+        L.orq_encode_rows_cr_f32.argtypes = [c.c_long, c.c_int, c.c_int, c.c_int, c.c_int,
+                                             c.c_uint64, u16p, c.c_void_p, u32p, u16p,
+                                             c.c_void_p, c.c_void_p]
+        L.orq_encode_rows_cr_f32.restype = None
+        L.orq_reconstruct_row_cr_f64.argtypes = [c.c_int, c.c_int, c.c_int, c.c_int, i8p, u32p,
+                                                 u16p, c.c_void_p, c.c_void_p, f64p]
+        L.orq_reconstruct_row_cr_f64.restype = None
         _lib = L
     return _lib
 
@@ -246,6 +253,48 @@ def encode_rows_refined_f32(x, ref, bits, group, seed, iters):
     scales = np.empty(x.shape[:-1] + (d // group,), dtype=np.uint16)
     lib().orq_encode_rows_refined_f32(n, d, group, bits, seed, iters, x, ref, words, scales)
     return words, scales
+
+
+def encode_rows_cr_f32(x, ref, ref_bits, bits, group, seed):
+    """Compressed-reference encode of rows [..., d] (bf16 bits); x None
+    encodes only the reference.  Returns (ref_words, ref_scales, words,
+    scales), the last two None without x."""
+    ref = _u16(ref)
+    d = ref.shape[-1]
+    n = int(np.prod(ref.shape[:-1])) if ref.ndim > 1 else 1
+    lead = ref.shape[:-1]
+    rw = np.empty(lead + ((d * ref_bits + 31) // 32,), dtype=np.uint32)
+    rs = np.empty(lead + (d // group,), dtype=np.uint16)
+    w = s = None
+    xp = wp = sp = None
+    if x is not None:
+        x = _u16(x)
+        assert x.shape == ref.shape
+        w = np.empty(lead + ((d * bits + 31) // 32,), dtype=np.uint32)
+        s = np.empty(lead + (d // group,), dtype=np.uint16)
+        xp, wp, sp = x.ctypes.data, w.ctypes.data, s.ctypes.data
+    lib().orq_encode_rows_cr_f32(n, d, group, ref_bits, bits, seed, ref, xp, rw, rs, wp, sp)
+    return rw, rs, w, s
+
+
+def reconstruct_rows_cr_f64(ref_words, ref_scales, words, scales, ref_bits, bits, group, seed,
+                            d):
+    """fp64 rows of a compressed-reference loop (words None: the reference)."""
+    rw = np.ascontiguousarray(ref_words, dtype=np.uint32).reshape(-1, (d * ref_bits + 31) // 32)
+    rs = np.ascontiguousarray(ref_scales, dtype=np.uint16).reshape(-1, d // group)
+    n = rw.shape[0]
+    if words is not None:
+        w = np.ascontiguousarray(words, dtype=np.uint32).reshape(n, -1)
+        sc = np.ascontiguousarray(scales, dtype=np.uint16).reshape(n, -1)
+    out = np.empty((n, d), dtype=np.float64)
+    D = signs(seed, d)
+    for i in range(n):
+        row = out[i]
+        lib().orq_reconstruct_row_cr_f64(
+            d, group, ref_bits, bits, D, np.ascontiguousarray(rw[i]), np.ascontiguousarray(rs[i]),
+            None if words is None else w[i].ctypes.data,
+            None if words is None else sc[i].ctypes.data, row)
+    return out
 
 
 def encode_row_f64(x, ref, bits, group, seed):

@@ -416,6 +416,79 @@ int orq_quantize_group_refined_f64(int g, int bits, const double *y, int iters,
     return done;
 }
 
+/* ------------------------------------------------------------------------ */
+/* compressed reference                                                      */
+/* ------------------------------------------------------------------------ */
+
+void orq_encode_rows_cr_f32(long n_rows, int d, int g, int ref_bits, int bits, uint64_t seed,
+                            const uint16_t *ref, const uint16_t *x,
+                            uint32_t *ref_words, uint16_t *ref_scales,
+                            uint32_t *words, uint16_t *scales)
+{
+    int8_t D[ORQ_MAX_D];
+    orq_signs(seed, d, D);
+    const int rwpr = (d * ref_bits + 31) / 32;
+    const int wpr = (d * bits + 31) / 32;
+    const int rtop = (1 << ref_bits) - 1;
+    for (long row = 0; row < n_rows; ++row) {
+        float r[ORQ_MAX_D], y[ORQ_MAX_D], z[ORQ_MAX_D];
+        uint8_t c[ORQ_MAX_D];
+        for (int i = 0; i < d; ++i)
+            r[i] = orq_bf16_to_f32(ref[row * d + i]);
+        orq_rotate_f32(d, D, r, y);
+        for (int k = 0; k < d / g; ++k) {
+            uint16_t h;
+            orq_quantize_group_refined_f32(g, ref_bits, y + k * g, 0, c + k * g, NULL, &h);
+            if (ref_scales)
+                ref_scales[row * (d / g) + k] = h;
+            const float s = (float)orq_f16_to_f64(h);
+            for (int i = 0; i < g; ++i)
+                z[k * g + i] = s * (float)(2 * c[k * g + i] - rtop);
+        }
+        if (ref_words)
+            orq_pack_codes(d, ref_bits, c, ref_words + row * rwpr);
+        if (!x)
+            continue;
+        for (int i = 0; i < d; ++i)
+            r[i] = orq_bf16_to_f32(x[row * d + i]);
+        orq_rotate_f32(d, D, r, y);
+        for (int i = 0; i < d; ++i)
+            y[i] = y[i] - z[i];
+        for (int k = 0; k < d / g; ++k)
+            orq_quantize_group_refined_f32(g, bits, y + k * g, 0, c + k * g, NULL,
+                                           scales + row * (d / g) + k);
+        orq_pack_codes(d, bits, c, words + row * wpr);
+    }
+}
+
+void orq_reconstruct_row_cr_f64(int d, int g, int ref_bits, int bits, const int8_t *D,
+                                const uint32_t *ref_words, const uint16_t *ref_scales,
+                                const uint32_t *words, const uint16_t *scales, double *out)
+{
+    uint8_t cr[ORQ_MAX_D], c[ORQ_MAX_D];
+    double w[ORQ_MAX_D];
+    double *R = (double *)malloc(sizeof(double) * (size_t)d * d);
+    orq_rotation_matrix_f64(d, D, R);
+    orq_unpack_codes(d, ref_bits, ref_words, cr);
+    if (words)
+        orq_unpack_codes(d, bits, words, c);
+    const int rtop = (1 << ref_bits) - 1, top = (1 << bits) - 1;
+    for (int i = 0; i < d; ++i) {
+        const int k = i / g;
+        w[i] = orq_f16_to_f64(ref_scales[k]) * (2 * cr[i] - rtop);
+        if (words)
+            w[i] += orq_f16_to_f64(scales[k]) * (2 * c[i] - top);
+    }
+    /* out = R^T w */
+    for (int j = 0; j < d; ++j) {
+        double acc = 0.0;
+        for (int i = 0; i < d; ++i)
+            acc += R[(size_t)i * d + j] * w[i];
+        out[j] = acc;
+    }
+    free(R);
+}
+
 /* fp64 definitional encoder: y = R r with the explicit matrix, the same code
  * rule evaluated in double, and the least-squares scale in double. */
 void orq_encode_row_f64(int d, int g, int bits, const int8_t *D,

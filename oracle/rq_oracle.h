@@ -113,6 +113,30 @@ void orq_encode_rows_refined_f32(long n_rows, int d, int g, int bits, uint64_t s
 int orq_quantize_group_refined_f64(int g, int bits, const double *y, int iters,
                                    uint8_t *codes, double *s_out, double *err);
 
+/* ---- compressed reference (the reference loop itself as rotated codes) --- */
+/* Reading of the pages' storage figure (80.7% less than BF16, beyond what a
+ * BF16 reference allows): the final loop is stored as rotated low-bit codes
+ * too, and every other loop as its residual against the RECONSTRUCTED
+ * reference, taken in the rotated domain.  Per row, in binary32:
+ *   y_ref = Rot f32(ref)            (the FWHT specification above)
+ *   reference codes/scales          quantiser above with ref_bits (4 or 8),
+ *                                   scale in the fixed <y,l> order
+ *                                   (refinement section, zero refits)
+ *   z_i   = f32(s16_ref) * l_ref,i  (exact: 11 x 9 significant bits)
+ *   e_i   = RN(y_i - z_i),  y = Rot f32(x)  for a non-final loop x
+ *   residual codes/scales           quantiser with bits (2 or 4), same
+ *                                   scale order
+ * so codes AND scales are reproducible bit for bit.  Reconstruction:
+ *   K_L^ = Rot^T z,   K_l^ = Rot^T (z + s16_l l_l). */
+void orq_encode_rows_cr_f32(long n_rows, int d, int g, int ref_bits, int bits, uint64_t seed,
+                            const uint16_t *ref, const uint16_t *x,
+                            uint32_t *ref_words, uint16_t *ref_scales,
+                            uint32_t *words, uint16_t *scales);
+/* out[d] in double; words/scales NULL reconstructs the reference loop. */
+void orq_reconstruct_row_cr_f64(int d, int g, int ref_bits, int bits, const int8_t *D,
+                                const uint32_t *ref_words, const uint16_t *ref_scales,
+                                const uint32_t *words, const uint16_t *scales, double *out);
+
 /* ---- reconstruction and attention (fp64 definitional) ------------------- */
 /* out[d] = f64(ref) + Rot^T (s16 * level), for one row. bits==16 => ref. */
 void orq_reconstruct_row_f64(int d, int g, int bits, const int8_t *D,

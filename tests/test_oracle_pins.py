@@ -475,3 +475,85 @@ def test_fixed_order_dot_within_its_rounding_bound():
         yi = rng.integers(-50, 50, size=g).astype(np.float32)     # all sums exact
         lv = rng.choice([-3, -1, 1, 3], size=g)
         assert oracle.ls_dot_f32(yi, lv) == float(np.sum(yi.astype(np.int64) * lv))
+
+
+# ---------------------------------------------------------------------------
+# compressed reference (the final loop stored as rotated codes)
+# ---------------------------------------------------------------------------
+
+def _bf16(v):
+    a = np.asarray(v, dtype=np.float32)
+    return (a.view(np.uint32) >> 16).astype(np.uint16)
+
+
+def _rand_bf16(rng, shape, scale=1.0):
+    return _bf16((rng.standard_normal(shape) * scale).astype(np.float32))
+
+
+def test_cr_reference_codes_are_the_zero_reference_encoder():
+    # quantising Rot(ref) is what the plain encoder does to ref against a
+    # zero reference: same codes (scales differ only in their sum order)
+    rng = np.random.default_rng(41)
+    ref = _rand_bf16(rng, (50, 128))
+    rw, rs, _, _ = oracle.encode_rows_cr_f32(None, ref, 4, 2, 32, 9)
+    w4, s4, _ = oracle.encode_rows_f32(ref, np.zeros_like(ref), 4, 32, 9)
+    assert np.array_equal(rw, w4)
+    a = np.vectorize(oracle.f16_to_f64)(rs)
+    b = np.vectorize(oracle.f16_to_f64)(s4)
+    assert np.all(np.abs(a - b) <= 1e-3 * np.abs(b) + 2.0 ** -24)
+
+
+def test_cr_exact_grid_reference_round_trips_exactly():
+    # d = 4, Rot = (1/2) H D: choose the rotated reference on the INT4 grid
+    # s l with s = 1/4 (levels include +-15), so that ref = D H y / 2 is a
+    # short dyadic vector, exact in bf16; then the reference reconstructs
+    # exactly, and a non-final loop equal to it gets a zero residual
+    d, seed = 4, 20                      # seed 20: all signs +1 for d = 4
+    assert list(oracle.signs(seed, d)) == [1, 1, 1, 1]
+    lv = np.array([15, -1, 3, -5])
+    y = 0.25 * lv
+    H = np.array([[oracle.hadamard_entry(i, j) for j in range(d)] for i in range(d)])
+    ref = H.T @ y / 2.0
+    rb = _bf16(ref)
+    assert np.array_equal(oracle.bf16_to_f32(rb).astype(np.float64), ref)
+    rw, rs, w, s = oracle.encode_rows_cr_f32(rb[None], rb[None], 4, 2, 4, seed)
+    codes = oracle.unpack_codes(rw[0], 4, d)
+    assert np.array_equal(2 * codes.astype(int) - 15, lv)
+    assert oracle.f16_to_f64(int(rs[0, 0])) == 0.25
+    K_ref = oracle.reconstruct_rows_cr_f64(rw, rs, None, None, 4, 2, 4, seed, d)
+    K_l = oracle.reconstruct_rows_cr_f64(rw, rs, w, s, 4, 2, 4, seed, d)
+    assert np.array_equal(K_ref[0], ref) and np.array_equal(K_l[0], ref)
+    assert oracle.f16_to_f64(int(s[0, 0])) == 0.0
+
+
+def test_cr_reconstruction_is_orthogonal():
+    # ||K^_l - x|| equals the rotated-domain error ||z + s l - R x||, with R
+    # the explicit rotation matrix: checks that reconstruction applies R^T
+    rng = np.random.default_rng(43)
+    d, g, seed = 64, 32, 12
+    ref = _rand_bf16(rng, (6, d))
+    x = _bf16(oracle.bf16_to_f32(ref) + 0.2 * rng.standard_normal((6, d)).astype(np.float32))
+    rw, rs, w, s = oracle.encode_rows_cr_f32(x, ref, 8, 4, g, seed)
+    K = oracle.reconstruct_rows_cr_f64(rw, rs, w, s, 8, 4, g, seed, d)
+    R = oracle.rotation_matrix_f64(d, seed)
+    xf = oracle.bf16_to_f32(x).astype(np.float64)
+    for i in range(6):
+        cr = oracle.unpack_codes(rw[i], 8, d).astype(int)
+        c = oracle.unpack_codes(w[i], 4, d).astype(int)
+        sr = np.repeat([oracle.f16_to_f64(int(h)) for h in rs[i]], g)
+        sl = np.repeat([oracle.f16_to_f64(int(h)) for h in s[i]], g)
+        z = sr * (2 * cr - 255) + sl * (2 * c - 15)
+        assert abs(np.linalg.norm(K[i] - xf[i]) - np.linalg.norm(z - R @ xf[i])) < 1e-9
+
+
+@pytest.mark.parametrize("ref_bits", [4, 8])
+def test_cr_residual_moves_the_loop_closer(ref_bits):
+    rng = np.random.default_rng(44 + ref_bits)
+    d, g, seed = 128, 32, 3
+    ref = _rand_bf16(rng, (40, d))
+    x = _bf16(oracle.bf16_to_f32(ref) + 0.1 * rng.standard_normal((40, d)).astype(np.float32))
+    rw, rs, w, s = oracle.encode_rows_cr_f32(x, ref, ref_bits, 2, g, seed)
+    xf = oracle.bf16_to_f32(x).astype(np.float64)
+    K_ref = oracle.reconstruct_rows_cr_f64(rw, rs, None, None, ref_bits, 2, g, seed, d)
+    K_l = oracle.reconstruct_rows_cr_f64(rw, rs, w, s, ref_bits, 2, g, seed, d)
+    assert np.linalg.norm(K_l - xf) < np.linalg.norm(K_ref - xf)
