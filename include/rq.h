@@ -85,7 +85,8 @@ int rq_version(void);
 /* Static text for a status code; never NULL. */
 const char *rq_status_string(rq_status s);
 
-/* Bytes of the codes of ONE loop at `bits` (2 or 4) for `shape`:
+/* Bytes of the codes of ONE loop at `bits` (2, 4, or 8 for a compressed
+ * reference) for `shape`:
  * batch*kv_heads*T*head_dim*bits/8 rounded up to 16, T = ctx_cap (ctx when
  * 0).  0 for bits == 16 or an invalid shape.  Host-only arithmetic. */
 size_t rq_codes_bytes(const rq_shape *shape, int bits);
@@ -165,6 +166,41 @@ rq_status rq_encode_at(const rq_shape *shape, int src_pitch, int src_offset, int
                        const uint16_t *ref, const uint8_t *bits_per_loop, uint64_t seed,
                        uint32_t *const *codes_out, uint16_t *const *scales_out,
                        uint16_t *ref_out, void *stream);
+
+/*
+ * rq_encode_cr_at -- encode into the compressed-reference format: the final
+ * loop itself is stored as rotated low-bit codes, and every other loop as its
+ * residual against the reconstructed reference, in the rotated domain (the
+ * reading of the pages' storage figure under which a decode step reads fewer
+ * bytes than BF16: ResidualQuant page, Abstract).  Per row, in binary32:
+ *   y_ref = Rot ref;  reference codes/scales: the group quantiser with
+ *           ref_bits, its least-squares sum in the fixed order of
+ *           rq_encode_at_ex;  z = f32(s16_ref) * l_ref (exact);
+ *   e     = RN(Rot x - z) for each non-final loop x, quantised with its bits.
+ * Codes and scales are bit-exact.  Reconstruction: K_L = Rot^T z and
+ * K_l = Rot^T (z + s16_l l_l); rq_reconstruct_cr and
+ * rq_decode_attention_cr read this format.
+ *
+ *   shape          : rows [batch][Hkv][ctx][d] of contiguous sources;
+ *                    ctx_cap ignored.
+ *   dst_pitch/offset: token pitch of the outputs and first token written
+ *                    (as rq_encode_at), so a step's new token can be retired
+ *                    into a cache position.
+ *   kv_loops, n_loops (0 .. RQ_MAX_LOOPS), bits_per_loop (2, 4 or 16),
+ *   codes_out, scales_out: as rq_encode_at; HOST arrays (may be NULL when
+ *                    n_loops is 0).
+ *   ref            : device bf16 final loop, contiguous.
+ *   ref_bits       : 4 or 8.
+ *   ref_codes_out  : rq_codes_bytes(dst shape, ref_bits) bytes.
+ *   ref_scales_out : rq_scales_bytes(dst shape, ref_bits) bytes.
+ * Errors: as rq_encode_at; RQ_ERR_UNSUPPORTED for other ref_bits.
+ */
+rq_status rq_encode_cr_at(const rq_shape *shape, int dst_pitch, int dst_offset,
+                          const uint16_t *const *kv_loops, int n_loops, const uint16_t *ref,
+                          int ref_bits, const uint8_t *bits_per_loop, uint64_t seed,
+                          uint32_t *ref_codes_out, uint16_t *ref_scales_out,
+                          uint32_t *const *codes_out, uint16_t *const *scales_out,
+                          void *stream);
 
 /* Most least-squares refits rq_encode_at_ex accepts. */
 #define RQ_MAX_REFINE 8
@@ -292,6 +328,33 @@ rq_status rq_decode_attention_varlen(const rq_shape *shape, const int32_t *ctx_l
                                      float *out, void *workspace, size_t workspace_bytes,
                                      void *stream);
 
+/*
+ * rq_decode_attention_cr -- decode attention of one loop over a cache in the
+ * compressed-reference format (rq_encode_cr_at): scores and values are formed
+ * from the reference codes plus (bits 2 or 4) the loop's residual codes, all
+ * in the rotated domain -- s = sigma <q~, s_ref l_ref + s l>, one Rot^T per
+ * output row -- so no BF16 row is read; bits == 16 decodes the final loop
+ * from the reference codes alone (codes/scales may then be NULL).
+ * One query row per kv head (q_heads == kv_heads; others RQ_ERR_UNSUPPORTED).
+ *   ctx_lens  : NULL (every sequence has shape->ctx tokens; workspace of
+ *               rq_decode_workspace_bytes) or a device int32 [batch] as in
+ *               rq_decode_attention_varlen (workspace of
+ *               rq_decode_workspace_bytes_varlen).
+ *   ref_codes_k/v, ref_scales_k/v, ref_bits (4 or 8): the reference's
+ *               codes and fp16 scales, [batch][Hkv][T_cap][...].
+ * Tail tokens (BF16 K/V of the current token) and every other argument as
+ * rq_decode_attention_tail.
+ */
+rq_status rq_decode_attention_cr(const rq_shape *shape, const int32_t *ctx_lens,
+                                 const uint16_t *q, const uint32_t *ref_codes_k,
+                                 const uint32_t *ref_codes_v, const uint16_t *ref_scales_k,
+                                 const uint16_t *ref_scales_v, int ref_bits,
+                                 const uint32_t *codes_k, const uint32_t *codes_v,
+                                 const uint16_t *scales_k, const uint16_t *scales_v, int bits,
+                                 uint64_t seed, float softmax_scale, const uint16_t *tail_k,
+                                 const uint16_t *tail_v, int n_tail, int tail_pitch, float *out,
+                                 void *workspace, size_t workspace_bytes, void *stream);
+
 /* Workspace bytes for rq_decode_attention_varlen with this shape (any
  * lengths up to the capacity); 0 if the shape is unsupported. */
 size_t rq_decode_workspace_bytes_varlen(const rq_shape *shape);
@@ -349,6 +412,16 @@ rq_status rq_decode_attention_noalloc(const rq_shape *shape, const uint16_t *q,
 rq_status rq_reconstruct(const rq_shape *shape, const uint16_t *ref, const uint32_t *codes,
                          const uint16_t *scales, int bits, uint64_t seed, void *out,
                          int out_bf16, void *stream);
+
+/* rq_reconstruct_cr -- rq_reconstruct for the compressed-reference format
+ * (rq_encode_cr_at): out = Rot^T (s_ref l_ref + s l), or Rot^T (s_ref l_ref)
+ * for bits == 16 (the reference loop; codes/scales may then be NULL).
+ * ref_codes/ref_scales as written by rq_encode_cr_at with ref_bits (4 or 8);
+ * layout, capacity and errors as rq_reconstruct. */
+rq_status rq_reconstruct_cr(const rq_shape *shape, const uint32_t *ref_codes,
+                            const uint16_t *ref_scales, int ref_bits, const uint32_t *codes,
+                            const uint16_t *scales, int bits, uint64_t seed, void *out,
+                            int out_bf16, void *stream);
 
 /* Reads and clears the encoders' sticky status word of the current device
  * (blocking; waits for all work on the device).  0 means every rq_encode /

@@ -13,7 +13,8 @@ from ._abi import (RQ_ERR_ALIGNMENT, RQ_ERR_CUDA, RQ_ERR_INVALID_ARG, RQ_ERR_UNS
                    rq_decode_attention_tail, rq_decode_workspace_bytes, rq_encode, rq_encode_at,
                    rq_encode_at_ex, rq_encode_take_status, rq_reconstruct, RQ_MAX_REFINE,
                    RQ_MAX_VARLEN_BATCH, rq_decode_attention_varlen,
-                   rq_decode_workspace_bytes_varlen,
+                   rq_decode_workspace_bytes_varlen, rq_encode_cr_at, rq_reconstruct_cr,
+                   rq_decode_attention_cr,
                    rq_scales_bytes, rq_shape, rq_status_string, rq_version,
                    rq_workspace_status)
 
@@ -23,7 +24,8 @@ __all__ = [
     "rq_status_string", "rq_codes_bytes", "rq_scales_bytes", "rq_decode_workspace_bytes",
     "rq_encode", "rq_encode_at", "rq_encode_at_ex", "RQ_MAX_REFINE", "rq_decode_attention", "rq_decode_attention_tail",
     "rq_decode_attention_noalloc", "rq_decode_attention_varlen", "rq_decode_workspace_bytes_varlen",
-    "RQ_MAX_VARLEN_BATCH", "rq_reconstruct", "rq_workspace_status", "rq_encode_take_status",
+    "RQ_MAX_VARLEN_BATCH", "rq_reconstruct", "rq_encode_cr_at", "rq_reconstruct_cr",
+    "rq_decode_attention_cr", "encode_cr", "reconstruct_cr", "decode_attention_cr", "rq_workspace_status", "rq_encode_take_status",
     "alloc_codes", "alloc_scales", "alloc_workspace", "encode", "decode_attention", "reconstruct",
 ]
 
@@ -105,4 +107,49 @@ def decode_attention(q, ref_k, ref_v, codes_k, codes_v, scales_k, scales_v, bits
     else:
         rq_decode_attention(shape, q, ref_k, ref_v, codes_k, codes_v, scales_k, scales_v, bits,
                             seed, softmax_scale, out, workspace, stream=stream)
+    return out
+
+
+def encode_cr(kv_loops, ref, ref_bits, bits_per_loop, group, seed, stream=None):
+    """Compressed-reference encode of contiguous [rows, Hkv, T, d] bf16 tensors.
+    Returns ((ref_codes, ref_scales), codes, scales)."""
+    rows, hkv, t, d = ref.shape
+    shape = make_shape(rows, hkv, t, d, group)
+    rc, rs = alloc_codes(shape, ref_bits, ref.device), alloc_scales(shape, ref_bits, ref.device)
+    codes = [alloc_codes(shape, b, ref.device) for b in bits_per_loop]
+    scales = [alloc_scales(shape, b, ref.device) for b in bits_per_loop]
+    rq_encode_cr_at(shape, t, 0, kv_loops, ref, ref_bits, bits_per_loop, seed, rc, rs, codes,
+                    scales, stream=stream)
+    return (rc, rs), codes, scales
+
+
+def reconstruct_cr(shape4, ref_codes, ref_scales, ref_bits, codes, scales, bits, group, seed,
+                   device="cuda", out_bf16=False, stream=None):
+    """Rows [rows, Hkv, T, d] of a compressed-reference loop (bits 16: the reference)."""
+    import torch
+    rows, hkv, t, d = shape4
+    shape = make_shape(rows, hkv, t, d, group)
+    out = torch.empty(shape4, dtype=torch.bfloat16 if out_bf16 else torch.float32,
+                      device=device)
+    rq_reconstruct_cr(shape, ref_codes, ref_scales, ref_bits, codes, scales, bits, seed, out,
+                      out_bf16, stream)
+    return out
+
+
+def decode_attention_cr(q, ref, codes_k, codes_v, scales_k, scales_v, bits, group, seed, ctx_cap,
+                        ctx=None, ctx_lens=None, tail_k=None, tail_v=None, n_tail=0,
+                        softmax_scale=0.0, out=None, workspace=None, stream=None):
+    """Decode attention over a compressed-reference cache.  ref = (ref_codes_k,
+    ref_scales_k, ref_codes_v, ref_scales_v, ref_bits); q [B, H, d]."""
+    import torch
+    rck, rsk, rcv, rsv, ref_bits = ref
+    b, h, d = q.shape
+    shape = make_shape(b, h, ctx if ctx is not None else ctx_cap, d, group, ctx_cap=ctx_cap)
+    if out is None:
+        out = torch.empty((b, h, d), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(shape, q.device, varlen=ctx_lens is not None)
+    rq_decode_attention_cr(shape, ctx_lens, q, rck, rcv, rsk, rsv, ref_bits, codes_k, codes_v,
+                           scales_k, scales_v, bits, seed, softmax_scale, tail_k, tail_v, n_tail,
+                           tail_k.shape[2] if n_tail else 0, out, workspace, stream=stream)
     return out

@@ -96,6 +96,22 @@ def lib():
         L.rq_decode_attention_varlen.restype = c.c_int
         L.rq_decode_workspace_bytes_varlen.argtypes = [sp]
         L.rq_decode_workspace_bytes_varlen.restype = c.c_size_t
+        L.rq_encode_cr_at.argtypes = [sp, c.c_int, c.c_int, c.POINTER(c.c_void_p), c.c_int,
+                                      c.c_void_p, c.c_int, c.POINTER(c.c_uint8), c.c_uint64,
+                                      c.c_void_p, c.c_void_p, c.POINTER(c.c_void_p),
+                                      c.POINTER(c.c_void_p), c.c_void_p]
+        L.rq_encode_cr_at.restype = c.c_int
+        L.rq_reconstruct_cr.argtypes = [sp, c.c_void_p, c.c_void_p, c.c_int, c.c_void_p,
+                                        c.c_void_p, c.c_int, c.c_uint64, c.c_void_p, c.c_int,
+                                        c.c_void_p]
+        L.rq_reconstruct_cr.restype = c.c_int
+        L.rq_decode_attention_cr.argtypes = [sp, c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p,
+                                             c.c_void_p, c.c_void_p, c.c_int, c.c_void_p,
+                                             c.c_void_p, c.c_void_p, c.c_void_p, c.c_int,
+                                             c.c_uint64, c.c_float, c.c_void_p, c.c_void_p,
+                                             c.c_int, c.c_int, c.c_void_p, c.c_void_p,
+                                             c.c_size_t, c.c_void_p]
+        L.rq_decode_attention_cr.restype = c.c_int
         L.rq_decode_attention_tail.argtypes = [sp, c.c_void_p, c.c_void_p, c.c_void_p,
                                                c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p,
                                                c.c_int, c.c_uint64, c.c_float, c.c_void_p,
@@ -299,3 +315,45 @@ def rq_encode_take_status():
     v = ctypes.c_uint32(0)
     _check(lib().rq_encode_take_status(ctypes.byref(v)), "rq_encode_take_status")
     return v.value
+
+
+def rq_encode_cr_at(shape, dst_pitch, dst_offset, kv_loops, ref, ref_bits, bits_per_loop, seed,
+                    ref_codes_out, ref_scales_out, codes_out, scales_out, stream=None,
+                    check=True):
+    n = len(bits_per_loop)
+    ptrs = lambda seq: (ctypes.c_void_p * max(n, 1))(*[_ptr(v) for v in seq])
+    bits = (ctypes.c_uint8 * max(n, 1))(*[int(b) for b in bits_per_loop])
+    st = lib().rq_encode_cr_at(_shp(shape), int(dst_pitch), int(dst_offset), ptrs(kv_loops), n,
+                               _ptr(ref), int(ref_bits), bits, ctypes.c_uint64(seed),
+                               _ptr(ref_codes_out), _ptr(ref_scales_out), ptrs(codes_out),
+                               ptrs(scales_out), _stream(stream))
+    if check:
+        _check(st, "rq_encode_cr_at")
+    return st
+
+
+def rq_reconstruct_cr(shape, ref_codes, ref_scales, ref_bits, codes, scales, bits, seed, out,
+                      out_bf16=False, stream=None, check=True):
+    st = lib().rq_reconstruct_cr(_shp(shape), _ptr(ref_codes), _ptr(ref_scales), int(ref_bits),
+                                 _ptr(codes), _ptr(scales), int(bits), ctypes.c_uint64(seed),
+                                 _ptr(out), 1 if out_bf16 else 0, _stream(stream))
+    if check:
+        _check(st, "rq_reconstruct_cr")
+    return st
+
+
+def rq_decode_attention_cr(shape, ctx_lens, q, ref_codes_k, ref_codes_v, ref_scales_k,
+                           ref_scales_v, ref_bits, codes_k, codes_v, scales_k, scales_v, bits,
+                           seed, softmax_scale, tail_k, tail_v, n_tail, tail_pitch, out,
+                           workspace, workspace_bytes=None, stream=None, check=True):
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    st = lib().rq_decode_attention_cr(
+        _shp(shape), _ptr(ctx_lens), _ptr(q), _ptr(ref_codes_k), _ptr(ref_codes_v),
+        _ptr(ref_scales_k), _ptr(ref_scales_v), int(ref_bits), _ptr(codes_k), _ptr(codes_v),
+        _ptr(scales_k), _ptr(scales_v), int(bits), ctypes.c_uint64(seed), float(softmax_scale),
+        _ptr(tail_k), _ptr(tail_v), int(n_tail), int(tail_pitch), _ptr(out), _ptr(workspace),
+        int(workspace_bytes), _stream(stream))
+    if check:
+        _check(st, "rq_decode_attention_cr")
+    return st

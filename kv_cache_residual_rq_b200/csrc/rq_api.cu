@@ -114,14 +114,14 @@ const char* rq_status_string(rq_status s) {
 }
 
 size_t rq_codes_bytes(const rq_shape* shape, int bits) {
-  if (!shape_ok(shape, false) || (bits != 2 && bits != 4)) return 0;
+  if (!shape_ok(shape, false) || (bits != 2 && bits != 4 && bits != 8)) return 0;
   const size_t elems =
       (size_t)shape->batch * shape->kv_heads * pitch_of(shape) * (size_t)shape->head_dim;
   return round16(elems * bits / 8);
 }
 
 size_t rq_scales_bytes(const rq_shape* shape, int bits) {
-  if (!shape_ok(shape, false) || (bits != 2 && bits != 4)) return 0;
+  if (!shape_ok(shape, false) || (bits != 2 && bits != 4 && bits != 8)) return 0;
   const size_t groups = (size_t)shape->batch * shape->kv_heads * pitch_of(shape) *
                         (size_t)(shape->head_dim / shape->group);
   return round16(groups * 2);
@@ -188,6 +188,58 @@ rq_status rq_encode_at_ex(const rq_shape* shape, int src_pitch, int src_offset,
   return e == cudaSuccess ? RQ_OK : RQ_ERR_CUDA;
 }
 
+rq_status rq_encode_cr_at(const rq_shape* shape, int dst_pitch, int dst_offset,
+                          const uint16_t* const* kv_loops, int n_loops, const uint16_t* ref,
+                          int ref_bits, const uint8_t* bits_per_loop, uint64_t seed,
+                          uint32_t* ref_codes_out, uint16_t* ref_scales_out,
+                          uint32_t* const* codes_out, uint16_t* const* scales_out,
+                          void* stream) {
+  if (!shape || (n_loops > 0 && (!kv_loops || !bits_per_loop || !codes_out || !scales_out)))
+    return RQ_ERR_INVALID_ARG;
+  if (shape->batch < 1 || shape->kv_heads < 1 || shape->ctx < 0) return RQ_ERR_INVALID_ARG;
+  if (dst_offset < 0 || dst_pitch < 1 || (long long)dst_offset + shape->ctx > dst_pitch)
+    return RQ_ERR_INVALID_ARG;
+  if (n_loops < 0 || n_loops > RQ_MAX_LOOPS) return RQ_ERR_INVALID_ARG;
+  if (ref_bits != 4 && ref_bits != 8) return RQ_ERR_UNSUPPORTED;
+  if (!supported_dims(shape->head_dim, shape->group)) return RQ_ERR_UNSUPPORTED;
+  if (!ref || !ref_codes_out || !ref_scales_out) return RQ_ERR_INVALID_ARG;
+  if (!aligned16(ref) || !aligned16(ref_codes_out) || !aligned16(ref_scales_out))
+    return RQ_ERR_ALIGNMENT;
+  EncodeParams p;
+  std::memset(&p, 0, sizeof p);
+  for (int l = 0; l < n_loops; ++l) {
+    const int b = bits_per_loop[l];
+    if (b != 2 && b != 4 && b != 16) return RQ_ERR_UNSUPPORTED;
+    p.bits[l] = b;
+    if (b == 16) continue;
+    if (!kv_loops[l] || !codes_out[l] || !scales_out[l]) return RQ_ERR_INVALID_ARG;
+    if (!aligned16(kv_loops[l]) || !aligned16(codes_out[l]) || !aligned16(scales_out[l]))
+      return RQ_ERR_ALIGNMENT;
+    p.x[l] = kv_loops[l];
+    p.codes[l] = codes_out[l];
+    p.scales[l] = scales_out[l];
+  }
+  p.ref = ref;
+  p.ref_bits = ref_bits;
+  p.ref_codes = ref_codes_out;
+  p.ref_scales = ref_scales_out;
+  p.n_loops = n_loops;
+  p.seed = seed;
+  p.ctx = shape->ctx;
+  p.src_pitch = shape->ctx;
+  p.src_offset = 0;
+  p.dst_pitch = dst_pitch;
+  p.dst_offset = dst_offset;
+  p.n_rows = (long long)shape->batch * shape->kv_heads * shape->ctx;
+  if (p.n_rows == 0) return RQ_OK;
+  if (p.n_rows > kEncodeTmaMaxRows) return RQ_ERR_UNSUPPORTED;
+  const int sms = device_sm_count();
+  if (sms <= 0) return RQ_ERR_CUDA;
+  cudaError_t e = launch_encode_tma(shape->head_dim, shape->group, p, sms,
+                                    static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? RQ_OK : RQ_ERR_CUDA;
+}
+
 rq_status rq_encode_at(const rq_shape* shape, int src_pitch, int src_offset, int dst_pitch,
                        int dst_offset, const uint16_t* const* kv_loops, int n_loops,
                        const uint16_t* ref, const uint8_t* bits_per_loop, uint64_t seed,
@@ -213,14 +265,33 @@ namespace {
 
 // Shared body of the decode entry points; ctx_lens null: every sequence has
 // shape->ctx cached tokens.
+struct CrRef {                 // compressed reference (ref_bits 0: BF16 rows)
+  int ref_bits = 0;
+  const uint32_t* codes_k = nullptr;
+  const uint32_t* codes_v = nullptr;
+  const uint16_t* scales_k = nullptr;
+  const uint16_t* scales_v = nullptr;
+};
+
 rq_status decode_impl(const rq_shape* shape, const int32_t* ctx_lens, const uint16_t* q,
                       const uint16_t* ref_k, const uint16_t* ref_v, const uint32_t* codes_k,
                       const uint32_t* codes_v, const uint16_t* scales_k,
                       const uint16_t* scales_v, int bits, uint64_t seed, float softmax_scale,
                       const uint16_t* tail_k, const uint16_t* tail_v, int n_tail,
                       int tail_pitch, float* out, void* workspace, size_t workspace_bytes,
-                      void* stream) {
+                      void* stream, const CrRef& cr = CrRef()) {
   const bool varlen = ctx_lens != nullptr;
+  if (cr.ref_bits != 0) {
+    if (cr.ref_bits != 4 && cr.ref_bits != 8) return RQ_ERR_UNSUPPORTED;
+    if (!shape || shape->q_heads != shape->kv_heads) return RQ_ERR_UNSUPPORTED;
+    if (!cr.codes_k || !cr.codes_v || !cr.scales_k || !cr.scales_v) return RQ_ERR_INVALID_ARG;
+    if (!aligned16(cr.codes_k) || !aligned16(cr.codes_v) || !aligned16(cr.scales_k) ||
+        !aligned16(cr.scales_v))
+      return RQ_ERR_ALIGNMENT;
+    // the reference rows are not read: stand-ins keep the checks below uniform
+    ref_k = reinterpret_cast<const uint16_t*>(cr.codes_k);
+    ref_v = reinterpret_cast<const uint16_t*>(cr.codes_v);
+  }
   if (!shape) return RQ_ERR_INVALID_ARG;
   if (shape->batch < 1 || shape->kv_heads < 1 || shape->ctx < 1 ||
       shape->q_heads < shape->kv_heads)
@@ -275,6 +346,11 @@ rq_status decode_impl(const rq_shape* shape, const int32_t* ctx_lens, const uint
   p.tail_pitch = n_tail > 0 ? tail_pitch : 0;
   p.ctx_lens = ctx_lens;
   if (varlen) p.ctx = pitch_of(shape);
+  p.ref_bits = cr.ref_bits;
+  p.rcodes_k = cr.codes_k;
+  p.rcodes_v = cr.codes_v;
+  p.rscales_k = cr.scales_k;
+  p.rscales_v = cr.scales_v;
   p.nt = pl.nt;
   p.n_tiles = pl.n_tiles;
   p.ctas = pl.ctas;
@@ -322,6 +398,27 @@ rq_status rq_decode_attention_varlen(const rq_shape* shape, const int32_t* ctx_l
                      workspace, workspace_bytes, stream);
 }
 
+rq_status rq_decode_attention_cr(const rq_shape* shape, const int32_t* ctx_lens,
+                                 const uint16_t* q, const uint32_t* ref_codes_k,
+                                 const uint32_t* ref_codes_v, const uint16_t* ref_scales_k,
+                                 const uint16_t* ref_scales_v, int ref_bits,
+                                 const uint32_t* codes_k, const uint32_t* codes_v,
+                                 const uint16_t* scales_k, const uint16_t* scales_v, int bits,
+                                 uint64_t seed, float softmax_scale, const uint16_t* tail_k,
+                                 const uint16_t* tail_v, int n_tail, int tail_pitch, float* out,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+  CrRef cr;
+  cr.ref_bits = ref_bits;
+  cr.codes_k = ref_codes_k;
+  cr.codes_v = ref_codes_v;
+  cr.scales_k = ref_scales_k;
+  cr.scales_v = ref_scales_v;
+  if (ref_bits != 4 && ref_bits != 8) return RQ_ERR_UNSUPPORTED;
+  return decode_impl(shape, ctx_lens, q, nullptr, nullptr, codes_k, codes_v, scales_k, scales_v,
+                     bits, seed, softmax_scale, tail_k, tail_v, n_tail, tail_pitch, out,
+                     workspace, workspace_bytes, stream, cr);
+}
+
 size_t rq_decode_workspace_bytes_varlen(const rq_shape* shape) {
   if (!decode_shape_ok(shape) || shape->batch > RQ_MAX_VARLEN_BATCH) return 0;
   return decode_workspace_bytes(*shape, true);
@@ -351,6 +448,7 @@ rq_status rq_reconstruct(const rq_shape* shape, const uint16_t* ref, const uint3
       (bits != 16 && (!aligned16(codes) || !aligned16(scales))))
     return RQ_ERR_ALIGNMENT;
   ReconstructParams p;
+  std::memset(&p, 0, sizeof p);
   p.ref = ref;
   p.codes = bits == 16 ? nullptr : codes;
   p.scales = bits == 16 ? nullptr : scales;
@@ -365,6 +463,40 @@ rq_status rq_reconstruct(const rq_shape* shape, const uint16_t* ref, const uint3
   if (sms <= 0) return RQ_ERR_CUDA;
   cudaError_t e = launch_reconstruct(shape->head_dim, shape->group, bits, p, sms,
                                      static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? RQ_OK : RQ_ERR_CUDA;
+}
+
+rq_status rq_reconstruct_cr(const rq_shape* shape, const uint32_t* ref_codes,
+                            const uint16_t* ref_scales, int ref_bits, const uint32_t* codes,
+                            const uint16_t* scales, int bits, uint64_t seed, void* out,
+                            int out_bf16, void* stream) {
+  if (!shape || !ref_codes || !ref_scales || !out) return RQ_ERR_INVALID_ARG;
+  if (shape->batch < 1 || shape->kv_heads < 1 || shape->ctx < 0) return RQ_ERR_INVALID_ARG;
+  if (shape->ctx_cap != 0 && shape->ctx_cap < shape->ctx) return RQ_ERR_INVALID_ARG;
+  if (!supported_dims(shape->head_dim, shape->group)) return RQ_ERR_UNSUPPORTED;
+  if (ref_bits != 4 && ref_bits != 8) return RQ_ERR_UNSUPPORTED;
+  if (bits != 2 && bits != 4 && bits != 16) return RQ_ERR_UNSUPPORTED;
+  if (bits != 16 && (!codes || !scales)) return RQ_ERR_INVALID_ARG;
+  if (!aligned16(ref_codes) || !aligned16(ref_scales) || !aligned16(out) ||
+      (bits != 16 && (!aligned16(codes) || !aligned16(scales))))
+    return RQ_ERR_ALIGNMENT;
+  ReconstructParams p;
+  std::memset(&p, 0, sizeof p);
+  p.ref_codes = ref_codes;
+  p.ref_scales = ref_scales;
+  p.codes = bits == 16 ? nullptr : codes;
+  p.scales = bits == 16 ? nullptr : scales;
+  p.out = out;
+  p.ctx = shape->ctx;
+  p.pitch = pitch_of(shape);
+  p.n_rows = (long long)shape->batch * shape->kv_heads * shape->ctx;
+  p.out_bf16 = out_bf16 ? 1 : 0;
+  p.seed = seed;
+  if (p.n_rows == 0) return RQ_OK;
+  const int sms = device_sm_count();
+  if (sms <= 0) return RQ_ERR_CUDA;
+  cudaError_t e = launch_reconstruct_cr(shape->head_dim, shape->group, ref_bits, bits, p, sms,
+                                        static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? RQ_OK : RQ_ERR_CUDA;
 }
 

@@ -125,9 +125,10 @@ __device__ __forceinline__ void load_row(const uint8_t* slot, int r, int q, uint
 // y_{m+16}} with step 1/(2 inv): packed code words, <y,l> in the fixed order
 // (fma chains over coordinates 0..15 and 16..31, the two runs added; the
 // partner lane's block added for groups of 64) and <l,l> (exact).
-template <int BITS, int GROUP, int RPW, bool CLAMP>
+template <int BITS, int GROUP, int RPW, bool CLAMP, bool WANT_LV = false>
 __device__ __forceinline__ void quant_pass(const float2 (&P)[16], float inv, uint32_t (&w)[BITS],
-                                           float& dot_out, float& nrm_out) {
+                                           float& dot_out, float& nrm_out,
+                                           float2* lv_out = nullptr) {
   const float2 inv2 = make_float2(inv, inv);
   const float2 mg = make_float2(kFloorMagic, kFloorMagic);
   const float2 two = make_float2(2.0f, 2.0f), one = make_float2(1.0f, 1.0f);
@@ -147,18 +148,23 @@ __device__ __forceinline__ void quant_pass(const float2 (&P)[16], float inv, uin
     if constexpr (BITS == 2) {
       w[0] += __float_as_uint(t.x) << (2 * m);
       w[1] += __float_as_uint(t.y) << (2 * m);
-    } else {
+    } else if constexpr (BITS == 4) {
       w[m / 8] += __float_as_uint(t.x) << (4 * (m % 8));
       w[2 + m / 8] += __float_as_uint(t.y) << (4 * (m % 8));
+    } else {
+      w[m / 4] += __float_as_uint(t.x) << (8 * (m % 4));
+      w[4 + m / 4] += __float_as_uint(t.y) << (8 * (m % 4));
     }
     const float2 fl = fsub2(t, mg);                 // floor(u)
     const float2 lv = __ffma2_rn(fl, two, one);     // level 2 floor(u) + 1 = 2c - (2^b - 1)
+    if constexpr (WANT_LV) lv_out[m] = lv;
     dot = __ffma2_rn(P[m], lv, dot);
-    if constexpr (BITS == 4) nrm = __ffma2_rn(lv, lv, nrm);
+    if constexpr (BITS != 2) nrm = __ffma2_rn(lv, lv, nrm);
   }
   // every field received (0x4B400000 + floor(u)); code c = floor(u) + 2^(b-1)
   constexpr uint32_t kOff = kFloorMagicBits - (1u << (BITS - 1));
-  constexpr uint32_t kSpread = BITS == 2 ? 0x55555555u : 0x11111111u;
+  constexpr uint32_t kSpread =
+      BITS == 2 ? 0x55555555u : (BITS == 4 ? 0x11111111u : 0x01010101u);
 #pragma unroll
   for (int k = 0; k < BITS; ++k) w[k] -= kOff * kSpread;
   float d = dot.x + dot.y, n;
@@ -183,10 +189,10 @@ __device__ __forceinline__ void quant_pass(const float2 (&P)[16], float inv, uin
 // then `iters` least-squares refits (nearest level of the current scale,
 // then the scale refitted); a group whose scale is below FLT_MIN keeps its
 // codes.  The loop runs the same number of times in every lane.
-template <int BITS, int GROUP, int RPW>
+template <int BITS, int GROUP, int RPW, bool WANT_Z = false>
 __device__ __forceinline__ void quantize_store(const float2 (&P)[16], uint32_t* codes_row,
                                                uint16_t* scales_row, int q, bool valid,
-                                               int iters) {
+                                               int iters, float2* z = nullptr) {
   float amax = 0.0f;
 #pragma unroll
   for (int m = 0; m < 16; ++m) amax = fmax3_abs(amax, P[m].x, P[m].y);
@@ -195,7 +201,7 @@ __device__ __forceinline__ void quantize_store(const float2 (&P)[16], uint32_t* 
   const float inv = (amax < 1.17549435e-38f) ? 0.0f : __fdiv_rn(outer, amax);
   uint32_t w[BITS];
   float d, n;
-  quant_pass<BITS, GROUP, RPW, false>(P, inv, w, d, n);
+  quant_pass<BITS, GROUP, RPW, false, WANT_Z>(P, inv, w, d, n, z);
   float s = d / n;                                  // least-squares scale
   for (int k = 0; k < iters; ++k) {
     const bool live = s >= 1.17549435e-38f;
@@ -209,15 +215,71 @@ __device__ __forceinline__ void quantize_store(const float2 (&P)[16], uint32_t* 
     }
   }
   s = fminf(fmaxf(s, -65504.0f), 65504.0f);
+  const __half s16 = __float2half_rn(s);
+  if constexpr (WANT_Z) {
+    // the reconstructed rotated row s16 * l (exact: 11 x 9 significant bits)
+    const float sf = __half2float(s16);
+    const float2 s2 = make_float2(sf, sf);
+#pragma unroll
+    for (int m = 0; m < 16; ++m) z[m] = __fmul2_rn(z[m], s2);
+  }
   if (!valid) return;
-  if constexpr (BITS == 2)
+  if constexpr (BITS == 2) {
     *reinterpret_cast<uint2*>(codes_row + 2 * q) = make_uint2(w[0], w[1]);
-  else
+  } else if constexpr (BITS == 4) {
     *reinterpret_cast<uint4*>(codes_row + 4 * q) = make_uint4(w[0], w[1], w[2], w[3]);
+  } else {
+    uint4* o = reinterpret_cast<uint4*>(codes_row + 8 * q);
+    o[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    o[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  }
   if (GROUP == 32)
-    scales_row[q] = __half_as_ushort(__float2half_rn(s));
+    scales_row[q] = __half_as_ushort(s16);
   else if (!(q & 1))
-    scales_row[q >> 1] = __half_as_ushort(__float2half_rn(s));
+    scales_row[q >> 1] = __half_as_ushort(s16);
+}
+
+// the row's 32 coordinates of this lane, v (signs applied), rotated in place
+// into P[m] = {y_m, y_{m+16}}: Walsh-Hadamard strides ascending, a butterfly
+// (a + b, a - b), then x c_d
+template <int D, int LPR, int RPW>
+__device__ __forceinline__ void rotate_lane(const float (&v)[32], float2 (&P)[16], int q) {
+#pragma unroll
+  for (int m = 0; m < 16; ++m) P[m] = make_float2(v[m], v[m + 16]);
+#pragma unroll
+  for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+      if (!(m & h)) {
+        const float2 a = P[m], b = P[m + h];
+        P[m] = __fadd2_rn(a, b);
+        P[m + h] = fsub2(a, b);
+      }
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < 16; ++m) {
+    const float a = P[m].x, b = P[m].y;
+    P[m] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
+  }
+#pragma unroll
+  for (int k = 1; k < LPR; k <<= 1) {
+    // the lower partner keeps a + b, the upper one a - b (fma with +-1 is
+    // exactly one rounded add or subtract)
+    const float sg = (q & k) ? -1.0f : 1.0f;
+    const float2 sg2 = make_float2(sg, sg);
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+      float2 o;
+      o.x = __shfl_xor_sync(kFull, P[m].x, RPW * k);
+      o.y = __shfl_xor_sync(kFull, P[m].y, RPW * k);
+      P[m] = __ffma2_rn(sg2, P[m], o);
+    }
+  }
+  const float cd = rot_scale<D>();
+  const float2 cd2 = make_float2(cd, cd);
+#pragma unroll
+  for (int m = 0; m < 16; ++m) P[m] = __fmul2_rn(P[m], cd2);
 }
 
 template <int D, int GROUP, int CW>
@@ -283,7 +345,6 @@ encode_tma_kernel(const __grid_constant__ EncodeTmaParams tp) {
   const int rw = lane % C::RPW;          // row within the warp
   const int q = lane / C::RPW;           // which 32 coordinates of the row
   const int r = warp * C::RPW + rw;      // row within the tile
-  const float cd = rot_scale<D>();
   long long it = 0;
   for (int t = blockIdx.x; t < tp.n_tiles; t += gridDim.x) {
     const long long idx = (long long)t * C::R + r;
@@ -308,8 +369,13 @@ encode_tma_kernel(const __grid_constant__ EncodeTmaParams tp) {
       for (int i = 0; i < 4; ++i)
         o[i] = make_uint4(wv[4 * i], wv[4 * i + 1], wv[4 * i + 2], wv[4 * i + 3]);
     }
-    float nref[32];
-    {
+    // BF16 reference: -D_i ref_i for the residual fma of every loop.
+    // Compressed reference: the rotated reference is quantised (its codes
+    // stored) and zr holds its reconstruction s16 * l, subtracted from every
+    // loop's rotated row.
+    float zr[32];
+    const bool cr = p.ref_bits != 0;
+    if (!cr) {
       const uint4* nd4 = reinterpret_cast<const uint4*>(ndtab + q * 16);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -317,9 +383,37 @@ encode_tma_kernel(const __grid_constant__ EncodeTmaParams tp) {
         const uint32_t ndw[4] = {nd.x, nd.y, nd.z, nd.w};
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          nref[8 * i + 2 * k] = fma_bf16<0>(wv[4 * i + k], ndw[k], 0.0f);
-          nref[8 * i + 2 * k + 1] = fma_bf16<1>(wv[4 * i + k], ndw[k], 0.0f);
+          zr[8 * i + 2 * k] = fma_bf16<0>(wv[4 * i + k], ndw[k], 0.0f);
+          zr[8 * i + 2 * k + 1] = fma_bf16<1>(wv[4 * i + k], ndw[k], 0.0f);
         }
+      }
+    } else {
+      float v[32];
+      const uint4* d4 = reinterpret_cast<const uint4*>(dtab + q * 16);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint4 dd = d4[i];
+        const uint32_t dw[4] = {dd.x, dd.y, dd.z, dd.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          v[8 * i + 2 * k] = fma_bf16<0>(wv[4 * i + k], dw[k], 0.0f);        // D_i ref_i
+          v[8 * i + 2 * k + 1] = fma_bf16<1>(wv[4 * i + k], dw[k], 0.0f);
+        }
+      }
+      float2 P[16], Z[16];
+      rotate_lane<D, C::LPR, C::RPW>(v, P, q);
+      if (p.ref_bits == 8)
+        quantize_store<8, GROUP, C::RPW, true>(P, p.ref_codes + (size_t)row * (D / 4),
+                                               p.ref_scales + (size_t)row * (D / GROUP), q,
+                                               valid, 0, Z);
+      else
+        quantize_store<4, GROUP, C::RPW, true>(P, p.ref_codes + (size_t)row * (D / 8),
+                                               p.ref_scales + (size_t)row * (D / GROUP), q,
+                                               valid, 0, Z);
+#pragma unroll
+      for (int m = 0; m < 16; ++m) {
+        zr[m] = Z[m].x;
+        zr[m + 16] = Z[m].y;
       }
     }
 
@@ -334,7 +428,8 @@ encode_tma_kernel(const __grid_constant__ EncodeTmaParams tp) {
       if (lane == 0) mbar_arrive(&empty[s]);
       ++it;
 
-      // residual with the seeded signs: y = D_i x_i + (-D_i ref_i), one rounding
+      // BF16 reference: y = D_i x_i + (-D_i ref_i), one rounding, then rotated.
+      // Compressed reference: D_i x_i (exact), rotated, then e = RN(y - zr).
       float v[32];
       {
         const uint4* d4 = reinterpret_cast<const uint4*>(dtab + q * 16);
@@ -344,48 +439,19 @@ encode_tma_kernel(const __grid_constant__ EncodeTmaParams tp) {
           const uint32_t dw[4] = {dd.x, dd.y, dd.z, dd.w};
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            v[8 * i + 2 * k] = fma_bf16<0>(wv[4 * i + k], dw[k], nref[8 * i + 2 * k]);
-            v[8 * i + 2 * k + 1] = fma_bf16<1>(wv[4 * i + k], dw[k], nref[8 * i + 2 * k + 1]);
+            const float a0 = cr ? 0.0f : zr[8 * i + 2 * k];
+            const float a1 = cr ? 0.0f : zr[8 * i + 2 * k + 1];
+            v[8 * i + 2 * k] = fma_bf16<0>(wv[4 * i + k], dw[k], a0);
+            v[8 * i + 2 * k + 1] = fma_bf16<1>(wv[4 * i + k], dw[k], a1);
           }
         }
       }
       float2 P[16];
+      rotate_lane<D, C::LPR, C::RPW>(v, P, q);
+      if (cr) {
 #pragma unroll
-      for (int m = 0; m < 16; ++m) P[m] = make_float2(v[m], v[m + 16]);
-      // Walsh-Hadamard, ascending strides; a butterfly is (a + b, a - b)
-#pragma unroll
-      for (int h = 1; h < 16; h <<= 1) {
-#pragma unroll
-        for (int m = 0; m < 16; ++m) {
-          if (!(m & h)) {
-            const float2 a = P[m], b = P[m + h];
-            P[m] = __fadd2_rn(a, b);
-            P[m + h] = fsub2(a, b);
-          }
-        }
+        for (int m = 0; m < 16; ++m) P[m] = fsub2(P[m], make_float2(zr[m], zr[m + 16]));
       }
-#pragma unroll
-      for (int m = 0; m < 16; ++m) {
-        const float a = P[m].x, b = P[m].y;
-        P[m] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
-      }
-#pragma unroll
-      for (int k = 1; k < C::LPR; k <<= 1) {
-        // the lower partner keeps a + b, the upper one a - b (fma with +-1 is
-        // exactly one rounded add or subtract)
-        const float sg = (q & k) ? -1.0f : 1.0f;
-        const float2 sg2 = make_float2(sg, sg);
-#pragma unroll
-        for (int m = 0; m < 16; ++m) {
-          float2 o;
-          o.x = __shfl_xor_sync(kFull, P[m].x, C::RPW * k);
-          o.y = __shfl_xor_sync(kFull, P[m].y, C::RPW * k);
-          P[m] = __ffma2_rn(sg2, P[m], o);
-        }
-      }
-      const float2 cd2 = make_float2(cd, cd);
-#pragma unroll
-      for (int m = 0; m < 16; ++m) P[m] = __fmul2_rn(P[m], cd2);
 
       const int l = tp.active[j];
       if (p.bits[l] == 2)

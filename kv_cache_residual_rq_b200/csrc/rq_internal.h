@@ -55,6 +55,9 @@ struct EncodeParams {
   int dst_pitch, dst_offset;         // token pitch / first token of the outputs
   int n_loops;
   int refine_iters;                  // least-squares refits after the absmax codes
+  int ref_bits;                      // 0: BF16 reference; 4 or 8: compressed reference
+  uint32_t* ref_codes;               // compressed reference: codes and scales out
+  uint16_t* ref_scales;
   uint64_t seed;
 };
 
@@ -74,7 +77,9 @@ cudaError_t encode_take_status(uint32_t* bits);
 // reconstruction (the format's decoder)
 // ---------------------------------------------------------------------------
 struct ReconstructParams {
-  const uint16_t* ref;
+  const uint16_t* ref;        // BF16 reference rows (null for a compressed reference)
+  const uint32_t* ref_codes;  // compressed reference: codes and fp16 scales
+  const uint16_t* ref_scales;
   const uint32_t* codes;      // unused for bits 16
   const uint16_t* scales;
   void* out;                  // fp32 or bf16 rows
@@ -86,6 +91,9 @@ struct ReconstructParams {
 
 cudaError_t launch_reconstruct(int head_dim, int group, int bits, const ReconstructParams& p,
                                int num_sms, cudaStream_t stream);
+// compressed reference with ref_bits (4 or 8); bits 16 = the reference loop
+cudaError_t launch_reconstruct_cr(int head_dim, int group, int ref_bits, int bits,
+                                  const ReconstructParams& p, int num_sms, cudaStream_t stream);
 
 // ---------------------------------------------------------------------------
 // decode attention
@@ -142,6 +150,11 @@ struct DecodeParams {
   const uint16_t* tail_k;   // optional BF16 tail tokens [heads][tail_pitch][d]
   const uint16_t* tail_v;
   int n_tail, tail_pitch;
+  int ref_bits;          // 0: BF16 reference rows; 4 or 8: compressed reference
+  const uint32_t* rcodes_k;   // compressed reference: codes and fp16 scales
+  const uint32_t* rcodes_v;
+  const uint16_t* rscales_k;
+  const uint16_t* rscales_v;
   const int* ctx_lens;   // variable-length call: cached tokens per sequence
                          // [batch] (device int32), else null (ctx for all)
   int nt;

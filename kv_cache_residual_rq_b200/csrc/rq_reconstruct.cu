@@ -17,7 +17,9 @@ namespace {
 
 constexpr int kThreads = 256;
 
-template <int D, int GROUP, int BITS, bool OUT_BF16>
+// RB: 0 = BF16 reference rows; 4 or 8 = compressed reference (codes and
+// scales in the rotated domain: out = Rot^T (s_ref l_ref + s l))
+template <int D, int GROUP, int BITS, bool OUT_BF16, int RB>
 __global__ void __launch_bounds__(kThreads)
 reconstruct_kernel(const ReconstructParams p) {
   constexpr int DPL = 8;
@@ -44,21 +46,44 @@ reconstruct_kernel(const ReconstructParams p) {
     const long long hd = idx / p.ctx, t = idx % p.ctx;
     const long long row = hd * p.pitch + t;
     const size_t eoff = (size_t)row * D + li * DPL;
-    const uint4 rw = valid ? __ldcs(reinterpret_cast<const uint4*>(p.ref + eoff))
-                           : make_uint4(0, 0, 0, 0);
+    uint4 rw = make_uint4(0, 0, 0, 0);
+    if constexpr (RB == 0) {
+      if (valid) rw = __ldcs(reinterpret_cast<const uint4*>(p.ref + eoff));
+    }
     float v[DPL];
-    if constexpr (BITS != 16) {
+    float vr[DPL];                    // compressed reference: s_ref l_ref
+#pragma unroll
+    for (int k = 0; k < DPL; ++k) vr[k] = 0.0f;
+    if constexpr (RB != 0) {
+      constexpr int RTOP = (1 << RB) - 1;
+      uint32_t rc[2] = {0u, 0u};
+      float sr = 0.0f;
+      if (valid) {
+        const uint32_t* cw = p.ref_codes + (size_t)row * (D * RB / 32) + li * DPL * RB / 32;
+        rc[0] = cw[0];
+        if constexpr (RB == 8) rc[1] = cw[1];
+        sr = __half2float(__ushort_as_half(p.ref_scales[(size_t)row * (D / GROUP) + li / LPG]));
+      }
+#pragma unroll
+      for (int k = 0; k < DPL; ++k) {
+        const int c = (int)((rc[(k * RB) / 32] >> ((k * RB) % 32)) & (uint32_t)RTOP);
+        vr[k] = sr * (float)(2 * c - RTOP);
+      }
+    }
+    if constexpr (BITS != 16 || RB != 0) {
       uint32_t x = 0;
       float s = 0.0f;
-      if (valid) {
-        const int bit0 = li * DPL * BITS;
-        x = p.codes[(size_t)row * (D * BITS / 32) + bit0 / 32] >> (bit0 % 32);
-        s = __half2float(__ushort_as_half(p.scales[(size_t)row * (D / GROUP) + li / LPG]));
+      if constexpr (BITS != 16) {
+        if (valid) {
+          const int bit0 = li * DPL * BITS;
+          x = p.codes[(size_t)row * (D * BITS / 32) + bit0 / 32] >> (bit0 % 32);
+          s = __half2float(__ushort_as_half(p.scales[(size_t)row * (D / GROUP) + li / LPG]));
+        }
       }
 #pragma unroll
       for (int k = 0; k < DPL; ++k) {
         const int c = (int)((x >> (BITS * k)) & (uint32_t)TOP);
-        v[k] = s * (float)(2 * c - TOP);
+        v[k] = (BITS == 16) ? vr[k] : vr[k] + s * (float)(2 * c - TOP);
       }
       // Rot^T: butterflies (strides 1, 2, 4 in registers, the rest across lanes)
 #pragma unroll
@@ -112,7 +137,7 @@ reconstruct_kernel(const ReconstructParams p) {
   }
 }
 
-template <int D, int GROUP, int BITS>
+template <int D, int GROUP, int BITS, int RB = 0>
 cudaError_t launch_t(const ReconstructParams& p, int num_sms, cudaStream_t stream) {
   constexpr int rows_per_block = kThreads / 32 * (32 / (D / 8));
   long long blocks = (p.n_rows + rows_per_block - 1) / rows_per_block;
@@ -120,9 +145,9 @@ cudaError_t launch_t(const ReconstructParams& p, int num_sms, cudaStream_t strea
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
   if (p.out_bf16)
-    reconstruct_kernel<D, GROUP, BITS, true><<<(unsigned)blocks, kThreads, 0, stream>>>(p);
+    reconstruct_kernel<D, GROUP, BITS, true, RB><<<(unsigned)blocks, kThreads, 0, stream>>>(p);
   else
-    reconstruct_kernel<D, GROUP, BITS, false><<<(unsigned)blocks, kThreads, 0, stream>>>(p);
+    reconstruct_kernel<D, GROUP, BITS, false, RB><<<(unsigned)blocks, kThreads, 0, stream>>>(p);
   return cudaGetLastError();
 }
 
@@ -134,7 +159,32 @@ cudaError_t launch_g(int bits, const ReconstructParams& p, int num_sms, cudaStre
   return cudaErrorInvalidValue;
 }
 
+template <int D, int GROUP, int RB>
+cudaError_t launch_cr_b(int bits, const ReconstructParams& p, int num_sms, cudaStream_t stream) {
+  if (bits == 2) return launch_t<D, GROUP, 2, RB>(p, num_sms, stream);
+  if (bits == 4) return launch_t<D, GROUP, 4, RB>(p, num_sms, stream);
+  if (bits == 16) return launch_t<D, GROUP, 16, RB>(p, num_sms, stream);
+  return cudaErrorInvalidValue;
+}
+
+template <int D, int GROUP>
+cudaError_t launch_cr_g(int ref_bits, int bits, const ReconstructParams& p, int num_sms,
+                        cudaStream_t stream) {
+  if (ref_bits == 8) return launch_cr_b<D, GROUP, 8>(bits, p, num_sms, stream);
+  if (ref_bits == 4) return launch_cr_b<D, GROUP, 4>(bits, p, num_sms, stream);
+  return cudaErrorInvalidValue;
+}
+
 }  // namespace
+
+cudaError_t launch_reconstruct_cr(int head_dim, int group, int ref_bits, int bits,
+                                  const ReconstructParams& p, int num_sms, cudaStream_t stream) {
+  if (head_dim == 128 && group == 32) return launch_cr_g<128, 32>(ref_bits, bits, p, num_sms, stream);
+  if (head_dim == 128 && group == 64) return launch_cr_g<128, 64>(ref_bits, bits, p, num_sms, stream);
+  if (head_dim == 64 && group == 32) return launch_cr_g<64, 32>(ref_bits, bits, p, num_sms, stream);
+  if (head_dim == 64 && group == 64) return launch_cr_g<64, 64>(ref_bits, bits, p, num_sms, stream);
+  return cudaErrorInvalidValue;
+}
 
 cudaError_t launch_reconstruct(int head_dim, int group, int bits, const ReconstructParams& p,
                                int num_sms, cudaStream_t stream) {

@@ -104,6 +104,36 @@ def measure(w, reps, peak, emit):
               "tokens_per_s_per_head_call": w.batch / t})
     assert rq.rq_workspace_status(ws) == 0
     if w.G == 1 and w.name == "ouro1.4b_decode":
+        # compressed reference (reference loop as rotated INT8 / INT4 codes)
+        xk1 = synth.loop_kv(w, 0, 0, 1, refk)
+        xv1 = synth.loop_kv(w, 0, 1, 1, refv)
+        for rb in (8, 4):
+            t = _time(lambda: rq.encode_cr([xk1], refk, rb, [2], w.group, w.seed), reps, flush)
+            nb_e = (rows * w.head_dim * 2 * 2 + rows * (w.head_dim * (rb + 2) // 8
+                                                      + 2 * 2 * (w.head_dim // w.group)))
+            emit({"workload": w.name, "kernel": f"encode compressed ref INT{rb} + 1 loop INT2",
+                  "us": t * 1e6, "bytes": nb_e, "gbs": nb_e / t / 1e9,
+                  "frac": nb_e / t / 1e9 / peak})
+            (rck, rsk), ckc, skc = rq.encode_cr([xk1], refk, rb, [2], w.group, w.seed)
+            (rcv, rsv), cvc, svc = rq.encode_cr([xv1], refv, rb, [2], w.group, w.seed)
+            heads_t = w.batch * w.kv_heads * w.ctx
+            for b in (2, 16):
+                per_tok = 2 * (w.head_dim * rb // 8 + 2 * (w.head_dim // w.group))
+                if b != 16:
+                    per_tok += 2 * (w.head_dim * b // 8 + 2 * (w.head_dim // w.group))
+                nb = heads_t * per_tok + w.batch * w.q_heads * w.head_dim * 6
+                args = (ckc[0], cvc[0], skc[0], svc[0]) if b != 16 else (None,) * 4
+                fn = lambda: rq.rq_decode_attention_cr(shape, None, q, rck, rcv, rsk, rsv, rb,
+                                                       *args, b, w.seed, 0.0, None, None, 0, 0,
+                                                       out, ws)
+                t = _time(fn, reps, None)
+                emit({"workload": w.name, "kernel": f"decode compressed ref INT{rb} bits={b}",
+                      "G": w.G, "us": t * 1e6, "bytes": nb, "gbs": nb / t / 1e9,
+                      "frac": nb / t / 1e9 / peak})
+            assert rq.rq_workspace_status(ws) == 0
+            del rck, rsk, ckc, skc, rcv, rsv, cvc, svc
+        del xk1, xv1
+        torch.cuda.empty_cache()
         # variable-length batch: seeded lengths in [ctx/8, ctx], the cache at
         # full capacity; bytes are those of the tokens actually present
         g = torch.Generator().manual_seed(w.seed * 977 + 5)

@@ -67,6 +67,34 @@ def study(w, emit):
                 del c, s, xh
             del x, xf
             torch.cuda.empty_cache()
+    # compressed reference: the final loop itself as rotated INT8 / INT4 codes,
+    # the other loops as residuals against its reconstruction
+    for kind, name in ((0, "K"), (1, "V")):
+        ref = synth.reference(w, 0, kind, dev)
+        xs = [synth.loop_kv(w, 0, kind, l, ref) for l in range(1, w.loops)]
+        rbits = [b if b != 16 else 2 for b in w.bits]
+        for rb in (8, 4):
+            (rc, rs), codes, scales = rq.encode_cr(xs, ref, rb, rbits, w.group, w.seed)
+            bpp = (rb + 16.0 / w.group) + sum(b + 16.0 / w.group for b in rbits)
+            xh = rq.reconstruct_cr(ref.shape, rc, rs, rb, None, None, 16, w.group, w.seed)
+            rf = ref.float()
+            emit({"workload": w.name, "tensor": name, "loop": w.loops,
+                  "scheme": f"compressed_ref_int{rb}", "bits": rb,
+                  "rel_recon_err": (torch.linalg.vector_norm(xh - rf) /
+                                    torch.linalg.vector_norm(rf)).item(),
+                  "bits_per_position_all_loops": bpp})
+            for l in range(1, w.loops):
+                xf = xs[l - 1].float()
+                xh = rq.reconstruct_cr(ref.shape, rc, rs, rb, codes[l - 1], scales[l - 1],
+                                       rbits[l - 1], w.group, w.seed)
+                emit({"workload": w.name, "tensor": name, "loop": l,
+                      "scheme": f"compressed_ref_int{rb}", "bits": rbits[l - 1],
+                      "rel_recon_err": (torch.linalg.vector_norm(xh - xf) /
+                                        torch.linalg.vector_norm(xf)).item(),
+                      "bits_per_position_all_loops": bpp})
+            del rc, rs, codes, scales, xh
+        del xs
+        torch.cuda.empty_cache()
     # attention output: quantise loop 1 (the most sensitive) of both K and V
     refk = synth.reference(w, 0, 0, dev)
     refv = synth.reference(w, 0, 1, dev)
@@ -88,6 +116,16 @@ def study(w, emit):
         err = (torch.linalg.vector_norm(out - exact) / torch.linalg.vector_norm(exact)).item()
         emit({"workload": w.name, "tensor": "attention(loop 1)", "scheme": scheme, "bits": bits,
               "rel_output_err": err})
+    if G == 1:
+        for rb in (8, 4):
+            b1 = w.bits[0] if w.bits[0] != 16 else 2
+            (rck, rsk), ck, sk = rq.encode_cr([xk], refk, rb, [b1], w.group, w.seed)
+            (rcv, rsv), cv, sv = rq.encode_cr([xv], refv, rb, [b1], w.group, w.seed)
+            out = rq.decode_attention_cr(q, (rck, rsk, rcv, rsv, rb), ck[0], cv[0], sk[0], sv[0],
+                                         b1, w.group, w.seed, refk.shape[2])
+            err = (torch.linalg.vector_norm(out - exact) / torch.linalg.vector_norm(exact)).item()
+            emit({"workload": w.name, "tensor": "attention(loop 1)",
+                  "scheme": f"compressed_ref_int{rb}", "bits": b1, "rel_output_err": err})
 
 
 def main(argv=None):
