@@ -163,6 +163,33 @@ __host__ __device__ constexpr float ref_pos_factor(int k) {
   return RB == 8 ? ((k & 1) ? 1.0f / 256.0f : 1.0f) : pos_factor<4, DPL>(k);
 }
 
+// sum_k a_k b_k + c over 4 byte lanes, a signed or unsigned, b unsigned
+__device__ __forceinline__ int dp4a_su(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ int dp4a_uu(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.u32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// acc + w * (1024 + c) for the half (0 low, 1 high) of a packed pair of fp16
+// values 0x6400 | c, w an fp16 weight: one rounding, fp32 accumulator
+template <int H>
+__device__ __forceinline__ float fma_f16_half(uint32_t w16x2, uint32_t cpair, float acc) {
+  if constexpr (H == 0)
+    asm("{\n\t.reg .b16 wl, wh, cl, ch;\n\tmov.b32 {wl, wh}, %1;\n\tmov.b32 {cl, ch}, %2;\n\t"
+        "fma.rn.f32.f16 %0, wl, cl, %0;\n\t}"
+        : "+f"(acc) : "r"(w16x2), "r"(cpair));
+  else
+    asm("{\n\t.reg .b16 wl, wh, cl, ch;\n\tmov.b32 {wl, wh}, %1;\n\tmov.b32 {cl, ch}, %2;\n\t"
+        "fma.rn.f32.f16 %0, wl, ch, %0;\n\t}"
+        : "+f"(acc) : "r"(w16x2), "r"(cpair));
+  return acc;
+}
+
 template <int D, int G, int BITS, int RB>
 __global__ void __launch_bounds__(kThreads, 2)
 decode_kernel(const DecodeParams p) {
@@ -323,6 +350,10 @@ decode_kernel(const DecodeParams p) {
   float2 qr[G][NP];                   // compressed reference: 2 q~ 2^-pos
   float roff[G];                      // compressed reference: (2^RB - 1) sum q~ (lane dims)
   float wsumR[G];                     // compressed reference: sum of p s_ref^V
+  // INT8 compressed reference: q~ of the lane's dims as 16-bit fixed point
+  // (step qsig), split into signed high and unsigned low bytes for dp4a
+  uint32_t qhi[G][2], qlo[G][2];
+  float qsig[G];
   float2 qc[G][NP];                   // 2 q~ 2^-pos (codes at their bit position)
   float qoff[G];                      // (2^b - 1) * sum q~ over the lane's dims
   // running state
@@ -394,6 +425,24 @@ decode_kernel(const DecodeParams p) {
       }
       qoff[r] = (float)TOPLVL * sum;
       roff[r] = (float)((1 << (RB ? RB : 1)) - 1) * sum;
+      if constexpr (RB == 8 && DPL == 8) {
+        float t[8], mx = 0.0f;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          t[k] = cd * qt[r * D + dim0 + k];
+          mx = fmaxf(mx, fabsf(t[k]));
+        }
+        const float sig = fmaxf(mx, 1e-30f) * (1.0f / 32512.0f);   // |Q| <= 127 * 256
+        const float inv_sig = 1.0f / sig;
+        qsig[r] = sig;
+        qhi[r][0] = qhi[r][1] = qlo[r][0] = qlo[r][1] = 0u;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int Q = __float2int_rn(t[k] * inv_sig);
+          qhi[r][k / 4] |= ((uint32_t)(Q >> 8) & 0xFFu) << (8 * (k % 4));
+          qlo[r][k / 4] |= ((uint32_t)Q & 0xFFu) << (8 * (k % 4));
+        }
+      }
     }
   };
 
@@ -450,8 +499,14 @@ decode_kernel(const DecodeParams p) {
           } else {
             // the reference is in the rotated domain too: accV holds its codes
             constexpr float RT = (float)((1 << RB) - 1);
-            z0 += 2.0f * ref_pos_factor<RB, DPL>(2 * j) * accV[r][j].x - RT * wsumR[r];
-            z1 += 2.0f * ref_pos_factor<RB, DPL>(2 * j + 1) * accV[r][j].y - RT * wsumR[r];
+            if constexpr (RB == 8 && DPL == 8) {
+              // accV = sum w (1024 + c): sum w l = 2 accV - (2048 + RT) sum w
+              z0 += 2.0f * accV[r][j].x - (2048.0f + RT) * wsumR[r];
+              z1 += 2.0f * accV[r][j].y - (2048.0f + RT) * wsumR[r];
+            } else {
+              z0 += 2.0f * ref_pos_factor<RB, DPL>(2 * j) * accV[r][j].x - RT * wsumR[r];
+              z1 += 2.0f * ref_pos_factor<RB, DPL>(2 * j + 1) * accV[r][j].y - RT * wsumR[r];
+            }
             rec[2 + dim0 + 2 * j] = 0.0f;
             rec[2 + dim0 + 2 * j + 1] = 0.0f;
           }
@@ -468,6 +523,13 @@ decode_kernel(const DecodeParams p) {
 
   // compressed reference: <q~, l_ref> of the lane's dims (without s_ref)
   auto ref_code_dot = [&](const unsigned char* kp, int r) {
+    if constexpr (RB == 8 && DPL == 8) {
+      // sum_k Q_k c_k exactly in integers: Q = 256 hi + lo
+      const uint2 w = *reinterpret_cast<const uint2*>(kp);
+      const int dh = dp4a_su(qhi[r][1], w.y, dp4a_su(qhi[r][0], w.x, 0));
+      const int dl = dp4a_uu(qlo[r][1], w.y, dp4a_uu(qlo[r][0], w.x, 0));
+      return fmaf(2.0f * qsig[r], __int2float_rn(dh * 256 + dl), -roff[r]);
+    }
     float f[DPL];
     ref_codes_positional<RB ? RB : 4, DPL>(kp, f);
     float2 acc = make_float2(-roff[r], 0.0f);
@@ -617,6 +679,21 @@ decode_kernel(const DecodeParams p) {
         float s_rv = 1.0f;
         if constexpr (RB == 0) {
           v_pairs(st + C::OFF_V + tok * C::KROW + dim0 * 2, vf);
+        } else if constexpr (RB == 8 && DPL == 8) {
+          // codes as exact fp16 values 1024 + c, weight p s_ref^V rounded to
+          // fp16 once (the same rounded weight goes into the offset sum)
+          s_rv = half_at(st + C::OFF_RSV + sc_off + tok * SB + grp * 2);
+          const __half w16 = __float2half_rn(pu * s_rv);
+          const uint32_t w2 = (uint32_t)__half_as_ushort(w16) * 0x10001u;
+          wsumR[0] += __half2float(w16);
+          const uint2 cw2 = *reinterpret_cast<const uint2*>(st + C::OFF_V + tok * C::KROW + dim0);
+#pragma unroll
+          for (int j = 0; j < NP; ++j) {
+            const uint32_t src = j < 2 ? cw2.x : cw2.y;
+            const uint32_t cp = __byte_perm(src, 0x64646464u, (j & 1) ? 0x7362u : 0x5140u);
+            accV[0][j].x = fma_f16_half<0>(w2, cp, accV[0][j].x);
+            accV[0][j].y = fma_f16_half<1>(w2, cp, accV[0][j].y);
+          }
         } else {
           float f[DPL];
           ref_codes_positional<RB ? RB : 4, DPL>(st + C::OFF_V + tok * C::KROW + dim0 * RB / 8, f);
@@ -629,7 +706,18 @@ decode_kernel(const DecodeParams p) {
           code_pairs(reinterpret_cast<const uint32_t*>(st + C::OFF_CV)[tok * C::CWORDS + cw], cf);
           s_v = half_at(st + C::OFF_SV + sc_off + tok * SB + grp * 2);
         }
-        accumulate_v(0, pu, vf, cf, s_v, s_rv);
+        if constexpr (RB == 8 && DPL == 8) {
+          // reference part done above; only the residual remains
+          if constexpr (C::RES) {
+            const float wv = pu * s_v;
+            const float2 w2 = make_float2(wv, wv);
+            wsum[0] += wv;
+#pragma unroll
+            for (int j = 0; j < NP; ++j) accC[0][j] = __ffma2_rn(w2, cf[j], accC[0][j]);
+          }
+        } else {
+          accumulate_v(0, pu, vf, cf, s_v, s_rv);
+        }
       }
     }
   };
