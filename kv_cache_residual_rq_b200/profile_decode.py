@@ -29,6 +29,8 @@ def main(argv=None):
     ap.add_argument("--encode", action="store_true", help="also time rq_encode of the layer")
     ap.add_argument("--tail", type=int, default=0,
                     help="BF16 tail tokens per call (1 = the benchmark's launch: cache + new token)")
+    ap.add_argument("--ref-bits", type=int, default=0,
+                    help="4 or 8: decode a compressed-reference cache instead")
     args = ap.parse_args(argv)
     w = synth.BY_NAME[args.workload]
     bits = args.bits or w.bits[0]
@@ -61,10 +63,25 @@ def main(argv=None):
         tail_k = torch.randn((w.batch, w.kv_heads, args.tail, w.head_dim), generator=g,
                              device=dev).to(torch.bfloat16)
         tail_v = torch.randn(tail_k.shape, generator=g, device=dev).to(torch.bfloat16)
+    crref = None
+    if args.ref_bits:
+        xk1 = synth.loop_kv(w, 0, 0, 1, refk)
+        xv1 = synth.loop_kv(w, 0, 1, 1, refv)
+        b1 = bits if bits != 16 else 2
+        (rck, rsk), ckc, skc = rq.encode_cr([xk1], refk, args.ref_bits, [b1], w.group, w.seed)
+        (rcv, rsv), cvc, svc = rq.encode_cr([xv1], refv, args.ref_bits, [b1], w.group, w.seed)
+        crref = (rck, rsk, rcv, rsv, args.ref_bits)
+        del xk1, xv1
     for _ in range(args.calls):
         start.record()
-        rq.decode_attention(q, refk, refv, ck, cv, sk, sv, bits, w.group, w.seed, out=out,
-                            workspace=ws, tail_k=tail_k, tail_v=tail_v, n_tail=args.tail)
+        if crref is not None:
+            rq.decode_attention_cr(q, crref, *((ckc[0], cvc[0], skc[0], svc[0]) if bits != 16
+                                              else (None,) * 4), bits, w.group, w.seed, w.ctx,
+                                   out=out, workspace=ws, tail_k=tail_k, tail_v=tail_v,
+                                   n_tail=args.tail)
+        else:
+            rq.decode_attention(q, refk, refv, ck, cv, sk, sv, bits, w.group, w.seed, out=out,
+                                workspace=ws, tail_k=tail_k, tail_v=tail_v, n_tail=args.tail)
         end.record()
         torch.cuda.synchronize()
         times.append(start.elapsed_time(end))
