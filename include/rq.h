@@ -230,6 +230,28 @@ rq_status rq_encode_at_ex(const rq_shape *shape, int src_pitch, int src_offset,
                           uint16_t *const *scales_out, uint16_t *ref_out, void *stream);
 
 /*
+ * rq_encode_paged -- rq_encode_at_ex into paged pools (the layout read by
+ * rq_decode_attention_paged): token t of sequence b, head h of the sources
+ * is written at position pos = dst_pos[b] + t of that sequence, i.e. row
+ * (page_table[b][pos / 64] * Hkv + h) * 64 + pos % 64 of every pool.
+ *   kv_loops, ref : contiguous device bf16 [batch][Hkv][ctx][d] (the tokens
+ *                   to retire, e.g. one per sequence per decode step).
+ *   dst_pos       : DEVICE int32 [batch], first position written per sequence.
+ *   page_table    : DEVICE int32 [batch][max_pages]; pools of n_pages pages.
+ *   codes_out, scales_out : HOST arrays of device pool pointers, sized by
+ *                   rq_codes_bytes / rq_scales_bytes of a shape with batch =
+ *                   n_pages and ctx = 64.
+ *   ref_out       : optional bf16 reference pool [n_pages][Hkv][64][d].
+ * A position past the table or a page id outside the pool writes nothing.
+ * Arithmetic, refits and errors as rq_encode_at_ex.
+ */
+rq_status rq_encode_paged(const rq_shape *shape, const uint16_t *const *kv_loops, int n_loops,
+                          const uint16_t *ref, const uint8_t *bits_per_loop, uint64_t seed,
+                          int refine_iters, const int32_t *dst_pos, const int32_t *page_table,
+                          int max_pages, int n_pages, uint32_t *const *codes_out,
+                          uint16_t *const *scales_out, uint16_t *ref_out, void *stream);
+
+/*
  * rq_decode_attention -- fused ResidualQuant decode attention for one loop
  * (Abstract: the reconstruction stays efficient; the reduced KV traffic is
  * what speeds decode up).
@@ -354,6 +376,35 @@ rq_status rq_decode_attention_cr(const rq_shape *shape, const int32_t *ctx_lens,
                                  uint64_t seed, float softmax_scale, const uint16_t *tail_k,
                                  const uint16_t *tail_v, int n_tail, int tail_pitch, float *out,
                                  void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * rq_decode_attention_paged -- rq_decode_attention_varlen over paged caches:
+ * the cache is a pool of pages of 64 tokens (one decode tile), and each
+ * sequence's tokens live in the pages its row of a page table names.
+ *   page_table : DEVICE int32 [batch][max_pages], 4-byte aligned: tokens
+ *                64 j .. 64 j + 63 of sequence b are page page_table[b][j].
+ *                Entries past a sequence's length are not read.  An entry
+ *                outside 0 .. n_pages-1 is treated as an empty page and sets
+ *                status bit 32 (the pool is never addressed out of range).
+ *   ref_k, ref_v : pools bf16 [n_pages][Hkv][64][d];
+ *   codes_k/v, scales_k/v : pools [n_pages][Hkv][64][d*b/32] and [...][d/g]
+ *                (rq_codes_bytes / rq_scales_bytes of a shape with batch =
+ *                n_pages, ctx = 64).
+ *   shape      : ctx must equal max_pages * 64 (the capacity per sequence;
+ *                ctx_cap 0 or equal); workspace of
+ *                rq_decode_workspace_bytes_varlen(shape).
+ *   ctx_lens   : as rq_decode_attention_varlen (required).
+ * Everything else as rq_decode_attention_varlen; BF16 reference only.
+ */
+rq_status rq_decode_attention_paged(const rq_shape *shape, const int32_t *ctx_lens,
+                                    const int32_t *page_table, int max_pages, int n_pages,
+                                    const uint16_t *q, const uint16_t *ref_k,
+                                    const uint16_t *ref_v, const uint32_t *codes_k,
+                                    const uint32_t *codes_v, const uint16_t *scales_k,
+                                    const uint16_t *scales_v, int bits, uint64_t seed,
+                                    float softmax_scale, const uint16_t *tail_k,
+                                    const uint16_t *tail_v, int n_tail, int tail_pitch, float *out,
+                                    void *workspace, size_t workspace_bytes, void *stream);
 
 /* Workspace bytes for rq_decode_attention_varlen with this shape (any
  * lengths up to the capacity); 0 if the shape is unsupported. */

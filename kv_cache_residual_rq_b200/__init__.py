@@ -14,7 +14,7 @@ from ._abi import (RQ_ERR_ALIGNMENT, RQ_ERR_CUDA, RQ_ERR_INVALID_ARG, RQ_ERR_UNS
                    rq_encode_at_ex, rq_encode_take_status, rq_reconstruct, RQ_MAX_REFINE,
                    RQ_MAX_VARLEN_BATCH, rq_decode_attention_varlen,
                    rq_decode_workspace_bytes_varlen, rq_encode_cr_at, rq_reconstruct_cr,
-                   rq_decode_attention_cr,
+                   rq_decode_attention_cr, rq_decode_attention_paged, rq_encode_paged,
                    rq_scales_bytes, rq_shape, rq_status_string, rq_version,
                    rq_workspace_status)
 
@@ -25,7 +25,8 @@ __all__ = [
     "rq_encode", "rq_encode_at", "rq_encode_at_ex", "RQ_MAX_REFINE", "rq_decode_attention", "rq_decode_attention_tail",
     "rq_decode_attention_noalloc", "rq_decode_attention_varlen", "rq_decode_workspace_bytes_varlen",
     "RQ_MAX_VARLEN_BATCH", "rq_reconstruct", "rq_encode_cr_at", "rq_reconstruct_cr",
-    "rq_decode_attention_cr", "encode_cr", "reconstruct_cr", "decode_attention_cr", "rq_workspace_status", "rq_encode_take_status",
+    "rq_decode_attention_cr", "encode_cr", "reconstruct_cr", "decode_attention_cr",
+    "rq_decode_attention_paged", "rq_encode_paged", "rq_workspace_status", "rq_encode_take_status",
     "alloc_codes", "alloc_scales", "alloc_workspace", "encode", "decode_attention", "reconstruct",
 ]
 

@@ -112,6 +112,18 @@ def lib():
                                              c.c_int, c.c_int, c.c_void_p, c.c_void_p,
                                              c.c_size_t, c.c_void_p]
         L.rq_decode_attention_cr.restype = c.c_int
+        L.rq_decode_attention_paged.argtypes = [sp, c.c_void_p, c.c_void_p, c.c_int, c.c_int,
+                                                c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p,
+                                                c.c_void_p, c.c_void_p, c.c_void_p, c.c_int,
+                                                c.c_uint64, c.c_float, c.c_void_p, c.c_void_p,
+                                                c.c_int, c.c_int, c.c_void_p, c.c_void_p,
+                                                c.c_size_t, c.c_void_p]
+        L.rq_decode_attention_paged.restype = c.c_int
+        L.rq_encode_paged.argtypes = [sp, c.POINTER(c.c_void_p), c.c_int, c.c_void_p,
+                                      c.POINTER(c.c_uint8), c.c_uint64, c.c_int, c.c_void_p,
+                                      c.c_void_p, c.c_int, c.c_int, c.POINTER(c.c_void_p),
+                                      c.POINTER(c.c_void_p), c.c_void_p, c.c_void_p]
+        L.rq_encode_paged.restype = c.c_int
         L.rq_decode_attention_tail.argtypes = [sp, c.c_void_p, c.c_void_p, c.c_void_p,
                                                c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p,
                                                c.c_int, c.c_uint64, c.c_float, c.c_void_p,
@@ -356,4 +368,36 @@ def rq_decode_attention_cr(shape, ctx_lens, q, ref_codes_k, ref_codes_v, ref_sca
         int(workspace_bytes), _stream(stream))
     if check:
         _check(st, "rq_decode_attention_cr")
+    return st
+
+
+def rq_decode_attention_paged(shape, ctx_lens, page_table, max_pages, n_pages, q, ref_k, ref_v,
+                              codes_k, codes_v, scales_k, scales_v, bits, seed, softmax_scale,
+                              tail_k, tail_v, n_tail, tail_pitch, out, workspace,
+                              workspace_bytes=None, stream=None, check=True):
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    st = lib().rq_decode_attention_paged(
+        _shp(shape), _ptr(ctx_lens), _ptr(page_table), int(max_pages), int(n_pages), _ptr(q),
+        _ptr(ref_k), _ptr(ref_v), _ptr(codes_k), _ptr(codes_v), _ptr(scales_k), _ptr(scales_v),
+        int(bits), ctypes.c_uint64(seed), float(softmax_scale), _ptr(tail_k), _ptr(tail_v),
+        int(n_tail), int(tail_pitch), _ptr(out), _ptr(workspace), int(workspace_bytes),
+        _stream(stream))
+    if check:
+        _check(st, "rq_decode_attention_paged")
+    return st
+
+
+def rq_encode_paged(shape, kv_loops, ref, bits_per_loop, seed, refine_iters, dst_pos, page_table,
+                    max_pages, n_pages, codes_out, scales_out, ref_out=None, stream=None,
+                    check=True):
+    n = len(bits_per_loop)
+    ptrs = lambda seq: (ctypes.c_void_p * max(n, 1))(*[_ptr(v) for v in seq])
+    bits = (ctypes.c_uint8 * max(n, 1))(*[int(b) for b in bits_per_loop])
+    st = lib().rq_encode_paged(_shp(shape), ptrs(kv_loops), n, _ptr(ref), bits,
+                               ctypes.c_uint64(seed), int(refine_iters), _ptr(dst_pos),
+                               _ptr(page_table), int(max_pages), int(n_pages), ptrs(codes_out),
+                               ptrs(scales_out), _ptr(ref_out), _stream(stream))
+    if check:
+        _check(st, "rq_encode_paged")
     return st

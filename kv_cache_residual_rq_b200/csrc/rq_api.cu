@@ -169,6 +169,7 @@ rq_status rq_encode_at_ex(const rq_shape* shape, int src_pitch, int src_offset,
   p.ref_out = ref_out;
   p.n_loops = n_loops;
   p.refine_iters = refine_iters;
+  p.kv_heads = shape->kv_heads;
   p.seed = seed;
   p.ctx = shape->ctx;
   p.src_pitch = src_pitch;
@@ -224,6 +225,7 @@ rq_status rq_encode_cr_at(const rq_shape* shape, int dst_pitch, int dst_offset,
   p.ref_codes = ref_codes_out;
   p.ref_scales = ref_scales_out;
   p.n_loops = n_loops;
+  p.kv_heads = shape->kv_heads;
   p.seed = seed;
   p.ctx = shape->ctx;
   p.src_pitch = shape->ctx;
@@ -237,6 +239,64 @@ rq_status rq_encode_cr_at(const rq_shape* shape, int dst_pitch, int dst_offset,
   if (sms <= 0) return RQ_ERR_CUDA;
   cudaError_t e = launch_encode_tma(shape->head_dim, shape->group, p, sms,
                                     static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? RQ_OK : RQ_ERR_CUDA;
+}
+
+rq_status rq_encode_paged(const rq_shape* shape, const uint16_t* const* kv_loops, int n_loops,
+                          const uint16_t* ref, const uint8_t* bits_per_loop, uint64_t seed,
+                          int refine_iters, const int32_t* dst_pos, const int32_t* page_table,
+                          int max_pages, int n_pages, uint32_t* const* codes_out,
+                          uint16_t* const* scales_out, uint16_t* ref_out, void* stream) {
+  if (!shape || !kv_loops || !bits_per_loop || !codes_out || !scales_out || !dst_pos ||
+      !page_table)
+    return RQ_ERR_INVALID_ARG;
+  if (shape->batch < 1 || shape->kv_heads < 1 || shape->ctx < 0) return RQ_ERR_INVALID_ARG;
+  if (max_pages < 1 || n_pages < 1) return RQ_ERR_INVALID_ARG;
+  if (refine_iters < 0 || refine_iters > RQ_MAX_REFINE) return RQ_ERR_INVALID_ARG;
+  if (n_loops < 1 || n_loops > RQ_MAX_LOOPS) return RQ_ERR_INVALID_ARG;
+  if (!supported_dims(shape->head_dim, shape->group)) return RQ_ERR_UNSUPPORTED;
+  if (!ref) return RQ_ERR_INVALID_ARG;
+  if (!aligned16(ref) || (ref_out && !aligned16(ref_out))) return RQ_ERR_ALIGNMENT;
+  if ((reinterpret_cast<uintptr_t>(dst_pos) & 3u) || (reinterpret_cast<uintptr_t>(page_table) & 3u))
+    return RQ_ERR_ALIGNMENT;
+  EncodeParams p;
+  std::memset(&p, 0, sizeof p);
+  int active = 0;
+  for (int l = 0; l < n_loops; ++l) {
+    const int b = bits_per_loop[l];
+    if (b != 2 && b != 4 && b != 16) return RQ_ERR_UNSUPPORTED;
+    p.bits[l] = b;
+    if (b == 16) continue;
+    if (!kv_loops[l] || !codes_out[l] || !scales_out[l]) return RQ_ERR_INVALID_ARG;
+    if (!aligned16(kv_loops[l]) || !aligned16(codes_out[l]) || !aligned16(scales_out[l]))
+      return RQ_ERR_ALIGNMENT;
+    p.x[l] = kv_loops[l];
+    p.codes[l] = codes_out[l];
+    p.scales[l] = scales_out[l];
+    ++active;
+  }
+  p.ref = ref;
+  p.ref_out = ref_out;
+  p.n_loops = n_loops;
+  p.refine_iters = refine_iters;
+  p.kv_heads = shape->kv_heads;
+  p.page_table = page_table;
+  p.dst_pos = dst_pos;
+  p.max_pages = max_pages;
+  p.n_pages = n_pages;
+  p.seed = seed;
+  p.ctx = shape->ctx;
+  p.src_pitch = shape->ctx;
+  p.src_offset = 0;
+  p.n_rows = (long long)shape->batch * shape->kv_heads * shape->ctx;
+  if (p.n_rows == 0 || (active == 0 && !ref_out)) return RQ_OK;
+  const int sms = device_sm_count();
+  if (sms <= 0) return RQ_ERR_CUDA;
+  cudaError_t e = p.n_rows <= kEncodeTmaMaxRows
+                      ? launch_encode_tma(shape->head_dim, shape->group, p, sms,
+                                          static_cast<cudaStream_t>(stream))
+                      : launch_encode(shape->head_dim, shape->group, p, sms,
+                                      static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? RQ_OK : RQ_ERR_CUDA;
 }
 
@@ -265,6 +325,12 @@ namespace {
 
 // Shared body of the decode entry points; ctx_lens null: every sequence has
 // shape->ctx cached tokens.
+struct Paged {                 // paged cache (table null: dense arrays)
+  const int32_t* table = nullptr;
+  int max_pages = 0;
+  int n_pages = 0;
+};
+
 struct CrRef {                 // compressed reference (ref_bits 0: BF16 rows)
   int ref_bits = 0;
   const uint32_t* codes_k = nullptr;
@@ -279,8 +345,16 @@ rq_status decode_impl(const rq_shape* shape, const int32_t* ctx_lens, const uint
                       const uint16_t* scales_v, int bits, uint64_t seed, float softmax_scale,
                       const uint16_t* tail_k, const uint16_t* tail_v, int n_tail,
                       int tail_pitch, float* out, void* workspace, size_t workspace_bytes,
-                      void* stream, const CrRef& cr = CrRef()) {
+                      void* stream, const CrRef& cr = CrRef(), const Paged& pg = Paged()) {
   const bool varlen = ctx_lens != nullptr;
+  if (pg.table) {
+    if (!varlen || !shape) return RQ_ERR_INVALID_ARG;
+    if (pg.max_pages < 1 || pg.n_pages < 1) return RQ_ERR_INVALID_ARG;
+    if ((long long)pg.max_pages * kDecodeTile != shape->ctx ||
+        (shape->ctx_cap != 0 && shape->ctx_cap != shape->ctx))
+      return RQ_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(pg.table) & 3u) return RQ_ERR_ALIGNMENT;
+  }
   if (cr.ref_bits != 0) {
     if (cr.ref_bits != 4 && cr.ref_bits != 8) return RQ_ERR_UNSUPPORTED;
     if (!shape || shape->q_heads != shape->kv_heads) return RQ_ERR_UNSUPPORTED;
@@ -346,6 +420,9 @@ rq_status decode_impl(const rq_shape* shape, const int32_t* ctx_lens, const uint
   p.tail_pitch = n_tail > 0 ? tail_pitch : 0;
   p.ctx_lens = ctx_lens;
   if (varlen) p.ctx = pitch_of(shape);
+  p.page_table = pg.table;
+  p.max_pages = pg.max_pages;
+  p.n_pages = pg.n_pages;
   p.ref_bits = cr.ref_bits;
   p.rcodes_k = cr.codes_k;
   p.rcodes_v = cr.codes_v;
@@ -417,6 +494,25 @@ rq_status rq_decode_attention_cr(const rq_shape* shape, const int32_t* ctx_lens,
   return decode_impl(shape, ctx_lens, q, nullptr, nullptr, codes_k, codes_v, scales_k, scales_v,
                      bits, seed, softmax_scale, tail_k, tail_v, n_tail, tail_pitch, out,
                      workspace, workspace_bytes, stream, cr);
+}
+
+rq_status rq_decode_attention_paged(const rq_shape* shape, const int32_t* ctx_lens,
+                                    const int32_t* page_table, int max_pages, int n_pages,
+                                    const uint16_t* q, const uint16_t* ref_k,
+                                    const uint16_t* ref_v, const uint32_t* codes_k,
+                                    const uint32_t* codes_v, const uint16_t* scales_k,
+                                    const uint16_t* scales_v, int bits, uint64_t seed,
+                                    float softmax_scale, const uint16_t* tail_k,
+                                    const uint16_t* tail_v, int n_tail, int tail_pitch, float* out,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
+  if (!ctx_lens || !page_table) return RQ_ERR_INVALID_ARG;
+  Paged pg;
+  pg.table = page_table;
+  pg.max_pages = max_pages;
+  pg.n_pages = n_pages;
+  return decode_impl(shape, ctx_lens, q, ref_k, ref_v, codes_k, codes_v, scales_k, scales_v, bits,
+                     seed, softmax_scale, tail_k, tail_v, n_tail, tail_pitch, out, workspace,
+                     workspace_bytes, stream, CrRef(), pg);
 }
 
 size_t rq_decode_workspace_bytes_varlen(const rq_shape* shape) {

@@ -260,11 +260,11 @@ decode_kernel(const DecodeParams p) {
           }
         }
         if (flags[0]) break;
-        const long long hd = cur.hd;
-        const int t0 = cur.t0();
-        const int n = cur.n();
+        size_t row;
+        const bool page_ok = tile_row(p, cur, row);
+        if (!page_ok && cur.n() > 0) flag_error(p.status, 32u);
+        const int n = page_ok ? cur.n() : 0;
         cur.next(p);
-        const size_t row = (size_t)hd * p.ctx_pitch + t0;       // first token row of the tile
         unsigned char* st = ring + s * C::STAGE_BYTES;
         if (n <= 0) {                   // the empty tile of an empty sequence
           mbar_arrive(&full_bar[s]);
@@ -801,8 +801,8 @@ decode_kernel(const DecodeParams p) {
   TileCursor cur = first_cur;
   for (int i = 0; i < n_my; ++i) {
     const long long hd = cur.hd;
-    const int t0 = cur.t0();
-    const int n = cur.n();
+    size_t row;
+    const int n = tile_row(p, cur, row) ? cur.n() : 0;
     if (hd != cur_head) {
       if (cur_head >= 0) {
         flush_head(cur_head, cur_first, cur_nt);
@@ -825,7 +825,6 @@ decode_kernel(const DecodeParams p) {
     }
     if (!aborted && n > 0) {
       const unsigned char* st = ring + s * C::STAGE_BYTES;
-      const size_t row = (size_t)hd * p.ctx_pitch + t0;
       const int sc_off = (int)((row * SB) & 15);
       const int grp = dim0 / p.group;
       if constexpr (G == 1) tile_g1(st, n, sc_off, grp);

@@ -73,6 +73,28 @@ struct TileCursor {
   }
 };
 
+// First row of the cursor's tile in the K/V, code and scale arrays.  Dense
+// caches: head hd's token t0 is row hd * ctx_pitch + t0.  Paged caches (page
+// = one 64-token tile): sequence b's tile j is page page_table[b][j] of a pool
+// [pages][kv_heads][64][...], rows (page * kv_heads + h) * 64 ...  Returns
+// false for a page id outside the pool; the caller then treats the tile as
+// empty (and the producer raises status bit 32), so a bad table entry cannot
+// address memory outside the pool.
+__device__ __forceinline__ bool tile_row(const DecodeParams& p, const TileCursor& c,
+                                         size_t& row) {
+  if (!p.page_table) {
+    row = (size_t)c.hd * p.ctx_pitch + c.t0();
+    return true;
+  }
+  const int page = p.page_table[(size_t)c.b * p.max_pages + c.j];
+  if (page < 0 || page >= p.n_pages) {
+    row = 0;
+    return false;
+  }
+  row = ((size_t)page * p.kv_heads + c.h) * kDecodeTile;
+  return true;
+}
+
 // The split of a call over its CTAs: n_tiles tiles in `ctas` equal runs.
 struct CallSplit {
   long long n_tiles;

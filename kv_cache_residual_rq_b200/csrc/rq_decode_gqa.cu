@@ -236,11 +236,11 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
           }
         }
         if (flags[0]) break;
-        const long long hd = cur.hd;
-        const int t0 = cur.t0();
-        const int n = cur.n();
+        size_t row;
+        const bool page_ok = tile_row(p, cur, row);
+        if (!page_ok && cur.n() > 0) flag_error(p.status, 32u);
+        const int n = page_ok ? cur.n() : 0;
         cur.next(p);
-        const size_t row = (size_t)hd * p.ctx_pitch + t0;
         unsigned char* st = ring + s * C::STAGE_BYTES;
         if (n <= 0) {                   // the empty tile of an empty sequence
           mbar_arrive(&full_bar[s]);
@@ -570,8 +570,8 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
   TileCursor cur = first_cur;
   for (int i = 0; i < n_my; ++i) {
     const long long hd = cur.hd;
-    const int t0 = cur.t0();
-    const int n = cur.n();
+    size_t row;
+    const int n = tile_row(p, cur, row) ? cur.n() : 0;
     if (hd != cur_head) {
       if (cur_head >= 0) {
         flush_head(cur_head, cur_first, cur_nt);
@@ -593,7 +593,6 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
       flags[0] = 1;
     }
     if (!aborted && n > 0) {
-      const size_t row = (size_t)hd * p.ctx_pitch + t0;
       tile_mma(ring + s * C::STAGE_BYTES, n, (int)((row * SB) & 15));
     }
     __syncwarp();
@@ -646,7 +645,9 @@ cudaError_t launch_decode_gqa(int head_dim, int G, int bits, const DecodeParams&
                               cudaStream_t stream) {
   GqaParams gp;
   gp.p = p;
-  const unsigned long long rows = (unsigned long long)p.batch * p.kv_heads * p.ctx_pitch;
+  const unsigned long long rows =
+      p.page_table ? (unsigned long long)p.n_pages * p.kv_heads * kDecodeTile
+                   : (unsigned long long)p.batch * p.kv_heads * p.ctx_pitch;
   if (!encode_rows_map(&gp.tmap_k, p.ref_k, rows, head_dim, kDecodeTile) ||
       !encode_rows_map(&gp.tmap_v, p.ref_v, rows, head_dim, kDecodeTile))
     return cudaErrorInvalidValue;

@@ -54,10 +54,11 @@ encode_kernel(const EncodeParams p) {
     const bool valid = idx < p.n_rows;
     const long long hd = idx / p.ctx, t = idx % p.ctx;
     const long long src_row = hd * p.src_pitch + p.src_offset + t;
-    const long long row = hd * p.dst_pitch + p.dst_offset + t;    // destination row
+    long long row = 0;                                             // destination row
+    const bool wvalid = valid && enc_dst_row(p, hd, t, row);
     const size_t eoff = (size_t)src_row * D + li * DPL;
     const uint4 rw = valid ? ld_stream(p.ref + eoff) : make_uint4(0, 0, 0, 0);
-    if (valid && p.ref_out)
+    if (wvalid && p.ref_out)
       *reinterpret_cast<uint4*>(p.ref_out + (size_t)row * D + li * DPL) = rw;
 
     for (int lb = 0; lb < p.n_loops; lb += kLoopBatch) {
@@ -199,12 +200,12 @@ encode_kernel(const EncodeParams p) {
         if (bits == 2) {
           // 16 codes per word: lanes 2w and 2w+1 of a row share word w
           const uint32_t upper = __shfl_down_sync(FULL, packed, 1);
-          if (valid && !(li & 1))
+          if (wvalid && !(li & 1))
             p.codes[l][(size_t)row * (D / 16) + (li >> 1)] = packed | (upper << 16);
         } else {
-          if (valid) p.codes[l][(size_t)row * (D / 8) + li] = packed;
+          if (wvalid) p.codes[l][(size_t)row * (D / 8) + li] = packed;
         }
-        if (valid && (li % LPG) == 0)
+        if (wvalid && (li % LPG) == 0)
           p.scales[l][(size_t)row * (D / GROUP) + li / LPG] =
               __half_as_ushort(__float2half_rn(s));
       }

@@ -348,9 +348,9 @@ encode_tma_kernel(const __grid_constant__ EncodeTmaParams tp) {
   long long it = 0;
   for (int t = blockIdx.x; t < tp.n_tiles; t += gridDim.x) {
     const long long idx = (long long)t * C::R + r;
-    const bool valid = idx < p.n_rows;
     const long long hd = idx / p.ctx, tok = idx - hd * p.ctx;
-    const long long row = hd * p.dst_pitch + p.dst_offset + tok;
+    long long row = 0;
+    const bool valid = idx < p.n_rows && enc_dst_row(p, hd, tok, row);
 
     // reference: -D_i ref_i, kept for every loop of these rows
     int s = (int)(it % kSlots);

@@ -55,11 +55,37 @@ struct EncodeParams {
   int dst_pitch, dst_offset;         // token pitch / first token of the outputs
   int n_loops;
   int refine_iters;                  // least-squares refits after the absmax codes
+  int kv_heads;                      // heads per row of the shape (paged destinations)
+  const int* page_table;             // paged destination pools: page of token block j of
+  const int* dst_pos;                //   sequence b at [b * max_pages + j]; first position
+  int max_pages, n_pages;            //   written per sequence; null for dense outputs
   int ref_bits;                      // 0: BF16 reference; 4 or 8: compressed reference
   uint32_t* ref_codes;               // compressed reference: codes and scales out
   uint16_t* ref_scales;
   uint64_t seed;
 };
+
+#ifdef __CUDACC__
+// Destination row of token t of head hd (hd = b * kv_heads + h).  Dense
+// outputs: hd * dst_pitch + dst_offset + t.  Paged pools of 64-token pages:
+// position pos = dst_pos[b] + t of sequence b lives in page page_table[b][pos / 64]
+// at row (page * kv_heads + h) * 64 + pos % 64.  Returns false -- nothing is
+// written -- for a position past the table or a page id outside the pool.
+__device__ __forceinline__ bool enc_dst_row(const EncodeParams& p, long long hd, long long t,
+                                            long long& row) {
+  if (!p.page_table) {
+    row = hd * p.dst_pitch + p.dst_offset + t;
+    return true;
+  }
+  const long long b = hd / p.kv_heads, h = hd - b * p.kv_heads;
+  const long long pos = (long long)p.dst_pos[b] + t;
+  if (pos < 0 || pos >= (long long)p.max_pages * 64) return false;
+  const int page = p.page_table[b * p.max_pages + pos / 64];
+  if (page < 0 || page >= p.n_pages) return false;
+  row = ((long long)page * p.kv_heads + h) * 64 + pos % 64;
+  return true;
+}
+#endif
 
 // streaming encoder: any token pitch and offset (rq_encode.cu)
 cudaError_t launch_encode(int head_dim, int group, const EncodeParams& p, int num_sms,
@@ -155,6 +181,8 @@ struct DecodeParams {
   const uint32_t* rcodes_v;
   const uint16_t* rscales_k;
   const uint16_t* rscales_v;
+  const int* page_table; // paged cache: page of tile j of sequence b at
+  int max_pages, n_pages; //   [b * max_pages + j], pool of n_pages pages; else null
   const int* ctx_lens;   // variable-length call: cached tokens per sequence
                          // [batch] (device int32), else null (ctx for all)
   int nt;

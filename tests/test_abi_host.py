@@ -239,3 +239,22 @@ def test_varlen_decode_rejects_bad_arguments_before_launch():
         cap, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, 0, 0.0, None, None, 0, 0, FAKE,
         FAKE, 64, stream=0, check=False)
     assert small_ws == rq.RQ_ERR_WORKSPACE
+
+
+def test_paged_entry_points_validate_before_launch():
+    s = rq.make_shape(2, 2, 4 * 64, 128, 32)
+    dec = lambda shape=s, lens=FAKE, table=FAKE, mp=4, npg=10: rq.rq_decode_attention_paged(
+        shape, lens, table, mp, npg, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, 0, 0.0, None,
+        None, 0, 0, FAKE, FAKE, 1 << 30, stream=0, check=False)
+    assert dec(lens=None) == rq.RQ_ERR_INVALID_ARG
+    assert dec(table=None) == rq.RQ_ERR_INVALID_ARG
+    assert dec(mp=3) == rq.RQ_ERR_INVALID_ARG          # ctx must be max_pages * 64
+    assert dec(npg=0) == rq.RQ_ERR_INVALID_ARG
+    assert dec(table=FAKE + 2) == rq.RQ_ERR_ALIGNMENT
+    enc = lambda pos=FAKE, table=FAKE, it=0: rq.rq_encode_paged(
+        rq.make_shape(2, 2, 1, 128, 32), [FAKE], FAKE, [2], 0, it, pos, table, 4, 10, [FAKE],
+        [FAKE], stream=0, check=False)
+    assert enc(pos=None) == rq.RQ_ERR_INVALID_ARG
+    assert enc(table=None) == rq.RQ_ERR_INVALID_ARG
+    assert enc(it=rq.RQ_MAX_REFINE + 1) == rq.RQ_ERR_INVALID_ARG
+    assert enc(pos=FAKE + 1) == rq.RQ_ERR_ALIGNMENT
