@@ -69,9 +69,12 @@ struct GCfg {
   static constexpr int SB = 2 * NG;                        // scale bytes per token
   static constexpr int WSUM_FLOATS = kConsumerWarps * G * NG;
   static constexpr int QFRAG_WORDS = 3 * KT * 32 * 2;       // q, q~ high, q~ remainder (bf16)
+  // INT2: per (row, scale group) sum of the q~ fragments' values (offset of
+  // the 128 + 2c operands), even count to keep the barriers 8-byte aligned
+  static constexpr int SQ_FLOATS = (G * NG + 1) / 2 * 2;
   static constexpr int SMEM_BYTES = 1024 /* base alignment slack */ + RING_BYTES +
                                     4 * (MERGE_FLOATS + QBUF_FLOATS + WSUM_FLOATS +
-                                         QFRAG_WORDS) +
+                                         QFRAG_WORDS + SQ_FLOATS) +
                                     2 * STAGES * 8 + 16;
   static_assert(G == 2 || G == 4 || G == 8, "grouped queries");
   static_assert(MERGE_FLOATS >= kVarlenMaxBatch + 1, "merge area holds the length scan");
@@ -171,6 +174,15 @@ __device__ __forceinline__ void k_levels(uint32_t w0, uint32_t w1, int q, uint32
   }
 }
 
+// INT2 K-residual B fragment with the k permutation of the q~ fragments:
+// register 0 = dims (2q, 2q+8), register 1 = dims (2q+1, 2q+9) of the
+// 16-dim step, each half the exact bf16 value 128 + 2c (code c at mantissa
+// bits 1-2; the codes of a register are 16 bits apart in the packed word).
+__device__ __forceinline__ void k_levels2(uint32_t w, int q, uint32_t& b0, uint32_t& b1) {
+  b0 = (((w << 1) >> (4 * q)) & 0x00060006u) | kMagic;
+  b1 = ((w >> (4 * q + 1)) & 0x00060006u) | kMagic;
+}
+
 template <int D, int G, int BITS, int GROUP>
 __global__ void __launch_bounds__(kDecodeThreads, 2)
 decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
@@ -190,7 +202,8 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
   float* qbuf = merge + C::MERGE_FLOATS;
   float* wsum_s = qbuf + C::QBUF_FLOATS;
   uint32_t* qfrag = reinterpret_cast<uint32_t*>(wsum_s + C::WSUM_FLOATS);  // [3][KT][32][2]
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(qfrag + C::QFRAG_WORDS);
+  float* sq_s = reinterpret_cast<float*>(qfrag + C::QFRAG_WORDS);           // [G][NG]
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(sq_s + C::SQ_FLOATS);
   uint64_t* empty_bar = full_bar + STAGES;
   volatile int* flags = reinterpret_cast<volatile int*>(empty_bar + STAGES);
 
@@ -319,7 +332,8 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
     load_rotate_queries<D, G>(p, hd, qs, qt, tid);
     const float cd = rot_scale<D>();
     if (warp == 0) {
-#pragma unroll
+      float sqj = 0.0f;      // running sum of the current scale group (INT2)
+#pragma unroll 1
       for (int kk = 0; kk < KT; ++kk) {
         uint32_t* fa = qfrag + ((0 * KT + kk) * 32 + lane) * 2;
         uint32_t* fh = qfrag + ((1 * KT + kk) * 32 + lane) * 2;
@@ -329,10 +343,27 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
           const float* trow = qt + g * D + 16 * kk + 2 * q;
           fa[0] = pack_bf16(qrow[0], qrow[1]);       // exact: q is bf16
           fa[1] = pack_bf16(qrow[8], qrow[9]);
-          split_bf16(cd * trow[0], cd * trow[1], fh[0], fl[0]);
-          split_bf16(cd * trow[8], cd * trow[9], fh[1], fl[1]);
+          if constexpr (BITS == 2) {
+            // k positions 2q, 2q+1 | 2q+8, 2q+9 carry dims 2q, 2q+8 | 2q+1, 2q+9,
+            // so the two codes of a B register sit 16 bits apart (k_levels2)
+            split_bf16(cd * trow[0], cd * trow[8], fh[0], fl[0]);
+            split_bf16(cd * trow[1], cd * trow[9], fh[1], fl[1]);
+            sqj += ((bf16_lo_f(fh[0]) + bf16_lo_f(fl[0])) +
+                    (bf16_hi_f(fh[0]) + bf16_hi_f(fl[0]))) +
+                   ((bf16_lo_f(fh[1]) + bf16_lo_f(fl[1])) +
+                    (bf16_hi_f(fh[1]) + bf16_hi_f(fl[1])));
+          } else {
+            split_bf16(cd * trow[0], cd * trow[1], fh[0], fl[0]);
+            split_bf16(cd * trow[8], cd * trow[9], fh[1], fl[1]);
+          }
         } else {
           fa[0] = fa[1] = fh[0] = fh[1] = fl[0] = fl[1] = 0u;
+        }
+        if (BITS == 2 && (kk + 1) % KSG == 0) {      // end of a scale group
+          sqj += __shfl_xor_sync(FULL, sqj, 1);
+          sqj += __shfl_xor_sync(FULL, sqj, 2);
+          if (row_ok && q == 0) sq_s[g * NG + kk / KSG] = sqj;
+          sqj = 0.0f;
         }
       }
     }
@@ -436,7 +467,7 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
           const uint32_t* cw = reinterpret_cast<const uint32_t*>(st + C::OFF_CK + tb[nt] * C::CROW);
           uint32_t b0, b1;
           if constexpr (BITS == 2) {
-            k_levels<2>(cw[kk], 0u, q, b0, b1);
+            k_levels2(cw[kk], q, b0, b1);
           } else {
             const uint2 w2 = *reinterpret_cast<const uint2*>(cw + 2 * kk);
             k_levels<4>(w2.x, w2.y, q, b0, b1);
@@ -451,8 +482,10 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
           for (int nt = 0; nt < 2; ++nt) {
             const float sk0 = half_at(st + C::OFF_SK + sc_off + tok0[nt] * SB + 2 * j);
             const float sk1 = half_at(st + C::OFF_SK + sc_off + (tok0[nt] + 1) * SB + 2 * j);
-            cref[nt][0] = fmaf(sk0, ct[nt][0], cref[nt][0]);
-            cref[nt][1] = fmaf(sk1, ct[nt][1], cref[nt][1]);
+            // INT2 operands are 128 + 2c: q~ . l = result - 131 sum q~
+            const float off = (BITS == 2 && row_ok) ? 131.0f * sq_s[g * NG + j] : 0.0f;
+            cref[nt][0] = fmaf(sk0, ct[nt][0] - off, cref[nt][0]);
+            cref[nt][1] = fmaf(sk1, ct[nt][1] - off, cref[nt][1]);
 #pragma unroll
             for (int e = 0; e < 4; ++e) ct[nt][e] = 0.0f;
           }
