@@ -169,3 +169,41 @@ def test_uniform_call_ignores_nan_in_spare_capacity(G):
             want = oracle_head(w, q, refk_h, refv_h, xk, xv, 2, b, h, ctx, None, None, 0)
             got = out[b, h * G:(h + 1) * G].double().cpu().numpy()
             assert np.abs(got - want).max() <= OUT_TOL
+
+
+@pytest.mark.parametrize("G", [1, 4])
+def test_one_captured_graph_serves_changing_lengths(G):
+    # capture a variable-length call once; new lengths written on the device
+    # between replays change the work each replay does
+    cap, bits = 200, 2
+    w, refk, refv, xk, xv, ck, cv, sk, sv, q, tail_k, tail_v = build_case(G, bits, [cap] * 3, cap,
+                                                                          1, 61 + G)
+    B, Hkv, d = 3, w.kv_heads, w.head_dim
+    shape = rq.make_shape(B, Hkv, cap, d, w.group, q_heads=Hkv * G)
+    ws = rq.alloc_workspace(shape, varlen=True)
+    lens_d = torch.tensor([cap] * B, dtype=torch.int32, device="cuda")
+    out = torch.empty((B, Hkv * G, d), dtype=torch.float32, device="cuda")
+    s = torch.cuda.Stream()
+    call = lambda: rq.rq_decode_attention_varlen(shape, lens_d, q, refk, refv, ck, cv, sk, sv,
+                                                 bits, w.seed, 0.0, tail_k, tail_v, 1,
+                                                 tail_k.shape[2], out, ws,
+                                                 stream=torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        call()                                       # warm-up outside the capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        call()
+    torch.cuda.synchronize()
+    for lens in ([5, 200, 64], [130, 1, 0], [200, 200, 200]):
+        lens_d.copy_(torch.tensor(lens, dtype=torch.int32))
+        g.replay()
+        torch.cuda.synchronize()
+        got = out.clone()
+        want = torch.empty_like(out)
+        rq.rq_decode_attention_varlen(shape, lens_d, q, refk, refv, ck, cv, sk, sv, bits, w.seed,
+                                      0.0, tail_k, tail_v, 1, tail_k.shape[2], want,
+                                      rq.alloc_workspace(shape, varlen=True))
+        torch.cuda.synchronize()
+        assert torch.equal(got, want), lens
+    assert rq.rq_workspace_status(ws) == 0
