@@ -139,13 +139,16 @@ def reconstruct_cr(shape4, ref_codes, ref_scales, ref_bits, codes, scales, bits,
 
 def decode_attention_cr(q, ref, codes_k, codes_v, scales_k, scales_v, bits, group, seed, ctx_cap,
                         ctx=None, ctx_lens=None, tail_k=None, tail_v=None, n_tail=0,
-                        softmax_scale=0.0, out=None, workspace=None, stream=None):
+                        softmax_scale=0.0, out=None, workspace=None, stream=None, kv_heads=None):
     """Decode attention over a compressed-reference cache.  ref = (ref_codes_k,
-    ref_scales_k, ref_codes_v, ref_scales_v, ref_bits); q [B, H, d]."""
+    ref_scales_k, ref_codes_v, ref_scales_v, ref_bits); q [B, Hq, d]; the
+    cache has kv_heads heads (default Hq)."""
     import torch
     rck, rsk, rcv, rsv, ref_bits = ref
     b, h, d = q.shape
-    shape = make_shape(b, h, ctx if ctx is not None else ctx_cap, d, group, ctx_cap=ctx_cap)
+    hkv = h if kv_heads is None else kv_heads
+    shape = make_shape(b, hkv, ctx if ctx is not None else ctx_cap, d, group, q_heads=h,
+                       ctx_cap=ctx_cap)
     if out is None:
         out = torch.empty((b, h, d), dtype=torch.float32, device=q.device)
     if workspace is None:

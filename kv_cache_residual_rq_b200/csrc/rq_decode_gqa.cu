@@ -22,9 +22,20 @@
 // completed when the warp flushes.  Rows beyond G are zero and their weights
 // are forced to zero.
 //
-// The reference K/V tiles arrive by TMA tensor copies with the 128-byte
-// swizzle (conflict-free ldmatrix); codes and scales by plain bulk copies, as
-// in the single-query kernel.  The work split, the partial records and the
+// Compressed INT8 reference (same page, the reference loop itself stored as
+// rotated codes): the reference term is one more quantised term in the
+// rotated domain, s_ref <q~, l_ref> for the scores and sum_t p s_ref l_ref for
+// the values, l_ref = 2c - 255.  Its K codes enter an f16 MMA as the exact
+// values 1024 + c (one byte permute per two codes) against q~ scaled by a
+// power of two per row and split into f16 high and remainder parts; its V
+// codes enter a bf16 MMA split into nibbles, 128 + 2 c_lo and 128 + 2 c_hi
+// (exact), the high nibble against 16 x the weights.  The offsets are removed
+// once per scale group (scores) or when the warp flushes (values).
+//
+// The reference K/V tiles (BF16 rows, or INT8 code rows) arrive by TMA
+// tensor copies with the swizzle of their line width (conflict-free
+// ldmatrix); codes and scales by plain bulk copies, as in the single-query
+// kernel.  The work split, the partial records and the
 // last-arriving-CTA merge with the single inverse rotation are shared with it
 // (rq_decode_common.cuh).  Every mbarrier wait is bounded.
 #include <cuda.h>
@@ -42,24 +53,30 @@ struct alignas(64) GqaParams {
   DecodeParams p;
 };
 
-template <int D, int G, int BITS, int GROUP>
+template <int D, int G, int BITS, int GROUP, int RB>
 struct GCfg {
   static constexpr int TILE = kDecodeTile;                 // 64 tokens
   static constexpr int WTOK = TILE / kConsumerWarps;       // 16 tokens per warp
   static constexpr bool RES = (BITS != 16);
+  static constexpr bool CR = (RB == 8);                    // INT8 compressed reference
   static constexpr int NBOX = D / 64;                      // 64-column boxes per row
   static constexpr int BOX_BYTES = 64 * 128;               // 64 rows x 128 B
+  // one K or V reference tile: BF16 boxes, or the INT8 code rows (D bytes each)
+  static constexpr int REF_TILE_BYTES = CR ? TILE * D : NBOX * BOX_BYTES;
   static constexpr int KT = D / 16;                        // k-steps of 16 dims
   static constexpr int CROW = RES ? D * BITS / 8 : 0;      // code bytes per token
   static constexpr int CWORDS = CROW / 4;
   static constexpr int SC_BYTES = RES ? TILE * (2 * D / 32) + 32 : 0;
+  static constexpr int RSC_BYTES = CR ? TILE * (2 * D / 32) + 32 : 0;   // reference scales
   static constexpr int OFF_K = 0;
-  static constexpr int OFF_V = OFF_K + NBOX * BOX_BYTES;
-  static constexpr int OFF_CK = OFF_V + NBOX * BOX_BYTES;
+  static constexpr int OFF_V = OFF_K + REF_TILE_BYTES;
+  static constexpr int OFF_CK = OFF_V + REF_TILE_BYTES;
   static constexpr int OFF_CV = OFF_CK + TILE * CROW;
   static constexpr int OFF_SK = OFF_CV + TILE * CROW;
   static constexpr int OFF_SV = OFF_SK + SC_BYTES;
-  static constexpr int STAGE_BYTES = (OFF_SV + SC_BYTES + 1023) / 1024 * 1024;
+  static constexpr int OFF_RSK = OFF_SV + SC_BYTES;
+  static constexpr int OFF_RSV = OFF_RSK + RSC_BYTES;
+  static constexpr int STAGE_BYTES = (OFF_RSV + RSC_BYTES + 1023) / 1024 * 1024;
   static constexpr int STAGES = 2;
   static constexpr int RING_BYTES = STAGES * STAGE_BYTES;
   static constexpr int MERGE_FLOATS = kConsumerWarps * G * (2 + 2 * D);
@@ -67,11 +84,14 @@ struct GCfg {
   static constexpr int NG = D / GROUP;                      // scale groups per token
   static constexpr int KSG = GROUP / 16;                   // k-steps per scale group
   static constexpr int SB = 2 * NG;                        // scale bytes per token
-  static constexpr int WSUM_FLOATS = kConsumerWarps * G * NG;
-  static constexpr int QFRAG_WORDS = 3 * KT * 32 * 2;       // q, q~ high, q~ remainder (bf16)
+  // per warp, row and scale group: sum of p s^V (and of p s_ref^V)
+  static constexpr int WSUM_FLOATS = kConsumerWarps * G * NG * (CR ? 2 : 1);
+  // q, q~ high, q~ remainder (bf16); with CR also q~ 2^E high, remainder (f16)
+  static constexpr int QFRAG_WORDS = (CR ? 5 : 3) * KT * 32 * 2;
   // INT2: per (row, scale group) sum of the q~ fragments' values (offset of
-  // the 128 + 2c operands), even count to keep the barriers 8-byte aligned
-  static constexpr int SQ_FLOATS = (G * NG + 1) / 2 * 2;
+  // the 128 + 2c operands); CR: the same for the f16 fragments (offset of
+  // 1024 + c) and per row 2^-E; even count to keep the barriers 8-byte aligned
+  static constexpr int SQ_FLOATS = (G * NG * (CR ? 2 : 1) + (CR ? G : 0) + 1) / 2 * 2;
   static constexpr int SMEM_BYTES = 1024 /* base alignment slack */ + RING_BYTES +
                                     4 * (MERGE_FLOATS + QBUF_FLOATS + WSUM_FLOATS +
                                          QFRAG_WORDS + SQ_FLOATS) +
@@ -80,6 +100,8 @@ struct GCfg {
   static_assert(MERGE_FLOATS >= kVarlenMaxBatch + 1, "merge area holds the length scan");
   static_assert(GROUP == 32 || GROUP == 64, "scale group");
   static_assert(D == 64 || D == 128, "head_dim");
+  static_assert(RB == 0 || RB == 8, "reference: BF16 rows or INT8 codes");
+  static_assert(OFF_V % 1024 == 0, "swizzled tiles start on the pattern's period");
 };
 
 // ---- PTX wrappers -----------------------------------------------------------
@@ -115,6 +137,26 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// the same with f16 operands
+__device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                        uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Byte offset of 16-byte chunk `chunk` of row `row` in a tile of rows of
+// RROW bytes (64 or 128) written by a TMA copy with the swizzle of that
+// width: address bits 4.. are XORed with bits 7.. (3 bits for 128 B, 2 for 64 B).
+template <int RROW>
+__device__ __forceinline__ uint32_t swz_offset(int row, int chunk) {
+  const uint32_t o = (uint32_t)(row * RROW + chunk * 16);
+  constexpr uint32_t mask = RROW == 128 ? 7u : 3u;
+  return o ^ (((o >> 7) & mask) << 4);
+}
+
 
 // {lo, hi} -> packed bf16x2 / f16x2 (round to nearest)
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -139,6 +181,23 @@ __device__ __forceinline__ float bf16_hi_f(uint32_t w) { return __uint_as_float(
 __device__ __forceinline__ void split_bf16(float lo, float hi, uint32_t& h, uint32_t& r) {
   h = pack_bf16(lo, hi);
   r = pack_bf16(lo - bf16_lo_f(h), hi - bf16_hi_f(h));
+}
+
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ float f16_lo_f(uint32_t w) {
+  return __half2float(__ushort_as_half((unsigned short)(w & 0xFFFFu)));
+}
+__device__ __forceinline__ float f16_hi_f(uint32_t w) {
+  return __half2float(__ushort_as_half((unsigned short)(w >> 16)));
+}
+// {lo, hi} as an f16 pair h plus an f16 pair of remainders r
+__device__ __forceinline__ void split_f16(float lo, float hi, uint32_t& h, uint32_t& r) {
+  h = pack_f16(lo, hi);
+  r = pack_f16(lo - f16_lo_f(h), hi - f16_hi_f(h));
 }
 
 constexpr uint32_t kMagic = 0x43004300u;   // bf16 128.0 in both halves (mantissa unit 1)
@@ -183,10 +242,10 @@ __device__ __forceinline__ void k_levels2(uint32_t w, int q, uint32_t& b0, uint3
   b1 = ((w >> (4 * q + 1)) & 0x00060006u) | kMagic;
 }
 
-template <int D, int G, int BITS, int GROUP>
+template <int D, int G, int BITS, int GROUP, int RB>
 __global__ void __launch_bounds__(kDecodeThreads, 2)
 decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
-  using C = GCfg<D, G, BITS, GROUP>;
+  using C = GCfg<D, G, BITS, GROUP, RB>;
   const DecodeParams& p = gp.p;
   constexpr int STAGES = C::STAGES, TILE = C::TILE, KT = C::KT;
   constexpr unsigned FULL = 0xffffffffu;
@@ -203,6 +262,9 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
   float* wsum_s = qbuf + C::QBUF_FLOATS;
   uint32_t* qfrag = reinterpret_cast<uint32_t*>(wsum_s + C::WSUM_FLOATS);  // [3][KT][32][2]
   float* sq_s = reinterpret_cast<float*>(qfrag + C::QFRAG_WORDS);           // [G][NG]
+  float* sqh_s = sq_s + G * NG;              // CR: [G][NG] sums of the f16 q~ fragments
+  float* rsig_s = sqh_s + G * NG;            // CR: [G] 2^-E of each row's f16 q~
+  float* wsumR_s = wsum_s + kConsumerWarps * G * NG;   // CR: sums of p s_ref^V
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(sq_s + C::SQ_FLOATS);
   uint64_t* empty_bar = full_bar + STAGES;
   volatile int* flags = reinterpret_cast<volatile int*>(empty_bar + STAGES);
@@ -260,20 +322,33 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
           ++issued;
           continue;
         }
-        uint32_t bytes = 2u * C::NBOX * C::BOX_BYTES;     // full boxes, OOB rows zero-filled
+        uint32_t bytes = 2u * C::REF_TILE_BYTES;          // full boxes, OOB rows zero-filled
         size_t sc_lo = 0;
         uint32_t sc_bytes = 0;
-        if constexpr (C::RES) {
+        if constexpr (C::RES || C::CR) {
           const size_t start = row * SB;
           sc_lo = start & ~(size_t)15;
           sc_bytes = (uint32_t)(((start + (size_t)n * SB + 15) & ~(size_t)15) - sc_lo);
-          bytes += 2u * n * C::CROW + 2u * sc_bytes;
         }
+        if constexpr (C::RES) bytes += 2u * n * C::CROW + 2u * sc_bytes;
+        if constexpr (C::CR) bytes += 2u * sc_bytes;
         mbar_arrive_expect_tx(&full_bar[s], bytes);
+        if constexpr (C::CR) {
+          // one box of whole code rows each
+          tma_load_2d(st + C::OFF_K, &gp.tmap_k, 0, (int)row, &full_bar[s]);
+          tma_load_2d(st + C::OFF_V, &gp.tmap_v, 0, (int)row, &full_bar[s]);
+          bulk_g2s(st + C::OFF_RSK, reinterpret_cast<const unsigned char*>(p.rscales_k) + sc_lo,
+                   sc_bytes, &full_bar[s]);
+          bulk_g2s(st + C::OFF_RSV, reinterpret_cast<const unsigned char*>(p.rscales_v) + sc_lo,
+                   sc_bytes, &full_bar[s]);
+        } else {
 #pragma unroll
-        for (int bx = 0; bx < C::NBOX; ++bx) {
-          tma_load_2d(st + C::OFF_K + bx * C::BOX_BYTES, &gp.tmap_k, 64 * bx, (int)row, &full_bar[s]);
-          tma_load_2d(st + C::OFF_V + bx * C::BOX_BYTES, &gp.tmap_v, 64 * bx, (int)row, &full_bar[s]);
+          for (int bx = 0; bx < C::NBOX; ++bx) {
+            tma_load_2d(st + C::OFF_K + bx * C::BOX_BYTES, &gp.tmap_k, 64 * bx, (int)row,
+                        &full_bar[s]);
+            tma_load_2d(st + C::OFF_V + bx * C::BOX_BYTES, &gp.tmap_v, 64 * bx, (int)row,
+                        &full_bar[s]);
+          }
         }
         if constexpr (C::RES) {
           bulk_g2s(st + C::OFF_CK, p.codes_k + row * C::CWORDS, n * C::CROW, &full_bar[s]);
@@ -302,21 +377,25 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
   // and lane, {a0, a2} of the bf16 query (kind 0) and of the rotated query
   // q~ as bf16 high part (kind 1) and bf16 remainder (kind 2): rows g, dims
   // 16kk + 2q.. and 16kk + 2q + 8..; rows g >= G are zero, and a1 = a3 = 0
-  // (rows g + 8).
+  // (rows g + 8).  With the INT8 reference, kinds 3 and 4 are the f16 high
+  // part and remainder of q~ 2^E (dims 16kk + 4q ..).
   auto qfrag_addr = [&](int kind, int kk) {
     return smem_u32(qfrag + ((kind * KT + kk) * 32 + lane) * 2);
   };
   // softmax state of row g (lanes with row_ok), and the output accumulators
   // (O^T fragments: dims 16mt + g (+8), rows 2q, 2q + 1)
   float m_run = kNegInf, l_run = 0.0f;
-  float wsum[NG];
+  float wsum[NG], wsumR[NG];
   float oref[KT][4], ores[KT][4];
 
   auto reset_state = [&]() {
     m_run = kNegInf;
     l_run = 0.0f;
 #pragma unroll
-    for (int j = 0; j < NG; ++j) wsum[j] = 0.0f;
+    for (int j = 0; j < NG; ++j) {
+      wsum[j] = 0.0f;
+      wsumR[j] = 0.0f;
+    }
 #pragma unroll
     for (int mt = 0; mt < KT; ++mt)
 #pragma unroll
@@ -331,6 +410,45 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
     float* qt = qbuf + G * D;
     load_rotate_queries<D, G>(p, hd, qs, qt, tid);
     const float cd = rot_scale<D>();
+    if constexpr (C::CR) {
+      if (warp == 0) {
+        // f16 fragments of q~ 2^E, E per row so that max |q~| 2^E is in
+        // [2^13, 2^14): the high parts keep 11 bits, the remainders the next
+        // 11, and no value leaves f16's normal range.  k positions 2q, 2q+1 |
+        // 2q+8, 2q+9 of k-step kk carry dims 16kk + 4q .. 4q+3, the four codes
+        // one 32-bit ldmatrix word of the INT8 rows holds.
+        float mx = 0.0f;
+        if (row_ok)
+          for (int d = q; d < D; d += 4) mx = fmaxf(mx, fabsf(cd * qt[g * D + d]));
+        mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 2));
+        const int ex = (int)((__float_as_uint(mx) >> 23) & 0xFFu) - 127;
+        const int E = min(13 - ex, 126);
+        const float up = __uint_as_float((uint32_t)(127 + E) << 23);
+        if (row_ok && q == 0) rsig_s[g] = __uint_as_float((uint32_t)(127 - E) << 23);
+        float sqh = 0.0f;
+#pragma unroll 1
+        for (int kk = 0; kk < KT; ++kk) {
+          uint32_t* f3 = qfrag + ((3 * KT + kk) * 32 + lane) * 2;
+          uint32_t* f4 = qfrag + ((4 * KT + kk) * 32 + lane) * 2;
+          if (row_ok) {
+            const float* trow = qt + g * D + 16 * kk + 4 * q;
+            split_f16(cd * trow[0] * up, cd * trow[1] * up, f3[0], f4[0]);
+            split_f16(cd * trow[2] * up, cd * trow[3] * up, f3[1], f4[1]);
+            sqh += ((f16_lo_f(f3[0]) + f16_lo_f(f4[0])) + (f16_hi_f(f3[0]) + f16_hi_f(f4[0]))) +
+                   ((f16_lo_f(f3[1]) + f16_lo_f(f4[1])) + (f16_hi_f(f3[1]) + f16_hi_f(f4[1])));
+          } else {
+            f3[0] = f3[1] = f4[0] = f4[1] = 0u;
+          }
+          if ((kk + 1) % KSG == 0) {                   // end of a scale group
+            sqh += __shfl_xor_sync(FULL, sqh, 1);
+            sqh += __shfl_xor_sync(FULL, sqh, 2);
+            if (row_ok && q == 0) sqh_s[g * NG + kk / KSG] = sqh;
+            sqh = 0.0f;
+          }
+        }
+      }
+    }
     if (warp == 0) {
       float sqj = 0.0f;      // running sum of the current scale group (INT2)
 #pragma unroll 1
@@ -378,47 +496,65 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
     for (int j = 0; j < NG; ++j) {
       wsum[j] += __shfl_xor_sync(FULL, wsum[j], 1);
       wsum[j] += __shfl_xor_sync(FULL, wsum[j], 2);
+      if constexpr (C::CR) {
+        wsumR[j] += __shfl_xor_sync(FULL, wsumR[j], 1);
+        wsumR[j] += __shfl_xor_sync(FULL, wsumR[j], 2);
+      }
     }
     named_bar_sync(1, kConsumerThreads);          // merge area free
     float* mw = merge + warp * G * (2 + 2 * D);
     if (row_ok && q == 0) {
       mw[g * (2 + 2 * D)] = m_run;
       mw[g * (2 + 2 * D) + 1] = l_run;
-      if constexpr (C::RES) {
 #pragma unroll
-        for (int j = 0; j < NG; ++j) wsum_s[(warp * G + g) * NG + j] = wsum[j];
+      for (int j = 0; j < NG; ++j) {
+        if constexpr (C::RES) wsum_s[(warp * G + g) * NG + j] = wsum[j];
+        if constexpr (C::CR) wsumR_s[(warp * G + g) * NG + j] = wsumR[j];
       }
     }
-    // O^T fragments: c0 (dim 16mt+g, row 2q), c1 (.., row 2q+1), c2/c3 dim +8
+    // O^T fragments: c0 (dim 16mt+g, row 2q), c1 (.., row 2q+1), c2/c3 dim +8;
+    // the INT8 reference's m-rows g, g + 8 are dims 16mt + 2g, 16mt + 2g + 1
 #pragma unroll
     for (int mt = 0; mt < KT; ++mt) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int r = 2 * q + (e & 1);
         const int dim = 16 * mt + g + 8 * (e >> 1);
+        const int dim_ref = C::CR ? 16 * mt + 2 * g + (e >> 1) : dim;
         if (r < G) {
-          mw[r * (2 + 2 * D) + 2 + dim] = oref[mt][e];
+          mw[r * (2 + 2 * D) + 2 + dim_ref] = oref[mt][e];
           if constexpr (C::RES) mw[r * (2 + 2 * D) + 2 + D + dim] = 2.0f * ores[mt][e];
           else mw[r * (2 + 2 * D) + 2 + D + dim] = 0.0f;
         }
       }
     }
     named_bar_sync(1, kConsumerThreads);
-    if constexpr (C::RES) {
-      // complete sum_t p s (2c - top) = 2 sum p s c - top sum p s
+    if constexpr (C::RES || C::CR) {
+      // complete sum_t p s (2c - top) = 2 sum p s c - top sum p s; the INT8
+      // reference's sum_t p s_ref (2c - 255) = acc - (2176 + 255) sum p s_ref
+      // (acc = sum w (128 + 2 c_lo) + 16 w (128 + 2 c_hi)), moved to the
+      // rotated part
       for (int e = tid; e < kConsumerWarps * G * D; e += kConsumerThreads) {
         const int w = e / (G * D), r = (e / D) % G, dim = e % D;
-        merge[(w * G + r) * (2 + 2 * D) + 2 + D + dim] -=
-            (float)TOPLVL * wsum_s[(w * G + r) * NG + dim / GROUP];
+        float* rec = merge + (w * G + r) * (2 + 2 * D);
+        const int wi = (w * G + r) * NG + dim / GROUP;
+        float z = rec[2 + D + dim];
+        if constexpr (C::RES) z -= (float)TOPLVL * wsum_s[wi];
+        if constexpr (C::CR) {
+          z += rec[2 + dim] - 2431.0f * wsumR_s[wi];
+          rec[2 + dim] = 0.0f;
+        }
+        rec[2 + D + dim] = z;
       }
       named_bar_sync(1, kConsumerThreads);
     }
-    finish_head<D, G, C::RES>(p, hd, first_tile, nt_h, split, cta, merge, qbuf, flags, tid);
+    finish_head<D, G, C::RES || C::CR>(p, hd, first_tile, nt_h, split, cta, merge, qbuf, flags,
+                                       tid);
   };
 
   // ---- one tile ----
   auto tile_mma = [&](const unsigned char* st, int n, int sc_off) {
-    if (n < TILE) {
+    if (!C::CR && n < TILE) {
       // rows past the head's last token (spare capacity, the next head, or
       // nothing ever written) are not part of the context: their weights are
       // 0, and zeroing this warp's such V rows keeps a non-finite value there
@@ -444,19 +580,57 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
     // ldmatrix: matrices (tile 0, dims +0..7), (tile 0, +8..15), (tile 1, ..), (tile 1, ..)
     const int ktr = wtok + ((lane >> 4) & 1) * 8 + r7;
     const int kch = (lane >> 3) & 1;
+    // INT8 reference: per-group f16 sums sum_k q~_k 2^E (1024 + c_k)
+    float c8[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
+    uint32_t b8[4];          // ldmatrix words of two k-steps: (nt 0, kk), (nt 1, kk), (nt 0, kk + 1), ..
 #pragma unroll
     for (int kk = 0; kk < KT; ++kk) {
-      const int chunk = 2 * kk + kch;
-      uint32_t b[4];
-      ldsm_x4(sK + (chunk >> 3) * C::BOX_BYTES + ktr * 128 + (((chunk & 7) ^ r7) << 4), b);
-      uint32_t a[4] = {0u, 0u, 0u, 0u};
-      {
-        const uint2 f = *reinterpret_cast<const uint2*>(qfrag + ((0 * KT + kk) * 32 + lane) * 2);
-        a[0] = f.x;
-        a[2] = f.y;
+      if constexpr (C::CR) {
+        if ((kk & 1) == 0) {
+          const int m = lane >> 3;
+          ldsm_x4(sK + swz_offset<D>(wtok + (m & 1) * 8 + r7, kk + (m >> 1)), b8);
+        }
+        const uint2 fh = *reinterpret_cast<const uint2*>(qfrag + ((3 * KT + kk) * 32 + lane) * 2);
+        const uint2 fl = *reinterpret_cast<const uint2*>(qfrag + ((4 * KT + kk) * 32 + lane) * 2);
+        const uint32_t ah[4] = {fh.x, 0u, fh.y, 0u};
+        const uint32_t al[4] = {fl.x, 0u, fl.y, 0u};
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          // codes 4q .. 4q+3 of the k-step's 16 as f16 1024 + c, exact
+          const uint32_t w = b8[2 * (kk & 1) + nt];
+          const uint32_t b0 = __byte_perm(w, 0x64u, 0x4140);
+          const uint32_t b1 = __byte_perm(w, 0x64u, 0x4342);
+          mma_f16(c8[nt], ah, b0, b1);
+          mma_f16(c8[nt], al, b0, b1);
+        }
+      } else {
+        const int chunk = 2 * kk + kch;
+        uint32_t b[4];
+        ldsm_x4(sK + (chunk >> 3) * C::BOX_BYTES + ktr * 128 + (((chunk & 7) ^ r7) << 4), b);
+        uint32_t a[4] = {0u, 0u, 0u, 0u};
+        {
+          const uint2 f = *reinterpret_cast<const uint2*>(qfrag + ((0 * KT + kk) * 32 + lane) * 2);
+          a[0] = f.x;
+          a[2] = f.y;
+        }
+        mma_bf16(cref[0], a, b[0], b[1]);
+        mma_bf16(cref[1], a, b[2], b[3]);
       }
-      mma_bf16(cref[0], a, b[0], b[1]);
-      mma_bf16(cref[1], a, b[2], b[3]);
+      if (C::CR && (kk + 1) % KSG == 0) {
+        // end of scale group j: S += s_ref_{t, j} 2^-E (2 acc - (2048 + 255) sum q~ 2^E)
+        const int j = kk / KSG;
+        const float rs = row_ok ? rsig_s[g] : 0.0f;
+        const float off = row_ok ? 2303.0f * sqh_s[g * NG + j] : 0.0f;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          const float r0 = half_at(st + C::OFF_RSK + sc_off + tok0[nt] * SB + 2 * j);
+          const float r1 = half_at(st + C::OFF_RSK + sc_off + (tok0[nt] + 1) * SB + 2 * j);
+          cref[nt][0] = fmaf(r0 * rs, fmaf(2.0f, c8[nt][0], -off), cref[nt][0]);
+          cref[nt][1] = fmaf(r1 * rs, fmaf(2.0f, c8[nt][1], -off), cref[nt][1]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) c8[nt][e] = 0.0f;
+        }
+      }
       if constexpr (C::RES) {
         const uint2 fh = *reinterpret_cast<const uint2*>(qfrag + ((1 * KT + kk) * 32 + lane) * 2);
         const uint2 fl = *reinterpret_cast<const uint2*>(qfrag + ((2 * KT + kk) * 32 + lane) * 2);
@@ -531,25 +705,76 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
         }
       }
 #pragma unroll
-      for (int j = 0; j < NG; ++j) wsum[j] *= alpha;
+      for (int j = 0; j < NG; ++j) {
+        wsum[j] *= alpha;
+        wsumR[j] *= alpha;
+      }
     }
     // P^T fragments (k = tokens 2q, 2q+1 / +8, n = row g): bf16 hi + lo
     const uint32_t ph0 = pack_bf16(pr[0][0], pr[0][1]);
     const uint32_t ph1 = pack_bf16(pr[1][0], pr[1][1]);
     const uint32_t pl0 = pack_bf16(pr[0][0] - bf16_lo_f(ph0), pr[0][1] - bf16_hi_f(ph0));
     const uint32_t pl1 = pack_bf16(pr[1][0] - bf16_lo_f(ph1), pr[1][1] - bf16_hi_f(ph1));
-    // ---- O_ref^T += V^T P^T ----
+    if constexpr (C::CR) {
+      // ---- O_ref^T += L_ref^T (P s_ref^V)^T, INT8 codes in nibbles ----
+      // ldmatrix.trans of the code rows: word = codes (token 2q: dims 2g,
+      // 2g+1; token 2q+1: dims 2g, 2g+1) of a 16-dim chunk; m-row g is dim
+      // 2g, m-row g + 8 dim 2g + 1
+      const int tk[4] = {wtok + 2 * q, wtok + 2 * q + 1, wtok + 2 * q + 8, wtok + 2 * q + 9};
+      const float pk[4] = {pr[0][0], pr[0][1], pr[1][0], pr[1][1]};
+      constexpr uint32_t NIB = 0x001E001Eu;
+      const uint32_t x16 = 0x41804180u, nzero = 0x80008000u;   // {16, 16}, {-0, -0}
 #pragma unroll
-    for (int mt = 0; mt < KT; ++mt) {
-      const int m = lane >> 3;                         // matrix this lane addresses
-      const int tr = wtok + (m >> 1) * 8 + r7;
-      const int chunk = 2 * mt + (m & 1);
-      const uint32_t addr = sV + (chunk >> 3) * C::BOX_BYTES + tr * 128 +
-                            ((((chunk & 7) ^ r7)) << 4);
-      uint32_t a[4];
-      ldsm_x4_trans(addr, a);
-      mma_bf16(oref[mt], a, ph0, ph1);
-      mma_bf16(oref[mt], a, pl0, pl1);
+      for (int j = 0; j < NG; ++j) {
+        float wv[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float sr = half_at(st + C::OFF_RSV + sc_off + tk[k] * SB + 2 * j);
+          wv[k] = (tk[k] < n) ? pk[k] * sr : 0.0f;       // weight 0 beyond the tile
+        }
+        wsumR[j] += (wv[0] + wv[1]) + (wv[2] + wv[3]);
+        uint32_t bh0, bl0, bh1, bl1;
+        split_bf16(wv[0], wv[1], bh0, bl0);
+        split_bf16(wv[2], wv[3], bh1, bl1);
+        // 16 w, exact
+        const uint32_t Bh0 = bfma2_u(bh0, x16, nzero), Bl0 = bfma2_u(bl0, x16, nzero);
+        const uint32_t Bh1 = bfma2_u(bh1, x16, nzero), Bl1 = bfma2_u(bl1, x16, nzero);
+#pragma unroll
+        for (int mt2 = j * KSG / 2; mt2 < (j + 1) * KSG / 2; ++mt2) {
+          const int m = lane >> 3;
+          uint32_t v[4];     // (tokens 0-7, chunk 2mt2), (8-15, 2mt2), (0-7, 2mt2+1), (8-15, ..)
+          ldsm_x4_trans(sV + swz_offset<D>(wtok + (m & 1) * 8 + r7, 2 * mt2 + (m >> 1)), v);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int mt = 2 * mt2 + h;
+            const uint32_t R0 = v[2 * h], R1 = v[2 * h + 1];
+            // 128 + 2 c_lo and 128 + 2 c_hi of the codes in bytes 0, 2 (dim 2g)
+            // and bytes 1, 3 (dim 2g + 1), one bf16 half each
+            const uint32_t alo[4] = {((R0 << 1) & NIB) | kMagic, ((R0 >> 7) & NIB) | kMagic,
+                                     ((R1 << 1) & NIB) | kMagic, ((R1 >> 7) & NIB) | kMagic};
+            const uint32_t ahi[4] = {((R0 >> 3) & NIB) | kMagic, ((R0 >> 11) & NIB) | kMagic,
+                                     ((R1 >> 3) & NIB) | kMagic, ((R1 >> 11) & NIB) | kMagic};
+            mma_bf16(oref[mt], alo, bh0, bh1);
+            mma_bf16(oref[mt], alo, bl0, bl1);
+            mma_bf16(oref[mt], ahi, Bh0, Bh1);
+            mma_bf16(oref[mt], ahi, Bl0, Bl1);
+          }
+        }
+      }
+    } else {
+      // ---- O_ref^T += V^T P^T ----
+#pragma unroll
+      for (int mt = 0; mt < KT; ++mt) {
+        const int m = lane >> 3;                         // matrix this lane addresses
+        const int tr = wtok + (m >> 1) * 8 + r7;
+        const int chunk = 2 * mt + (m & 1);
+        const uint32_t addr = sV + (chunk >> 3) * C::BOX_BYTES + tr * 128 +
+                              ((((chunk & 7) ^ r7)) << 4);
+        uint32_t a[4];
+        ldsm_x4_trans(addr, a);
+        mma_bf16(oref[mt], a, ph0, ph1);
+        mma_bf16(oref[mt], a, pl0, pl1);
+      }
     }
     // ---- O_res^T += C_V^T (P s^V)^T ----
     if constexpr (C::RES) {
@@ -636,38 +861,47 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
 
 // ---- host side ---------------------------------------------------------------
 
-template <int D, int G, int BITS, int GROUP>
+template <int D, int G, int BITS, int GROUP, int RB>
 cudaError_t launch_gqa_t(const GqaParams& gp, cudaStream_t stream) {
-  using C = GCfg<D, G, BITS, GROUP>;
+  using C = GCfg<D, G, BITS, GROUP, RB>;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(decode_gqa_kernel<D, G, BITS, GROUP>,
+    cudaError_t e = cudaFuncSetAttribute(decode_gqa_kernel<D, G, BITS, GROUP, RB>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  return launch_pdl(decode_gqa_kernel<D, G, BITS, GROUP>, gp.p.ctas, kDecodeThreads,
+  return launch_pdl(decode_gqa_kernel<D, G, BITS, GROUP, RB>, gp.p.ctas, kDecodeThreads,
                     C::SMEM_BYTES, stream, gp);
 }
 
-template <int D, int G>
+template <int D, int G, int RB>
 cudaError_t launch_gqa_g(int bits, const GqaParams& gp, cudaStream_t stream) {
   const int group = gp.p.group;
-  if (bits == 16) return launch_gqa_t<D, G, 16, 32>(gp, stream);   // no scales are read
+  if (bits == 16) {
+    if constexpr (RB == 0) {
+      return launch_gqa_t<D, G, 16, 32, RB>(gp, stream);   // no scales are read
+    } else {
+      return group == 32 ? launch_gqa_t<D, G, 16, 32, RB>(gp, stream)
+                         : launch_gqa_t<D, G, 16, 64, RB>(gp, stream);
+    }
+  }
   if (bits == 2)
-    return group == 32 ? launch_gqa_t<D, G, 2, 32>(gp, stream) : launch_gqa_t<D, G, 2, 64>(gp, stream);
+    return group == 32 ? launch_gqa_t<D, G, 2, 32, RB>(gp, stream)
+                       : launch_gqa_t<D, G, 2, 64, RB>(gp, stream);
   if (bits == 4)
-    return group == 32 ? launch_gqa_t<D, G, 4, 32>(gp, stream) : launch_gqa_t<D, G, 4, 64>(gp, stream);
+    return group == 32 ? launch_gqa_t<D, G, 4, 32, RB>(gp, stream)
+                       : launch_gqa_t<D, G, 4, 64, RB>(gp, stream);
   return cudaErrorInvalidValue;
 }
 
-template <int D>
+template <int D, int RB>
 cudaError_t launch_gqa_d(int G, int bits, const GqaParams& gp, cudaStream_t stream) {
   switch (G) {
-    case 2: return launch_gqa_g<D, 2>(bits, gp, stream);
-    case 4: return launch_gqa_g<D, 4>(bits, gp, stream);
-    case 8: return launch_gqa_g<D, 8>(bits, gp, stream);
+    case 2: return launch_gqa_g<D, 2, RB>(bits, gp, stream);
+    case 4: return launch_gqa_g<D, 4, RB>(bits, gp, stream);
+    case 8: return launch_gqa_g<D, 8, RB>(bits, gp, stream);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -681,11 +915,21 @@ cudaError_t launch_decode_gqa(int head_dim, int G, int bits, const DecodeParams&
   const unsigned long long rows =
       p.page_table ? (unsigned long long)p.n_pages * p.kv_heads * kDecodeTile
                    : (unsigned long long)p.batch * p.kv_heads * p.ctx_pitch;
+  if (p.ref_bits == 8) {
+    // the reference is INT8 code rows (head_dim bytes each)
+    if (!encode_bytes_map(&gp.tmap_k, p.rcodes_k, rows, head_dim, kDecodeTile) ||
+        !encode_bytes_map(&gp.tmap_v, p.rcodes_v, rows, head_dim, kDecodeTile))
+      return cudaErrorInvalidValue;
+    if (head_dim == 128) return launch_gqa_d<128, 8>(G, bits, gp, stream);
+    if (head_dim == 64) return launch_gqa_d<64, 8>(G, bits, gp, stream);
+    return cudaErrorInvalidValue;
+  }
+  if (p.ref_bits != 0) return cudaErrorInvalidValue;
   if (!encode_rows_map(&gp.tmap_k, p.ref_k, rows, head_dim, kDecodeTile) ||
       !encode_rows_map(&gp.tmap_v, p.ref_v, rows, head_dim, kDecodeTile))
     return cudaErrorInvalidValue;
-  if (head_dim == 128) return launch_gqa_d<128>(G, bits, gp, stream);
-  if (head_dim == 64) return launch_gqa_d<64>(G, bits, gp, stream);
+  if (head_dim == 128) return launch_gqa_d<128, 0>(G, bits, gp, stream);
+  if (head_dim == 64) return launch_gqa_d<64, 0>(G, bits, gp, stream);
   return cudaErrorInvalidValue;
 }
 

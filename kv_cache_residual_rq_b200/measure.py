@@ -103,11 +103,12 @@ def measure(w, reps, peak, emit):
               "bytes": nb, "gbs": nb / t / 1e9, "frac": nb / t / 1e9 / peak,
               "tokens_per_s_per_head_call": w.batch / t})
     assert rq.rq_workspace_status(ws) == 0
-    if w.G == 1 and w.name == "ouro1.4b_decode":
-        # compressed reference (reference loop as rotated INT8 / INT4 codes)
+    if w.name in ("ouro1.4b_decode", "deep_loop_gqa"):
+        # compressed reference (reference loop as rotated INT8 / INT4 codes;
+        # grouped queries: INT8)
         xk1 = synth.loop_kv(w, 0, 0, 1, refk)
         xv1 = synth.loop_kv(w, 0, 1, 1, refv)
-        for rb in (8, 4):
+        for rb in ((8, 4) if w.G == 1 else (8,)):
             t = _time(lambda: rq.encode_cr([xk1], refk, rb, [2], w.group, w.seed), reps, flush)
             nb_e = (rows * w.head_dim * 2 * 2 + rows * (w.head_dim * (rb + 2) // 8
                                                       + 2 * 2 * (w.head_dim // w.group)))
@@ -134,6 +135,7 @@ def measure(w, reps, peak, emit):
             del rck, rsk, ckc, skc, rcv, rsv, cvc, svc
         del xk1, xv1
         torch.cuda.empty_cache()
+    if w.G == 1 and w.name == "ouro1.4b_decode":
         # variable-length batch: seeded lengths in [ctx/8, ctx], the cache at
         # full capacity; bytes are those of the tokens actually present
         g = torch.Generator().manual_seed(w.seed * 977 + 5)

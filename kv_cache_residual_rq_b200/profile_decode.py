@@ -78,7 +78,7 @@ def main(argv=None):
             rq.decode_attention_cr(q, crref, *((ckc[0], cvc[0], skc[0], svc[0]) if bits != 16
                                               else (None,) * 4), bits, w.group, w.seed, w.ctx,
                                    out=out, workspace=ws, tail_k=tail_k, tail_v=tail_v,
-                                   n_tail=args.tail)
+                                   n_tail=args.tail, kv_heads=w.kv_heads)
         else:
             rq.decode_attention(q, refk, refv, ck, cv, sk, sv, bits, w.group, w.seed, out=out,
                                 workspace=ws, tail_k=tail_k, tail_v=tail_v, n_tail=args.tail)

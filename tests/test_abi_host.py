@@ -81,6 +81,27 @@ def _decode(shape, bits=2, q=FAKE, rk=FAKE, rv=FAKE, ck=FAKE, cv=FAKE, sk=FAKE, 
                                   ws_bytes, stream=0, check=False)
 
 
+
+def _decode_cr(shape, ref_bits=8, rck=FAKE, rsv=FAKE, bits=16, q=FAKE):
+    ws_bytes = rq.rq_decode_workspace_bytes(shape) or 1 << 30
+    return rq.rq_decode_attention_cr(shape, None, q, rck, FAKE, FAKE, rsv, ref_bits, None, None,
+                                      None, None, bits, 1, 0.0, None, None, 0, 0, FAKE, FAKE,
+                                      ws_bytes, stream=0, check=False)
+
+
+def test_cr_decode_rejects_bad_arguments_before_launch():
+    E = rq
+    gqa = rq.make_shape(2, 2, 100, 128, 32, q_heads=8)
+    # grouped queries need the INT8 reference; an INT4 one is refused
+    assert _decode_cr(gqa, ref_bits=4) == E.RQ_ERR_UNSUPPORTED
+    assert _decode_cr(gqa, ref_bits=3) == E.RQ_ERR_UNSUPPORTED
+    assert _decode_cr(rq.make_shape(2, 2, 100, 128, 32), ref_bits=16) == E.RQ_ERR_UNSUPPORTED
+    # past the format checks, INT8 with grouped queries reaches the pointer checks
+    assert _decode_cr(gqa, rck=None) == E.RQ_ERR_INVALID_ARG
+    assert _decode_cr(gqa, rsv=MISALIGNED) == E.RQ_ERR_ALIGNMENT
+    assert _decode_cr(gqa, q=MISALIGNED) == E.RQ_ERR_ALIGNMENT
+    assert _decode_cr(rq.make_shape(2, 1, 100, 128, 32, q_heads=16)) == E.RQ_ERR_UNSUPPORTED
+
 def test_decode_rejects_bad_arguments_before_launch():
     good = rq.make_shape(2, 2, 100, 128, 32, q_heads=8)
     E = rq

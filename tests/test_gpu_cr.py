@@ -179,3 +179,73 @@ def test_cr_decode_matches_oracle(ref_bits, bits, varlen):
             worst = max(worst, float(np.abs(got - want).max()))
     assert worst <= OUT_TOL
     print(f"ref INT{ref_bits} bits {bits} varlen {varlen}: max-abs {worst:.2e}")
+
+
+def oracle_cr_kv(xk, xv, refk, refv, ref_bits, bits, g, seed, b, h, ctx):
+    """fp64 K_hat, V_hat of (sequence b, kv head h) from the oracle's own encode."""
+    d = refk.shape[-1]
+    out = []
+    for src_x, src_r in ((xk, refk), (xv, refv)):
+        rw, rs, ww, ws = oracle.encode_rows_cr_f32(u16(src_x[b, h, :ctx]), u16(src_r[b, h, :ctx]),
+                                                   ref_bits, bits if bits != 16 else 2, g, seed)
+        out.append(oracle.reconstruct_rows_cr_f64(
+            rw, rs, ww if bits != 16 else None, ws if bits != 16 else None, ref_bits,
+            bits if bits != 16 else 2, g, seed, d))
+    return out
+
+
+@pytest.mark.parametrize("G,d,g,bits,varlen", [
+    (2, 128, 32, 2, False), (4, 128, 32, 4, True), (8, 128, 64, 2, True), (8, 128, 32, 16, False),
+    (4, 64, 32, 2, False), (2, 64, 64, 4, True), (8, 64, 32, 2, False), (4, 128, 64, 16, True)])
+def test_cr_decode_grouped_queries(G, d, g, bits, varlen):
+    """Grouped queries over an INT8 compressed reference (the tensor-core
+    kernel): G query rows per kv head, several tiles, ragged and empty lengths,
+    one tail token."""
+    lens = [0, 1, 130, 200] if varlen else [177, 177]
+    B, Hkv, cap, n_tail, ref_bits = len(lens), 2, 200, 1, 8
+    w = synth.Workload("crgqa", 2, 1, B, cap, Hkv * G, Hkv, d, g, (2,), (0.25,), 140 + G + d)
+    refk, refv = synth.reference(w, 0, 0), synth.reference(w, 0, 1)
+    xk, xv = synth.loop_kv(w, 0, 0, 1, refk), synth.loop_kv(w, 0, 1, 1, refv)
+    rb = bits if bits != 16 else 2
+    (rck, rsk), ck, sk = rq.encode_cr([xk], refk, ref_bits, [rb], g, w.seed)
+    (rcv, rsv), cv, sv = rq.encode_cr([xv], refv, ref_bits, [rb], g, w.seed)
+    q = synth.query(w, 0, 1)
+    tail_k = synth.reference(w, 0, 0, batch=B, ctx=n_tail + 2)
+    tail_v = synth.reference(w, 0, 1, batch=B, ctx=n_tail + 2)
+    if varlen:
+        # garbage past every length: NaN scales, all-ones codes
+        for buf in (rsk, rsv, sk[0], sv[0]):
+            v = buf[: B * Hkv * cap * (d // g) * 2].view(torch.int16).view(B, Hkv, cap, -1)
+            for bi, n in enumerate(lens):
+                v[bi, :, n:] = F16_NAN
+        for buf, bb in ((rck, ref_bits), (rcv, ref_bits), (ck[0], rb), (cv[0], rb)):
+            v = buf[: B * Hkv * cap * d * bb // 8].view(torch.int32).view(B, Hkv, cap, -1)
+            for bi, n in enumerate(lens):
+                v[bi, :, n:] = -1
+    ctx_lens = torch.tensor(lens, dtype=torch.int32, device="cuda") if varlen else None
+    out = rq.decode_attention_cr(q, (rck, rsk, rcv, rsv, ref_bits),
+                                 None if bits == 16 else ck[0], None if bits == 16 else cv[0],
+                                 None if bits == 16 else sk[0], None if bits == 16 else sv[0],
+                                 bits, g, w.seed, cap, ctx=None if varlen else lens[0],
+                                 ctx_lens=ctx_lens, tail_k=tail_k, tail_v=tail_v, n_tail=n_tail,
+                                 kv_heads=Hkv)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out).all()
+    worst = 0.0
+    for b in range(B):
+        for h in range(Hkv):
+            parts_k, parts_v = [], []
+            if lens[b] > 0:
+                kh, vh = oracle_cr_kv(xk, xv, refk, refv, ref_bits, bits, g, w.seed, b, h, lens[b])
+                parts_k.append(kh)
+                parts_v.append(vh)
+            parts_k.append(oracle.bf16_to_f32(u16(tail_k[b, h, :n_tail])).astype(np.float64))
+            parts_v.append(oracle.bf16_to_f32(u16(tail_v[b, h, :n_tail])).astype(np.float64))
+            qh = oracle.bf16_to_f32(u16(q[b, h * G:(h + 1) * G])).astype(np.float64)
+            want = oracle.attention_f64(qh, np.concatenate(parts_k), np.concatenate(parts_v),
+                                        1.0 / np.sqrt(d))
+            got = out[b, h * G:(h + 1) * G].double().cpu().numpy()
+            worst = max(worst, float(np.abs(got - want).max()))
+    assert worst <= OUT_TOL
+    print(f"G {G} d {d} group {g} bits {bits} varlen {varlen}: max-abs {worst:.2e}")
+
