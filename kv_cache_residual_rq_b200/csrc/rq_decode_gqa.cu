@@ -28,9 +28,10 @@
 // the values, l_ref = 2c - 255.  Its K codes enter an f16 MMA as the exact
 // values 1024 + c (one byte permute per two codes) against q~ scaled by a
 // power of two per row and split into f16 high and remainder parts; its V
-// codes enter a bf16 MMA split into nibbles, 128 + 2 c_lo and 128 + 2 c_hi
-// (exact), the high nibble against 16 x the weights.  The offsets are removed
-// once per scale group (scores) or when the warp flushes (values).
+// codes enter an f16 MMA the same way against the weights p s_ref, split into
+// f16 parts after a lazily updated power of two keeps them in f16's range.
+// The offsets are removed once per scale group (scores) or when the warp
+// flushes (values).
 //
 // The reference K/V tiles (BF16 rows, or INT8 code rows) arrive by TMA
 // tensor copies with the swizzle of their line width (conflict-free
@@ -386,11 +387,13 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
   // (O^T fragments: dims 16mt + g (+8), rows 2q, 2q + 1)
   float m_run = kNegInf, l_run = 0.0f;
   float wsum[NG], wsumR[NG];
+  float vscale = 1.0f;     // INT8 reference: power of two applied to the V weights
   float oref[KT][4], ores[KT][4];
 
   auto reset_state = [&]() {
     m_run = kNegInf;
     l_run = 0.0f;
+    vscale = 1.0f;
 #pragma unroll
     for (int j = 0; j < NG; ++j) {
       wsum[j] = 0.0f;
@@ -509,7 +512,7 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
 #pragma unroll
       for (int j = 0; j < NG; ++j) {
         if constexpr (C::RES) wsum_s[(warp * G + g) * NG + j] = wsum[j];
-        if constexpr (C::CR) wsumR_s[(warp * G + g) * NG + j] = wsumR[j];
+        if constexpr (C::CR) wsumR_s[(warp * G + g) * NG + j] = wsumR[j] * (1.0f / vscale);
       }
     }
     // O^T fragments: c0 (dim 16mt+g, row 2q), c1 (.., row 2q+1), c2/c3 dim +8;
@@ -522,7 +525,8 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
         const int dim = 16 * mt + g + 8 * (e >> 1);
         const int dim_ref = C::CR ? 16 * mt + 2 * g + (e >> 1) : dim;
         if (r < G) {
-          mw[r * (2 + 2 * D) + 2 + dim_ref] = oref[mt][e];
+          if constexpr (C::CR) mw[r * (2 + 2 * D) + 2 + dim_ref] = oref[mt][e] * (2.0f / vscale);
+          else mw[r * (2 + 2 * D) + 2 + dim_ref] = oref[mt][e];
           if constexpr (C::RES) mw[r * (2 + 2 * D) + 2 + D + dim] = 2.0f * ores[mt][e];
           else mw[r * (2 + 2 * D) + 2 + D + dim] = 0.0f;
         }
@@ -531,9 +535,9 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
     named_bar_sync(1, kConsumerThreads);
     if constexpr (C::RES || C::CR) {
       // complete sum_t p s (2c - top) = 2 sum p s c - top sum p s; the INT8
-      // reference's sum_t p s_ref (2c - 255) = acc - (2176 + 255) sum p s_ref
-      // (acc = sum w (128 + 2 c_lo) + 16 w (128 + 2 c_hi)), moved to the
-      // rotated part
+      // reference's sum_t p s_ref (2c - 255) = 2 acc - (2048 + 255) sum p s_ref
+      // (acc = sum p s_ref (1024 + c), written as 2 acc), moved to the rotated
+      // part
       for (int e = tid; e < kConsumerWarps * G * D; e += kConsumerThreads) {
         const int w = e / (G * D), r = (e / D) % G, dim = e % D;
         float* rec = merge + (w * G + r) * (2 + 2 * D);
@@ -541,7 +545,7 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
         float z = rec[2 + D + dim];
         if constexpr (C::RES) z -= (float)TOPLVL * wsum_s[wi];
         if constexpr (C::CR) {
-          z += rec[2 + dim] - 2431.0f * wsumR_s[wi];
+          z += rec[2 + dim] - 2303.0f * wsumR_s[wi];
           rec[2 + dim] = 0.0f;
         }
         rec[2 + D + dim] = z;
@@ -716,29 +720,52 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
     const uint32_t pl0 = pack_bf16(pr[0][0] - bf16_lo_f(ph0), pr[0][1] - bf16_hi_f(ph0));
     const uint32_t pl1 = pack_bf16(pr[1][0] - bf16_lo_f(ph1), pr[1][1] - bf16_hi_f(ph1));
     if constexpr (C::CR) {
-      // ---- O_ref^T += L_ref^T (P s_ref^V)^T, INT8 codes in nibbles ----
+      // ---- O_ref^T += C_ref^T (P s_ref^V 2^Ev)^T, codes as f16 1024 + c ----
       // ldmatrix.trans of the code rows: word = codes (token 2q: dims 2g,
       // 2g+1; token 2q+1: dims 2g, 2g+1) of a 16-dim chunk; m-row g is dim
-      // 2g, m-row g + 8 dim 2g + 1
+      // 2g, m-row g + 8 dim 2g + 1.  The weights p s_ref are f16 high parts
+      // and remainders after a warp-wide power of two vscale that keeps the
+      // tile's largest scale in [2^8, 2^15): no weight can overflow f16, and
+      // the remainders stay far above its subnormals for every weight that
+      // matters.  vscale changes lazily; the accumulators follow it exactly.
       const int tk[4] = {wtok + 2 * q, wtok + 2 * q + 1, wtok + 2 * q + 8, wtok + 2 * q + 9};
-      const float pk[4] = {pr[0][0], pr[0][1], pr[1][0], pr[1][1]};
-      constexpr uint32_t NIB = 0x001E001Eu;
-      const uint32_t x16 = 0x41804180u, nzero = 0x80008000u;   // {16, 16}, {-0, -0}
+      auto s_ref_v = [&](int k, int j) {               // 0 beyond the tile
+        const float v = half_at(st + C::OFF_RSV + sc_off + tk[k] * SB + 2 * j);
+        return (tk[k] < n) ? v : 0.0f;
+      };
+      float smax = 0.0f;
+#pragma unroll
+      for (int j = 0; j < NG; ++j)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) smax = fmaxf(smax, fabsf(s_ref_v(k, j)));
+      smax = fmaxf(smax, __shfl_xor_sync(FULL, smax, 1));
+      smax = fmaxf(smax, __shfl_xor_sync(FULL, smax, 2));
+      {
+        const float big = smax * vscale;                 // the same in every lane
+        if (smax > 0.0f && !(big >= 256.0f && big < 32768.0f)) {
+          const int ex = (int)((__float_as_uint(smax) >> 23) & 0xFFu) - 127;
+          const float nv = __uint_as_float((uint32_t)(127 + 12 - ex) << 23);
+          const float f = nv / vscale;                     // a power of two, exact
+#pragma unroll
+          for (int mt = 0; mt < KT; ++mt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) oref[mt][e] *= f;
+#pragma unroll
+          for (int j = 0; j < NG; ++j) wsumR[j] *= f;
+          vscale = nv;
+        }
+      }
+      const float pk[4] = {pr[0][0] * vscale, pr[0][1] * vscale, pr[1][0] * vscale,
+                           pr[1][1] * vscale};
 #pragma unroll
       for (int j = 0; j < NG; ++j) {
         float wv[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float sr = half_at(st + C::OFF_RSV + sc_off + tk[k] * SB + 2 * j);
-          wv[k] = (tk[k] < n) ? pk[k] * sr : 0.0f;       // weight 0 beyond the tile
-        }
+        for (int k = 0; k < 4; ++k) wv[k] = pk[k] * s_ref_v(k, j);
         wsumR[j] += (wv[0] + wv[1]) + (wv[2] + wv[3]);
         uint32_t bh0, bl0, bh1, bl1;
-        split_bf16(wv[0], wv[1], bh0, bl0);
-        split_bf16(wv[2], wv[3], bh1, bl1);
-        // 16 w, exact
-        const uint32_t Bh0 = bfma2_u(bh0, x16, nzero), Bl0 = bfma2_u(bl0, x16, nzero);
-        const uint32_t Bh1 = bfma2_u(bh1, x16, nzero), Bl1 = bfma2_u(bl1, x16, nzero);
+        split_f16(wv[0], wv[1], bh0, bl0);
+        split_f16(wv[2], wv[3], bh1, bl1);
 #pragma unroll
         for (int mt2 = j * KSG / 2; mt2 < (j + 1) * KSG / 2; ++mt2) {
           const int m = lane >> 3;
@@ -748,16 +775,11 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
           for (int h = 0; h < 2; ++h) {
             const int mt = 2 * mt2 + h;
             const uint32_t R0 = v[2 * h], R1 = v[2 * h + 1];
-            // 128 + 2 c_lo and 128 + 2 c_hi of the codes in bytes 0, 2 (dim 2g)
-            // and bytes 1, 3 (dim 2g + 1), one bf16 half each
-            const uint32_t alo[4] = {((R0 << 1) & NIB) | kMagic, ((R0 >> 7) & NIB) | kMagic,
-                                     ((R1 << 1) & NIB) | kMagic, ((R1 >> 7) & NIB) | kMagic};
-            const uint32_t ahi[4] = {((R0 >> 3) & NIB) | kMagic, ((R0 >> 11) & NIB) | kMagic,
-                                     ((R1 >> 3) & NIB) | kMagic, ((R1 >> 11) & NIB) | kMagic};
-            mma_bf16(oref[mt], alo, bh0, bh1);
-            mma_bf16(oref[mt], alo, bl0, bl1);
-            mma_bf16(oref[mt], ahi, Bh0, Bh1);
-            mma_bf16(oref[mt], ahi, Bl0, Bl1);
+            // bytes 0, 2 (dim 2g) and bytes 1, 3 (dim 2g + 1) as f16 1024 + c
+            const uint32_t a[4] = {__byte_perm(R0, 0x64u, 0x4240), __byte_perm(R0, 0x64u, 0x4341),
+                                   __byte_perm(R1, 0x64u, 0x4240), __byte_perm(R1, 0x64u, 0x4341)};
+            mma_f16(oref[mt], a, bh0, bh1);
+            mma_f16(oref[mt], a, bl0, bl1);
           }
         }
       }
