@@ -366,7 +366,11 @@ rq_status rq_decode_attention_varlen(const rq_shape *shape, const int32_t *ctx_l
  *   ref_codes_k/v, ref_scales_k/v, ref_bits (4 or 8): the reference's
  *               codes and fp16 scales, [batch][Hkv][T_cap][...].
  * Tail tokens (BF16 K/V of the current token) and every other argument as
- * rq_decode_attention_tail.
+ * rq_decode_attention_tail.  Range: with G = 1 and ref_bits 8 the value
+ * weights p s_ref are fp16 with p < 2^8, so reference scales above 2^8
+ * (groups of rotated reference values beyond ~32000) are outside the format;
+ * such a call, or one whose reference scales are not finite, sets workspace
+ * status bit 64 and its output is not valid.
  */
 rq_status rq_decode_attention_cr(const rq_shape *shape, const int32_t *ctx_lens,
                                  const uint16_t *q, const uint32_t *ref_codes_k,
@@ -485,9 +489,11 @@ rq_status rq_encode_take_status(uint32_t *host_status);
 
 /* Copies the workspace's device status word to *host_status (blocking read
  * on `stream`).  0 means every decode call since the workspace was zeroed
- * ran clean; non-zero means a bounded wait inside a kernel ran out, its
- * output is invalid, and the workspace must be zeroed again.  This is the
- * only entry point that synchronises. */
+ * ran clean; non-zero means a call's output is invalid and the workspace must
+ * be zeroed again: bits 1, 2, 8 a bounded wait inside a kernel ran out, 4 a
+ * partial-record slot out of range, 16 a sequence length clamped to the
+ * capacity, 32 a page id outside the pool, 64 a compressed-reference weight
+ * out of range.  This is the only entry point that synchronises. */
 rq_status rq_workspace_status(const void *workspace, size_t workspace_bytes,
                               uint32_t *host_status, void *stream);
 

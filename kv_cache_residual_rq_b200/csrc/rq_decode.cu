@@ -478,6 +478,11 @@ decode_kernel(const DecodeParams p) {
     }
     named_bar_sync(1, kConsumerThreads);          // merge area (and table) free
     float* mw = merge + warp * G * (2 + 2 * D);
+    if constexpr (RB == 8 && DPL == 8) {
+      // an fp16 weight p s_ref overflowed (reference scales above 2^8 with
+      // the lazy softmax's p up to 2^8): the output is not valid
+      if (lane == 0 && !isfinite(wsumR[0])) flag_error(p.status, 64u);
+    }
     if (slot == 0) {
 #pragma unroll
       for (int r = 0; r < G; ++r) {

@@ -506,6 +506,13 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
     }
     named_bar_sync(1, kConsumerThreads);          // merge area free
     float* mw = merge + warp * G * (2 + 2 * D);
+    if constexpr (C::CR) {
+      // non-finite reference weights (invalid scales): the output is not valid
+      bool bad = false;
+#pragma unroll
+      for (int j = 0; j < NG; ++j) bad |= !isfinite(wsumR[j]);
+      if (row_ok && q == 0 && bad) flag_error(p.status, 64u);
+    }
     if (row_ok && q == 0) {
       mw[g * (2 + 2 * D)] = m_run;
       mw[g * (2 + 2 * D) + 1] = l_run;
@@ -725,9 +732,11 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
       // 2g+1; token 2q+1: dims 2g, 2g+1) of a 16-dim chunk; m-row g is dim
       // 2g, m-row g + 8 dim 2g + 1.  The weights p s_ref are f16 high parts
       // and remainders after a warp-wide power of two vscale that keeps the
-      // tile's largest scale in [2^8, 2^15): no weight can overflow f16, and
-      // the remainders stay far above its subnormals for every weight that
-      // matters.  vscale changes lazily; the accumulators follow it exactly.
+      // tile's largest scale in [1, 2^7): with p < 2^kLazyMax = 2^8 (the
+      // lazy softmax max) no weight reaches 2^15, below f16's largest value,
+      // and the remainders stay far above its subnormals for every weight
+      // that matters.  vscale changes lazily; the accumulators follow it
+      // exactly.
       const int tk[4] = {wtok + 2 * q, wtok + 2 * q + 1, wtok + 2 * q + 8, wtok + 2 * q + 9};
       auto s_ref_v = [&](int k, int j) {               // 0 beyond the tile
         const float v = half_at(st + C::OFF_RSV + sc_off + tk[k] * SB + 2 * j);
@@ -742,9 +751,10 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
       smax = fmaxf(smax, __shfl_xor_sync(FULL, smax, 2));
       {
         const float big = smax * vscale;                 // the same in every lane
-        if (smax > 0.0f && !(big >= 256.0f && big < 32768.0f)) {
+        static_assert(kLazyMax <= 8.0f, "p s_ref vscale < 2^(kLazyMax + 7) must fit f16");
+        if (smax > 0.0f && !(big >= 1.0f && big < 128.0f)) {
           const int ex = (int)((__float_as_uint(smax) >> 23) & 0xFFu) - 127;
-          const float nv = __uint_as_float((uint32_t)(127 + 12 - ex) << 23);
+          const float nv = __uint_as_float((uint32_t)(127 + 3 - ex) << 23);   // [2^3, 2^4)
           const float f = nv / vscale;                     // a power of two, exact
 #pragma unroll
           for (int mt = 0; mt < KT; ++mt)

@@ -249,3 +249,55 @@ def test_cr_decode_grouped_queries(G, d, g, bits, varlen):
     assert worst <= OUT_TOL
     print(f"G {G} d {d} group {g} bits {bits} varlen {varlen}: max-abs {worst:.2e}")
 
+
+
+def test_cr_grouped_peaky_scores_long_context():
+    """Scores spread wide over many tiles: the lazy softmax lets weights grow
+    to 2^8 before the running max moves, which the INT8 reference's f16 value
+    weights must absorb without overflow."""
+    G, d, g, bits, B, Hkv, T = 4, 128, 32, 2, 2, 2, 1500
+    w = synth.Workload("crpeak", 2, 1, B, T, Hkv * G, Hkv, d, g, (bits,), (0.25,), 177)
+    refk, refv = synth.reference(w, 0, 0), synth.reference(w, 0, 1)
+    xk, xv = synth.loop_kv(w, 0, 0, 1, refk), synth.loop_kv(w, 0, 1, 1, refv)
+    (rck, rsk), ck, sk = rq.encode_cr([xk], refk, 8, [bits], g, w.seed)
+    (rcv, rsv), cv, sv = rq.encode_cr([xv], refv, 8, [bits], g, w.seed)
+    q = (synth.query(w, 0, 1).float() * 8.0).to(torch.bfloat16)
+    shape = rq.make_shape(B, Hkv, T, d, g, q_heads=Hkv * G)
+    ws = rq.alloc_workspace(shape, q.device)
+    out = rq.decode_attention_cr(q, (rck, rsk, rcv, rsv, 8), ck[0], cv[0], sk[0], sv[0], bits, g,
+                                 w.seed, T, workspace=ws, kv_heads=Hkv)
+    torch.cuda.synchronize()
+    assert rq.rq_workspace_status(ws) == 0
+    assert torch.isfinite(out).all()
+    worst = 0.0
+    for b in range(B):
+        for h in range(Hkv):
+            kh, vh = oracle_cr_kv(xk, xv, refk, refv, 8, bits, g, w.seed, b, h, T)
+            qh = oracle.bf16_to_f32(u16(q[b, h * G:(h + 1) * G])).astype(np.float64)
+            want = oracle.attention_f64(qh, kh, vh, 1.0 / np.sqrt(d))
+            worst = max(worst, float(np.abs(out[b, h * G:(h + 1) * G].double().cpu().numpy()
+                                            - want).max()))
+    assert worst <= OUT_TOL
+    print(f"peaky G {G}: max-abs {worst:.2e}")
+
+
+def test_cr_single_query_weight_overflow_sets_status():
+    """With one query row per kv head the INT8 reference's value weights are
+    fp16; reference scales at the fp16 maximum overflow them once a weight
+    exceeds 1, and the call reports it in workspace status bit 64.  The
+    context is long enough that every CTA's run spans several tiles (a later
+    tile's scores above the first tile's max give weights above 1)."""
+    d, g, B, H, T = 128, 32, 2, 2, 16384
+    w = synth.Workload("crovf", 2, 1, B, T, H, H, d, g, (2,), (0.25,), 178)
+    refk, refv = synth.reference(w, 0, 0), synth.reference(w, 0, 1)
+    xk, xv = synth.loop_kv(w, 0, 0, 1, refk), synth.loop_kv(w, 0, 1, 1, refv)
+    (rck, rsk), ck, sk = rq.encode_cr([xk], refk, 8, [2], g, w.seed)
+    (rcv, rsv), cv, sv = rq.encode_cr([xv], refv, 8, [2], g, w.seed)
+    rsv.view(torch.int16)[: B * H * T * (d // g)] = 0x7BFF          # fp16 65504
+    q = (synth.query(w, 0, 1).float() * 4.0).to(torch.bfloat16)
+    shape = rq.make_shape(B, H, T, d, g)
+    ws = rq.alloc_workspace(shape, q.device)
+    rq.decode_attention_cr(q, (rck, rsk, rcv, rsv, 8), ck[0], cv[0], sk[0], sv[0], 2, g, w.seed,
+                           T, workspace=ws)
+    torch.cuda.synchronize()
+    assert rq.rq_workspace_status(ws) & 64
