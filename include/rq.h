@@ -357,8 +357,7 @@ rq_status rq_decode_attention_varlen(const rq_shape *shape, const int32_t *ctx_l
  * in the rotated domain -- s = sigma <q~, s_ref l_ref + s l>, one Rot^T per
  * output row -- so no BF16 row is read; bits == 16 decodes the final loop
  * from the reference codes alone (codes/scales may then be NULL).
- * Query rows per kv head G = q_heads / kv_heads in {1, 2, 4, 8}; G > 1 needs
- * ref_bits 8 (RQ_ERR_UNSUPPORTED for an INT4 reference with G > 1).
+ * Query rows per kv head G = q_heads / kv_heads in {1, 2, 4, 8}.
  *   ctx_lens  : NULL (every sequence has shape->ctx tokens; workspace of
  *               rq_decode_workspace_bytes) or a device int32 [batch] as in
  *               rq_decode_attention_varlen (workspace of

@@ -358,8 +358,6 @@ rq_status decode_impl(const rq_shape* shape, const int32_t* ctx_lens, const uint
   if (cr.ref_bits != 0) {
     if (cr.ref_bits != 4 && cr.ref_bits != 8) return RQ_ERR_UNSUPPORTED;
     if (!shape) return RQ_ERR_INVALID_ARG;
-    // grouped queries run on the tensor-core kernel, which reads INT8 references
-    if (shape->q_heads != shape->kv_heads && cr.ref_bits != 8) return RQ_ERR_UNSUPPORTED;
     if (!cr.codes_k || !cr.codes_v || !cr.scales_k || !cr.scales_v) return RQ_ERR_INVALID_ARG;
     if (!aligned16(cr.codes_k) || !aligned16(cr.codes_v) || !aligned16(cr.scales_k) ||
         !aligned16(cr.scales_v))

@@ -60,15 +60,19 @@ struct GCfg {
   static constexpr int WTOK = TILE / kConsumerWarps;       // 16 tokens per warp
   static constexpr bool RES = (BITS != 16);
   static constexpr bool CR = (RB == 8);                    // INT8 compressed reference
+  static constexpr bool CR4 = (RB == 4);                   // INT4 compressed reference
+  static constexpr bool CRX = (RB != 0);                   // either
+  static constexpr int RCROW = CR4 ? D / 2 : 0;            // INT4 reference code bytes per token
+  static constexpr int RCWORDS = RCROW / 4;
   static constexpr int NBOX = D / 64;                      // 64-column boxes per row
   static constexpr int BOX_BYTES = 64 * 128;               // 64 rows x 128 B
   // one K or V reference tile: BF16 boxes, or the INT8 code rows (D bytes each)
-  static constexpr int REF_TILE_BYTES = CR ? TILE * D : NBOX * BOX_BYTES;
+  static constexpr int REF_TILE_BYTES = CR ? TILE * D : CR4 ? TILE * RCROW : NBOX * BOX_BYTES;
   static constexpr int KT = D / 16;                        // k-steps of 16 dims
   static constexpr int CROW = RES ? D * BITS / 8 : 0;      // code bytes per token
   static constexpr int CWORDS = CROW / 4;
   static constexpr int SC_BYTES = RES ? TILE * (2 * D / 32) + 32 : 0;
-  static constexpr int RSC_BYTES = CR ? TILE * (2 * D / 32) + 32 : 0;   // reference scales
+  static constexpr int RSC_BYTES = CRX ? TILE * (2 * D / 32) + 32 : 0;  // reference scales
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + REF_TILE_BYTES;
   static constexpr int OFF_CK = OFF_V + REF_TILE_BYTES;
@@ -86,9 +90,10 @@ struct GCfg {
   static constexpr int KSG = GROUP / 16;                   // k-steps per scale group
   static constexpr int SB = 2 * NG;                        // scale bytes per token
   // per warp, row and scale group: sum of p s^V (and of p s_ref^V)
-  static constexpr int WSUM_FLOATS = kConsumerWarps * G * NG * (CR ? 2 : 1);
-  // q, q~ high, q~ remainder (bf16); with CR also q~ 2^E high, remainder (f16)
-  static constexpr int QFRAG_WORDS = (CR ? 5 : 3) * KT * 32 * 2;
+  static constexpr int WSUM_FLOATS = kConsumerWarps * G * NG * (CRX ? 2 : 1);
+  // q, q~ high, q~ remainder (bf16); with CR also q~ 2^E high, remainder
+  // (f16); with CR4 q~ high, remainder (bf16, dims in order)
+  static constexpr int QFRAG_WORDS = (CRX ? 5 : 3) * KT * 32 * 2;
   // INT2: per (row, scale group) sum of the q~ fragments' values (offset of
   // the 128 + 2c operands); CR: the same for the f16 fragments (offset of
   // 1024 + c) and per row 2^-E; even count to keep the barriers 8-byte aligned
@@ -101,7 +106,7 @@ struct GCfg {
   static_assert(MERGE_FLOATS >= kVarlenMaxBatch + 1, "merge area holds the length scan");
   static_assert(GROUP == 32 || GROUP == 64, "scale group");
   static_assert(D == 64 || D == 128, "head_dim");
-  static_assert(RB == 0 || RB == 8, "reference: BF16 rows or INT8 codes");
+  static_assert(RB == 0 || RB == 4 || RB == 8, "reference: BF16 rows, INT4 or INT8 codes");
   static_assert(OFF_V % 1024 == 0, "swizzled tiles start on the pattern's period");
 };
 
@@ -323,18 +328,26 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
           ++issued;
           continue;
         }
-        uint32_t bytes = 2u * C::REF_TILE_BYTES;          // full boxes, OOB rows zero-filled
+        // full boxes (OOB rows zero-filled), or n rows of INT4 reference codes
+        uint32_t bytes = C::CR4 ? 2u * n * C::RCROW : 2u * C::REF_TILE_BYTES;
         size_t sc_lo = 0;
         uint32_t sc_bytes = 0;
-        if constexpr (C::RES || C::CR) {
+        if constexpr (C::RES || C::CRX) {
           const size_t start = row * SB;
           sc_lo = start & ~(size_t)15;
           sc_bytes = (uint32_t)(((start + (size_t)n * SB + 15) & ~(size_t)15) - sc_lo);
         }
         if constexpr (C::RES) bytes += 2u * n * C::CROW + 2u * sc_bytes;
-        if constexpr (C::CR) bytes += 2u * sc_bytes;
+        if constexpr (C::CRX) bytes += 2u * sc_bytes;
         mbar_arrive_expect_tx(&full_bar[s], bytes);
-        if constexpr (C::CR) {
+        if constexpr (C::CR4) {
+          bulk_g2s(st + C::OFF_K, p.rcodes_k + row * C::RCWORDS, n * C::RCROW, &full_bar[s]);
+          bulk_g2s(st + C::OFF_V, p.rcodes_v + row * C::RCWORDS, n * C::RCROW, &full_bar[s]);
+          bulk_g2s(st + C::OFF_RSK, reinterpret_cast<const unsigned char*>(p.rscales_k) + sc_lo,
+                   sc_bytes, &full_bar[s]);
+          bulk_g2s(st + C::OFF_RSV, reinterpret_cast<const unsigned char*>(p.rscales_v) + sc_lo,
+                   sc_bytes, &full_bar[s]);
+        } else if constexpr (C::CR) {
           // one box of whole code rows each
           tma_load_2d(st + C::OFF_K, &gp.tmap_k, 0, (int)row, &full_bar[s]);
           tma_load_2d(st + C::OFF_V, &gp.tmap_v, 0, (int)row, &full_bar[s]);
@@ -452,6 +465,23 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
         }
       }
     }
+    if constexpr (C::CR4) {
+      if (warp == 0) {
+        // bf16 high part and remainder of q~, dims in order (INT4 levels)
+#pragma unroll 1
+        for (int kk = 0; kk < KT; ++kk) {
+          uint32_t* f3 = qfrag + ((3 * KT + kk) * 32 + lane) * 2;
+          uint32_t* f4 = qfrag + ((4 * KT + kk) * 32 + lane) * 2;
+          if (row_ok) {
+            const float* trow = qt + g * D + 16 * kk + 2 * q;
+            split_bf16(cd * trow[0], cd * trow[1], f3[0], f4[0]);
+            split_bf16(cd * trow[8], cd * trow[9], f3[1], f4[1]);
+          } else {
+            f3[0] = f3[1] = f4[0] = f4[1] = 0u;
+          }
+        }
+      }
+    }
     if (warp == 0) {
       float sqj = 0.0f;      // running sum of the current scale group (INT2)
 #pragma unroll 1
@@ -499,14 +529,14 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
     for (int j = 0; j < NG; ++j) {
       wsum[j] += __shfl_xor_sync(FULL, wsum[j], 1);
       wsum[j] += __shfl_xor_sync(FULL, wsum[j], 2);
-      if constexpr (C::CR) {
+      if constexpr (C::CRX) {
         wsumR[j] += __shfl_xor_sync(FULL, wsumR[j], 1);
         wsumR[j] += __shfl_xor_sync(FULL, wsumR[j], 2);
       }
     }
     named_bar_sync(1, kConsumerThreads);          // merge area free
     float* mw = merge + warp * G * (2 + 2 * D);
-    if constexpr (C::CR) {
+    if constexpr (C::CRX) {
       // non-finite reference weights (invalid scales): the output is not valid
       bool bad = false;
 #pragma unroll
@@ -520,6 +550,7 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
       for (int j = 0; j < NG; ++j) {
         if constexpr (C::RES) wsum_s[(warp * G + g) * NG + j] = wsum[j];
         if constexpr (C::CR) wsumR_s[(warp * G + g) * NG + j] = wsumR[j] * (1.0f / vscale);
+        if constexpr (C::CR4) wsumR_s[(warp * G + g) * NG + j] = wsumR[j];
       }
     }
     // O^T fragments: c0 (dim 16mt+g, row 2q), c1 (.., row 2q+1), c2/c3 dim +8;
@@ -533,6 +564,7 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
         const int dim_ref = C::CR ? 16 * mt + 2 * g + (e >> 1) : dim;
         if (r < G) {
           if constexpr (C::CR) mw[r * (2 + 2 * D) + 2 + dim_ref] = oref[mt][e] * (2.0f / vscale);
+          else if constexpr (C::CR4) mw[r * (2 + 2 * D) + 2 + dim] = 2.0f * oref[mt][e];
           else mw[r * (2 + 2 * D) + 2 + dim_ref] = oref[mt][e];
           if constexpr (C::RES) mw[r * (2 + 2 * D) + 2 + D + dim] = 2.0f * ores[mt][e];
           else mw[r * (2 + 2 * D) + 2 + D + dim] = 0.0f;
@@ -540,8 +572,9 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
       }
     }
     named_bar_sync(1, kConsumerThreads);
-    if constexpr (C::RES || C::CR) {
-      // complete sum_t p s (2c - top) = 2 sum p s c - top sum p s; the INT8
+    if constexpr (C::RES || C::CRX) {
+      // complete sum_t p s (2c - top) = 2 sum p s c - top sum p s (the INT4
+      // reference the same way, written as 2 sum p s_ref c); the INT8
       // reference's sum_t p s_ref (2c - 255) = 2 acc - (2048 + 255) sum p s_ref
       // (acc = sum p s_ref (1024 + c), written as 2 acc), moved to the rotated
       // part
@@ -551,21 +584,21 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
         const int wi = (w * G + r) * NG + dim / GROUP;
         float z = rec[2 + D + dim];
         if constexpr (C::RES) z -= (float)TOPLVL * wsum_s[wi];
-        if constexpr (C::CR) {
-          z += rec[2 + dim] - 2303.0f * wsumR_s[wi];
+        if constexpr (C::CRX) {
+          z += rec[2 + dim] - (C::CR ? 2303.0f : 15.0f) * wsumR_s[wi];
           rec[2 + dim] = 0.0f;
         }
         rec[2 + D + dim] = z;
       }
       named_bar_sync(1, kConsumerThreads);
     }
-    finish_head<D, G, C::RES || C::CR>(p, hd, first_tile, nt_h, split, cta, merge, qbuf, flags,
-                                       tid);
+    finish_head<D, G, C::RES || C::CRX>(p, hd, first_tile, nt_h, split, cta, merge, qbuf, flags,
+                                        tid);
   };
 
   // ---- one tile ----
   auto tile_mma = [&](const unsigned char* st, int n, int sc_off) {
-    if (!C::CR && n < TILE) {
+    if (!C::CRX && n < TILE) {
       // rows past the head's last token (spare capacity, the next head, or
       // nothing ever written) are not part of the context: their weights are
       // 0, and zeroing this warp's such V rows keeps a non-finite value there
@@ -614,6 +647,20 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
           mma_f16(c8[nt], ah, b0, b1);
           mma_f16(c8[nt], al, b0, b1);
         }
+      } else if constexpr (C::CR4) {
+        // INT4 reference levels 2c - 15, exact in bf16, against q~ high + remainder
+        const uint2 fh = *reinterpret_cast<const uint2*>(qfrag + ((3 * KT + kk) * 32 + lane) * 2);
+        const uint2 fl = *reinterpret_cast<const uint2*>(qfrag + ((4 * KT + kk) * 32 + lane) * 2);
+        const uint32_t ah[4] = {fh.x, 0u, fh.y, 0u};
+        const uint32_t al[4] = {fl.x, 0u, fl.y, 0u};
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          const uint2 w2 = *reinterpret_cast<const uint2*>(st + C::OFF_K + tb[nt] * C::RCROW + 8 * kk);
+          uint32_t b0, b1;
+          k_levels<4>(w2.x, w2.y, q, b0, b1);
+          mma_bf16(c8[nt], ah, b0, b1);
+          mma_bf16(c8[nt], al, b0, b1);
+        }
       } else {
         const int chunk = 2 * kk + kch;
         uint32_t b[4];
@@ -627,17 +674,26 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
         mma_bf16(cref[0], a, b[0], b[1]);
         mma_bf16(cref[1], a, b[2], b[3]);
       }
-      if (C::CR && (kk + 1) % KSG == 0) {
+      if (C::CRX && (kk + 1) % KSG == 0) {
         // end of scale group j: S += s_ref_{t, j} 2^-E (2 acc - (2048 + 255) sum q~ 2^E)
+        // (INT8), S += s_ref_{t, j} acc (INT4: the levels themselves)
         const int j = kk / KSG;
-        const float rs = row_ok ? rsig_s[g] : 0.0f;
-        const float off = row_ok ? 2303.0f * sqh_s[g * NG + j] : 0.0f;
+        float rs = 1.0f, off = 0.0f;
+        if constexpr (C::CR) {
+          rs = row_ok ? rsig_s[g] : 0.0f;
+          off = row_ok ? 2303.0f * sqh_s[g * NG + j] : 0.0f;
+        }
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
           const float r0 = half_at(st + C::OFF_RSK + sc_off + tok0[nt] * SB + 2 * j);
           const float r1 = half_at(st + C::OFF_RSK + sc_off + (tok0[nt] + 1) * SB + 2 * j);
-          cref[nt][0] = fmaf(r0 * rs, fmaf(2.0f, c8[nt][0], -off), cref[nt][0]);
-          cref[nt][1] = fmaf(r1 * rs, fmaf(2.0f, c8[nt][1], -off), cref[nt][1]);
+          if constexpr (C::CR) {
+            cref[nt][0] = fmaf(r0 * rs, fmaf(2.0f, c8[nt][0], -off), cref[nt][0]);
+            cref[nt][1] = fmaf(r1 * rs, fmaf(2.0f, c8[nt][1], -off), cref[nt][1]);
+          } else {
+            cref[nt][0] = fmaf(r0, c8[nt][0], cref[nt][0]);
+            cref[nt][1] = fmaf(r1, c8[nt][1], cref[nt][1]);
+          }
 #pragma unroll
           for (int e = 0; e < 4; ++e) c8[nt][e] = 0.0f;
         }
@@ -726,7 +782,44 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
     const uint32_t ph1 = pack_bf16(pr[1][0], pr[1][1]);
     const uint32_t pl0 = pack_bf16(pr[0][0] - bf16_lo_f(ph0), pr[0][1] - bf16_hi_f(ph0));
     const uint32_t pl1 = pack_bf16(pr[1][0] - bf16_lo_f(ph1), pr[1][1] - bf16_hi_f(ph1));
-    if constexpr (C::CR) {
+    if constexpr (C::CR4) {
+      // ---- O_ref^T += C_ref^T (P s_ref^V)^T, INT4 codes exact in bf16 ----
+      const int tk[4] = {wtok + 2 * q, wtok + 2 * q + 1, wtok + 2 * q + 8, wtok + 2 * q + 9};
+      const float pk[4] = {pr[0][0], pr[0][1], pr[1][0], pr[1][1]};
+#pragma unroll
+      for (int j = 0; j < NG; ++j) {
+        float wv[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float sr = half_at(st + C::OFF_RSV + sc_off + tk[k] * SB + 2 * j);
+          wv[k] = (tk[k] < n) ? pk[k] * sr : 0.0f;       // weight 0 beyond the tile
+        }
+        wsumR[j] += (wv[0] + wv[1]) + (wv[2] + wv[3]);
+        uint32_t bh0, bl0, bh1, bl1;
+        split_bf16(wv[0], wv[1], bh0, bl0);
+        split_bf16(wv[2], wv[3], bh1, bl1);
+#pragma unroll
+        for (int mt = j * KSG; mt < (j + 1) * KSG; ++mt) {
+          // codes of dims 16mt + g (lo halves) and 16mt + g + 8 (hi halves)
+          uint32_t x[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t* cw = reinterpret_cast<const uint32_t*>(st + C::OFF_V + tk[k] * C::RCROW);
+            const uint32_t lo = (cw[2 * mt] >> (4 * g)) & 0xFu;
+            const uint32_t hi = (cw[2 * mt + 1] >> (4 * g)) & 0xFu;
+            x[k] = lo | (hi << 16) | kMagic;
+          }
+          const uint32_t m128 = 0xC300C300u;   // {-128, -128}
+          uint32_t a[4];
+          a[0] = badd2_u(__byte_perm(x[0], x[1], 0x5410), m128);   // dim g,   tokens 2q, 2q+1
+          a[1] = badd2_u(__byte_perm(x[0], x[1], 0x7632), m128);   // dim g+8
+          a[2] = badd2_u(__byte_perm(x[2], x[3], 0x5410), m128);   // dim g,   tokens 2q+8, 2q+9
+          a[3] = badd2_u(__byte_perm(x[2], x[3], 0x7632), m128);   // dim g+8
+          mma_bf16(oref[mt], a, bh0, bh1);
+          mma_bf16(oref[mt], a, bl0, bl1);
+        }
+      }
+    } else if constexpr (C::CR) {
       // ---- O_ref^T += C_ref^T (P s_ref^V 2^Ev)^T, codes as f16 1024 + c ----
       // ldmatrix.trans of the code rows: word = codes (token 2q: dims 2g,
       // 2g+1; token 2q+1: dims 2g, 2g+1) of a 16-dim chunk; m-row g is dim
@@ -954,6 +1047,12 @@ cudaError_t launch_decode_gqa(int head_dim, int G, int bits, const DecodeParams&
       return cudaErrorInvalidValue;
     if (head_dim == 128) return launch_gqa_d<128, 8>(G, bits, gp, stream);
     if (head_dim == 64) return launch_gqa_d<64, 8>(G, bits, gp, stream);
+    return cudaErrorInvalidValue;
+  }
+  if (p.ref_bits == 4) {
+    // INT4 reference code rows by bulk copies (no tensor maps)
+    if (head_dim == 128) return launch_gqa_d<128, 4>(G, bits, gp, stream);
+    if (head_dim == 64) return launch_gqa_d<64, 4>(G, bits, gp, stream);
     return cudaErrorInvalidValue;
   }
   if (p.ref_bits != 0) return cudaErrorInvalidValue;

@@ -104,11 +104,10 @@ def measure(w, reps, peak, emit):
               "tokens_per_s_per_head_call": w.batch / t})
     assert rq.rq_workspace_status(ws) == 0
     if w.name in ("ouro1.4b_decode", "deep_loop_gqa"):
-        # compressed reference (reference loop as rotated INT8 / INT4 codes;
-        # grouped queries: INT8)
+        # compressed reference (reference loop as rotated INT8 / INT4 codes)
         xk1 = synth.loop_kv(w, 0, 0, 1, refk)
         xv1 = synth.loop_kv(w, 0, 1, 1, refv)
-        for rb in ((8, 4) if w.G == 1 else (8,)):
+        for rb in (8, 4):
             t = _time(lambda: rq.encode_cr([xk1], refk, rb, [2], w.group, w.seed), reps, flush)
             nb_e = (rows * w.head_dim * 2 * 2 + rows * (w.head_dim * (rb + 2) // 8
                                                       + 2 * 2 * (w.head_dim // w.group)))

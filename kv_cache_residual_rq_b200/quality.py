@@ -116,7 +116,7 @@ def study(w, emit):
         err = (torch.linalg.vector_norm(out - exact) / torch.linalg.vector_norm(exact)).item()
         emit({"workload": w.name, "tensor": "attention(loop 1)", "scheme": scheme, "bits": bits,
               "rel_output_err": err})
-    for rb in ((8, 4) if G == 1 else (8,)):
+    for rb in (8, 4):
         b1 = w.bits[0] if w.bits[0] != 16 else 2
         (rck, rsk), ck, sk = rq.encode_cr([xk], refk, rb, [b1], w.group, w.seed)
         (rcv, rsv), cv, sv = rq.encode_cr([xv], refv, rb, [b1], w.group, w.seed)

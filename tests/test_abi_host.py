@@ -92,12 +92,13 @@ def _decode_cr(shape, ref_bits=8, rck=FAKE, rsv=FAKE, bits=16, q=FAKE):
 def test_cr_decode_rejects_bad_arguments_before_launch():
     E = rq
     gqa = rq.make_shape(2, 2, 100, 128, 32, q_heads=8)
-    # grouped queries need the INT8 reference; an INT4 one is refused
-    assert _decode_cr(gqa, ref_bits=4) == E.RQ_ERR_UNSUPPORTED
     assert _decode_cr(gqa, ref_bits=3) == E.RQ_ERR_UNSUPPORTED
     assert _decode_cr(rq.make_shape(2, 2, 100, 128, 32), ref_bits=16) == E.RQ_ERR_UNSUPPORTED
-    # past the format checks, INT8 with grouped queries reaches the pointer checks
+    # past the format checks, INT8 and INT4 with grouped queries reach the
+    # pointer checks
     assert _decode_cr(gqa, rck=None) == E.RQ_ERR_INVALID_ARG
+    assert _decode_cr(gqa, ref_bits=4, rck=None) == E.RQ_ERR_INVALID_ARG
+    assert _decode_cr(gqa, ref_bits=4, rsv=MISALIGNED) == E.RQ_ERR_ALIGNMENT
     assert _decode_cr(gqa, rsv=MISALIGNED) == E.RQ_ERR_ALIGNMENT
     assert _decode_cr(gqa, q=MISALIGNED) == E.RQ_ERR_ALIGNMENT
     assert _decode_cr(rq.make_shape(2, 1, 100, 128, 32, q_heads=16)) == E.RQ_ERR_UNSUPPORTED

@@ -194,15 +194,18 @@ def oracle_cr_kv(xk, xv, refk, refv, ref_bits, bits, g, seed, b, h, ctx):
     return out
 
 
-@pytest.mark.parametrize("G,d,g,bits,varlen", [
-    (2, 128, 32, 2, False), (4, 128, 32, 4, True), (8, 128, 64, 2, True), (8, 128, 32, 16, False),
-    (4, 64, 32, 2, False), (2, 64, 64, 4, True), (8, 64, 32, 2, False), (4, 128, 64, 16, True)])
-def test_cr_decode_grouped_queries(G, d, g, bits, varlen):
-    """Grouped queries over an INT8 compressed reference (the tensor-core
-    kernel): G query rows per kv head, several tiles, ragged and empty lengths,
-    one tail token."""
+@pytest.mark.parametrize("ref_bits,G,d,g,bits,varlen", [
+    (8, 2, 128, 32, 2, False), (8, 4, 128, 32, 4, True), (8, 8, 128, 64, 2, True),
+    (8, 8, 128, 32, 16, False), (8, 4, 64, 32, 2, False), (8, 2, 64, 64, 4, True),
+    (8, 8, 64, 32, 2, False), (8, 4, 128, 64, 16, True),
+    (4, 4, 128, 32, 2, False), (4, 2, 128, 64, 4, True), (4, 8, 64, 32, 2, True),
+    (4, 4, 64, 64, 16, False), (4, 8, 128, 32, 16, True)])
+def test_cr_decode_grouped_queries(ref_bits, G, d, g, bits, varlen):
+    """Grouped queries over an INT8 or INT4 compressed reference (the
+    tensor-core kernel): G query rows per kv head, several tiles, ragged and
+    empty lengths, one tail token."""
     lens = [0, 1, 130, 200] if varlen else [177, 177]
-    B, Hkv, cap, n_tail, ref_bits = len(lens), 2, 200, 1, 8
+    B, Hkv, cap, n_tail = len(lens), 2, 200, 1
     w = synth.Workload("crgqa", 2, 1, B, cap, Hkv * G, Hkv, d, g, (2,), (0.25,), 140 + G + d)
     refk, refv = synth.reference(w, 0, 0), synth.reference(w, 0, 1)
     xk, xv = synth.loop_kv(w, 0, 0, 1, refk), synth.loop_kv(w, 0, 1, 1, refv)
@@ -247,7 +250,8 @@ def test_cr_decode_grouped_queries(G, d, g, bits, varlen):
             got = out[b, h * G:(h + 1) * G].double().cpu().numpy()
             worst = max(worst, float(np.abs(got - want).max()))
     assert worst <= OUT_TOL
-    print(f"G {G} d {d} group {g} bits {bits} varlen {varlen}: max-abs {worst:.2e}")
+    print(f"ref INT{ref_bits} G {G} d {d} group {g} bits {bits} varlen {varlen}: "
+          f"max-abs {worst:.2e}")
 
 
 
