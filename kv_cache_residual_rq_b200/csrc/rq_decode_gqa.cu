@@ -22,18 +22,22 @@
 // completed when the warp flushes.  Rows beyond G are zero and their weights
 // are forced to zero.
 //
-// Compressed INT8 reference (same page, the reference loop itself stored as
-// rotated codes): the reference term is one more quantised term in the
-// rotated domain, s_ref <q~, l_ref> for the scores and sum_t p s_ref l_ref for
-// the values, l_ref = 2c - 255.  Its K codes enter an f16 MMA as the exact
-// values 1024 + c (one byte permute per two codes) against q~ scaled by a
-// power of two per row and split into f16 high and remainder parts; its V
-// codes enter an f16 MMA the same way against the weights p s_ref, split into
-// f16 parts after a lazily updated power of two keeps them in f16's range.
-// The offsets are removed once per scale group (scores) or when the warp
-// flushes (values).
+// Compressed INT8 / INT4 reference (same page, the reference loop itself
+// stored as rotated codes): the reference term is one more quantised term in
+// the rotated domain, s_ref <q~, l_ref> for the scores and sum_t p s_ref l_ref
+// for the values, l_ref = 2c - (2^b - 1).  Its codes enter f16 MMAs as the
+// exact subnormals c 2^-24 -- the code in the low mantissa bits: one byte
+// permute per two INT8 codes, one shift and one mask per two INT4 codes, no
+// offset to cancel -- against q~ scaled by a power of two per row and split
+// into f16 high and remainder parts (scores), or against the weights p s_ref
+// split into f16 parts after a lazily updated power of two keeps them in
+// f16's range (values); the 2^24 returns with the scales, once per scale
+// group (scores) or when the warp flushes (values).  The reference rows (d or
+// d/2 bytes) arrive swizzled; the k order of the q~ fragments and the m-row
+// order of the value accumulators follow the codes' positions in the 32-bit
+// ldmatrix words.
 //
-// The reference K/V tiles (BF16 rows, or INT8 code rows) arrive by TMA
+// The reference K/V tiles (BF16 rows, or code rows) arrive by TMA
 // tensor copies with the swizzle of their line width (conflict-free
 // ldmatrix); codes and scales by plain bulk copies, as in the single-query
 // kernel.  The work split, the partial records and the
@@ -62,12 +66,16 @@ struct GCfg {
   static constexpr bool CR = (RB == 8);                    // INT8 compressed reference
   static constexpr bool CR4 = (RB == 4);                   // INT4 compressed reference
   static constexpr bool CRX = (RB != 0);                   // either
-  static constexpr int RCROW = CR4 ? D / 2 : 0;            // INT4 reference code bytes per token
-  static constexpr int RCWORDS = RCROW / 4;
+  static constexpr int RROW = CRX ? D * RB / 8 : 0;        // reference code bytes per token
+  // f16 operands of the reference codes: the exact subnormals c 2^-24 (the
+  // code in the low mantissa bits, no offset).  A sum acc over those operands
+  // gives the level sum  sum w (2c - (2^RB - 1)) = 2^25 acc - (2^RB - 1) sum w.
+  static constexpr float CSCALE = 33554432.0f;                        // 2^25
+  static constexpr float LOFF = (float)((1 << RB) - 1);
   static constexpr int NBOX = D / 64;                      // 64-column boxes per row
   static constexpr int BOX_BYTES = 64 * 128;               // 64 rows x 128 B
   // one K or V reference tile: BF16 boxes, or the INT8 code rows (D bytes each)
-  static constexpr int REF_TILE_BYTES = CR ? TILE * D : CR4 ? TILE * RCROW : NBOX * BOX_BYTES;
+  static constexpr int REF_TILE_BYTES = CRX ? TILE * RROW : NBOX * BOX_BYTES;
   static constexpr int KT = D / 16;                        // k-steps of 16 dims
   static constexpr int CROW = RES ? D * BITS / 8 : 0;      // code bytes per token
   static constexpr int CWORDS = CROW / 4;
@@ -91,13 +99,14 @@ struct GCfg {
   static constexpr int SB = 2 * NG;                        // scale bytes per token
   // per warp, row and scale group: sum of p s^V (and of p s_ref^V)
   static constexpr int WSUM_FLOATS = kConsumerWarps * G * NG * (CRX ? 2 : 1);
-  // q, q~ high, q~ remainder (bf16); with CR also q~ 2^E high, remainder
-  // (f16); with CR4 q~ high, remainder (bf16, dims in order)
+  // q, q~ high, q~ remainder (bf16); with a compressed reference also
+  // q~ 2^E high, remainder (f16, k-permuted for the reference's codes)
   static constexpr int QFRAG_WORDS = (CRX ? 5 : 3) * KT * 32 * 2;
   // INT2: per (row, scale group) sum of the q~ fragments' values (offset of
-  // the 128 + 2c operands); CR: the same for the f16 fragments (offset of
-  // 1024 + c) and per row 2^-E; even count to keep the barriers 8-byte aligned
-  static constexpr int SQ_FLOATS = (G * NG * (CR ? 2 : 1) + (CR ? G : 0) + 1) / 2 * 2;
+  // the 128 + 2c operands); compressed reference: the same for the f16
+  // fragments (the levels' 2^b - 1) and per row 2^-E; even count to keep the
+  // barriers 8-byte aligned
+  static constexpr int SQ_FLOATS = (G * NG * (CRX ? 2 : 1) + (CRX ? G : 0) + 1) / 2 * 2;
   static constexpr int SMEM_BYTES = 1024 /* base alignment slack */ + RING_BYTES +
                                     4 * (MERGE_FLOATS + QBUF_FLOATS + WSUM_FLOATS +
                                          QFRAG_WORDS + SQ_FLOATS) +
@@ -107,7 +116,8 @@ struct GCfg {
   static_assert(GROUP == 32 || GROUP == 64, "scale group");
   static_assert(D == 64 || D == 128, "head_dim");
   static_assert(RB == 0 || RB == 4 || RB == 8, "reference: BF16 rows, INT4 or INT8 codes");
-  static_assert(OFF_V % 1024 == 0, "swizzled tiles start on the pattern's period");
+  // the swizzle pattern repeats every 8 lines: 1024 B for 128-byte lines
+  static_assert(OFF_V % (CRX ? 8 * RROW : 1024) == 0, "swizzled tiles start on the period");
 };
 
 // ---- PTX wrappers -----------------------------------------------------------
@@ -124,6 +134,12 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x2_trans(uint32_t addr, uint32_t (&r)[2]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
+               : "=r"(r[0]), "=r"(r[1])
                : "r"(addr));
 }
 
@@ -154,12 +170,14 @@ __device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], u
 }
 
 // Byte offset of 16-byte chunk `chunk` of row `row` in a tile of rows of
-// RROW bytes (64 or 128) written by a TMA copy with the swizzle of that
-// width: address bits 4.. are XORed with bits 7.. (3 bits for 128 B, 2 for 64 B).
+// RROW bytes (32, 64 or 128) written by a TMA copy with the swizzle of that
+// width: address bits 4.. are XORed with bits 7.. (3 bits for 128 B, 2 for
+// 64 B, 1 for 32 B).
 template <int RROW>
 __device__ __forceinline__ uint32_t swz_offset(int row, int chunk) {
+  static_assert(RROW == 32 || RROW == 64 || RROW == 128, "swizzle width");
   const uint32_t o = (uint32_t)(row * RROW + chunk * 16);
-  constexpr uint32_t mask = RROW == 128 ? 7u : 3u;
+  constexpr uint32_t mask = RROW / 16 - 1;
   return o ^ (((o >> 7) & mask) << 4);
 }
 
@@ -328,8 +346,7 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
           ++issued;
           continue;
         }
-        // full boxes (OOB rows zero-filled), or n rows of INT4 reference codes
-        uint32_t bytes = C::CR4 ? 2u * n * C::RCROW : 2u * C::REF_TILE_BYTES;
+        uint32_t bytes = 2u * C::REF_TILE_BYTES;          // full boxes, OOB rows zero-filled
         size_t sc_lo = 0;
         uint32_t sc_bytes = 0;
         if constexpr (C::RES || C::CRX) {
@@ -340,14 +357,7 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
         if constexpr (C::RES) bytes += 2u * n * C::CROW + 2u * sc_bytes;
         if constexpr (C::CRX) bytes += 2u * sc_bytes;
         mbar_arrive_expect_tx(&full_bar[s], bytes);
-        if constexpr (C::CR4) {
-          bulk_g2s(st + C::OFF_K, p.rcodes_k + row * C::RCWORDS, n * C::RCROW, &full_bar[s]);
-          bulk_g2s(st + C::OFF_V, p.rcodes_v + row * C::RCWORDS, n * C::RCROW, &full_bar[s]);
-          bulk_g2s(st + C::OFF_RSK, reinterpret_cast<const unsigned char*>(p.rscales_k) + sc_lo,
-                   sc_bytes, &full_bar[s]);
-          bulk_g2s(st + C::OFF_RSV, reinterpret_cast<const unsigned char*>(p.rscales_v) + sc_lo,
-                   sc_bytes, &full_bar[s]);
-        } else if constexpr (C::CR) {
+        if constexpr (C::CRX) {
           // one box of whole code rows each
           tma_load_2d(st + C::OFF_K, &gp.tmap_k, 0, (int)row, &full_bar[s]);
           tma_load_2d(st + C::OFF_V, &gp.tmap_v, 0, (int)row, &full_bar[s]);
@@ -426,13 +436,17 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
     float* qt = qbuf + G * D;
     load_rotate_queries<D, G>(p, hd, qs, qt, tid);
     const float cd = rot_scale<D>();
-    if constexpr (C::CR) {
+    if constexpr (C::CRX) {
       if (warp == 0) {
         // f16 fragments of q~ 2^E, E per row so that max |q~| 2^E is in
         // [2^13, 2^14): the high parts keep 11 bits, the remainders the next
-        // 11, and no value leaves f16's normal range.  k positions 2q, 2q+1 |
-        // 2q+8, 2q+9 of k-step kk carry dims 16kk + 4q .. 4q+3, the four codes
-        // one 32-bit ldmatrix word of the INT8 rows holds.
+        // 11, and no value leaves f16's normal range.  The k positions
+        // follow the codes a 32-bit ldmatrix word holds: INT8, k positions
+        // 2q, 2q+1 | 2q+8, 2q+9 of k-step kk carry dims 16kk + 4q .. 4q+3;
+        // INT4, a word holds dims 8q .. 8q+7 of a 32-dim chunk (two k-steps),
+        // code i at bits 4i, and k-step kk (half h = kk & 1 of chunk kk / 2)
+        // carries dims 8q + 2h + {0, 4 | 1, 5} (a register's two codes then
+        // sit 16 bits apart).
         float mx = 0.0f;
         if (row_ok)
           for (int d = q; d < D; d += 4) mx = fmaxf(mx, fabsf(cd * qt[g * D + d]));
@@ -448,9 +462,21 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
           uint32_t* f3 = qfrag + ((3 * KT + kk) * 32 + lane) * 2;
           uint32_t* f4 = qfrag + ((4 * KT + kk) * 32 + lane) * 2;
           if (row_ok) {
-            const float* trow = qt + g * D + 16 * kk + 4 * q;
-            split_f16(cd * trow[0] * up, cd * trow[1] * up, f3[0], f4[0]);
-            split_f16(cd * trow[2] * up, cd * trow[3] * up, f3[1], f4[1]);
+            int d0, d1, d2, d3;
+            if constexpr (C::CR) {
+              d0 = 16 * kk + 4 * q;
+              d1 = d0 + 1;
+              d2 = d0 + 2;
+              d3 = d0 + 3;
+            } else {
+              d0 = 32 * (kk >> 1) + 8 * q + 2 * (kk & 1);
+              d1 = d0 + 4;
+              d2 = d0 + 1;
+              d3 = d0 + 5;
+            }
+            const float* trow = qt + g * D;
+            split_f16(cd * trow[d0] * up, cd * trow[d1] * up, f3[0], f4[0]);
+            split_f16(cd * trow[d2] * up, cd * trow[d3] * up, f3[1], f4[1]);
             sqh += ((f16_lo_f(f3[0]) + f16_lo_f(f4[0])) + (f16_hi_f(f3[0]) + f16_hi_f(f4[0]))) +
                    ((f16_lo_f(f3[1]) + f16_lo_f(f4[1])) + (f16_hi_f(f3[1]) + f16_hi_f(f4[1])));
           } else {
@@ -461,23 +487,6 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
             sqh += __shfl_xor_sync(FULL, sqh, 2);
             if (row_ok && q == 0) sqh_s[g * NG + kk / KSG] = sqh;
             sqh = 0.0f;
-          }
-        }
-      }
-    }
-    if constexpr (C::CR4) {
-      if (warp == 0) {
-        // bf16 high part and remainder of q~, dims in order (INT4 levels)
-#pragma unroll 1
-        for (int kk = 0; kk < KT; ++kk) {
-          uint32_t* f3 = qfrag + ((3 * KT + kk) * 32 + lane) * 2;
-          uint32_t* f4 = qfrag + ((4 * KT + kk) * 32 + lane) * 2;
-          if (row_ok) {
-            const float* trow = qt + g * D + 16 * kk + 2 * q;
-            split_bf16(cd * trow[0], cd * trow[1], f3[0], f4[0]);
-            split_bf16(cd * trow[8], cd * trow[9], f3[1], f4[1]);
-          } else {
-            f3[0] = f3[1] = f4[0] = f4[1] = 0u;
           }
         }
       }
@@ -549,22 +558,23 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
 #pragma unroll
       for (int j = 0; j < NG; ++j) {
         if constexpr (C::RES) wsum_s[(warp * G + g) * NG + j] = wsum[j];
-        if constexpr (C::CR) wsumR_s[(warp * G + g) * NG + j] = wsumR[j] * (1.0f / vscale);
-        if constexpr (C::CR4) wsumR_s[(warp * G + g) * NG + j] = wsumR[j];
+        if constexpr (C::CRX) wsumR_s[(warp * G + g) * NG + j] = wsumR[j] * (1.0f / vscale);
       }
     }
     // O^T fragments: c0 (dim 16mt+g, row 2q), c1 (.., row 2q+1), c2/c3 dim +8;
-    // the INT8 reference's m-rows g, g + 8 are dims 16mt + 2g, 16mt + 2g + 1
+    // the INT8 reference's m-rows g, g + 8 are dims 16mt + 2g, 16mt + 2g + 1,
+    // the INT4 reference's 32 (mt / 2) + 4g + 2 (mt & 1) (+ 1)
 #pragma unroll
     for (int mt = 0; mt < KT; ++mt) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int r = 2 * q + (e & 1);
         const int dim = 16 * mt + g + 8 * (e >> 1);
-        const int dim_ref = C::CR ? 16 * mt + 2 * g + (e >> 1) : dim;
+        const int dim_ref = C::CR    ? 16 * mt + 2 * g + (e >> 1)
+                            : C::CR4 ? 32 * (mt >> 1) + 4 * g + 2 * (mt & 1) + (e >> 1)
+                                     : dim;
         if (r < G) {
-          if constexpr (C::CR) mw[r * (2 + 2 * D) + 2 + dim_ref] = oref[mt][e] * (2.0f / vscale);
-          else if constexpr (C::CR4) mw[r * (2 + 2 * D) + 2 + dim] = 2.0f * oref[mt][e];
+          if constexpr (C::CRX) mw[r * (2 + 2 * D) + 2 + dim_ref] = oref[mt][e] * (C::CSCALE / vscale);
           else mw[r * (2 + 2 * D) + 2 + dim_ref] = oref[mt][e];
           if constexpr (C::RES) mw[r * (2 + 2 * D) + 2 + D + dim] = 2.0f * ores[mt][e];
           else mw[r * (2 + 2 * D) + 2 + D + dim] = 0.0f;
@@ -573,11 +583,10 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
     }
     named_bar_sync(1, kConsumerThreads);
     if constexpr (C::RES || C::CRX) {
-      // complete sum_t p s (2c - top) = 2 sum p s c - top sum p s (the INT4
-      // reference the same way, written as 2 sum p s_ref c); the INT8
-      // reference's sum_t p s_ref (2c - 255) = 2 acc - (2048 + 255) sum p s_ref
-      // (acc = sum p s_ref (1024 + c), written as 2 acc), moved to the rotated
-      // part
+      // complete sum_t p s (2c - top) = 2 sum p s c - top sum p s; the
+      // compressed reference's sum_t p s_ref (2c - (2^RB - 1)) = CSCALE acc -
+      // LOFF sum p s_ref (acc over the f16 code operands, written as
+      // CSCALE acc), moved to the rotated part
       for (int e = tid; e < kConsumerWarps * G * D; e += kConsumerThreads) {
         const int w = e / (G * D), r = (e / D) % G, dim = e % D;
         float* rec = merge + (w * G + r) * (2 + 2 * D);
@@ -585,7 +594,7 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
         float z = rec[2 + D + dim];
         if constexpr (C::RES) z -= (float)TOPLVL * wsum_s[wi];
         if constexpr (C::CRX) {
-          z += rec[2 + dim] - (C::CR ? 2303.0f : 15.0f) * wsumR_s[wi];
+          z += rec[2 + dim] - C::LOFF * wsumR_s[wi];
           rec[2 + dim] = 0.0f;
         }
         rec[2 + D + dim] = z;
@@ -624,7 +633,7 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
     // ldmatrix: matrices (tile 0, dims +0..7), (tile 0, +8..15), (tile 1, ..), (tile 1, ..)
     const int ktr = wtok + ((lane >> 4) & 1) * 8 + r7;
     const int kch = (lane >> 3) & 1;
-    // INT8 reference: per-group f16 sums sum_k q~_k 2^E (1024 + c_k)
+    // compressed reference: per-group f16 sums sum_k q~_k 2^E c_k 2^-24
     float c8[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
     uint32_t b8[4];          // ldmatrix words of two k-steps: (nt 0, kk), (nt 1, kk), (nt 0, kk + 1), ..
 #pragma unroll
@@ -632,7 +641,7 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
       if constexpr (C::CR) {
         if ((kk & 1) == 0) {
           const int m = lane >> 3;
-          ldsm_x4(sK + swz_offset<D>(wtok + (m & 1) * 8 + r7, kk + (m >> 1)), b8);
+          ldsm_x4(sK + swz_offset<C::RROW>(wtok + (m & 1) * 8 + r7, kk + (m >> 1)), b8);
         }
         const uint2 fh = *reinterpret_cast<const uint2*>(qfrag + ((3 * KT + kk) * 32 + lane) * 2);
         const uint2 fl = *reinterpret_cast<const uint2*>(qfrag + ((4 * KT + kk) * 32 + lane) * 2);
@@ -640,26 +649,33 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
         const uint32_t al[4] = {fl.x, 0u, fl.y, 0u};
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
-          // codes 4q .. 4q+3 of the k-step's 16 as f16 1024 + c, exact
+          // codes 4q .. 4q+3 of the k-step's 16 as f16 subnormals c 2^-24, exact
           const uint32_t w = b8[2 * (kk & 1) + nt];
-          const uint32_t b0 = __byte_perm(w, 0x64u, 0x4140);
-          const uint32_t b1 = __byte_perm(w, 0x64u, 0x4342);
+          const uint32_t b0 = __byte_perm(w, 0u, 0x4140);
+          const uint32_t b1 = __byte_perm(w, 0u, 0x4342);
           mma_f16(c8[nt], ah, b0, b1);
           mma_f16(c8[nt], al, b0, b1);
         }
       } else if constexpr (C::CR4) {
-        // INT4 reference levels 2c - 15, exact in bf16, against q~ high + remainder
+        // one ldmatrix.x4 every four k-steps: words (nt 0, chunk), (nt 1,
+        // chunk), (nt 0, chunk + 1), (nt 1, chunk + 1) of two 32-dim chunks
+        if ((kk & 3) == 0) {
+          const int m = lane >> 3;
+          ldsm_x4(sK + swz_offset<C::RROW>(wtok + (m & 1) * 8 + r7, (kk >> 1) + (m >> 1)), b8);
+        }
         const uint2 fh = *reinterpret_cast<const uint2*>(qfrag + ((3 * KT + kk) * 32 + lane) * 2);
         const uint2 fl = *reinterpret_cast<const uint2*>(qfrag + ((4 * KT + kk) * 32 + lane) * 2);
         const uint32_t ah[4] = {fh.x, 0u, fh.y, 0u};
         const uint32_t al[4] = {fl.x, 0u, fl.y, 0u};
+        const int sh = 8 * (kk & 1);
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
-          const uint2 w2 = *reinterpret_cast<const uint2*>(st + C::OFF_K + tb[nt] * C::RCROW + 8 * kk);
-          uint32_t b0, b1;
-          k_levels<4>(w2.x, w2.y, q, b0, b1);
-          mma_bf16(c8[nt], ah, b0, b1);
-          mma_bf16(c8[nt], al, b0, b1);
+          // codes i, i + 4 of the word (bits 4i, 4i + 16) as f16 subnormals c 2^-24
+          const uint32_t w = b8[2 * ((kk >> 1) & 1) + nt];
+          const uint32_t b0 = (w >> sh) & 0x000F000Fu;
+          const uint32_t b1 = (w >> (sh + 4)) & 0x000F000Fu;
+          mma_f16(c8[nt], ah, b0, b1);
+          mma_f16(c8[nt], al, b0, b1);
         }
       } else {
         const int chunk = 2 * kk + kch;
@@ -675,25 +691,16 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
         mma_bf16(cref[1], a, b[2], b[3]);
       }
       if (C::CRX && (kk + 1) % KSG == 0) {
-        // end of scale group j: S += s_ref_{t, j} 2^-E (2 acc - (2048 + 255) sum q~ 2^E)
-        // (INT8), S += s_ref_{t, j} acc (INT4: the levels themselves)
+        // end of scale group j: S += s_ref_{t, j} 2^-E (CSCALE acc - LOFF sum q~ 2^E)
         const int j = kk / KSG;
-        float rs = 1.0f, off = 0.0f;
-        if constexpr (C::CR) {
-          rs = row_ok ? rsig_s[g] : 0.0f;
-          off = row_ok ? 2303.0f * sqh_s[g * NG + j] : 0.0f;
-        }
+        const float rs = row_ok ? rsig_s[g] : 0.0f;
+        const float off = row_ok ? C::LOFF * sqh_s[g * NG + j] : 0.0f;
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
           const float r0 = half_at(st + C::OFF_RSK + sc_off + tok0[nt] * SB + 2 * j);
           const float r1 = half_at(st + C::OFF_RSK + sc_off + (tok0[nt] + 1) * SB + 2 * j);
-          if constexpr (C::CR) {
-            cref[nt][0] = fmaf(r0 * rs, fmaf(2.0f, c8[nt][0], -off), cref[nt][0]);
-            cref[nt][1] = fmaf(r1 * rs, fmaf(2.0f, c8[nt][1], -off), cref[nt][1]);
-          } else {
-            cref[nt][0] = fmaf(r0, c8[nt][0], cref[nt][0]);
-            cref[nt][1] = fmaf(r1, c8[nt][1], cref[nt][1]);
-          }
+          cref[nt][0] = fmaf(r0 * rs, fmaf(C::CSCALE, c8[nt][0], -off), cref[nt][0]);
+          cref[nt][1] = fmaf(r1 * rs, fmaf(C::CSCALE, c8[nt][1], -off), cref[nt][1]);
 #pragma unroll
           for (int e = 0; e < 4; ++e) c8[nt][e] = 0.0f;
         }
@@ -782,48 +789,14 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
     const uint32_t ph1 = pack_bf16(pr[1][0], pr[1][1]);
     const uint32_t pl0 = pack_bf16(pr[0][0] - bf16_lo_f(ph0), pr[0][1] - bf16_hi_f(ph0));
     const uint32_t pl1 = pack_bf16(pr[1][0] - bf16_lo_f(ph1), pr[1][1] - bf16_hi_f(ph1));
-    if constexpr (C::CR4) {
-      // ---- O_ref^T += C_ref^T (P s_ref^V)^T, INT4 codes exact in bf16 ----
-      const int tk[4] = {wtok + 2 * q, wtok + 2 * q + 1, wtok + 2 * q + 8, wtok + 2 * q + 9};
-      const float pk[4] = {pr[0][0], pr[0][1], pr[1][0], pr[1][1]};
-#pragma unroll
-      for (int j = 0; j < NG; ++j) {
-        float wv[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float sr = half_at(st + C::OFF_RSV + sc_off + tk[k] * SB + 2 * j);
-          wv[k] = (tk[k] < n) ? pk[k] * sr : 0.0f;       // weight 0 beyond the tile
-        }
-        wsumR[j] += (wv[0] + wv[1]) + (wv[2] + wv[3]);
-        uint32_t bh0, bl0, bh1, bl1;
-        split_bf16(wv[0], wv[1], bh0, bl0);
-        split_bf16(wv[2], wv[3], bh1, bl1);
-#pragma unroll
-        for (int mt = j * KSG; mt < (j + 1) * KSG; ++mt) {
-          // codes of dims 16mt + g (lo halves) and 16mt + g + 8 (hi halves)
-          uint32_t x[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint32_t* cw = reinterpret_cast<const uint32_t*>(st + C::OFF_V + tk[k] * C::RCROW);
-            const uint32_t lo = (cw[2 * mt] >> (4 * g)) & 0xFu;
-            const uint32_t hi = (cw[2 * mt + 1] >> (4 * g)) & 0xFu;
-            x[k] = lo | (hi << 16) | kMagic;
-          }
-          const uint32_t m128 = 0xC300C300u;   // {-128, -128}
-          uint32_t a[4];
-          a[0] = badd2_u(__byte_perm(x[0], x[1], 0x5410), m128);   // dim g,   tokens 2q, 2q+1
-          a[1] = badd2_u(__byte_perm(x[0], x[1], 0x7632), m128);   // dim g+8
-          a[2] = badd2_u(__byte_perm(x[2], x[3], 0x5410), m128);   // dim g,   tokens 2q+8, 2q+9
-          a[3] = badd2_u(__byte_perm(x[2], x[3], 0x7632), m128);   // dim g+8
-          mma_bf16(oref[mt], a, bh0, bh1);
-          mma_bf16(oref[mt], a, bl0, bl1);
-        }
-      }
-    } else if constexpr (C::CR) {
-      // ---- O_ref^T += C_ref^T (P s_ref^V 2^Ev)^T, codes as f16 1024 + c ----
-      // ldmatrix.trans of the code rows: word = codes (token 2q: dims 2g,
-      // 2g+1; token 2q+1: dims 2g, 2g+1) of a 16-dim chunk; m-row g is dim
-      // 2g, m-row g + 8 dim 2g + 1.  The weights p s_ref are f16 high parts
+    if constexpr (C::CRX) {
+      // ---- O_ref^T += C_ref^T (P s_ref^V 2^Ev)^T, codes as f16 subnormals ----
+      // ldmatrix.trans of the code rows.  INT8: word = codes (token 2q: dims
+      // 2g, 2g+1; token 2q+1: dims 2g, 2g+1) of a 16-dim chunk; m-row g is
+      // dim 2g, m-row g + 8 dim 2g + 1.  INT4: word = codes of dims 4g .. 4g+3
+      // of a 32-dim chunk (token 2q low half, 2q+1 high half, code i at bits
+      // 4i); m-tile 2 chunk has m-rows g, g + 8 = dims 4g, 4g + 1, m-tile
+      // 2 chunk + 1 dims 4g + 2, 4g + 3.  The weights p s_ref are f16 high parts
       // and remainders after a warp-wide power of two vscale that keeps the
       // tile's largest scale in [1, 2^7): with p < 2^kLazyMax = 2^8 (the
       // lazy softmax max) no weight reaches 2^15, below f16's largest value,
@@ -869,20 +842,39 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
         uint32_t bh0, bl0, bh1, bl1;
         split_f16(wv[0], wv[1], bh0, bl0);
         split_f16(wv[2], wv[3], bh1, bl1);
+        if constexpr (C::CR4) {
 #pragma unroll
-        for (int mt2 = j * KSG / 2; mt2 < (j + 1) * KSG / 2; ++mt2) {
-          const int m = lane >> 3;
-          uint32_t v[4];     // (tokens 0-7, chunk 2mt2), (8-15, 2mt2), (0-7, 2mt2+1), (8-15, ..)
-          ldsm_x4_trans(sV + swz_offset<D>(wtok + (m & 1) * 8 + r7, 2 * mt2 + (m >> 1)), v);
+          for (int ch = j * GROUP / 32; ch < (j + 1) * GROUP / 32; ++ch) {
+            const int m = (lane >> 3) & 1;
+            uint32_t v[2];   // (tokens 0-7, chunk ch), (tokens 8-15, chunk ch)
+            ldsm_x2_trans(sV + swz_offset<C::RROW>(wtok + m * 8 + r7, ch), v);
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int mt = 2 * mt2 + h;
-            const uint32_t R0 = v[2 * h], R1 = v[2 * h + 1];
-            // bytes 0, 2 (dim 2g) and bytes 1, 3 (dim 2g + 1) as f16 1024 + c
-            const uint32_t a[4] = {__byte_perm(R0, 0x64u, 0x4240), __byte_perm(R0, 0x64u, 0x4341),
-                                   __byte_perm(R1, 0x64u, 0x4240), __byte_perm(R1, 0x64u, 0x4341)};
-            mma_f16(oref[mt], a, bh0, bh1);
-            mma_f16(oref[mt], a, bl0, bl1);
+            for (int h = 0; h < 2; ++h) {
+              const int sh = 8 * h;
+              const uint32_t a[4] = {(v[0] >> sh) & 0x000F000Fu, (v[0] >> (sh + 4)) & 0x000F000Fu,
+                                     (v[1] >> sh) & 0x000F000Fu, (v[1] >> (sh + 4)) & 0x000F000Fu};
+              mma_f16(oref[2 * ch + h], a, bh0, bh1);
+              mma_f16(oref[2 * ch + h], a, bl0, bl1);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int mt2 = j * KSG / 2; mt2 < (j + 1) * KSG / 2; ++mt2) {
+            const int m = lane >> 3;
+            uint32_t v[4];   // (tokens 0-7, chunk 2mt2), (8-15, 2mt2), (0-7, 2mt2+1), (8-15, ..)
+            ldsm_x4_trans(sV + swz_offset<C::RROW>(wtok + (m & 1) * 8 + r7, 2 * mt2 + (m >> 1)),
+                          v);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int mt = 2 * mt2 + h;
+              const uint32_t R0 = v[2 * h], R1 = v[2 * h + 1];
+              // bytes 0, 2 (dim 2g) and bytes 1, 3 (dim 2g + 1) as f16 subnormals
+              const uint32_t a[4] = {
+                  __byte_perm(R0, 0u, 0x4240), __byte_perm(R0, 0u, 0x4341),
+                  __byte_perm(R1, 0u, 0x4240), __byte_perm(R1, 0u, 0x4341)};
+              mma_f16(oref[mt], a, bh0, bh1);
+              mma_f16(oref[mt], a, bl0, bl1);
+            }
           }
         }
       }
@@ -1040,19 +1032,19 @@ cudaError_t launch_decode_gqa(int head_dim, int G, int bits, const DecodeParams&
   const unsigned long long rows =
       p.page_table ? (unsigned long long)p.n_pages * p.kv_heads * kDecodeTile
                    : (unsigned long long)p.batch * p.kv_heads * p.ctx_pitch;
-  if (p.ref_bits == 8) {
-    // the reference is INT8 code rows (head_dim bytes each)
-    if (!encode_bytes_map(&gp.tmap_k, p.rcodes_k, rows, head_dim, kDecodeTile) ||
-        !encode_bytes_map(&gp.tmap_v, p.rcodes_v, rows, head_dim, kDecodeTile))
+  if (p.ref_bits == 8 || p.ref_bits == 4) {
+    // the reference is code rows of head_dim * ref_bits / 8 bytes
+    const int rrow = head_dim * p.ref_bits / 8;
+    if (!encode_bytes_map(&gp.tmap_k, p.rcodes_k, rows, rrow, kDecodeTile) ||
+        !encode_bytes_map(&gp.tmap_v, p.rcodes_v, rows, rrow, kDecodeTile))
       return cudaErrorInvalidValue;
-    if (head_dim == 128) return launch_gqa_d<128, 8>(G, bits, gp, stream);
-    if (head_dim == 64) return launch_gqa_d<64, 8>(G, bits, gp, stream);
-    return cudaErrorInvalidValue;
-  }
-  if (p.ref_bits == 4) {
-    // INT4 reference code rows by bulk copies (no tensor maps)
-    if (head_dim == 128) return launch_gqa_d<128, 4>(G, bits, gp, stream);
-    if (head_dim == 64) return launch_gqa_d<64, 4>(G, bits, gp, stream);
+    if (p.ref_bits == 8) {
+      if (head_dim == 128) return launch_gqa_d<128, 8>(G, bits, gp, stream);
+      if (head_dim == 64) return launch_gqa_d<64, 8>(G, bits, gp, stream);
+    } else {
+      if (head_dim == 128) return launch_gqa_d<128, 4>(G, bits, gp, stream);
+      if (head_dim == 64) return launch_gqa_d<64, 4>(G, bits, gp, stream);
+    }
     return cudaErrorInvalidValue;
   }
   if (p.ref_bits != 0) return cudaErrorInvalidValue;

@@ -206,8 +206,8 @@ int device_sm_count();   // SMs of the current device, cached per device
 // rows, 128-byte swizzle, rows past the end read as zeros (rq_tma.cu).
 bool encode_rows_map(CUtensorMap* map, const void* base, unsigned long long rows, int d,
                      int box_rows);
-// TMA map of a row-major [rows][row_bytes] byte array (row_bytes 64 or 128):
-// box = whole rows x box_rows, swizzle of the row's width (64 or 128 bytes).
+// TMA map of a row-major [rows][row_bytes] byte array (row_bytes 32, 64 or
+// 128): box = whole rows x box_rows, swizzle of the row's width.
 bool encode_bytes_map(CUtensorMap* map, const void* base, unsigned long long rows, int row_bytes,
                       int box_rows);
 
