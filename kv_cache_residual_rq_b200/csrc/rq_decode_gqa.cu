@@ -63,6 +63,10 @@ struct GCfg {
   static constexpr int TILE = kDecodeTile;                 // 64 tokens
   static constexpr int WTOK = TILE / kConsumerWarps;       // 16 tokens per warp
   static constexpr bool RES = (BITS != 16);
+  // INT2 residual with 64-dim scale groups: a 16-byte row chunk of codes is
+  // exactly one scale group, so ldmatrix reads the code rows directly
+  static constexpr bool LDM2 = (BITS == 2 && GROUP == 64);
+  static constexpr int NCH = D / 64;                        // 64-dim chunks per row
   static constexpr bool CR = (RB == 8);                    // INT8 compressed reference
   static constexpr bool CR4 = (RB == 4);                   // INT4 compressed reference
   static constexpr bool CRX = (RB != 0);                   // either
@@ -134,6 +138,12 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t (&r)[2]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];"
+               : "=r"(r[0]), "=r"(r[1])
                : "r"(addr));
 }
 
@@ -500,7 +510,11 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
         uint32_t* fl = qfrag + ((2 * KT + kk) * 32 + lane) * 2;
         if (row_ok) {
           const float* qrow = qs + g * D + 16 * kk + 2 * q;
-          const float* trow = qt + g * D + 16 * kk + 2 * q;
+          // INT2 with ldmatrix words: k-step kk = 4c + t of chunk c carries
+          // dims 64c + 16q + 2t + {0, 8 | 1, 9} (codes 2t, 2t+8 | 2t+1, 2t+9
+          // of the word holding the chunk's dims 16q .. 16q+15)
+          const float* trow = qt + g * D +
+                              (C::LDM2 ? 64 * (kk >> 2) + 16 * q + 2 * (kk & 3) : 16 * kk + 2 * q);
           fa[0] = pack_bf16(qrow[0], qrow[1]);       // exact: q is bf16
           fa[1] = pack_bf16(qrow[8], qrow[9]);
           if constexpr (BITS == 2) {
@@ -570,13 +584,14 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
       for (int e = 0; e < 4; ++e) {
         const int r = 2 * q + (e & 1);
         const int dim = 16 * mt + g + 8 * (e >> 1);
+        const int dim_res = C::LDM2 ? 64 * (mt >> 2) + 8 * g + 2 * (mt & 3) + (e >> 1) : dim;
         const int dim_ref = C::CR    ? 16 * mt + 2 * g + (e >> 1)
                             : C::CR4 ? 32 * (mt >> 1) + 4 * g + 2 * (mt & 1) + (e >> 1)
                                      : dim;
         if (r < G) {
           if constexpr (C::CRX) mw[r * (2 + 2 * D) + 2 + dim_ref] = oref[mt][e] * (C::CSCALE / vscale);
           else mw[r * (2 + 2 * D) + 2 + dim_ref] = oref[mt][e];
-          if constexpr (C::RES) mw[r * (2 + 2 * D) + 2 + D + dim] = 2.0f * ores[mt][e];
+          if constexpr (C::RES) mw[r * (2 + 2 * D) + 2 + D + dim_res] = 2.0f * ores[mt][e];
           else mw[r * (2 + 2 * D) + 2 + D + dim] = 0.0f;
         }
       }
@@ -636,6 +651,7 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
     // compressed reference: per-group f16 sums sum_k q~_k 2^E c_k 2^-24
     float c8[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
     uint32_t b8[4];          // ldmatrix words of two k-steps: (nt 0, kk), (nt 1, kk), (nt 0, kk + 1), ..
+    uint32_t ck4[4];         // INT2 residual (64-dim groups): the tile's K code words
 #pragma unroll
     for (int kk = 0; kk < KT; ++kk) {
       if constexpr (C::CR) {
@@ -710,11 +726,35 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
         const uint2 fl = *reinterpret_cast<const uint2*>(qfrag + ((2 * KT + kk) * 32 + lane) * 2);
         const uint32_t ah[4] = {fh.x, 0u, fh.y, 0u};
         const uint32_t al[4] = {fl.x, 0u, fl.y, 0u};
+        if constexpr (C::LDM2) {
+          // the whole warp tile's K codes in one ldmatrix: words (nt 0, chunk
+          // 0), (nt 1, chunk 0)[, (nt 0, chunk 1), (nt 1, chunk 1)]
+          if (kk == 0) {
+            const int m = (lane >> 3) & (2 * C::NCH - 1);
+            const uint32_t a = smem_u32(st + C::OFF_CK + (wtok + (m & 1) * 8 + r7) * C::CROW +
+                                        (m >> 1) * 16);
+            if constexpr (C::NCH == 2) {
+              ldsm_x4(a, ck4);
+            } else {
+              uint32_t r2[2];
+              ldsm_x2(a, r2);
+              ck4[0] = r2[0];
+              ck4[1] = r2[1];
+            }
+          }
+        }
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
           const uint32_t* cw = reinterpret_cast<const uint32_t*>(st + C::OFF_CK + tb[nt] * C::CROW);
           uint32_t b0, b1;
-          if constexpr (BITS == 2) {
+          if constexpr (C::LDM2) {
+            // codes 2t, 2t+8 | 2t+1, 2t+9 of the word at mantissa bits 1-2:
+            // bf16 128 + 2c, exact (as k_levels2)
+            const uint32_t w = ck4[2 * (kk >> 2) + nt];
+            const int t = kk & 3;
+            b0 = ((t == 0 ? (w << 1) : (w >> (4 * t - 1))) & 0x00060006u) | kMagic;
+            b1 = ((w >> (4 * t + 1)) & 0x00060006u) | kMagic;
+          } else if constexpr (BITS == 2) {
             k_levels2(cw[kk], q, b0, b1);
           } else {
             const uint2 w2 = *reinterpret_cast<const uint2*>(cw + 2 * kk);
@@ -897,6 +937,24 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
     if constexpr (C::RES) {
       const int tk[4] = {wtok + 2 * q, wtok + 2 * q + 1, wtok + 2 * q + 8, wtok + 2 * q + 9};
       const float pk[4] = {pr[0][0], pr[0][1], pr[1][0], pr[1][1]};
+      // INT2, 64-dim groups: the warp tile's V code words by one
+      // ldmatrix.trans: word = codes of dims 8g .. 8g+7 of a 64-dim chunk
+      // (token 2q low half, 2q+1 high half, code i at bits 2i); (tokens 0-7,
+      // chunk 0), (8-15, chunk 0)[, (0-7, chunk 1), (8-15, chunk 1)]
+      uint32_t cv4[4];
+      if constexpr (C::LDM2) {
+        const int m = (lane >> 3) & (2 * C::NCH - 1);
+        const uint32_t a = smem_u32(st + C::OFF_CV + (wtok + (m & 1) * 8 + r7) * C::CROW +
+                                    (m >> 1) * 16);
+        if constexpr (C::NCH == 2) {
+          ldsm_x4_trans(a, cv4);
+        } else {
+          uint32_t r2[2];
+          ldsm_x2_trans(a, r2);
+          cv4[0] = r2[0];
+          cv4[1] = r2[1];
+        }
+      }
 #pragma unroll
       for (int j = 0; j < NG; ++j) {
         float wv[4];
@@ -909,6 +967,23 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
         uint32_t bh0, bl0, bh1, bl1;
         split_bf16(wv[0], wv[1], bh0, bl0);
         split_bf16(wv[2], wv[3], bh1, bl1);
+        if constexpr (C::LDM2) {
+          // chunk j: m-tile 4j + i has m-rows g, g + 8 = dims 64j + 8g + 2i (+ 1);
+          // operands (128 + c) - 128 = c, exact (the accumulator carries no
+          // offset across the head's tiles)
+          const uint32_t m128 = 0xC300C300u;   // {-128, -128}
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t R0 = cv4[2 * j], R1 = cv4[2 * j + 1];
+            const uint32_t a[4] = {badd2_u(((R0 >> (4 * i)) & 0x00030003u) | kMagic, m128),
+                                   badd2_u(((R0 >> (4 * i + 2)) & 0x00030003u) | kMagic, m128),
+                                   badd2_u(((R1 >> (4 * i)) & 0x00030003u) | kMagic, m128),
+                                   badd2_u(((R1 >> (4 * i + 2)) & 0x00030003u) | kMagic, m128)};
+            mma_bf16(ores[4 * j + i], a, bh0, bh1);
+            mma_bf16(ores[4 * j + i], a, bl0, bl1);
+          }
+          continue;
+        }
 #pragma unroll
         for (int mt = j * KSG; mt < (j + 1) * KSG; ++mt) {
           // codes of dims 16mt + g (lo halves) and 16mt + g + 8 (hi halves)

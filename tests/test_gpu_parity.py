@@ -219,6 +219,8 @@ def test_decode_full_size_sampled(name, loops):
     (64, 64, 4, 4, 257, 2, 1),
     (128, 32, 1, 16, 333, 2, 2),       # reference loop, ragged
     (128, 32, 4, 2, 20000, 1, 1),      # one head spread over many CTAs
+    (64, 64, 2, 2, 300, 2, 2),         # INT2, 64-dim groups (ldmatrix code words), d 64
+    (128, 64, 8, 2, 777, 1, 3),        # the same at d 128, G = 8, ragged
 ])
 def test_decode_edge_shapes(d, group, G, bits, ctx, batch, hkv):
     bl = (bits, 16) if bits != 16 else (2, 16)
