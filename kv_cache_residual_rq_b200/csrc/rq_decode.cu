@@ -33,8 +33,9 @@
 //   - INT2 K residual: per head, a shared-memory table holds, for every
 //     4-dim slice of q~ and every byte of 4 codes, the partial product
 //     sum_k q~_k l(c_k); a lane's 8 dims cost two table reads.
-//   - Codes become floats with one AND/OR and one subtract (the 2^23
-//     exponent trick, the code left at its bit position); the position's
+//   - Codes become floats with one AND/OR each and one paired subtract per
+//     two codes (the 2^23 exponent trick, the code left at its bit
+//     position, `sub.rn.f32x2`); the position's
 //     power of two is folded into the query constants or applied once when
 //     the V accumulator is flushed.
 //   - Scores are reduce-scattered across the lanes of a token (one shuffle
@@ -105,22 +106,44 @@ __device__ __forceinline__ float code_at(uint32_t masked) {
   return __uint_as_float(0x4B000000u | masked) - 8388608.0f;
 }
 
+// {a.x - b.x, a.y - b.y}, one paired instruction
+__device__ __forceinline__ float2 sub2_rn(float2 a, float2 b) {
+  float2 r;
+  asm("{\n\t.reg .b64 ra, rb, rr;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "sub.rn.f32x2 rr, ra, rb;\n\tmov.b64 {%0, %1}, rr;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+
 // The lane's DPL codes as floats c_k * 2^pos_k (pos_k = the bit position the
-// code sits at inside `x`, the lane's bits already shifted down to bit 0).
+// code sits at inside `x`, the lane's bits already shifted down to bit 0):
+// each masked code ORed into the bit pattern of 2^23, then 2^23 subtracted
+// (exact), two codes per paired subtraction.
 template <int BITS, int DPL>
 __device__ __forceinline__ void codes_positional(uint32_t x, float (&f)[DPL]) {
   constexpr uint32_t M = (1u << BITS) - 1u;
+  uint32_t m[DPL];
   if constexpr (BITS * DPL > 16) {
     // 8 INT4 codes: split so no code sits above bit 16 (exactness needs < 2^23)
     const uint32_t lo = x & 0xFFFFu, hi = x >> 16;
 #pragma unroll
     for (int k = 0; k < DPL / 2; ++k) {
-      f[k] = code_at(lo & (M << (BITS * k)));
-      f[k + DPL / 2] = code_at(hi & (M << (BITS * k)));
+      m[k] = lo & (M << (BITS * k));
+      m[k + DPL / 2] = hi & (M << (BITS * k));
     }
   } else {
 #pragma unroll
-    for (int k = 0; k < DPL; ++k) f[k] = code_at(x & (M << (BITS * k)));
+    for (int k = 0; k < DPL; ++k) m[k] = x & (M << (BITS * k));
+  }
+  const float2 big = make_float2(8388608.0f, 8388608.0f);
+#pragma unroll
+  for (int j = 0; j < DPL / 2; ++j) {
+    const float2 v = sub2_rn(make_float2(__uint_as_float(0x4B000000u | m[2 * j]),
+                                         __uint_as_float(0x4B000000u | m[2 * j + 1])),
+                             big);
+    f[2 * j] = v.x;
+    f[2 * j + 1] = v.y;
   }
 }
 
