@@ -1107,6 +1107,8 @@ cudaError_t launch_decode_gqa(int head_dim, int G, int bits, const DecodeParams&
   const unsigned long long rows =
       p.page_table ? (unsigned long long)p.n_pages * p.kv_heads * kDecodeTile
                    : (unsigned long long)p.batch * p.kv_heads * p.ctx_pitch;
+  // tensor-copy row coordinates are 32-bit signed
+  if (rows > 0x7FFFFFFFull) return cudaErrorInvalidValue;
   if (p.ref_bits == 8 || p.ref_bits == 4) {
     // the reference is code rows of head_dim * ref_bits / 8 bytes
     const int rrow = head_dim * p.ref_bits / 8;
