@@ -282,10 +282,14 @@ __device__ __forceinline__ void rotate_lane(const float (&v)[32], float2 (&P)[16
   for (int m = 0; m < 16; ++m) P[m] = __fmul2_rn(P[m], cd2);
 }
 
-template <int D, int GROUP, int CW>
+// MODE 0: BF16 reference, no refits; 1: BF16 reference with least-squares
+// refits; 2: compressed reference.  Separate instantiations keep the plain
+// encode free of the other modes' registers and branches.
+template <int D, int GROUP, int CW, int MODE>
 __global__ void __launch_bounds__(ECfg<D, CW>::THREADS, 1)
 encode_tma_kernel(const __grid_constant__ EncodeTmaParams tp) {
   using C = ECfg<D, CW>;
+  const int iters = (MODE == 0) ? 0 : tp.p.refine_iters;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -374,8 +378,8 @@ encode_tma_kernel(const __grid_constant__ EncodeTmaParams tp) {
     // stored) and zr holds its reconstruction s16 * l, subtracted from every
     // loop's rotated row.
     float zr[32];
-    const bool cr = p.ref_bits != 0;
-    if (!cr) {
+    constexpr bool cr = (MODE == 2);
+    if constexpr (!cr) {
       const uint4* nd4 = reinterpret_cast<const uint4*>(ndtab + q * 16);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -448,7 +452,7 @@ encode_tma_kernel(const __grid_constant__ EncodeTmaParams tp) {
       }
       float2 P[16];
       rotate_lane<D, C::LPR, C::RPW>(v, P, q);
-      if (cr) {
+      if constexpr (cr) {
 #pragma unroll
         for (int m = 0; m < 16; ++m) P[m] = fsub2(P[m], make_float2(zr[m], zr[m + 16]));
       }
@@ -457,26 +461,33 @@ encode_tma_kernel(const __grid_constant__ EncodeTmaParams tp) {
       if (p.bits[l] == 2)
         quantize_store<2, GROUP, C::RPW>(P, p.codes[l] + (size_t)row * (D / 16),
                                          p.scales[l] + (size_t)row * (D / GROUP), q, valid,
-                                         p.refine_iters);
+                                         iters);
       else
         quantize_store<4, GROUP, C::RPW>(P, p.codes[l] + (size_t)row * (D / 8),
                                          p.scales[l] + (size_t)row * (D / GROUP), q, valid,
-                                         p.refine_iters);
+                                         iters);
     }
   }
 }
 
 constexpr int kConsumerWarps = 15;   // + 1 producer = 16 warps, 4 per scheduler
 
-template <int D, int GROUP>
-cudaError_t launch_t(const EncodeTmaParams& tp, int num_sms, cudaStream_t stream) {
+template <int D, int GROUP, int MODE>
+cudaError_t launch_tm(const EncodeTmaParams& tp, int num_sms, cudaStream_t stream) {
   using C = ECfg<D, kConsumerWarps>;
-  cudaError_t e = cudaFuncSetAttribute(encode_tma_kernel<D, GROUP, kConsumerWarps>,
+  cudaError_t e = cudaFuncSetAttribute(encode_tma_kernel<D, GROUP, kConsumerWarps, MODE>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   const int grid = tp.n_tiles < num_sms ? tp.n_tiles : num_sms;
-  return launch_pdl(encode_tma_kernel<D, GROUP, kConsumerWarps>, (unsigned)grid, C::THREADS,
-                    C::SMEM, stream, tp);
+  return launch_pdl(encode_tma_kernel<D, GROUP, kConsumerWarps, MODE>, (unsigned)grid,
+                    C::THREADS, C::SMEM, stream, tp);
+}
+
+template <int D, int GROUP>
+cudaError_t launch_t(const EncodeTmaParams& tp, int num_sms, cudaStream_t stream) {
+  if (tp.p.ref_bits != 0) return launch_tm<D, GROUP, 2>(tp, num_sms, stream);
+  if (tp.p.refine_iters > 0) return launch_tm<D, GROUP, 1>(tp, num_sms, stream);
+  return launch_tm<D, GROUP, 0>(tp, num_sms, stream);
 }
 
 }  // namespace
