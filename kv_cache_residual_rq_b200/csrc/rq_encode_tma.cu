@@ -352,7 +352,9 @@ encode_tma_kernel(const __grid_constant__ EncodeTmaParams tp) {
   long long it = 0;
   for (int t = blockIdx.x; t < tp.n_tiles; t += gridDim.x) {
     const long long idx = (long long)t * C::R + r;
-    const long long hd = idx / p.ctx, tok = idx - hd * p.ctx;
+    // idx < n_tiles * R <= kEncodeTmaMaxRows + R < 2^31: a 32-bit division
+    const uint32_t hd32 = (uint32_t)idx / (uint32_t)p.ctx;
+    const long long hd = hd32, tok = idx - (long long)hd32 * p.ctx;
     long long row = 0;
     const bool valid = idx < p.n_rows && enc_dst_row(p, hd, tok, row);
 
