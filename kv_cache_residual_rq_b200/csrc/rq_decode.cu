@@ -95,7 +95,8 @@ struct Cfg {
   static constexpr int QPRE_HEADS = 4;
   static constexpr int QPRE_BYTES = QPRE_HEADS * G * D * 2;
   static constexpr int SMEM_BYTES =
-      RING_BYTES + 4 * (AREA_FLOATS + QBUF_FLOATS) + 2 * STAGES * 8 + 16 + QPRE_BYTES;
+      RING_BYTES + 4 * (AREA_FLOATS + QBUF_FLOATS) + 2 * STAGES * 8 + 16 + QPRE_BYTES +
+      STAGES * 8;   // + the stages' resolved rows
   static_assert(TPW % TPS == 0 && STEPS % CH == 0, "tile split");
   static_assert(G != 1 || CH == STEPS, "G == 1 processes a whole tile per chunk");
   static_assert(STAGE_BYTES % 16 == 0, "stage alignment");
@@ -234,6 +235,8 @@ decode_kernel(const DecodeParams p) {
   volatile int* flags = reinterpret_cast<volatile int*>(empty_bar + STAGES);  // [0] abort, [1] last
   uint16_t* qpre = reinterpret_cast<uint16_t*>(
       reinterpret_cast<unsigned char*>(empty_bar + STAGES) + 16);      // [QPRE_HEADS][G][D]
+  volatile unsigned long long* stage_row = reinterpret_cast<volatile unsigned long long*>(
+      reinterpret_cast<unsigned char*>(qpre) + C::QPRE_BYTES);          // [STAGES], paged
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -273,8 +276,15 @@ decode_kernel(const DecodeParams p) {
     if (lane == 0) {
       int issued = 0;
       TileCursor cur = first_cur;
+      // paged caches: the next tile's page id is read one tile ahead, so its
+      // latency overlaps the wait for a free stage
+      int page_next = (p.page_table && n_my > 0) ? tile_page(p, cur) : 0;
       for (int i = 0; i < n_my; ++i) {
         const int s = i % STAGES;
+        const TileCursor tc = cur;
+        const int page = page_next;
+        cur.next(p);
+        if (p.page_table && i + 1 < n_my) page_next = tile_page(p, cur);
         if (i >= STAGES) {
           if (!mbar_wait_bounded(&empty_bar[s], ((i / STAGES) - 1) & 1)) {
             flag_error(p.status, 1u);
@@ -284,10 +294,10 @@ decode_kernel(const DecodeParams p) {
         }
         if (flags[0]) break;
         size_t row;
-        const bool page_ok = tile_row(p, cur, row);
-        if (!page_ok && cur.n() > 0) flag_error(p.status, 32u);
-        const int n = page_ok ? cur.n() : 0;
-        cur.next(p);
+        const bool page_ok = p.page_table ? tile_row_page(p, tc, page, row) : tile_row(p, tc, row);
+        if (!page_ok && tc.n() > 0) flag_error(p.status, 32u);
+        const int n = page_ok ? tc.n() : 0;
+        if (p.page_table) stage_row[s] = page_ok ? (unsigned long long)row : kBadRow;
         unsigned char* st = ring + s * C::STAGE_BYTES;
         if (n <= 0) {                   // the empty tile of an empty sequence
           mbar_arrive(&full_bar[s]);
@@ -829,8 +839,9 @@ decode_kernel(const DecodeParams p) {
   TileCursor cur = first_cur;
   for (int i = 0; i < n_my; ++i) {
     const long long hd = cur.hd;
-    size_t row;
-    const int n = tile_row(p, cur, row) ? cur.n() : 0;
+    size_t row = 0;
+    int n = cur.n();
+    if (!p.page_table) tile_row(p, cur, row);   // paged: the stage's row, below
     if (hd != cur_head) {
       if (cur_head >= 0) {
         flush_head(cur_head, cur_first, cur_nt);
@@ -850,6 +861,11 @@ decode_kernel(const DecodeParams p) {
       if (!aborted && lane == 0) flag_error(p.status, 8u);
       aborted = true;
       flags[0] = 1;
+    }
+    if (!aborted && p.page_table) {
+      const unsigned long long r = stage_row[s];   // written before the stage's arrive
+      if (r == kBadRow) n = 0;
+      else row = (size_t)r;
     }
     if (!aborted && n > 0) {
       const unsigned char* st = ring + s * C::STAGE_BYTES;

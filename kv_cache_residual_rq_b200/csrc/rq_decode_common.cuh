@@ -80,13 +80,13 @@ struct TileCursor {
 // false for a page id outside the pool; the caller then treats the tile as
 // empty (and the producer raises status bit 32), so a bad table entry cannot
 // address memory outside the pool.
-__device__ __forceinline__ bool tile_row(const DecodeParams& p, const TileCursor& c,
-                                         size_t& row) {
-  if (!p.page_table) {
-    row = (size_t)c.hd * p.ctx_pitch + c.t0();
-    return true;
-  }
-  const int page = p.page_table[(size_t)c.b * p.max_pages + c.j];
+// Paged caches: the page id of the cursor's tile (read ahead by the
+// producer), and the row of a page id already read.
+__device__ __forceinline__ int tile_page(const DecodeParams& p, const TileCursor& c) {
+  return p.page_table[(size_t)c.b * p.max_pages + c.j];
+}
+__device__ __forceinline__ bool tile_row_page(const DecodeParams& p, const TileCursor& c,
+                                              int page, size_t& row) {
   if (page < 0 || page >= p.n_pages) {
     row = 0;
     return false;
@@ -94,6 +94,20 @@ __device__ __forceinline__ bool tile_row(const DecodeParams& p, const TileCursor
   row = ((size_t)page * p.kv_heads + c.h) * kDecodeTile;
   return true;
 }
+
+__device__ __forceinline__ bool tile_row(const DecodeParams& p, const TileCursor& c,
+                                         size_t& row) {
+  if (!p.page_table) {
+    row = (size_t)c.hd * p.ctx_pitch + c.t0();
+    return true;
+  }
+  return tile_row_page(p, c, tile_page(p, c), row);
+}
+
+// A stage's row as the producer resolved it (paged caches), kBadRow for a
+// page id outside the pool; the consumers read it after the stage's barrier
+// instead of the page table.
+constexpr unsigned long long kBadRow = ~0ull;
 
 // The split of a call over its CTAs: n_tiles tiles in `ctas` equal runs.
 struct CallSplit {

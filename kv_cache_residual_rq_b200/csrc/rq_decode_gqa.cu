@@ -114,7 +114,7 @@ struct GCfg {
   static constexpr int SMEM_BYTES = 1024 /* base alignment slack */ + RING_BYTES +
                                     4 * (MERGE_FLOATS + QBUF_FLOATS + WSUM_FLOATS +
                                          QFRAG_WORDS + SQ_FLOATS) +
-                                    2 * STAGES * 8 + 16;
+                                    2 * STAGES * 8 + 16 + STAGES * 8;   // + stage rows
   static_assert(G == 2 || G == 4 || G == 8, "grouped queries");
   static_assert(MERGE_FLOATS >= kVarlenMaxBatch + 1, "merge area holds the length scan");
   static_assert(GROUP == 32 || GROUP == 64, "scale group");
@@ -302,6 +302,8 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(sq_s + C::SQ_FLOATS);
   uint64_t* empty_bar = full_bar + STAGES;
   volatile int* flags = reinterpret_cast<volatile int*>(empty_bar + STAGES);
+  volatile unsigned long long* stage_row = reinterpret_cast<volatile unsigned long long*>(
+      reinterpret_cast<unsigned char*>(empty_bar + STAGES) + 16);    // [STAGES], paged
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -335,8 +337,14 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
     if (lane == 0) {
       int issued = 0;
       TileCursor cur = first_cur;
+      // paged caches: the next tile's page id is read one tile ahead
+      int page_next = (p.page_table && n_my > 0) ? tile_page(p, cur) : 0;
       for (int i = 0; i < n_my; ++i) {
         const int s = i % STAGES;
+        const TileCursor tc = cur;
+        const int page = page_next;
+        cur.next(p);
+        if (p.page_table && i + 1 < n_my) page_next = tile_page(p, cur);
         if (i >= STAGES) {
           if (!mbar_wait_bounded(&empty_bar[s], ((i / STAGES) - 1) & 1)) {
             flag_error(p.status, 1u);
@@ -346,10 +354,10 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
         }
         if (flags[0]) break;
         size_t row;
-        const bool page_ok = tile_row(p, cur, row);
-        if (!page_ok && cur.n() > 0) flag_error(p.status, 32u);
-        const int n = page_ok ? cur.n() : 0;
-        cur.next(p);
+        const bool page_ok = p.page_table ? tile_row_page(p, tc, page, row) : tile_row(p, tc, row);
+        if (!page_ok && tc.n() > 0) flag_error(p.status, 32u);
+        const int n = page_ok ? tc.n() : 0;
+        if (p.page_table) stage_row[s] = page_ok ? (unsigned long long)row : kBadRow;
         unsigned char* st = ring + s * C::STAGE_BYTES;
         if (n <= 0) {                   // the empty tile of an empty sequence
           mbar_arrive(&full_bar[s]);
@@ -1020,8 +1028,9 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
   TileCursor cur = first_cur;
   for (int i = 0; i < n_my; ++i) {
     const long long hd = cur.hd;
-    size_t row;
-    const int n = tile_row(p, cur, row) ? cur.n() : 0;
+    size_t row = 0;
+    int n = cur.n();
+    if (!p.page_table) tile_row(p, cur, row);   // paged: the stage's row, below
     if (hd != cur_head) {
       if (cur_head >= 0) {
         flush_head(cur_head, cur_first, cur_nt);
@@ -1041,6 +1050,11 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
       if (!aborted && lane == 0) flag_error(p.status, 8u);
       aborted = true;
       flags[0] = 1;
+    }
+    if (!aborted && p.page_table) {
+      const unsigned long long r = stage_row[s];   // written before the stage's arrive
+      if (r == kBadRow) n = 0;
+      else row = (size_t)r;
     }
     if (!aborted && n > 0) {
       tile_mma(ring + s * C::STAGE_BYTES, n, (int)((row * SB) & 15));

@@ -61,6 +61,48 @@ def _time(fn, reps, flush):
     return times[len(times) // 2]
 
 
+def _to_pool(flat, B, H, T, perm):
+    """A dense [B, H, T, X] cache (flat device buffer) as a pool of 64-token
+    pages [pages, H, 64, X]: page (b, j) stored at pool index perm[b * P + j]."""
+    import torch
+    P = T // 64
+    x = flat[: B * H * T * (flat.numel() // (B * H * T))].view(B, H, P, 64, -1)
+    pages = x.permute(0, 2, 1, 3, 4).reshape(B * P, H, 64, -1)
+    pool = torch.empty_like(pages)
+    pool[perm] = pages
+    return pool
+
+
+def measure_paged(w, refk, refv, ck, cv, sk, sv, q, out, peak, reps, emit):
+    """The loop-1 residual call with the cache scattered over a shuffled pool
+    of 64-token pages (every sequence at full length): the same bytes as the
+    dense call, addressed through the page table."""
+    import torch
+    import kv_cache_residual_rq_b200 as rq
+    dev = refk.device
+    B, H, T, d = w.batch, w.kv_heads, w.ctx, w.head_dim
+    P = T // 64
+    g = torch.Generator(device="cpu").manual_seed(w.seed * 131 + 7)
+    perm = torch.randperm(B * P, generator=g).to(dev)
+    table = perm.view(B, P).to(torch.int32).contiguous()
+    u8 = lambda t: t.contiguous().view(torch.uint8).view(-1)
+    pk, pv = _to_pool(u8(refk), B, H, T, perm), _to_pool(u8(refv), B, H, T, perm)
+    pck, pcv = _to_pool(ck, B, H, T, perm), _to_pool(cv, B, H, T, perm)
+    psk, psv = _to_pool(sk, B, H, T, perm), _to_pool(sv, B, H, T, perm)
+    shape = rq.make_shape(B, H, T, d, w.group, w.q_heads)
+    lens = torch.full((B,), T, dtype=torch.int32, device=dev)
+    ws = rq.alloc_workspace(shape, dev, varlen=True)
+    b = w.bits[0]
+    fn = lambda: rq.rq_decode_attention_paged(shape, lens, table, P, B * P, q, pk, pv, pck, pcv,
+                                              psk, psv, b, w.seed, 0.0, None, None, 0, 0, out,
+                                              ws)
+    t = _time(fn, reps, None)
+    nb = decode_bytes(w, b)
+    emit({"workload": w.name, "kernel": f"decode paged bits={b} (shuffled 64-token pages)",
+          "G": w.G, "us": t * 1e6, "bytes": nb, "gbs": nb / t / 1e9, "frac": nb / t / 1e9 / peak})
+    assert rq.rq_workspace_status(ws) == 0
+
+
 def measure(w, reps, peak, emit):
     import torch
     import kv_cache_residual_rq_b200 as rq
@@ -103,6 +145,9 @@ def measure(w, reps, peak, emit):
               "bytes": nb, "gbs": nb / t / 1e9, "frac": nb / t / 1e9 / peak,
               "tokens_per_s_per_head_call": w.batch / t})
     assert rq.rq_workspace_status(ws) == 0
+    if w.name in ("ouro1.4b_decode", "deep_loop_gqa"):
+        measure_paged(w, refk, refv, ck[0], cv[0], sk[0], sv[0], q, out, peak, reps, emit)
+        torch.cuda.empty_cache()
     if w.name in ("ouro1.4b_decode", "deep_loop_gqa"):
         # compressed reference (reference loop as rotated INT8 / INT4 codes)
         xk1 = synth.loop_kv(w, 0, 0, 1, refk)
