@@ -199,7 +199,9 @@ def oracle_cr_kv(xk, xv, refk, refv, ref_bits, bits, g, seed, b, h, ctx):
     (8, 8, 128, 32, 16, False), (8, 4, 64, 32, 2, False), (8, 2, 64, 64, 4, True),
     (8, 8, 64, 32, 2, False), (8, 4, 128, 64, 16, True),
     (4, 4, 128, 32, 2, False), (4, 2, 128, 64, 4, True), (4, 8, 64, 32, 2, True),
-    (4, 4, 64, 64, 16, False), (4, 8, 128, 32, 16, True)])
+    (4, 4, 64, 64, 16, False), (4, 8, 128, 32, 16, True),
+    # INT2 residuals with 64-dim groups (ldmatrix code words) at d 64
+    (8, 4, 64, 64, 2, True), (4, 2, 64, 64, 2, False)])
 def test_cr_decode_grouped_queries(ref_bits, G, d, g, bits, varlen):
     """Grouped queries over an INT8 or INT4 compressed reference (the
     tensor-core kernel): G query rows per kv head, several tiles, ragged and
