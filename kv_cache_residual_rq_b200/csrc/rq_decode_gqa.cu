@@ -990,31 +990,31 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
             mma_bf16(ores[4 * j + i], a, bh0, bh1);
             mma_bf16(ores[4 * j + i], a, bl0, bl1);
           }
-          continue;
-        }
+        } else {
 #pragma unroll
-        for (int mt = j * KSG; mt < (j + 1) * KSG; ++mt) {
-          // codes of dims 16mt + g (lo halves) and 16mt + g + 8 (hi halves)
-          uint32_t x[4];
+          for (int mt = j * KSG; mt < (j + 1) * KSG; ++mt) {
+            // codes of dims 16mt + g (lo halves) and 16mt + g + 8 (hi halves)
+            uint32_t x[4];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint32_t* cw = reinterpret_cast<const uint32_t*>(st + C::OFF_CV + tk[k] * C::CROW);
-            if constexpr (BITS == 2) {
-              x[k] = ((cw[mt] >> (2 * g)) & 0x00030003u) | kMagic;
-            } else {
-              const uint32_t lo = (cw[2 * mt] >> (4 * g)) & 0xFu;
-              const uint32_t hi = (cw[2 * mt + 1] >> (4 * g)) & 0xFu;
-              x[k] = lo | (hi << 16) | kMagic;
+            for (int k = 0; k < 4; ++k) {
+              const uint32_t* cw = reinterpret_cast<const uint32_t*>(st + C::OFF_CV + tk[k] * C::CROW);
+              if constexpr (BITS == 2) {
+                x[k] = ((cw[mt] >> (2 * g)) & 0x00030003u) | kMagic;
+              } else {
+                const uint32_t lo = (cw[2 * mt] >> (4 * g)) & 0xFu;
+                const uint32_t hi = (cw[2 * mt + 1] >> (4 * g)) & 0xFu;
+                x[k] = lo | (hi << 16) | kMagic;
+              }
             }
+            const uint32_t m128 = 0xC300C300u;   // {-128, -128}
+            uint32_t a[4];
+            a[0] = badd2_u(__byte_perm(x[0], x[1], 0x5410), m128);   // dim g,   tokens 2q, 2q+1
+            a[1] = badd2_u(__byte_perm(x[0], x[1], 0x7632), m128);   // dim g+8
+            a[2] = badd2_u(__byte_perm(x[2], x[3], 0x5410), m128);   // dim g,   tokens 2q+8, 2q+9
+            a[3] = badd2_u(__byte_perm(x[2], x[3], 0x7632), m128);   // dim g+8
+            mma_bf16(ores[mt], a, bh0, bh1);
+            mma_bf16(ores[mt], a, bl0, bl1);
           }
-          const uint32_t m128 = 0xC300C300u;   // {-128, -128}
-          uint32_t a[4];
-          a[0] = badd2_u(__byte_perm(x[0], x[1], 0x5410), m128);   // dim g,   tokens 2q, 2q+1
-          a[1] = badd2_u(__byte_perm(x[0], x[1], 0x7632), m128);   // dim g+8
-          a[2] = badd2_u(__byte_perm(x[2], x[3], 0x5410), m128);   // dim g,   tokens 2q+8, 2q+9
-          a[3] = badd2_u(__byte_perm(x[2], x[3], 0x7632), m128);   // dim g+8
-          mma_bf16(ores[mt], a, bh0, bh1);
-          mma_bf16(ores[mt], a, bl0, bl1);
         }
       }
     }
