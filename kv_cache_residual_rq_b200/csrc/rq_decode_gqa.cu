@@ -63,9 +63,11 @@ struct GCfg {
   static constexpr int TILE = kDecodeTile;                 // 64 tokens
   static constexpr int WTOK = TILE / kConsumerWarps;       // 16 tokens per warp
   static constexpr bool RES = (BITS != 16);
-  // INT2 residual with 64-dim scale groups: a 16-byte row chunk of codes is
-  // exactly one scale group, so ldmatrix reads the code rows directly
-  static constexpr bool LDM2 = (BITS == 2 && GROUP == 64);
+  // INT2 residual: ldmatrix reads the code rows directly.  With 64-dim scale
+  // groups a 16-byte row chunk is exactly one group; with 32-dim groups it
+  // holds two, and lanes exchange words (one shuffle) so that every k-step
+  // and every m-tile stays inside one group.
+  static constexpr bool LDM2 = (BITS == 2);
   static constexpr int NCH = D / 64;                        // 64-dim chunks per row
   static constexpr bool CR = (RB == 8);                    // INT8 compressed reference
   static constexpr bool CR4 = (RB == 4);                   // INT4 compressed reference
@@ -521,8 +523,13 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
           // INT2 with ldmatrix words: k-step kk = 4c + t of chunk c carries
           // dims 64c + 16q + 2t + {0, 8 | 1, 9} (codes 2t, 2t+8 | 2t+1, 2t+9
           // of the word holding the chunk's dims 16q .. 16q+15)
-          const float* trow = qt + g * D +
-                              (C::LDM2 ? 64 * (kk >> 2) + 16 * q + 2 * (kk & 3) : 16 * kk + 2 * q);
+          // (32-dim groups: k-step kk is half t = kk & 1 of group (kk >> 1) & 1 of
+          // chunk kk >> 2; lane q reads the word of dims 16 (q & 1) .. of that
+          // group and takes its codes 2u, 2u+8 | 2u+1, 2u+9, u = 2t + (q >> 1))
+          const int lo2 = GROUP == 64 ? 16 * q + 2 * (kk & 3)
+                                      : 32 * ((kk >> 1) & 1) + 16 * (q & 1) +
+                                            2 * (2 * (kk & 1) + (q >> 1));
+          const float* trow = qt + g * D + (C::LDM2 ? 64 * (kk >> 2) + lo2 : 16 * kk + 2 * q);
           fa[0] = pack_bf16(qrow[0], qrow[1]);       // exact: q is bf16
           fa[1] = pack_bf16(qrow[8], qrow[9]);
           if constexpr (BITS == 2) {
@@ -592,7 +599,11 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
       for (int e = 0; e < 4; ++e) {
         const int r = 2 * q + (e & 1);
         const int dim = 16 * mt + g + 8 * (e >> 1);
-        const int dim_res = C::LDM2 ? 64 * (mt >> 2) + 8 * g + 2 * (mt & 3) + (e >> 1) : dim;
+        const int dim_res =
+            !C::LDM2      ? dim
+            : GROUP == 64 ? 64 * (mt >> 2) + 8 * g + 2 * (mt & 3) + (e >> 1)
+                          : 64 * (mt >> 2) + 32 * ((mt >> 1) & 1) + 8 * (g & 3) + 4 * (mt & 1) +
+                                2 * (g >> 2) + (e >> 1);
         const int dim_ref = C::CR    ? 16 * mt + 2 * g + (e >> 1)
                             : C::CR4 ? 32 * (mt >> 1) + 4 * g + 2 * (mt & 1) + (e >> 1)
                                      : dim;
@@ -659,7 +670,8 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
     // compressed reference: per-group f16 sums sum_k q~_k 2^E c_k 2^-24
     float c8[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
     uint32_t b8[4];          // ldmatrix words of two k-steps: (nt 0, kk), (nt 1, kk), (nt 0, kk + 1), ..
-    uint32_t ck4[4];         // INT2 residual (64-dim groups): the tile's K code words
+    uint32_t ck4[4];         // INT2 residual: the tile's K code words
+    uint32_t ckp[4];         // 32-dim groups: the same words of lane ^ 2
 #pragma unroll
     for (int kk = 0; kk < KT; ++kk) {
       if constexpr (C::CR) {
@@ -749,6 +761,10 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
               ck4[0] = r2[0];
               ck4[1] = r2[1];
             }
+            if constexpr (GROUP == 32) {
+#pragma unroll
+              for (int m = 0; m < 2 * C::NCH; ++m) ckp[m] = __shfl_xor_sync(FULL, ck4[m], 2);
+            }
           }
         }
 #pragma unroll
@@ -756,12 +772,21 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
           const uint32_t* cw = reinterpret_cast<const uint32_t*>(st + C::OFF_CK + tb[nt] * C::CROW);
           uint32_t b0, b1;
           if constexpr (C::LDM2) {
-            // codes 2t, 2t+8 | 2t+1, 2t+9 of the word at mantissa bits 1-2:
-            // bf16 128 + 2c, exact (as k_levels2)
-            const uint32_t w = ck4[2 * (kk >> 2) + nt];
-            const int t = kk & 3;
-            b0 = ((t == 0 ? (w << 1) : (w >> (4 * t - 1))) & 0x00060006u) | kMagic;
-            b1 = ((w >> (4 * t + 1)) & 0x00060006u) | kMagic;
+            // codes 2u, 2u+8 | 2u+1, 2u+9 of the word at mantissa bits 1-2:
+            // bf16 128 + 2c, exact (as k_levels2); bit 31 (code 15) is not
+            // among the codes the shifted copy serves
+            uint32_t w;
+            int u;
+            if constexpr (GROUP == 64) {
+              w = ck4[2 * (kk >> 2) + nt];
+              u = kk & 3;
+            } else {
+              const int idx = 2 * (kk >> 2) + nt;
+              w = ((q >> 1) == ((kk >> 1) & 1)) ? ck4[idx] : ckp[idx];
+              u = 2 * (kk & 1) + (q >> 1);
+            }
+            b0 = (((w << 1) >> (4 * u)) & 0x00060006u) | kMagic;
+            b1 = ((w >> (4 * u + 1)) & 0x00060006u) | kMagic;
           } else if constexpr (BITS == 2) {
             k_levels2(cw[kk], q, b0, b1);
           } else {
@@ -949,7 +974,7 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
       // ldmatrix.trans: word = codes of dims 8g .. 8g+7 of a 64-dim chunk
       // (token 2q low half, 2q+1 high half, code i at bits 2i); (tokens 0-7,
       // chunk 0), (8-15, chunk 0)[, (0-7, chunk 1), (8-15, chunk 1)]
-      uint32_t cv4[4];
+      uint32_t cv4[4], cvp[4];   // cvp (32-dim groups): the words of lane ^ 16
       if constexpr (C::LDM2) {
         const int m = (lane >> 3) & (2 * C::NCH - 1);
         const uint32_t a = smem_u32(st + C::OFF_CV + (wtok + (m & 1) * 8 + r7) * C::CROW +
@@ -961,6 +986,10 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
           ldsm_x2_trans(a, r2);
           cv4[0] = r2[0];
           cv4[1] = r2[1];
+        }
+        if constexpr (GROUP == 32) {
+#pragma unroll
+          for (int m2 = 0; m2 < 2 * C::NCH; ++m2) cvp[m2] = __shfl_xor_sync(FULL, cv4[m2], 16);
         }
       }
 #pragma unroll
@@ -976,19 +1005,39 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
         split_bf16(wv[0], wv[1], bh0, bl0);
         split_bf16(wv[2], wv[3], bh1, bl1);
         if constexpr (C::LDM2) {
-          // chunk j: m-tile 4j + i has m-rows g, g + 8 = dims 64j + 8g + 2i (+ 1);
           // operands (128 + c) - 128 = c, exact (the accumulator carries no
           // offset across the head's tiles)
           const uint32_t m128 = 0xC300C300u;   // {-128, -128}
+          if constexpr (GROUP == 64) {
+            // chunk j: m-tile 4j + i has m-rows g, g + 8 = dims 64j + 8g + 2i (+ 1)
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint32_t R0 = cv4[2 * j], R1 = cv4[2 * j + 1];
-            const uint32_t a[4] = {badd2_u(((R0 >> (4 * i)) & 0x00030003u) | kMagic, m128),
-                                   badd2_u(((R0 >> (4 * i + 2)) & 0x00030003u) | kMagic, m128),
-                                   badd2_u(((R1 >> (4 * i)) & 0x00030003u) | kMagic, m128),
-                                   badd2_u(((R1 >> (4 * i + 2)) & 0x00030003u) | kMagic, m128)};
-            mma_bf16(ores[4 * j + i], a, bh0, bh1);
-            mma_bf16(ores[4 * j + i], a, bl0, bl1);
+            for (int i = 0; i < 4; ++i) {
+              const uint32_t R0 = cv4[2 * j], R1 = cv4[2 * j + 1];
+              const uint32_t a[4] = {badd2_u(((R0 >> (4 * i)) & 0x00030003u) | kMagic, m128),
+                                     badd2_u(((R0 >> (4 * i + 2)) & 0x00030003u) | kMagic, m128),
+                                     badd2_u(((R1 >> (4 * i)) & 0x00030003u) | kMagic, m128),
+                                     badd2_u(((R1 >> (4 * i + 2)) & 0x00030003u) | kMagic, m128)};
+              mma_bf16(ores[4 * j + i], a, bh0, bh1);
+              mma_bf16(ores[4 * j + i], a, bl0, bl1);
+            }
+          } else {
+            // group j = half gc of chunk c: lanes g and g ^ 4 both hold the
+            // word of dims 8 (g & 3) .. +7 of the group; m-tile 2j + i has
+            // m-rows g, g + 8 = dims 64c + 32gc + 8 (g & 3) + 4i + 2 (g >> 2) (+ 1)
+            const int c = j >> 1, gc = j & 1;
+            const bool own = (g >> 2) == gc;
+            const uint32_t R0 = own ? cv4[2 * c] : cvp[2 * c];
+            const uint32_t R1 = own ? cv4[2 * c + 1] : cvp[2 * c + 1];
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              const int sh = 2 * (4 * i + 2 * (g >> 2));
+              const uint32_t a[4] = {badd2_u(((R0 >> sh) & 0x00030003u) | kMagic, m128),
+                                     badd2_u(((R0 >> (sh + 2)) & 0x00030003u) | kMagic, m128),
+                                     badd2_u(((R1 >> sh) & 0x00030003u) | kMagic, m128),
+                                     badd2_u(((R1 >> (sh + 2)) & 0x00030003u) | kMagic, m128)};
+              mma_bf16(ores[2 * j + i], a, bh0, bh1);
+              mma_bf16(ores[2 * j + i], a, bl0, bl1);
+            }
           }
         } else {
 #pragma unroll
