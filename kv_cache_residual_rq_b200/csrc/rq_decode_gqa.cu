@@ -68,6 +68,9 @@ struct GCfg {
   // holds two, and lanes exchange words (one shuffle) so that every k-step
   // and every m-tile stays inside one group.
   static constexpr bool LDM2 = (BITS == 2);
+  // INT4 residual: a 16-byte row chunk (32 dims) always lies inside one scale
+  // group; ldmatrix words of eight codes, no exchange needed
+  static constexpr bool LDM4 = (BITS == 4);
   static constexpr int NCH = D / 64;                        // 64-dim chunks per row
   static constexpr bool CR = (RB == 8);                    // INT8 compressed reference
   static constexpr bool CR4 = (RB == 4);                   // INT4 compressed reference
@@ -541,6 +544,17 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
                     (bf16_hi_f(fh[0]) + bf16_hi_f(fl[0]))) +
                    ((bf16_lo_f(fh[1]) + bf16_lo_f(fl[1])) +
                     (bf16_hi_f(fh[1]) + bf16_hi_f(fl[1])));
+          } else if constexpr (C::LDM4) {
+            // k-step kk = half h of 32-dim chunk kk >> 1: k positions 2q, 2q+1 |
+            // 2q+8, 2q+9 carry dims 8q + 2h + {0, 4 | 1, 5} (the word's codes
+            // 2h, 2h+4 | 2h+1, 2h+5, each register's two codes 16 bits apart)
+            const float* t4 = qt + g * D + 32 * (kk >> 1) + 8 * q + 2 * (kk & 1);
+            split_bf16(cd * t4[0], cd * t4[4], fh[0], fl[0]);
+            split_bf16(cd * t4[1], cd * t4[5], fh[1], fl[1]);
+            sqj += ((bf16_lo_f(fh[0]) + bf16_lo_f(fl[0])) +
+                    (bf16_hi_f(fh[0]) + bf16_hi_f(fl[0]))) +
+                   ((bf16_lo_f(fh[1]) + bf16_lo_f(fl[1])) +
+                    (bf16_hi_f(fh[1]) + bf16_hi_f(fl[1])));
           } else {
             split_bf16(cd * trow[0], cd * trow[1], fh[0], fl[0]);
             split_bf16(cd * trow[8], cd * trow[9], fh[1], fl[1]);
@@ -548,7 +562,7 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
         } else {
           fa[0] = fa[1] = fh[0] = fh[1] = fl[0] = fl[1] = 0u;
         }
-        if (BITS == 2 && (kk + 1) % KSG == 0) {      // end of a scale group
+        if ((BITS == 2 || C::LDM4) && (kk + 1) % KSG == 0) {      // end of a scale group
           sqj += __shfl_xor_sync(FULL, sqj, 1);
           sqj += __shfl_xor_sync(FULL, sqj, 2);
           if (row_ok && q == 0) sq_s[g * NG + kk / KSG] = sqj;
@@ -600,7 +614,8 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
         const int r = 2 * q + (e & 1);
         const int dim = 16 * mt + g + 8 * (e >> 1);
         const int dim_res =
-            !C::LDM2      ? dim
+            C::LDM4       ? 32 * (mt >> 1) + 4 * g + 2 * (mt & 1) + (e >> 1)
+            : !C::LDM2    ? dim
             : GROUP == 64 ? 64 * (mt >> 2) + 8 * g + 2 * (mt & 3) + (e >> 1)
                           : 64 * (mt >> 2) + 32 * ((mt >> 1) & 1) + 8 * (g & 3) + 4 * (mt & 1) +
                                 2 * (g >> 2) + (e >> 1);
@@ -746,6 +761,16 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
         const uint2 fl = *reinterpret_cast<const uint2*>(qfrag + ((2 * KT + kk) * 32 + lane) * 2);
         const uint32_t ah[4] = {fh.x, 0u, fh.y, 0u};
         const uint32_t al[4] = {fl.x, 0u, fl.y, 0u};
+        if constexpr (C::LDM4) {
+          // every fourth k-step: words (nt 0, chunk), (nt 1, chunk), (nt 0,
+          // chunk + 1), (nt 1, chunk + 1) of two 32-dim chunks
+          if ((kk & 3) == 0) {
+            const int m = lane >> 3;
+            ldsm_x4(smem_u32(st + C::OFF_CK + (wtok + (m & 1) * 8 + r7) * C::CROW +
+                             ((kk >> 1) + (m >> 1)) * 16),
+                    ck4);
+          }
+        }
         if constexpr (C::LDM2) {
           // the whole warp tile's K codes in one ldmatrix: words (nt 0, chunk
           // 0), (nt 1, chunk 0)[, (nt 0, chunk 1), (nt 1, chunk 1)]
@@ -787,6 +812,12 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
             }
             b0 = (((w << 1) >> (4 * u)) & 0x00060006u) | kMagic;
             b1 = ((w >> (4 * u + 1)) & 0x00060006u) | kMagic;
+          } else if constexpr (C::LDM4) {
+            // codes 2h, 2h+4 | 2h+1, 2h+5 at mantissa bits 1-4: bf16 128 + 2c, exact
+            const uint32_t w = ck4[2 * ((kk >> 1) & 1) + nt];
+            const int h = kk & 1;
+            b0 = (((w << 1) >> (8 * h)) & 0x001E001Eu) | kMagic;
+            b1 = ((w >> (8 * h + 3)) & 0x001E001Eu) | kMagic;
           } else if constexpr (BITS == 2) {
             k_levels2(cw[kk], q, b0, b1);
           } else {
@@ -803,8 +834,11 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
           for (int nt = 0; nt < 2; ++nt) {
             const float sk0 = half_at(st + C::OFF_SK + sc_off + tok0[nt] * SB + 2 * j);
             const float sk1 = half_at(st + C::OFF_SK + sc_off + (tok0[nt] + 1) * SB + 2 * j);
-            // INT2 operands are 128 + 2c: q~ . l = result - 131 sum q~
-            const float off = (BITS == 2 && row_ok) ? 131.0f * sq_s[g * NG + j] : 0.0f;
+            // INT2 operands are 128 + 2c: q~ . l = result - 131 sum q~; INT4
+            // (ldmatrix words) 128 + 2c: result - 143 sum q~
+            const float off = ((BITS == 2 || C::LDM4) && row_ok)
+                                  ? (BITS == 2 ? 131.0f : 143.0f) * sq_s[g * NG + j]
+                                  : 0.0f;
             cref[nt][0] = fmaf(sk0, ct[nt][0] - off, cref[nt][0]);
             cref[nt][1] = fmaf(sk1, ct[nt][1] - off, cref[nt][1]);
 #pragma unroll
@@ -1037,6 +1071,28 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
                                      badd2_u(((R1 >> (sh + 2)) & 0x00030003u) | kMagic, m128)};
               mma_bf16(ores[2 * j + i], a, bh0, bh1);
               mma_bf16(ores[2 * j + i], a, bl0, bl1);
+            }
+          }
+        } else if constexpr (C::LDM4) {
+          // the group's 32-dim chunks by ldmatrix.trans: word = codes of dims
+          // 4g .. 4g+3 of the chunk (token 2q low half, 2q+1 high half, code i
+          // at bits 4i); m-tile 2 ch has m-rows g, g + 8 = dims 4g, 4g + 1,
+          // m-tile 2 ch + 1 dims 4g + 2, 4g + 3; operands (128 + c) - 128 = c
+          const uint32_t m128 = 0xC300C300u;   // {-128, -128}
+#pragma unroll
+          for (int ch = j * GROUP / 32; ch < (j + 1) * GROUP / 32; ++ch) {
+            const int m = (lane >> 3) & 1;
+            uint32_t v[2];   // (tokens 0-7, chunk ch), (tokens 8-15, chunk ch)
+            ldsm_x2_trans(smem_u32(st + C::OFF_CV + (wtok + m * 8 + r7) * C::CROW + ch * 16), v);
+#pragma unroll
+            for (int xy = 0; xy < 2; ++xy) {
+              const int sh = 8 * xy;
+              const uint32_t a[4] = {badd2_u(((v[0] >> sh) & 0x000F000Fu) | kMagic, m128),
+                                     badd2_u(((v[0] >> (sh + 4)) & 0x000F000Fu) | kMagic, m128),
+                                     badd2_u(((v[1] >> sh) & 0x000F000Fu) | kMagic, m128),
+                                     badd2_u(((v[1] >> (sh + 4)) & 0x000F000Fu) | kMagic, m128)};
+              mma_bf16(ores[2 * ch + xy], a, bh0, bh1);
+              mma_bf16(ores[2 * ch + xy], a, bl0, bl1);
             }
           }
         } else {
