@@ -557,3 +557,77 @@ def test_cr_residual_moves_the_loop_closer(ref_bits):
     K_ref = oracle.reconstruct_rows_cr_f64(rw, rs, None, None, ref_bits, 2, g, seed, d)
     K_l = oracle.reconstruct_rows_cr_f64(rw, rs, w, s, ref_bits, 2, g, seed, d)
     assert np.linalg.norm(K_l - xf) < np.linalg.norm(K_ref - xf)
+
+
+def _nearest_levels_on_absmax_grid(e, bits):
+    """Brute force over the 2^b points amax*l/(2^b - 1), l odd: the level of
+    the nearest point per coordinate, and the gap to the runner-up (how far
+    the coordinate sits from a decision boundary)."""
+    top = (1 << bits) - 1
+    levels = np.arange(-top, top + 1, 2)
+    grid = np.abs(e).max() * levels / top
+    dist = np.abs(e[:, None] - grid[None, :])
+    order = np.argsort(dist, axis=1, kind="stable")
+    near = np.take_along_axis(dist, order[:, :2], axis=1)
+    return levels[order[:, 0]], near[:, 1] - near[:, 0]
+
+
+def _check_cr_residual_base(x, ref, ref_bits, bits, g, seed):
+    """The residual of a non-final loop is quantised against the
+    reconstructed reference in the rotated domain, e = R x - z with
+    z = s_ref l_ref (ResidualQuant Abstract: the final loop is the reference;
+    this format stores that reference itself as rotated codes).  e is formed
+    here in fp64 from the explicit rotation matrix and the reference's own
+    codes and scales; the loop's codes must be the nearest levels of e on its
+    absmax grid (away from decision boundaries) and its scales the
+    least-squares optimum for those codes, to one fp16 step."""
+    d = x.shape[-1]
+    rw, rs, w, s = oracle.encode_rows_cr_f32(x, ref, ref_bits, bits, g, seed)
+    R = oracle.rotation_matrix_f64(d, seed)
+    xf = oracle.bf16_to_f32(x).astype(np.float64)
+    rtop, top = (1 << ref_bits) - 1, (1 << bits) - 1
+    checked = 0
+    for i in range(x.shape[0]):
+        cr = oracle.unpack_codes(rw[i], ref_bits, d).astype(int)
+        sr = np.repeat([oracle.f16_to_f64(int(h)) for h in rs[i]], g)
+        e = R @ xf[i] - sr * (2 * cr - rtop)
+        lv = 2 * oracle.unpack_codes(w[i], bits, d).astype(int) - top
+        for k in range(d // g):
+            eg, lg = e[k * g:(k + 1) * g], lv[k * g:(k + 1) * g]
+            want, gap = _nearest_levels_on_absmax_grid(eg, bits)
+            clear = gap > 1e-4 * np.abs(eg).max()
+            assert clear.sum() >= g // 2
+            assert np.array_equal(lg[clear], want[clear]), (i, k)
+            s_opt = float(eg @ lg) / float(lg @ lg)
+            s16 = oracle.f16_to_f64(int(s[i, k]))
+            step = 2.0 ** (math.floor(math.log2(abs(s_opt))) - 10)
+            assert abs(s16 - s_opt) <= step + 1e-6 * abs(s_opt), (i, k, s16, s_opt)
+            checked += 1
+    return checked
+
+
+@pytest.mark.parametrize("ref_bits", [4, 8])
+def test_cr_loop_equal_to_reference_encodes_the_reference_error(ref_bits):
+    # a non-final loop identical to the final loop: its residual is the
+    # reference's own quantisation error R ref - z, which is not zero, so the
+    # loop must end up strictly closer to ref than the reference codes alone
+    rng = np.random.default_rng(60 + ref_bits)
+    d, g, seed = 128, 32, 5
+    ref = _rand_bf16(rng, (12, d), scale=2.0)
+    assert _check_cr_residual_base(ref, ref, ref_bits, 2, g, seed) == 12 * d // g
+    rw, rs, w, s = oracle.encode_rows_cr_f32(ref, ref, ref_bits, 2, g, seed)
+    assert np.all(s != 0)
+    rf = oracle.bf16_to_f32(ref).astype(np.float64)
+    K_ref = oracle.reconstruct_rows_cr_f64(rw, rs, None, None, ref_bits, 2, g, seed, d)
+    K_l = oracle.reconstruct_rows_cr_f64(rw, rs, w, s, ref_bits, 2, g, seed, d)
+    for i in range(ref.shape[0]):
+        assert np.linalg.norm(K_l[i] - rf[i]) < np.linalg.norm(K_ref[i] - rf[i])
+
+
+@pytest.mark.parametrize("ref_bits,bits,g", [(4, 2, 32), (4, 4, 64), (8, 2, 64)])
+def test_cr_residual_is_taken_against_the_reconstructed_reference(ref_bits, bits, g):
+    rng = np.random.default_rng(70 + ref_bits + bits + g)
+    d, seed = 128, 8
+    ref = _rand_bf16(rng, (10, d))
+    x = _bf16(oracle.bf16_to_f32(ref) + 0.1 * rng.standard_normal((10, d)).astype(np.float32))
+    assert _check_cr_residual_base(x, ref, ref_bits, bits, g, seed) == 10 * d // g
