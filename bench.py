@@ -14,6 +14,19 @@ INT2 residuals with group 32), synthetic seeded data.
 Under torchrun each rank runs its own copy of the workload (weak scaling);
 the timed region is bracketed by a barrier and a device synchronize, the
 elapsed time is the max over ranks.  Rank 0 prints one JSON line.
+
+Besides the headline (the --steps timed region) the line carries:
+  sustained   the same step held for --sustain-s seconds, with its own clock
+              record (the 1 kW power cap lowers the SM clock in steady state)
+  workloads   (N=1) the other configured workloads, timed in the same run
+              with CUDA events around back-to-back launches and the SM clock
+              sampled meanwhile: the mixed-precision 32K decode calls (loop 1
+              INT4, loop 2 INT2, loop 4 BF16), the deep-loop grouped-query
+              decode calls (INT2, BF16), the whole 32K-prefill rq_encode in one
+              call, and the budgeted batch sweep's maximum batches with their
+              full 24-layer caches allocated in HBM
+  cpu_baseline (N=1) the oracle on this host's cores: decode on one thread
+              and on every core, and the encoder's GB/s
 """
 import argparse
 import hashlib
@@ -129,116 +142,7 @@ def gpu_id_for(device_index):
 # workload
 # ---------------------------------------------------------------------------
 
-def algorithmic_bytes(w, bits):
-    """HBM bytes one decode call must move: reference K/V, codes, scales, q, out."""
-    heads_t = w.batch * w.kv_heads * w.ctx
-    b = 2 * heads_t * w.head_dim * 2
-    if bits != 16:
-        b += 2 * heads_t * w.head_dim * bits // 8 + 2 * heads_t * (w.head_dim // w.group) * 2
-    b += w.batch * w.q_heads * w.head_dim * (2 + 4)
-    return b
-
-
-class DecodeStep:
-    """Device-resident cache of every layer plus the per-step inputs.
-
-    Cache arrays are contiguous across layers, [layers][K, V][B][Hkv][T][...],
-    so the step's append-encode covers every layer in one call."""
-
-    def __init__(self, w, device):
-        import torch
-        import kv_cache_residual_rq_b200 as rq
-        from kv_cache_residual_rq_b200 import synth
-        self.w, self.rq, self.torch = w, rq, torch
-        L, N, B, H, T, d = w.loops, w.layers, w.batch, w.kv_heads, w.ctx, w.head_dim
-        self.shape = rq.make_shape(B, H, T, d, w.group, w.q_heads)
-        cache_shape = rq.make_shape(N * 2 * B, H, T, d, w.group)
-        self.ref = torch.empty((N, 2, B, H, T, d), dtype=torch.bfloat16, device=device)
-        self.codes = [rq.alloc_codes(cache_shape, b, device) for b in w.bits]
-        self.scales = [rq.alloc_scales(cache_shape, b, device) for b in w.bits]
-        # exact bytes of one (layer, K or V) part: parts are packed back to back
-        self.code_bytes = [B * H * T * d * b // 8 for b in w.bits]
-        self.scale_bytes = [B * H * T * (d // w.group) * 2 for b in w.bits]
-        assert all(n % 16 == 0 for n in self.code_bytes + self.scale_bytes)
-        layer_shape = rq.make_shape(B, H, T, d, w.group)
-        for layer in range(N):
-            for kind in (0, 1):
-                r = synth.reference(w, layer, kind, device)
-                self.ref[layer, kind].copy_(r)
-                loops = [synth.loop_kv(w, layer, kind, l, r) for l in range(1, L)]
-                part = layer * 2 + kind
-                rq.rq_encode(layer_shape, loops, self.ref[layer, kind], list(w.bits), w.seed,
-                             [self._slice(self.codes[l], self.code_bytes[l], part)
-                              for l in range(L - 1)],
-                             [self._slice(self.scales[l], self.scale_bytes[l], part)
-                              for l in range(L - 1)])
-                del loops, r
-            torch.cuda.empty_cache()
-        # per-step inputs: one query per (loop, layer), and the new token's K/V
-        # of every loop and layer ([loop][layer][K, V][B][Hkv][1][d])
-        self.q = torch.stack([torch.stack([synth.query(w, layer, loop, device)
-                                           for layer in range(N)]) for loop in range(1, L + 1)])
-        g = torch.Generator(device=device)
-        g.manual_seed(w.seed * 31 + 7)
-        newref = torch.randn((N, 2, B, H, 1, d), generator=g, device=device)
-        self.new_kv = torch.stack(
-            [(newref + w.sigma[l] * torch.randn(newref.shape, generator=g, device=device))
-             .to(torch.bfloat16) for l in range(L - 1)] + [newref.to(torch.bfloat16)])
-        self.append_shape = rq.make_shape(N * 2 * B, H, 1, d, w.group)
-        self.out = torch.empty((L, N, B, w.q_heads, d), dtype=torch.float32, device=device)
-        self.ws = rq.alloc_workspace(self.shape, device)
-        self.ws_bytes = self.ws.numel()
-        self.launches_per_step = L * N + 1
-
-    @staticmethod
-    def _slice(buf, nbytes, part):
-        return buf[part * nbytes:(part + 1) * nbytes]
-
-    def run(self, stream, timers=None, bufs=None):
-        """One decode step: every (loop, layer) attends over the cache plus the
-        new token's BF16 K/V of that loop; then the new token is encoded into
-        the cache (the last slot is reused every step, so T stays fixed).
-        timers: list to append (start, end, bits, calls) per loop segment --
-        events only at loop boundaries, so consecutive calls of a loop stay
-        back to back and each launch overlaps its predecessor's tail
-        (programmatic dependent launch); an event between two launches would
-        serialise them.  bufs: (q, new_kv, out) tensors to use instead of the
-        step's own (double-buffered end-to-end loop)."""
-        rq, w, torch = self.rq, self.w, self.torch
-        st = stream.cuda_stream
-        q_all, kv_all, out_all = bufs if bufs is not None else (self.q, self.new_kv, self.out)
-        T = w.ctx
-        for li in range(w.loops):
-            bits = w.bits[li] if li < w.loops - 1 else 16
-            ev = None
-            if timers is not None:
-                ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                ev[0].record(stream)
-            for layer in range(w.layers):
-                ck = cv = sk = sv = None
-                if bits != 16:
-                    ck = self._slice(self.codes[li], self.code_bytes[li], 2 * layer)
-                    cv = self._slice(self.codes[li], self.code_bytes[li], 2 * layer + 1)
-                    sk = self._slice(self.scales[li], self.scale_bytes[li], 2 * layer)
-                    sv = self._slice(self.scales[li], self.scale_bytes[li], 2 * layer + 1)
-                rq.rq_decode_attention_tail(
-                    self.shape, q_all[li, layer], self.ref[layer, 0], self.ref[layer, 1],
-                    ck, cv, sk, sv, bits, w.seed, 0.0, kv_all[li, layer, 0],
-                    kv_all[li, layer, 1], 1, 1, out_all[li, layer], self.ws, self.ws_bytes, st)
-            if ev is not None:
-                ev[1].record(stream)
-                timers.append((ev[0], ev[1], bits, w.layers))
-        rq.rq_encode_at(self.append_shape, 1, 0, T, T - 1, list(kv_all[:w.loops - 1]),
-                        kv_all[w.loops - 1], list(w.bits), w.seed, self.codes, self.scales,
-                        self.ref, st)
-
-    def step_bytes(self):
-        w = self.w
-        total = 0
-        for li in range(w.loops):
-            bits = w.bits[li] if li < w.loops - 1 else 16
-            total += w.layers * algorithmic_bytes(w, bits)
-        return total
+from kv_cache_residual_rq_b200.step import DecodeStep, algorithmic_bytes  # noqa: E402
 
 
 # the sources that make up the single-query decode kernel the roofline names
@@ -316,6 +220,34 @@ def hbm_peak():
 # ---------------------------------------------------------------------------
 
 _ORACLE_INPUTS = {}
+_ORACLE_CODES = {}
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        return os.cpu_count() or 1
+
+
+def cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
+def _pool_map(fn, items, threads):
+    """Run fn over items on `threads` host threads (the oracle is called
+    through ctypes, which releases the GIL for the duration of each call)."""
+    if threads <= 1:
+        return [fn(i) for i in items]
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(threads) as ex:
+        return list(ex.map(fn, items))
 
 
 def _oracle_inputs(w):
@@ -334,30 +266,50 @@ def _oracle_inputs(w):
     return _ORACLE_INPUTS[w.name]
 
 
-def oracle_head_seconds(w, n_res, n_ref, seed_offset=0):
-    """Time the oracle's decode attention on sampled heads of layer 0.
+def _oracle_head_codes(w, h):
+    """The oracle's own encode of kv head h's loop-1 K/V (prepared, not timed)."""
+    key = (w.name, h)
+    if key not in _ORACLE_CODES:
+        import oracle
+        rk, rv, xk, xv, _ = _oracle_inputs(w)
+        ck, sk, _ = oracle.encode_rows_f32(xk[h], rk[h], w.bits[0], w.group, w.seed)
+        cv, sv, _ = oracle.encode_rows_f32(xv[h], rv[h], w.bits[0], w.group, w.seed)
+        _ORACLE_CODES[key] = (ck, cv, sk, sv)
+    return _ORACLE_CODES[key]
 
-    Returns (seconds per residual head, seconds per reference head).  Inputs
-    are the workload's generator run on the CPU; the oracle encodes them
-    itself (not timed), then its decode attention is timed."""
+
+def oracle_head_seconds(w, n_res, n_ref, threads=1, seed_offset=0):
+    """Time the oracle's decode attention on sampled heads of layer 0, run on
+    `threads` host threads.
+
+    Returns (wall seconds per residual head, wall seconds per reference
+    head): each batch of heads is timed as a whole, so with several threads
+    these are throughput figures.  Inputs are the workload's generator run on
+    the CPU; the oracle encodes them itself beforehand (not timed)."""
     import oracle
-    rk, rv, xk, xv, q = _oracle_inputs(w)
+    oracle.lib()
+    rk, rv, _, _, q = _oracle_inputs(w)
     bits = w.bits[0]
-    t_res = t_ref = 0.0
-    for i in range(n_res):
-        h = (i + seed_offset) % w.kv_heads
-        ck, sk, _ = oracle.encode_rows_f32(xk[h], rk[h], bits, w.group, w.seed)
-        cv, sv, _ = oracle.encode_rows_f32(xv[h], rv[h], bits, w.group, w.seed)
-        qh = q[h * w.G:(h + 1) * w.G]
-        t0 = time.perf_counter()
-        oracle.decode_attention_f64(qh, rk[h], rv[h], ck, cv, sk, sv, bits, w.group, w.seed)
-        t_res += time.perf_counter() - t0
-    for i in range(n_ref):
-        h = (i + seed_offset) % w.kv_heads
-        qh = q[h * w.G:(h + 1) * w.G]
-        t0 = time.perf_counter()
-        oracle.decode_attention_f64(qh, rk[h], rv[h], None, None, None, None, 16, w.group, w.seed)
-        t_ref += time.perf_counter() - t0
+    res_heads = [(i + seed_offset) % w.kv_heads for i in range(n_res)]
+    ref_heads = [(i + seed_offset) % w.kv_heads for i in range(n_ref)]
+    for h in set(res_heads):
+        _oracle_head_codes(w, h)
+
+    def res(h):
+        ck, cv, sk, sv = _oracle_head_codes(w, h)
+        oracle.decode_attention_f64(q[h * w.G:(h + 1) * w.G], rk[h], rv[h], ck, cv, sk, sv,
+                                    bits, w.group, w.seed)
+
+    def ref(h):
+        oracle.decode_attention_f64(q[h * w.G:(h + 1) * w.G], rk[h], rv[h], None, None, None,
+                                    None, 16, w.group, w.seed)
+
+    t0 = time.perf_counter()
+    _pool_map(res, res_heads, threads)
+    t_res = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    _pool_map(ref, ref_heads, threads)
+    t_ref = time.perf_counter() - t0
     return t_res / max(n_res, 1), t_ref / max(n_ref, 1)
 
 
@@ -368,18 +320,63 @@ def oracle_step_seconds(w, s_res, s_ref):
     return heads * (n_res_calls * s_res + n_ref_calls * s_ref)
 
 
-def cpu_baseline(w):
-    n_res, n_ref = 64, 32
+def oracle_encode_gbs(threads, rows_per_job=16384):
+    """The fp32 exact-spec oracle encoder on rows of the 32K-prefill workload
+    (16 heads x rows_per_job/16 tokens of layer 0's K, its 3 INT2 loops),
+    one job per thread.  Returns (GB/s of algorithmic bytes, wall seconds)."""
+    import numpy as np
+    import torch
+    import oracle
+    from kv_cache_residual_rq_b200 import synth
+    from kv_cache_residual_rq_b200.measure import encode_bytes
+    w = synth.ENCODE
+    oracle.lib()
+    key = ("encode", rows_per_job)
+    if key not in _ORACLE_INPUTS:
+        u16 = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)
+        t = rows_per_job // w.kv_heads
+        rk = synth.reference(w, 0, 0, "cpu", batch=1, ctx=t)
+        xs = [synth.loop_kv(w, 0, 0, l, rk) for l in range(1, w.loops)]
+        _ORACLE_INPUTS[key] = (u16(rk[0]).reshape(-1, w.head_dim),
+                               [u16(x[0]).reshape(-1, w.head_dim) for x in xs])
+    ref, xs = _ORACLE_INPUTS[key]
+
+    def job(_):
+        for x, b in zip(xs, w.bits):
+            oracle.encode_rows_f32(x, ref, b, w.group, w.seed)
+
     t0 = time.perf_counter()
-    s_res, s_ref = oracle_head_seconds(w, n_res, n_ref)
+    _pool_map(job, range(threads), threads)
+    wall = time.perf_counter() - t0
+    return encode_bytes(w, rows_per_job) * threads / wall / 1e9, wall
+
+
+def cpu_baseline(w):
+    """The oracle timed on this host: decode (the bench's metric) on one
+    thread and on every core, and the encoder's GB/s likewise."""
+    cores = host_cores()
+    t0 = time.perf_counter()
+    s_res1, s_ref1 = oracle_head_seconds(w, 32, 16, threads=1)
+    single = w.batch / oracle_step_seconds(w, s_res1, s_ref1)
+    s_resn, s_refn = oracle_head_seconds(w, 8 * cores, 4 * cores, threads=cores)
+    multi = w.batch / oracle_step_seconds(w, s_resn, s_refn)
+    enc1, _ = oracle_encode_gbs(1, 65536)
+    encn, _ = oracle_encode_gbs(cores, 16384)
     spent = time.perf_counter() - t0
-    step = oracle_step_seconds(w, s_res, s_ref)
-    return {"value": w.batch / step, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": (f"fp64 oracle decode attention of {n_res} residual-INT2 heads and {n_ref} "
-                       f"reference heads (T={w.ctx}, d={w.head_dim}) of one layer, "
-                       f"{spent:.1f} s single-threaded, scaled to the full step "
-                       f"({w.layers} layers x {w.loops} loops x {w.batch * w.kv_heads} heads); "
-                       f"the append-encode (<0.1% of the step) is not included")}
+    return {"value": multi, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "extrapolated": True, "nproc": os.cpu_count(), "cpu_model": cpu_model(),
+            "single_thread": {"value": single, "unit": UNIT, "cores": 1},
+            "encode": {"unit": "GB/s", "single_thread": enc1, "all_cores": encn,
+                       "sample": ("fp32 exact-spec oracle encoder, 3 INT2 loops of layer 0's "
+                                  "K of the 32K-prefill workload: 65536 rows on 1 thread, "
+                                  f"16384 rows per thread on {cores} threads")},
+            "sample": (f"fp64 oracle decode attention of layer-0 heads (T={w.ctx}, "
+                       f"d={w.head_dim}): {8 * cores} residual-INT2 + {4 * cores} reference "
+                       f"heads on {cores} threads (value), 32 + 16 heads on 1 thread "
+                       f"(single_thread), scaled to the full step ({w.layers} layers x "
+                       f"{w.loops} loops x {w.batch * w.kv_heads} heads); {spent:.1f} s in "
+                       f"all with the encode timing; the append-encode (<0.1% of the step) "
+                       f"is not included")}
 
 
 # ---------------------------------------------------------------------------
@@ -399,26 +396,60 @@ def run_reference(args, w):
     rank, _, world = dist_env()
     if rank != 0:
         return
+    cores = host_cores()
+    n_res, n_ref = cores, max(1, cores // 2)
     for i in range(args.warmup):
-        oracle_head_seconds(w, 1, 1, seed_offset=i)
-    times = []
+        oracle_head_seconds(w, n_res, n_ref, threads=cores, seed_offset=i)
+    times, walls = [], []
     for i in range(args.steps):
-        s_res, s_ref = oracle_head_seconds(w, 1, 1, seed_offset=i)
+        t0 = time.perf_counter()
+        s_res, s_ref = oracle_head_seconds(w, n_res, n_ref, threads=cores, seed_offset=i)
+        walls.append(time.perf_counter() - t0)
         times.append(oracle_step_seconds(w, s_res, s_ref))
     step = statistics.mean(times)
     value = w.batch / step
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step * 1e3,
+        "extrapolated": True,
+        "sampled_heads_per_step": {"residual": n_res, "reference": n_ref},
+        "sample_wall_ms_per_step": statistics.mean(walls) * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded; Ouro-1.4B-shaped KV, no model or dataset)",
         "config": config_dict(w, "n/a (CPU)"),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": (f"each step: fp64 oracle decode attention of 1 residual and 1 "
-                                    f"reference head of layer 0, scaled to the full step")},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "nproc": os.cpu_count(), "cpu_model": cpu_model(),
+                         "sample": (f"each step: fp64 oracle decode attention of {n_res} "
+                                    f"residual and {n_ref} reference heads of layer 0 on "
+                                    f"{cores} threads, scaled to the full step "
+                                    f"(ms_per_step is that extrapolation; the sample itself "
+                                    f"took sample_wall_ms_per_step)")},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def other_workloads(peak, local_rank, args):
+    """The other configured workloads, timed in this run: the mixed-precision
+    32K and deep-loop grouped-query decode calls, the whole 32K-prefill
+    encode, and the budgeted batch sweep at its maximum batches with the full
+    caches held in HBM."""
+    from kv_cache_residual_rq_b200 import capacity, measure, synth
+    make_sampler = lambda: ClockSampler(gpu_id_for(local_rank))
+    entries = measure.bench_workloads(peak, make_sampler)
+    w = synth.ENCODE
+    rows, maxb = capacity.plan(w, w.ctx, synth.SWEEP_BATCHES, synth.KV_BUDGET_BYTES)
+    cap = {"budget_bytes": synth.KV_BUDGET_BYTES, "ctx": w.ctx, "max_batch": maxb,
+           "exceeds_budget": sorted({f"{s} {b}" for s, b, _, ok in rows if not ok}),
+           "runs": []}
+    for scheme in ("rq", "bf16"):
+        r = capacity.run_batch(w, w.ctx, maxb[scheme], scheme, args.capacity_steps, peak,
+                               synth.KV_BUDGET_BYTES)
+        cap["runs"].append({k: r[k] for k in ("scheme", "batch", "cache_bytes_allocated",
+                                              "device_bytes_held", "step_ms", "tokens_per_s",
+                                              "frac_hbm", "workspace_status",
+                                              "outputs_finite")})
+    return {"entries": entries, "capacity": cap}
 
 
 def run_ours(args, w):
@@ -533,6 +564,36 @@ def run_ours(args, w):
     e_elapsed, e_tokens = aggregate(e_start.elapsed_time(e_end) / 1e3, w.batch * args.steps)
     status = rq.rq_workspace_status(state.ws)
 
+    # ---- the same step held for a few seconds (power-capped steady state) ----
+    sustained = None
+    if args.sustain_s > 0:
+        n_sus = max(args.steps, int(args.sustain_s / (max_elapsed / args.steps)))
+        sus_timers = []
+        clocks = ClockSampler(gpu_id_for(local_rank))
+        clocks.start()
+        time.sleep(0.3)
+        barrier()
+        torch.cuda.synchronize(device)
+        s_start = torch.cuda.Event(enable_timing=True)
+        s_end = torch.cuda.Event(enable_timing=True)
+        s_start.record(stream)
+        for _ in range(n_sus):
+            state.run(stream, sus_timers)
+        s_end.record(stream)
+        torch.cuda.synchronize(device)
+        barrier()
+        s_clk = clocks.stop()
+        s_elapsed, s_tokens = aggregate(s_start.elapsed_time(s_end) / 1e3, w.batch * n_sus)
+        s_res = statistics.mean(a.elapsed_time(b) / n for a, b, bits, n in sus_timers
+                                if bits != 16) / 1e3
+        sustained = {"steps": n_sus, "ms_per_step": s_elapsed / n_sus * 1e3,
+                     "value": s_tokens / s_elapsed, "avg_launch_us": s_res * 1e6,
+                     "frac": bytes_res / s_res / 1e9 / peak, "clocks": s_clk,
+                     "launch_kcycles": (s_res * 1e3 * s_clk["sm_mhz"]
+                                        if s_clk.get("sm_mhz") else None)}
+        del sus_timers
+    status = status | rq.rq_workspace_status(state.ws)
+
     if rank == 0:
         step_bytes = state.step_bytes()
         line = {
@@ -550,6 +611,8 @@ def run_ours(args, w):
             "gpu_launches": state.launches_per_step * args.steps,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic,
+                         "launch_kcycles": (avg_res_s * 1e3 * clk["sm_mhz"]
+                                            if clk.get("sm_mhz") else None),
                          "kernel": f"decode_kernel<128,1,{w.bits[0]}> (residual loop)",
                          "algorithmic_bytes_per_launch": bytes_res,
                          "avg_launch_us": avg_res_s * 1e6, "peak_source": peak_kind + " hbm_gbs",
@@ -561,6 +624,12 @@ def run_ours(args, w):
             "workspace_status": status,
             "kernel_source_hash": khash,
         }
+        if sustained is not None:
+            line["sustained"] = sustained
+        if world == 1 and not args.no_workloads:
+            del state, bufs
+            torch.cuda.empty_cache()
+            line["workloads"] = other_workloads(peak, local_rank, args)
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(w)
         print(json.dumps(line), flush=True)
@@ -575,6 +644,11 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the other workloads' block (N=1 only)")
+    ap.add_argument("--sustain-s", type=float, default=3.0,
+                    help="seconds of a second, longer timed region (0: skip)")
+    ap.add_argument("--capacity-steps", type=int, default=3)
     ap.add_argument("--record-traffic", metavar="NCU_CSV",
                     help="write the decode kernel's ncu DRAM bytes into profiles/ and exit")
     args = ap.parse_args(argv)

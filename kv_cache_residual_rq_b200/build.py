@@ -2,9 +2,10 @@
 
     python -m kv_cache_residual_rq_b200.build [--force]
 
-nvcc compiles every .cu under csrc/ for compute_100a/sm_100a and links them
-into kv_cache_residual_rq_b200/librq.so with the CUDA runtime linked
-statically, so the library loads without a CUDA toolkit on the path.
+nvcc compiles every .cu under csrc/ for compute_100a/sm_100a (one process
+per file, in parallel) and links them into kv_cache_residual_rq_b200/librq.so
+with the CUDA runtime linked statically, so the library loads without a CUDA
+toolkit on the path.
 """
 import glob
 import os
@@ -39,21 +40,46 @@ def _stale():
     return max(os.path.getmtime(d) for d in deps) > os.path.getmtime(LIB)
 
 
-def build(force=False, verbose=False):
-    if not force and not _stale():
-        return LIB
+def _nvcc():
     nvcc = os.environ.get("NVCC", "nvcc")
     if os.path.exists("/usr/local/cuda/bin/nvcc") and nvcc == "nvcc":
         nvcc = "/usr/local/cuda/bin/nvcc"
-    cmd = [nvcc, *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-shared", "-o", LIB + ".tmp", *sources()]
-    r = subprocess.run(cmd, capture_output=True, text=True)
-    if r.returncode != 0:
-        sys.stderr.write(r.stdout + r.stderr)
-        raise RuntimeError("nvcc failed building librq.so")
-    if verbose:
-        sys.stderr.write(r.stderr)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    return nvcc
+
+
+def build(force=False, verbose=False, extra_flags=(), lib=LIB):
+    """Compile every translation unit for sm_100a in parallel (one nvcc per
+    .cu file), then link them into `lib`."""
+    import tempfile
+    from concurrent.futures import ThreadPoolExecutor
+    if lib == LIB and not force and not _stale():
+        return lib
+    nvcc = _nvcc()
+    flags = [*NVCC_FLAGS, *extra_flags, "-I", INCLUDE, "-I", CSRC]
+    with tempfile.TemporaryDirectory(prefix="rq_build_") as tmp:
+        def compile_one(src):
+            obj = os.path.join(tmp, os.path.basename(src) + ".o")
+            r = subprocess.run([nvcc, *flags, "-c", "-o", obj, src], capture_output=True,
+                               text=True)
+            return src, obj, r
+        srcs = sources()
+        with ThreadPoolExecutor(max(1, min(len(srcs), os.cpu_count() or 1))) as ex:
+            results = list(ex.map(compile_one, srcs))
+        for src, _, r in results:
+            if r.returncode != 0:
+                sys.stderr.write(r.stdout + r.stderr)
+                raise RuntimeError(f"nvcc failed on {os.path.basename(src)}")
+            if verbose:
+                sys.stderr.write(r.stderr)
+        r = subprocess.run([nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-cudart",
+                            "static", "-shared", "-o", lib + ".tmp",
+                            *[obj for _, obj, _ in results]],
+                           capture_output=True, text=True)
+        if r.returncode != 0:
+            sys.stderr.write(r.stdout + r.stderr)
+            raise RuntimeError("nvcc failed linking " + os.path.basename(lib))
+    os.replace(lib + ".tmp", lib)
+    return lib
 
 
 if __name__ == "__main__":

@@ -15,16 +15,19 @@ group 32, loops 1-3 INT2):
 
 For every batch of the sweep the full cache size is computed; a batch whose
 cache exceeds the budget (120e9 bytes, decimal) is reported as such and not
-run.  A batch within budget is run as a whole decode step, loop-major like a
-looped model (loop 1 over all layers, then loop 2, ...), with two layers'
-worth of cache resident and alternated between consecutive calls: each call
-streams at least 268 MB, more than the 126 MB L2, so the bytes a step moves
-are those of a full 24-layer cache.  Time: CUDA events around whole steps,
-median over --steps after warm-up.  tokens/s = batch / step time.
+run.  A batch within budget allocates its whole 24-layer cache in HBM, fills
+it from the seeded generator (the ResidualQuant cache through the library's
+encoder), and runs whole decode steps over it, loop-major like a looped
+model (loop 1 over all layers, then loop 2, ...); every call also attends
+over the new token's own BF16 K/V of its loop.  The step is attention only
+(no append), the same for both schemes.  Time: CUDA events around whole
+steps, median over --steps after 3 warm-up steps.  tokens/s = batch / step
+time.
 
 Prints one JSON line per (scheme, batch).
 """
 import argparse
+import dataclasses
 import json
 import os
 import sys
@@ -32,8 +35,6 @@ import sys
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
-
-RESIDENT_LAYERS = 2
 
 
 def step_bytes(w, ctx, batch, scheme):
@@ -50,69 +51,95 @@ def step_bytes(w, ctx, batch, scheme):
     return w.layers * (per_layer + q_out)
 
 
-def run_batch(w, ctx, batch, scheme, steps, emit, peak):
+class BF16Step:
+    """Every loop's K/V of every layer in BF16, [loops][layers][K, V][B][Hkv][T][d],
+    with the per-step inputs of DecodeStep (queries, new-token K/V)."""
+
+    def __init__(self, w, device):
+        import torch
+        import kv_cache_residual_rq_b200 as rq
+        from kv_cache_residual_rq_b200 import synth
+        self.w, self.rq = w, rq
+        L, N, B, H, T, d = w.loops, w.layers, w.batch, w.kv_heads, w.ctx, w.head_dim
+        self.shape = rq.make_shape(B, H, T, d, w.group, w.q_heads)
+        self.kv = torch.empty((L, N, 2, B, H, T, d), dtype=torch.bfloat16, device=device)
+        for layer in range(N):
+            for kind in (0, 1):
+                r = synth.reference(w, layer, kind, device)
+                self.kv[L - 1, layer, kind].copy_(r)
+                for l in range(1, L):
+                    self.kv[l - 1, layer, kind].copy_(synth.loop_kv(w, layer, kind, l, r))
+                del r
+            torch.cuda.empty_cache()
+        self.q = torch.stack([torch.stack([synth.query(w, layer, loop, device)
+                                           for layer in range(N)]) for loop in range(1, L + 1)])
+        g = torch.Generator(device=device)
+        g.manual_seed(w.seed * 31 + 7)
+        self.new_kv = torch.randn((L, N, 2, B, H, 1, d), generator=g,
+                                  device=device).to(torch.bfloat16)
+        self.out = torch.empty((L, N, B, w.q_heads, d), dtype=torch.float32, device=device)
+        self.ws = rq.alloc_workspace(self.shape, device)
+        self.ws_bytes = self.ws.numel()
+
+    def cache_bytes(self):
+        return self.kv.numel() * 2
+
+    def run(self, stream, append=False):
+        st = stream.cuda_stream
+        for li in range(self.w.loops):
+            for layer in range(self.w.layers):
+                self.rq.rq_decode_attention_tail(
+                    self.shape, self.q[li, layer], self.kv[li, layer, 0], self.kv[li, layer, 1],
+                    None, None, None, None, 16, self.w.seed, 0.0, self.new_kv[li, layer, 0],
+                    self.new_kv[li, layer, 1], 1, 1, self.out[li, layer], self.ws,
+                    self.ws_bytes, st)
+
+
+def run_batch(w, ctx, batch, scheme, steps, peak, budget):
+    """Allocate and fill the full cache of `batch` sequences, check it against
+    the budget, time whole decode steps.  Returns the result line."""
     import torch
     import kv_cache_residual_rq_b200 as rq
     from kv_cache_residual_rq_b200 import synth
-    dev = torch.device("cuda:0")
-    L = w.loops
-    shape = rq.make_shape(batch, w.kv_heads, ctx, w.head_dim, w.group, w.q_heads)
-    layers = []
-    for layer in range(RESIDENT_LAYERS):
-        ent = {}
-        for kind, name in ((0, "k"), (1, "v")):
-            ref = synth.reference(w, layer, kind, dev, batch=batch, ctx=ctx)
-            loops = [synth.loop_kv(w, layer, kind, l, ref) for l in range(1, L)]
-            if scheme == "bf16":
-                ent[name] = loops + [ref]                    # loop l's own K/V
-            else:
-                codes, scales = rq.encode(loops, ref, list(w.bits), w.group, w.seed)
-                ent[name] = ref
-                ent["c" + name], ent["s" + name] = codes, scales
-            del loops
-        layers.append(ent)
-        torch.cuda.empty_cache()
-    qs = [synth.query(w, 0, li + 1, dev, batch=batch) for li in range(L)]
-    out = torch.empty((batch, w.q_heads, w.head_dim), dtype=torch.float32, device=dev)
-    ws = rq.alloc_workspace(shape, dev)
-
-    def step():
-        for li in range(L):
-            for layer in range(w.layers):
-                e = layers[layer % RESIDENT_LAYERS]
-                if scheme == "bf16":
-                    rq.rq_decode_attention(shape, qs[li], e["k"][li], e["v"][li], None, None,
-                                           None, None, 16, w.seed, 0.0, out, ws)
-                elif li < L - 1:
-                    rq.rq_decode_attention(shape, qs[li], e["k"], e["v"], e["ck"][li],
-                                           e["cv"][li], e["sk"][li], e["sv"][li], w.bits[li],
-                                           w.seed, 0.0, out, ws)
-                else:
-                    rq.rq_decode_attention(shape, qs[li], e["k"], e["v"], None, None, None,
-                                           None, 16, w.seed, 0.0, out, ws)
-
+    from kv_cache_residual_rq_b200.step import DecodeStep
+    dev = torch.device("cuda", torch.cuda.current_device())
+    wb = dataclasses.replace(w, batch=batch, ctx=ctx)
+    torch.cuda.empty_cache()
+    base = torch.cuda.memory_allocated(dev)
+    state = (DecodeStep if scheme == "rq" else BF16Step)(wb, dev)
+    torch.cuda.synchronize(dev)
+    torch.cuda.empty_cache()
+    held = torch.cuda.memory_allocated(dev) - base
+    cache = state.cache_bytes()
+    if cache > budget:
+        raise RuntimeError(f"{scheme} batch {batch}: cache of {cache} bytes exceeds the budget")
+    stream = torch.cuda.current_stream(dev)
     for _ in range(3):
-        step()
+        state.run(stream, append=False)
     times = []
     for _ in range(steps):
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
-        a.record()
-        step()
-        b.record()
-        torch.cuda.synchronize()
+        a.record(stream)
+        state.run(stream, append=False)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
         times.append(a.elapsed_time(b) / 1e3)
-    assert rq.rq_workspace_status(ws) == 0
+    status = rq.rq_workspace_status(state.ws)
+    finite = bool(torch.isfinite(state.out).all().item())
     times.sort()
     t = times[len(times) // 2]
     nb = step_bytes(w, ctx, batch, scheme)
-    emit({"scheme": scheme, "batch": batch, "ctx": ctx, "status": "run",
-          "kv_bytes": batch * synth.kv_bytes_per_sequence(w, ctx, scheme == "rq"),
-          "step_ms": t * 1e3, "tokens_per_s": batch / t, "step_bytes": nb,
-          "gbs": nb / t / 1e9, "frac_hbm": nb / t / 1e9 / peak,
-          "calls_per_step": L * w.layers, "resident_layers": RESIDENT_LAYERS})
-    del layers, qs, out, ws
+    line = {"scheme": scheme, "batch": batch, "ctx": ctx, "status": "run",
+            "kv_bytes": batch * synth.kv_bytes_per_sequence(w, ctx, scheme == "rq"),
+            "cache_bytes_allocated": cache, "device_bytes_held": held,
+            "budget_bytes": budget, "step_ms": t * 1e3, "tokens_per_s": batch / t,
+            "step_bytes": nb, "gbs": nb / t / 1e9, "frac_hbm": nb / t / 1e9 / peak,
+            "calls_per_step": w.loops * w.layers, "layers_resident": w.layers,
+            "workspace_status": status, "outputs_finite": finite}
+    del state
     torch.cuda.empty_cache()
+    return line
 
 
 def plan(w, ctx, batches, budget):
@@ -151,7 +178,7 @@ def main(argv=None):
             emit({"scheme": scheme, "batch": b, "ctx": ctx, "status": "exceeds budget",
                   "kv_bytes": kv})
             continue
-        run_batch(w, ctx, b, scheme, args.steps, emit, peak)
+        emit(run_batch(w, ctx, b, scheme, args.steps, peak, args.budget))
 
 
 if __name__ == "__main__":

@@ -212,3 +212,126 @@ def main(argv=None):
 
 if __name__ == "__main__":
     main()
+
+
+# ---------------------------------------------------------------------------
+# the bench's per-workload block: back-to-back launches with sampled clocks
+# ---------------------------------------------------------------------------
+
+def _back_to_back(fn, stream, target_s, sampler):
+    """Average duration of `fn` launched back to back on `stream` (CUDA events
+    around n launches, n chosen so the timed region lasts about target_s),
+    with the SM clock sampled during the timed region."""
+    import time
+    import torch
+    for _ in range(3):
+        fn()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(3):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    est = a.elapsed_time(b) / 3e3
+    n = int(min(5000, max(10, target_s / max(est, 1e-6))))
+    if sampler is not None:
+        sampler.start()
+        time.sleep(0.25)
+    a.record(stream)
+    for _ in range(n):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    clk = sampler.stop() if sampler is not None else {}
+    return a.elapsed_time(b) / 1e3 / n, n, clk
+
+
+def _entry(name, t, n, clk, nbytes, peak, **extra):
+    mhz = clk.get("sm_mhz")
+    e = {"name": name, "us": round(t * 1e6, 2), "launches": n, "bytes": nbytes,
+         "gbs": round(nbytes / t / 1e9, 1), "frac": round(nbytes / t / 1e9 / peak, 4),
+         "sm_mhz": mhz, "kcycles": round(t * 1e6 * mhz / 1e3, 1) if mhz else None}
+    if clk.get("reasons"):
+        e["reasons"] = clk["reasons"]
+    e.update(extra)
+    return e
+
+
+def bench_workloads(peak, make_sampler, target_s=0.4):
+    """Entries for the bench's `workloads` block: the configured decode calls
+    of the mixed-precision 32K workload (loop 1 INT4, loop 2 INT2, loop 4 BF16)
+    and of the deep-loop grouped-query workload (INT2 loop, BF16 reference),
+    one full layer each (every call streams more than 1 GB, far beyond L2),
+    and rq_encode of the whole 32K prefill (24 layers x K/V x 4 loops in one
+    call, 25.8 GB read).  make_sampler() returns a clock sampler with
+    start()/stop()."""
+    import torch
+    import kv_cache_residual_rq_b200 as rq
+    from kv_cache_residual_rq_b200 import synth
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream(dev)
+    st = stream.cuda_stream
+    out_entries = []
+
+    for w, loops in ((synth.MIXED, (1, 2, None)), (synth.DEEP, (1, None))):
+        refk = synth.reference(w, 0, 0, dev)
+        refv = synth.reference(w, 0, 1, dev)
+        shape = rq.make_shape(w.batch, w.kv_heads, w.ctx, w.head_dim, w.group, w.q_heads)
+        ws = rq.alloc_workspace(shape, dev)
+        out = torch.empty((w.batch, w.q_heads, w.head_dim), dtype=torch.float32, device=dev)
+        per_call = {}
+        for loop in loops:
+            if loop is None:
+                bits, args = 16, (None,) * 4
+                q = synth.query(w, 0, w.loops, dev)
+            else:
+                bits = w.bits[loop - 1]
+                (ck,), (sk,) = rq.encode([synth.loop_kv(w, 0, 0, loop, refk)], refk, [bits],
+                                         w.group, w.seed)
+                (cv,), (sv,) = rq.encode([synth.loop_kv(w, 0, 1, loop, refv)], refv, [bits],
+                                         w.group, w.seed)
+                args = (ck, cv, sk, sv)
+                q = synth.query(w, 0, loop, dev)
+            fn = lambda: rq.rq_decode_attention(shape, q, refk, refv, *args, bits, w.seed, 0.0,
+                                                out, ws, stream=st)
+            t, n, clk = _back_to_back(fn, stream, target_s, make_sampler())
+            per_call[bits] = t
+            label = f"loop {loop} INT{bits}" if loop else f"loop {w.loops} BF16 reference"
+            out_entries.append(_entry(f"{w.name} decode {label}", t, n, clk,
+                                      decode_bytes(w, bits), peak, G=w.G))
+            del args
+            torch.cuda.empty_cache()
+        assert rq.rq_workspace_status(ws) == 0
+        # the configured step from these per-call times: every non-final loop
+        # at its bits, the final loop BF16, over all layers
+        step_s = w.layers * (sum(per_call[b] for b in w.bits) + per_call[16])
+        out_entries[-1]["step_tokens_per_s_from_calls"] = round(w.batch / step_s, 1)
+        del refk, refv, ws, out
+        torch.cuda.empty_cache()
+
+    # the whole 32K prefill encode in one call
+    w = synth.ENCODE
+    N, H, T, d = w.layers, w.kv_heads, w.ctx, w.head_dim
+    rows_batch = N * 2 * w.batch
+    x = torch.empty((w.loops, rows_batch, H, T, d), dtype=torch.bfloat16, device=dev)
+    for layer in range(N):
+        for kind in (0, 1):
+            r = synth.reference(w, layer, kind, dev)
+            part = slice((layer * 2 + kind) * w.batch, (layer * 2 + kind + 1) * w.batch)
+            x[w.loops - 1, part].copy_(r)
+            for l in range(1, w.loops):
+                x[l - 1, part].copy_(synth.loop_kv(w, layer, kind, l, r))
+            del r
+    shape = rq.make_shape(rows_batch, H, T, d, w.group)
+    codes = [rq.alloc_codes(shape, b, dev) for b in w.bits]
+    scales = [rq.alloc_scales(shape, b, dev) for b in w.bits]
+    fn = lambda: rq.rq_encode(shape, list(x[:w.loops - 1]), x[w.loops - 1], list(w.bits),
+                              w.seed, codes, scales, st)
+    t, n, clk = _back_to_back(fn, stream, target_s, make_sampler())
+    nb = encode_bytes(w, rows_batch * H * T)
+    out_entries.append(_entry(f"{w.name} encode (24 layers x K/V x {w.loops} loops, one call)",
+                              t, n, clk, nb, peak, rows=rows_batch * H * T))
+    del x, codes, scales
+    torch.cuda.empty_cache()
+    return out_entries
