@@ -10,7 +10,9 @@ import ctypes
 import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "librq.so")
+# RQ_LIBRARY selects another build of the same library (the bounds-checked
+# librq_bounds.so); default: the in-tree librq.so
+LIB_PATH = os.environ.get("RQ_LIBRARY") or os.path.join(HERE, "librq.so")
 
 RQ_OK = 0
 RQ_ERR_INVALID_ARG = 1

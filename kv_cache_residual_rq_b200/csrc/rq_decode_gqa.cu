@@ -203,11 +203,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
-__device__ __forceinline__ uint32_t bfma2_u(uint32_t a, uint32_t b, uint32_t c) {
-  uint32_t r;
-  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
-  return r;
-}
 __device__ __forceinline__ uint32_t badd2_u(uint32_t a, uint32_t b) {
   uint32_t r;
   asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
@@ -240,46 +235,6 @@ __device__ __forceinline__ void split_f16(float lo, float hi, uint32_t& h, uint3
 }
 
 constexpr uint32_t kMagic = 0x43004300u;   // bf16 128.0 in both halves (mantissa unit 1)
-
-// Levels of the K codes for the B fragment of one k-step (16 dims) of one
-// token: b0 = {l(2q), l(2q+1)}, b1 = {l(2q+8), l(2q+9)}, bf16, exact.  INT2:
-// w0 is the k-step's word (code j at bits 2j); INT4: w0, w1 are its two words
-// (code j at bits 4j of word j / 8).
-template <int BITS>
-__device__ __forceinline__ void k_levels(uint32_t w0, uint32_t w1, int q, uint32_t& b0,
-                                         uint32_t& b1) {
-  if constexpr (BITS == 2) {
-    // lo halves take the code at mantissa bit 1 (value 128 + 2c, level =
-    // v - 131), hi halves at bit 18 = mantissa bit 2 (value 128 + 4c,
-    // level = v/2 - 67); every step is exact in bf16
-    const uint32_t x = w0 >> (4 * q);
-    const uint32_t v0 = ((x << 1) & 0x6u) | ((x << 16) & 0xC0000u) | kMagic;
-    const uint32_t v1 = ((x >> 15) & 0x6u) | (x & 0xC0000u) | kMagic;
-    const uint32_t mul = 0x3F003F80u;   // {1.0, 0.5}
-    const uint32_t add = 0xC286C303u;   // {-131, -67}
-    b0 = bfma2_u(v0, mul, add);
-    b1 = bfma2_u(v1, mul, add);
-  } else {
-    // both halves take the code at mantissa bit 1 (value 128 + 2c, level
-    // 2c - 15 = v - 143)
-    const uint32_t x0 = w0 >> (8 * q);
-    const uint32_t x1 = w1 >> (8 * q);
-    const uint32_t v0 = ((x0 << 1) & 0x1Eu) | ((x0 << 13) & 0x1E0000u) | kMagic;
-    const uint32_t v1 = ((x1 << 1) & 0x1Eu) | ((x1 << 13) & 0x1E0000u) | kMagic;
-    const uint32_t add = 0xC30FC30Fu;   // {-143, -143}
-    b0 = badd2_u(v0, add);
-    b1 = badd2_u(v1, add);
-  }
-}
-
-// INT2 K-residual B fragment with the k permutation of the q~ fragments:
-// register 0 = dims (2q, 2q+8), register 1 = dims (2q+1, 2q+9) of the
-// 16-dim step, each half the exact bf16 value 128 + 2c (code c at mantissa
-// bits 1-2; the codes of a register are 16 bits apart in the packed word).
-__device__ __forceinline__ void k_levels2(uint32_t w, int q, uint32_t& b0, uint32_t& b1) {
-  b0 = (((w << 1) >> (4 * q)) & 0x00060006u) | kMagic;
-  b1 = ((w >> (4 * q + 1)) & 0x00060006u) | kMagic;
-}
 
 template <int D, int G, int BITS, int GROUP, int RB>
 __global__ void __launch_bounds__(kDecodeThreads, 2)
@@ -537,7 +492,7 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
           fa[1] = pack_bf16(qrow[8], qrow[9]);
           if constexpr (BITS == 2) {
             // k positions 2q, 2q+1 | 2q+8, 2q+9 carry dims 2q, 2q+8 | 2q+1, 2q+9,
-            // so the two codes of a B register sit 16 bits apart (k_levels2)
+            // so the two codes of a B register sit 16 bits apart
             split_bf16(cd * trow[0], cd * trow[8], fh[0], fl[0]);
             split_bf16(cd * trow[1], cd * trow[9], fh[1], fl[1]);
             sqj += ((bf16_lo_f(fh[0]) + bf16_lo_f(fl[0])) +
@@ -678,7 +633,6 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
     float cref[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
     float ct[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
     const int tok0[2] = {wtok + 2 * q, wtok + 8 + 2 * q};     // tokens of c0 per tile
-    const int tb[2] = {wtok + g, wtok + 8 + g};               // B-fragment token per tile
     // ldmatrix: matrices (tile 0, dims +0..7), (tile 0, +8..15), (tile 1, ..), (tile 1, ..)
     const int ktr = wtok + ((lane >> 4) & 1) * 8 + r7;
     const int kch = (lane >> 3) & 1;
@@ -794,12 +748,12 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
         }
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
-          const uint32_t* cw = reinterpret_cast<const uint32_t*>(st + C::OFF_CK + tb[nt] * C::CROW);
           uint32_t b0, b1;
           if constexpr (C::LDM2) {
             // codes 2u, 2u+8 | 2u+1, 2u+9 of the word at mantissa bits 1-2:
-            // bf16 128 + 2c, exact (as k_levels2); bit 31 (code 15) is not
-            // among the codes the shifted copy serves
+            // bf16 128 + 2c, exact (the q~ fragments' k permutation puts the
+            // two codes of a B register 16 bits apart); bit 31 (code 15) is
+            // not among the codes the shifted copy serves
             uint32_t w;
             int u;
             if constexpr (GROUP == 64) {
@@ -812,17 +766,13 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
             }
             b0 = (((w << 1) >> (4 * u)) & 0x00060006u) | kMagic;
             b1 = ((w >> (4 * u + 1)) & 0x00060006u) | kMagic;
-          } else if constexpr (C::LDM4) {
+          } else {
+            static_assert(C::LDM4, "residual codes are INT2 or INT4");
             // codes 2h, 2h+4 | 2h+1, 2h+5 at mantissa bits 1-4: bf16 128 + 2c, exact
             const uint32_t w = ck4[2 * ((kk >> 1) & 1) + nt];
             const int h = kk & 1;
             b0 = (((w << 1) >> (8 * h)) & 0x001E001Eu) | kMagic;
             b1 = ((w >> (8 * h + 3)) & 0x001E001Eu) | kMagic;
-          } else if constexpr (BITS == 2) {
-            k_levels2(cw[kk], q, b0, b1);
-          } else {
-            const uint2 w2 = *reinterpret_cast<const uint2*>(cw + 2 * kk);
-            k_levels<4>(w2.x, w2.y, q, b0, b1);
           }
           mma_bf16(ct[nt], ah, b0, b1);
           mma_bf16(ct[nt], al, b0, b1);
@@ -1073,7 +1023,8 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
               mma_bf16(ores[2 * j + i], a, bl0, bl1);
             }
           }
-        } else if constexpr (C::LDM4) {
+        } else {
+          static_assert(C::LDM4, "residual codes are INT2 or INT4");
           // the group's 32-dim chunks by ldmatrix.trans: word = codes of dims
           // 4g .. 4g+3 of the chunk (token 2q low half, 2q+1 high half, code i
           // at bits 4i); m-tile 2 ch has m-rows g, g + 8 = dims 4g, 4g + 1,
@@ -1094,31 +1045,6 @@ decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
               mma_bf16(ores[2 * ch + xy], a, bh0, bh1);
               mma_bf16(ores[2 * ch + xy], a, bl0, bl1);
             }
-          }
-        } else {
-#pragma unroll
-          for (int mt = j * KSG; mt < (j + 1) * KSG; ++mt) {
-            // codes of dims 16mt + g (lo halves) and 16mt + g + 8 (hi halves)
-            uint32_t x[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const uint32_t* cw = reinterpret_cast<const uint32_t*>(st + C::OFF_CV + tk[k] * C::CROW);
-              if constexpr (BITS == 2) {
-                x[k] = ((cw[mt] >> (2 * g)) & 0x00030003u) | kMagic;
-              } else {
-                const uint32_t lo = (cw[2 * mt] >> (4 * g)) & 0xFu;
-                const uint32_t hi = (cw[2 * mt + 1] >> (4 * g)) & 0xFu;
-                x[k] = lo | (hi << 16) | kMagic;
-              }
-            }
-            const uint32_t m128 = 0xC300C300u;   // {-128, -128}
-            uint32_t a[4];
-            a[0] = badd2_u(__byte_perm(x[0], x[1], 0x5410), m128);   // dim g,   tokens 2q, 2q+1
-            a[1] = badd2_u(__byte_perm(x[0], x[1], 0x7632), m128);   // dim g+8
-            a[2] = badd2_u(__byte_perm(x[2], x[3], 0x5410), m128);   // dim g,   tokens 2q+8, 2q+9
-            a[3] = badd2_u(__byte_perm(x[2], x[3], 0x7632), m128);   // dim g+8
-            mma_bf16(ores[mt], a, bh0, bh1);
-            mma_bf16(ores[mt], a, bl0, bl1);
           }
         }
       }

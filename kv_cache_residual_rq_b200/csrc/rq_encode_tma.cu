@@ -38,22 +38,29 @@ __device__ uint32_t g_encode_status;
 
 namespace {
 
-constexpr int kSlots = 6;
 constexpr float kFloorMagic = 12582912.0f;          // 1.5 * 2^23
 constexpr uint32_t kFloorMagicBits = 0x4B400000u;
 constexpr unsigned kFull = 0xffffffffu;
 
+// consumer warps per CTA (+ 1 producer warp) and ring slots
+template <int D>
+constexpr int consumer_warps() { return D == 128 ? 11 : 8; }
+template <int D>
+constexpr int ring_slots() { return D == 128 ? 5 : 6; }
+
 template <int D, int CW>
 struct ECfg {
-  static constexpr int LPR = D / 32;                // lanes per row
+  static constexpr int LPR = D / 64;                // lanes per row, 64 coordinates each
   static constexpr int RPW = 32 / LPR;              // rows per consumer warp
   static constexpr int R = CW * RPW;                // rows per tile
   static constexpr int NBOX = D / 64;               // 64-column boxes per row
   static constexpr int BOX_BYTES = R * 128;
   static constexpr int SLOT_BYTES = NBOX * BOX_BYTES;
+  static constexpr int SLOTS = ring_slots<D>();
   static constexpr int THREADS = (CW + 1) * 32;
-  static constexpr int SMEM = 1024 + kSlots * SLOT_BYTES + 2 * (D / 2) * 4 + 2 * kSlots * 8;
+  static constexpr int SMEM = 1024 + SLOTS * SLOT_BYTES + 2 * (D / 2) * 4 + 2 * SLOTS * 8;
   static_assert(R <= 256, "tensor-copy box is at most 256 rows");
+  static_assert(SMEM <= 232448, "shared memory of one CTA");
 };
 
 struct alignas(64) EncodeTmaParams {
@@ -104,152 +111,48 @@ __device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
   return r;
 }
 
-// 32 bf16 of one lane: row r of the slot, 16-byte chunks c0 .. c0+3 of box b
-template <int D, int CW>
-__device__ __forceinline__ void load_row(const uint8_t* slot, int r, int q, uint32_t (&w)[16]) {
+// The lane's 64 coordinates of row r (q: which half of a 128-wide row), as
+// P[m] = {c_m, c_{m+32}}: chunk c of the row's 128-byte box line holds
+// coordinates 8c .. 8c+7, so P[m].x comes from chunk m/8 and P[m].y from
+// chunk m/8 + 4.  For each coordinate i: out_i = a_i * b_i + add_i, a the
+// slot's bf16 row, b the lane's bf16 sign words (word k = coordinates 2k,
+// 2k+1), add the float2 addends in the same layout (or zero).
+template <int D, int CW, bool ADD>
+__device__ __forceinline__ void row_fma(const uint8_t* slot, const uint32_t* signs, int r, int q,
+                                        const float2 (&add)[32], float2 (&P)[32]) {
   using C = ECfg<D, CW>;
-  const int b = (D == 128) ? (q >> 1) : 0;
-  const int c0 = (D == 128) ? (q & 1) * 4 : q * 4;
-  const uint8_t* rp = slot + b * C::BOX_BYTES + r * 128;
+  const uint8_t* rp = slot + q * C::BOX_BYTES + r * 128;
+  const uint4* s4 = reinterpret_cast<const uint4*>(signs + 32 * q);
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint4 v = *reinterpret_cast<const uint4*>(rp + (((c0 + i) ^ (r & 7)) << 4));
-    w[4 * i] = v.x;
-    w[4 * i + 1] = v.y;
-    w[4 * i + 2] = v.z;
-    w[4 * i + 3] = v.w;
+  for (int c = 0; c < 8; ++c) {
+    const uint4 v = *reinterpret_cast<const uint4*>(rp + ((c ^ (r & 7)) << 4));
+    const uint4 dd = s4[c];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    const uint32_t dw[4] = {dd.x, dd.y, dd.z, dd.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int i = 8 * c + 2 * k + h;            // coordinate within the lane's 64
+        const int m = i & 31;
+        const float a = ADD ? ((i < 32) ? add[m].x : add[m].y) : 0.0f;
+        const float o = h ? fma_bf16<1>(w[k], dw[k], a) : fma_bf16<0>(w[k], dw[k], a);
+        if (i < 32) P[m].x = o; else P[m].y = o;
+      }
+    }
   }
 }
 
-// One quantisation pass of a lane's 32 rotated coordinates P[m] = {y_m,
-// y_{m+16}} with step 1/(2 inv): packed code words, <y,l> in the fixed order
-// (fma chains over coordinates 0..15 and 16..31, the two runs added; the
-// partner lane's block added for groups of 64) and <l,l> (exact).
-template <int BITS, int GROUP, int RPW, bool CLAMP, bool WANT_LV = false>
-__device__ __forceinline__ void quant_pass(const float2 (&P)[16], float inv, uint32_t (&w)[BITS],
-                                           float& dot_out, float& nrm_out,
-                                           float2* lv_out = nullptr) {
-  const float2 inv2 = make_float2(inv, inv);
-  const float2 mg = make_float2(kFloorMagic, kFloorMagic);
-  const float2 two = make_float2(2.0f, 2.0f), one = make_float2(1.0f, 1.0f);
-  constexpr float lo = kFloorMagic - (float)(1 << (BITS - 1));
-  constexpr float hi = kFloorMagic + (float)((1 << (BITS - 1)) - 1);
-  float2 dot = make_float2(0.0f, 0.0f), nrm = make_float2(0.0f, 0.0f);
+// The lane's 64 coordinates (signs applied) rotated in place: Walsh-Hadamard
+// strides ascending, each butterfly (a + b, a - b) one rounded operation --
+// strides 1..16 as packed pairs, 32 inside each pair, 64 (head_dim 128) with
+// the partner lane -- then x c_d.
+template <int D, int RPW>
+__device__ __forceinline__ void rotate64(float2 (&P)[32], int q) {
 #pragma unroll
-  for (int k = 0; k < BITS; ++k) w[k] = 0;
+  for (int h = 1; h < 32; h <<= 1) {
 #pragma unroll
-  for (int m = 0; m < 16; ++m) {
-    const float2 u = __fmul2_rn(P[m], inv2);
-    float2 t = __fadd2_rd(u, mg);                   // 1.5*2^23 + floor(u), exact
-    if constexpr (CLAMP) {
-      t.x = fminf(fmaxf(t.x, lo), hi);
-      t.y = fminf(fmaxf(t.y, lo), hi);
-    }
-    if constexpr (BITS == 2) {
-      w[0] += __float_as_uint(t.x) << (2 * m);
-      w[1] += __float_as_uint(t.y) << (2 * m);
-    } else if constexpr (BITS == 4) {
-      w[m / 8] += __float_as_uint(t.x) << (4 * (m % 8));
-      w[2 + m / 8] += __float_as_uint(t.y) << (4 * (m % 8));
-    } else {
-      w[m / 4] += __float_as_uint(t.x) << (8 * (m % 4));
-      w[4 + m / 4] += __float_as_uint(t.y) << (8 * (m % 4));
-    }
-    const float2 fl = fsub2(t, mg);                 // floor(u)
-    const float2 lv = __ffma2_rn(fl, two, one);     // level 2 floor(u) + 1 = 2c - (2^b - 1)
-    if constexpr (WANT_LV) lv_out[m] = lv;
-    dot = __ffma2_rn(P[m], lv, dot);
-    if constexpr (BITS != 2) nrm = __ffma2_rn(lv, lv, nrm);
-  }
-  // every field received (0x4B400000 + floor(u)); code c = floor(u) + 2^(b-1)
-  constexpr uint32_t kOff = kFloorMagicBits - (1u << (BITS - 1));
-  constexpr uint32_t kSpread =
-      BITS == 2 ? 0x55555555u : (BITS == 4 ? 0x11111111u : 0x01010101u);
-#pragma unroll
-  for (int k = 0; k < BITS; ++k) w[k] -= kOff * kSpread;
-  float d = dot.x + dot.y, n;
-  if constexpr (BITS == 2) {
-    // <l, l> = 32 + 8 * (number of outer levels +-3, i.e. codes 0 and 3,
-    // whose two bits are equal): an exact integer either way
-    const uint32_t e = __popc(~(w[0] ^ (w[0] >> 1)) & 0x55555555u) +
-                       __popc(~(w[1] ^ (w[1] >> 1)) & 0x55555555u);
-    n = (float)(32u + 8u * e);
-  } else {
-    n = nrm.x + nrm.y;
-  }
-  if (GROUP == 64) {
-    d += __shfl_xor_sync(kFull, d, RPW);
-    n += __shfl_xor_sync(kFull, n, RPW);
-  }
-  dot_out = d;
-  nrm_out = n;
-}
-
-// codes and scale of one lane's 32 rotated coordinates: the absmax step,
-// then `iters` least-squares refits (nearest level of the current scale,
-// then the scale refitted); a group whose scale is below FLT_MIN keeps its
-// codes.  The loop runs the same number of times in every lane.
-template <int BITS, int GROUP, int RPW, bool WANT_Z = false>
-__device__ __forceinline__ void quantize_store(const float2 (&P)[16], uint32_t* codes_row,
-                                               uint16_t* scales_row, int q, bool valid,
-                                               int iters, float2* z = nullptr) {
-  float amax = 0.0f;
-#pragma unroll
-  for (int m = 0; m < 16; ++m) amax = fmax3_abs(amax, P[m].x, P[m].y);
-  if (GROUP == 64) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, RPW));
-  constexpr float outer = (float)(1 << (BITS - 1)) - 0.5f;
-  const float inv = (amax < 1.17549435e-38f) ? 0.0f : __fdiv_rn(outer, amax);
-  uint32_t w[BITS];
-  float d, n;
-  quant_pass<BITS, GROUP, RPW, false, WANT_Z>(P, inv, w, d, n, z);
-  float s = d / n;                                  // least-squares scale
-  for (int k = 0; k < iters; ++k) {
-    const bool live = s >= 1.17549435e-38f;
-    uint32_t w2[BITS];
-    float d2, n2;
-    quant_pass<BITS, GROUP, RPW, true>(P, live ? __fdiv_rn(0.5f, s) : 0.0f, w2, d2, n2);
-    if (live) {
-#pragma unroll
-      for (int j = 0; j < BITS; ++j) w[j] = w2[j];
-      s = d2 / n2;
-    }
-  }
-  s = fminf(fmaxf(s, -65504.0f), 65504.0f);
-  const __half s16 = __float2half_rn(s);
-  if constexpr (WANT_Z) {
-    // the reconstructed rotated row s16 * l (exact: 11 x 9 significant bits)
-    const float sf = __half2float(s16);
-    const float2 s2 = make_float2(sf, sf);
-#pragma unroll
-    for (int m = 0; m < 16; ++m) z[m] = __fmul2_rn(z[m], s2);
-  }
-  if (!valid) return;
-  if constexpr (BITS == 2) {
-    *reinterpret_cast<uint2*>(codes_row + 2 * q) = make_uint2(w[0], w[1]);
-  } else if constexpr (BITS == 4) {
-    *reinterpret_cast<uint4*>(codes_row + 4 * q) = make_uint4(w[0], w[1], w[2], w[3]);
-  } else {
-    uint4* o = reinterpret_cast<uint4*>(codes_row + 8 * q);
-    o[0] = make_uint4(w[0], w[1], w[2], w[3]);
-    o[1] = make_uint4(w[4], w[5], w[6], w[7]);
-  }
-  if (GROUP == 32)
-    scales_row[q] = __half_as_ushort(s16);
-  else if (!(q & 1))
-    scales_row[q >> 1] = __half_as_ushort(s16);
-}
-
-// the row's 32 coordinates of this lane, v (signs applied), rotated in place
-// into P[m] = {y_m, y_{m+16}}: Walsh-Hadamard strides ascending, a butterfly
-// (a + b, a - b), then x c_d
-template <int D, int LPR, int RPW>
-__device__ __forceinline__ void rotate_lane(const float (&v)[32], float2 (&P)[16], int q) {
-#pragma unroll
-  for (int m = 0; m < 16; ++m) P[m] = make_float2(v[m], v[m + 16]);
-#pragma unroll
-  for (int h = 1; h < 16; h <<= 1) {
-#pragma unroll
-    for (int m = 0; m < 16; ++m) {
+    for (int m = 0; m < 32; ++m) {
       if (!(m & h)) {
         const float2 a = P[m], b = P[m + h];
         P[m] = __fadd2_rn(a, b);
@@ -258,28 +161,190 @@ __device__ __forceinline__ void rotate_lane(const float (&v)[32], float2 (&P)[16
     }
   }
 #pragma unroll
-  for (int m = 0; m < 16; ++m) {
+  for (int m = 0; m < 32; ++m) {
     const float a = P[m].x, b = P[m].y;
     P[m] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
   }
-#pragma unroll
-  for (int k = 1; k < LPR; k <<= 1) {
+  if constexpr (D == 128) {
     // the lower partner keeps a + b, the upper one a - b (fma with +-1 is
     // exactly one rounded add or subtract)
-    const float sg = (q & k) ? -1.0f : 1.0f;
+    const float sg = q ? -1.0f : 1.0f;
     const float2 sg2 = make_float2(sg, sg);
 #pragma unroll
-    for (int m = 0; m < 16; ++m) {
+    for (int m = 0; m < 32; ++m) {
       float2 o;
-      o.x = __shfl_xor_sync(kFull, P[m].x, RPW * k);
-      o.y = __shfl_xor_sync(kFull, P[m].y, RPW * k);
+      o.x = __shfl_xor_sync(kFull, P[m].x, RPW);
+      o.y = __shfl_xor_sync(kFull, P[m].y, RPW);
       P[m] = __ffma2_rn(sg2, P[m], o);
     }
   }
   const float cd = rot_scale<D>();
   const float2 cd2 = make_float2(cd, cd);
 #pragma unroll
-  for (int m = 0; m < 16; ++m) P[m] = __fmul2_rn(P[m], cd2);
+  for (int m = 0; m < 32; ++m) P[m] = __fmul2_rn(P[m], cd2);
+}
+
+// One quantisation pass over the lane's two 32-coordinate blocks, A = P[].x
+// and B = P[].y, with steps 1/(2 inv.x), 1/(2 inv.y): code words (A's BITS
+// words, then B's), <y,l> and <l,l> of each block (.x, .y).
+// FIXED: <y,l> in the fixed order (fma chains over coordinates 0..15 and
+// 16..31 of a block, the two runs added), which the least-squares refits and
+// the compressed reference need bit for bit.  Otherwise the sum runs as four
+// interleaved chains (the plain encode's scale is an fp16 rounding of it, so
+// its order is free).  Code words are integer sums: any order.
+template <int BITS, bool CLAMP, bool FIXED, bool WANT_LV = false>
+__device__ __forceinline__ void quant_pass(const float2 (&P)[32], float2 inv2,
+                                           uint32_t (&w)[2 * BITS], float2& dot_out,
+                                           float2& nrm_out, float2* lv_out = nullptr) {
+  constexpr int PER = 32 / BITS;                    // codes per word
+  const float2 mg = make_float2(kFloorMagic, kFloorMagic);
+  const float2 two = make_float2(2.0f, 2.0f), one = make_float2(1.0f, 1.0f);
+  constexpr float lo = kFloorMagic - (float)(1 << (BITS - 1));
+  constexpr float hi = kFloorMagic + (float)((1 << (BITS - 1)) - 1);
+  constexpr int NC = FIXED ? 2 : 4;                 // independent chains
+  float2 dot[NC], nrm[NC];
+#pragma unroll
+  for (int c = 0; c < NC; ++c) {
+    dot[c] = make_float2(0.0f, 0.0f);
+    nrm[c] = make_float2(0.0f, 0.0f);
+  }
+#pragma unroll
+  for (int k = 0; k < 2 * BITS; ++k) w[k] = 0;
+#pragma unroll
+  for (int m = 0; m < 32; ++m) {
+    const int c = FIXED ? m / 16 : m % 4;           // FIXED: chain = run of 16
+    const float2 u = __fmul2_rn(P[m], inv2);
+    float2 t = __fadd2_rd(u, mg);                   // 1.5*2^23 + floor(u), exact
+    if constexpr (CLAMP) {
+      t.x = fminf(fmaxf(t.x, lo), hi);
+      t.y = fminf(fmaxf(t.y, lo), hi);
+    }
+    w[m / PER] += __float_as_uint(t.x) << (BITS * (m % PER));
+    w[BITS + m / PER] += __float_as_uint(t.y) << (BITS * (m % PER));
+    const float2 fl = fsub2(t, mg);                 // floor(u)
+    const float2 lv = __ffma2_rn(fl, two, one);     // level 2 floor(u) + 1 = 2c - (2^b - 1)
+    if constexpr (WANT_LV) lv_out[m] = lv;
+    dot[c] = __ffma2_rn(P[m], lv, dot[c]);
+    if constexpr (BITS != 2) nrm[c] = __ffma2_rn(lv, lv, nrm[c]);
+  }
+  // every field received (0x4B400000 + floor(u)); code c = floor(u) + 2^(b-1)
+  constexpr uint32_t kOff = kFloorMagicBits - (1u << (BITS - 1));
+  constexpr uint32_t kSpread =
+      BITS == 2 ? 0x55555555u : (BITS == 4 ? 0x11111111u : 0x01010101u);
+#pragma unroll
+  for (int k = 0; k < 2 * BITS; ++k) w[k] -= kOff * kSpread;
+  if constexpr (FIXED) {
+    dot_out = __fadd2_rn(dot[0], dot[1]);           // run 0 + run 1 of each block
+  } else {
+    dot_out = __fadd2_rn(__fadd2_rn(dot[0], dot[1]), __fadd2_rn(dot[2], dot[3]));
+  }
+  if constexpr (BITS == 2) {
+    // <l, l> = 32 + 8 * (number of outer levels +-3, i.e. codes 0 and 3,
+    // whose two bits are equal): an exact integer
+    const uint32_t ea = __popc(~(w[0] ^ (w[0] >> 1)) & 0x55555555u) +
+                        __popc(~(w[1] ^ (w[1] >> 1)) & 0x55555555u);
+    const uint32_t eb = __popc(~(w[2] ^ (w[2] >> 1)) & 0x55555555u) +
+                        __popc(~(w[3] ^ (w[3] >> 1)) & 0x55555555u);
+    nrm_out = make_float2((float)(32u + 8u * ea), (float)(32u + 8u * eb));
+  } else {
+    // integers below 2^24 in every partial sum: exact in any order
+    float2 n = nrm[0];
+#pragma unroll
+    for (int c = 1; c < NC; ++c) n = __fadd2_rn(n, nrm[c]);
+    nrm_out = n;
+  }
+}
+
+__device__ __forceinline__ float2 f2(float x) { return make_float2(x, x); }
+
+// Codes and scales of the lane's 64 rotated coordinates: blocks A (P[].x)
+// and B (P[].y) are one 32-wide scale group each, or together one group of
+// 64.  The absmax step, then `iters` least-squares refits (nearest level of
+// the current scale, then the scale refitted); a group whose scale is below
+// FLT_MIN keeps its codes.  WANT_Z: z = s16 * l (the rotated reconstruction).
+template <int BITS, int GROUP, bool FIXED, bool WANT_Z = false>
+__device__ __forceinline__ void quantize_store(const float2 (&P)[32], uint32_t* codes_row,
+                                               uint16_t* scales_row, int q, bool valid,
+                                               int iters, float2* z = nullptr) {
+  // absmax of each block as four interleaved chains (max is exact in any order)
+  float ax[4], ay[4];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    ax[c] = fmax3_abs(0.0f, P[2 * c].x, P[2 * c + 1].x);
+    ay[c] = fmax3_abs(0.0f, P[2 * c].y, P[2 * c + 1].y);
+  }
+#pragma unroll
+  for (int m = 8; m < 32; m += 2) {
+    const int c = (m / 2) % 4;
+    ax[c] = fmax3_abs(ax[c], P[m].x, P[m + 1].x);
+    ay[c] = fmax3_abs(ay[c], P[m].y, P[m + 1].y);
+  }
+  float amx = fmaxf(fmaxf(ax[0], ax[1]), fmaxf(ax[2], ax[3]));
+  float amy = fmaxf(fmaxf(ay[0], ay[1]), fmaxf(ay[2], ay[3]));
+  if constexpr (GROUP == 64) amx = amy = fmaxf(amx, amy);
+  constexpr float outer = (float)(1 << (BITS - 1)) - 0.5f;
+  float2 inv;
+  inv.x = (amx < 1.17549435e-38f) ? 0.0f : __fdiv_rn(outer, amx);
+  inv.y = (GROUP == 64) ? inv.x : ((amy < 1.17549435e-38f) ? 0.0f : __fdiv_rn(outer, amy));
+  uint32_t w[2 * BITS];
+  float2 d, n;
+  quant_pass<BITS, false, FIXED, WANT_Z>(P, inv, w, d, n, z);
+  if constexpr (GROUP == 64) {
+    d = f2(d.x + d.y);                              // block A + block B
+    n = f2(n.x + n.y);
+  }
+  // least-squares scale: IEEE division where later steps depend on its bits
+  // (refits, the compressed reference); else only its fp16 rounding is kept
+  float2 s;
+  if constexpr (FIXED) {
+    s.x = d.x / n.x;
+    s.y = (GROUP == 64) ? s.x : d.y / n.y;
+  } else {
+    s.x = __fdividef(d.x, n.x);
+    s.y = (GROUP == 64) ? s.x : __fdividef(d.y, n.y);
+  }
+  for (int k = 0; k < iters; ++k) {
+    const bool lx = s.x >= 1.17549435e-38f, ly = s.y >= 1.17549435e-38f;
+    float2 inv2;
+    inv2.x = lx ? __fdiv_rn(0.5f, s.x) : 0.0f;
+    inv2.y = (GROUP == 64) ? inv2.x : (ly ? __fdiv_rn(0.5f, s.y) : 0.0f);
+    uint32_t w2[2 * BITS];
+    float2 d2, n2;
+    quant_pass<BITS, true, true>(P, inv2, w2, d2, n2);
+    if constexpr (GROUP == 64) {
+      d2 = f2(d2.x + d2.y);
+      n2 = f2(n2.x + n2.y);
+    }
+    if (lx) {
+#pragma unroll
+      for (int j = 0; j < BITS; ++j) w[j] = w2[j];
+      s.x = d2.x / n2.x;
+    }
+    if (ly) {
+#pragma unroll
+      for (int j = BITS; j < 2 * BITS; ++j) w[j] = w2[j];
+      s.y = (GROUP == 64) ? s.x : d2.y / n2.y;
+    }
+  }
+  s.x = fminf(fmaxf(s.x, -65504.0f), 65504.0f);
+  s.y = fminf(fmaxf(s.y, -65504.0f), 65504.0f);
+  const __half hx = __float2half_rn(s.x), hy = __float2half_rn(s.y);
+  if constexpr (WANT_Z) {
+    // the reconstructed rotated block s16 * l (exact: 11 x 9 significant bits)
+    const float2 s2 = make_float2(__half2float(hx), __half2float(hy));
+#pragma unroll
+    for (int m = 0; m < 32; ++m) z[m] = __fmul2_rn(z[m], s2);
+  }
+  if (!valid) return;
+  uint4* o = reinterpret_cast<uint4*>(codes_row + 2 * BITS * q);
+#pragma unroll
+  for (int k = 0; k < 2 * BITS / 4; ++k)
+    o[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+  if constexpr (GROUP == 32)
+    *reinterpret_cast<uint32_t*>(scales_row + 2 * q) =
+        (uint32_t)__half_as_ushort(hx) | ((uint32_t)__half_as_ushort(hy) << 16);
+  else
+    scales_row[q] = __half_as_ushort(hx);
 }
 
 // MODE 0: BF16 reference, no refits; 1: BF16 reference with least-squares
@@ -289,14 +354,16 @@ template <int D, int GROUP, int CW, int MODE>
 __global__ void __launch_bounds__(ECfg<D, CW>::THREADS, 1)
 encode_tma_kernel(const __grid_constant__ EncodeTmaParams tp) {
   using C = ECfg<D, CW>;
+  constexpr int SLOTS = C::SLOTS;
+  constexpr bool FIXED = (MODE != 0);
   const int iters = (MODE == 0) ? 0 : tp.p.refine_iters;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint32_t* dtab = reinterpret_cast<uint32_t*>(ring + kSlots * C::SLOT_BYTES);  // D_i as bf16 pairs
+  uint32_t* dtab = reinterpret_cast<uint32_t*>(ring + SLOTS * C::SLOT_BYTES);  // D_i as bf16 pairs
   uint32_t* ndtab = dtab + D / 2;                                            // -D_i
   uint64_t* full = reinterpret_cast<uint64_t*>(ndtab + D / 2);
-  uint64_t* empty = full + kSlots;
+  uint64_t* empty = full + SLOTS;
   const EncodeParams& p = tp.p;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_allow_next();
@@ -308,7 +375,7 @@ encode_tma_kernel(const __grid_constant__ EncodeTmaParams tp) {
     ndtab[i] = dtab[i] ^ 0x80008000u;
   }
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kSlots; ++s) {
+    for (int s = 0; s < SLOTS; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], CW);
     }
@@ -325,8 +392,8 @@ encode_tma_kernel(const __grid_constant__ EncodeTmaParams tp) {
     bool ok = true;
     for (int t = blockIdx.x; ok && t < tp.n_tiles; t += gridDim.x) {
       for (int j = 0; j < per_tile; ++j, ++it) {
-        const int s = (int)(it % kSlots);
-        if (it >= kSlots && !mbar_wait_bounded(&empty[s], (uint32_t)((it / kSlots - 1) & 1))) {
+        const int s = (int)(it % SLOTS);
+        if (it >= SLOTS && !mbar_wait_bounded(&empty[s], (uint32_t)((it / SLOTS - 1) & 1))) {
           atomicOr(&g_encode_status, 1u);
           ok = false;
           break;
@@ -339,15 +406,15 @@ encode_tma_kernel(const __grid_constant__ EncodeTmaParams tp) {
       }
     }
     // do not leave while copies into this CTA's shared memory are in flight
-    for (long long k = (it > kSlots ? it - kSlots : 0); k < it; ++k)
-      if (!mbar_wait_bounded(&full[k % kSlots], (uint32_t)((k / kSlots) & 1)))
+    for (long long k = (it > SLOTS ? it - SLOTS : 0); k < it; ++k)
+      if (!mbar_wait_bounded(&full[k % SLOTS], (uint32_t)((k / SLOTS) & 1)))
         atomicOr(&g_encode_status, 2u);
     return;
   }
 
   // ---------------- consumers ----------------
   const int rw = lane % C::RPW;          // row within the warp
-  const int q = lane / C::RPW;           // which 32 coordinates of the row
+  const int q = lane / C::RPW;           // which 64 coordinates of the row
   const int r = warp * C::RPW + rw;      // row within the tile
   long long it = 0;
   for (int t = blockIdx.x; t < tp.n_tiles; t += gridDim.x) {
@@ -358,131 +425,83 @@ encode_tma_kernel(const __grid_constant__ EncodeTmaParams tp) {
     long long row = 0;
     const bool valid = idx < p.n_rows && enc_dst_row(p, hd, tok, row);
 
-    // reference: -D_i ref_i, kept for every loop of these rows
-    int s = (int)(it % kSlots);
-    if (!mbar_wait_bounded(&full[s], (uint32_t)((it / kSlots) & 1))) {
+    // reference: -D_i ref_i (BF16 reference), kept for every loop of these
+    // rows; or, compressed reference, the rotated reference is quantised
+    // (its codes stored) and zr holds its reconstruction s16 * l, which is
+    // subtracted from every loop's rotated row
+    int s = (int)(it % SLOTS);
+    if (!mbar_wait_bounded(&full[s], (uint32_t)((it / SLOTS) & 1))) {
       atomicOr(&g_encode_status, 4u);
       return;
     }
-    uint32_t wv[16];
-    load_row<D, CW>(ring + s * C::SLOT_BYTES, r, q, wv);
+    const uint8_t* slot = ring + s * C::SLOT_BYTES;
+    if (valid && p.ref_out) {
+      const uint8_t* rp = slot + q * C::BOX_BYTES + r * 128;
+      uint4* o = reinterpret_cast<uint4*>(p.ref_out + (size_t)row * D + q * 64);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) o[c] = *reinterpret_cast<const uint4*>(rp + ((c ^ (r & 7)) << 4));
+    }
+    float2 zr[32];
+    if constexpr (MODE != 2) {
+      row_fma<D, CW, false>(slot, ndtab, r, q, zr, zr);
+    } else {
+      float2 P[32];
+      row_fma<D, CW, false>(slot, dtab, r, q, zr, P);         // D_i ref_i, exact
+      rotate64<D, C::RPW>(P, q);
+      if (p.ref_bits == 8)
+        quantize_store<8, GROUP, true, true>(P, p.ref_codes + (size_t)row * (D / 4),
+                                             p.ref_scales + (size_t)row * (D / GROUP), q,
+                                             valid, 0, zr);
+      else
+        quantize_store<4, GROUP, true, true>(P, p.ref_codes + (size_t)row * (D / 8),
+                                             p.ref_scales + (size_t)row * (D / GROUP), q,
+                                             valid, 0, zr);
+    }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
     ++it;
-    if (valid && p.ref_out) {
-      uint4* o = reinterpret_cast<uint4*>(p.ref_out + (size_t)row * D + q * 32);
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        o[i] = make_uint4(wv[4 * i], wv[4 * i + 1], wv[4 * i + 2], wv[4 * i + 3]);
-    }
-    // BF16 reference: -D_i ref_i for the residual fma of every loop.
-    // Compressed reference: the rotated reference is quantised (its codes
-    // stored) and zr holds its reconstruction s16 * l, subtracted from every
-    // loop's rotated row.
-    float zr[32];
-    constexpr bool cr = (MODE == 2);
-    if constexpr (!cr) {
-      const uint4* nd4 = reinterpret_cast<const uint4*>(ndtab + q * 16);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint4 nd = nd4[i];
-        const uint32_t ndw[4] = {nd.x, nd.y, nd.z, nd.w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          zr[8 * i + 2 * k] = fma_bf16<0>(wv[4 * i + k], ndw[k], 0.0f);
-          zr[8 * i + 2 * k + 1] = fma_bf16<1>(wv[4 * i + k], ndw[k], 0.0f);
-        }
-      }
-    } else {
-      float v[32];
-      const uint4* d4 = reinterpret_cast<const uint4*>(dtab + q * 16);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint4 dd = d4[i];
-        const uint32_t dw[4] = {dd.x, dd.y, dd.z, dd.w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          v[8 * i + 2 * k] = fma_bf16<0>(wv[4 * i + k], dw[k], 0.0f);        // D_i ref_i
-          v[8 * i + 2 * k + 1] = fma_bf16<1>(wv[4 * i + k], dw[k], 0.0f);
-        }
-      }
-      float2 P[16], Z[16];
-      rotate_lane<D, C::LPR, C::RPW>(v, P, q);
-      if (p.ref_bits == 8)
-        quantize_store<8, GROUP, C::RPW, true>(P, p.ref_codes + (size_t)row * (D / 4),
-                                               p.ref_scales + (size_t)row * (D / GROUP), q,
-                                               valid, 0, Z);
-      else
-        quantize_store<4, GROUP, C::RPW, true>(P, p.ref_codes + (size_t)row * (D / 8),
-                                               p.ref_scales + (size_t)row * (D / GROUP), q,
-                                               valid, 0, Z);
-#pragma unroll
-      for (int m = 0; m < 16; ++m) {
-        zr[m] = Z[m].x;
-        zr[m + 16] = Z[m].y;
-      }
-    }
 
     for (int j = 0; j < tp.n_active; ++j) {
-      s = (int)(it % kSlots);
-      if (!mbar_wait_bounded(&full[s], (uint32_t)((it / kSlots) & 1))) {
+      s = (int)(it % SLOTS);
+      if (!mbar_wait_bounded(&full[s], (uint32_t)((it / SLOTS) & 1))) {
         atomicOr(&g_encode_status, 4u);
         return;
       }
-      load_row<D, CW>(ring + s * C::SLOT_BYTES, r, q, wv);
+      // BF16 reference: y = D_i x_i + (-D_i ref_i), one rounding, then rotated.
+      // Compressed reference: D_i x_i (exact), rotated, then e = RN(y - zr).
+      float2 P[32];
+      row_fma<D, CW, MODE != 2>(ring + s * C::SLOT_BYTES, dtab, r, q, zr, P);
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
       ++it;
-
-      // BF16 reference: y = D_i x_i + (-D_i ref_i), one rounding, then rotated.
-      // Compressed reference: D_i x_i (exact), rotated, then e = RN(y - zr).
-      float v[32];
-      {
-        const uint4* d4 = reinterpret_cast<const uint4*>(dtab + q * 16);
+      rotate64<D, C::RPW>(P, q);
+      if constexpr (MODE == 2) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint4 dd = d4[i];
-          const uint32_t dw[4] = {dd.x, dd.y, dd.z, dd.w};
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const float a0 = cr ? 0.0f : zr[8 * i + 2 * k];
-            const float a1 = cr ? 0.0f : zr[8 * i + 2 * k + 1];
-            v[8 * i + 2 * k] = fma_bf16<0>(wv[4 * i + k], dw[k], a0);
-            v[8 * i + 2 * k + 1] = fma_bf16<1>(wv[4 * i + k], dw[k], a1);
-          }
-        }
+        for (int m = 0; m < 32; ++m) P[m] = fsub2(P[m], zr[m]);
       }
-      float2 P[16];
-      rotate_lane<D, C::LPR, C::RPW>(v, P, q);
-      if constexpr (cr) {
-#pragma unroll
-        for (int m = 0; m < 16; ++m) P[m] = fsub2(P[m], make_float2(zr[m], zr[m + 16]));
-      }
-
       const int l = tp.active[j];
       if (p.bits[l] == 2)
-        quantize_store<2, GROUP, C::RPW>(P, p.codes[l] + (size_t)row * (D / 16),
-                                         p.scales[l] + (size_t)row * (D / GROUP), q, valid,
-                                         iters);
+        quantize_store<2, GROUP, FIXED>(P, p.codes[l] + (size_t)row * (D / 16),
+                                        p.scales[l] + (size_t)row * (D / GROUP), q, valid,
+                                        iters);
       else
-        quantize_store<4, GROUP, C::RPW>(P, p.codes[l] + (size_t)row * (D / 8),
-                                         p.scales[l] + (size_t)row * (D / GROUP), q, valid,
-                                         iters);
+        quantize_store<4, GROUP, FIXED>(P, p.codes[l] + (size_t)row * (D / 8),
+                                        p.scales[l] + (size_t)row * (D / GROUP), q, valid,
+                                        iters);
     }
   }
 }
 
-constexpr int kConsumerWarps = 15;   // + 1 producer = 16 warps, 4 per scheduler
-
 template <int D, int GROUP, int MODE>
 cudaError_t launch_tm(const EncodeTmaParams& tp, int num_sms, cudaStream_t stream) {
-  using C = ECfg<D, kConsumerWarps>;
-  cudaError_t e = cudaFuncSetAttribute(encode_tma_kernel<D, GROUP, kConsumerWarps, MODE>,
+  constexpr int CW = consumer_warps<D>();
+  using C = ECfg<D, CW>;
+  cudaError_t e = cudaFuncSetAttribute(encode_tma_kernel<D, GROUP, CW, MODE>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   const int grid = tp.n_tiles < num_sms ? tp.n_tiles : num_sms;
-  return launch_pdl(encode_tma_kernel<D, GROUP, kConsumerWarps, MODE>, (unsigned)grid,
-                    C::THREADS, C::SMEM, stream, tp);
+  return launch_pdl(encode_tma_kernel<D, GROUP, CW, MODE>, (unsigned)grid, C::THREADS, C::SMEM,
+                    stream, tp);
 }
 
 template <int D, int GROUP>
@@ -495,7 +514,7 @@ cudaError_t launch_t(const EncodeTmaParams& tp, int num_sms, cudaStream_t stream
 }  // namespace
 
 int encode_tma_rows_per_tile(int head_dim) {
-  return head_dim == 128 ? ECfg<128, kConsumerWarps>::R : ECfg<64, kConsumerWarps>::R;
+  return head_dim == 128 ? ECfg<128, consumer_warps<128>()>::R : ECfg<64, consumer_warps<64>()>::R;
 }
 
 cudaError_t launch_encode_tma(int head_dim, int group, const EncodeParams& p, int num_sms,

@@ -1,6 +1,6 @@
 """Per-workload kernel timings (one layer each), for the measured tables.
 
-    python -m kv_cache_residual_rq_b200.measure [--workloads a,b] [--reps N]
+    python -m kv_cache_residual_rq_b200.measure [--workloads a,b] [--reps N] [--gqa-variants]
 
 For every workload: the decode call of each distinct loop kind (residual INT2,
 INT4, BF16 reference) over one full layer, and rq_encode of one layer's K
@@ -199,15 +199,54 @@ def measure(w, reps, peak, emit):
         assert rq.rq_workspace_status(wsv) == 0
 
 
+def measure_gqa_variants(reps, peak, emit):
+    """Deep-loop shapes (B 32, Hkv 8, G 4, T 8192, d 128) with the residual
+    formats the configured workload does not use: INT4 with 64- and 32-dim
+    scale groups, INT2 with 32-dim groups (the configured call is INT2 with
+    64-dim groups)."""
+    import dataclasses
+    import torch
+    import kv_cache_residual_rq_b200 as rq
+    from kv_cache_residual_rq_b200 import synth
+    dev = torch.device("cuda:0")
+    base = synth.DEEP
+    for bits, group in ((4, 64), (4, 32), (2, 32)):
+        w = dataclasses.replace(base, group=group, bits=(bits,) * (base.loops - 1))
+        refk = synth.reference(w, 0, 0, dev)
+        refv = synth.reference(w, 0, 1, dev)
+        q = synth.query(w, 0, 1, dev)
+        (ck,), (sk,) = rq.encode([synth.loop_kv(w, 0, 0, 1, refk)], refk, [bits], group, w.seed)
+        (cv,), (sv,) = rq.encode([synth.loop_kv(w, 0, 1, 1, refv)], refv, [bits], group, w.seed)
+        shape = rq.make_shape(w.batch, w.kv_heads, w.ctx, w.head_dim, group, w.q_heads)
+        ws = rq.alloc_workspace(shape, dev)
+        out = torch.empty((w.batch, w.q_heads, w.head_dim), dtype=torch.float32, device=dev)
+        fn = lambda: rq.rq_decode_attention(shape, q, refk, refv, ck, cv, sk, sv, bits, w.seed,
+                                            0.0, out, ws)
+        t = _time(fn, reps, None)
+        nb = decode_bytes(w, bits)
+        emit({"workload": f"{w.name} shapes", "kernel": f"decode bits={bits} group={group}",
+              "G": w.G, "us": t * 1e6, "bytes": nb, "gbs": nb / t / 1e9,
+              "frac": nb / t / 1e9 / peak})
+        assert rq.rq_workspace_status(ws) == 0
+        del refk, refv, ck, cv, sk, sv, ws, out
+        torch.cuda.empty_cache()
+
+
 def main(argv=None):
     from kv_cache_residual_rq_b200 import synth
     ap = argparse.ArgumentParser()
     ap.add_argument("--workloads", default=",".join(w.name for w in synth.WORKLOADS))
     ap.add_argument("--reps", type=int, default=20)
+    ap.add_argument("--gqa-variants", action="store_true",
+                    help="also time the deep-loop shapes with INT4 residuals (64- and 32-dim "
+                         "groups) and INT2 with 32-dim groups")
     args = ap.parse_args(argv)
     peak = _peak()
-    for name in args.workloads.split(","):
-        measure(synth.BY_NAME[name], args.reps, peak, lambda d: print(json.dumps(d), flush=True))
+    emit = lambda d: print(json.dumps(d), flush=True)
+    for name in args.workloads.split(",") if args.workloads else []:
+        measure(synth.BY_NAME[name], args.reps, peak, emit)
+    if args.gqa_variants:
+        measure_gqa_variants(args.reps, peak, emit)
 
 
 if __name__ == "__main__":

@@ -68,11 +68,15 @@ def encode_layer(w, layer, kind, device="cuda", batch=None, ctx=None):
 
 
 def compare_encode_rows(w, ref, loops, codes, scales, rows):
-    """rows: flat row indices into [B*Hkv*T]."""
+    """rows: flat row indices into [B*Hkv*T].  Codes must equal the oracle's
+    bit for bit, scales within one fp16 step.  Returns the oracle's tie count
+    per quantised loop (coordinates with y*inv exactly an integer, which the
+    floor rule sends to the upper level); the rows holding a tie are checked
+    on their own as well, so agreement at every counted tie is explicit."""
     d = w.head_dim
     rows_t = torch.as_tensor(rows, device=ref.device)
     r_flat = ref.reshape(-1, d)
-    ties = 0
+    ties = []
     for l, bits in enumerate(w.bits):
         if bits == 16:
             assert codes[l] is None and scales[l] is None
@@ -80,13 +84,19 @@ def compare_encode_rows(w, ref, loops, codes, scales, rows):
         x_flat = loops[l].reshape(-1, d)
         gw = codes_view(codes[l], (r_flat.shape[0],), d, bits)[rows_t]
         gs = scales_view(scales[l], (r_flat.shape[0],), d, w.group)[rows_t]
-        want_w, want_s, t = oracle.encode_rows_f32(u16(x_flat[rows_t]), u16(r_flat[rows_t]), bits,
-                                                   w.group, w.seed)
-        ties += t
+        xs, rs = u16(x_flat[rows_t]), u16(r_flat[rows_t])
+        want_w, want_s, t = oracle.encode_rows_f32(xs, rs, bits, w.group, w.seed)
         got_w = gw.cpu().numpy().view(np.uint32)
         mism = (got_w != want_w)
         assert not mism.any(), f"loop {l + 1}: {mism.sum()} code words differ"
         check_scales(gs.cpu().numpy().view(np.uint16), want_s)
+        if t:
+            tie_rows = [i for i in range(len(rows))
+                        if oracle.encode_rows_f32(xs[i:i + 1], rs[i:i + 1], bits, w.group,
+                                                  w.seed)[2]]
+            assert tie_rows and np.array_equal(got_w[tie_rows], want_w[tie_rows]), \
+                f"loop {l + 1}: codes differ at a tie"
+        ties.append(t)
     return ties
 
 
@@ -96,7 +106,8 @@ def test_encode_tiny_full():
         ref, loops, codes, scales = encode_layer(w, 0, kind)
         n = ref.numel() // w.head_dim
         ties = compare_encode_rows(w, ref, loops, codes, scales, np.arange(n))
-        print(f"tiny kind={kind}: {n} rows x {w.loops - 1} loops bit-exact, ties={ties}")
+        print(f"ties tiny kind {kind}: {n} rows x {w.loops - 1} loops bit-exact, "
+              f"ties per loop {ties}")
 
 
 @pytest.mark.parametrize("name", ["ouro1.4b_decode", "mixed_precision_32k", "deep_loop_gqa",
@@ -109,7 +120,8 @@ def test_encode_full_size_sampled(name):
     rng = np.random.default_rng(7)
     rows = np.unique(np.concatenate([rng.integers(0, n, 3000), [0, 1, n - 1]]))
     ties = compare_encode_rows(w, ref, loops, codes, scales, rows)
-    print(f"{name}: {rows.size} sampled rows bit-exact, ties={ties}")
+    print(f"ties {name} layer {layer} V: {rows.size} sampled rows x {len(ties)} loops "
+          f"bit-exact, ties per loop {ties}")
 
 
 @pytest.mark.parametrize("d,group,bits", [(64, 64, 2), (128, 64, 4), (64, 32, 4)])
@@ -221,6 +233,9 @@ def test_decode_full_size_sampled(name, loops):
     (128, 32, 4, 2, 20000, 1, 1),      # one head spread over many CTAs
     (64, 64, 2, 2, 300, 2, 2),         # INT2, 64-dim groups (ldmatrix code words), d 64
     (128, 64, 8, 2, 777, 1, 3),        # the same at d 128, G = 8, ragged
+    (64, 32, 4, 4, 257, 2, 1),         # INT4, 32-dim groups at d 64: two chunks per row
+    (128, 32, 8, 4, 777, 1, 3),        # INT4, 32-dim groups, G = 8, ragged
+    (64, 32, 2, 2, 191, 3, 2),         # INT2, 32-dim groups at d 64 (word exchange)
 ])
 def test_decode_edge_shapes(d, group, G, bits, ctx, batch, hkv):
     bl = (bits, 16) if bits != 16 else (2, 16)
