@@ -487,10 +487,12 @@ def run_ours(args, w):
     torch.cuda.synchronize(device)
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.nvtx.range_push(f"{w.name} timed steps")
     t_start.record(stream)
     for _ in range(args.steps):
         state.run(stream, timers)
     t_end.record(stream)
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize(device)
     barrier()
     clk = clocks.stop()
@@ -558,7 +560,9 @@ def run_ours(args, w):
     torch.cuda.synchronize(device)
     e_start = torch.cuda.Event(enable_timing=True)
     e_end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.nvtx.range_push(f"{w.name} end-to-end steps")
     e2e_loop(args.steps, e_start, e_end)
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize(device)
     barrier()
     e_elapsed, e_tokens = aggregate(e_start.elapsed_time(e_end) / 1e3, w.batch * args.steps)
@@ -576,10 +580,12 @@ def run_ours(args, w):
         torch.cuda.synchronize(device)
         s_start = torch.cuda.Event(enable_timing=True)
         s_end = torch.cuda.Event(enable_timing=True)
+        torch.cuda.nvtx.range_push(f"{w.name} sustained steps")
         s_start.record(stream)
         for _ in range(n_sus):
             state.run(stream, sus_timers)
         s_end.record(stream)
+        torch.cuda.nvtx.range_pop()
         torch.cuda.synchronize(device)
         barrier()
         s_clk = clocks.stop()

@@ -483,7 +483,11 @@ rq_status rq_reconstruct_cr(const rq_shape *shape, const uint32_t *ref_codes,
  * rq_encode_at since the last read ran clean; non-zero means a bounded wait
  * inside the encoder ran out (bit 0: the copy engine's slot was never
  * released, bit 1: a copy never completed, bit 2: a consumer's tile never
- * arrived) and the codes written since then are invalid. */
+ * arrived) and the codes written since then are invalid.  Bit 3 (value 8)
+ * exists only in the bounds-checked build of this library (librq_bounds.so,
+ * compiled with RQ_BOUNDS_CHECK): an encoder or reconstruction kernel found
+ * an index outside its buffer and skipped that access.  The reconstruction
+ * entry points report here too. */
 rq_status rq_encode_take_status(uint32_t *host_status);
 
 /* Copies the workspace's device status word to *host_status (blocking read
@@ -492,7 +496,10 @@ rq_status rq_encode_take_status(uint32_t *host_status);
  * be zeroed again: bits 1, 2, 8 a bounded wait inside a kernel ran out, 4 a
  * partial-record slot out of range, 16 a sequence length clamped to the
  * capacity, 32 a page id outside the pool, 64 a compressed-reference weight
- * out of range.  This is the only entry point that synchronises. */
+ * out of range; 128, only in the bounds-checked build (librq_bounds.so), an
+ * index a decode kernel computed fell outside its buffer or shared-memory
+ * area and that access was skipped.  This is the only entry point that
+ * synchronises. */
 rq_status rq_workspace_status(const void *workspace, size_t workspace_bytes,
                               uint32_t *host_status, void *stream);
 

@@ -16,6 +16,9 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "librq.so")
+# the same library with every computed index checked before its access
+# (-DRQ_BOUNDS_CHECK; a failed check raises a status bit, nothing traps)
+LIB_BOUNDS = os.path.join(HERE, "librq_bounds.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -32,12 +35,12 @@ def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _stale():
-    if not os.path.exists(LIB):
+def _stale(lib=LIB):
+    if not os.path.exists(lib):
         return True
     deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")) \
         + glob.glob(os.path.join(INCLUDE, "*.h"))
-    return max(os.path.getmtime(d) for d in deps) > os.path.getmtime(LIB)
+    return max(os.path.getmtime(d) for d in deps) > os.path.getmtime(lib)
 
 
 def _nvcc():
@@ -47,12 +50,15 @@ def _nvcc():
     return nvcc
 
 
-def build(force=False, verbose=False, extra_flags=(), lib=LIB):
+def build(force=False, verbose=False, bounds=False):
     """Compile every translation unit for sm_100a in parallel (one nvcc per
-    .cu file), then link them into `lib`."""
+    .cu file), then link them into librq.so (bounds: librq_bounds.so, built
+    with -DRQ_BOUNDS_CHECK)."""
     import tempfile
     from concurrent.futures import ThreadPoolExecutor
-    if lib == LIB and not force and not _stale():
+    lib = LIB_BOUNDS if bounds else LIB
+    extra_flags = ("-DRQ_BOUNDS_CHECK",) if bounds else ()
+    if not force and not _stale(lib):
         return lib
     nvcc = _nvcc()
     flags = [*NVCC_FLAGS, *extra_flags, "-I", INCLUDE, "-I", CSRC]
@@ -83,4 +89,5 @@ def build(force=False, verbose=False, extra_flags=(), lib=LIB):
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv,
+                bounds="--bounds" in sys.argv))

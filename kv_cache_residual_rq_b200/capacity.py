@@ -117,6 +117,7 @@ def run_batch(w, ctx, batch, scheme, steps, peak, budget):
     for _ in range(3):
         state.run(stream, append=False)
     times = []
+    torch.cuda.nvtx.range_push(f"{w.name} capacity {scheme} batch {batch}")
     for _ in range(steps):
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
@@ -125,6 +126,7 @@ def run_batch(w, ctx, batch, scheme, steps, peak, budget):
         b.record(stream)
         torch.cuda.synchronize(dev)
         times.append(a.elapsed_time(b) / 1e3)
+    torch.cuda.nvtx.range_pop()
     status = rq.rq_workspace_status(state.ws)
     finite = bool(torch.isfinite(state.out).all().item())
     times.sort()

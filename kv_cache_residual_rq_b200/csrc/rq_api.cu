@@ -35,6 +35,17 @@ bool shape_ok(const rq_shape* s, bool need_ctx) {
   return supported_dims(s->head_dim, s->group);
 }
 
+// Extents and status word every encoder launch carries (the bounds-checked
+// build tests its indices against them); false if the status word's device
+// address is not available.
+bool finish_encode_params(EncodeParams& p, const rq_shape& s) {
+  const long long heads = (long long)s.batch * s.kv_heads;
+  p.n_src_rows = heads * p.src_pitch;
+  p.n_dst_rows = p.page_table ? (long long)p.n_pages * s.kv_heads * 64 : heads * p.dst_pitch;
+  p.status = encode_status_ptr();
+  return p.status != nullptr;
+}
+
 bool decode_shape_ok(const rq_shape* s) {
   if (!shape_ok(s, true)) return false;
   if (s->q_heads < s->kv_heads || s->q_heads % s->kv_heads) return false;
@@ -178,6 +189,7 @@ rq_status rq_encode_at_ex(const rq_shape* shape, int src_pitch, int src_offset,
   p.dst_offset = dst_offset;
   p.n_rows = (long long)shape->batch * shape->kv_heads * shape->ctx;
   if (p.n_rows == 0 || (active == 0 && !ref_out)) return RQ_OK;
+  if (!finish_encode_params(p, *shape)) return RQ_ERR_CUDA;
   const int sms = device_sm_count();
   if (sms <= 0) return RQ_ERR_CUDA;
   const bool contiguous = src_pitch == shape->ctx && src_offset == 0 &&
@@ -235,6 +247,7 @@ rq_status rq_encode_cr_at(const rq_shape* shape, int dst_pitch, int dst_offset,
   p.n_rows = (long long)shape->batch * shape->kv_heads * shape->ctx;
   if (p.n_rows == 0) return RQ_OK;
   if (p.n_rows > kEncodeTmaMaxRows) return RQ_ERR_UNSUPPORTED;
+  if (!finish_encode_params(p, *shape)) return RQ_ERR_CUDA;
   const int sms = device_sm_count();
   if (sms <= 0) return RQ_ERR_CUDA;
   cudaError_t e = launch_encode_tma(shape->head_dim, shape->group, p, sms,
@@ -290,6 +303,7 @@ rq_status rq_encode_paged(const rq_shape* shape, const uint16_t* const* kv_loops
   p.src_offset = 0;
   p.n_rows = (long long)shape->batch * shape->kv_heads * shape->ctx;
   if (p.n_rows == 0 || (active == 0 && !ref_out)) return RQ_OK;
+  if (!finish_encode_params(p, *shape)) return RQ_ERR_CUDA;
   const int sms = device_sm_count();
   if (sms <= 0) return RQ_ERR_CUDA;
   cudaError_t e = p.n_rows <= kEncodeTmaMaxRows
@@ -555,6 +569,8 @@ rq_status rq_reconstruct(const rq_shape* shape, const uint16_t* ref, const uint3
   p.out_bf16 = out_bf16 ? 1 : 0;
   p.seed = seed;
   if (p.n_rows == 0) return RQ_OK;
+  p.status = encode_status_ptr();
+  if (!p.status) return RQ_ERR_CUDA;
   const int sms = device_sm_count();
   if (sms <= 0) return RQ_ERR_CUDA;
   cudaError_t e = launch_reconstruct(shape->head_dim, shape->group, bits, p, sms,
@@ -589,6 +605,8 @@ rq_status rq_reconstruct_cr(const rq_shape* shape, const uint32_t* ref_codes,
   p.out_bf16 = out_bf16 ? 1 : 0;
   p.seed = seed;
   if (p.n_rows == 0) return RQ_OK;
+  p.status = encode_status_ptr();
+  if (!p.status) return RQ_ERR_CUDA;
   const int sms = device_sm_count();
   if (sms <= 0) return RQ_ERR_CUDA;
   cudaError_t e = launch_reconstruct_cr(shape->head_dim, shape->group, ref_bits, bits, p, sms,

@@ -270,6 +270,15 @@ decode_kernel(const DecodeParams p) {
     const size_t start = row * SB;
     return (uint32_t)(((start + (size_t)n * SB + 15) & ~(size_t)15) - (start & ~(size_t)15));
   };
+  // scale bytes a stage holds (per array), for the bounds-checked build
+  constexpr int SCAP = C::RES ? C::SC_BYTES : (RB != 0 ? C::RSC_BYTES : 0);
+  // a tile's copies stay inside the call's arrays and the stage
+  auto copies_in_bounds = [&](size_t row, int n) {
+    const size_t lo = (row * SB) & ~(size_t)15;
+    const uint32_t nb = sc_bytes_ref(row, n);
+    return tile_in_bounds(p, row, n, lo, nb, SB) &&
+           RQ_IN_BOUNDS(SCAP == 0 || (int)nb <= SCAP, p.status, kStatusBounds);
+  };
 
   // ========================= producer warp ================================
   if (warp == kConsumerWarps) {
@@ -299,7 +308,8 @@ decode_kernel(const DecodeParams p) {
         const int n = page_ok ? tc.n() : 0;
         if (p.page_table) stage_row[s] = page_ok ? (unsigned long long)row : kBadRow;
         unsigned char* st = ring + s * C::STAGE_BYTES;
-        if (n <= 0) {                   // the empty tile of an empty sequence
+        if (n <= 0 || !copies_in_bounds(row, n)) {   // the empty tile of an empty sequence
+          if (n > 0 && p.page_table) stage_row[s] = kBadRow;
           mbar_arrive(&full_bar[s]);
           ++issued;
           continue;
@@ -354,8 +364,11 @@ decode_kernel(const DecodeParams p) {
     const int hh = e / (G * D / 8), rem = e % (G * D / 8);
     const long long hd = h_first + hh;
     const int b = (int)(hd / p.kv_heads), h = (int)(hd % p.kv_heads);
-    reinterpret_cast<uint4*>(qpre)[e] =
-        reinterpret_cast<const uint4*>(p.q + ((size_t)b * p.q_heads + (size_t)h * G) * D)[rem];
+    if (RQ_IN_BOUNDS(hd >= 0 && hd < (long long)p.batch * p.kv_heads &&
+                         (size_t)h * G + G <= (size_t)p.q_heads,
+                     p.status, kStatusBounds))
+      reinterpret_cast<uint4*>(qpre)[e] =
+          reinterpret_cast<const uint4*>(p.q + ((size_t)b * p.q_heads + (size_t)h * G) * D)[rem];
   }
 
   const int li = lane % LPT;          // lane within its token
@@ -866,6 +879,15 @@ decode_kernel(const DecodeParams p) {
       const unsigned long long r = stage_row[s];   // written before the stage's arrive
       if (r == kBadRow) n = 0;
       else row = (size_t)r;
+    }
+    if (!aborted && n > 0) {
+      const unsigned char* st = ring + s * C::STAGE_BYTES;
+      const int sc_off = (int)((row * SB) & 15);
+      const int grp = dim0 / p.group;
+      // the consumers' stage reads: token rows < n, scales of n tokens
+      if (!RQ_IN_BOUNDS(n <= TILE && (SCAP == 0 || sc_off + n * SB <= SCAP), p.status,
+                        kStatusBounds))
+        n = 0;
     }
     if (!aborted && n > 0) {
       const unsigned char* st = ring + s * C::STAGE_BYTES;

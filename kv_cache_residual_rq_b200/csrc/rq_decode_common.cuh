@@ -83,6 +83,7 @@ struct TileCursor {
 // Paged caches: the page id of the cursor's tile (read ahead by the
 // producer), and the row of a page id already read.
 __device__ __forceinline__ int tile_page(const DecodeParams& p, const TileCursor& c) {
+  if (!RQ_IN_BOUNDS(c.b < p.batch && c.j < p.max_pages, p.status, kStatusBounds)) return -1;
   return p.page_table[(size_t)c.b * p.max_pages + c.j];
 }
 __device__ __forceinline__ bool tile_row_page(const DecodeParams& p, const TileCursor& c,
@@ -102,6 +103,25 @@ __device__ __forceinline__ bool tile_row(const DecodeParams& p, const TileCursor
     return true;
   }
   return tile_row_page(p, c, tile_page(p, c), row);
+}
+
+// Rows of the call's K/V, code and scale arrays: heads * ctx_pitch for dense
+// caches, the pool's n_pages * kv_heads * 64 for paged ones.
+__device__ __forceinline__ size_t call_rows(const DecodeParams& p) {
+  return p.page_table ? (size_t)p.n_pages * p.kv_heads * kDecodeTile
+                      : (size_t)p.batch * p.kv_heads * p.ctx_pitch;
+}
+
+// A tile's copies stay inside the call's arrays: tokens [row, row + n) and
+// the 16-byte-aligned scale bytes [sc_lo, sc_lo + sc_bytes) of arrays of
+// call_rows(p) rows of sb scale bytes each (sizes rounded up to 16 bytes).
+__device__ __forceinline__ bool tile_in_bounds(const DecodeParams& p, size_t row, int n,
+                                               size_t sc_lo, uint32_t sc_bytes, int sb) {
+  const size_t rows = call_rows(p);
+  const size_t sc_total = (rows * (size_t)sb + 15) / 16 * 16;
+  return RQ_IN_BOUNDS(n >= 0 && n <= kDecodeTile && row + (size_t)n <= rows &&
+                          sc_lo + sc_bytes <= sc_total,
+                      p.status, kStatusBounds);
 }
 
 // A stage's row as the producer resolved it (paged caches), kBadRow for a
@@ -130,6 +150,8 @@ __device__ __forceinline__ bool plan_cta(const DecodeParams& p, int cta, int* sc
     split.ctas = p.ctas;
   } else {
     const int tid = threadIdx.x;
+    // the scan writes batch + 1 ints of scratch (sized for kVarlenMaxBatch + 1)
+    if (!RQ_IN_BOUNDS(p.batch <= kVarlenMaxBatch, p.status, kStatusBounds)) return false;
     if (tid < 32) {
       // exclusive prefix of per-head tile counts over the sequences
       const int per = (p.batch + 31) / 32;
@@ -228,6 +250,10 @@ __device__ __forceinline__ void load_rotate_queries(const DecodeParams& p, long 
   const int b = (int)(hd / p.kv_heads);
   const int h = (int)(hd % p.kv_heads);
   const int warp = tid >> 5, lane = tid & 31;
+  // rows b * q_heads + h * G + r of q: inside the call's batch * q_heads rows
+  const bool hd_ok = qrows || RQ_IN_BOUNDS(hd >= 0 && hd < (long long)p.batch * p.kv_heads &&
+                                               (size_t)h * G + G <= (size_t)p.q_heads,
+                                           p.status, kStatusBounds);
   named_bar_sync(1, kConsumerThreads);          // previous users of the buffers done
   const uint16_t* qbase = qrows ? qrows : p.q + ((size_t)b * p.q_heads + (size_t)h * G) * D;
   for (int r = warp; r < G; r += kConsumerWarps) {
@@ -235,7 +261,7 @@ __device__ __forceinline__ void load_rotate_queries(const DecodeParams& p, long 
     float v[E];
 #pragma unroll
     for (int k = 0; k < E; ++k) {
-      const float x = __uint_as_float((uint32_t)qr[k] << 16);
+      const float x = hd_ok ? __uint_as_float((uint32_t)qr[k] << 16) : 0.0f;
       qs[r * D + lane * E + k] = x;
       v[k] = flip_sign(x, sign_bit(p.seed, lane * E + k));
     }
@@ -271,6 +297,14 @@ __device__ __forceinline__ void finish_head(const DecodeParams& p, long long hd,
   if (j < 0 || j >= p.max_contrib || ncontrib > p.max_contrib) {
     if (tid == 0) flag_error(p.status, 4u);
     return;
+  }
+  // head hd's records and counter, its output rows, its tail tokens and the
+  // tail scratch (G * n_tail floats of the merge area)
+  {
+    const bool ok = hd >= 0 && hd < (long long)p.batch * p.kv_heads &&
+                    (size_t)h * G + G <= (size_t)p.q_heads && p.n_tail >= 0 &&
+                    p.n_tail <= RQ_MAX_TAIL && (p.n_tail == 0 || p.n_tail <= p.tail_pitch);
+    if (!RQ_IN_BOUNDS(ok, p.status, kStatusBounds)) return;
   }
   float* recs = p.records + (size_t)hd * p.max_contrib * G * (4 + 2 * D);
   // per query row: the warps' common max and each warp's weight, once

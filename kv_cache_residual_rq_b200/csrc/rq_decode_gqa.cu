@@ -1,1149 +1,9 @@
-// rq_decode_gqa.cu -- ResidualQuant decode attention for grouped queries
-// (G = q_heads / kv_heads in {2, 4, 8}) on the sm_100a tensor cores.
-//
-// Method: "ResidualQuant: KV Cache Quantization for Looped Transformers with
-// 2-Bit Residuals", Abstract -- decode rebuilds each non-final loop's K/V
-// from the BF16 final-loop reference plus the loop's rotated low-bit residual.
-//
-// With G query rows per kv head every K/V tile is shared by G rows, so the
-// four products of the fused attention are small dense contractions and go to
-// the tensor cores (mma.sync m16n8k16, fp32 accumulation), per warp and per
-// 16 tokens of a 64-token tile:
-//   S_ref = Q  K^T              (K from shared memory, ldmatrix)
-//   S_res = Q~ L_K^T            per scale group, then x s^K
-//   O_ref^T += V^T P^T          (V via ldmatrix.trans)
-//   O_res^T += C_V^T (P s^V)^T
-// all in bf16 x bf16 with fp32 accumulation.  L_K are the levels
-// 2c - (2^b - 1) and C_V the codes c, small integers that bf16 holds exactly,
-// built from the packed words in registers; q~, P and P s^V, which are not
-// bf16 values, are split into a bf16 high part and a bf16 remainder and
-// multiplied twice, so they keep ~16 significant bits and bf16's range.
-// sum_t p s (2c - (2^b-1)) = 2 (C_V^T (P s)^T) - (2^b - 1) sum_t p s is
-// completed when the warp flushes.  Rows beyond G are zero and their weights
-// are forced to zero.
-//
-// Compressed INT8 / INT4 reference (same page, the reference loop itself
-// stored as rotated codes): the reference term is one more quantised term in
-// the rotated domain, s_ref <q~, l_ref> for the scores and sum_t p s_ref l_ref
-// for the values, l_ref = 2c - (2^b - 1).  Its codes enter f16 MMAs as the
-// exact subnormals c 2^-24 -- the code in the low mantissa bits: one byte
-// permute per two INT8 codes, one shift and one mask per two INT4 codes, no
-// offset to cancel -- against q~ scaled by a power of two per row and split
-// into f16 high and remainder parts (scores), or against the weights p s_ref
-// split into f16 parts after a lazily updated power of two keeps them in
-// f16's range (values); the 2^24 returns with the scales, once per scale
-// group (scores) or when the warp flushes (values).  The reference rows (d or
-// d/2 bytes) arrive swizzled; the k order of the q~ fragments and the m-row
-// order of the value accumulators follow the codes' positions in the 32-bit
-// ldmatrix words.
-//
-// The reference K/V tiles (BF16 rows, or code rows) arrive by TMA
-// tensor copies with the swizzle of their line width (conflict-free
-// ldmatrix); codes and scales by plain bulk copies, as in the single-query
-// kernel.  The work split, the partial records and the
-// last-arriving-CTA merge with the single inverse rotation are shared with it
-// (rq_decode_common.cuh).  Every mbarrier wait is bounded.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-#include <cuda_bf16.h>
-
-#include "rq_decode_common.cuh"
+// rq_decode_gqa.cu -- host entry of the grouped-query decode kernel
+// (rq_decode_gqa.cuh): tensor maps of the call's reference rows, then the
+// launch of the instance for its head size and reference type.
+#include "rq_decode_gqa.cuh"
 
 namespace rq {
-namespace {
-
-struct alignas(64) GqaParams {
-  CUtensorMap tmap_k;        // reference K viewed as [rows][d] bf16, box 64 x 64, swizzle 128B
-  CUtensorMap tmap_v;
-  DecodeParams p;
-};
-
-template <int D, int G, int BITS, int GROUP, int RB>
-struct GCfg {
-  static constexpr int TILE = kDecodeTile;                 // 64 tokens
-  static constexpr int WTOK = TILE / kConsumerWarps;       // 16 tokens per warp
-  static constexpr bool RES = (BITS != 16);
-  // INT2 residual: ldmatrix reads the code rows directly.  With 64-dim scale
-  // groups a 16-byte row chunk is exactly one group; with 32-dim groups it
-  // holds two, and lanes exchange words (one shuffle) so that every k-step
-  // and every m-tile stays inside one group.
-  static constexpr bool LDM2 = (BITS == 2);
-  // INT4 residual: a 16-byte row chunk (32 dims) always lies inside one scale
-  // group; ldmatrix words of eight codes, no exchange needed
-  static constexpr bool LDM4 = (BITS == 4);
-  static constexpr int NCH = D / 64;                        // 64-dim chunks per row
-  static constexpr bool CR = (RB == 8);                    // INT8 compressed reference
-  static constexpr bool CR4 = (RB == 4);                   // INT4 compressed reference
-  static constexpr bool CRX = (RB != 0);                   // either
-  static constexpr int RROW = CRX ? D * RB / 8 : 0;        // reference code bytes per token
-  // f16 operands of the reference codes: the exact subnormals c 2^-24 (the
-  // code in the low mantissa bits, no offset).  A sum acc over those operands
-  // gives the level sum  sum w (2c - (2^RB - 1)) = 2^25 acc - (2^RB - 1) sum w.
-  static constexpr float CSCALE = 33554432.0f;                        // 2^25
-  static constexpr float LOFF = (float)((1 << RB) - 1);
-  static constexpr int NBOX = D / 64;                      // 64-column boxes per row
-  static constexpr int BOX_BYTES = 64 * 128;               // 64 rows x 128 B
-  // one K or V reference tile: BF16 boxes, or the INT8 code rows (D bytes each)
-  static constexpr int REF_TILE_BYTES = CRX ? TILE * RROW : NBOX * BOX_BYTES;
-  static constexpr int KT = D / 16;                        // k-steps of 16 dims
-  static constexpr int CROW = RES ? D * BITS / 8 : 0;      // code bytes per token
-  static constexpr int CWORDS = CROW / 4;
-  static constexpr int SC_BYTES = RES ? TILE * (2 * D / 32) + 32 : 0;
-  static constexpr int RSC_BYTES = CRX ? TILE * (2 * D / 32) + 32 : 0;  // reference scales
-  static constexpr int OFF_K = 0;
-  static constexpr int OFF_V = OFF_K + REF_TILE_BYTES;
-  static constexpr int OFF_CK = OFF_V + REF_TILE_BYTES;
-  static constexpr int OFF_CV = OFF_CK + TILE * CROW;
-  static constexpr int OFF_SK = OFF_CV + TILE * CROW;
-  static constexpr int OFF_SV = OFF_SK + SC_BYTES;
-  static constexpr int OFF_RSK = OFF_SV + SC_BYTES;
-  static constexpr int OFF_RSV = OFF_RSK + RSC_BYTES;
-  static constexpr int STAGE_BYTES = (OFF_RSV + RSC_BYTES + 1023) / 1024 * 1024;
-  static constexpr int STAGES = 2;
-  static constexpr int RING_BYTES = STAGES * STAGE_BYTES;
-  static constexpr int MERGE_FLOATS = kConsumerWarps * G * (2 + 2 * D);
-  static constexpr int QBUF_FLOATS = 2 * G * D;
-  static constexpr int NG = D / GROUP;                      // scale groups per token
-  static constexpr int KSG = GROUP / 16;                   // k-steps per scale group
-  static constexpr int SB = 2 * NG;                        // scale bytes per token
-  // per warp, row and scale group: sum of p s^V (and of p s_ref^V)
-  static constexpr int WSUM_FLOATS = kConsumerWarps * G * NG * (CRX ? 2 : 1);
-  // q, q~ high, q~ remainder (bf16); with a compressed reference also
-  // q~ 2^E high, remainder (f16, k-permuted for the reference's codes)
-  static constexpr int QFRAG_WORDS = (CRX ? 5 : 3) * KT * 32 * 2;
-  // INT2: per (row, scale group) sum of the q~ fragments' values (offset of
-  // the 128 + 2c operands); compressed reference: the same for the f16
-  // fragments (the levels' 2^b - 1) and per row 2^-E; even count to keep the
-  // barriers 8-byte aligned
-  static constexpr int SQ_FLOATS = (G * NG * (CRX ? 2 : 1) + (CRX ? G : 0) + 1) / 2 * 2;
-  static constexpr int SMEM_BYTES = 1024 /* base alignment slack */ + RING_BYTES +
-                                    4 * (MERGE_FLOATS + QBUF_FLOATS + WSUM_FLOATS +
-                                         QFRAG_WORDS + SQ_FLOATS) +
-                                    2 * STAGES * 8 + 16 + STAGES * 8;   // + stage rows
-  static_assert(G == 2 || G == 4 || G == 8, "grouped queries");
-  static_assert(MERGE_FLOATS >= kVarlenMaxBatch + 1, "merge area holds the length scan");
-  static_assert(GROUP == 32 || GROUP == 64, "scale group");
-  static_assert(D == 64 || D == 128, "head_dim");
-  static_assert(RB == 0 || RB == 4 || RB == 8, "reference: BF16 rows, INT4 or INT8 codes");
-  // the swizzle pattern repeats every 8 lines: 1024 B for 128-byte lines
-  static_assert(OFF_V % (CRX ? 8 * RROW : 1024) == 0, "swizzled tiles start on the period");
-};
-
-// ---- PTX wrappers -----------------------------------------------------------
-
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
-                                            uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
-      : "memory");
-}
-
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-
-__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t (&r)[2]) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];"
-               : "=r"(r[0]), "=r"(r[1])
-               : "r"(addr));
-}
-
-__device__ __forceinline__ void ldsm_x2_trans(uint32_t addr, uint32_t (&r)[2]) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
-               : "=r"(r[0]), "=r"(r[1])
-               : "r"(addr));
-}
-
-__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-
-// D(16x8, f32) += A(16x16) B(16x8); A row-major, B column-major fragments.
-__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
-                                         uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
-      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// the same with f16 operands
-__device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
-                                        uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, "
-      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// Byte offset of 16-byte chunk `chunk` of row `row` in a tile of rows of
-// RROW bytes (32, 64 or 128) written by a TMA copy with the swizzle of that
-// width: address bits 4.. are XORed with bits 7.. (3 bits for 128 B, 2 for
-// 64 B, 1 for 32 B).
-template <int RROW>
-__device__ __forceinline__ uint32_t swz_offset(int row, int chunk) {
-  static_assert(RROW == 32 || RROW == 64 || RROW == 128, "swizzle width");
-  const uint32_t o = (uint32_t)(row * RROW + chunk * 16);
-  constexpr uint32_t mask = RROW / 16 - 1;
-  return o ^ (((o >> 7) & mask) << 4);
-}
-
-
-// {lo, hi} -> packed bf16x2 / f16x2 (round to nearest)
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  uint32_t r;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-__device__ __forceinline__ uint32_t badd2_u(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-  return r;
-}
-__device__ __forceinline__ float bf16_lo_f(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi_f(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-
-// {lo, hi} as a bf16 pair h plus a bf16 pair of remainders r, lo ~ h.lo + r.lo
-__device__ __forceinline__ void split_bf16(float lo, float hi, uint32_t& h, uint32_t& r) {
-  h = pack_bf16(lo, hi);
-  r = pack_bf16(lo - bf16_lo_f(h), hi - bf16_hi_f(h));
-}
-
-__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
-  uint32_t r;
-  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-__device__ __forceinline__ float f16_lo_f(uint32_t w) {
-  return __half2float(__ushort_as_half((unsigned short)(w & 0xFFFFu)));
-}
-__device__ __forceinline__ float f16_hi_f(uint32_t w) {
-  return __half2float(__ushort_as_half((unsigned short)(w >> 16)));
-}
-// {lo, hi} as an f16 pair h plus an f16 pair of remainders r
-__device__ __forceinline__ void split_f16(float lo, float hi, uint32_t& h, uint32_t& r) {
-  h = pack_f16(lo, hi);
-  r = pack_f16(lo - f16_lo_f(h), hi - f16_hi_f(h));
-}
-
-constexpr uint32_t kMagic = 0x43004300u;   // bf16 128.0 in both halves (mantissa unit 1)
-
-template <int D, int G, int BITS, int GROUP, int RB>
-__global__ void __launch_bounds__(kDecodeThreads, 2)
-decode_gqa_kernel(const __grid_constant__ GqaParams gp) {
-  using C = GCfg<D, G, BITS, GROUP, RB>;
-  const DecodeParams& p = gp.p;
-  constexpr int STAGES = C::STAGES, TILE = C::TILE, KT = C::KT;
-  constexpr unsigned FULL = 0xffffffffu;
-  constexpr int TOPLVL = C::RES ? (1 << BITS) - 1 : 0;
-  constexpr int NG = C::NG, KSG = C::KSG, SB = C::SB;
-
-  extern __shared__ unsigned char smem_raw[];
-  // the swizzled boxes need 1024-byte alignment
-  unsigned char* smem = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  unsigned char* ring = smem;
-  float* merge = reinterpret_cast<float*>(smem + C::RING_BYTES);
-  float* qbuf = merge + C::MERGE_FLOATS;
-  float* wsum_s = qbuf + C::QBUF_FLOATS;
-  uint32_t* qfrag = reinterpret_cast<uint32_t*>(wsum_s + C::WSUM_FLOATS);  // [3][KT][32][2]
-  float* sq_s = reinterpret_cast<float*>(qfrag + C::QFRAG_WORDS);           // [G][NG]
-  float* sqh_s = sq_s + G * NG;              // CR: [G][NG] sums of the f16 q~ fragments
-  float* rsig_s = sqh_s + G * NG;            // CR: [G] 2^-E of each row's f16 q~
-  float* wsumR_s = wsum_s + kConsumerWarps * G * NG;   // CR: sums of p s_ref^V
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(sq_s + C::SQ_FLOATS);
-  uint64_t* empty_bar = full_bar + STAGES;
-  volatile int* flags = reinterpret_cast<volatile int*>(empty_bar + STAGES);
-  volatile unsigned long long* stage_row = reinterpret_cast<volatile unsigned long long*>(
-      reinterpret_cast<unsigned char*>(empty_bar + STAGES) + 16);    // [STAGES], paged
-
-  const int tid = threadIdx.x;
-  const int warp = tid >> 5;
-  const int lane = tid & 31;
-  const int cta = blockIdx.x;
-  pdl_allow_next();
-  if (cta >= p.ctas) return;
-
-  if (tid == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full_bar[s], 1);
-      mbar_init(&empty_bar[s], kConsumerWarps);
-    }
-    flags[0] = 0;
-    flags[1] = 0;
-    fence_mbar_init();
-  }
-  __syncthreads();
-  pdl_wait_prev();     // inputs and workspace may come from the previous kernel
-
-  // this CTA's run of tiles (the merge area is free scratch until the first head)
-  CallSplit split;
-  long long tile_begin, tile_end;
-  TileCursor first_cur;
-  if (!plan_cta(p, cta, reinterpret_cast<int*>(merge), split, tile_begin, tile_end, first_cur))
-    return;
-  const int n_my = (int)(tile_end - tile_begin);
-
-  // ========================= producer warp ================================
-  if (warp == kConsumerWarps) {
-    if (lane == 0) {
-      int issued = 0;
-      TileCursor cur = first_cur;
-      // paged caches: the next tile's page id is read one tile ahead
-      int page_next = (p.page_table && n_my > 0) ? tile_page(p, cur) : 0;
-      for (int i = 0; i < n_my; ++i) {
-        const int s = i % STAGES;
-        const TileCursor tc = cur;
-        const int page = page_next;
-        cur.next(p);
-        if (p.page_table && i + 1 < n_my) page_next = tile_page(p, cur);
-        if (i >= STAGES) {
-          if (!mbar_wait_bounded(&empty_bar[s], ((i / STAGES) - 1) & 1)) {
-            flag_error(p.status, 1u);
-            flags[0] = 1;
-            break;
-          }
-        }
-        if (flags[0]) break;
-        size_t row;
-        const bool page_ok = p.page_table ? tile_row_page(p, tc, page, row) : tile_row(p, tc, row);
-        if (!page_ok && tc.n() > 0) flag_error(p.status, 32u);
-        const int n = page_ok ? tc.n() : 0;
-        if (p.page_table) stage_row[s] = page_ok ? (unsigned long long)row : kBadRow;
-        unsigned char* st = ring + s * C::STAGE_BYTES;
-        if (n <= 0) {                   // the empty tile of an empty sequence
-          mbar_arrive(&full_bar[s]);
-          ++issued;
-          continue;
-        }
-        uint32_t bytes = 2u * C::REF_TILE_BYTES;          // full boxes, OOB rows zero-filled
-        size_t sc_lo = 0;
-        uint32_t sc_bytes = 0;
-        if constexpr (C::RES || C::CRX) {
-          const size_t start = row * SB;
-          sc_lo = start & ~(size_t)15;
-          sc_bytes = (uint32_t)(((start + (size_t)n * SB + 15) & ~(size_t)15) - sc_lo);
-        }
-        if constexpr (C::RES) bytes += 2u * n * C::CROW + 2u * sc_bytes;
-        if constexpr (C::CRX) bytes += 2u * sc_bytes;
-        mbar_arrive_expect_tx(&full_bar[s], bytes);
-        if constexpr (C::CRX) {
-          // one box of whole code rows each
-          tma_load_2d(st + C::OFF_K, &gp.tmap_k, 0, (int)row, &full_bar[s]);
-          tma_load_2d(st + C::OFF_V, &gp.tmap_v, 0, (int)row, &full_bar[s]);
-          bulk_g2s(st + C::OFF_RSK, reinterpret_cast<const unsigned char*>(p.rscales_k) + sc_lo,
-                   sc_bytes, &full_bar[s]);
-          bulk_g2s(st + C::OFF_RSV, reinterpret_cast<const unsigned char*>(p.rscales_v) + sc_lo,
-                   sc_bytes, &full_bar[s]);
-        } else {
-#pragma unroll
-          for (int bx = 0; bx < C::NBOX; ++bx) {
-            tma_load_2d(st + C::OFF_K + bx * C::BOX_BYTES, &gp.tmap_k, 64 * bx, (int)row,
-                        &full_bar[s]);
-            tma_load_2d(st + C::OFF_V + bx * C::BOX_BYTES, &gp.tmap_v, 64 * bx, (int)row,
-                        &full_bar[s]);
-          }
-        }
-        if constexpr (C::RES) {
-          bulk_g2s(st + C::OFF_CK, p.codes_k + row * C::CWORDS, n * C::CROW, &full_bar[s]);
-          bulk_g2s(st + C::OFF_CV, p.codes_v + row * C::CWORDS, n * C::CROW, &full_bar[s]);
-          bulk_g2s(st + C::OFF_SK, reinterpret_cast<const unsigned char*>(p.scales_k) + sc_lo,
-                   sc_bytes, &full_bar[s]);
-          bulk_g2s(st + C::OFF_SV, reinterpret_cast<const unsigned char*>(p.scales_v) + sc_lo,
-                   sc_bytes, &full_bar[s]);
-        }
-        ++issued;
-      }
-      for (int j = (issued > STAGES ? issued - STAGES : 0); j < issued; ++j)
-        if (!mbar_wait_bounded(&full_bar[j % STAGES], (j / STAGES) & 1)) flag_error(p.status, 2u);
-    }
-    return;
-  }
-
-  // ========================= consumer warps ===============================
-  const int g = lane >> 2;            // fragment row group
-  const int q = lane & 3;             // fragment column pair
-  const int wtok = warp * C::WTOK;    // this warp's first token in a tile
-  const bool row_ok = g < G;          // lanes whose S/P row is a real query row
-  const float score_scale = p.score_scale;
-
-  // The per-head Q A-fragments live in shared memory (qfrag): for k-step kk
-  // and lane, {a0, a2} of the bf16 query (kind 0) and of the rotated query
-  // q~ as bf16 high part (kind 1) and bf16 remainder (kind 2): rows g, dims
-  // 16kk + 2q.. and 16kk + 2q + 8..; rows g >= G are zero, and a1 = a3 = 0
-  // (rows g + 8).  With the INT8 reference, kinds 3 and 4 are the f16 high
-  // part and remainder of q~ 2^E (dims 16kk + 4q ..).
-  auto qfrag_addr = [&](int kind, int kk) {
-    return smem_u32(qfrag + ((kind * KT + kk) * 32 + lane) * 2);
-  };
-  // softmax state of row g (lanes with row_ok), and the output accumulators
-  // (O^T fragments: dims 16mt + g (+8), rows 2q, 2q + 1)
-  float m_run = kNegInf, l_run = 0.0f;
-  float wsum[NG], wsumR[NG];
-  float vscale = 1.0f;     // INT8 reference: power of two applied to the V weights
-  float oref[KT][4], ores[KT][4];
-
-  auto reset_state = [&]() {
-    m_run = kNegInf;
-    l_run = 0.0f;
-    vscale = 1.0f;
-#pragma unroll
-    for (int j = 0; j < NG; ++j) {
-      wsum[j] = 0.0f;
-      wsumR[j] = 0.0f;
-    }
-#pragma unroll
-    for (int mt = 0; mt < KT; ++mt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        oref[mt][e] = 0.0f;
-        ores[mt][e] = 0.0f;
-      }
-  };
-
-  auto setup_head = [&](long long hd) {
-    float* qs = qbuf;
-    float* qt = qbuf + G * D;
-    load_rotate_queries<D, G>(p, hd, qs, qt, tid);
-    const float cd = rot_scale<D>();
-    if constexpr (C::CRX) {
-      if (warp == 0) {
-        // f16 fragments of q~ 2^E, E per row so that max |q~| 2^E is in
-        // [2^13, 2^14): the high parts keep 11 bits, the remainders the next
-        // 11, and no value leaves f16's normal range.  The k positions
-        // follow the codes a 32-bit ldmatrix word holds: INT8, k positions
-        // 2q, 2q+1 | 2q+8, 2q+9 of k-step kk carry dims 16kk + 4q .. 4q+3;
-        // INT4, a word holds dims 8q .. 8q+7 of a 32-dim chunk (two k-steps),
-        // code i at bits 4i, and k-step kk (half h = kk & 1 of chunk kk / 2)
-        // carries dims 8q + 2h + {0, 4 | 1, 5} (a register's two codes then
-        // sit 16 bits apart).
-        float mx = 0.0f;
-        if (row_ok)
-          for (int d = q; d < D; d += 4) mx = fmaxf(mx, fabsf(cd * qt[g * D + d]));
-        mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 1));
-        mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 2));
-        const int ex = (int)((__float_as_uint(mx) >> 23) & 0xFFu) - 127;
-        const int E = min(13 - ex, 126);
-        const float up = __uint_as_float((uint32_t)(127 + E) << 23);
-        if (row_ok && q == 0) rsig_s[g] = __uint_as_float((uint32_t)(127 - E) << 23);
-        float sqh = 0.0f;
-#pragma unroll 1
-        for (int kk = 0; kk < KT; ++kk) {
-          uint32_t* f3 = qfrag + ((3 * KT + kk) * 32 + lane) * 2;
-          uint32_t* f4 = qfrag + ((4 * KT + kk) * 32 + lane) * 2;
-          if (row_ok) {
-            int d0, d1, d2, d3;
-            if constexpr (C::CR) {
-              d0 = 16 * kk + 4 * q;
-              d1 = d0 + 1;
-              d2 = d0 + 2;
-              d3 = d0 + 3;
-            } else {
-              d0 = 32 * (kk >> 1) + 8 * q + 2 * (kk & 1);
-              d1 = d0 + 4;
-              d2 = d0 + 1;
-              d3 = d0 + 5;
-            }
-            const float* trow = qt + g * D;
-            split_f16(cd * trow[d0] * up, cd * trow[d1] * up, f3[0], f4[0]);
-            split_f16(cd * trow[d2] * up, cd * trow[d3] * up, f3[1], f4[1]);
-            sqh += ((f16_lo_f(f3[0]) + f16_lo_f(f4[0])) + (f16_hi_f(f3[0]) + f16_hi_f(f4[0]))) +
-                   ((f16_lo_f(f3[1]) + f16_lo_f(f4[1])) + (f16_hi_f(f3[1]) + f16_hi_f(f4[1])));
-          } else {
-            f3[0] = f3[1] = f4[0] = f4[1] = 0u;
-          }
-          if ((kk + 1) % KSG == 0) {                   // end of a scale group
-            sqh += __shfl_xor_sync(FULL, sqh, 1);
-            sqh += __shfl_xor_sync(FULL, sqh, 2);
-            if (row_ok && q == 0) sqh_s[g * NG + kk / KSG] = sqh;
-            sqh = 0.0f;
-          }
-        }
-      }
-    }
-    if (warp == 0) {
-      float sqj = 0.0f;      // running sum of the current scale group (INT2)
-#pragma unroll 1
-      for (int kk = 0; kk < KT; ++kk) {
-        uint32_t* fa = qfrag + ((0 * KT + kk) * 32 + lane) * 2;
-        uint32_t* fh = qfrag + ((1 * KT + kk) * 32 + lane) * 2;
-        uint32_t* fl = qfrag + ((2 * KT + kk) * 32 + lane) * 2;
-        if (row_ok) {
-          const float* qrow = qs + g * D + 16 * kk + 2 * q;
-          // INT2 with ldmatrix words: k-step kk = 4c + t of chunk c carries
-          // dims 64c + 16q + 2t + {0, 8 | 1, 9} (codes 2t, 2t+8 | 2t+1, 2t+9
-          // of the word holding the chunk's dims 16q .. 16q+15)
-          // (32-dim groups: k-step kk is half t = kk & 1 of group (kk >> 1) & 1 of
-          // chunk kk >> 2; lane q reads the word of dims 16 (q & 1) .. of that
-          // group and takes its codes 2u, 2u+8 | 2u+1, 2u+9, u = 2t + (q >> 1))
-          const int lo2 = GROUP == 64 ? 16 * q + 2 * (kk & 3)
-                                      : 32 * ((kk >> 1) & 1) + 16 * (q & 1) +
-                                            2 * (2 * (kk & 1) + (q >> 1));
-          const float* trow = qt + g * D + (C::LDM2 ? 64 * (kk >> 2) + lo2 : 16 * kk + 2 * q);
-          fa[0] = pack_bf16(qrow[0], qrow[1]);       // exact: q is bf16
-          fa[1] = pack_bf16(qrow[8], qrow[9]);
-          if constexpr (BITS == 2) {
-            // k positions 2q, 2q+1 | 2q+8, 2q+9 carry dims 2q, 2q+8 | 2q+1, 2q+9,
-            // so the two codes of a B register sit 16 bits apart
-            split_bf16(cd * trow[0], cd * trow[8], fh[0], fl[0]);
-            split_bf16(cd * trow[1], cd * trow[9], fh[1], fl[1]);
-            sqj += ((bf16_lo_f(fh[0]) + bf16_lo_f(fl[0])) +
-                    (bf16_hi_f(fh[0]) + bf16_hi_f(fl[0]))) +
-                   ((bf16_lo_f(fh[1]) + bf16_lo_f(fl[1])) +
-                    (bf16_hi_f(fh[1]) + bf16_hi_f(fl[1])));
-          } else if constexpr (C::LDM4) {
-            // k-step kk = half h of 32-dim chunk kk >> 1: k positions 2q, 2q+1 |
-            // 2q+8, 2q+9 carry dims 8q + 2h + {0, 4 | 1, 5} (the word's codes
-            // 2h, 2h+4 | 2h+1, 2h+5, each register's two codes 16 bits apart)
-            const float* t4 = qt + g * D + 32 * (kk >> 1) + 8 * q + 2 * (kk & 1);
-            split_bf16(cd * t4[0], cd * t4[4], fh[0], fl[0]);
-            split_bf16(cd * t4[1], cd * t4[5], fh[1], fl[1]);
-            sqj += ((bf16_lo_f(fh[0]) + bf16_lo_f(fl[0])) +
-                    (bf16_hi_f(fh[0]) + bf16_hi_f(fl[0]))) +
-                   ((bf16_lo_f(fh[1]) + bf16_lo_f(fl[1])) +
-                    (bf16_hi_f(fh[1]) + bf16_hi_f(fl[1])));
-          } else {
-            split_bf16(cd * trow[0], cd * trow[1], fh[0], fl[0]);
-            split_bf16(cd * trow[8], cd * trow[9], fh[1], fl[1]);
-          }
-        } else {
-          fa[0] = fa[1] = fh[0] = fh[1] = fl[0] = fl[1] = 0u;
-        }
-        if ((BITS == 2 || C::LDM4) && (kk + 1) % KSG == 0) {      // end of a scale group
-          sqj += __shfl_xor_sync(FULL, sqj, 1);
-          sqj += __shfl_xor_sync(FULL, sqj, 2);
-          if (row_ok && q == 0) sq_s[g * NG + kk / KSG] = sqj;
-          sqj = 0.0f;
-        }
-      }
-    }
-    named_bar_sync(1, kConsumerThreads);
-  };
-
-  auto flush_head = [&](long long hd, long long first_tile, int nt_h) {
-    // l and the V weight sums of row g over the four lanes of its row group
-    l_run += __shfl_xor_sync(FULL, l_run, 1);
-    l_run += __shfl_xor_sync(FULL, l_run, 2);
-#pragma unroll
-    for (int j = 0; j < NG; ++j) {
-      wsum[j] += __shfl_xor_sync(FULL, wsum[j], 1);
-      wsum[j] += __shfl_xor_sync(FULL, wsum[j], 2);
-      if constexpr (C::CRX) {
-        wsumR[j] += __shfl_xor_sync(FULL, wsumR[j], 1);
-        wsumR[j] += __shfl_xor_sync(FULL, wsumR[j], 2);
-      }
-    }
-    named_bar_sync(1, kConsumerThreads);          // merge area free
-    float* mw = merge + warp * G * (2 + 2 * D);
-    if constexpr (C::CRX) {
-      // non-finite reference weights (invalid scales): the output is not valid
-      bool bad = false;
-#pragma unroll
-      for (int j = 0; j < NG; ++j) bad |= !isfinite(wsumR[j]);
-      if (row_ok && q == 0 && bad) flag_error(p.status, 64u);
-    }
-    if (row_ok && q == 0) {
-      mw[g * (2 + 2 * D)] = m_run;
-      mw[g * (2 + 2 * D) + 1] = l_run;
-#pragma unroll
-      for (int j = 0; j < NG; ++j) {
-        if constexpr (C::RES) wsum_s[(warp * G + g) * NG + j] = wsum[j];
-        if constexpr (C::CRX) wsumR_s[(warp * G + g) * NG + j] = wsumR[j] * (1.0f / vscale);
-      }
-    }
-    // O^T fragments: c0 (dim 16mt+g, row 2q), c1 (.., row 2q+1), c2/c3 dim +8;
-    // the INT8 reference's m-rows g, g + 8 are dims 16mt + 2g, 16mt + 2g + 1,
-    // the INT4 reference's 32 (mt / 2) + 4g + 2 (mt & 1) (+ 1)
-#pragma unroll
-    for (int mt = 0; mt < KT; ++mt) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int r = 2 * q + (e & 1);
-        const int dim = 16 * mt + g + 8 * (e >> 1);
-        const int dim_res =
-            C::LDM4       ? 32 * (mt >> 1) + 4 * g + 2 * (mt & 1) + (e >> 1)
-            : !C::LDM2    ? dim
-            : GROUP == 64 ? 64 * (mt >> 2) + 8 * g + 2 * (mt & 3) + (e >> 1)
-                          : 64 * (mt >> 2) + 32 * ((mt >> 1) & 1) + 8 * (g & 3) + 4 * (mt & 1) +
-                                2 * (g >> 2) + (e >> 1);
-        const int dim_ref = C::CR    ? 16 * mt + 2 * g + (e >> 1)
-                            : C::CR4 ? 32 * (mt >> 1) + 4 * g + 2 * (mt & 1) + (e >> 1)
-                                     : dim;
-        if (r < G) {
-          if constexpr (C::CRX) mw[r * (2 + 2 * D) + 2 + dim_ref] = oref[mt][e] * (C::CSCALE / vscale);
-          else mw[r * (2 + 2 * D) + 2 + dim_ref] = oref[mt][e];
-          if constexpr (C::RES) mw[r * (2 + 2 * D) + 2 + D + dim_res] = 2.0f * ores[mt][e];
-          else mw[r * (2 + 2 * D) + 2 + D + dim] = 0.0f;
-        }
-      }
-    }
-    named_bar_sync(1, kConsumerThreads);
-    if constexpr (C::RES || C::CRX) {
-      // complete sum_t p s (2c - top) = 2 sum p s c - top sum p s; the
-      // compressed reference's sum_t p s_ref (2c - (2^RB - 1)) = CSCALE acc -
-      // LOFF sum p s_ref (acc over the f16 code operands, written as
-      // CSCALE acc), moved to the rotated part
-      for (int e = tid; e < kConsumerWarps * G * D; e += kConsumerThreads) {
-        const int w = e / (G * D), r = (e / D) % G, dim = e % D;
-        float* rec = merge + (w * G + r) * (2 + 2 * D);
-        const int wi = (w * G + r) * NG + dim / GROUP;
-        float z = rec[2 + D + dim];
-        if constexpr (C::RES) z -= (float)TOPLVL * wsum_s[wi];
-        if constexpr (C::CRX) {
-          z += rec[2 + dim] - C::LOFF * wsumR_s[wi];
-          rec[2 + dim] = 0.0f;
-        }
-        rec[2 + D + dim] = z;
-      }
-      named_bar_sync(1, kConsumerThreads);
-    }
-    finish_head<D, G, C::RES || C::CRX>(p, hd, first_tile, nt_h, split, cta, merge, qbuf, flags,
-                                        tid);
-  };
-
-  // ---- one tile ----
-  auto tile_mma = [&](const unsigned char* st, int n, int sc_off) {
-    if (!C::CRX && n < TILE) {
-      // rows past the head's last token (spare capacity, the next head, or
-      // nothing ever written) are not part of the context: their weights are
-      // 0, and zeroing this warp's such V rows keeps a non-finite value there
-      // out of the products
-      unsigned char* vrows = const_cast<unsigned char*>(st) + C::OFF_V;
-      for (int e = lane; e < C::WTOK * C::NBOX * 8; e += 32) {
-        const int tok = wtok + e / (C::NBOX * 8), c = e % (C::NBOX * 8);
-        if (tok >= n)
-          *reinterpret_cast<uint4*>(vrows + (c >> 3) * C::BOX_BYTES + tok * 128 + (c & 7) * 16) =
-              make_uint4(0u, 0u, 0u, 0u);
-      }
-      __syncwarp();
-    }
-    const uint32_t sK = smem_u32(st + C::OFF_K);
-    const uint32_t sV = smem_u32(st + C::OFF_V);
-    const int r7 = lane & 7;
-    // ---- scores for the warp's two 8-token tiles, k-steps outermost ----
-    // c[nt]: S_ref (then + s x S_res) fragments, row g, tokens 2q, 2q+1 of nt
-    float cref[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
-    float ct[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
-    const int tok0[2] = {wtok + 2 * q, wtok + 8 + 2 * q};     // tokens of c0 per tile
-    // ldmatrix: matrices (tile 0, dims +0..7), (tile 0, +8..15), (tile 1, ..), (tile 1, ..)
-    const int ktr = wtok + ((lane >> 4) & 1) * 8 + r7;
-    const int kch = (lane >> 3) & 1;
-    // compressed reference: per-group f16 sums sum_k q~_k 2^E c_k 2^-24
-    float c8[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
-    uint32_t b8[4];          // ldmatrix words of two k-steps: (nt 0, kk), (nt 1, kk), (nt 0, kk + 1), ..
-    uint32_t ck4[4];         // INT2 residual: the tile's K code words
-    uint32_t ckp[4];         // 32-dim groups: the same words of lane ^ 2
-#pragma unroll
-    for (int kk = 0; kk < KT; ++kk) {
-      if constexpr (C::CR) {
-        if ((kk & 1) == 0) {
-          const int m = lane >> 3;
-          ldsm_x4(sK + swz_offset<C::RROW>(wtok + (m & 1) * 8 + r7, kk + (m >> 1)), b8);
-        }
-        const uint2 fh = *reinterpret_cast<const uint2*>(qfrag + ((3 * KT + kk) * 32 + lane) * 2);
-        const uint2 fl = *reinterpret_cast<const uint2*>(qfrag + ((4 * KT + kk) * 32 + lane) * 2);
-        const uint32_t ah[4] = {fh.x, 0u, fh.y, 0u};
-        const uint32_t al[4] = {fl.x, 0u, fl.y, 0u};
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-          // codes 4q .. 4q+3 of the k-step's 16 as f16 subnormals c 2^-24, exact
-          const uint32_t w = b8[2 * (kk & 1) + nt];
-          const uint32_t b0 = __byte_perm(w, 0u, 0x4140);
-          const uint32_t b1 = __byte_perm(w, 0u, 0x4342);
-          mma_f16(c8[nt], ah, b0, b1);
-          mma_f16(c8[nt], al, b0, b1);
-        }
-      } else if constexpr (C::CR4) {
-        // one ldmatrix.x4 every four k-steps: words (nt 0, chunk), (nt 1,
-        // chunk), (nt 0, chunk + 1), (nt 1, chunk + 1) of two 32-dim chunks
-        if ((kk & 3) == 0) {
-          const int m = lane >> 3;
-          ldsm_x4(sK + swz_offset<C::RROW>(wtok + (m & 1) * 8 + r7, (kk >> 1) + (m >> 1)), b8);
-        }
-        const uint2 fh = *reinterpret_cast<const uint2*>(qfrag + ((3 * KT + kk) * 32 + lane) * 2);
-        const uint2 fl = *reinterpret_cast<const uint2*>(qfrag + ((4 * KT + kk) * 32 + lane) * 2);
-        const uint32_t ah[4] = {fh.x, 0u, fh.y, 0u};
-        const uint32_t al[4] = {fl.x, 0u, fl.y, 0u};
-        const int sh = 8 * (kk & 1);
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-          // codes i, i + 4 of the word (bits 4i, 4i + 16) as f16 subnormals c 2^-24
-          const uint32_t w = b8[2 * ((kk >> 1) & 1) + nt];
-          const uint32_t b0 = (w >> sh) & 0x000F000Fu;
-          const uint32_t b1 = (w >> (sh + 4)) & 0x000F000Fu;
-          mma_f16(c8[nt], ah, b0, b1);
-          mma_f16(c8[nt], al, b0, b1);
-        }
-      } else {
-        const int chunk = 2 * kk + kch;
-        uint32_t b[4];
-        ldsm_x4(sK + (chunk >> 3) * C::BOX_BYTES + ktr * 128 + (((chunk & 7) ^ r7) << 4), b);
-        uint32_t a[4] = {0u, 0u, 0u, 0u};
-        {
-          const uint2 f = *reinterpret_cast<const uint2*>(qfrag + ((0 * KT + kk) * 32 + lane) * 2);
-          a[0] = f.x;
-          a[2] = f.y;
-        }
-        mma_bf16(cref[0], a, b[0], b[1]);
-        mma_bf16(cref[1], a, b[2], b[3]);
-      }
-      if (C::CRX && (kk + 1) % KSG == 0) {
-        // end of scale group j: S += s_ref_{t, j} 2^-E (CSCALE acc - LOFF sum q~ 2^E)
-        const int j = kk / KSG;
-        const float rs = row_ok ? rsig_s[g] : 0.0f;
-        const float off = row_ok ? C::LOFF * sqh_s[g * NG + j] : 0.0f;
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-          const float r0 = half_at(st + C::OFF_RSK + sc_off + tok0[nt] * SB + 2 * j);
-          const float r1 = half_at(st + C::OFF_RSK + sc_off + (tok0[nt] + 1) * SB + 2 * j);
-          cref[nt][0] = fmaf(r0 * rs, fmaf(C::CSCALE, c8[nt][0], -off), cref[nt][0]);
-          cref[nt][1] = fmaf(r1 * rs, fmaf(C::CSCALE, c8[nt][1], -off), cref[nt][1]);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) c8[nt][e] = 0.0f;
-        }
-      }
-      if constexpr (C::RES) {
-        const uint2 fh = *reinterpret_cast<const uint2*>(qfrag + ((1 * KT + kk) * 32 + lane) * 2);
-        const uint2 fl = *reinterpret_cast<const uint2*>(qfrag + ((2 * KT + kk) * 32 + lane) * 2);
-        const uint32_t ah[4] = {fh.x, 0u, fh.y, 0u};
-        const uint32_t al[4] = {fl.x, 0u, fl.y, 0u};
-        if constexpr (C::LDM4) {
-          // every fourth k-step: words (nt 0, chunk), (nt 1, chunk), (nt 0,
-          // chunk + 1), (nt 1, chunk + 1) of two 32-dim chunks
-          if ((kk & 3) == 0) {
-            const int m = lane >> 3;
-            ldsm_x4(smem_u32(st + C::OFF_CK + (wtok + (m & 1) * 8 + r7) * C::CROW +
-                             ((kk >> 1) + (m >> 1)) * 16),
-                    ck4);
-          }
-        }
-        if constexpr (C::LDM2) {
-          // the whole warp tile's K codes in one ldmatrix: words (nt 0, chunk
-          // 0), (nt 1, chunk 0)[, (nt 0, chunk 1), (nt 1, chunk 1)]
-          if (kk == 0) {
-            const int m = (lane >> 3) & (2 * C::NCH - 1);
-            const uint32_t a = smem_u32(st + C::OFF_CK + (wtok + (m & 1) * 8 + r7) * C::CROW +
-                                        (m >> 1) * 16);
-            if constexpr (C::NCH == 2) {
-              ldsm_x4(a, ck4);
-            } else {
-              uint32_t r2[2];
-              ldsm_x2(a, r2);
-              ck4[0] = r2[0];
-              ck4[1] = r2[1];
-            }
-            if constexpr (GROUP == 32) {
-#pragma unroll
-              for (int m = 0; m < 2 * C::NCH; ++m) ckp[m] = __shfl_xor_sync(FULL, ck4[m], 2);
-            }
-          }
-        }
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-          uint32_t b0, b1;
-          if constexpr (C::LDM2) {
-            // codes 2u, 2u+8 | 2u+1, 2u+9 of the word at mantissa bits 1-2:
-            // bf16 128 + 2c, exact (the q~ fragments' k permutation puts the
-            // two codes of a B register 16 bits apart); bit 31 (code 15) is
-            // not among the codes the shifted copy serves
-            uint32_t w;
-            int u;
-            if constexpr (GROUP == 64) {
-              w = ck4[2 * (kk >> 2) + nt];
-              u = kk & 3;
-            } else {
-              const int idx = 2 * (kk >> 2) + nt;
-              w = ((q >> 1) == ((kk >> 1) & 1)) ? ck4[idx] : ckp[idx];
-              u = 2 * (kk & 1) + (q >> 1);
-            }
-            b0 = (((w << 1) >> (4 * u)) & 0x00060006u) | kMagic;
-            b1 = ((w >> (4 * u + 1)) & 0x00060006u) | kMagic;
-          } else {
-            static_assert(C::LDM4, "residual codes are INT2 or INT4");
-            // codes 2h, 2h+4 | 2h+1, 2h+5 at mantissa bits 1-4: bf16 128 + 2c, exact
-            const uint32_t w = ck4[2 * ((kk >> 1) & 1) + nt];
-            const int h = kk & 1;
-            b0 = (((w << 1) >> (8 * h)) & 0x001E001Eu) | kMagic;
-            b1 = ((w >> (8 * h + 3)) & 0x001E001Eu) | kMagic;
-          }
-          mma_bf16(ct[nt], ah, b0, b1);
-          mma_bf16(ct[nt], al, b0, b1);
-        }
-        if ((kk + 1) % KSG == 0) {
-          // end of scale group j: S += s^K_{t, j} x (q~_j . l_j) for c0, c1
-          const int j = kk / KSG;
-#pragma unroll
-          for (int nt = 0; nt < 2; ++nt) {
-            const float sk0 = half_at(st + C::OFF_SK + sc_off + tok0[nt] * SB + 2 * j);
-            const float sk1 = half_at(st + C::OFF_SK + sc_off + (tok0[nt] + 1) * SB + 2 * j);
-            // INT2 operands are 128 + 2c: q~ . l = result - 131 sum q~; INT4
-            // (ldmatrix words) 128 + 2c: result - 143 sum q~
-            const float off = ((BITS == 2 || C::LDM4) && row_ok)
-                                  ? (BITS == 2 ? 131.0f : 143.0f) * sq_s[g * NG + j]
-                                  : 0.0f;
-            cref[nt][0] = fmaf(sk0, ct[nt][0] - off, cref[nt][0]);
-            cref[nt][1] = fmaf(sk1, ct[nt][1] - off, cref[nt][1]);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) ct[nt][e] = 0.0f;
-          }
-        }
-      }
-    }
-    float sc[2][2];          // row g, tokens 2q, 2q+1 of tile nt
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      sc[nt][0] = (row_ok && tok0[nt] < n) ? score_scale * cref[nt][0] : kNegInf;
-      sc[nt][1] = (row_ok && tok0[nt] + 1 < n) ? score_scale * cref[nt][1] : kNegInf;
-    }
-    // ---- online softmax of row g (four lanes per row), rescaled lazily ----
-    float mc = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
-    float alpha = 1.0f;
-    if (__any_sync(FULL, mc > m_run + kLazyMax)) {
-      mc = fmaxf(mc, __shfl_xor_sync(FULL, mc, 1));
-      mc = fmaxf(mc, __shfl_xor_sync(FULL, mc, 2));
-      const float m_new = fmaxf(m_run, mc);
-      alpha = (m_new == m_run) ? 1.0f : (m_run == kNegInf ? 0.0f : exp2f(m_run - m_new));
-      m_run = m_new;
-    }
-    float pr[2][2];
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-      for (int e = 0; e < 2; ++e) pr[nt][e] = (sc[nt][e] == kNegInf) ? 0.0f : exp2f(sc[nt][e] - m_run);
-    l_run = l_run * alpha + (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
-    if (!__all_sync(FULL, alpha == 1.0f)) {
-      // rows 2q and 2q+1 of the O^T fragments: their alphas live in lanes 8q, 8q+4
-      const float a0 = __shfl_sync(FULL, alpha, 8 * q);
-      const float a1 = __shfl_sync(FULL, alpha, 8 * q + 4);
-      const float2 a01 = make_float2(a0, a1);
-#pragma unroll
-      for (int mt = 0; mt < KT; ++mt) {
-        float2 x = __fmul2_rn(make_float2(oref[mt][0], oref[mt][1]), a01);
-        float2 y = __fmul2_rn(make_float2(oref[mt][2], oref[mt][3]), a01);
-        oref[mt][0] = x.x; oref[mt][1] = x.y; oref[mt][2] = y.x; oref[mt][3] = y.y;
-        if constexpr (C::RES) {
-          x = __fmul2_rn(make_float2(ores[mt][0], ores[mt][1]), a01);
-          y = __fmul2_rn(make_float2(ores[mt][2], ores[mt][3]), a01);
-          ores[mt][0] = x.x; ores[mt][1] = x.y; ores[mt][2] = y.x; ores[mt][3] = y.y;
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < NG; ++j) {
-        wsum[j] *= alpha;
-        wsumR[j] *= alpha;
-      }
-    }
-    // P^T fragments (k = tokens 2q, 2q+1 / +8, n = row g): bf16 hi + lo
-    const uint32_t ph0 = pack_bf16(pr[0][0], pr[0][1]);
-    const uint32_t ph1 = pack_bf16(pr[1][0], pr[1][1]);
-    const uint32_t pl0 = pack_bf16(pr[0][0] - bf16_lo_f(ph0), pr[0][1] - bf16_hi_f(ph0));
-    const uint32_t pl1 = pack_bf16(pr[1][0] - bf16_lo_f(ph1), pr[1][1] - bf16_hi_f(ph1));
-    if constexpr (C::CRX) {
-      // ---- O_ref^T += C_ref^T (P s_ref^V 2^Ev)^T, codes as f16 subnormals ----
-      // ldmatrix.trans of the code rows.  INT8: word = codes (token 2q: dims
-      // 2g, 2g+1; token 2q+1: dims 2g, 2g+1) of a 16-dim chunk; m-row g is
-      // dim 2g, m-row g + 8 dim 2g + 1.  INT4: word = codes of dims 4g .. 4g+3
-      // of a 32-dim chunk (token 2q low half, 2q+1 high half, code i at bits
-      // 4i); m-tile 2 chunk has m-rows g, g + 8 = dims 4g, 4g + 1, m-tile
-      // 2 chunk + 1 dims 4g + 2, 4g + 3.  The weights p s_ref are f16 high parts
-      // and remainders after a warp-wide power of two vscale that keeps the
-      // tile's largest scale in [1, 2^7): with p < 2^kLazyMax = 2^8 (the
-      // lazy softmax max) no weight reaches 2^15, below f16's largest value,
-      // and the remainders stay far above its subnormals for every weight
-      // that matters.  vscale changes lazily; the accumulators follow it
-      // exactly.
-      const int tk[4] = {wtok + 2 * q, wtok + 2 * q + 1, wtok + 2 * q + 8, wtok + 2 * q + 9};
-      auto s_ref_v = [&](int k, int j) {               // 0 beyond the tile
-        const float v = half_at(st + C::OFF_RSV + sc_off + tk[k] * SB + 2 * j);
-        return (tk[k] < n) ? v : 0.0f;
-      };
-      float smax = 0.0f;
-#pragma unroll
-      for (int j = 0; j < NG; ++j)
-#pragma unroll
-        for (int k = 0; k < 4; ++k) smax = fmaxf(smax, fabsf(s_ref_v(k, j)));
-      smax = fmaxf(smax, __shfl_xor_sync(FULL, smax, 1));
-      smax = fmaxf(smax, __shfl_xor_sync(FULL, smax, 2));
-      {
-        const float big = smax * vscale;                 // the same in every lane
-        static_assert(kLazyMax <= 8.0f, "p s_ref vscale < 2^(kLazyMax + 7) must fit f16");
-        if (smax > 0.0f && !(big >= 1.0f && big < 128.0f)) {
-          const int ex = (int)((__float_as_uint(smax) >> 23) & 0xFFu) - 127;
-          const float nv = __uint_as_float((uint32_t)(127 + 3 - ex) << 23);   // [2^3, 2^4)
-          const float f = nv / vscale;                     // a power of two, exact
-#pragma unroll
-          for (int mt = 0; mt < KT; ++mt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) oref[mt][e] *= f;
-#pragma unroll
-          for (int j = 0; j < NG; ++j) wsumR[j] *= f;
-          vscale = nv;
-        }
-      }
-      const float pk[4] = {pr[0][0] * vscale, pr[0][1] * vscale, pr[1][0] * vscale,
-                           pr[1][1] * vscale};
-#pragma unroll
-      for (int j = 0; j < NG; ++j) {
-        float wv[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) wv[k] = pk[k] * s_ref_v(k, j);
-        wsumR[j] += (wv[0] + wv[1]) + (wv[2] + wv[3]);
-        uint32_t bh0, bl0, bh1, bl1;
-        split_f16(wv[0], wv[1], bh0, bl0);
-        split_f16(wv[2], wv[3], bh1, bl1);
-        if constexpr (C::CR4) {
-#pragma unroll
-          for (int ch = j * GROUP / 32; ch < (j + 1) * GROUP / 32; ++ch) {
-            const int m = (lane >> 3) & 1;
-            uint32_t v[2];   // (tokens 0-7, chunk ch), (tokens 8-15, chunk ch)
-            ldsm_x2_trans(sV + swz_offset<C::RROW>(wtok + m * 8 + r7, ch), v);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int sh = 8 * h;
-              const uint32_t a[4] = {(v[0] >> sh) & 0x000F000Fu, (v[0] >> (sh + 4)) & 0x000F000Fu,
-                                     (v[1] >> sh) & 0x000F000Fu, (v[1] >> (sh + 4)) & 0x000F000Fu};
-              mma_f16(oref[2 * ch + h], a, bh0, bh1);
-              mma_f16(oref[2 * ch + h], a, bl0, bl1);
-            }
-          }
-        } else {
-#pragma unroll
-          for (int mt2 = j * KSG / 2; mt2 < (j + 1) * KSG / 2; ++mt2) {
-            const int m = lane >> 3;
-            uint32_t v[4];   // (tokens 0-7, chunk 2mt2), (8-15, 2mt2), (0-7, 2mt2+1), (8-15, ..)
-            ldsm_x4_trans(sV + swz_offset<C::RROW>(wtok + (m & 1) * 8 + r7, 2 * mt2 + (m >> 1)),
-                          v);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int mt = 2 * mt2 + h;
-              const uint32_t R0 = v[2 * h], R1 = v[2 * h + 1];
-              // bytes 0, 2 (dim 2g) and bytes 1, 3 (dim 2g + 1) as f16 subnormals
-              const uint32_t a[4] = {
-                  __byte_perm(R0, 0u, 0x4240), __byte_perm(R0, 0u, 0x4341),
-                  __byte_perm(R1, 0u, 0x4240), __byte_perm(R1, 0u, 0x4341)};
-              mma_f16(oref[mt], a, bh0, bh1);
-              mma_f16(oref[mt], a, bl0, bl1);
-            }
-          }
-        }
-      }
-    } else {
-      // ---- O_ref^T += V^T P^T ----
-#pragma unroll
-      for (int mt = 0; mt < KT; ++mt) {
-        const int m = lane >> 3;                         // matrix this lane addresses
-        const int tr = wtok + (m >> 1) * 8 + r7;
-        const int chunk = 2 * mt + (m & 1);
-        const uint32_t addr = sV + (chunk >> 3) * C::BOX_BYTES + tr * 128 +
-                              ((((chunk & 7) ^ r7)) << 4);
-        uint32_t a[4];
-        ldsm_x4_trans(addr, a);
-        mma_bf16(oref[mt], a, ph0, ph1);
-        mma_bf16(oref[mt], a, pl0, pl1);
-      }
-    }
-    // ---- O_res^T += C_V^T (P s^V)^T ----
-    if constexpr (C::RES) {
-      const int tk[4] = {wtok + 2 * q, wtok + 2 * q + 1, wtok + 2 * q + 8, wtok + 2 * q + 9};
-      const float pk[4] = {pr[0][0], pr[0][1], pr[1][0], pr[1][1]};
-      // INT2, 64-dim groups: the warp tile's V code words by one
-      // ldmatrix.trans: word = codes of dims 8g .. 8g+7 of a 64-dim chunk
-      // (token 2q low half, 2q+1 high half, code i at bits 2i); (tokens 0-7,
-      // chunk 0), (8-15, chunk 0)[, (0-7, chunk 1), (8-15, chunk 1)]
-      uint32_t cv4[4], cvp[4];   // cvp (32-dim groups): the words of lane ^ 16
-      if constexpr (C::LDM2) {
-        const int m = (lane >> 3) & (2 * C::NCH - 1);
-        const uint32_t a = smem_u32(st + C::OFF_CV + (wtok + (m & 1) * 8 + r7) * C::CROW +
-                                    (m >> 1) * 16);
-        if constexpr (C::NCH == 2) {
-          ldsm_x4_trans(a, cv4);
-        } else {
-          uint32_t r2[2];
-          ldsm_x2_trans(a, r2);
-          cv4[0] = r2[0];
-          cv4[1] = r2[1];
-        }
-        if constexpr (GROUP == 32) {
-#pragma unroll
-          for (int m2 = 0; m2 < 2 * C::NCH; ++m2) cvp[m2] = __shfl_xor_sync(FULL, cv4[m2], 16);
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < NG; ++j) {
-        float wv[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float sv = half_at(st + C::OFF_SV + sc_off + tk[k] * SB + 2 * j);
-          wv[k] = (tk[k] < n) ? pk[k] * sv : 0.0f;       // weight 0 beyond the tile
-        }
-        wsum[j] += (wv[0] + wv[1]) + (wv[2] + wv[3]);
-        uint32_t bh0, bl0, bh1, bl1;
-        split_bf16(wv[0], wv[1], bh0, bl0);
-        split_bf16(wv[2], wv[3], bh1, bl1);
-        if constexpr (C::LDM2) {
-          // operands (128 + c) - 128 = c, exact (the accumulator carries no
-          // offset across the head's tiles)
-          const uint32_t m128 = 0xC300C300u;   // {-128, -128}
-          if constexpr (GROUP == 64) {
-            // chunk j: m-tile 4j + i has m-rows g, g + 8 = dims 64j + 8g + 2i (+ 1)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const uint32_t R0 = cv4[2 * j], R1 = cv4[2 * j + 1];
-              const uint32_t a[4] = {badd2_u(((R0 >> (4 * i)) & 0x00030003u) | kMagic, m128),
-                                     badd2_u(((R0 >> (4 * i + 2)) & 0x00030003u) | kMagic, m128),
-                                     badd2_u(((R1 >> (4 * i)) & 0x00030003u) | kMagic, m128),
-                                     badd2_u(((R1 >> (4 * i + 2)) & 0x00030003u) | kMagic, m128)};
-              mma_bf16(ores[4 * j + i], a, bh0, bh1);
-              mma_bf16(ores[4 * j + i], a, bl0, bl1);
-            }
-          } else {
-            // group j = half gc of chunk c: lanes g and g ^ 4 both hold the
-            // word of dims 8 (g & 3) .. +7 of the group; m-tile 2j + i has
-            // m-rows g, g + 8 = dims 64c + 32gc + 8 (g & 3) + 4i + 2 (g >> 2) (+ 1)
-            const int c = j >> 1, gc = j & 1;
-            const bool own = (g >> 2) == gc;
-            const uint32_t R0 = own ? cv4[2 * c] : cvp[2 * c];
-            const uint32_t R1 = own ? cv4[2 * c + 1] : cvp[2 * c + 1];
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-              const int sh = 2 * (4 * i + 2 * (g >> 2));
-              const uint32_t a[4] = {badd2_u(((R0 >> sh) & 0x00030003u) | kMagic, m128),
-                                     badd2_u(((R0 >> (sh + 2)) & 0x00030003u) | kMagic, m128),
-                                     badd2_u(((R1 >> sh) & 0x00030003u) | kMagic, m128),
-                                     badd2_u(((R1 >> (sh + 2)) & 0x00030003u) | kMagic, m128)};
-              mma_bf16(ores[2 * j + i], a, bh0, bh1);
-              mma_bf16(ores[2 * j + i], a, bl0, bl1);
-            }
-          }
-        } else {
-          static_assert(C::LDM4, "residual codes are INT2 or INT4");
-          // the group's 32-dim chunks by ldmatrix.trans: word = codes of dims
-          // 4g .. 4g+3 of the chunk (token 2q low half, 2q+1 high half, code i
-          // at bits 4i); m-tile 2 ch has m-rows g, g + 8 = dims 4g, 4g + 1,
-          // m-tile 2 ch + 1 dims 4g + 2, 4g + 3; operands (128 + c) - 128 = c
-          const uint32_t m128 = 0xC300C300u;   // {-128, -128}
-#pragma unroll
-          for (int ch = j * GROUP / 32; ch < (j + 1) * GROUP / 32; ++ch) {
-            const int m = (lane >> 3) & 1;
-            uint32_t v[2];   // (tokens 0-7, chunk ch), (tokens 8-15, chunk ch)
-            ldsm_x2_trans(smem_u32(st + C::OFF_CV + (wtok + m * 8 + r7) * C::CROW + ch * 16), v);
-#pragma unroll
-            for (int xy = 0; xy < 2; ++xy) {
-              const int sh = 8 * xy;
-              const uint32_t a[4] = {badd2_u(((v[0] >> sh) & 0x000F000Fu) | kMagic, m128),
-                                     badd2_u(((v[0] >> (sh + 4)) & 0x000F000Fu) | kMagic, m128),
-                                     badd2_u(((v[1] >> sh) & 0x000F000Fu) | kMagic, m128),
-                                     badd2_u(((v[1] >> (sh + 4)) & 0x000F000Fu) | kMagic, m128)};
-              mma_bf16(ores[2 * ch + xy], a, bh0, bh1);
-              mma_bf16(ores[2 * ch + xy], a, bl0, bl1);
-            }
-          }
-        }
-      }
-    }
-  };
-
-  // ---- main loop over this CTA's tiles ----
-  long long cur_head = -1, cur_first = 0;
-  int cur_nt = 0;
-  bool aborted = false;
-  reset_state();
-  TileCursor cur = first_cur;
-  for (int i = 0; i < n_my; ++i) {
-    const long long hd = cur.hd;
-    size_t row = 0;
-    int n = cur.n();
-    if (!p.page_table) tile_row(p, cur, row);   // paged: the stage's row, below
-    if (hd != cur_head) {
-      if (cur_head >= 0) {
-        flush_head(cur_head, cur_first, cur_nt);
-        reset_state();
-      }
-      cur_head = hd;
-      cur_first = cur.head_first();
-      cur_nt = cur.nt;
-      setup_head(hd);
-    }
-    cur.next(p);
-    const int s = i % STAGES;
-    bool ok = !aborted && !flags[0];
-    if (ok) ok = mbar_wait_bounded(&full_bar[s], (i / STAGES) & 1);
-    ok = __all_sync(FULL, ok);
-    if (!ok) {
-      if (!aborted && lane == 0) flag_error(p.status, 8u);
-      aborted = true;
-      flags[0] = 1;
-    }
-    if (!aborted && p.page_table) {
-      const unsigned long long r = stage_row[s];   // written before the stage's arrive
-      if (r == kBadRow) n = 0;
-      else row = (size_t)r;
-    }
-    if (!aborted && n > 0) {
-      tile_mma(ring + s * C::STAGE_BYTES, n, (int)((row * SB) & 15));
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty_bar[s]);
-  }
-  if (cur_head >= 0) flush_head(cur_head, cur_first, cur_nt);
-}
-
-// ---- host side ---------------------------------------------------------------
-
-template <int D, int G, int BITS, int GROUP, int RB>
-cudaError_t launch_gqa_t(const GqaParams& gp, cudaStream_t stream) {
-  using C = GCfg<D, G, BITS, GROUP, RB>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(decode_gqa_kernel<D, G, BITS, GROUP, RB>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
-  return launch_pdl(decode_gqa_kernel<D, G, BITS, GROUP, RB>, gp.p.ctas, kDecodeThreads,
-                    C::SMEM_BYTES, stream, gp);
-}
-
-template <int D, int G, int RB>
-cudaError_t launch_gqa_g(int bits, const GqaParams& gp, cudaStream_t stream) {
-  const int group = gp.p.group;
-  if (bits == 16) {
-    if constexpr (RB == 0) {
-      return launch_gqa_t<D, G, 16, 32, RB>(gp, stream);   // no scales are read
-    } else {
-      return group == 32 ? launch_gqa_t<D, G, 16, 32, RB>(gp, stream)
-                         : launch_gqa_t<D, G, 16, 64, RB>(gp, stream);
-    }
-  }
-  if (bits == 2)
-    return group == 32 ? launch_gqa_t<D, G, 2, 32, RB>(gp, stream)
-                       : launch_gqa_t<D, G, 2, 64, RB>(gp, stream);
-  if (bits == 4)
-    return group == 32 ? launch_gqa_t<D, G, 4, 32, RB>(gp, stream)
-                       : launch_gqa_t<D, G, 4, 64, RB>(gp, stream);
-  return cudaErrorInvalidValue;
-}
-
-template <int D, int RB>
-cudaError_t launch_gqa_d(int G, int bits, const GqaParams& gp, cudaStream_t stream) {
-  switch (G) {
-    case 2: return launch_gqa_g<D, 2, RB>(bits, gp, stream);
-    case 4: return launch_gqa_g<D, 4, RB>(bits, gp, stream);
-    case 8: return launch_gqa_g<D, 8, RB>(bits, gp, stream);
-    default: return cudaErrorInvalidValue;
-  }
-}
-
-}  // namespace
 
 cudaError_t launch_decode_gqa(int head_dim, int G, int bits, const DecodeParams& p,
                               cudaStream_t stream) {
@@ -1161,11 +21,11 @@ cudaError_t launch_decode_gqa(int head_dim, int G, int bits, const DecodeParams&
         !encode_bytes_map(&gp.tmap_v, p.rcodes_v, rows, rrow, kDecodeTile))
       return cudaErrorInvalidValue;
     if (p.ref_bits == 8) {
-      if (head_dim == 128) return launch_gqa_d<128, 8>(G, bits, gp, stream);
-      if (head_dim == 64) return launch_gqa_d<64, 8>(G, bits, gp, stream);
+      if (head_dim == 128) return launch_gqa_d128_r8(G, bits, gp, stream);
+      if (head_dim == 64) return launch_gqa_d64_r8(G, bits, gp, stream);
     } else {
-      if (head_dim == 128) return launch_gqa_d<128, 4>(G, bits, gp, stream);
-      if (head_dim == 64) return launch_gqa_d<64, 4>(G, bits, gp, stream);
+      if (head_dim == 128) return launch_gqa_d128_r4(G, bits, gp, stream);
+      if (head_dim == 64) return launch_gqa_d64_r4(G, bits, gp, stream);
     }
     return cudaErrorInvalidValue;
   }
@@ -1173,8 +33,8 @@ cudaError_t launch_decode_gqa(int head_dim, int G, int bits, const DecodeParams&
   if (!encode_rows_map(&gp.tmap_k, p.ref_k, rows, head_dim, kDecodeTile) ||
       !encode_rows_map(&gp.tmap_v, p.ref_v, rows, head_dim, kDecodeTile))
     return cudaErrorInvalidValue;
-  if (head_dim == 128) return launch_gqa_d<128, 0>(G, bits, gp, stream);
-  if (head_dim == 64) return launch_gqa_d<64, 0>(G, bits, gp, stream);
+  if (head_dim == 128) return launch_gqa_d128_r0(G, bits, gp, stream);
+  if (head_dim == 64) return launch_gqa_d64_r0(G, bits, gp, stream);
   return cudaErrorInvalidValue;
 }
 

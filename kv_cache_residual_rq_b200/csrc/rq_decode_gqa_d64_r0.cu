@@ -1,0 +1,13 @@
+// rq_decode_gqa_d64_r0.cu -- the grouped-query decode kernel's instances for
+// head_dim 64 and BF16 reference rows (one translation unit each, compiled in
+// parallel).
+#define RQ_GQA_KERNEL_DEFINITIONS
+#include "rq_decode_gqa.cuh"
+
+namespace rq {
+
+cudaError_t launch_gqa_d64_r0(int G, int bits, const GqaParams& gp, cudaStream_t stream) {
+  return launch_gqa_d<64, 0>(G, bits, gp, stream);
+}
+
+}  // namespace rq

@@ -59,6 +59,27 @@ __device__ __forceinline__ float flip_sign(float x, uint32_t neg) {
 }
 
 // ---------------------------------------------------------------------------
+// Bounds-checked builds (nvcc -DRQ_BOUNDS_CHECK: librq_bounds.so).  Before
+// an access whose index a kernel computes at run time, RQ_IN_BOUNDS(ok,
+// status, bit) tests that index against the extent of its buffer -- the
+// sizes the C ABI's size queries give for the call's shape -- or of its
+// shared-memory area.  A failed test raises `bit` in the call's status word
+// and the access is skipped; nothing traps.  In normal builds the test is
+// the constant true and the condition is never evaluated.
+// ---------------------------------------------------------------------------
+#ifdef RQ_BOUNDS_CHECK
+__device__ __forceinline__ bool rq_in_bounds(bool ok, uint32_t* status, uint32_t bit) {
+  if (!ok) atomicOr(status, bit);
+  return ok;
+}
+#define RQ_IN_BOUNDS(ok, status, bit) (::rq::rq_in_bounds((ok), (status), (bit)))
+#else
+#define RQ_IN_BOUNDS(ok, status, bit) (true)
+#endif
+constexpr uint32_t kStatusBounds = 128u;         // decode workspace status word
+constexpr uint32_t kEncodeStatusBounds = 8u;     // encoder status word
+
+// ---------------------------------------------------------------------------
 // mbarrier + bulk async copy (global -> shared, completion via mbarrier tx)
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

@@ -51,11 +51,15 @@ encode_kernel(const EncodeParams p) {
 
   for (long long row0 = warp * RPW; row0 < p.n_rows; row0 += nwarps * RPW) {
     const long long idx = row0 + slot;             // (head, token) index of this call
-    const bool valid = idx < p.n_rows;
     const long long hd = idx / p.ctx, t = idx % p.ctx;
     const long long src_row = hd * p.src_pitch + p.src_offset + t;
+    const bool valid = idx < p.n_rows &&
+                       RQ_IN_BOUNDS(src_row >= 0 && src_row < p.n_src_rows, p.status,
+                                    kEncodeStatusBounds);
     long long row = 0;                                             // destination row
-    const bool wvalid = valid && enc_dst_row(p, hd, t, row);
+    const bool wvalid = valid && enc_dst_row(p, hd, t, row) &&
+                        RQ_IN_BOUNDS(row >= 0 && row < p.n_dst_rows, p.status,
+                                     kEncodeStatusBounds);
     const size_t eoff = (size_t)src_row * D + li * DPL;
     const uint4 rw = valid ? ld_stream(p.ref + eoff) : make_uint4(0, 0, 0, 0);
     if (wvalid && p.ref_out)

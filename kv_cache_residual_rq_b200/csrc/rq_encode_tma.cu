@@ -27,6 +27,7 @@
 #include <cudaTypedefs.h>
 
 #include <cstring>
+#include <mutex>
 
 #include "rq_device.cuh"
 #include "rq_internal.h"
@@ -393,6 +394,10 @@ encode_tma_kernel(const __grid_constant__ EncodeTmaParams tp) {
     for (int t = blockIdx.x; ok && t < tp.n_tiles; t += gridDim.x) {
       for (int j = 0; j < per_tile; ++j, ++it) {
         const int s = (int)(it % SLOTS);
+        // the tile's first row lies inside the sources (the tensor maps zero-fill
+        // the rows of a partial tile past the end)
+        RQ_IN_BOUNDS((long long)t * C::R < p.n_rows && j < RQ_MAX_LOOPS + 1, p.status,
+                     kEncodeStatusBounds);
         if (it >= SLOTS && !mbar_wait_bounded(&empty[s], (uint32_t)((it / SLOTS - 1) & 1))) {
           atomicOr(&g_encode_status, 1u);
           ok = false;
@@ -416,6 +421,8 @@ encode_tma_kernel(const __grid_constant__ EncodeTmaParams tp) {
   const int rw = lane % C::RPW;          // row within the warp
   const int q = lane / C::RPW;           // which 64 coordinates of the row
   const int r = warp * C::RPW + rw;      // row within the tile
+  // shared-memory reads of this lane: line r of box q of a slot
+  if (!RQ_IN_BOUNDS(r < C::R && q < C::NBOX, p.status, kEncodeStatusBounds)) return;
   long long it = 0;
   for (int t = blockIdx.x; t < tp.n_tiles; t += gridDim.x) {
     const long long idx = (long long)t * C::R + r;
@@ -423,7 +430,11 @@ encode_tma_kernel(const __grid_constant__ EncodeTmaParams tp) {
     const uint32_t hd32 = (uint32_t)idx / (uint32_t)p.ctx;
     const long long hd = hd32, tok = idx - (long long)hd32 * p.ctx;
     long long row = 0;
-    const bool valid = idx < p.n_rows && enc_dst_row(p, hd, tok, row);
+    bool valid = idx < p.n_rows && enc_dst_row(p, hd, tok, row);
+    // every output of the row (codes, scales, reference copy) is written at
+    // destination row `row`
+    if (valid)
+      valid = RQ_IN_BOUNDS(row >= 0 && row < p.n_dst_rows, p.status, kEncodeStatusBounds);
 
     // reference: -D_i ref_i (BF16 reference), kept for every loop of these
     // rows; or, compressed reference, the rotated reference is quantised
@@ -538,6 +549,21 @@ cudaError_t launch_encode_tma(int head_dim, int group, const EncodeParams& p, in
   if (head_dim == 64 && group == 32) return launch_t<64, 32>(tp, num_sms, stream);
   if (head_dim == 64 && group == 64) return launch_t<64, 64>(tp, num_sms, stream);
   return cudaErrorInvalidValue;
+}
+
+uint32_t* encode_status_ptr() {
+  constexpr int kMaxDevices = 64;
+  static uint32_t* addr[kMaxDevices] = {nullptr};
+  static std::mutex mu;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_encode_status) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<uint32_t*>(ptr);
+  }
+  return addr[dev];
 }
 
 cudaError_t encode_take_status(uint32_t* bits) {

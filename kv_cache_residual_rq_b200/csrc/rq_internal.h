@@ -63,6 +63,11 @@ struct EncodeParams {
   uint32_t* ref_codes;               // compressed reference: codes and scales out
   uint16_t* ref_scales;
   uint64_t seed;
+  // extents the bounds-checked build tests indices against: rows of the
+  // sources (heads * src_pitch) and of the outputs (heads * dst_pitch, or a
+  // paged pool's n_pages * kv_heads * 64), and the encoders' status word
+  long long n_src_rows, n_dst_rows;
+  uint32_t* status;
 };
 
 #ifdef __CUDACC__
@@ -98,6 +103,9 @@ cudaError_t launch_encode_tma(int head_dim, int group, const EncodeParams& p, in
                               cudaStream_t stream);
 // read and clear the sticky error bits of the encoders on the current device
 cudaError_t encode_take_status(uint32_t* bits);
+// device address of that status word on the current device (looked up once
+// per device); null if the runtime cannot provide it
+uint32_t* encode_status_ptr();
 
 // ---------------------------------------------------------------------------
 // reconstruction (the format's decoder)
@@ -113,6 +121,7 @@ struct ReconstructParams {
   int ctx, pitch;
   int out_bf16;
   uint64_t seed;
+  uint32_t* status;           // the encoders' status word (bounds-checked build)
 };
 
 cudaError_t launch_reconstruct(int head_dim, int group, int bits, const ReconstructParams& p,

@@ -42,9 +42,12 @@ reconstruct_kernel(const ReconstructParams p) {
 
   for (long long row0 = warp * RPW; row0 < p.n_rows; row0 += nwarps * RPW) {
     const long long idx = row0 + slot;
-    const bool valid = idx < p.n_rows;
     const long long hd = idx / p.ctx, t = idx % p.ctx;
     const long long row = hd * p.pitch + t;
+    // every array of the call holds heads * pitch rows
+    const bool valid = idx < p.n_rows &&
+                       RQ_IN_BOUNDS(row >= 0 && row < (p.n_rows / p.ctx) * p.pitch, p.status,
+                                    kEncodeStatusBounds);
     const size_t eoff = (size_t)row * D + li * DPL;
     uint4 rw = make_uint4(0, 0, 0, 0);
     if constexpr (RB == 0) {

@@ -257,7 +257,7 @@ if __name__ == "__main__":
 # the bench's per-workload block: back-to-back launches with sampled clocks
 # ---------------------------------------------------------------------------
 
-def _back_to_back(fn, stream, target_s, sampler):
+def _back_to_back(fn, stream, target_s, sampler, label="timed launches"):
     """Average duration of `fn` launched back to back on `stream` (CUDA events
     around n launches, n chosen so the timed region lasts about target_s),
     with the SM clock sampled during the timed region."""
@@ -277,10 +277,12 @@ def _back_to_back(fn, stream, target_s, sampler):
     if sampler is not None:
         sampler.start()
         time.sleep(0.25)
+    torch.cuda.nvtx.range_push(label)
     a.record(stream)
     for _ in range(n):
         fn()
     b.record(stream)
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     clk = sampler.stop() if sampler is not None else {}
     return a.elapsed_time(b) / 1e3 / n, n, clk
@@ -334,9 +336,10 @@ def bench_workloads(peak, make_sampler, target_s=0.4):
                 q = synth.query(w, 0, loop, dev)
             fn = lambda: rq.rq_decode_attention(shape, q, refk, refv, *args, bits, w.seed, 0.0,
                                                 out, ws, stream=st)
-            t, n, clk = _back_to_back(fn, stream, target_s, make_sampler())
-            per_call[bits] = t
             label = f"loop {loop} INT{bits}" if loop else f"loop {w.loops} BF16 reference"
+            t, n, clk = _back_to_back(fn, stream, target_s, make_sampler(),
+                                      f"{w.name} decode {label}")
+            per_call[bits] = t
             out_entries.append(_entry(f"{w.name} decode {label}", t, n, clk,
                                       decode_bytes(w, bits), peak, G=w.G))
             del args
@@ -367,7 +370,7 @@ def bench_workloads(peak, make_sampler, target_s=0.4):
     scales = [rq.alloc_scales(shape, b, dev) for b in w.bits]
     fn = lambda: rq.rq_encode(shape, list(x[:w.loops - 1]), x[w.loops - 1], list(w.bits),
                               w.seed, codes, scales, st)
-    t, n, clk = _back_to_back(fn, stream, target_s, make_sampler())
+    t, n, clk = _back_to_back(fn, stream, target_s, make_sampler(), f"{w.name} encode")
     nb = encode_bytes(w, rows_batch * H * T)
     out_entries.append(_entry(f"{w.name} encode (24 layers x K/V x {w.loops} loops, one call)",
                               t, n, clk, nb, peak, rows=rows_batch * H * T))

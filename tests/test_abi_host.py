@@ -47,6 +47,15 @@ def test_library_exports_every_declared_symbol():
         assert hasattr(lib, name), name
 
 
+def test_bounds_checked_library_exports_every_declared_symbol():
+    # librq_bounds.so: the same ABI, built with every computed index checked
+    if rq_build._stale(rq_build.LIB_BOUNDS):
+        pytest.skip("librq_bounds.so not built from the current sources")
+    lib = ctypes.CDLL(rq_build.LIB_BOUNDS)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
 def test_version_and_status_strings():
     assert rq.rq_version() >= 100
     for s in range(6):
