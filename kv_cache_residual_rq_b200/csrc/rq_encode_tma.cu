@@ -8,21 +8,25 @@
 // identical binary32 operations in the identical order.
 //
 // Used when every source array is a contiguous [rows][head_dim] block (the
-// whole-cache encode).  One CTA per SM:
+// whole-cache encode).  This file holds the plain mode (absmax codes, one
+// least-squares scale); the refit and compressed-reference modes, whose
+// scales must follow the specification's summation order, are in
+// rq_encode_tma_fixed.cu.  One CTA per SM:
 //   * a producer warp streams tiles of R rows -- the reference tile, then the
 //     same rows of every quantised loop -- into a ring of shared-memory slots
 //     with 2-D tensor copies (128-byte swizzle), completion on mbarriers;
-//   * each consumer warp owns 8 rows (head_dim 128; 16 rows for 64) of the
-//     tile, 4 (2) lanes per row, 32 consecutive coordinates per lane, so a
-//     scale group of 32 is one lane and needs no cross-lane reduction.
+//   * a consumer lane owns 64 consecutive coordinates of a row (two lanes per
+//     row at head_dim 128, one at 64), as 32 packed pairs {c_m, c_m+32}.
 // Per lane and loop: residual and seeded sign in one mixed bf16 x bf16 + f32
 // fma per coordinate (D_i x_i + (-D_i ref_i), exact product, one rounding);
-// the Walsh-Hadamard stages 1..16 in registers as packed fp32x2 adds and
-// subtracts (stage 16 scalar), stages 32 and 64 by shfl.xor; codes from
-// floor(u) obtained as (u + 1.5*2^23) rounded down, whose bit pattern is
-// 0x4B400000 + floor(u), packed by shifted adds with one constant correction
-// per word.  Every wait is bounded; on a timeout the kernel raises a bit in
-// the encoder status word and stops.
+// the Walsh-Hadamard strides 1..16 as packed fp32x2 adds and subtracts,
+// stride 32 inside each pair, stride 64 (head_dim 128) by shfl.xor; the
+// lane's two 32-wide blocks are the two scale groups of 32 (or together one
+// of 64), quantised side by side as packed pairs; codes from floor(u)
+// obtained as (u + 1.5*2^23) rounded down, whose bit pattern is 0x4B400000 +
+// floor(u), packed by shifted adds with one constant correction per word.
+// Every wait is bounded; on a timeout the kernel raises a bit in the encoder
+// status word and stops.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -187,22 +191,17 @@ __device__ __forceinline__ void rotate64(float2 (&P)[32], int q) {
 
 // One quantisation pass over the lane's two 32-coordinate blocks, A = P[].x
 // and B = P[].y, with steps 1/(2 inv.x), 1/(2 inv.y): code words (A's BITS
-// words, then B's), <y,l> and <l,l> of each block (.x, .y).
-// FIXED: <y,l> in the fixed order (fma chains over coordinates 0..15 and
-// 16..31 of a block, the two runs added), which the least-squares refits and
-// the compressed reference need bit for bit.  Otherwise the sum runs as four
-// interleaved chains (the plain encode's scale is an fp16 rounding of it, so
-// its order is free).  Code words are integer sums: any order.
-template <int BITS, bool CLAMP, bool FIXED, bool WANT_LV = false>
+// words, then B's), <y,l> and <l,l> of each block (.x, .y).  The scale is
+// kept only as its fp16 rounding, so <y,l> runs as four interleaved chains;
+// code words are integer sums (any order).
+template <int BITS>
 __device__ __forceinline__ void quant_pass(const float2 (&P)[32], float2 inv2,
                                            uint32_t (&w)[2 * BITS], float2& dot_out,
-                                           float2& nrm_out, float2* lv_out = nullptr) {
+                                           float2& nrm_out) {
   constexpr int PER = 32 / BITS;                    // codes per word
   const float2 mg = make_float2(kFloorMagic, kFloorMagic);
   const float2 two = make_float2(2.0f, 2.0f), one = make_float2(1.0f, 1.0f);
-  constexpr float lo = kFloorMagic - (float)(1 << (BITS - 1));
-  constexpr float hi = kFloorMagic + (float)((1 << (BITS - 1)) - 1);
-  constexpr int NC = FIXED ? 2 : 4;                 // independent chains
+  constexpr int NC = 4;                             // independent chains
   float2 dot[NC], nrm[NC];
 #pragma unroll
   for (int c = 0; c < NC; ++c) {
@@ -213,32 +212,22 @@ __device__ __forceinline__ void quant_pass(const float2 (&P)[32], float2 inv2,
   for (int k = 0; k < 2 * BITS; ++k) w[k] = 0;
 #pragma unroll
   for (int m = 0; m < 32; ++m) {
-    const int c = FIXED ? m / 16 : m % 4;           // FIXED: chain = run of 16
+    const int c = m % NC;
     const float2 u = __fmul2_rn(P[m], inv2);
-    float2 t = __fadd2_rd(u, mg);                   // 1.5*2^23 + floor(u), exact
-    if constexpr (CLAMP) {
-      t.x = fminf(fmaxf(t.x, lo), hi);
-      t.y = fminf(fmaxf(t.y, lo), hi);
-    }
+    const float2 t = __fadd2_rd(u, mg);             // 1.5*2^23 + floor(u), exact
     w[m / PER] += __float_as_uint(t.x) << (BITS * (m % PER));
     w[BITS + m / PER] += __float_as_uint(t.y) << (BITS * (m % PER));
     const float2 fl = fsub2(t, mg);                 // floor(u)
     const float2 lv = __ffma2_rn(fl, two, one);     // level 2 floor(u) + 1 = 2c - (2^b - 1)
-    if constexpr (WANT_LV) lv_out[m] = lv;
     dot[c] = __ffma2_rn(P[m], lv, dot[c]);
     if constexpr (BITS != 2) nrm[c] = __ffma2_rn(lv, lv, nrm[c]);
   }
   // every field received (0x4B400000 + floor(u)); code c = floor(u) + 2^(b-1)
   constexpr uint32_t kOff = kFloorMagicBits - (1u << (BITS - 1));
-  constexpr uint32_t kSpread =
-      BITS == 2 ? 0x55555555u : (BITS == 4 ? 0x11111111u : 0x01010101u);
+  constexpr uint32_t kSpread = BITS == 2 ? 0x55555555u : 0x11111111u;
 #pragma unroll
   for (int k = 0; k < 2 * BITS; ++k) w[k] -= kOff * kSpread;
-  if constexpr (FIXED) {
-    dot_out = __fadd2_rn(dot[0], dot[1]);           // run 0 + run 1 of each block
-  } else {
-    dot_out = __fadd2_rn(__fadd2_rn(dot[0], dot[1]), __fadd2_rn(dot[2], dot[3]));
-  }
+  dot_out = __fadd2_rn(__fadd2_rn(dot[0], dot[1]), __fadd2_rn(dot[2], dot[3]));
   if constexpr (BITS == 2) {
     // <l, l> = 32 + 8 * (number of outer levels +-3, i.e. codes 0 and 3,
     // whose two bits are equal): an exact integer
@@ -249,10 +238,7 @@ __device__ __forceinline__ void quant_pass(const float2 (&P)[32], float2 inv2,
     nrm_out = make_float2((float)(32u + 8u * ea), (float)(32u + 8u * eb));
   } else {
     // integers below 2^24 in every partial sum: exact in any order
-    float2 n = nrm[0];
-#pragma unroll
-    for (int c = 1; c < NC; ++c) n = __fadd2_rn(n, nrm[c]);
-    nrm_out = n;
+    nrm_out = __fadd2_rn(__fadd2_rn(nrm[0], nrm[1]), __fadd2_rn(nrm[2], nrm[3]));
   }
 }
 
@@ -260,13 +246,10 @@ __device__ __forceinline__ float2 f2(float x) { return make_float2(x, x); }
 
 // Codes and scales of the lane's 64 rotated coordinates: blocks A (P[].x)
 // and B (P[].y) are one 32-wide scale group each, or together one group of
-// 64.  The absmax step, then `iters` least-squares refits (nearest level of
-// the current scale, then the scale refitted); a group whose scale is below
-// FLT_MIN keeps its codes.  WANT_Z: z = s16 * l (the rotated reconstruction).
-template <int BITS, int GROUP, bool FIXED, bool WANT_Z = false>
+// 64.  The absmax step, then the least-squares scale of those codes.
+template <int BITS, int GROUP>
 __device__ __forceinline__ void quantize_store(const float2 (&P)[32], uint32_t* codes_row,
-                                               uint16_t* scales_row, int q, bool valid,
-                                               int iters, float2* z = nullptr) {
+                                               uint16_t* scales_row, int q, bool valid) {
   // absmax of each block as four interleaved chains (max is exact in any order)
   float ax[4], ay[4];
 #pragma unroll
@@ -289,53 +272,19 @@ __device__ __forceinline__ void quantize_store(const float2 (&P)[32], uint32_t* 
   inv.y = (GROUP == 64) ? inv.x : ((amy < 1.17549435e-38f) ? 0.0f : __fdiv_rn(outer, amy));
   uint32_t w[2 * BITS];
   float2 d, n;
-  quant_pass<BITS, false, FIXED, WANT_Z>(P, inv, w, d, n, z);
+  quant_pass<BITS>(P, inv, w, d, n);
   if constexpr (GROUP == 64) {
     d = f2(d.x + d.y);                              // block A + block B
     n = f2(n.x + n.y);
   }
-  // least-squares scale: IEEE division where later steps depend on its bits
-  // (refits, the compressed reference); else only its fp16 rounding is kept
+  // least-squares scale; only its fp16 rounding is kept, so the fast
+  // reciprocal division serves
   float2 s;
-  if constexpr (FIXED) {
-    s.x = d.x / n.x;
-    s.y = (GROUP == 64) ? s.x : d.y / n.y;
-  } else {
-    s.x = __fdividef(d.x, n.x);
-    s.y = (GROUP == 64) ? s.x : __fdividef(d.y, n.y);
-  }
-  for (int k = 0; k < iters; ++k) {
-    const bool lx = s.x >= 1.17549435e-38f, ly = s.y >= 1.17549435e-38f;
-    float2 inv2;
-    inv2.x = lx ? __fdiv_rn(0.5f, s.x) : 0.0f;
-    inv2.y = (GROUP == 64) ? inv2.x : (ly ? __fdiv_rn(0.5f, s.y) : 0.0f);
-    uint32_t w2[2 * BITS];
-    float2 d2, n2;
-    quant_pass<BITS, true, true>(P, inv2, w2, d2, n2);
-    if constexpr (GROUP == 64) {
-      d2 = f2(d2.x + d2.y);
-      n2 = f2(n2.x + n2.y);
-    }
-    if (lx) {
-#pragma unroll
-      for (int j = 0; j < BITS; ++j) w[j] = w2[j];
-      s.x = d2.x / n2.x;
-    }
-    if (ly) {
-#pragma unroll
-      for (int j = BITS; j < 2 * BITS; ++j) w[j] = w2[j];
-      s.y = (GROUP == 64) ? s.x : d2.y / n2.y;
-    }
-  }
+  s.x = __fdividef(d.x, n.x);
+  s.y = (GROUP == 64) ? s.x : __fdividef(d.y, n.y);
   s.x = fminf(fmaxf(s.x, -65504.0f), 65504.0f);
   s.y = fminf(fmaxf(s.y, -65504.0f), 65504.0f);
   const __half hx = __float2half_rn(s.x), hy = __float2half_rn(s.y);
-  if constexpr (WANT_Z) {
-    // the reconstructed rotated block s16 * l (exact: 11 x 9 significant bits)
-    const float2 s2 = make_float2(__half2float(hx), __half2float(hy));
-#pragma unroll
-    for (int m = 0; m < 32; ++m) z[m] = __fmul2_rn(z[m], s2);
-  }
   if (!valid) return;
   uint4* o = reinterpret_cast<uint4*>(codes_row + 2 * BITS * q);
 #pragma unroll
@@ -348,16 +297,12 @@ __device__ __forceinline__ void quantize_store(const float2 (&P)[32], uint32_t* 
     scales_row[q] = __half_as_ushort(hx);
 }
 
-// MODE 0: BF16 reference, no refits; 1: BF16 reference with least-squares
-// refits; 2: compressed reference.  Separate instantiations keep the plain
-// encode free of the other modes' registers and branches.
-template <int D, int GROUP, int CW, int MODE>
+// The plain mode: BF16 reference, absmax codes, one least-squares scale.
+template <int D, int GROUP, int CW>
 __global__ void __launch_bounds__(ECfg<D, CW>::THREADS, 1)
 encode_tma_kernel(const __grid_constant__ EncodeTmaParams tp) {
   using C = ECfg<D, CW>;
   constexpr int SLOTS = C::SLOTS;
-  constexpr bool FIXED = (MODE != 0);
-  const int iters = (MODE == 0) ? 0 : tp.p.refine_iters;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -396,8 +341,8 @@ encode_tma_kernel(const __grid_constant__ EncodeTmaParams tp) {
         const int s = (int)(it % SLOTS);
         // the tile's first row lies inside the sources (the tensor maps zero-fill
         // the rows of a partial tile past the end)
-        RQ_IN_BOUNDS((long long)t * C::R < p.n_rows && j < RQ_MAX_LOOPS + 1, p.status,
-                     kEncodeStatusBounds);
+        (void)RQ_IN_BOUNDS((long long)t * C::R < p.n_rows && j < RQ_MAX_LOOPS + 1, p.status,
+                           kEncodeStatusBounds);
         if (it >= SLOTS && !mbar_wait_bounded(&empty[s], (uint32_t)((it / SLOTS - 1) & 1))) {
           atomicOr(&g_encode_status, 1u);
           ok = false;
@@ -436,10 +381,7 @@ encode_tma_kernel(const __grid_constant__ EncodeTmaParams tp) {
     if (valid)
       valid = RQ_IN_BOUNDS(row >= 0 && row < p.n_dst_rows, p.status, kEncodeStatusBounds);
 
-    // reference: -D_i ref_i (BF16 reference), kept for every loop of these
-    // rows; or, compressed reference, the rotated reference is quantised
-    // (its codes stored) and zr holds its reconstruction s16 * l, which is
-    // subtracted from every loop's rotated row
+    // reference: -D_i ref_i, kept for every loop of these rows
     int s = (int)(it % SLOTS);
     if (!mbar_wait_bounded(&full[s], (uint32_t)((it / SLOTS) & 1))) {
       atomicOr(&g_encode_status, 4u);
@@ -453,21 +395,7 @@ encode_tma_kernel(const __grid_constant__ EncodeTmaParams tp) {
       for (int c = 0; c < 8; ++c) o[c] = *reinterpret_cast<const uint4*>(rp + ((c ^ (r & 7)) << 4));
     }
     float2 zr[32];
-    if constexpr (MODE != 2) {
-      row_fma<D, CW, false>(slot, ndtab, r, q, zr, zr);
-    } else {
-      float2 P[32];
-      row_fma<D, CW, false>(slot, dtab, r, q, zr, P);         // D_i ref_i, exact
-      rotate64<D, C::RPW>(P, q);
-      if (p.ref_bits == 8)
-        quantize_store<8, GROUP, true, true>(P, p.ref_codes + (size_t)row * (D / 4),
-                                             p.ref_scales + (size_t)row * (D / GROUP), q,
-                                             valid, 0, zr);
-      else
-        quantize_store<4, GROUP, true, true>(P, p.ref_codes + (size_t)row * (D / 8),
-                                             p.ref_scales + (size_t)row * (D / GROUP), q,
-                                             valid, 0, zr);
-    }
+    row_fma<D, CW, false>(slot, ndtab, r, q, zr, zr);
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
     ++it;
@@ -478,48 +406,34 @@ encode_tma_kernel(const __grid_constant__ EncodeTmaParams tp) {
         atomicOr(&g_encode_status, 4u);
         return;
       }
-      // BF16 reference: y = D_i x_i + (-D_i ref_i), one rounding, then rotated.
-      // Compressed reference: D_i x_i (exact), rotated, then e = RN(y - zr).
+      // y = D_i x_i + (-D_i ref_i), one rounding, then rotated
       float2 P[32];
-      row_fma<D, CW, MODE != 2>(ring + s * C::SLOT_BYTES, dtab, r, q, zr, P);
+      row_fma<D, CW, true>(ring + s * C::SLOT_BYTES, dtab, r, q, zr, P);
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
       ++it;
       rotate64<D, C::RPW>(P, q);
-      if constexpr (MODE == 2) {
-#pragma unroll
-        for (int m = 0; m < 32; ++m) P[m] = fsub2(P[m], zr[m]);
-      }
       const int l = tp.active[j];
       if (p.bits[l] == 2)
-        quantize_store<2, GROUP, FIXED>(P, p.codes[l] + (size_t)row * (D / 16),
-                                        p.scales[l] + (size_t)row * (D / GROUP), q, valid,
-                                        iters);
+        quantize_store<2, GROUP>(P, p.codes[l] + (size_t)row * (D / 16),
+                                 p.scales[l] + (size_t)row * (D / GROUP), q, valid);
       else
-        quantize_store<4, GROUP, FIXED>(P, p.codes[l] + (size_t)row * (D / 8),
-                                        p.scales[l] + (size_t)row * (D / GROUP), q, valid,
-                                        iters);
+        quantize_store<4, GROUP>(P, p.codes[l] + (size_t)row * (D / 8),
+                                 p.scales[l] + (size_t)row * (D / GROUP), q, valid);
     }
   }
 }
 
-template <int D, int GROUP, int MODE>
-cudaError_t launch_tm(const EncodeTmaParams& tp, int num_sms, cudaStream_t stream) {
+template <int D, int GROUP>
+cudaError_t launch_t(const EncodeTmaParams& tp, int num_sms, cudaStream_t stream) {
   constexpr int CW = consumer_warps<D>();
   using C = ECfg<D, CW>;
-  cudaError_t e = cudaFuncSetAttribute(encode_tma_kernel<D, GROUP, CW, MODE>,
+  cudaError_t e = cudaFuncSetAttribute(encode_tma_kernel<D, GROUP, CW>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   const int grid = tp.n_tiles < num_sms ? tp.n_tiles : num_sms;
-  return launch_pdl(encode_tma_kernel<D, GROUP, CW, MODE>, (unsigned)grid, C::THREADS, C::SMEM,
-                    stream, tp);
-}
-
-template <int D, int GROUP>
-cudaError_t launch_t(const EncodeTmaParams& tp, int num_sms, cudaStream_t stream) {
-  if (tp.p.ref_bits != 0) return launch_tm<D, GROUP, 2>(tp, num_sms, stream);
-  if (tp.p.refine_iters > 0) return launch_tm<D, GROUP, 1>(tp, num_sms, stream);
-  return launch_tm<D, GROUP, 0>(tp, num_sms, stream);
+  return launch_pdl(encode_tma_kernel<D, GROUP, CW>, (unsigned)grid, C::THREADS, C::SMEM, stream,
+                    tp);
 }
 
 }  // namespace
@@ -530,6 +444,9 @@ int encode_tma_rows_per_tile(int head_dim) {
 
 cudaError_t launch_encode_tma(int head_dim, int group, const EncodeParams& p, int num_sms,
                               cudaStream_t stream) {
+  // least-squares refits and the compressed reference: rq_encode_tma_fixed.cu
+  if (p.ref_bits != 0 || p.refine_iters > 0)
+    return launch_encode_tma_fixed(head_dim, group, p, num_sms, stream);
   EncodeTmaParams tp;
   std::memset(&tp, 0, sizeof tp);
   tp.p = p;

@@ -101,6 +101,10 @@ cudaError_t launch_encode(int head_dim, int group, const EncodeParams& p, int nu
 constexpr long long kEncodeTmaMaxRows = (1ll << 31) - 512;
 cudaError_t launch_encode_tma(int head_dim, int group, const EncodeParams& p, int num_sms,
                               cudaStream_t stream);
+// its least-squares-refit and compressed-reference modes (called by
+// launch_encode_tma; rq_encode_tma_fixed.cu)
+cudaError_t launch_encode_tma_fixed(int head_dim, int group, const EncodeParams& p, int num_sms,
+                                    cudaStream_t stream);
 // read and clear the sticky error bits of the encoders on the current device
 cudaError_t encode_take_status(uint32_t* bits);
 // device address of that status word on the current device (looked up once
