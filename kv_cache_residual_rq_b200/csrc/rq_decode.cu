@@ -52,7 +52,7 @@ namespace {
 
 constexpr int kThreads = kDecodeThreads;
 
-template <int D, int G, int BITS, int RB>
+template <int D, int G, int BITS>
 struct Cfg {
   static constexpr int DPL = (G >= 4) ? 4 : 8;              // dims per lane
   static constexpr int LPT = D / DPL;                       // lanes per token
@@ -64,8 +64,7 @@ struct Cfg {
   static constexpr int CH = (G == 1) ? LPT / 2 : (STEPS < 4 ? STEPS : 4);
   static constexpr bool RES = (BITS != 16);
   static constexpr bool LUT = (G == 1 && BITS == 2);
-  // reference rows: bf16 (RB 0) or compressed-reference codes of RB bits
-  static constexpr int KROW = RB ? D * RB / 8 : D * 2;
+  static constexpr int KROW = D * 2;                        // BF16 reference row bytes
   static constexpr int CROW = RES ? D * BITS / 8 : 0;       // code bytes per token
   static constexpr int CWORDS = CROW / 4;
   static constexpr int SC_BYTES = RES ? TILE * (2 * D / 32) + 32 : 0;
@@ -75,11 +74,8 @@ struct Cfg {
   static constexpr int OFF_CV = OFF_CK + TILE * CROW;
   static constexpr int OFF_SK = OFF_CV + TILE * CROW;
   static constexpr int OFF_SV = OFF_SK + SC_BYTES;
-  static constexpr int RSC_BYTES = RB ? TILE * (2 * D / 32) + 32 : 0;   // reference scales
-  static constexpr int OFF_RSK = OFF_SV + SC_BYTES;
-  static constexpr int OFF_RSV = OFF_RSK + RSC_BYTES;
-  static constexpr int STAGE_BYTES = OFF_RSV + RSC_BYTES;
-  static constexpr int STAGES = (RES && !RB) ? 2 : 3;
+  static constexpr int STAGE_BYTES = OFF_SV + SC_BYTES;
+  static constexpr int STAGES = RES ? 2 : 3;
   static constexpr int RING_BYTES = STAGES * STAGE_BYTES;
   // K-residual table: [256 byte values][32 slices] floats
   static constexpr int LUT_FLOATS = LUT ? 256 * 32 : 0;
@@ -155,69 +151,10 @@ __host__ __device__ constexpr float pos_factor(int k) {
                            : 1.0f / (float)(1u << (BITS * k));
 }
 
-// The lane's DPL compressed-reference codes (RB bits each, at byte address
-// p in shared memory) as floats c_k * 2^pos_k; 2^-pos_k is ref_pos_factor.
-template <int RB, int DPL>
-__device__ __forceinline__ void ref_codes_positional(const unsigned char* p, float (&f)[DPL]) {
-  if constexpr (RB == 8) {
-    // two codes per 16-bit half, at bit 0 and bit 8
-    uint32_t w[DPL / 4];
-    if constexpr (DPL == 8) {
-      const uint2 v = *reinterpret_cast<const uint2*>(p);
-      w[0] = v.x;
-      w[1] = v.y;
-    } else {
-      w[0] = *reinterpret_cast<const uint32_t*>(p);
-    }
-#pragma unroll
-    for (int k = 0; k < DPL; ++k) {
-      const uint32_t h = (w[k / 4] >> (16 * ((k / 2) & 1))) & 0xFFFFu;
-      f[k] = code_at(h & (0xFFu << (8 * (k & 1))));
-    }
-  } else {
-    uint32_t x;
-    if constexpr (DPL == 8) x = *reinterpret_cast<const uint32_t*>(p);
-    else x = *reinterpret_cast<const uint16_t*>(p);
-    codes_positional<4, DPL>(x, f);
-  }
-}
-
-template <int RB, int DPL>
-__host__ __device__ constexpr float ref_pos_factor(int k) {
-  return RB == 8 ? ((k & 1) ? 1.0f / 256.0f : 1.0f) : pos_factor<4, DPL>(k);
-}
-
-// sum_k a_k b_k + c over 4 byte lanes, a signed or unsigned, b unsigned
-__device__ __forceinline__ int dp4a_su(uint32_t a, uint32_t b, int c) {
-  int d;
-  asm("dp4a.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
-}
-__device__ __forceinline__ int dp4a_uu(uint32_t a, uint32_t b, int c) {
-  int d;
-  asm("dp4a.u32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
-}
-
-// acc + w * (1024 + c) for the half (0 low, 1 high) of a packed pair of fp16
-// values 0x6400 | c, w an fp16 weight: one rounding, fp32 accumulator
-template <int H>
-__device__ __forceinline__ float fma_f16_half(uint32_t w16x2, uint32_t cpair, float acc) {
-  if constexpr (H == 0)
-    asm("{\n\t.reg .b16 wl, wh, cl, ch;\n\tmov.b32 {wl, wh}, %1;\n\tmov.b32 {cl, ch}, %2;\n\t"
-        "fma.rn.f32.f16 %0, wl, cl, %0;\n\t}"
-        : "+f"(acc) : "r"(w16x2), "r"(cpair));
-  else
-    asm("{\n\t.reg .b16 wl, wh, cl, ch;\n\tmov.b32 {wl, wh}, %1;\n\tmov.b32 {cl, ch}, %2;\n\t"
-        "fma.rn.f32.f16 %0, wl, ch, %0;\n\t}"
-        : "+f"(acc) : "r"(w16x2), "r"(cpair));
-  return acc;
-}
-
-template <int D, int G, int BITS, int RB>
+template <int D, int G, int BITS>
 __global__ void __launch_bounds__(kThreads, 2)
 decode_kernel(const DecodeParams p) {
-  using C = Cfg<D, G, BITS, RB>;
+  using C = Cfg<D, G, BITS>;
   constexpr int DPL = C::DPL, LPT = C::LPT, TPS = C::TPS, TILE = C::TILE;
   constexpr int STAGES = C::STAGES, CH = C::CH;
   constexpr unsigned FULL = 0xffffffffu;
@@ -271,7 +208,7 @@ decode_kernel(const DecodeParams p) {
     return (uint32_t)(((start + (size_t)n * SB + 15) & ~(size_t)15) - (start & ~(size_t)15));
   };
   // scale bytes a stage holds (per array), for the bounds-checked build
-  constexpr int SCAP = C::RES ? C::SC_BYTES : (RB != 0 ? C::RSC_BYTES : 0);
+  constexpr int SCAP = C::RES ? C::SC_BYTES : 0;
   // a tile's copies stay inside the call's arrays and the stage
   auto copies_in_bounds = [&](size_t row, int n) {
     const size_t lo = (row * SB) & ~(size_t)15;
@@ -323,20 +260,9 @@ decode_kernel(const DecodeParams p) {
           sc_bytes = (uint32_t)(((start + (size_t)n * SB + 15) & ~(size_t)15) - sc_lo);
           bytes += 2u * n * C::CROW + 2u * sc_bytes;
         }
-        if constexpr (RB != 0) bytes += 2u * sc_bytes_ref(row, n);
         mbar_arrive_expect_tx(&full_bar[s], bytes);
-        if constexpr (RB == 0) {
-          bulk_g2s(st + C::OFF_K, p.ref_k + row * D, n * C::KROW, &full_bar[s]);
-          bulk_g2s(st + C::OFF_V, p.ref_v + row * D, n * C::KROW, &full_bar[s]);
-        } else {
-          bulk_g2s(st + C::OFF_K, p.rcodes_k + row * (C::KROW / 4), n * C::KROW, &full_bar[s]);
-          bulk_g2s(st + C::OFF_V, p.rcodes_v + row * (C::KROW / 4), n * C::KROW, &full_bar[s]);
-          const size_t rlo = (row * SB) & ~(size_t)15;
-          bulk_g2s(st + C::OFF_RSK, reinterpret_cast<const unsigned char*>(p.rscales_k) + rlo,
-                   sc_bytes_ref(row, n), &full_bar[s]);
-          bulk_g2s(st + C::OFF_RSV, reinterpret_cast<const unsigned char*>(p.rscales_v) + rlo,
-                   sc_bytes_ref(row, n), &full_bar[s]);
-        }
+        bulk_g2s(st + C::OFF_K, p.ref_k + row * D, n * C::KROW, &full_bar[s]);
+        bulk_g2s(st + C::OFF_V, p.ref_v + row * D, n * C::KROW, &full_bar[s]);
         if constexpr (C::RES) {
           bulk_g2s(st + C::OFF_CK, p.codes_k + row * C::CWORDS, n * C::CROW, &full_bar[s]);
           bulk_g2s(st + C::OFF_CV, p.codes_v + row * C::CWORDS, n * C::CROW, &full_bar[s]);
@@ -393,13 +319,6 @@ decode_kernel(const DecodeParams p) {
   // per-lane constants of the current head (scores are accumulated without
   // the softmax scale, which multiplies each reduced score once)
   uint32_t qbf[G][NP];                // q as packed bf16 pairs
-  float2 qr[G][NP];                   // compressed reference: 2 q~ 2^-pos
-  float roff[G];                      // compressed reference: (2^RB - 1) sum q~ (lane dims)
-  float wsumR[G];                     // compressed reference: sum of p s_ref^V
-  // INT8 compressed reference: q~ of the lane's dims as 16-bit fixed point
-  // (step qsig), split into signed high and unsigned low bytes for dp4a
-  uint32_t qhi[G][2], qlo[G][2];
-  float qsig[G];
   float2 qc[G][NP];                   // 2 q~ 2^-pos (codes at their bit position)
   float qoff[G];                      // (2^b - 1) * sum q~ over the lane's dims
   // running state
@@ -412,7 +331,6 @@ decode_kernel(const DecodeParams p) {
       m_run[r] = kNegInf;
       l_run[r] = 0.0f;
       wsum[r] = 0.0f;
-      wsumR[r] = 0.0f;
 #pragma unroll
       for (int j = 0; j < NP; ++j) {
         accV[r][j] = make_float2(0.0f, 0.0f);
@@ -464,31 +382,9 @@ decode_kernel(const DecodeParams p) {
         const float t1 = cd * qt[r * D + dim0 + 2 * j + 1];
         qc[r][j] = make_float2(2.0f * t0 * pos_factor<PB, DPL>(2 * j),
                                2.0f * t1 * pos_factor<PB, DPL>(2 * j + 1));
-        if constexpr (RB != 0)
-          qr[r][j] = make_float2(2.0f * t0 * ref_pos_factor<RB, DPL>(2 * j),
-                                 2.0f * t1 * ref_pos_factor<RB, DPL>(2 * j + 1));
         sum += t0 + t1;
       }
       qoff[r] = (float)TOPLVL * sum;
-      roff[r] = (float)((1 << (RB ? RB : 1)) - 1) * sum;
-      if constexpr (RB == 8 && DPL == 8) {
-        float t[8], mx = 0.0f;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          t[k] = cd * qt[r * D + dim0 + k];
-          mx = fmaxf(mx, fabsf(t[k]));
-        }
-        const float sig = fmaxf(mx, 1e-30f) * (1.0f / 32512.0f);   // |Q| <= 127 * 256
-        const float inv_sig = 1.0f / sig;
-        qsig[r] = sig;
-        qhi[r][0] = qhi[r][1] = qlo[r][0] = qlo[r][1] = 0u;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int Q = __float2int_rn(t[k] * inv_sig);
-          qhi[r][k / 4] |= ((uint32_t)(Q >> 8) & 0xFFu) << (8 * (k % 4));
-          qlo[r][k / 4] |= ((uint32_t)Q & 0xFFu) << (8 * (k % 4));
-        }
-      }
     }
   };
 
@@ -510,7 +406,6 @@ decode_kernel(const DecodeParams p) {
 #pragma unroll
       for (int m = LPT; m < 32; m <<= 1) {
         if constexpr (C::RES) wsum[r] += __shfl_xor_sync(FULL, wsum[r], m);
-        if constexpr (RB != 0) wsumR[r] += __shfl_xor_sync(FULL, wsumR[r], m);
 #pragma unroll
         for (int j = 0; j < NP; ++j) {
           accV[r][j].x += __shfl_xor_sync(FULL, accV[r][j].x, m);
@@ -524,11 +419,6 @@ decode_kernel(const DecodeParams p) {
     }
     named_bar_sync(1, kConsumerThreads);          // merge area (and table) free
     float* mw = merge + warp * G * (2 + 2 * D);
-    if constexpr (RB == 8 && DPL == 8) {
-      // an fp16 weight p s_ref overflowed (reference scales above 2^8 with
-      // the lazy softmax's p up to 2^8): the output is not valid
-      if (lane == 0 && !isfinite(wsumR[0])) flag_error(p.status, 64u);
-    }
     if (slot == 0) {
 #pragma unroll
       for (int r = 0; r < G; ++r) {
@@ -544,23 +434,8 @@ decode_kernel(const DecodeParams p) {
             z0 = 2.0f * pos_factor<PB, DPL>(2 * j) * accC[r][j].x - (float)TOPLVL * wsum[r];
             z1 = 2.0f * pos_factor<PB, DPL>(2 * j + 1) * accC[r][j].y - (float)TOPLVL * wsum[r];
           }
-          if constexpr (RB == 0) {
-            rec[2 + dim0 + 2 * j] = accV[r][j].x;
-            rec[2 + dim0 + 2 * j + 1] = accV[r][j].y;
-          } else {
-            // the reference is in the rotated domain too: accV holds its codes
-            constexpr float RT = (float)((1 << RB) - 1);
-            if constexpr (RB == 8 && DPL == 8) {
-              // accV = sum w (1024 + c): sum w l = 2 accV - (2048 + RT) sum w
-              z0 += 2.0f * accV[r][j].x - (2048.0f + RT) * wsumR[r];
-              z1 += 2.0f * accV[r][j].y - (2048.0f + RT) * wsumR[r];
-            } else {
-              z0 += 2.0f * ref_pos_factor<RB, DPL>(2 * j) * accV[r][j].x - RT * wsumR[r];
-              z1 += 2.0f * ref_pos_factor<RB, DPL>(2 * j + 1) * accV[r][j].y - RT * wsumR[r];
-            }
-            rec[2 + dim0 + 2 * j] = 0.0f;
-            rec[2 + dim0 + 2 * j + 1] = 0.0f;
-          }
+          rec[2 + dim0 + 2 * j] = accV[r][j].x;
+          rec[2 + dim0 + 2 * j + 1] = accV[r][j].y;
           rec[2 + D + dim0 + 2 * j] = z0;
           rec[2 + D + dim0 + 2 * j + 1] = z1;
         }
@@ -568,25 +443,7 @@ decode_kernel(const DecodeParams p) {
     }
     named_bar_sync(1, kConsumerThreads);
 
-    finish_head<D, G, C::RES || RB != 0>(p, hd, first_tile, nt_h, split, cta, merge, qbuf,
-                                         flags, tid);
-  };
-
-  // compressed reference: <q~, l_ref> of the lane's dims (without s_ref)
-  auto ref_code_dot = [&](const unsigned char* kp, int r) {
-    if constexpr (RB == 8 && DPL == 8) {
-      // sum_k Q_k c_k exactly in integers: Q = 256 hi + lo
-      const uint2 w = *reinterpret_cast<const uint2*>(kp);
-      const int dh = dp4a_su(qhi[r][1], w.y, dp4a_su(qhi[r][0], w.x, 0));
-      const int dl = dp4a_uu(qlo[r][1], w.y, dp4a_uu(qlo[r][0], w.x, 0));
-      return fmaf(2.0f * qsig[r], __int2float_rn(dh * 256 + dl), -roff[r]);
-    }
-    float f[DPL];
-    ref_codes_positional<RB ? RB : 4, DPL>(kp, f);
-    float2 acc = make_float2(-roff[r], 0.0f);
-#pragma unroll
-    for (int j = 0; j < NP; ++j) acc = __ffma2_rn(qr[r][j], make_float2(f[2 * j], f[2 * j + 1]), acc);
-    return acc.x + acc.y;
+    finish_head<D, G, C::RES>(p, hd, first_tile, nt_h, split, cta, merge, qbuf, flags, tid);
   };
 
   // <q, K row> of the lane's dims, straight from the packed bf16 row
@@ -633,7 +490,6 @@ decode_kernel(const DecodeParams p) {
     const float2 a2 = make_float2(alpha, alpha);
     l_run[r] *= alpha;
     if constexpr (C::RES) wsum[r] *= alpha;
-    if constexpr (RB != 0) wsumR[r] *= alpha;
 #pragma unroll
     for (int j = 0; j < NP; ++j) {
       accV[r][j] = __fmul2_rn(accV[r][j], a2);
@@ -643,11 +499,8 @@ decode_kernel(const DecodeParams p) {
 
   // adds weight pw of one token (lane's V row vf, codes word, scale s_v)
   auto accumulate_v = [&](int r, float pw, const float2 (&vf)[NP], const float2 (&cf)[NP],
-                          float s_v, float s_rv = 1.0f) {
-    // weight of the reference row: p (BF16 row) or p s_ref^V (reference codes)
-    const float pv = (RB != 0) ? pw * s_rv : pw;
-    if constexpr (RB != 0) wsumR[r] += pv;
-    const float2 p2 = make_float2(pv, pv);
+                          float s_v) {
+    const float2 p2 = make_float2(pw, pw);
 #pragma unroll
     for (int j = 0; j < NP; ++j) accV[r][j] = __ffma2_rn(p2, vf[j], accV[r][j]);
     if constexpr (C::RES) {
@@ -665,13 +518,7 @@ decode_kernel(const DecodeParams p) {
 #pragma unroll
     for (int u = 0; u < CH; ++u) {
       const int tok = warp * C::TPW + u * TPS + slot;
-      float dot;
-      if constexpr (RB == 0) {
-        dot = ref_dot(st + C::OFF_K + tok * C::KROW + dim0 * 2, 0);
-      } else {
-        const float s_rk = half_at(st + C::OFF_RSK + sc_off + tok * SB + grp * 2);
-        dot = s_rk * ref_code_dot(st + C::OFF_K + tok * C::KROW + dim0 * RB / 8, 0);
-      }
+      float dot = ref_dot(st + C::OFF_K + tok * C::KROW + dim0 * 2, 0);
       if constexpr (C::RES) {
         const uint32_t word = reinterpret_cast<const uint32_t*>(st + C::OFF_CK)[tok * C::CWORDS + cw];
         const float s_k = half_at(st + C::OFF_SK + sc_off + tok * SB + grp * 2);
@@ -727,48 +574,13 @@ decode_kernel(const DecodeParams p) {
       const int tok = warp * C::TPW + u * TPS + slot;
       if (tok < n) {
         float2 vf[NP], cf[NP];
-        float s_rv = 1.0f;
-        if constexpr (RB == 0) {
-          v_pairs(st + C::OFF_V + tok * C::KROW + dim0 * 2, vf);
-        } else if constexpr (RB == 8 && DPL == 8) {
-          // codes as exact fp16 values 1024 + c, weight p s_ref^V rounded to
-          // fp16 once (the same rounded weight goes into the offset sum)
-          s_rv = half_at(st + C::OFF_RSV + sc_off + tok * SB + grp * 2);
-          const __half w16 = __float2half_rn(pu * s_rv);
-          const uint32_t w2 = (uint32_t)__half_as_ushort(w16) * 0x10001u;
-          wsumR[0] += __half2float(w16);
-          const uint2 cw2 = *reinterpret_cast<const uint2*>(st + C::OFF_V + tok * C::KROW + dim0);
-#pragma unroll
-          for (int j = 0; j < NP; ++j) {
-            const uint32_t src = j < 2 ? cw2.x : cw2.y;
-            const uint32_t cp = __byte_perm(src, 0x64646464u, (j & 1) ? 0x7362u : 0x5140u);
-            accV[0][j].x = fma_f16_half<0>(w2, cp, accV[0][j].x);
-            accV[0][j].y = fma_f16_half<1>(w2, cp, accV[0][j].y);
-          }
-        } else {
-          float f[DPL];
-          ref_codes_positional<RB ? RB : 4, DPL>(st + C::OFF_V + tok * C::KROW + dim0 * RB / 8, f);
-#pragma unroll
-          for (int j = 0; j < NP; ++j) vf[j] = make_float2(f[2 * j], f[2 * j + 1]);
-          s_rv = half_at(st + C::OFF_RSV + sc_off + tok * SB + grp * 2);
-        }
+        v_pairs(st + C::OFF_V + tok * C::KROW + dim0 * 2, vf);
         float s_v = 0.0f;
         if constexpr (C::RES) {
           code_pairs(reinterpret_cast<const uint32_t*>(st + C::OFF_CV)[tok * C::CWORDS + cw], cf);
           s_v = half_at(st + C::OFF_SV + sc_off + tok * SB + grp * 2);
         }
-        if constexpr (RB == 8 && DPL == 8) {
-          // reference part done above; only the residual remains
-          if constexpr (C::RES) {
-            const float wv = pu * s_v;
-            const float2 w2 = make_float2(wv, wv);
-            wsum[0] += wv;
-#pragma unroll
-            for (int j = 0; j < NP; ++j) accC[0][j] = __ffma2_rn(w2, cf[j], accC[0][j]);
-          }
-        } else {
-          accumulate_v(0, pu, vf, cf, s_v, s_rv);
-        }
+        accumulate_v(0, pu, vf, cf, s_v);
       }
     }
   };
@@ -905,33 +717,33 @@ decode_kernel(const DecodeParams p) {
   if (cur_head >= 0) flush_head(cur_head, cur_first, cur_nt);
 }
 
-template <int D, int G, int BITS, int RB>
+template <int D, int G, int BITS>
 cudaError_t launch_decode_t(const DecodeParams& p, cudaStream_t stream) {
-  using C = Cfg<D, G, BITS, RB>;
+  using C = Cfg<D, G, BITS>;
   static bool attr_set = false;   // per process; harmless to repeat
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, G, BITS, RB>,
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, G, BITS>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  return launch_pdl(decode_kernel<D, G, BITS, RB>, p.ctas, kThreads, C::SMEM_BYTES, stream, p);
+  return launch_pdl(decode_kernel<D, G, BITS>, p.ctas, kThreads, C::SMEM_BYTES, stream, p);
 }
 
-template <int D, int G, int RB>
+template <int D, int G>
 cudaError_t launch_decode_b(int bits, const DecodeParams& p, cudaStream_t stream) {
-  if (bits == 2) return launch_decode_t<D, G, 2, RB>(p, stream);
-  if (bits == 4) return launch_decode_t<D, G, 4, RB>(p, stream);
-  if (bits == 16) return launch_decode_t<D, G, 16, RB>(p, stream);
+  if (bits == 2) return launch_decode_t<D, G, 2>(p, stream);
+  if (bits == 4) return launch_decode_t<D, G, 4>(p, stream);
+  if (bits == 16) return launch_decode_t<D, G, 16>(p, stream);
   return cudaErrorInvalidValue;
 }
 
 template <int D, int G>
 cudaError_t launch_decode_g(int bits, const DecodeParams& p, cudaStream_t stream) {
-  if (p.ref_bits == 0) return launch_decode_b<D, G, 0>(bits, p, stream);
-  if (p.ref_bits == 8) return launch_decode_b<D, G, 8>(bits, p, stream);
-  if (p.ref_bits == 4) return launch_decode_b<D, G, 4>(bits, p, stream);
+  if (p.ref_bits == 0) return launch_decode_b<D, G>(bits, p, stream);
+  // a compressed reference: the tensor-core kernel (rq_decode_cr1.cu)
+  if (p.ref_bits == 8 || p.ref_bits == 4) return launch_decode_cr1(D, bits, p, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -7,7 +7,7 @@ namespace rq {
 
 cudaError_t launch_decode_gqa(int head_dim, int G, int bits, const DecodeParams& p,
                               cudaStream_t stream) {
-  GqaParams gp;
+  TcParams gp;
   gp.p = p;
   const unsigned long long rows =
       p.page_table ? (unsigned long long)p.n_pages * p.kv_heads * kDecodeTile

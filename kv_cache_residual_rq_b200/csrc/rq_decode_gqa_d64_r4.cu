@@ -6,7 +6,7 @@
 
 namespace rq {
 
-cudaError_t launch_gqa_d64_r4(int G, int bits, const GqaParams& gp, cudaStream_t stream) {
+cudaError_t launch_gqa_d64_r4(int G, int bits, const TcParams& gp, cudaStream_t stream) {
   return launch_gqa_d<64, 4>(G, bits, gp, stream);
 }
 

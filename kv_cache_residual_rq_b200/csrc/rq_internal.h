@@ -212,6 +212,9 @@ cudaError_t launch_decode(int head_dim, int G, int bits, const DecodeParams& p,
 // grouped queries, G in {2, 4, 8} (tensor cores, TMA tensor copies)
 cudaError_t launch_decode_gqa(int head_dim, int G, int bits, const DecodeParams& p,
                               cudaStream_t stream);
+// one query row per kv head over a compressed reference (p.ref_bits 4 or 8):
+// the tensor-core kernel (rq_decode_cr1.cu)
+cudaError_t launch_decode_cr1(int head_dim, int bits, const DecodeParams& p, cudaStream_t stream);
 
 int device_sm_count();   // SMs of the current device, cached per device
 

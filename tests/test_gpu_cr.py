@@ -287,22 +287,45 @@ def test_cr_grouped_peaky_scores_long_context():
     print(f"peaky G {G}: max-abs {worst:.2e}")
 
 
-def test_cr_single_query_weight_overflow_sets_status():
-    """With one query row per kv head the INT8 reference's value weights are
-    fp16; reference scales at the fp16 maximum overflow them once a weight
-    exceeds 1, and the call reports it in workspace status bit 64.  The
-    context is long enough that every CTA's run spans several tiles (a later
-    tile's scores above the first tile's max give weights above 1)."""
-    d, g, B, H, T = 128, 32, 2, 2, 16384
-    w = synth.Workload("crovf", 2, 1, B, T, H, H, d, g, (2,), (0.25,), 178)
+def test_cr_single_query_large_value_scales():
+    """One query row per kv head: the value weights p s 2^Ev are f16 after a
+    lazily updated warp-wide power of two, so reference value scales at the
+    fp16 maximum decode without overflow (status 0) and match the oracle's
+    attention over the same scales.  A NaN scale of a cached token makes the
+    weights non-finite, which raises workspace status bit 64."""
+    d, g, B, H, T = 128, 32, 2, 2, 2000
+    w = synth.Workload("crbig", 2, 1, B, T, H, H, d, g, (2,), (0.25,), 178)
     refk, refv = synth.reference(w, 0, 0), synth.reference(w, 0, 1)
     xk, xv = synth.loop_kv(w, 0, 0, 1, refk), synth.loop_kv(w, 0, 1, 1, refv)
     (rck, rsk), ck, sk = rq.encode_cr([xk], refk, 8, [2], g, w.seed)
     (rcv, rsv), cv, sv = rq.encode_cr([xv], refv, 8, [2], g, w.seed)
-    rsv.view(torch.int16)[: B * H * T * (d // g)] = 0x7BFF          # fp16 65504
+    big = 0x7BFF                                                 # fp16 65504
+    rsv.view(torch.int16)[: B * H * T * (d // g)] = big
     q = (synth.query(w, 0, 1).float() * 4.0).to(torch.bfloat16)
     shape = rq.make_shape(B, H, T, d, g)
     ws = rq.alloc_workspace(shape, q.device)
+    out = rq.decode_attention_cr(q, (rck, rsk, rcv, rsv, 8), ck[0], cv[0], sk[0], sv[0], 2, g,
+                                 w.seed, T, workspace=ws)
+    torch.cuda.synchronize()
+    assert rq.rq_workspace_status(ws) == 0
+    assert torch.isfinite(out).all()
+    worst, top = 0.0, 0.0
+    for b in range(B):
+        for h in range(H):
+            parts = []
+            for src_x, src_r, v in ((xk, refk, False), (xv, refv, True)):
+                rw, rs, ww, wsc = oracle.encode_rows_cr_f32(u16(src_x[b, h, :T]),
+                                                            u16(src_r[b, h, :T]), 8, 2, g, w.seed)
+                if v:
+                    rs = np.full_like(rs, big)
+                parts.append(oracle.reconstruct_rows_cr_f64(rw, rs, ww, wsc, 8, 2, g, w.seed, d))
+            qh = oracle.bf16_to_f32(u16(q[b, h:h + 1])).astype(np.float64)
+            want = oracle.attention_f64(qh, parts[0], parts[1], 1.0 / np.sqrt(d))
+            worst = max(worst, float(np.abs(out[b, h:h + 1].double().cpu().numpy() - want).max()))
+            top = max(top, float(np.abs(want).max()))
+    print(f"value scales 65504: max-abs {worst:.3e} of max |out| {top:.3e}")
+    assert worst <= 1e-4 * top
+    rsv.view(torch.int16)[5 * (d // g) + 1] = F16_NAN           # token 5 of head (0, 0)
     rq.decode_attention_cr(q, (rck, rsk, rcv, rsv, 8), ck[0], cv[0], sk[0], sv[0], 2, g, w.seed,
                            T, workspace=ws)
     torch.cuda.synchronize()
