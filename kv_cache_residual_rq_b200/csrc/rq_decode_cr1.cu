@@ -71,10 +71,8 @@ struct C1Cfg {
   static constexpr int OFF_RSV = OFF_RSK + RSC_BYTES;
   static constexpr int STAGE_BYTES = (OFF_RSV + RSC_BYTES + 1023) / 1024 * 1024;
   // resident CTAs per SM (registers: 65536 / (CTAS x 160 threads), rounded to
-  // whole warps per scheduler), and the ring depth that fits their shared memory
+  // whole warps per scheduler)
   static constexpr int CTAS = 3;
-  static constexpr int STAGES = CTAS == 2 ? 3 : 2;
-  static constexpr int RING_BYTES = STAGES * STAGE_BYTES;
   // per consumer warp {m, l, o_ref[D], o~[D]}; also the scratch of the
   // sequence-length scan of a variable-length call
   static constexpr int MERGE_0 = kConsumerWarps * (2 + 2 * D);
@@ -84,10 +82,19 @@ struct C1Cfg {
   // score B fragments per lane: reference MMAs [NV], residual MMAs [4]
   static constexpr int KFRAG_WORDS = (NV + 4) * 32 * 2;
   static constexpr int WSUM_FLOATS = kConsumerWarps * NV * 2;
-  static constexpr int SMEM_BYTES = 1024 /* base alignment slack */ + RING_BYTES +
-                                    4 * (MERGE_FLOATS + QBUF_FLOATS + QI_WORDS + WSUM_FLOATS +
-                                         KFRAG_WORDS) +
-                                    2 * STAGES * 8 + 16 + STAGES * 8;   // + stage rows
+  static constexpr int MAX_STAGES = 4;
+  static constexpr int OTHER_BYTES = 1024 /* base alignment slack */ +
+                                     4 * (MERGE_FLOATS + QBUF_FLOATS + QI_WORDS + WSUM_FLOATS +
+                                          KFRAG_WORDS) +
+                                     2 * MAX_STAGES * 8 + 16 + MAX_STAGES * 8;   // + stage rows
+  // the ring: as many stages (2 .. 4) as the CTAS resident CTAs' shared
+  // memory allows (228 KB per SM, 1 KB of it reserved per CTA)
+  static constexpr int SMEM_PER_CTA = 228 * 1024 / CTAS - 1024;
+  static constexpr int FIT = (SMEM_PER_CTA - OTHER_BYTES) / STAGE_BYTES;
+  static constexpr int STAGES = FIT > MAX_STAGES ? MAX_STAGES : FIT;
+  static constexpr int RING_BYTES = STAGES * STAGE_BYTES;
+  static constexpr int SMEM_BYTES = OTHER_BYTES + RING_BYTES;
+  static_assert(STAGES >= 2, "a double-buffered ring fits");
   static_assert(D == 64 || D == 128, "head_dim");
   static_assert(GROUP == 32 || GROUP == 64, "scale group");
   static_assert(RB == 4 || RB == 8, "compressed reference: INT4 or INT8 codes");
@@ -425,8 +432,10 @@ decode_cr1_kernel(const __grid_constant__ TcParams gp) {
       f1 += __shfl_xor_sync(FULL, f1, 1);
       f0 += __shfl_xor_sync(FULL, f0, 2);
       f1 += __shfl_xor_sync(FULL, f1, 2);
-      if (tok0 >= n) f0 = kNegInf;
-      if (tok1 >= n) f1 = kNegInf;
+      if (n < C::TILE) {               // a partial tile: tokens from n on are not cached
+        if (tok0 >= n) f0 = kNegInf;
+        if (tok1 >= n) f1 = kNegInf;
+      }
     }
     // ---- online softmax, one row per warp, rescaled lazily ----
     {
@@ -466,14 +475,18 @@ decode_cr1_kernel(const __grid_constant__ TcParams gp) {
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const int tok = wtok + tk[k];
-        const float a = half_at(st + C::OFF_RSV + sc_off + tok * SB + 2 * rg);
-        sr[k] = (tok < n) ? a : 0.0f;                 // weight 0 beyond the tile
+        sr[k] = half_at(st + C::OFF_RSV + sc_off + tok * SB + 2 * rg);
+        if constexpr (C::RES) sv[k] = half_at(st + C::OFF_SV + sc_off + tok * SB + 2 * rg);
+      }
+      if (n < C::TILE) {                 // weight 0 beyond the tile
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          if (wtok + tk[k] >= n) sr[k] = sv[k] = 0.0f;
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
         smax = fmaxf(smax, fabsf(sr[k]));
-        if constexpr (C::RES) {
-          const float b = half_at(st + C::OFF_SV + sc_off + tok * SB + 2 * rg);
-          sv[k] = (tok < n) ? b : 0.0f;
-          smax = fmaxf(smax, fabsf(sv[k]));
-        }
+        if constexpr (C::RES) smax = fmaxf(smax, fabsf(sv[k]));
       }
       // 2^Ev moves only when the tile's largest value scale times 2^Ev leaves
       // [1, 2^7): one vote decides, the warp's max is formed only then
@@ -515,6 +528,15 @@ decode_cr1_kernel(const __grid_constant__ TcParams gp) {
     uint32_t br0, br1, bv0 = 0u, bv1 = 0u;
     weight_frags(sr, br0, br1, wr_sum);
     if constexpr (C::RES) weight_frags(sv, bv0, bv1, wv_sum);
+    // INT8 reference: the residual codes of the odd m-tiles enter masked in
+    // place (4c for INT2, 16c for INT4; exact subnormals), their weights
+    // scaled down by the same power of two (exact)
+    uint32_t bv0o = bv0, bv1o = bv1;
+    if constexpr (C::RES && RB == 8) {
+      const uint32_t f = (BITS == 2) ? 0x34003400u : 0x2C002C00u;   // {1/4, 1/4} / {1/16, 1/16}
+      bv0o = hmul2_u(bv0, f);
+      bv1o = hmul2_u(bv1, f);
+    }
 
     // ---- values: o~^T += C^T W^T, reference then residual codes ----
     const unsigned char* cvb = st + C::OFF_CV;
@@ -538,10 +560,12 @@ decode_cr1_kernel(const __grid_constant__ TcParams gp) {
 #pragma unroll
             for (int k = 0; k < 4; ++k)
               w[k] = *reinterpret_cast<const uint2*>(cvb + (wtok + tk[k]) * C::CROW + 8 * cp);
-            X[0] = __byte_perm(w[0].x, w[1].x, psel);
-            X[1] = __byte_perm(w[0].y, w[1].y, psel);
-            X[2] = __byte_perm(w[2].x, w[3].x, psel);
-            X[3] = __byte_perm(w[2].y, w[3].y, psel);
+            // the nibble of m-row g down to bit 0
+            const int sh = 4 * (g & 1);
+            X[0] = __byte_perm(w[0].x, w[1].x, psel) >> sh;
+            X[1] = __byte_perm(w[0].y, w[1].y, psel) >> sh;
+            X[2] = __byte_perm(w[2].x, w[3].x, psel) >> sh;
+            X[3] = __byte_perm(w[2].y, w[3].y, psel) >> sh;
           } else {
             // words 4cp + (g >> 2) (m-rows g) and 4cp + 2 + (g >> 2)
             const int wo = 4 * (4 * cp + (g >> 2));
@@ -566,11 +590,12 @@ decode_cr1_kernel(const __grid_constant__ TcParams gp) {
                                  __byte_perm(R[2], 0u, sel), __byte_perm(R[3], 0u, sel)};
           mma_f16(acc[2 * cp + e], a, br0, br1);
           if constexpr (C::RES) {
-            const int sh = (BITS == 2) ? 4 * (g & 1) + 2 * e : 4 * e;
+            // m-rows g: INT2 bits 2e of the nibble (Y), INT4 nibble e of the byte
             constexpr uint32_t M = (BITS == 2) ? 0x00030003u : 0x000F000Fu;
-            const uint32_t c[4] = {(X[0] >> sh) & M, (X[1] >> sh) & M, (X[2] >> sh) & M,
-                                   (X[3] >> sh) & M};
-            mma_f16(acc[2 * cp + e], c, bv0, bv1);
+            const uint32_t Me = e ? (BITS == 2 ? M << 2 : M << 4) : M;
+            const uint32_t c[4] = {X[0] & Me, X[1] & Me, X[2] & Me, X[3] & Me};
+            if (e) mma_f16(acc[2 * cp + e], c, bv0o, bv1o);
+            else mma_f16(acc[2 * cp + e], c, bv0, bv1);
           }
         }
       }
