@@ -27,14 +27,16 @@
 // Compressed INT8 / INT4 reference (same page, the reference loop itself
 // stored as rotated codes): the reference term is one more quantised term in
 // the rotated domain, s_ref <q~, l_ref> for the scores and sum_t p s_ref l_ref
-// for the values, l_ref = 2c - (2^b - 1).  Its codes enter f16 MMAs as the
-// exact subnormals c 2^-24 -- the code in the low mantissa bits: one byte
-// permute per two INT8 codes, one shift and one mask per two INT4 codes, no
-// offset to cancel -- against q~ scaled by a power of two per row and split
-// into f16 high and remainder parts (scores), or against the weights p s_ref
-// split into f16 parts after a lazily updated power of two keeps them in
-// f16's range (values); the 2^24 returns with the scales, once per scale
-// group (scores) or when the warp flushes (values).  The reference rows (d or
+// for the values, l_ref = 2c - (2^b - 1).  Scores: integer MMAs (m16n8k32,
+// s8 x u8) per 32-dim slice, the rows' q~ as 16-bit fixed point Q = q~ / sig
+// split into signed bytes h (rows g) and l (rows g + 8) against the codes one
+// per byte (INT8 rows as ldmatrix reads them, INT4 nibbles by one mask or a
+// shift and a mask per four); per scale group sig (2 <Q, c> - (2^b - 1) sum
+// Q) is exact in integers until the scale.  Values: the codes enter f16 MMAs
+// as the exact subnormals c 2^-24 (one byte permute per two INT8 codes, one
+// shift and one mask per two INT4 codes) against the weights p s_ref split
+// into f16 parts after a lazily updated power of two keeps them in f16's
+// range; the 2^24 returns when the warp flushes.  The reference rows (d or
 // d/2 bytes) arrive swizzled; the k order of the q~ fragments and the m-row
 // order of the value accumulators follow the codes' positions in the 32-bit
 // ldmatrix words.
@@ -110,18 +112,21 @@ struct GCfg {
   static constexpr int MERGE_FLOATS = kConsumerWarps * G * (2 + 2 * D);
   static constexpr int QBUF_FLOATS = 2 * G * D;
   static constexpr int NG = D / GROUP;                      // scale groups per token
+  static constexpr int NV = D / 32;                        // 32-dim slices
+  static constexpr int SPG = GROUP / 32;                   // slices per scale group
   static constexpr int KSG = GROUP / 16;                   // k-steps per scale group
   static constexpr int SB = 2 * NG;                        // scale bytes per token
   // per warp, row and scale group: sum of p s^V (and of p s_ref^V)
   static constexpr int WSUM_FLOATS = kConsumerWarps * G * NG * (CRX ? 2 : 1);
   // q, q~ high, q~ remainder (bf16); with a compressed reference also
   // q~ 2^E high, remainder (f16, k-permuted for the reference's codes)
-  static constexpr int QFRAG_WORDS = (CRX ? 5 : 3) * KT * 32 * 2;
+  static constexpr int QFRAG_WORDS = 3 * KT * 32 * 2 + (CRX ? NV * 32 * 4 : 0);
   // INT2: per (row, scale group) sum of the q~ fragments' values (offset of
   // the 128 + 2c operands); compressed reference: the same for the f16
   // fragments (the levels' 2^b - 1) and per row 2^-E; even count to keep the
   // barriers 8-byte aligned
-  static constexpr int SQ_FLOATS = (G * NG * (CRX ? 2 : 1) + ((CRX || RES) ? G : 0) + 1) / 2 * 2;
+  static constexpr int SQ_FLOATS =
+      (G * NG * (CRX ? 2 : 1) + ((CRX || RES) ? G : 0) + (CRX ? G : 0) + 1) / 2 * 2;
   static constexpr int SMEM_BYTES = 1024 /* base alignment slack */ + RING_BYTES +
                                     4 * (MERGE_FLOATS + QBUF_FLOATS + WSUM_FLOATS +
                                          QFRAG_WORDS + SQ_FLOATS) +
@@ -156,9 +161,10 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
   float* wsum_s = qbuf + C::QBUF_FLOATS;
   uint32_t* qfrag = reinterpret_cast<uint32_t*>(wsum_s + C::WSUM_FLOATS);  // [3][KT][32][2]
   float* sq_s = reinterpret_cast<float*>(qfrag + C::QFRAG_WORDS);           // [G][NG]
-  float* sqh_s = sq_s + G * NG;              // CR: [G][NG] sums of the f16 q~ fragments
+  float* sqh_s = sq_s + G * NG;              // CR: [G][NG] sums of Q per scale group
   // [G] 2^-E of each row's f16 q~ fragments (residual and compressed reference)
   float* rsig_s = sq_s + G * NG * (C::CRX ? 2 : 1);
+  float* rsigc_s = rsig_s + G;               // CR: [G] sig of each row's Q
   float* wsumR_s = wsum_s + kConsumerWarps * G * NG;   // CR: sums of p s_ref^V
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(sq_s + C::SQ_FLOATS);
   uint64_t* empty_bar = full_bar + STAGES;
@@ -212,9 +218,10 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
   // and lane, {a0, a2} of the bf16 query (kind 0) and, with a residual, of
   // the rotated query as f16 q~ 2^E (kind 1; kind 2 is unused): rows g, dims
   // in the k order of the residual's code words; rows g >= G are zero, and
-  // a1 = a3 = 0 (rows g + 8).  With a compressed reference, kinds 3 and 4
-  // are the f16 high part and remainder of q~ 2^E in the k order of the
-  // reference's code words.
+  // a1 = a3 = 0 (rows g + 8).  With a compressed reference, the region after
+  // kind 2 holds per 32-dim slice and lane the four s8 A words {a0, a1, a2,
+  // a3} of the reference's integer MMAs (rows g: bytes h of Q, rows g + 8:
+  // bytes l, in the k order of the reference's code words).
   auto qfrag_addr = [&](int kind, int kk) {
     return smem_u32(qfrag + ((kind * KT + kk) * 32 + lane) * 2);
   };
@@ -250,55 +257,46 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
     const float cd = rot_scale<D>();
     if constexpr (C::CRX) {
       if (warp == 0) {
-        // f16 fragments of q~ 2^E, E per row so that max |q~| 2^E is in
-        // [2^13, 2^14): the high parts keep 11 bits, the remainders the next
-        // 11, and no value leaves f16's normal range.  The k positions
-        // follow the codes a 32-bit ldmatrix word holds: INT8, k positions
-        // 2q, 2q+1 | 2q+8, 2q+9 of k-step kk carry dims 16kk + 4q .. 4q+3;
-        // INT4, a word holds dims 8q .. 8q+7 of a 32-dim chunk (two k-steps),
-        // code i at bits 4i, and k-step kk (half h = kk & 1 of chunk kk / 2)
-        // carries dims 8q + 2h + {0, 4 | 1, 5} (a register's two codes then
-        // sit 16 bits apart).
+        // row g of q~ as 16-bit fixed point Q = q~ / sig (sig = max |q~| /
+        // 32639, so Q = 256 h + l with signed bytes h, l), as the A fragments
+        // of the compressed reference's integer MMAs: per 32-dim slice j,
+        // rows g carry the h bytes and rows g + 8 the l bytes; the k
+        // positions 4q + b and 16 + 4q + b carry the dims of the codes the
+        // ldmatrix words hold there (INT8: 32j + 4q + b, + 16; INT4: nibbles
+        // 0 and 1 of byte 4q + b of chunk j, dims 32j + 8q + 2b, + 1)
         float mx = 0.0f;
         if (row_ok)
           for (int d = q; d < D; d += 4) mx = fmaxf(mx, fabsf(cd * qt[g * D + d]));
         mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 1));
         mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 2));
-        const int ex = (int)((__float_as_uint(mx) >> 23) & 0xFFu) - 127;
-        const int E = min(13 - ex, 126);
-        const float up = __uint_as_float((uint32_t)(127 + E) << 23);
-        if (row_ok && q == 0) rsig_s[g] = __uint_as_float((uint32_t)(127 - E) << 23);
-        float sqh = 0.0f;
+        const float sig = mx > 0.0f ? mx * (1.0f / 32639.0f) : 1.0f;
+        const float inv = 1.0f / sig;
+        if (row_ok && q == 0) rsigc_s[g] = sig;
+        int sq = 0;          // sum of Q over the lane's dims of the current scale group
 #pragma unroll 1
-        for (int kk = 0; kk < KT; ++kk) {
-          uint32_t* f3 = qfrag + ((3 * KT + kk) * 32 + lane) * 2;
-          uint32_t* f4 = qfrag + ((4 * KT + kk) * 32 + lane) * 2;
+        for (int j = 0; j < C::NV; ++j) {
+          uint32_t a[4] = {0u, 0u, 0u, 0u};
           if (row_ok) {
-            int d0, d1, d2, d3;
-            if constexpr (C::CR) {
-              d0 = 16 * kk + 4 * q;
-              d1 = d0 + 1;
-              d2 = d0 + 2;
-              d3 = d0 + 3;
-            } else {
-              d0 = 32 * (kk >> 1) + 8 * q + 2 * (kk & 1);
-              d1 = d0 + 4;
-              d2 = d0 + 1;
-              d3 = d0 + 5;
-            }
-            const float* trow = qt + g * D;
-            split_f16(cd * trow[d0] * up, cd * trow[d1] * up, f3[0], f4[0]);
-            split_f16(cd * trow[d2] * up, cd * trow[d3] * up, f3[1], f4[1]);
-            sqh += ((f16_lo_f(f3[0]) + f16_lo_f(f4[0])) + (f16_hi_f(f3[0]) + f16_hi_f(f4[0]))) +
-                   ((f16_lo_f(f3[1]) + f16_lo_f(f4[1])) + (f16_hi_f(f3[1]) + f16_hi_f(f4[1])));
-          } else {
-            f3[0] = f3[1] = f4[0] = f4[1] = 0u;
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2)
+#pragma unroll
+              for (int b = 0; b < 4; ++b) {
+                const int dim = C::CR ? 32 * j + 16 * h2 + 4 * q + b : 32 * j + 8 * q + 2 * b + h2;
+                const int Q = min(max(__float2int_rn(cd * qt[g * D + dim] * inv), -32639), 32639);
+                const int lo = ((Q + 128) & 255) - 128;
+                const int hi = (Q - lo) >> 8;
+                a[2 * h2] |= (uint32_t)(hi & 0xFF) << (8 * b);
+                a[2 * h2 + 1] |= (uint32_t)(lo & 0xFF) << (8 * b);
+                sq += Q;
+              }
           }
-          if ((kk + 1) % KSG == 0) {                   // end of a scale group
-            sqh += __shfl_xor_sync(FULL, sqh, 1);
-            sqh += __shfl_xor_sync(FULL, sqh, 2);
-            if (row_ok && q == 0) sqh_s[g * NG + kk / KSG] = sqh;
-            sqh = 0.0f;
+          *reinterpret_cast<uint4*>(qfrag + ((3 * KT) * 32 * 2) + (j * 32 + lane) * 4) =
+              make_uint4(a[0], a[1], a[2], a[3]);
+          if ((j + 1) % C::SPG == 0) {                // end of a scale group
+            sq += __shfl_xor_sync(FULL, sq, 1);
+            sq += __shfl_xor_sync(FULL, sq, 2);
+            if (row_ok && q == 0) sqh_s[g * NG + j / C::SPG] = (float)sq;
+            sq = 0;
           }
         }
       }
@@ -480,53 +478,61 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
     // ldmatrix: matrices (tile 0, dims +0..7), (tile 0, +8..15), (tile 1, ..), (tile 1, ..)
     const int ktr = wtok + ((lane >> 4) & 1) * 8 + r7;
     const int kch = (lane >> 3) & 1;
-    // compressed reference: per-group f16 sums sum_k q~_k 2^E c_k 2^-24
-    float c8[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
-    uint32_t b8[4];          // ldmatrix words of two k-steps: (nt 0, kk), (nt 1, kk), (nt 0, kk + 1), ..
+    if constexpr (C::CRX) {
+      // ---- compressed reference: S_ref = Q C_ref^T per 32-dim slice j as
+      // integer MMAs: A = the rows' Q bytes (rows g: h, rows g + 8: l; kind
+      // 3 of qfrag), B = the codes of the n-tile's 8 tokens (ldmatrix words,
+      // one code per byte: INT8 as stored, INT4 nibble 0 | nibble 1) ----
+      int ci[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
+      uint32_t b8[4];      // (nt 0, chunk), (nt 1, chunk), (nt 0, chunk + 1), (nt 1, chunk + 1)
+      const int m = lane >> 3;
+#pragma unroll
+      for (int j = 0; j < C::NV; ++j) {
+        if constexpr (C::CR) {
+          ldsm_x4(sK + swz_offset<C::RROW>(wtok + (m & 1) * 8 + r7, 2 * j + (m >> 1)), b8);
+        } else if ((j & 1) == 0) {
+          ldsm_x4(sK + swz_offset<C::RROW>(wtok + (m & 1) * 8 + r7, j + (m >> 1)), b8);
+        }
+        const uint4 af = *reinterpret_cast<const uint4*>(qfrag + ((3 * KT) * 32 * 2) +
+                                                         (j * 32 + lane) * 4);
+        const uint32_t a[4] = {af.x, af.y, af.z, af.w};
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          uint32_t b0, b1;
+          if constexpr (C::CR) {
+            b0 = b8[nt];
+            b1 = b8[2 + nt];
+          } else {
+            const uint32_t w = b8[2 * (j & 1) + nt];
+            b0 = w & 0x0F0F0F0Fu;
+            b1 = (w >> 4) & 0x0F0F0F0Fu;
+          }
+          mma_s8u8(ci[nt], a, b0, b1);
+        }
+        if ((j + 1) % C::SPG == 0) {
+          // end of scale group jg: S += s_ref[t, jg] sig (2 <Q, c> - (2^RB - 1) sum Q)
+          const int jg = j / C::SPG;
+          const float sg = row_ok ? rsigc_s[g] : 0.0f;
+          const int off = row_ok ? (int)((1 << RB) - 1) * __float2int_rn(sqh_s[g * NG + jg]) : 0;
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) {
+            const float r0 = half_at(st + C::OFF_RSK + sc_off + tok0[nt] * SB + 2 * jg);
+            const float r1 = half_at(st + C::OFF_RSK + sc_off + (tok0[nt] + 1) * SB + 2 * jg);
+            const int x0 = 512 * ci[nt][0] + 2 * ci[nt][2] - off;
+            const int x1 = 512 * ci[nt][1] + 2 * ci[nt][3] - off;
+            cref[nt][0] = fmaf(r0 * sg, (float)x0, cref[nt][0]);
+            cref[nt][1] = fmaf(r1 * sg, (float)x1, cref[nt][1]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) ci[nt][e] = 0;
+          }
+        }
+      }
+    }
     uint32_t ck4[4];         // INT2 residual: the tile's K code words
     uint32_t ckp[4];         // 32-dim groups: the same words of lane ^ 2
 #pragma unroll
     for (int kk = 0; kk < KT; ++kk) {
-      if constexpr (C::CR) {
-        if ((kk & 1) == 0) {
-          const int m = lane >> 3;
-          ldsm_x4(sK + swz_offset<C::RROW>(wtok + (m & 1) * 8 + r7, kk + (m >> 1)), b8);
-        }
-        const uint2 fh = *reinterpret_cast<const uint2*>(qfrag + ((3 * KT + kk) * 32 + lane) * 2);
-        const uint2 fl = *reinterpret_cast<const uint2*>(qfrag + ((4 * KT + kk) * 32 + lane) * 2);
-        const uint32_t ah[4] = {fh.x, 0u, fh.y, 0u};
-        const uint32_t al[4] = {fl.x, 0u, fl.y, 0u};
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-          // codes 4q .. 4q+3 of the k-step's 16 as f16 subnormals c 2^-24, exact
-          const uint32_t w = b8[2 * (kk & 1) + nt];
-          const uint32_t b0 = __byte_perm(w, 0u, 0x4140);
-          const uint32_t b1 = __byte_perm(w, 0u, 0x4342);
-          mma_f16(c8[nt], ah, b0, b1);
-          mma_f16(c8[nt], al, b0, b1);
-        }
-      } else if constexpr (C::CR4) {
-        // one ldmatrix.x4 every four k-steps: words (nt 0, chunk), (nt 1,
-        // chunk), (nt 0, chunk + 1), (nt 1, chunk + 1) of two 32-dim chunks
-        if ((kk & 3) == 0) {
-          const int m = lane >> 3;
-          ldsm_x4(sK + swz_offset<C::RROW>(wtok + (m & 1) * 8 + r7, (kk >> 1) + (m >> 1)), b8);
-        }
-        const uint2 fh = *reinterpret_cast<const uint2*>(qfrag + ((3 * KT + kk) * 32 + lane) * 2);
-        const uint2 fl = *reinterpret_cast<const uint2*>(qfrag + ((4 * KT + kk) * 32 + lane) * 2);
-        const uint32_t ah[4] = {fh.x, 0u, fh.y, 0u};
-        const uint32_t al[4] = {fl.x, 0u, fl.y, 0u};
-        const int sh = 8 * (kk & 1);
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-          // codes i, i + 4 of the word (bits 4i, 4i + 16) as f16 subnormals c 2^-24
-          const uint32_t w = b8[2 * ((kk >> 1) & 1) + nt];
-          const uint32_t b0 = (w >> sh) & 0x000F000Fu;
-          const uint32_t b1 = (w >> (sh + 4)) & 0x000F000Fu;
-          mma_f16(c8[nt], ah, b0, b1);
-          mma_f16(c8[nt], al, b0, b1);
-        }
-      } else {
+      if constexpr (!C::CRX) {
         const int chunk = 2 * kk + kch;
         uint32_t b[4];
         ldsm_x4(sK + (chunk >> 3) * C::BOX_BYTES + ktr * 128 + (((chunk & 7) ^ r7) << 4), b);
@@ -538,21 +544,6 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
         }
         mma_bf16(cref[0], a, b[0], b[1]);
         mma_bf16(cref[1], a, b[2], b[3]);
-      }
-      if (C::CRX && (kk + 1) % KSG == 0) {
-        // end of scale group j: S += s_ref_{t, j} 2^-E (CSCALE acc - LOFF sum q~ 2^E)
-        const int j = kk / KSG;
-        const float rs = row_ok ? rsig_s[g] : 0.0f;
-        const float off = row_ok ? C::LOFF * sqh_s[g * NG + j] : 0.0f;
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-          const float r0 = half_at(st + C::OFF_RSK + sc_off + tok0[nt] * SB + 2 * j);
-          const float r1 = half_at(st + C::OFF_RSK + sc_off + (tok0[nt] + 1) * SB + 2 * j);
-          cref[nt][0] = fmaf(r0 * rs, fmaf(C::CSCALE, c8[nt][0], -off), cref[nt][0]);
-          cref[nt][1] = fmaf(r1 * rs, fmaf(C::CSCALE, c8[nt][1], -off), cref[nt][1]);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) c8[nt][e] = 0.0f;
-        }
       }
       if constexpr (C::RES) {
         const uint2 fh = *reinterpret_cast<const uint2*>(qfrag + ((1 * KT + kk) * 32 + lane) * 2);
