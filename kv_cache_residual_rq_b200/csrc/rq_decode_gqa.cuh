@@ -79,6 +79,9 @@ struct GCfg {
   // INT4 residual: a 16-byte row chunk (32 dims) always lies inside one scale
   // group; ldmatrix words of eight codes, no exchange needed
   static constexpr bool LDM4 = (BITS == 4);
+  // INT2 residual with 64-dim groups (a 16-byte chunk of a code row is one
+  // group): scores as integer MMAs, the q~ rows as 16-bit fixed point
+  static constexpr bool RIM = (BITS == 2 && GROUP == 64);
   static constexpr int NCH = D / 64;                        // 64-dim chunks per row
   static constexpr bool CR = (RB == 8);                    // INT8 compressed reference
   static constexpr bool CR4 = (RB == 4);                   // INT4 compressed reference
@@ -302,7 +305,51 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
       }
     }
     float upR = 1.0f;        // 2^E of the residual's f16 q~ fragments (row g)
-    if constexpr (C::RES) {
+    if constexpr (C::RIM) {
+      if (warp == 0) {
+        // row g of q~ as 16-bit fixed point Q = q~ / sig, as the s8 A
+        // fragments of the residual's integer MMAs: per 64-dim chunk c and
+        // code pair pp, rows g carry the h bytes and rows g + 8 the l bytes;
+        // k positions 4q + b | 16 + 4q + b carry dims 64c + 16q + 2pp + 4b | +1
+        // (codes 2pp + 4b | 2pp + 1 + 4b of the word holding dims 16q .. 16q+15)
+        float mx = 0.0f;
+        if (row_ok)
+          for (int d = q; d < D; d += 4) mx = fmaxf(mx, fabsf(cd * qt[g * D + d]));
+        mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 2));
+        const float sig = mx > 0.0f ? mx * (1.0f / 32639.0f) : 1.0f;
+        const float inv = 1.0f / sig;
+        if (row_ok && q == 0) rsig_s[g] = sig;
+#pragma unroll 1
+        for (int c = 0; c < C::NCH; ++c) {
+          int sq = 0;
+#pragma unroll
+          for (int pp = 0; pp < 2; ++pp) {
+            uint32_t a[4] = {0u, 0u, 0u, 0u};
+            if (row_ok) {
+#pragma unroll
+              for (int h2 = 0; h2 < 2; ++h2)
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                  const int dim = 64 * c + 16 * q + 2 * pp + h2 + 4 * b;
+                  const int Q =
+                      min(max(__float2int_rn(cd * qt[g * D + dim] * inv), -32639), 32639);
+                  const int lo = ((Q + 128) & 255) - 128;
+                  const int hi = (Q - lo) >> 8;
+                  a[2 * h2] |= (uint32_t)(hi & 0xFF) << (8 * b);
+                  a[2 * h2 + 1] |= (uint32_t)(lo & 0xFF) << (8 * b);
+                  sq += Q;
+                }
+            }
+            *reinterpret_cast<uint4*>(qfrag + (1 * KT) * 32 * 2 + ((2 * c + pp) * 32 + lane) * 4) =
+                make_uint4(a[0], a[1], a[2], a[3]);
+          }
+          sq += __shfl_xor_sync(FULL, sq, 1);
+          sq += __shfl_xor_sync(FULL, sq, 2);
+          if (row_ok && q == 0) sq_s[g * NG + c] = (float)sq;     // chunk c = scale group c
+        }
+      }
+    } else if constexpr (C::RES) {
       if (warp == 0) {
         float mx = 0.0f;
         if (row_ok)
@@ -336,7 +383,9 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
           const float* trow = qt + g * D + (C::LDM2 ? 64 * (kk >> 2) + lo2 : 16 * kk + 2 * q);
           fa[0] = pack_bf16(qrow[0], qrow[1]);       // exact: q is bf16
           fa[1] = pack_bf16(qrow[8], qrow[9]);
-          if constexpr (BITS == 2) {
+          if constexpr (C::RIM) {
+            // (the residual's fragments are the integer MMAs' above)
+          } else if constexpr (BITS == 2) {
             // k positions 2q, 2q+1 | 2q+8, 2q+9 carry dims 2q, 2q+8 | 2q+1, 2q+9,
             // so the two codes of a B register sit 16 bits apart
             fh[0] = pack_f16(cd * trow[0] * upR, cd * trow[8] * upR);
@@ -357,9 +406,10 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
             split_bf16(cd * trow[8], cd * trow[9], fh[1], fl[1]);
           }
         } else {
-          fa[0] = fa[1] = fh[0] = fh[1] = fl[0] = fl[1] = 0u;
+          fa[0] = fa[1] = 0u;
+          if constexpr (!C::RIM) fh[0] = fh[1] = fl[0] = fl[1] = 0u;
         }
-        if ((BITS == 2 || C::LDM4) && (kk + 1) % KSG == 0) {      // end of a scale group
+        if ((BITS == 2 || C::LDM4) && !C::RIM && (kk + 1) % KSG == 0) {   // end of a scale group
           sqj += __shfl_xor_sync(FULL, sqj, 1);
           sqj += __shfl_xor_sync(FULL, sqj, 2);
           if (row_ok && q == 0) sq_s[g * NG + kk / KSG] = sqj;
@@ -545,7 +595,7 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
         mma_bf16(cref[0], a, b[0], b[1]);
         mma_bf16(cref[1], a, b[2], b[3]);
       }
-      if constexpr (C::RES) {
+      if constexpr (C::RES && !C::RIM) {
         const uint2 fh = *reinterpret_cast<const uint2*>(qfrag + ((1 * KT + kk) * 32 + lane) * 2);
         const uint32_t ah[4] = {fh.x, 0u, fh.y, 0u};
         if constexpr (C::LDM4) {
@@ -622,6 +672,53 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) ct[nt][e] = 0.0f;
           }
+        }
+      }
+    }
+    if constexpr (C::RIM) {
+      // ---- residual scores as integer MMAs per 64-dim chunk (one scale
+      // group): A = the rows' Q bytes (h | l), B = the n-tile's code words
+      // (ldmatrix: lane q holds dims 16q .. 16q+15 of the chunk), one code
+      // per byte by a shift and a mask per four codes ----
+      uint32_t w4[4];        // (nt 0, chunk 0), (nt 1, chunk 0)[, (nt 0, chunk 1), (nt 1, chunk 1)]
+      {
+        const int m = (lane >> 3) & (2 * C::NCH - 1);
+        const uint32_t a = smem_u32(st + C::OFF_CK + (wtok + (m & 1) * 8 + r7) * C::CROW +
+                                    (m >> 1) * 16);
+        if constexpr (C::NCH == 2) {
+          ldsm_x4(a, w4);
+        } else {
+          uint32_t r2[2];
+          ldsm_x2(a, r2);
+          w4[0] = r2[0];
+          w4[1] = r2[1];
+        }
+      }
+      const float sg = row_ok ? rsig_s[g] : 0.0f;
+#pragma unroll
+      for (int c = 0; c < C::NCH; ++c) {
+        int ci[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
+#pragma unroll
+        for (int pp = 0; pp < 2; ++pp) {
+          const uint4 af = *reinterpret_cast<const uint4*>(qfrag + (1 * KT) * 32 * 2 +
+                                                           ((2 * c + pp) * 32 + lane) * 4);
+          const uint32_t a[4] = {af.x, af.y, af.z, af.w};
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) {
+            const uint32_t w = w4[2 * c + nt];
+            mma_s8u8(ci[nt], a, (w >> (4 * pp)) & 0x03030303u, (w >> (4 * pp + 2)) & 0x03030303u);
+          }
+        }
+        // scale group c: S += s^K[t, c] sig (2 <Q, c> - 3 sum Q)
+        const int off = row_ok ? TOPLVL * __float2int_rn(sq_s[g * NG + c]) : 0;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          const float sk0 = half_at(st + C::OFF_SK + sc_off + tok0[nt] * SB + 2 * c);
+          const float sk1 = half_at(st + C::OFF_SK + sc_off + (tok0[nt] + 1) * SB + 2 * c);
+          const int x0 = 512 * ci[nt][0] + 2 * ci[nt][2] - off;
+          const int x1 = 512 * ci[nt][1] + 2 * ci[nt][3] - off;
+          cref[nt][0] = fmaf(sk0 * sg, (float)x0, cref[nt][0]);
+          cref[nt][1] = fmaf(sk1 * sg, (float)x1, cref[nt][1]);
         }
       }
     }
