@@ -231,22 +231,24 @@ decode_cr1_kernel(const __grid_constant__ TcParams gp) {
     float* qt = qbuf + D;
     load_rotate_queries<D, 1>(p, hd, qs, qt, tid);
     const float cd = rot_scale<D>();
-    if (tid < NV) {
-      // slice v of q~ as 16-bit fixed point: Q = q~ / sig, |Q| <= 32639 so
-      // that Q = 256 h + l has signed-byte h and l
-      const int v = tid;
-      float mx = 0.0f;
-      for (int k = 0; k < 32; ++k) mx = fmaxf(mx, fabsf(cd * qt[32 * v + k]));
+    if (warp < NV) {
+      // slice v = warp of q~ as 16-bit fixed point, one dim per lane: Q =
+      // q~ / sig, |Q| <= 32639 so that Q = 256 h + l has signed-byte h and l
+      const float x = cd * qt[32 * warp + lane];
+      float mx = fabsf(x);
+#pragma unroll
+      for (int m = 1; m < 32; m <<= 1) mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, m));
       const float sig = mx > 0.0f ? mx * (1.0f / 32639.0f) : 1.0f;
       const float inv = 1.0f / sig;
-      int sum = 0;
-      for (int k = 0; k < 32; ++k) {
-        const int Q = min(max(__float2int_rn(cd * qt[32 * v + k] * inv), -32639), 32639);
-        qi[32 * v + k] = Q;
-        sum += Q;
+      const int Q = min(max(__float2int_rn(x * inv), -32639), 32639);
+      qi[32 * warp + lane] = Q;
+      int sum = Q;
+#pragma unroll
+      for (int m = 1; m < 32; m <<= 1) sum += __shfl_xor_sync(FULL, sum, m);
+      if (lane == 0) {
+        qsig_s[warp] = sig;
+        qsum_s[warp] = sum;
       }
-      qsig_s[v] = sig;
-      qsum_s[v] = sum;
     }
     named_bar_sync(1, kConsumerThreads);
     // byte (0: h, 1: l) of Q[dim] for this lane's B column (slice g / 2),
@@ -258,20 +260,20 @@ decode_cr1_kernel(const __grid_constant__ TcParams gp) {
       const int hi = (Q - lo) >> 8;
       return (uint32_t)(((g & 1) ? lo : hi) & 0xFF);
     };
-    if (warp == 0) {
+    // the MMAs' fragments, spread over the consumer warps
 #pragma unroll 1
-      for (int i = 0; i < NV + 4; ++i)
+    for (int i = warp; i < NV + 4; i += kConsumerWarps) {
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t w = 0u;
+      for (int h = 0; h < 2; ++h) {
+        uint32_t w = 0u;
 #pragma unroll
-          for (int b = 0; b < 4; ++b) {
-            const int dim = i < NV ? kdim_ref<RB>(i, 16 * h, t, b)
-                                   : kdim_res<BITS == 4 ? 4 : 2>(i - NV, 16 * h, t, b);
-            w |= qbyte(dim) << (8 * b);
-          }
-          kfrag[(i * 32 + lane) * 2 + h] = w;
+        for (int b = 0; b < 4; ++b) {
+          const int dim = i < NV ? kdim_ref<RB>(i, 16 * h, t, b)
+                                 : kdim_res<BITS == 4 ? 4 : 2>(i - NV, 16 * h, t, b);
+          w |= qbyte(dim) << (8 * b);
         }
+        kfrag[(i * 32 + lane) * 2 + h] = w;
+      }
     }
     const bool slice_ok = t < NV;
     ksig = slice_ok ? qsig_s[tv] * p.score_scale : 0.0f;
