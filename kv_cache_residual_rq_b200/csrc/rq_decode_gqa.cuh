@@ -86,6 +86,10 @@ struct GCfg {
   static constexpr bool CR = (RB == 8);                    // INT8 compressed reference
   static constexpr bool CR4 = (RB == 4);                   // INT4 compressed reference
   static constexpr bool CRX = (RB != 0);                   // either
+  // INT8 compressed reference with an INT2 residual: the residual's value
+  // products go into the reference's f16 accumulators (one set of value
+  // accumulators; the other combinations keep their own)
+  static constexpr bool VSH = (RB == 8 && BITS == 2);
   static constexpr int RROW = CRX ? D * RB / 8 : 0;        // reference code bytes per token
   // f16 operands of the reference codes: the exact subnormals c 2^-24 (the
   // code in the low mantissa bits, no offset).  A sum acc over those operands
@@ -111,6 +115,7 @@ struct GCfg {
   static constexpr int OFF_RSV = OFF_RSK + RSC_BYTES;
   static constexpr int STAGE_BYTES = (OFF_RSV + RSC_BYTES + 1023) / 1024 * 1024;
   static constexpr int STAGES = 2;
+
   static constexpr int RING_BYTES = STAGES * STAGE_BYTES;
   static constexpr int MERGE_FLOATS = kConsumerWarps * G * (2 + 2 * D);
   static constexpr int QBUF_FLOATS = 2 * G * D;
@@ -123,7 +128,15 @@ struct GCfg {
   static constexpr int WSUM_FLOATS = kConsumerWarps * G * NG * (CRX ? 2 : 1);
   // q, q~ high, q~ remainder (bf16); with a compressed reference also
   // q~ 2^E high, remainder (f16, k-permuted for the reference's codes)
-  static constexpr int QFRAG_WORDS = 3 * KT * 32 * 2 + (CRX ? NV * 32 * 4 : 0);
+  // qfrag regions (32-bit words): kind 0 at QF0 (the bf16 query; BF16
+  // reference only), kinds 1 and 2 at QF1, QF1 + KT * 64 (the residual's f16
+  // fragments), or at QF1 the residual's integer-MMA fragments (RIM), and the
+  // compressed reference's integer-MMA fragments at QFC
+  static constexpr int QF0 = 0;
+  static constexpr int QF1 = CRX ? 0 : KT * 64;
+  static constexpr int QF12_WORDS = RIM ? NCH * 256 : (RES ? 2 * KT * 64 : 0);
+  static constexpr int QFC = QF1 + QF12_WORDS;
+  static constexpr int QFRAG_WORDS = QFC + (CRX ? NV * 32 * 4 : 0);
   // INT2: per (row, scale group) sum of the q~ fragments' values (offset of
   // the 128 + 2c operands); compressed reference: the same for the f16
   // fragments (the levels' 2^b - 1) and per row 2^-E; even count to keep the
@@ -134,6 +147,12 @@ struct GCfg {
                                     4 * (MERGE_FLOATS + QBUF_FLOATS + WSUM_FLOATS +
                                          QFRAG_WORDS + SQ_FLOATS) +
                                     2 * STAGES * 8 + 16 + STAGES * 8;   // + stage rows
+  // resident CTAs per SM: two (168 registers); with one set of value
+  // accumulators (VSH, or a compressed reference alone) three (128
+  // registers) where their shared memory fits (228 KB per SM, 1 KB of it
+  // reserved per CTA)
+  static constexpr bool FITS3 = SMEM_BYTES <= 228 * 1024 / 3 - 1024;
+  static constexpr int CTAS = ((VSH || (CRX && !RES)) && FITS3) ? 3 : 2;
   static_assert(G == 2 || G == 4 || G == 8, "grouped queries");
   static_assert(MERGE_FLOATS >= kVarlenMaxBatch + 1, "merge area holds the length scan");
   static_assert(GROUP == 32 || GROUP == 64, "scale group");
@@ -145,7 +164,7 @@ struct GCfg {
 
 
 template <int D, int G, int BITS, int GROUP, int RB>
-__global__ void __launch_bounds__(kDecodeThreads, 2)
+__global__ void __launch_bounds__(kDecodeThreads, GCfg<D, G, BITS, GROUP, RB>::CTAS)
 decode_gqa_kernel(const __grid_constant__ TcParams gp) {
   using C = GCfg<D, G, BITS, GROUP, RB>;
   const DecodeParams& p = gp.p;
@@ -225,9 +244,6 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
   // kind 2 holds per 32-dim slice and lane the four s8 A words {a0, a1, a2,
   // a3} of the reference's integer MMAs (rows g: bytes h of Q, rows g + 8:
   // bytes l, in the k order of the reference's code words).
-  auto qfrag_addr = [&](int kind, int kk) {
-    return smem_u32(qfrag + ((kind * KT + kk) * 32 + lane) * 2);
-  };
   // softmax state of row g (lanes with row_ok), and the output accumulators
   // (O^T fragments: dims 16mt + g (+8), rows 2q, 2q + 1)
   float m_run = kNegInf, l_run = 0.0f;
@@ -293,7 +309,7 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
                 sq += Q;
               }
           }
-          *reinterpret_cast<uint4*>(qfrag + ((3 * KT) * 32 * 2) + (j * 32 + lane) * 4) =
+          *reinterpret_cast<uint4*>(qfrag + C::QFC + (j * 32 + lane) * 4) =
               make_uint4(a[0], a[1], a[2], a[3]);
           if ((j + 1) % C::SPG == 0) {                // end of a scale group
             sq += __shfl_xor_sync(FULL, sq, 1);
@@ -341,7 +357,7 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
                   sq += Q;
                 }
             }
-            *reinterpret_cast<uint4*>(qfrag + (1 * KT) * 32 * 2 + ((2 * c + pp) * 32 + lane) * 4) =
+            *reinterpret_cast<uint4*>(qfrag + C::QF1 + ((2 * c + pp) * 32 + lane) * 4) =
                 make_uint4(a[0], a[1], a[2], a[3]);
           }
           sq += __shfl_xor_sync(FULL, sq, 1);
@@ -366,9 +382,11 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
       float sqj = 0.0f;      // running sum of the current scale group (INT2)
 #pragma unroll 1
       for (int kk = 0; kk < KT; ++kk) {
-        uint32_t* fa = qfrag + ((0 * KT + kk) * 32 + lane) * 2;
-        uint32_t* fh = qfrag + ((1 * KT + kk) * 32 + lane) * 2;
-        uint32_t* fl = qfrag + ((2 * KT + kk) * 32 + lane) * 2;
+        // (kind 0 only for a BF16 reference, kinds 1 and 2 only for the f16
+        // residual form; the others' regions hold other fragments or none)
+        uint32_t* fa = qfrag + C::QF0 + (kk * 32 + lane) * 2;
+        uint32_t* fh = qfrag + C::QF1 + (kk * 32 + lane) * 2;
+        uint32_t* fl = qfrag + C::QF1 + KT * 64 + (kk * 32 + lane) * 2;
         if (row_ok) {
           const float* qrow = qs + g * D + 16 * kk + 2 * q;
           // INT2 with ldmatrix words: k-step kk = 4c + t of chunk c carries
@@ -381,9 +399,11 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
                                       : 32 * ((kk >> 1) & 1) + 16 * (q & 1) +
                                             2 * (2 * (kk & 1) + (q >> 1));
           const float* trow = qt + g * D + (C::LDM2 ? 64 * (kk >> 2) + lo2 : 16 * kk + 2 * q);
-          fa[0] = pack_bf16(qrow[0], qrow[1]);       // exact: q is bf16
-          fa[1] = pack_bf16(qrow[8], qrow[9]);
-          if constexpr (C::RIM) {
+          if constexpr (!C::CRX) {
+            fa[0] = pack_bf16(qrow[0], qrow[1]);     // exact: q is bf16
+            fa[1] = pack_bf16(qrow[8], qrow[9]);
+          }
+          if constexpr (C::RIM || !C::RES) {
             // (the residual's fragments are the integer MMAs' above)
           } else if constexpr (BITS == 2) {
             // k positions 2q, 2q+1 | 2q+8, 2q+9 carry dims 2q, 2q+8 | 2q+1, 2q+9,
@@ -401,13 +421,10 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
             fh[1] = pack_f16(cd * t4[1] * upR, cd * t4[5] * upR);
             fl[0] = fl[1] = 0u;
             sqj += (f16_lo_f(fh[0]) + f16_hi_f(fh[0])) + (f16_lo_f(fh[1]) + f16_hi_f(fh[1]));
-          } else {
-            split_bf16(cd * trow[0], cd * trow[1], fh[0], fl[0]);
-            split_bf16(cd * trow[8], cd * trow[9], fh[1], fl[1]);
           }
         } else {
-          fa[0] = fa[1] = 0u;
-          if constexpr (!C::RIM) fh[0] = fh[1] = fl[0] = fl[1] = 0u;
+          if constexpr (!C::CRX) fa[0] = fa[1] = 0u;
+          if constexpr (C::RES && !C::RIM) fh[0] = fh[1] = fl[0] = fl[1] = 0u;
         }
         if ((BITS == 2 || C::LDM4) && !C::RIM && (kk + 1) % KSG == 0) {   // end of a scale group
           sqj += __shfl_xor_sync(FULL, sqj, 1);
@@ -447,7 +464,7 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
       mw[g * (2 + 2 * D) + 1] = l_run;
 #pragma unroll
       for (int j = 0; j < NG; ++j) {
-        if constexpr (C::RES) wsum_s[(warp * G + g) * NG + j] = wsum[j];
+        if constexpr (C::RES) wsum_s[(warp * G + g) * NG + j] = wsum[j] * (C::VSH ? 1.0f / vscale : 1.0f);
         if constexpr (C::CRX) wsumR_s[(warp * G + g) * NG + j] = wsumR[j] * (1.0f / vscale);
       }
     }
@@ -472,7 +489,7 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
         if (r < G) {
           if constexpr (C::CRX) mw[r * (2 + 2 * D) + 2 + dim_ref] = oref[mt][e] * (C::CSCALE / vscale);
           else mw[r * (2 + 2 * D) + 2 + dim_ref] = oref[mt][e];
-          if constexpr (C::RES) mw[r * (2 + 2 * D) + 2 + D + dim_res] = 2.0f * ores[mt][e];
+          if constexpr (C::RES && !C::VSH) mw[r * (2 + 2 * D) + 2 + D + dim_res] = 2.0f * ores[mt][e];
           else mw[r * (2 + 2 * D) + 2 + D + dim] = 0.0f;
         }
       }
@@ -543,8 +560,7 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
         } else if ((j & 1) == 0) {
           ldsm_x4(sK + swz_offset<C::RROW>(wtok + (m & 1) * 8 + r7, j + (m >> 1)), b8);
         }
-        const uint4 af = *reinterpret_cast<const uint4*>(qfrag + ((3 * KT) * 32 * 2) +
-                                                         (j * 32 + lane) * 4);
+        const uint4 af = *reinterpret_cast<const uint4*>(qfrag + C::QFC + (j * 32 + lane) * 4);
         const uint32_t a[4] = {af.x, af.y, af.z, af.w};
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
@@ -588,7 +604,7 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
         ldsm_x4(sK + (chunk >> 3) * C::BOX_BYTES + ktr * 128 + (((chunk & 7) ^ r7) << 4), b);
         uint32_t a[4] = {0u, 0u, 0u, 0u};
         {
-          const uint2 f = *reinterpret_cast<const uint2*>(qfrag + ((0 * KT + kk) * 32 + lane) * 2);
+          const uint2 f = *reinterpret_cast<const uint2*>(qfrag + C::QF0 + (kk * 32 + lane) * 2);
           a[0] = f.x;
           a[2] = f.y;
         }
@@ -596,7 +612,7 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
         mma_bf16(cref[1], a, b[2], b[3]);
       }
       if constexpr (C::RES && !C::RIM) {
-        const uint2 fh = *reinterpret_cast<const uint2*>(qfrag + ((1 * KT + kk) * 32 + lane) * 2);
+        const uint2 fh = *reinterpret_cast<const uint2*>(qfrag + C::QF1 + (kk * 32 + lane) * 2);
         const uint32_t ah[4] = {fh.x, 0u, fh.y, 0u};
         if constexpr (C::LDM4) {
           // every fourth k-step: words (nt 0, chunk), (nt 1, chunk), (nt 0,
@@ -700,7 +716,7 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
         int ci[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
 #pragma unroll
         for (int pp = 0; pp < 2; ++pp) {
-          const uint4 af = *reinterpret_cast<const uint4*>(qfrag + (1 * KT) * 32 * 2 +
+          const uint4 af = *reinterpret_cast<const uint4*>(qfrag + C::QF1 +
                                                            ((2 * c + pp) * 32 + lane) * 4);
           const uint32_t a[4] = {af.x, af.y, af.z, af.w};
 #pragma unroll
@@ -754,7 +770,7 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
         float2 x = __fmul2_rn(make_float2(oref[mt][0], oref[mt][1]), a01);
         float2 y = __fmul2_rn(make_float2(oref[mt][2], oref[mt][3]), a01);
         oref[mt][0] = x.x; oref[mt][1] = x.y; oref[mt][2] = y.x; oref[mt][3] = y.y;
-        if constexpr (C::RES) {
+        if constexpr (C::RES && !C::VSH) {
           x = __fmul2_rn(make_float2(ores[mt][0], ores[mt][1]), a01);
           y = __fmul2_rn(make_float2(ores[mt][2], ores[mt][3]), a01);
           ores[mt][0] = x.x; ores[mt][1] = x.y; ores[mt][2] = y.x; ores[mt][3] = y.y;
@@ -790,11 +806,24 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
         const float v = half_at(st + C::OFF_RSV + sc_off + tk[k] * SB + 2 * j);
         return (tk[k] < n) ? v : 0.0f;
       };
+      // the residual's value products land in the same accumulators, with
+      // the same power of two on their weights p s^V
+      auto s_res_v = [&](int k, int j) {
+        if constexpr (C::VSH) {
+          const float v = half_at(st + C::OFF_SV + sc_off + tk[k] * SB + 2 * j);
+          return (tk[k] < n) ? v : 0.0f;
+        } else {
+          return 0.0f;
+        }
+      };
       float smax = 0.0f;
 #pragma unroll
       for (int j = 0; j < NG; ++j)
 #pragma unroll
-        for (int k = 0; k < 4; ++k) smax = fmaxf(smax, fabsf(s_ref_v(k, j)));
+        for (int k = 0; k < 4; ++k) {
+          smax = fmaxf(smax, fabsf(s_ref_v(k, j)));
+          if constexpr (C::VSH) smax = fmaxf(smax, fabsf(s_res_v(k, j)));
+        }
       smax = fmaxf(smax, __shfl_xor_sync(FULL, smax, 1));
       smax = fmaxf(smax, __shfl_xor_sync(FULL, smax, 2));
       {
@@ -809,12 +838,43 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) oref[mt][e] *= f;
 #pragma unroll
-          for (int j = 0; j < NG; ++j) wsumR[j] *= f;
+          for (int j = 0; j < NG; ++j) {
+            wsumR[j] *= f;
+            if constexpr (C::VSH) wsum[j] *= f;
+          }
           vscale = nv;
         }
       }
       const float pk[4] = {pr[0][0] * vscale, pr[0][1] * vscale, pr[1][0] * vscale,
                            pr[1][1] * vscale};
+      // The residual's V codes on the reference's m-rows, as f16 subnormals:
+      // m-row g (+ 8) of m-tile mt is dim d0 (+ 1), d0 = 16mt + 2g (INT8
+      // reference) or 32 (mt / 2) + 4g + 2 (mt & 1) (INT4 reference); one
+      // byte permute puts the byte holding d0's code of tokens 2q, 2q + 1
+      // (and 2q + 8, 2q + 9) into halves 0 and 1, a shift brings d0's code to
+      // bit 0 and d0 + 1's follows at bit BITS.
+      auto res_frag = [&](int mt, uint32_t (&a)[4]) {
+        if constexpr (C::VSH) {
+          const int d0 = C::CR ? 16 * mt + 2 * g : 32 * (mt >> 1) + 4 * g + 2 * (mt & 1);
+          const int wi = d0 * BITS / 32;                       // word holding d0's code
+          const int bit = (d0 * BITS) & 31;                    // its bit in the word
+          const uint32_t bs = (uint32_t)(bit >> 3);             // byte of the word
+          const uint32_t psel = bs | (bs << 4) | ((4u + bs) << 8) | ((4u + bs) << 12);
+          const int sh = bit & 7;
+          const unsigned char* cvb = st + C::OFF_CV + wi * 4;
+          const uint32_t x01 =
+              __byte_perm(*reinterpret_cast<const uint32_t*>(cvb + tk[0] * C::CROW),
+                          *reinterpret_cast<const uint32_t*>(cvb + tk[1] * C::CROW), psel) >> sh;
+          const uint32_t x23 =
+              __byte_perm(*reinterpret_cast<const uint32_t*>(cvb + tk[2] * C::CROW),
+                          *reinterpret_cast<const uint32_t*>(cvb + tk[3] * C::CROW), psel) >> sh;
+          constexpr uint32_t M = (BITS == 2) ? 0x00030003u : 0x000F000Fu;
+          a[0] = x01 & M;
+          a[1] = (x01 >> BITS) & M;
+          a[2] = x23 & M;
+          a[3] = (x23 >> BITS) & M;
+        }
+      };
 #pragma unroll
       for (int j = 0; j < NG; ++j) {
         float wv[4];
@@ -824,6 +884,23 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
         uint32_t bh0, bl0, bh1, bl1;
         split_f16(wv[0], wv[1], bh0, bl0);
         split_f16(wv[2], wv[3], bh1, bl1);
+        uint32_t rh0 = 0u, rl0 = 0u, rh1 = 0u, rl1 = 0u;   // the residual's weights
+        if constexpr (C::VSH) {
+          float wr[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) wr[k] = pk[k] * s_res_v(k, j);
+          wsum[j] += (wr[0] + wr[1]) + (wr[2] + wr[3]);
+          split_f16(wr[0], wr[1], rh0, rl0);
+          split_f16(wr[2], wr[3], rh1, rl1);
+        }
+        auto residual_mma = [&](int mt) {
+          if constexpr (C::VSH) {
+            uint32_t a[4];
+            res_frag(mt, a);
+            mma_f16(oref[mt], a, rh0, rh1);
+            mma_f16(oref[mt], a, rl0, rl1);
+          }
+        };
         if constexpr (C::CR4) {
 #pragma unroll
           for (int ch = j * GROUP / 32; ch < (j + 1) * GROUP / 32; ++ch) {
@@ -837,6 +914,7 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
                                      (v[1] >> sh) & 0x000F000Fu, (v[1] >> (sh + 4)) & 0x000F000Fu};
               mma_f16(oref[2 * ch + h], a, bh0, bh1);
               mma_f16(oref[2 * ch + h], a, bl0, bl1);
+              residual_mma(2 * ch + h);
             }
           }
         } else {
@@ -856,6 +934,7 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
                   __byte_perm(R1, 0u, 0x4240), __byte_perm(R1, 0u, 0x4341)};
               mma_f16(oref[mt], a, bh0, bh1);
               mma_f16(oref[mt], a, bl0, bl1);
+              residual_mma(mt);
             }
           }
         }
@@ -875,8 +954,9 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
         mma_bf16(oref[mt], a, pl0, pl1);
       }
     }
-    // ---- O_res^T += C_V^T (P s^V)^T ----
-    if constexpr (C::RES) {
+    // ---- O_res^T += C_V^T (P s^V)^T (an INT8 compressed reference with an
+    // INT2 residual takes these products into its accumulators above) ----
+    if constexpr (C::RES && !C::VSH) {
       const int tk[4] = {wtok + 2 * q, wtok + 2 * q + 1, wtok + 2 * q + 8, wtok + 2 * q + 9};
       const float pk[4] = {pr[0][0], pr[0][1], pr[1][0], pr[1][1]};
       // INT2, 64-dim groups: the warp tile's V code words by one
@@ -994,8 +1074,17 @@ cudaError_t launch_gqa_t(const TcParams& gp, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  return launch_pdl(decode_gqa_kernel<D, G, BITS, GROUP, RB>, gp.p.ctas, kDecodeThreads,
-                    C::SMEM_BYTES, stream, gp);
+  TcParams g2 = gp;
+  if constexpr (C::CTAS != kDecodeCtasPerSm) {
+    // the call's CTAs: CTAS per SM, no more than its tiles (uniform calls)
+    long long P = (long long)device_sm_count() * C::CTAS;
+    if (P > kDecodeMaxCtas) P = kDecodeMaxCtas;
+    if (!g2.p.ctx_lens && P > g2.p.n_tiles) P = g2.p.n_tiles;
+    if (P < 1) P = 1;
+    g2.p.ctas = (int)P;
+  }
+  return launch_pdl(decode_gqa_kernel<D, G, BITS, GROUP, RB>, g2.p.ctas, kDecodeThreads,
+                    C::SMEM_BYTES, stream, g2);
 }
 
 template <int D, int G, int RB>
