@@ -536,14 +536,18 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
     }
     const uint32_t sK = smem_u32(st + C::OFF_K);
     const uint32_t sV = smem_u32(st + C::OFF_V);
-    const int r7 = lane & 7;
+    // ldmatrix row order: the row addressed by lane r (of a matrix's eight)
+    // is token (r >> 1) + 4 (r & 1) of its 8-token half, so n / k positions
+    // 2q, 2q + 1 carry tokens q, q + 4 (the four lanes of a row group then
+    // read four consecutive rows of the plainly loaded code rows)
+    const int pr7 = ((lane & 7) >> 1) | ((lane & 1) << 2);
     // ---- scores for the warp's two 8-token tiles, k-steps outermost ----
-    // c[nt]: S_ref (then + s x S_res) fragments, row g, tokens 2q, 2q+1 of nt
+    // c[nt]: S_ref (then + s x S_res) fragments, row g, tokens q, q + 4 of nt
     float cref[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
     float ct[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
-    const int tok0[2] = {wtok + 2 * q, wtok + 8 + 2 * q};     // tokens of c0 per tile
+    const int tok0[2] = {wtok + q, wtok + 8 + q};     // tokens of c0 per tile (c1: + 4)
     // ldmatrix: matrices (tile 0, dims +0..7), (tile 0, +8..15), (tile 1, ..), (tile 1, ..)
-    const int ktr = wtok + ((lane >> 4) & 1) * 8 + r7;
+    const int ktr = wtok + ((lane >> 4) & 1) * 8 + pr7;
     const int kch = (lane >> 3) & 1;
     if constexpr (C::CRX) {
       // ---- compressed reference: S_ref = Q C_ref^T per 32-dim slice j as
@@ -556,9 +560,9 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
 #pragma unroll
       for (int j = 0; j < C::NV; ++j) {
         if constexpr (C::CR) {
-          ldsm_x4(sK + swz_offset<C::RROW>(wtok + (m & 1) * 8 + r7, 2 * j + (m >> 1)), b8);
+          ldsm_x4(sK + swz_offset<C::RROW>(wtok + (m & 1) * 8 + pr7, 2 * j + (m >> 1)), b8);
         } else if ((j & 1) == 0) {
-          ldsm_x4(sK + swz_offset<C::RROW>(wtok + (m & 1) * 8 + r7, j + (m >> 1)), b8);
+          ldsm_x4(sK + swz_offset<C::RROW>(wtok + (m & 1) * 8 + pr7, j + (m >> 1)), b8);
         }
         const uint4 af = *reinterpret_cast<const uint4*>(qfrag + C::QFC + (j * 32 + lane) * 4);
         const uint32_t a[4] = {af.x, af.y, af.z, af.w};
@@ -583,7 +587,7 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
 #pragma unroll
           for (int nt = 0; nt < 2; ++nt) {
             const float r0 = half_at(st + C::OFF_RSK + sc_off + tok0[nt] * SB + 2 * jg);
-            const float r1 = half_at(st + C::OFF_RSK + sc_off + (tok0[nt] + 1) * SB + 2 * jg);
+            const float r1 = half_at(st + C::OFF_RSK + sc_off + (tok0[nt] + 4) * SB + 2 * jg);
             const int x0 = 512 * ci[nt][0] + 2 * ci[nt][2] - off;
             const int x1 = 512 * ci[nt][1] + 2 * ci[nt][3] - off;
             cref[nt][0] = fmaf(r0 * sg, (float)x0, cref[nt][0]);
@@ -601,7 +605,7 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
       if constexpr (!C::CRX) {
         const int chunk = 2 * kk + kch;
         uint32_t b[4];
-        ldsm_x4(sK + (chunk >> 3) * C::BOX_BYTES + ktr * 128 + (((chunk & 7) ^ r7) << 4), b);
+        ldsm_x4(sK + (chunk >> 3) * C::BOX_BYTES + ktr * 128 + (((chunk & 7) ^ pr7) << 4), b);
         uint32_t a[4] = {0u, 0u, 0u, 0u};
         {
           const uint2 f = *reinterpret_cast<const uint2*>(qfrag + C::QF0 + (kk * 32 + lane) * 2);
@@ -619,7 +623,7 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
           // chunk + 1), (nt 1, chunk + 1) of two 32-dim chunks
           if ((kk & 3) == 0) {
             const int m = lane >> 3;
-            ldsm_x4(smem_u32(st + C::OFF_CK + (wtok + (m & 1) * 8 + r7) * C::CROW +
+            ldsm_x4(smem_u32(st + C::OFF_CK + (wtok + (m & 1) * 8 + pr7) * C::CROW +
                              ((kk >> 1) + (m >> 1)) * 16),
                     ck4);
           }
@@ -629,7 +633,7 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
           // 0), (nt 1, chunk 0)[, (nt 0, chunk 1), (nt 1, chunk 1)]
           if (kk == 0) {
             const int m = (lane >> 3) & (2 * C::NCH - 1);
-            const uint32_t a = smem_u32(st + C::OFF_CK + (wtok + (m & 1) * 8 + r7) * C::CROW +
+            const uint32_t a = smem_u32(st + C::OFF_CK + (wtok + (m & 1) * 8 + pr7) * C::CROW +
                                         (m >> 1) * 16);
             if constexpr (C::NCH == 2) {
               ldsm_x4(a, ck4);
@@ -682,7 +686,7 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
 #pragma unroll
           for (int nt = 0; nt < 2; ++nt) {
             const float sk0 = half_at(st + C::OFF_SK + sc_off + tok0[nt] * SB + 2 * j);
-            const float sk1 = half_at(st + C::OFF_SK + sc_off + (tok0[nt] + 1) * SB + 2 * j);
+            const float sk1 = half_at(st + C::OFF_SK + sc_off + (tok0[nt] + 4) * SB + 2 * j);
             cref[nt][0] = fmaf(sk0 * rsR, fmaf(C::CSCALE, ct[nt][0], -offR), cref[nt][0]);
             cref[nt][1] = fmaf(sk1 * rsR, fmaf(C::CSCALE, ct[nt][1], -offR), cref[nt][1]);
 #pragma unroll
@@ -699,7 +703,7 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
       uint32_t w4[4];        // (nt 0, chunk 0), (nt 1, chunk 0)[, (nt 0, chunk 1), (nt 1, chunk 1)]
       {
         const int m = (lane >> 3) & (2 * C::NCH - 1);
-        const uint32_t a = smem_u32(st + C::OFF_CK + (wtok + (m & 1) * 8 + r7) * C::CROW +
+        const uint32_t a = smem_u32(st + C::OFF_CK + (wtok + (m & 1) * 8 + pr7) * C::CROW +
                                     (m >> 1) * 16);
         if constexpr (C::NCH == 2) {
           ldsm_x4(a, w4);
@@ -730,7 +734,7 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
           const float sk0 = half_at(st + C::OFF_SK + sc_off + tok0[nt] * SB + 2 * c);
-          const float sk1 = half_at(st + C::OFF_SK + sc_off + (tok0[nt] + 1) * SB + 2 * c);
+          const float sk1 = half_at(st + C::OFF_SK + sc_off + (tok0[nt] + 4) * SB + 2 * c);
           const int x0 = 512 * ci[nt][0] + 2 * ci[nt][2] - off;
           const int x1 = 512 * ci[nt][1] + 2 * ci[nt][3] - off;
           cref[nt][0] = fmaf(sk0 * sg, (float)x0, cref[nt][0]);
@@ -738,11 +742,11 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
         }
       }
     }
-    float sc[2][2];          // row g, tokens 2q, 2q+1 of tile nt
+    float sc[2][2];          // row g, tokens q, q + 4 of tile nt
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
       sc[nt][0] = (row_ok && tok0[nt] < n) ? score_scale * cref[nt][0] : kNegInf;
-      sc[nt][1] = (row_ok && tok0[nt] + 1 < n) ? score_scale * cref[nt][1] : kNegInf;
+      sc[nt][1] = (row_ok && tok0[nt] + 4 < n) ? score_scale * cref[nt][1] : kNegInf;
     }
     // ---- online softmax of row g (four lanes per row), rescaled lazily ----
     float mc = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
@@ -782,17 +786,17 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
         wsumR[j] *= alpha;
       }
     }
-    // P^T fragments (k = tokens 2q, 2q+1 / +8, n = row g): bf16 hi + lo
+    // P^T fragments (k = tokens q, q + 4 / + 8, n = row g): bf16 hi + lo
     const uint32_t ph0 = pack_bf16(pr[0][0], pr[0][1]);
     const uint32_t ph1 = pack_bf16(pr[1][0], pr[1][1]);
     const uint32_t pl0 = pack_bf16(pr[0][0] - bf16_lo_f(ph0), pr[0][1] - bf16_hi_f(ph0));
     const uint32_t pl1 = pack_bf16(pr[1][0] - bf16_lo_f(ph1), pr[1][1] - bf16_hi_f(ph1));
     if constexpr (C::CRX) {
       // ---- O_ref^T += C_ref^T (P s_ref^V 2^Ev)^T, codes as f16 subnormals ----
-      // ldmatrix.trans of the code rows.  INT8: word = codes (token 2q: dims
-      // 2g, 2g+1; token 2q+1: dims 2g, 2g+1) of a 16-dim chunk; m-row g is
+      // ldmatrix.trans of the code rows.  INT8: word = codes (token q: dims
+      // 2g, 2g+1; token q + 4: dims 2g, 2g+1) of a 16-dim chunk; m-row g is
       // dim 2g, m-row g + 8 dim 2g + 1.  INT4: word = codes of dims 4g .. 4g+3
-      // of a 32-dim chunk (token 2q low half, 2q+1 high half, code i at bits
+      // of a 32-dim chunk (token q low half, q + 4 high half, code i at bits
       // 4i); m-tile 2 chunk has m-rows g, g + 8 = dims 4g, 4g + 1, m-tile
       // 2 chunk + 1 dims 4g + 2, 4g + 3.  The weights p s_ref are f16 high parts
       // and remainders after a warp-wide power of two vscale that keeps the
@@ -801,7 +805,7 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
       // and the remainders stay far above its subnormals for every weight
       // that matters.  vscale changes lazily; the accumulators follow it
       // exactly.
-      const int tk[4] = {wtok + 2 * q, wtok + 2 * q + 1, wtok + 2 * q + 8, wtok + 2 * q + 9};
+      const int tk[4] = {wtok + q, wtok + q + 4, wtok + q + 8, wtok + q + 12};
       auto s_ref_v = [&](int k, int j) {               // 0 beyond the tile
         const float v = half_at(st + C::OFF_RSV + sc_off + tk[k] * SB + 2 * j);
         return (tk[k] < n) ? v : 0.0f;
@@ -850,8 +854,8 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
       // The residual's V codes on the reference's m-rows, as f16 subnormals:
       // m-row g (+ 8) of m-tile mt is dim d0 (+ 1), d0 = 16mt + 2g (INT8
       // reference) or 32 (mt / 2) + 4g + 2 (mt & 1) (INT4 reference); one
-      // byte permute puts the byte holding d0's code of tokens 2q, 2q + 1
-      // (and 2q + 8, 2q + 9) into halves 0 and 1, a shift brings d0's code to
+      // byte permute puts the byte holding d0's code of tokens q, q + 4
+      // (and q + 8, q + 12) into halves 0 and 1, a shift brings d0's code to
       // bit 0 and d0 + 1's follows at bit BITS.
       auto res_frag = [&](int mt, uint32_t (&a)[4]) {
         if constexpr (C::VSH) {
@@ -906,7 +910,7 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
           for (int ch = j * GROUP / 32; ch < (j + 1) * GROUP / 32; ++ch) {
             const int m = (lane >> 3) & 1;
             uint32_t v[2];   // (tokens 0-7, chunk ch), (tokens 8-15, chunk ch)
-            ldsm_x2_trans(sV + swz_offset<C::RROW>(wtok + m * 8 + r7, ch), v);
+            ldsm_x2_trans(sV + swz_offset<C::RROW>(wtok + m * 8 + pr7, ch), v);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               const int sh = 8 * h;
@@ -922,7 +926,7 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
           for (int mt2 = j * KSG / 2; mt2 < (j + 1) * KSG / 2; ++mt2) {
             const int m = lane >> 3;
             uint32_t v[4];   // (tokens 0-7, chunk 2mt2), (8-15, 2mt2), (0-7, 2mt2+1), (8-15, ..)
-            ldsm_x4_trans(sV + swz_offset<C::RROW>(wtok + (m & 1) * 8 + r7, 2 * mt2 + (m >> 1)),
+            ldsm_x4_trans(sV + swz_offset<C::RROW>(wtok + (m & 1) * 8 + pr7, 2 * mt2 + (m >> 1)),
                           v);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
@@ -944,10 +948,10 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
 #pragma unroll
       for (int mt = 0; mt < KT; ++mt) {
         const int m = lane >> 3;                         // matrix this lane addresses
-        const int tr = wtok + (m >> 1) * 8 + r7;
+        const int tr = wtok + (m >> 1) * 8 + pr7;
         const int chunk = 2 * mt + (m & 1);
         const uint32_t addr = sV + (chunk >> 3) * C::BOX_BYTES + tr * 128 +
-                              ((((chunk & 7) ^ r7)) << 4);
+                              ((((chunk & 7) ^ pr7)) << 4);
         uint32_t a[4];
         ldsm_x4_trans(addr, a);
         mma_bf16(oref[mt], a, ph0, ph1);
@@ -957,16 +961,16 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
     // ---- O_res^T += C_V^T (P s^V)^T (an INT8 compressed reference with an
     // INT2 residual takes these products into its accumulators above) ----
     if constexpr (C::RES && !C::VSH) {
-      const int tk[4] = {wtok + 2 * q, wtok + 2 * q + 1, wtok + 2 * q + 8, wtok + 2 * q + 9};
+      const int tk[4] = {wtok + q, wtok + q + 4, wtok + q + 8, wtok + q + 12};
       const float pk[4] = {pr[0][0], pr[0][1], pr[1][0], pr[1][1]};
       // INT2, 64-dim groups: the warp tile's V code words by one
       // ldmatrix.trans: word = codes of dims 8g .. 8g+7 of a 64-dim chunk
-      // (token 2q low half, 2q+1 high half, code i at bits 2i); (tokens 0-7,
+      // (token q low half, q + 4 high half, code i at bits 2i); (tokens 0-7,
       // chunk 0), (8-15, chunk 0)[, (0-7, chunk 1), (8-15, chunk 1)]
       uint32_t cv4[4], cvp[4];   // cvp (32-dim groups): the words of lane ^ 16
       if constexpr (C::LDM2) {
         const int m = (lane >> 3) & (2 * C::NCH - 1);
-        const uint32_t a = smem_u32(st + C::OFF_CV + (wtok + (m & 1) * 8 + r7) * C::CROW +
+        const uint32_t a = smem_u32(st + C::OFF_CV + (wtok + (m & 1) * 8 + pr7) * C::CROW +
                                     (m >> 1) * 16);
         if constexpr (C::NCH == 2) {
           ldsm_x4_trans(a, cv4);
@@ -1031,7 +1035,7 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
         } else {
           static_assert(C::LDM4, "residual codes are INT2 or INT4");
           // the group's 32-dim chunks by ldmatrix.trans: word = codes of dims
-          // 4g .. 4g+3 of the chunk (token 2q low half, 2q+1 high half, code i
+          // 4g .. 4g+3 of the chunk (token q low half, q + 4 high half, code i
           // at bits 4i); m-tile 2 ch has m-rows g, g + 8 = dims 4g, 4g + 1,
           // m-tile 2 ch + 1 dims 4g + 2, 4g + 3; operands (128 + c) - 128 = c
           const uint32_t m128 = 0xC300C300u;   // {-128, -128}
@@ -1039,7 +1043,7 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
           for (int ch = j * GROUP / 32; ch < (j + 1) * GROUP / 32; ++ch) {
             const int m = (lane >> 3) & 1;
             uint32_t v[2];   // (tokens 0-7, chunk ch), (tokens 8-15, chunk ch)
-            ldsm_x2_trans(smem_u32(st + C::OFF_CV + (wtok + m * 8 + r7) * C::CROW + ch * 16), v);
+            ldsm_x2_trans(smem_u32(st + C::OFF_CV + (wtok + m * 8 + pr7) * C::CROW + ch * 16), v);
 #pragma unroll
             for (int xy = 0; xy < 2; ++xy) {
               const int sh = 8 * xy;
