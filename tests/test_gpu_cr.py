@@ -181,6 +181,47 @@ def test_cr_decode_matches_oracle(ref_bits, bits, varlen):
     print(f"ref INT{ref_bits} bits {bits} varlen {varlen}: max-abs {worst:.2e}")
 
 
+@pytest.mark.parametrize("ref_bits,bits,d,g", [
+    (8, 2, 64, 32), (8, 2, 64, 64), (8, 2, 128, 64), (8, 4, 64, 32), (8, 4, 128, 64),
+    (8, 16, 64, 64), (4, 2, 64, 32), (4, 2, 128, 64), (4, 4, 64, 64), (4, 4, 128, 32),
+    (4, 16, 64, 32)])
+def test_cr_decode_single_query_shapes(ref_bits, bits, d, g):
+    """One query row per kv head on the tensor-core kernel at every head size
+    and scale group: head_dim 64 uses two of the four 32-dim slices (the
+    score MMAs' k positions and B columns of the other two are zero), and
+    64-dim groups share one scale between two slices.  Ragged contexts (a
+    partial last tile, one token past a tile) and a BF16 tail token."""
+    lens = [193, 65]
+    B, Hkv, cap, n_tail = len(lens), 2, 200, 1
+    w = synth.Workload("crsq", 2, 1, B, cap, Hkv, Hkv, d, g, (2,), (0.25,),
+                       300 + ref_bits + bits + d + g)
+    refk, refv = synth.reference(w, 0, 0), synth.reference(w, 0, 1)
+    xk, xv = synth.loop_kv(w, 0, 0, 1, refk), synth.loop_kv(w, 0, 1, 1, refv)
+    rb = bits if bits != 16 else 2
+    (rck, rsk), ck, sk = rq.encode_cr([xk], refk, ref_bits, [rb], g, w.seed)
+    (rcv, rsv), cv, sv = rq.encode_cr([xv], refv, ref_bits, [rb], g, w.seed)
+    q = synth.query(w, 0, 1)
+    tail_k = synth.reference(w, 0, 0, batch=B, ctx=n_tail + 2)
+    tail_v = synth.reference(w, 0, 1, batch=B, ctx=n_tail + 2)
+    ctx_lens = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    out = rq.decode_attention_cr(q, (rck, rsk, rcv, rsv, ref_bits),
+                                 None if bits == 16 else ck[0], None if bits == 16 else cv[0],
+                                 None if bits == 16 else sk[0], None if bits == 16 else sv[0],
+                                 bits, g, w.seed, cap, ctx_lens=ctx_lens, tail_k=tail_k,
+                                 tail_v=tail_v, n_tail=n_tail)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out).all()
+    worst = 0.0
+    for b in range(B):
+        for h in range(Hkv):
+            want = oracle_cr_head(xk, xv, refk, refv, ref_bits, bits, g, w.seed, q, b, h, lens[b],
+                                  tail_k, tail_v, n_tail)
+            got = out[b, h:h + 1].double().cpu().numpy()
+            worst = max(worst, float(np.abs(got - want).max()))
+    assert worst <= OUT_TOL
+    print(f"single query ref INT{ref_bits} bits {bits} d {d} group {g}: max-abs {worst:.2e}")
+
+
 def oracle_cr_kv(xk, xv, refk, refv, ref_bits, bits, g, seed, b, h, ctx):
     """fp64 K_hat, V_hat of (sequence b, kv head h) from the oracle's own encode."""
     d = refk.shape[-1]
