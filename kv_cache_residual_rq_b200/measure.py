@@ -35,6 +35,17 @@ def decode_bytes(w, bits, batch=None):
     return n + b * w.q_heads * w.head_dim * 6
 
 
+def cr_decode_bytes(w, rb, bits):
+    """Algorithmic bytes of one decode call over a compressed reference of rb
+    bits (codes and scales of K and V) plus a residual loop of `bits` (none
+    for 16), q and out."""
+    heads_t = w.batch * w.kv_heads * w.ctx
+    per_tok = 2 * (w.head_dim * rb // 8 + 2 * (w.head_dim // w.group))
+    if bits != 16:
+        per_tok += 2 * (w.head_dim * bits // 8 + 2 * (w.head_dim // w.group))
+    return heads_t * per_tok + w.batch * w.q_heads * w.head_dim * 6
+
+
 def encode_bytes(w, rows):
     active = [b for b in w.bits if b != 16]
     read = rows * w.head_dim * 2 * (1 + len(active))
@@ -161,12 +172,8 @@ def measure(w, reps, peak, emit):
                   "frac": nb_e / t / 1e9 / peak})
             (rck, rsk), ckc, skc = rq.encode_cr([xk1], refk, rb, [2], w.group, w.seed)
             (rcv, rsv), cvc, svc = rq.encode_cr([xv1], refv, rb, [2], w.group, w.seed)
-            heads_t = w.batch * w.kv_heads * w.ctx
             for b in (2, 16):
-                per_tok = 2 * (w.head_dim * rb // 8 + 2 * (w.head_dim // w.group))
-                if b != 16:
-                    per_tok += 2 * (w.head_dim * b // 8 + 2 * (w.head_dim // w.group))
-                nb = heads_t * per_tok + w.batch * w.q_heads * w.head_dim * 6
+                nb = cr_decode_bytes(w, rb, b)
                 args = (ckc[0], cvc[0], skc[0], svc[0]) if b != 16 else (None,) * 4
                 fn = lambda: rq.rq_decode_attention_cr(shape, None, q, rck, rcv, rsk, rsv, rb,
                                                        *args, b, w.seed, 0.0, None, None, 0, 0,
@@ -303,10 +310,12 @@ def bench_workloads(peak, make_sampler, target_s=0.4):
     """Entries for the bench's `workloads` block: the configured decode calls
     of the mixed-precision 32K workload (loop 1 INT4, loop 2 INT2, loop 4 BF16)
     and of the deep-loop grouped-query workload (INT2 loop, BF16 reference),
-    one full layer each (every call streams more than 1 GB, far beyond L2),
-    and rq_encode of the whole 32K prefill (24 layers x K/V x 4 loops in one
-    call, 25.8 GB read).  make_sampler() returns a clock sampler with
-    start()/stop()."""
+    one full layer each (every call streams more than 1 GB, far beyond L2);
+    the compressed-reference format's call (INT8 reference + the first INT2
+    loop) on the Ouro-shaped and deep-loop layers, beside the same loop over
+    the BF16 reference; and rq_encode of the whole 32K prefill (24 layers x
+    K/V x 4 loops in one call, 25.8 GB read).  make_sampler() returns a clock
+    sampler with start()/stop()."""
     import torch
     import kv_cache_residual_rq_b200 as rq
     from kv_cache_residual_rq_b200 import synth
@@ -350,6 +359,40 @@ def bench_workloads(peak, make_sampler, target_s=0.4):
         step_s = w.layers * (sum(per_call[b] for b in w.bits) + per_call[16])
         out_entries[-1]["step_tokens_per_s_from_calls"] = round(w.batch / step_s, 1)
         del refk, refv, ws, out
+        torch.cuda.empty_cache()
+
+    # the compressed-reference format (next to the BF16-reference call of the
+    # same loop on the same layer)
+    for w in (synth.BY_NAME["ouro1.4b_decode"], synth.DEEP):
+        refk = synth.reference(w, 0, 0, dev)
+        refv = synth.reference(w, 0, 1, dev)
+        shape = rq.make_shape(w.batch, w.kv_heads, w.ctx, w.head_dim, w.group, w.q_heads)
+        ws = rq.alloc_workspace(shape, dev)
+        out = torch.empty((w.batch, w.q_heads, w.head_dim), dtype=torch.float32, device=dev)
+        q = synth.query(w, 0, 1, dev)
+        xk1 = synth.loop_kv(w, 0, 0, 1, refk)
+        xv1 = synth.loop_kv(w, 0, 1, 1, refv)
+        bits = w.bits[0]
+        if w is not synth.DEEP:          # (the deep-loop BF16-reference call is above)
+            (ck,), (sk,) = rq.encode([xk1], refk, [bits], w.group, w.seed)
+            (cv,), (sv,) = rq.encode([xv1], refv, [bits], w.group, w.seed)
+            fn = lambda: rq.rq_decode_attention(shape, q, refk, refv, ck, cv, sk, sv, bits,
+                                                w.seed, 0.0, out, ws, stream=st)
+            label = f"{w.name} decode loop 1 INT{bits} over the BF16 reference"
+            t, n, clk = _back_to_back(fn, stream, target_s, make_sampler(), label)
+            out_entries.append(_entry(label, t, n, clk, decode_bytes(w, bits), peak, G=w.G))
+            del ck, cv, sk, sv
+        (rck, rsk), (cck,), (csk,) = rq.encode_cr([xk1], refk, 8, [bits], w.group, w.seed)
+        (rcv, rsv), (ccv,), (csv,) = rq.encode_cr([xv1], refv, 8, [bits], w.group, w.seed)
+        del xk1, xv1
+        fn = lambda: rq.rq_decode_attention_cr(shape, None, q, rck, rcv, rsk, rsv, 8, cck, ccv,
+                                               csk, csv, bits, w.seed, 0.0, None, None, 0, 0,
+                                               out, ws, stream=st)
+        label = f"{w.name} decode compressed reference INT8 + loop 1 INT{bits}"
+        t, n, clk = _back_to_back(fn, stream, target_s, make_sampler(), label)
+        out_entries.append(_entry(label, t, n, clk, cr_decode_bytes(w, 8, bits), peak, G=w.G))
+        assert rq.rq_workspace_status(ws) == 0
+        del refk, refv, ws, out, rck, rsk, cck, csk, rcv, rsv, ccv, csv
         torch.cuda.empty_cache()
 
     # the whole 32K prefill encode in one call
