@@ -29,3 +29,17 @@ def test_step_bytes_reread_reference_each_loop():
     qo = 4 * 24 * 16 * 128 * 6
     assert capacity.step_bytes(W, CTX, 1, "bf16") == elems * 2 * 4 + qo
     assert capacity.step_bytes(W, CTX, 1, "rq") == elems * 2 * 4 + 3 * elems * 5 // 16 + qo
+
+
+def test_call_bytes_by_hand():
+    # one Ouro-shaped call: 16 x 16 heads x 4096 tokens, d 128, group 32
+    from kv_cache_residual_rq_b200 import measure
+    w = synth.BY_NAME["ouro1.4b_decode"]
+    heads_t = 16 * 16 * 4096
+    qo = 16 * 16 * 128 * 6                       # q bf16 in, out fp32
+    # BF16 K/V rows, INT2 codes of K and V, one fp16 scale per 32 dims each
+    assert measure.decode_bytes(w, 2) == heads_t * (2 * 256 + 2 * 32 + 2 * 8) + qo == 620953600
+    assert measure.decode_bytes(w, 16) == heads_t * 2 * 256 + qo
+    # compressed reference: INT8 (INT4) K/V codes and scales instead of the rows
+    assert measure.cr_decode_bytes(w, 8, 2) == heads_t * (2 * 136 + 2 * 40) + qo == 369295360
+    assert measure.cr_decode_bytes(w, 4, 16) == heads_t * 2 * 72 + qo
