@@ -328,6 +328,40 @@ def test_cr_grouped_peaky_scores_long_context():
     print(f"peaky G {G}: max-abs {worst:.2e}")
 
 
+@pytest.mark.parametrize("name", ["ouro1.4b_decode", "deep_loop_gqa"])
+def test_cr_decode_full_size_sampled(name):
+    """The compressed-reference call at full size, in the shape the bench's
+    workloads block times (INT8 reference + the first INT2 loop of one layer:
+    the single-query kernel on the Ouro-shaped call, the grouped-query kernel
+    with shared value accumulators on the deep-loop call), checked on sampled
+    heads against fp64 attention over the oracle's own encode."""
+    w = synth.BY_NAME[name]
+    G, d, g = w.G, w.head_dim, w.group
+    refk, refv = synth.reference(w, 0, 0), synth.reference(w, 0, 1)
+    xk, xv = synth.loop_kv(w, 0, 0, 1, refk), synth.loop_kv(w, 0, 1, 1, refv)
+    (rck, rsk), ck, sk = rq.encode_cr([xk], refk, 8, [2], g, w.seed)
+    (rcv, rsv), cv, sv = rq.encode_cr([xv], refv, 8, [2], g, w.seed)
+    q = synth.query(w, 0, 1)
+    shape = rq.make_shape(w.batch, w.kv_heads, w.ctx, d, g, w.q_heads)
+    ws = rq.alloc_workspace(shape, q.device)
+    out = rq.decode_attention_cr(q, (rck, rsk, rcv, rsv, 8), ck[0], cv[0], sk[0], sv[0], 2, g,
+                                 w.seed, w.ctx, workspace=ws, kv_heads=w.kv_heads)
+    torch.cuda.synchronize()
+    assert rq.rq_workspace_status(ws) == 0
+    rng = np.random.default_rng(5)
+    heads = {(0, 0), (w.batch - 1, w.kv_heads - 1)}
+    heads |= {(int(rng.integers(w.batch)), int(rng.integers(w.kv_heads))) for _ in range(2)}
+    worst = 0.0
+    for b, h in sorted(heads):
+        kh, vh = oracle_cr_kv(xk, xv, refk, refv, 8, 2, g, w.seed, b, h, w.ctx)
+        qh = oracle.bf16_to_f32(u16(q[b, h * G:(h + 1) * G])).astype(np.float64)
+        want = oracle.attention_f64(qh, kh, vh, 1.0 / np.sqrt(d))
+        got = out[b, h * G:(h + 1) * G].double().cpu().numpy()
+        worst = max(worst, float(np.abs(got - want).max()))
+    assert worst <= OUT_TOL
+    print(f"{name} compressed reference INT8 + INT2: {len(heads)} heads, max-abs {worst:.2e}")
+
+
 def test_cr_single_query_large_value_scales():
     """One query row per kv head: the value weights p s 2^Ev are f16 after a
     lazily updated warp-wide power of two, so reference value scales at the
