@@ -365,11 +365,11 @@ rq_status rq_decode_attention_varlen(const rq_shape *shape, const int32_t *ctx_l
  *   ref_codes_k/v, ref_scales_k/v, ref_bits (4 or 8): the reference's
  *               codes and fp16 scales, [batch][Hkv][T_cap][...].
  * Tail tokens (BF16 K/V of the current token) and every other argument as
- * rq_decode_attention_tail.  Range: with G = 1 and ref_bits 8 the value
- * weights p s_ref are fp16 with p < 2^8, so reference scales above 2^8
- * (groups of rotated reference values beyond ~32000) are outside the format;
- * such a call, or one whose reference scales are not finite, sets workspace
- * status bit 64 and its output is not valid.
+ * rq_decode_attention_tail.  The value weights p s are fp16 after a
+ * warp-wide power of two that follows the largest scale of each tile, so
+ * every finite fp16 scale is in range; a call whose reference or residual
+ * value scales are not finite sets workspace status bit 64 and its output is
+ * not valid.
  */
 rq_status rq_decode_attention_cr(const rq_shape *shape, const int32_t *ctx_lens,
                                  const uint16_t *q, const uint32_t *ref_codes_k,
@@ -495,8 +495,8 @@ rq_status rq_encode_take_status(uint32_t *host_status);
  * ran clean; non-zero means a call's output is invalid and the workspace must
  * be zeroed again: bits 1, 2, 8 a bounded wait inside a kernel ran out, 4 a
  * partial-record slot out of range, 16 a sequence length clamped to the
- * capacity, 32 a page id outside the pool, 64 a compressed-reference weight
- * out of range; 128, only in the bounds-checked build (librq_bounds.so), an
+ * capacity, 32 a page id outside the pool, 64 a compressed-reference value
+ * weight not finite; 128, only in the bounds-checked build (librq_bounds.so), an
  * index a decode kernel computed fell outside its buffer or shared-memory
  * area and that access was skipped.  This is the only entry point that
  * synchronises. */
