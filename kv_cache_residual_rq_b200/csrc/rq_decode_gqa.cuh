@@ -544,6 +544,9 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
     // ---- scores for the warp's two 8-token tiles, k-steps outermost ----
     // c[nt]: S_ref (then + s x S_res) fragments, row g, tokens q, q + 4 of nt
     float cref[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
+    // BF16 reference: the odd k-steps' products in a second accumulator (two
+    // chains of KT / 2 MMAs instead of one of KT), added before the softmax
+    float cref2[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
     float ct[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
     const int tok0[2] = {wtok + q, wtok + 8 + q};     // tokens of c0 per tile (c1: + 4)
     // ldmatrix: matrices (tile 0, dims +0..7), (tile 0, +8..15), (tile 1, ..), (tile 1, ..)
@@ -612,8 +615,8 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
           a[0] = f.x;
           a[2] = f.y;
         }
-        mma_bf16(cref[0], a, b[0], b[1]);
-        mma_bf16(cref[1], a, b[2], b[3]);
+        mma_bf16((kk & 1) ? cref2[0] : cref[0], a, b[0], b[1]);
+        mma_bf16((kk & 1) ? cref2[1] : cref[1], a, b[2], b[3]);
       }
       if constexpr (C::RES && !C::RIM) {
         const uint2 fh = *reinterpret_cast<const uint2*>(qfrag + C::QF1 + (kk * 32 + lane) * 2);
@@ -741,6 +744,12 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
           cref[nt][1] = fmaf(sk1 * sg, (float)x1, cref[nt][1]);
         }
       }
+    }
+    if constexpr (!C::CRX) {
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) cref[nt][e] += cref2[nt][e];
     }
     float sc[2][2];          // row g, tokens q, q + 4 of tile nt
 #pragma unroll
