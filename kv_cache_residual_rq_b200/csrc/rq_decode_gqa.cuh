@@ -13,12 +13,16 @@
 //   S_res = Q~ C_K^T            per scale group, then x s^K
 //   O_ref^T += V^T P^T          (V via ldmatrix.trans)
 //   O_res^T += C_V^T (P s^V)^T
-// with fp32 accumulation.  S_ref and O_ref are bf16 x bf16.  S_res is one
-// f16 MMA per k-step: q~ scaled by a power of two 2^E per row (max |q~| 2^E
-// in [2^13, 2^14)) and rounded to f16 (11 significant bits), against the K
-// codes as the exact f16 subnormals c 2^-24 (a shift and a mask per two
-// codes, no offset); per scale group q~ . l = 2^25 acc - (2^b - 1) sum q~,
-// times s^K 2^-E.  O_res: the V codes c are exact bf16 values, and P s^V, not
+// with fp32 accumulation.  S_ref and O_ref are bf16 x bf16.  S_res, INT2
+// residual with 64-dim groups: integer MMAs (m16n8k32) of the rows' q~ as
+// 16-bit fixed point (signed bytes h | l as A rows g | g + 8) against the
+// codes one per byte (a shift and a mask per four), exact integer level sums
+// per group until x s^K sig.  S_res otherwise: one f16 MMA per k-step, q~
+// scaled by a power of two 2^E per row (max |q~| 2^E in [2^13, 2^14)) and
+// rounded to f16 (11 significant bits), against the K codes as the exact f16
+// subnormals c 2^-24 (a shift and a mask per two codes, no offset); per scale
+// group q~ . l = 2^25 acc - (2^b - 1) sum q~, times s^K 2^-E.  O_res: the V
+// codes c are exact bf16 values, and P s^V, not
 // a bf16 value, is split into a bf16 high part and a bf16 remainder and
 // multiplied twice (~16 significant bits, bf16's range); sum_t p s (2c -
 // (2^b-1)) = 2 (C_V^T (P s)^T) - (2^b - 1) sum_t p s is completed when the
@@ -137,10 +141,11 @@ struct GCfg {
   static constexpr int QF12_WORDS = RIM ? NCH * 256 : (RES ? 2 * KT * 64 : 0);
   static constexpr int QFC = QF1 + QF12_WORDS;
   static constexpr int QFRAG_WORDS = QFC + (CRX ? NV * 32 * 4 : 0);
-  // INT2: per (row, scale group) sum of the q~ fragments' values (offset of
-  // the 128 + 2c operands); compressed reference: the same for the f16
-  // fragments (the levels' 2^b - 1) and per row 2^-E; even count to keep the
-  // barriers 8-byte aligned
+  // residual: per (row, scale group) the sum of the q~ fragments' values (f16
+  // form) or of Q (integer form), for the levels' 2^b - 1 offset; compressed
+  // reference: the same sums of its Q; per row the residual's scale (2^-E or
+  // sig) and the compressed reference's sig; even count to keep the barriers
+  // 8-byte aligned
   static constexpr int SQ_FLOATS =
       (G * NG * (CRX ? 2 : 1) + ((CRX || RES) ? G : 0) + (CRX ? G : 0) + 1) / 2 * 2;
   static constexpr int SMEM_BYTES = 1024 /* base alignment slack */ + RING_BYTES +
@@ -184,7 +189,8 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
   uint32_t* qfrag = reinterpret_cast<uint32_t*>(wsum_s + C::WSUM_FLOATS);  // [3][KT][32][2]
   float* sq_s = reinterpret_cast<float*>(qfrag + C::QFRAG_WORDS);           // [G][NG]
   float* sqh_s = sq_s + G * NG;              // CR: [G][NG] sums of Q per scale group
-  // [G] 2^-E of each row's f16 q~ fragments (residual and compressed reference)
+  // [G] the residual's per-row scale: 2^-E of the f16 q~ fragments, or sig
+  // of the integer form's Q
   float* rsig_s = sq_s + G * NG * (C::CRX ? 2 : 1);
   float* rsigc_s = rsig_s + G;               // CR: [G] sig of each row's Q
   float* wsumR_s = wsum_s + kConsumerWarps * G * NG;   // CR: sums of p s_ref^V
