@@ -328,7 +328,7 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
     }
     float upR = 1.0f;        // 2^E of the residual's f16 q~ fragments (row g)
     if constexpr (C::RIM) {
-      if (warp == 0) {
+      if (warp == (C::CRX ? 1 : kConsumerWarps - 1)) {   // beside warp 0's fragments
         // row g of q~ as 16-bit fixed point Q = q~ / sig, as the s8 A
         // fragments of the residual's integer MMAs: per 64-dim chunk c and
         // code pair pp, rows g carry the h bytes and rows g + 8 the l bytes;
