@@ -611,6 +611,26 @@ decode_cr1_kernel(const __grid_constant__ TcParams gp) {
                  ((4u + (g & 3)) << 12))
               : ((2u * h2) | ((2u * h2 + 1u) << 4) | ((4u + 2u * h2) << 8) |
                  ((5u + 2u * h2) << 12));
+      // codes are masked in place where they sit in the low 10 bits of a
+      // half (exact subnormals 2^k c 2^-24), their weights scaled by 2^-k
+      // (exact): the reference's odd nibbles (k = 4), the INT2 residual's
+      // fields 1-3 (k = 2, 4, 6), the INT4 residual's odd nibbles (k = 4);
+      // nibbles 2 and 3 of a half are first moved down by one shift of 8
+      const uint32_t br0q = hmul2_u(br0, 0x2C002C00u), br1q = hmul2_u(br1, 0x2C002C00u);
+      uint32_t bvs0[4] = {bv0, bv0, bv0, bv0}, bvs1[4] = {bv1, bv1, bv1, bv1};
+      if constexpr (C::RES) {
+        if constexpr (BITS == 2) {
+#pragma unroll
+          for (int s = 1; s < 4; ++s) {
+            const uint32_t f = s == 1 ? 0x34003400u : (s == 2 ? 0x2C002C00u : 0x24002400u);
+            bvs0[s] = hmul2_u(bv0, f);
+            bvs1[s] = hmul2_u(bv1, f);
+          }
+        } else {
+          bvs0[1] = bvs0[3] = hmul2_u(bv0, 0x2C002C00u);
+          bvs1[1] = bvs1[3] = hmul2_u(bv1, 0x2C002C00u);
+        }
+      }
 #pragma unroll
       for (int cq = 0; cq < NV / 2; ++cq) {
         uint32_t R[4];   // (tokens 0-7, chunk 2cq), (0-7, 2cq + 1), (8-15, 2cq), (8-15, 2cq + 1)
@@ -632,18 +652,25 @@ decode_cr1_kernel(const __grid_constant__ TcParams gp) {
           X[2] = __byte_perm(w[2][0], w[3][0], psel);
           X[3] = __byte_perm(w[2][1], w[3][1], psel);
         }
+        uint32_t R8[4], X8[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          R8[i] = R[i] >> 8;
+          X8[i] = (BITS == 4) ? X[i] >> 8 : X[i];
+        }
 #pragma unroll
         for (int s = 0; s < 4; ++s) {
           // nibble s of each half: dim 4g + s of tokens t, t + 4
-          const uint32_t a[4] = {(R[0] >> (4 * s)) & 0x000F000Fu, (R[1] >> (4 * s)) & 0x000F000Fu,
-                                 (R[2] >> (4 * s)) & 0x000F000Fu, (R[3] >> (4 * s)) & 0x000F000Fu};
-          mma_f16(acc[4 * cq + s], a, br0, br1);
+          const uint32_t* Rs = s < 2 ? R : R8;
+          const uint32_t Mr = (s & 1) ? 0x00F000F0u : 0x000F000Fu;
+          const uint32_t a[4] = {Rs[0] & Mr, Rs[1] & Mr, Rs[2] & Mr, Rs[3] & Mr};
+          mma_f16(acc[4 * cq + s], a, (s & 1) ? br0q : br0, (s & 1) ? br1q : br1);
           if constexpr (C::RES) {
-            const int sh = (BITS == 2) ? 2 * s : 4 * s;
-            constexpr uint32_t M = (BITS == 2) ? 0x00030003u : 0x000F000Fu;
-            const uint32_t c[4] = {(X[0] >> sh) & M, (X[1] >> sh) & M, (X[2] >> sh) & M,
-                                   (X[3] >> sh) & M};
-            mma_f16(acc[4 * cq + s], c, bv0, bv1);
+            const uint32_t* Xs = (BITS == 4 && s >= 2) ? X8 : X;
+            const uint32_t M = (BITS == 2) ? (0x00030003u << (2 * s))
+                                           : ((s & 1) ? 0x00F000F0u : 0x000F000Fu);
+            const uint32_t c[4] = {Xs[0] & M, Xs[1] & M, Xs[2] & M, Xs[3] & M};
+            mma_f16(acc[4 * cq + s], c, bvs0[s], bvs1[s]);
           }
         }
       }

@@ -24,7 +24,9 @@
 // lane's two 32-wide blocks are the two scale groups of 32 (or together one
 // of 64), quantised side by side as packed pairs; codes from floor(u)
 // obtained as (u + 1.5*2^23) rounded down, whose bit pattern is 0x4B400000 +
-// floor(u), packed by shifted adds with one constant correction per word.
+// floor(u), packed by shifted adds with one constant correction per word;
+// the least-squares numerator <y, l> = 2 <y, floor(u)> + sum y, the block's
+// sum y taken from four unrotated coordinates (no level per coordinate).
 // Every wait is bounded; on a timeout the kernel raises a bit in the encoder
 // status word and stops.
 #include <cuda.h>
@@ -140,18 +142,41 @@ __device__ __forceinline__ void rotate64(float2 (&P)[32], int q) {
   for (int m = 0; m < 32; ++m) P[m] = __fmul2_rn(P[m], cd2);
 }
 
+// Sum of the rotated coordinates over each of the lane's two 32-wide blocks,
+// taken from the unrotated ones.  In the Sylvester Hadamard matrix H the rows
+// 32a .. 32a + 31 (block a) sum to 32 (-1)^popcount(a & (j >> 5)) in the
+// columns j that are multiples of 32 and to zero in every other column, so
+// sum over block a of y = 32 c_d sum_j' (-1)^popcount(a & j') x_(32 j'): the
+// lane's x_0 and x_32 and, at head_dim 128, its partner's.  It differs from
+// the sum of the computed y by the rotation's roundings (a few units in the
+// last place of sum |y|), which the least-squares scale, kept as fp16, does
+// not see.
+template <int D, int RPW>
+__device__ __forceinline__ float2 block_sums(const float2 (&P)[32], int q) {
+  float2 a = make_float2(P[0].x + P[0].y, P[0].x - P[0].y);
+  if constexpr (D == 128) {
+    const float sg = q ? -1.0f : 1.0f;
+    float2 o;
+    o.x = __shfl_xor_sync(kFull, a.x, RPW);
+    o.y = __shfl_xor_sync(kFull, a.y, RPW);
+    a = make_float2(fmaf(sg, a.x, o.x), fmaf(sg, a.y, o.y));
+  }
+  const float k = 32.0f * rot_scale<D>();
+  return make_float2(k * a.x, k * a.y);
+}
+
 // One quantisation pass over the lane's two 32-coordinate blocks, A = P[].x
 // and B = P[].y, with steps 1/(2 inv.x), 1/(2 inv.y): code words (A's BITS
-// words, then B's), <y,l> and <l,l> of each block (.x, .y).  The scale is
-// kept only as its fp16 rounding, so <y,l> runs as four interleaved chains;
-// code words are integer sums (any order).
+// words, then B's), <y,f> with f = floor(u) and <l,l> of each block (.x,
+// .y).  With l = 2 f + 1, <y,l> = 2 <y,f> + sum y, and the caller supplies
+// sum y; the scale is kept only as its fp16 rounding, so <y,f> runs as four
+// interleaved chains; code words are integer sums (any order).
 template <int BITS>
 __device__ __forceinline__ void quant_pass(const float2 (&P)[32], float2 inv2,
                                            uint32_t (&w)[2 * BITS], float2& dot_out,
                                            float2& nrm_out) {
   constexpr int PER = 32 / BITS;                    // codes per word
   const float2 mg = make_float2(kFloorMagic, kFloorMagic);
-  const float2 two = make_float2(2.0f, 2.0f), one = make_float2(1.0f, 1.0f);
   constexpr int NC = 4;                             // independent chains
   float2 dot[NC], nrm[NC];
 #pragma unroll
@@ -168,10 +193,9 @@ __device__ __forceinline__ void quant_pass(const float2 (&P)[32], float2 inv2,
     const float2 t = __fadd2_rd(u, mg);             // 1.5*2^23 + floor(u), exact
     w[m / PER] += __float_as_uint(t.x) << (BITS * (m % PER));
     w[BITS + m / PER] += __float_as_uint(t.y) << (BITS * (m % PER));
-    const float2 fl = fsub2(t, mg);                 // floor(u)
-    const float2 lv = __ffma2_rn(fl, two, one);     // level 2 floor(u) + 1 = 2c - (2^b - 1)
-    dot[c] = __ffma2_rn(P[m], lv, dot[c]);
-    if constexpr (BITS != 2) nrm[c] = __ffma2_rn(lv, lv, nrm[c]);
+    const float2 fl = fsub2(t, mg);                 // floor(u); level 2 floor(u) + 1
+    dot[c] = __ffma2_rn(P[m], fl, dot[c]);
+    if constexpr (BITS != 2) nrm[c] = __ffma2_rn(fl, fl, nrm[c]);
   }
   // every field received (0x4B400000 + floor(u)); code c = floor(u) + 2^(b-1)
   constexpr uint32_t kOff = kFloorMagicBits - (1u << (BITS - 1));
@@ -188,8 +212,16 @@ __device__ __forceinline__ void quant_pass(const float2 (&P)[32], float2 inv2,
                         __popc(~(w[3] ^ (w[3] >> 1)) & 0x55555555u);
     nrm_out = make_float2((float)(32u + 8u * ea), (float)(32u + 8u * eb));
   } else {
-    // integers below 2^24 in every partial sum: exact in any order
-    nrm_out = __fadd2_rn(__fadd2_rn(nrm[0], nrm[1]), __fadd2_rn(nrm[2], nrm[3]));
+    // <l, l> = 4 (sum f^2 + sum f) + 32, sum f = sum c - 8 * 32 from the code
+    // words; integers below 2^24 in every partial sum: exact in any order
+    auto csum = [](uint32_t x) {
+      const uint32_t b = (x & 0x0F0F0F0Fu) + ((x >> 4) & 0x0F0F0F0Fu);
+      return (b * 0x01010101u) >> 24;
+    };
+    const int fa = (int)(csum(w[0]) + csum(w[1]) + csum(w[2]) + csum(w[3])) - 256;
+    const int fb = (int)(csum(w[4]) + csum(w[5]) + csum(w[6]) + csum(w[7])) - 256;
+    const float2 sq = __fadd2_rn(__fadd2_rn(nrm[0], nrm[1]), __fadd2_rn(nrm[2], nrm[3]));
+    nrm_out = make_float2(4.0f * (sq.x + (float)fa) + 32.0f, 4.0f * (sq.y + (float)fb) + 32.0f);
   }
 }
 
@@ -197,10 +229,12 @@ __device__ __forceinline__ float2 f2(float x) { return make_float2(x, x); }
 
 // Codes and scales of the lane's 64 rotated coordinates: blocks A (P[].x)
 // and B (P[].y) are one 32-wide scale group each, or together one group of
-// 64.  The absmax step, then the least-squares scale of those codes.
+// 64; ysum = sum y over each block.  The absmax step, then the least-squares
+// scale of those codes.
 template <int BITS, int GROUP>
-__device__ __forceinline__ void quantize_store(const float2 (&P)[32], uint32_t* codes_row,
-                                               uint16_t* scales_row, int q, bool valid) {
+__device__ __forceinline__ void quantize_store(const float2 (&P)[32], float2 ysum,
+                                               uint32_t* codes_row, uint16_t* scales_row, int q,
+                                               bool valid) {
   // absmax of each block as four interleaved chains (max is exact in any order)
   float ax[4], ay[4];
 #pragma unroll
@@ -224,6 +258,7 @@ __device__ __forceinline__ void quantize_store(const float2 (&P)[32], uint32_t* 
   uint32_t w[2 * BITS];
   float2 d, n;
   quant_pass<BITS>(P, inv, w, d, n);
+  d = make_float2(fmaf(2.0f, d.x, ysum.x), fmaf(2.0f, d.y, ysum.y));   // <y, l>
   if constexpr (GROUP == 64) {
     d = f2(d.x + d.y);                              // block A + block B
     n = f2(n.x + n.y);
@@ -363,13 +398,14 @@ encode_tma_kernel(const __grid_constant__ EncodeTmaParams tp) {
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
       ++it;
+      const float2 ysum = block_sums<D, C::RPW>(P, q);
       rotate64<D, C::RPW>(P, q);
       const int l = tp.active[j];
       if (p.bits[l] == 2)
-        quantize_store<2, GROUP>(P, p.codes[l] + (size_t)row * (D / 16),
+        quantize_store<2, GROUP>(P, ysum, p.codes[l] + (size_t)row * (D / 16),
                                  p.scales[l] + (size_t)row * (D / GROUP), q, valid);
       else
-        quantize_store<4, GROUP>(P, p.codes[l] + (size_t)row * (D / 8),
+        quantize_store<4, GROUP>(P, ysum, p.codes[l] + (size_t)row * (D / 8),
                                  p.scales[l] + (size_t)row * (D / GROUP), q, valid);
     }
   }
