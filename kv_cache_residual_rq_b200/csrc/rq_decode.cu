@@ -192,6 +192,37 @@ decode_kernel(const DecodeParams p) {
     fence_mbar_init();
   }
   __syncthreads();
+  // dense calls of uniform length (the run depends on the arguments alone):
+  // the first tiles of this CTA's run go into L2 while the previous grid
+  // finishes, so that the ring fills from L2 once the wait returns
+  if (warp == kConsumerWarps && lane == 0 && !p.ctx_lens && !p.page_table) {
+    CallSplit sp;
+    long long tb, te;
+    TileCursor c;
+    if (plan_cta(p, cta, nullptr, sp, tb, te, c)) {
+      const int sb = (D / p.group) * 2;
+      const long long npf = min(te - tb, (long long)kPrefetchTiles);
+      for (long long i = 0; i < npf; ++i) {
+        size_t row;
+        const int n = c.n();
+        if (n > 0 && tile_row(p, c, row)) {
+          const size_t lo = (row * sb) & ~(size_t)15;
+          const uint32_t nb = (uint32_t)(((row * sb + (size_t)n * sb + 15) & ~(size_t)15) - lo);
+          if (tile_in_bounds(p, row, n, lo, nb, sb)) {
+            bulk_prefetch_l2(p.ref_k + row * D, n * C::KROW);
+            bulk_prefetch_l2(p.ref_v + row * D, n * C::KROW);
+            if constexpr (C::RES) {
+              bulk_prefetch_l2(p.codes_k + row * C::CWORDS, n * C::CROW);
+              bulk_prefetch_l2(p.codes_v + row * C::CWORDS, n * C::CROW);
+              bulk_prefetch_l2(reinterpret_cast<const unsigned char*>(p.scales_k) + lo, nb);
+              bulk_prefetch_l2(reinterpret_cast<const unsigned char*>(p.scales_v) + lo, nb);
+            }
+          }
+        }
+        c.next(p);
+      }
+    }
+  }
   pdl_wait_prev();     // inputs and workspace may come from the previous kernel
 
   // this CTA's run of tiles (the merge area is free scratch until the first head)

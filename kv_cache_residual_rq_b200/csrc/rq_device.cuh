@@ -145,12 +145,20 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
+// cp.async.bulk prefetch of global memory into L2 (no data returned, no
+// completion to wait for).  src 16-byte aligned; bytes a multiple of 16.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // Programmatic dependent launch (sm_90 and later).  pdl_allow_next lets the
 // next kernel of the stream be scheduled once every CTA of this grid has
 // started; pdl_wait_prev blocks until the grids before this one have
 // completed and their writes are visible.  A kernel launched with the
 // programmatic-serialization attribute must call pdl_wait_prev before its
-// first global memory access.
+// first global memory read whose value it uses.  An L2 prefetch may come
+// earlier: it returns no data, and L2 is where the previous grid's writes
+// land, so every read after the wait sees them.
 __device__ __forceinline__ void pdl_allow_next() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
