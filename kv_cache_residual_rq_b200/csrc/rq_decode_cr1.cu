@@ -175,6 +175,7 @@ decode_cr1_kernel(const __grid_constant__ TcParams gp) {
     fence_mbar_init();
   }
   __syncthreads();
+  if (warp == kConsumerWarps && lane == 0) prefetch_first_tiles<C, D>(p, cta);
   pdl_wait_prev();     // inputs and workspace may come from the previous kernel
 
   CallSplit split;

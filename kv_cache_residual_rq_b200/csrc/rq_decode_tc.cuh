@@ -163,6 +163,46 @@ __device__ __forceinline__ uint32_t hmul2_u(uint32_t a, uint32_t b) {
 
 // ---- the tile pipeline --------------------------------------------------------
 
+// Dense calls of uniform length (the CTA's run depends on the arguments
+// alone): the first tiles of the run go into L2 before the grid-dependency
+// wait, so that the ring fills from L2 once the previous grid has finished.
+// Called by one lane.
+template <class C, int D>
+__device__ __forceinline__ void prefetch_first_tiles(const DecodeParams& p, int cta) {
+  if (p.ctx_lens || p.page_table) return;
+  CallSplit sp;
+  long long tb, te;
+  TileCursor c;
+  if (!plan_cta(p, cta, nullptr, sp, tb, te, c)) return;
+  constexpr int SB = C::SB;
+  const long long npf = min(te - tb, (long long)kPrefetchTiles);
+  for (long long i = 0; i < npf; ++i, c.next(p)) {
+    size_t row;
+    const int n = c.n();
+    if (n <= 0 || !tile_row(p, c, row)) continue;
+    const size_t lo = (row * SB) & ~(size_t)15;
+    const uint32_t nb = (uint32_t)(((row * SB + (size_t)n * SB + 15) & ~(size_t)15) - lo);
+    if (!tile_in_bounds(p, row, n, lo, nb, SB)) continue;
+    if constexpr (C::CRX) {
+      bulk_prefetch_l2(reinterpret_cast<const unsigned char*>(p.rcodes_k) + row * C::RROW,
+                       n * C::RROW);
+      bulk_prefetch_l2(reinterpret_cast<const unsigned char*>(p.rcodes_v) + row * C::RROW,
+                       n * C::RROW);
+      bulk_prefetch_l2(reinterpret_cast<const unsigned char*>(p.rscales_k) + lo, nb);
+      bulk_prefetch_l2(reinterpret_cast<const unsigned char*>(p.rscales_v) + lo, nb);
+    } else {
+      bulk_prefetch_l2(p.ref_k + row * D, n * 2 * D);
+      bulk_prefetch_l2(p.ref_v + row * D, n * 2 * D);
+    }
+    if constexpr (C::RES) {
+      bulk_prefetch_l2(p.codes_k + row * C::CWORDS, n * C::CROW);
+      bulk_prefetch_l2(p.codes_v + row * C::CWORDS, n * C::CROW);
+      bulk_prefetch_l2(reinterpret_cast<const unsigned char*>(p.scales_k) + lo, nb);
+      bulk_prefetch_l2(reinterpret_cast<const unsigned char*>(p.scales_v) + lo, nb);
+    }
+  }
+}
+
 // Producer warp (lane 0 issues): fills stage i % STAGES with tile i of the
 // CTA's run once the consumers have released it.  C: the kernel's stage
 // layout (STAGES, STAGE_BYTES, REF_TILE_BYTES, OFF_*, CROW, CWORDS, SB, RES,
