@@ -19,7 +19,7 @@ namespace rq {
 constexpr int kConsumerWarps = 4;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kMergeChunk = 64;   // records whose weights the head merge stages at once
-constexpr int kPrefetchTiles = 4;   // tiles a CTA fetches into L2 before the grid-dependency wait
+constexpr int kPrefetchTiles = 2;   // tiles a CTA fetches into L2 before the grid-dependency wait
 constexpr int kDecodeThreads = kConsumerThreads + 32;   // + one producer warp
 constexpr float kNegInf = -INFINITY;
 // lazy rescaling threshold of the online softmax (base-2 units)
