@@ -19,6 +19,7 @@ namespace rq {
 constexpr int kConsumerWarps = 4;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kMergeChunk = 64;   // records whose weights the head merge stages at once
+constexpr int kMergeFew = 8;      // up to this many records a head merge loads in one batch
 constexpr int kPrefetchTiles = 2;   // tiles a CTA fetches into L2 before the grid-dependency wait
 constexpr int kDecodeThreads = kConsumerThreads + 32;   // + one producer warp
 constexpr float kNegInf = -INFINITY;
@@ -356,9 +357,11 @@ __device__ __forceinline__ void finish_head(const DecodeParams& p, long long hd,
   // ---- last contributor: merge all records of the head, finish ----
   // Every record load of a pass is independent of the others, so each pass
   // costs about one L2 round trip per batch of loads instead of one per
-  // record: (1) the rows' maxima M_r over the records, (2) per chunk of
-  // records their weights exp2(m_c - M_r) and weighted sums l_c, (3) the
-  // weighted sums of the accumulators, eight records per batch.
+  // record.  Up to kMergeFew records: each thread loads all of them for its
+  // element at once (one round trip).  More: (1) the rows' maxima M_r over
+  // the records, (2) per chunk of records their weights exp2(m_c - M_r) and
+  // weighted sums l_c, (3) the weighted sums of the accumulators, eight
+  // records per batch.
   float* zres = merge;               // [G][D] rotated-domain residual sums
   float* zref = merge + G * D;       // [G][D]
   float* lsum = merge + 2 * G * D;   // [G]
@@ -376,76 +379,115 @@ __device__ __forceinline__ void finish_head(const DecodeParams& p, long long hd,
   const int rr = tid % G;                        // the row of this thread's records
   constexpr int RSTEP = kConsumerThreads / G;    // records per pass of the threads
   auto rec = [&](int c, int r) { return recs + ((size_t)c * G + r) * (4 + 2 * D); };
-  // (1) M_r
-  {
-    float pm = kNegInf;
-    for (int c = tid / G; c < ncontrib; c += RSTEP) pm = fmaxf(pm, __ldcg(rec(c, rr)));
-#pragma unroll
-    for (int m = G; m < 32; m <<= 1) pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, m));
-    if (lane_m < G) red[warp_m * G + lane_m] = pm;
-    named_bar_sync(1, kConsumerThreads);
-    if (tid < G) {
-      float M = kNegInf;
-#pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, red[w * G + tid]);
-      mrow[tid] = M;
-    }
-    named_bar_sync(1, kConsumerThreads);
-  }
-  float lpart = 0.0f;                            // threads tid < G: l of row tid
-  for (int c0 = 0; c0 < ncontrib; c0 += kMergeChunk) {
-    const int nc = min(kMergeChunk, ncontrib - c0);
-    // (2) the chunk's weights; a record without tokens (m = -inf) weighs 0
-    for (int e = tid; e < nc * G; e += kConsumerThreads) {
-      const int c = c0 + e / G, r = e % G;
-      const float* rc = rec(c, r);
-      const float mc = __ldcg(rc), lc = __ldcg(rc + 1);
-      const float wgt = (mc == kNegInf) ? 0.0f : exp2f(mc - mrow[r]);
-      wch[e] = wgt;
-      lch[e] = (mc == kNegInf) ? 0.0f : wgt * lc;
-    }
-    named_bar_sync(1, kConsumerThreads);
-    if (tid < G)
-      for (int cc = 0; cc < nc; ++cc) lpart += lch[cc * G + tid];
-    // (3) the accumulators, eight records per batch of loads
+  if (ncontrib <= kMergeFew) {
 #pragma unroll 1
     for (int eidx = tid; eidx < G * D; eidx += kConsumerThreads) {
       const int r = eidx / D, i = eidx % D;
-      float aref = 0.0f, ares = 0.0f;
-      int cc = 0;
-      for (; cc + 8 <= nc; cc += 8) {
-        float va[8], vr[8];
+      float mc[kMergeFew], lc[kMergeFew], va[kMergeFew], vr[kMergeFew];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const float* rc = rec(c0 + cc + u, r);
+      for (int u = 0; u < kMergeFew; ++u) {
+        mc[u] = kNegInf;
+        lc[u] = va[u] = vr[u] = 0.0f;
+        if (u < ncontrib) {
+          const float* rc = rec(u, r);
+          mc[u] = __ldcg(rc);
+          lc[u] = __ldcg(rc + 1);
           va[u] = __ldcg(rc + 4 + i);
-          vr[u] = RES ? __ldcg(rc + 4 + D + i) : 0.0f;
+          if constexpr (RES) vr[u] = __ldcg(rc + 4 + D + i);
         }
+      }
+      float M = kNegInf;
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const float wgt = wch[(cc + u) * G + r];
-          if (wgt != 0.0f) {
-            aref = fmaf(wgt, va[u], aref);
-            if constexpr (RES) ares = fmaf(wgt, vr[u], ares);
+      for (int u = 0; u < kMergeFew; ++u) M = fmaxf(M, mc[u]);
+      float l = 0.0f, aref = 0.0f, ares = 0.0f;
+#pragma unroll
+      for (int u = 0; u < kMergeFew; ++u) {
+        if (mc[u] != kNegInf) {          // a record without tokens weighs 0
+          const float wgt = exp2f(mc[u] - M);
+          l = fmaf(wgt, lc[u], l);
+          aref = fmaf(wgt, va[u], aref);
+          if constexpr (RES) ares = fmaf(wgt, vr[u], ares);
+        }
+      }
+      zref[eidx] = aref;
+      zres[eidx] = ares;
+      if (i == 0) {
+        lsum[r] = l;
+        mrow[r] = M;
+      }
+    }
+  } else {
+    // (1) M_r
+    {
+      float pm = kNegInf;
+      for (int c = tid / G; c < ncontrib; c += RSTEP) pm = fmaxf(pm, __ldcg(rec(c, rr)));
+  #pragma unroll
+      for (int m = G; m < 32; m <<= 1) pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, m));
+      if (lane_m < G) red[warp_m * G + lane_m] = pm;
+      named_bar_sync(1, kConsumerThreads);
+      if (tid < G) {
+        float M = kNegInf;
+  #pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, red[w * G + tid]);
+        mrow[tid] = M;
+      }
+      named_bar_sync(1, kConsumerThreads);
+    }
+    float lpart = 0.0f;                            // threads tid < G: l of row tid
+    for (int c0 = 0; c0 < ncontrib; c0 += kMergeChunk) {
+      const int nc = min(kMergeChunk, ncontrib - c0);
+      // (2) the chunk's weights; a record without tokens (m = -inf) weighs 0
+      for (int e = tid; e < nc * G; e += kConsumerThreads) {
+        const int c = c0 + e / G, r = e % G;
+        const float* rc = rec(c, r);
+        const float mc = __ldcg(rc), lc = __ldcg(rc + 1);
+        const float wgt = (mc == kNegInf) ? 0.0f : exp2f(mc - mrow[r]);
+        wch[e] = wgt;
+        lch[e] = (mc == kNegInf) ? 0.0f : wgt * lc;
+      }
+      named_bar_sync(1, kConsumerThreads);
+      if (tid < G)
+        for (int cc = 0; cc < nc; ++cc) lpart += lch[cc * G + tid];
+      // (3) the accumulators, eight records per batch of loads
+  #pragma unroll 1
+      for (int eidx = tid; eidx < G * D; eidx += kConsumerThreads) {
+        const int r = eidx / D, i = eidx % D;
+        float aref = 0.0f, ares = 0.0f;
+        int cc = 0;
+        for (; cc + 8 <= nc; cc += 8) {
+          float va[8], vr[8];
+  #pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const float* rc = rec(c0 + cc + u, r);
+            va[u] = __ldcg(rc + 4 + i);
+            vr[u] = RES ? __ldcg(rc + 4 + D + i) : 0.0f;
+          }
+  #pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const float wgt = wch[(cc + u) * G + r];
+            if (wgt != 0.0f) {
+              aref = fmaf(wgt, va[u], aref);
+              if constexpr (RES) ares = fmaf(wgt, vr[u], ares);
+            }
           }
         }
-      }
-      for (; cc < nc; ++cc) {
-        const float* rc = rec(c0 + cc, r);
-        const float wgt = wch[cc * G + r];
-        const float va = __ldcg(rc + 4 + i);
-        const float vr = RES ? __ldcg(rc + 4 + D + i) : 0.0f;
-        if (wgt != 0.0f) {
-          aref = fmaf(wgt, va, aref);
-          if constexpr (RES) ares = fmaf(wgt, vr, ares);
+        for (; cc < nc; ++cc) {
+          const float* rc = rec(c0 + cc, r);
+          const float wgt = wch[cc * G + r];
+          const float va = __ldcg(rc + 4 + i);
+          const float vr = RES ? __ldcg(rc + 4 + D + i) : 0.0f;
+          if (wgt != 0.0f) {
+            aref = fmaf(wgt, va, aref);
+            if constexpr (RES) ares = fmaf(wgt, vr, ares);
+          }
         }
+        zref[eidx] = c0 ? zref[eidx] + aref : aref;
+        zres[eidx] = c0 ? zres[eidx] + ares : ares;
       }
-      zref[eidx] = c0 ? zref[eidx] + aref : aref;
-      zres[eidx] = c0 ? zres[eidx] + ares : ares;
+      named_bar_sync(1, kConsumerThreads);      // the chunk's weights may be overwritten
     }
-    named_bar_sync(1, kConsumerThreads);      // the chunk's weights may be overwritten
+    if (tid < G) lsum[tid] = lpart;
   }
-  if (tid < G) lsum[tid] = lpart;
   const int nt = p.n_tail;
   if (nt > 0) {
     // BF16 tail tokens of this head (not encoded yet): same base-2 scores,
