@@ -222,6 +222,32 @@ def test_cr_decode_single_query_shapes(ref_bits, bits, d, g):
     print(f"single query ref INT{ref_bits} bits {bits} d {d} group {g}: max-abs {worst:.2e}")
 
 
+@pytest.mark.parametrize("ref_bits,bits,hkv,ctx", [(8, 2, 1, 20000), (4, 2, 8, 3000)])
+def test_cr_decode_many_records_per_head(ref_bits, bits, hkv, ctx):
+    """Few heads over a long context: one head spread over every CTA of the
+    single-query kernel (more records than one merge chunk), or a few dozen
+    records per head (above the one-batch merge, within one chunk)."""
+    B, d, g = 1, 128, 32
+    w = synth.Workload("crlong", 2, 1, B, ctx, hkv, hkv, d, g, (2,), (0.25,), 410 + hkv)
+    refk, refv = synth.reference(w, 0, 0), synth.reference(w, 0, 1)
+    xk, xv = synth.loop_kv(w, 0, 0, 1, refk), synth.loop_kv(w, 0, 1, 1, refv)
+    (rck, rsk), ck, sk = rq.encode_cr([xk], refk, ref_bits, [bits], g, w.seed)
+    (rcv, rsv), cv, sv = rq.encode_cr([xv], refv, ref_bits, [bits], g, w.seed)
+    q = synth.query(w, 0, 1)
+    out = rq.decode_attention_cr(q, (rck, rsk, rcv, rsv, ref_bits), ck[0], cv[0], sk[0], sv[0],
+                                 bits, g, w.seed, ctx, kv_heads=hkv)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out).all()
+    worst = 0.0
+    for h in range(hkv):
+        want = oracle_cr_head(xk, xv, refk, refv, ref_bits, bits, g, w.seed, q, 0, h, ctx,
+                              None, None, 0)
+        got = out[0, h:h + 1].double().cpu().numpy()
+        worst = max(worst, float(np.abs(got - want).max()))
+    assert worst <= OUT_TOL
+    print(f"ref INT{ref_bits} bits {bits} Hkv {hkv} T {ctx}: max-abs {worst:.2e}")
+
+
 def oracle_cr_kv(xk, xv, refk, refv, ref_bits, bits, g, seed, b, h, ctx):
     """fp64 K_hat, V_hat of (sequence b, kv head h) from the oracle's own encode."""
     d = refk.shape[-1]

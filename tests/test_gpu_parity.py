@@ -236,6 +236,8 @@ def test_decode_full_size_sampled(name, loops):
     (64, 32, 4, 4, 257, 2, 1),         # INT4, 32-dim groups at d 64: two chunks per row
     (128, 32, 8, 4, 777, 1, 3),        # INT4, 32-dim groups, G = 8, ragged
     (64, 32, 2, 2, 191, 3, 2),         # INT2, 32-dim groups at d 64 (word exchange)
+    (128, 32, 1, 2, 20000, 1, 1),      # G = 1, one head over every CTA: the merge's chunked passes
+    (128, 32, 1, 2, 4000, 1, 8),       # G = 1, ~37 records per head: one chunk
 ])
 def test_decode_edge_shapes(d, group, G, bits, ctx, batch, hkv):
     bl = (bits, 16) if bits != 16 else (2, 16)
