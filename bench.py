@@ -442,7 +442,7 @@ def other_workloads(peak, local_rank, args):
     cap = {"budget_bytes": synth.KV_BUDGET_BYTES, "ctx": w.ctx, "max_batch": maxb,
            "exceeds_budget": sorted({f"{s} {b}" for s, b, _, ok in rows if not ok}),
            "runs": []}
-    for scheme in ("rq", "bf16"):
+    for scheme in ("rq", "bf16", "rq_cr8"):
         r = capacity.run_batch(w, w.ctx, maxb[scheme], scheme, args.capacity_steps, peak,
                                synth.KV_BUDGET_BYTES)
         cap["runs"].append({k: r[k] for k in ("scheme", "batch", "cache_bytes_allocated",

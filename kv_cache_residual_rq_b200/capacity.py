@@ -12,6 +12,11 @@ group 32, loops 1-3 INT2):
          attention call per (loop, layer) over that loop's own K/V
   rq   : the final loop in BF16 plus INT2 residuals of loops 1-3; a step
          runs the residual call for loops 1-3 and the BF16 call for loop 4
+  rq_cr8 : the same with the final loop itself stored as rotated INT8 codes
+         with fp16 scales (the compressed reference), the residuals taken
+         against its reconstruction; a step runs the compressed-reference
+         call with loop l's residual for loops 1-3 and the reference alone
+         for loop 4
 
 For every batch of the sweep the full cache size is computed; a batch whose
 cache exceeds the budget (120e9 bytes, decimal) is reported as such and not
@@ -37,16 +42,39 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 
+SCHEMES = ("bf16", "rq", "rq_cr8")
+CR_REF_BITS = 8           # reference code bits of the rq_cr8 scheme
+
+
+def kv_bytes_per_sequence(w, ctx, scheme):
+    """KV bytes of one sequence across all layers and loops."""
+    if scheme != "rq_cr8":
+        return synth_kv_bytes(w, ctx, scheme == "rq")
+    per_elem_bits = CR_REF_BITS + 16.0 / w.group             # reference codes + scales
+    for b in w.bits:
+        per_elem_bits += b + 16.0 / w.group                  # each residual loop
+    return int(2 * w.layers * w.kv_heads * ctx * w.head_dim * per_elem_bits / 8)
+
+
+def synth_kv_bytes(w, ctx, quantized):
+    from kv_cache_residual_rq_b200 import synth
+    return synth.kv_bytes_per_sequence(w, ctx, quantized)
+
+
 def step_bytes(w, ctx, batch, scheme):
     """Algorithmic bytes one decode step reads (all loops and layers)."""
     heads_t = batch * w.kv_heads * ctx
-    ref = 2 * heads_t * w.head_dim * 2                       # K + V, bf16
+    scales = 2 * (w.head_dim // w.group)                     # fp16 scale bytes per token
+    if scheme == "rq_cr8":
+        ref = 2 * heads_t * (w.head_dim * CR_REF_BITS // 8 + scales)   # K + V codes, scales
+    else:
+        ref = 2 * heads_t * w.head_dim * 2                   # K + V, bf16
     per_layer = 0
     for li in range(w.loops):
-        per_layer += ref                                     # every call reads a BF16 K/V
-        if scheme == "rq" and li < w.loops - 1:
+        per_layer += ref                                     # every call reads the reference
+        if scheme != "bf16" and li < w.loops - 1:
             b = w.bits[li]
-            per_layer += 2 * heads_t * (w.head_dim * b // 8 + 2 * (w.head_dim // w.group))
+            per_layer += 2 * heads_t * (w.head_dim * b // 8 + scales)
     q_out = w.loops * batch * w.q_heads * w.head_dim * 6
     return w.layers * (per_layer + q_out)
 
@@ -95,6 +123,65 @@ class BF16Step:
                     self.ws_bytes, st)
 
 
+class CRStep:
+    """The rq_cr8 cache: per (layer, K or V) the final loop as INT8 reference
+    codes and scales and loops 1-3 as INT2 residuals against its
+    reconstruction, all from the library's compressed-reference encoder; the
+    per-step inputs as in BF16Step."""
+
+    def __init__(self, w, device):
+        import torch
+        import kv_cache_residual_rq_b200 as rq
+        from kv_cache_residual_rq_b200 import synth
+        self.w, self.rq = w, rq
+        L, N, B, H, T, d = w.loops, w.layers, w.batch, w.kv_heads, w.ctx, w.head_dim
+        self.shape = rq.make_shape(B, H, T, d, w.group, w.q_heads)
+        # [layer][K, V] -> ((ref codes, ref scales), [codes per loop], [scales per loop])
+        self.parts = []
+        for layer in range(N):
+            kinds = []
+            for kind in (0, 1):
+                r = synth.reference(w, layer, kind, device)
+                loops = [synth.loop_kv(w, layer, kind, l, r) for l in range(1, L)]
+                kinds.append(rq.encode_cr(loops, r, CR_REF_BITS, list(w.bits), w.group, w.seed))
+                del loops, r
+            self.parts.append(kinds)
+            torch.cuda.empty_cache()
+        self.q = torch.stack([torch.stack([synth.query(w, layer, loop, device)
+                                           for layer in range(N)]) for loop in range(1, L + 1)])
+        g = torch.Generator(device=device)
+        g.manual_seed(w.seed * 31 + 7)
+        self.new_kv = torch.randn((L, N, 2, B, H, 1, d), generator=g,
+                                  device=device).to(torch.bfloat16)
+        self.out = torch.empty((L, N, B, w.q_heads, d), dtype=torch.float32, device=device)
+        self.ws = rq.alloc_workspace(self.shape, device)
+        self.ws_bytes = self.ws.numel()
+
+    def cache_bytes(self):
+        n = 0
+        for kinds in self.parts:
+            for (rc, rs), codes, scales in kinds:
+                n += rc.numel() + rs.numel() + sum(c.numel() for c in codes)
+                n += sum(x.numel() for x in scales)
+        return n
+
+    def run(self, stream, append=False):
+        st = stream.cuda_stream
+        w = self.w
+        for li in range(w.loops):
+            res = li < w.loops - 1
+            for layer in range(w.layers):
+                (rck, rsk), ck, sk = self.parts[layer][0]
+                (rcv, rsv), cv, sv = self.parts[layer][1]
+                self.rq.rq_decode_attention_cr(
+                    self.shape, None, self.q[li, layer], rck, rcv, rsk, rsv, CR_REF_BITS,
+                    ck[li] if res else None, cv[li] if res else None,
+                    sk[li] if res else None, sv[li] if res else None,
+                    w.bits[li] if res else 16, w.seed, 0.0, self.new_kv[li, layer, 0],
+                    self.new_kv[li, layer, 1], 1, 1, self.out[li, layer], self.ws,
+                    self.ws_bytes, st)
+
+
 def run_batch(w, ctx, batch, scheme, steps, peak, budget):
     """Allocate and fill the full cache of `batch` sequences, check it against
     the budget, time whole decode steps.  Returns the result line."""
@@ -106,7 +193,7 @@ def run_batch(w, ctx, batch, scheme, steps, peak, budget):
     wb = dataclasses.replace(w, batch=batch, ctx=ctx)
     torch.cuda.empty_cache()
     base = torch.cuda.memory_allocated(dev)
-    state = (DecodeStep if scheme == "rq" else BF16Step)(wb, dev)
+    state = {"rq": DecodeStep, "bf16": BF16Step, "rq_cr8": CRStep}[scheme](wb, dev)
     torch.cuda.synchronize(dev)
     torch.cuda.empty_cache()
     held = torch.cuda.memory_allocated(dev) - base
@@ -133,7 +220,7 @@ def run_batch(w, ctx, batch, scheme, steps, peak, budget):
     t = times[len(times) // 2]
     nb = step_bytes(w, ctx, batch, scheme)
     line = {"scheme": scheme, "batch": batch, "ctx": ctx, "status": "run",
-            "kv_bytes": batch * synth.kv_bytes_per_sequence(w, ctx, scheme == "rq"),
+            "kv_bytes": batch * kv_bytes_per_sequence(w, ctx, scheme),
             "cache_bytes_allocated": cache, "device_bytes_held": held,
             "budget_bytes": budget, "step_ms": t * 1e3, "tokens_per_s": batch / t,
             "step_bytes": nb, "gbs": nb / t / 1e9, "frac_hbm": nb / t / 1e9 / peak,
@@ -146,11 +233,10 @@ def run_batch(w, ctx, batch, scheme, steps, peak, budget):
 
 def plan(w, ctx, batches, budget):
     """(scheme, batch, cache bytes, fits) for the sweep, plus the max batches."""
-    from kv_cache_residual_rq_b200 import synth
     rows = []
     maxb = {}
-    for scheme in ("bf16", "rq"):
-        per_seq = synth.kv_bytes_per_sequence(w, ctx, scheme == "rq")
+    for scheme in SCHEMES:
+        per_seq = kv_bytes_per_sequence(w, ctx, scheme)
         maxb[scheme] = int(budget // per_seq)
         for b in batches:
             rows.append((scheme, b, b * per_seq, b * per_seq <= budget))
@@ -171,8 +257,7 @@ def main(argv=None):
     rows, maxb = plan(w, ctx, batches, args.budget)
     emit = lambda d: print(json.dumps(d), flush=True)
     emit({"workload": w.name, "ctx": ctx, "budget_bytes": args.budget,
-          "kv_bytes_per_sequence": {s: synth.kv_bytes_per_sequence(w, ctx, s == "rq")
-                                    for s in ("bf16", "rq")},
+          "kv_bytes_per_sequence": {s: kv_bytes_per_sequence(w, ctx, s) for s in SCHEMES},
           "max_batch": maxb})
     peak = _peak()
     for scheme, b, kv, fits in rows:

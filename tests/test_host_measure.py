@@ -14,12 +14,23 @@ def test_kv_bytes_per_sequence_by_hand():
     assert synth.kv_bytes_per_sequence(W, CTX, True) == elems * 2 + 3 * elems * (2 + 0.5) // 8
 
 
+def test_compressed_reference_kv_bytes_by_hand():
+    # INT8 reference (8 bits + one fp16 scale per 32) + three INT2 loops
+    # (2 bits + one fp16 scale per 32 each): 16 bits per element, K and V
+    elems = 2 * 24 * 16 * CTX * 128
+    assert capacity.kv_bytes_per_sequence(W, CTX, "rq_cr8") == elems * 2      # 6.44 GB
+    assert capacity.kv_bytes_per_sequence(W, CTX, "bf16") == elems * 2 * 4
+    assert capacity.kv_bytes_per_sequence(W, CTX, "rq") == synth.kv_bytes_per_sequence(W, CTX, True)
+
+
 def test_budget_plan_max_batches():
     rows, maxb = capacity.plan(W, CTX, synth.SWEEP_BATCHES, 120e9)
-    assert maxb == {"bf16": 4, "rq": 12}
+    assert maxb == {"bf16": 4, "rq": 12, "rq_cr8": 18}
     fits = {(s, b) for s, b, _, ok in rows if ok}
     assert fits == {("bf16", 1), ("bf16", 2), ("bf16", 4),
-                    ("rq", 1), ("rq", 2), ("rq", 4), ("rq", 8), ("rq", 12)}
+                    ("rq", 1), ("rq", 2), ("rq", 4), ("rq", 8), ("rq", 12),
+                    ("rq_cr8", 1), ("rq_cr8", 2), ("rq_cr8", 4), ("rq_cr8", 8),
+                    ("rq_cr8", 12), ("rq_cr8", 16)}
 
 
 def test_step_bytes_reread_reference_each_loop():
@@ -29,6 +40,9 @@ def test_step_bytes_reread_reference_each_loop():
     qo = 4 * 24 * 16 * 128 * 6
     assert capacity.step_bytes(W, CTX, 1, "bf16") == elems * 2 * 4 + qo
     assert capacity.step_bytes(W, CTX, 1, "rq") == elems * 2 * 4 + 3 * elems * 5 // 16 + qo
+    # compressed reference: every call reads the INT8 reference codes and
+    # scales (136 bytes per token row of 128 dims), loops 1-3 add 40
+    assert capacity.step_bytes(W, CTX, 1, "rq_cr8") == elems * (4 * 136 + 3 * 40) // 128 + qo
 
 
 def test_call_bytes_by_hand():
