@@ -239,6 +239,54 @@ def measure_gqa_variants(reps, peak, emit):
         torch.cuda.empty_cache()
 
 
+def measure_cr_long(reps, peak, emit, batches=(1, 4, 16)):
+    """The compressed-reference decode (INT8 reference + one INT2 loop, and
+    the reference alone) at the 32K-prefill workload's shapes (16 KV heads,
+    32K context, one layer) for several batches: single launches (median of
+    `reps`) and ten back-to-back launches (best of three)."""
+    import dataclasses
+    import torch
+    import kv_cache_residual_rq_b200 as rq
+    from kv_cache_residual_rq_b200 import synth
+    dev = torch.device("cuda", torch.cuda.current_device())
+    for B in batches:
+        w = dataclasses.replace(synth.ENCODE, batch=B)
+        refk, refv = synth.reference(w, 0, 0, dev), synth.reference(w, 0, 1, dev)
+        q = synth.query(w, 0, 1, dev)
+        xk, xv = synth.loop_kv(w, 0, 0, 1, refk), synth.loop_kv(w, 0, 1, 1, refv)
+        (rck, rsk), ck, sk = rq.encode_cr([xk], refk, 8, [2], w.group, w.seed)
+        (rcv, rsv), cv, sv = rq.encode_cr([xv], refv, 8, [2], w.group, w.seed)
+        del xk, xv, refk, refv
+        torch.cuda.empty_cache()
+        shape = rq.make_shape(B, w.kv_heads, w.ctx, w.head_dim, w.group, w.q_heads)
+        ws = rq.alloc_workspace(shape, dev)
+        out = torch.empty((B, w.q_heads, w.head_dim), dtype=torch.float32, device=dev)
+        for b in (2, 16):
+            args = (ck[0], cv[0], sk[0], sv[0]) if b != 16 else (None,) * 4
+            fn = lambda: rq.rq_decode_attention_cr(shape, None, q, rck, rcv, rsk, rsv, 8, *args,
+                                                   b, w.seed, 0.0, None, None, 0, 0, out, ws)
+            t_iso = _time(fn, reps, None)
+            best = float("inf")
+            for _ in range(3):
+                a = torch.cuda.Event(enable_timing=True)
+                e = torch.cuda.Event(enable_timing=True)
+                a.record()
+                for _ in range(10):
+                    fn()
+                e.record()
+                torch.cuda.synchronize()
+                best = min(best, a.elapsed_time(e) / 1e3 / 10)
+            nb = cr_decode_bytes(w, 8, b)
+            emit({"workload": f"encode_prefill_32k batch {B}",
+                  "kernel": f"decode compressed ref INT8 bits={b}", "G": w.G,
+                  "us": t_iso * 1e6, "us_back_to_back": best * 1e6, "bytes": nb,
+                  "gbs": nb / t_iso / 1e9, "frac": nb / t_iso / 1e9 / peak,
+                  "frac_back_to_back": nb / best / 1e9 / peak})
+        assert rq.rq_workspace_status(ws) == 0
+        del rck, rsk, rcv, rsv, ck, cv, sk, sv, ws, out
+        torch.cuda.empty_cache()
+
+
 def main(argv=None):
     from kv_cache_residual_rq_b200 import synth
     ap = argparse.ArgumentParser()
@@ -247,6 +295,9 @@ def main(argv=None):
     ap.add_argument("--gqa-variants", action="store_true",
                     help="also time the deep-loop shapes with INT4 residuals (64- and 32-dim "
                          "groups) and INT2 with 32-dim groups")
+    ap.add_argument("--cr-long", action="store_true",
+                    help="also time the compressed-reference decode at 32K context for "
+                         "batches 1, 4, 16 (isolated and back to back)")
     args = ap.parse_args(argv)
     peak = _peak()
     emit = lambda d: print(json.dumps(d), flush=True)
@@ -254,6 +305,8 @@ def main(argv=None):
         measure(synth.BY_NAME[name], args.reps, peak, emit)
     if args.gqa_variants:
         measure_gqa_variants(args.reps, peak, emit)
+    if args.cr_long:
+        measure_cr_long(args.reps, peak, emit)
 
 
 if __name__ == "__main__":
