@@ -19,7 +19,7 @@ namespace rq {
 constexpr int kConsumerWarps = 4;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kMergeChunk = 64;   // records whose weights the head merge stages at once
-constexpr int kMergeFew = 8;      // up to this many records a head merge loads in one batch
+constexpr int kMergeFew = 8;      // default: up to this many records a head merge loads in one batch
 constexpr int kPrefetchTiles = 2;   // tiles a CTA fetches into L2 before the grid-dependency wait
 constexpr int kDecodeThreads = kConsumerThreads + 32;   // + one producer warp
 constexpr float kNegInf = -INFINITY;
@@ -282,7 +282,7 @@ __device__ __forceinline__ void load_rotate_queries(const DecodeParams& p, long 
 // folding in the head's BF16 tail tokens (if any).  qs holds the head's raw
 // query rows [G][D] as floats.  All consumer threads call it; `merge` is
 // reused as scratch (it holds at least 4 G (2 + 2 D) floats).
-template <int D, int G, bool RES>
+template <int D, int G, bool RES, int FEW = kMergeFew>
 __device__ __forceinline__ void finish_head(const DecodeParams& p, long long hd,
                                             long long first_tile, int nt_h,
                                             const CallSplit& split, int cta, float* merge,
@@ -357,7 +357,7 @@ __device__ __forceinline__ void finish_head(const DecodeParams& p, long long hd,
   // ---- last contributor: merge all records of the head, finish ----
   // Every record load of a pass is independent of the others, so each pass
   // costs about one L2 round trip per batch of loads instead of one per
-  // record.  Up to kMergeFew records: each thread loads all of them for its
+  // record.  Up to FEW records: each thread loads all of them for its
   // element at once (one round trip).  More: (1) the rows' maxima M_r over
   // the records, (2) per chunk of records their weights exp2(m_c - M_r) and
   // weighted sums l_c, (3) the weighted sums of the accumulators, eight
@@ -379,13 +379,13 @@ __device__ __forceinline__ void finish_head(const DecodeParams& p, long long hd,
   const int rr = tid % G;                        // the row of this thread's records
   constexpr int RSTEP = kConsumerThreads / G;    // records per pass of the threads
   auto rec = [&](int c, int r) { return recs + ((size_t)c * G + r) * (4 + 2 * D); };
-  if (ncontrib <= kMergeFew) {
+  if (ncontrib <= FEW) {
 #pragma unroll 1
     for (int eidx = tid; eidx < G * D; eidx += kConsumerThreads) {
       const int r = eidx / D, i = eidx % D;
-      float mc[kMergeFew], lc[kMergeFew], va[kMergeFew], vr[kMergeFew];
+      float mc[FEW], lc[FEW], va[FEW], vr[FEW];
 #pragma unroll
-      for (int u = 0; u < kMergeFew; ++u) {
+      for (int u = 0; u < FEW; ++u) {
         mc[u] = kNegInf;
         lc[u] = va[u] = vr[u] = 0.0f;
         if (u < ncontrib) {
@@ -398,10 +398,10 @@ __device__ __forceinline__ void finish_head(const DecodeParams& p, long long hd,
       }
       float M = kNegInf;
 #pragma unroll
-      for (int u = 0; u < kMergeFew; ++u) M = fmaxf(M, mc[u]);
+      for (int u = 0; u < FEW; ++u) M = fmaxf(M, mc[u]);
       float l = 0.0f, aref = 0.0f, ares = 0.0f;
 #pragma unroll
-      for (int u = 0; u < kMergeFew; ++u) {
+      for (int u = 0; u < FEW; ++u) {
         if (mc[u] != kNegInf) {          // a record without tokens weighs 0
           const float wgt = exp2f(mc[u] - M);
           l = fmaf(wgt, lc[u], l);

@@ -335,7 +335,8 @@ decode_cr1_kernel(const __grid_constant__ TcParams gp) {
       rec[2 + dim] = 0.0f;
     }
     named_bar_sync(1, kConsumerThreads);
-    finish_head<D, 1, true>(p, hd, first_tile, nt_h, split, cta, merge, qbuf, flags, tid);
+    // four records per batch: the smaller merge leaves the token loop more registers
+    finish_head<D, 1, true, 4>(p, hd, first_tile, nt_h, split, cta, merge, qbuf, flags, tid);
   };
 
   auto kfrag_at = [&](int i) {

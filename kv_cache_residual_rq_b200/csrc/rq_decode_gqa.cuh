@@ -521,8 +521,9 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
       }
       named_bar_sync(1, kConsumerThreads);
     }
-    finish_head<D, G, C::RES || C::CRX>(p, hd, first_tile, nt_h, split, cta, merge, qbuf, flags,
-                                        tid);
+    // compressed references: four records per merge batch (more registers for the token loop)
+    finish_head<D, G, C::RES || C::CRX, C::CRX ? 4 : kMergeFew>(p, hd, first_tile, nt_h, split,
+                                                                 cta, merge, qbuf, flags, tid);
   };
 
   // ---- one tile ----
