@@ -494,7 +494,10 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
                             : C::CR4 ? 32 * (mt >> 1) + 4 * g + 2 * (mt & 1) + (e >> 1)
                                      : dim;
         if (r < G) {
-          if constexpr (C::CRX) mw[r * (2 + 2 * D) + 2 + dim_ref] = oref[mt][e] * (C::CSCALE / vscale);
+          // (INT4 reference: m-rows g + 8 hold 16 x their codes' products)
+          if constexpr (C::CRX)
+            mw[r * (2 + 2 * D) + 2 + dim_ref] =
+                oref[mt][e] * (C::CSCALE / vscale) * ((C::CR4 && (e >> 1)) ? 0.0625f : 1.0f);
           else mw[r * (2 + 2 * D) + 2 + dim_ref] = oref[mt][e];
           if constexpr (C::RES && !C::VSH) mw[r * (2 + 2 * D) + 2 + D + dim_res] = 2.0f * ores[mt][e];
           else mw[r * (2 + 2 * D) + 2 + D + dim] = 0.0f;
@@ -930,9 +933,12 @@ decode_gqa_kernel(const __grid_constant__ TcParams gp) {
             ldsm_x2_trans(sV + swz_offset<C::RROW>(wtok + m * 8 + pr7, ch), v);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-              const int sh = 8 * h;
-              const uint32_t a[4] = {(v[0] >> sh) & 0x000F000Fu, (v[0] >> (sh + 4)) & 0x000F000Fu,
-                                     (v[1] >> sh) & 0x000F000Fu, (v[1] >> (sh + 4)) & 0x000F000Fu};
+              // nibbles 2h (m-rows g) and 2h + 1 (m-rows g + 8) of each half:
+              // the odd one masked in place as 16 c (an exact subnormal), its
+              // m-rows scaled back by 1/16 at the flush
+              const uint32_t v0 = h ? v[0] >> 8 : v[0], v1 = h ? v[1] >> 8 : v[1];
+              const uint32_t a[4] = {v0 & 0x000F000Fu, v0 & 0x00F000F0u, v1 & 0x000F000Fu,
+                                     v1 & 0x00F000F0u};
               mma_f16(oref[2 * ch + h], a, bh0, bh1);
               mma_f16(oref[2 * ch + h], a, bl0, bl1);
               residual_mma(2 * ch + h);
