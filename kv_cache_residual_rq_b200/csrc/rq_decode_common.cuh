@@ -281,9 +281,7 @@ __device__ __forceinline__ void load_rotate_queries(const DecodeParams& p, long 
 // if it is the last CTA of the head to arrive, the head's output, after
 // folding in the head's BF16 tail tokens (if any).  qs holds the head's raw
 // query rows [G][D] as floats.  All consumer threads call it; `merge` is
-// reused as scratch (it holds at least 4 G (2 + 2 D) floats).  FEW: the most
-// records the last contributor merges with one batch of loads per element
-// (a kernel whose token loop is short of registers takes fewer).
+// reused as scratch (it holds at least 4 G (2 + 2 D) floats).
 template <int D, int G, bool RES, int FEW = kMergeFew>
 __device__ __forceinline__ void finish_head(const DecodeParams& p, long long hd,
                                             long long first_tile, int nt_h,
