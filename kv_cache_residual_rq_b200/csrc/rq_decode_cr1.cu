@@ -366,10 +366,12 @@ decode_cr1_kernel(const __grid_constant__ TcParams gp) {
         for (int cq = 0; cq < NV / 2; ++cq) {
           uint32_t r[4];
           ldsm_x4(sK + swz_offset<C::RROW>(trow, 2 * cq + (mrow >> 1)), r);
+          // low nibbles, and the high ones masked in place as bytes 16 c (cr2
+          // then holds 16 x their sums, divided out below)
 #pragma unroll
           for (int s = 0; s < 2; ++s) {
-            const uint32_t a[4] = {(r[0] >> (4 * s)) & 0x0F0F0F0Fu, (r[1] >> (4 * s)) & 0x0F0F0F0Fu,
-                                   (r[2] >> (4 * s)) & 0x0F0F0F0Fu, (r[3] >> (4 * s)) & 0x0F0F0F0Fu};
+            const uint32_t mk = s ? 0xF0F0F0F0u : 0x0F0F0F0Fu;
+            const uint32_t a[4] = {r[0] & mk, r[1] & mk, r[2] & mk, r[3] & mk};
             const uint2 b = kfrag_at(2 * cq + s);
             mma_u8s8(s ? cr2 : cr, a, b.x, b.y);
           }
@@ -396,12 +398,12 @@ decode_cr1_kernel(const __grid_constant__ TcParams gp) {
         const uint4 w1 = *reinterpret_cast<const uint4*>(r1 + 16 * tv);
         const uint32_t x0[4] = {w0.x, w0.y, w0.z, w0.w};
         const uint32_t x1[4] = {w1.x, w1.y, w1.z, w1.w};
+        // odd m: the high nibbles masked in place (ck2 holds 16 x their sums)
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
-          const int wi = m >> 1, sh = 4 * (m & 1);
-          const uint32_t a[4] = {(x0[wi] >> sh) & 0x0F0F0F0Fu, (x1[wi] >> sh) & 0x0F0F0F0Fu,
-                                 (x0[2 + wi] >> sh) & 0x0F0F0F0Fu,
-                                 (x1[2 + wi] >> sh) & 0x0F0F0F0Fu};
+          const int wi = m >> 1;
+          const uint32_t mk = (m & 1) ? 0xF0F0F0F0u : 0x0F0F0F0Fu;
+          const uint32_t a[4] = {x0[wi] & mk, x1[wi] & mk, x0[2 + wi] & mk, x1[2 + wi] & mk};
           const uint2 b = kfrag_at(NV + m);
           mma_u8s8((m & 1) ? ck2 : ck, a, b.x, b.y);
         }
@@ -412,10 +414,11 @@ decode_cr1_kernel(const __grid_constant__ TcParams gp) {
       // level sums 2 <Q, c> - (2^b - 1) sum Q of slice t, exact in integers
       const int rg = tv >> RSH;
       const int tok0 = wtok + g, tok1 = tok0 + 8;
+      // (exact: an INT4 chain's second accumulator holds multiples of 16)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        cr[e] += cr2[e];
-        ck[e] += ck2[e];
+        cr[e] += (RB == 4) ? (cr2[e] >> 4) : cr2[e];
+        ck[e] += (BITS == 4) ? (ck2[e] >> 4) : ck2[e];
       }
       const int xr0 = 512 * cr[0] + 2 * cr[1] + koffR;
       const int xr1 = 512 * cr[2] + 2 * cr[3] + koffR;
